@@ -1,0 +1,455 @@
+"""Paged-decode benchmark: KV GB/s and sequence-steps/s on B200, % of HBM roofline.
+
+Workload (default): Llama-3-8B-shaped GQA decode with prefix sharing, bf16 -- 256
+sequences in 16 groups of 16 sharing a 512-token prefix (32 shared blocks), private
+lognormal suffixes (median 600, cap 8192), 32 query / 8 kv heads, head_dim 128,
+block_size 16.  One step = the whole decode hot path for one batch:
+pa_cache_write of the 256 new tokens' K/V through their slot mapping, then
+pa_decode over every sequence (split-K partitions of 512 tokens + LSE reduce).
+
+Timed region: K steps after W warm-up steps, CUDA events on the launching stream,
+barrier + synchronize on both sides, max over ranks.  The step's inputs (1.1 GB of
+KV) are larger than L2 (126 MB), so no flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank holds its own copy of the workload on its GPU
+(the path shards by sequence with no exchange) -> weak scaling; `value` is the
+total over ranks.  `--impl reference` times the CPU oracle on the host cores on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+PARTITION = 512
+CONFIG_ID = 3
+WORKLOAD_NAME = "llama3-8b-gqa-prefix-sharing-decode"
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------- accounting
+def step_bytes(wl, tables, lens):
+    """Algorithmic bytes of one decode launch: K+V of every token attended, q in,
+    out written.  'unique' counts each (physical block, token slot) once -- the
+    HBM floor when siblings share prefix blocks; 'logical' counts per sequence."""
+    e = wl.elem_bytes
+    row = wl.num_kv_heads * wl.head_dim * e * 2          # K + V of one token, all kv heads
+    qo = len(lens) * wl.num_q_heads * wl.head_dim * e * 2
+    used = {}
+    for s, L in enumerate(lens):
+        for j in range(-(-int(L) // 16)):
+            b = int(tables[s, j])
+            used[b] = max(used.get(b, 0), min(16, int(L) - 16 * j))
+    unique = sum(used.values()) * row + qo
+    logical = int(np.sum(lens)) * row + qo
+    return unique, logical
+
+
+def cache_write_bytes(wl, ntok):
+    return ntok * wl.num_kv_heads * wl.head_dim * wl.elem_bytes * 2 * 2   # K,V read + write
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """NVML polling of SM clock and clock-event reasons in a background thread."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle", 0x10: "sync_boost"}
+
+    def __init__(self, torch, device, period_s=0.005):
+        self.samples, self.period, self.ok = [], period_s, False
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            try:
+                props = torch.cuda.get_device_properties(device)
+                bus = "%08x:%02x:%02x.0" % (getattr(props, "pci_domain_id", 0), props.pci_bus_id,
+                                            props.pci_device_id)
+                self.h = nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+            except Exception:
+                self.h = nv.nvmlDeviceGetHandleByIndex(device)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as ex:  # NVML missing: report no clocks rather than guess
+            log("clock sampling unavailable:", ex)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _reasons(self):
+        nv = self.nv
+        f = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        return int(f(self.h))
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self, t0, t1):
+        if not self.ok:
+            return None
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed_region"
+        if not inside:   # region shorter than the poll period: nearest samples around it
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:2]
+            window = "nearest_to_timed_region"
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median([s[1] for s in inside])) if inside else None,
+                "sm_max_mhz": float(self.max_mhz), "reasons": reasons,
+                "samples": len(inside), "window": window}
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    if n_gpus != world:
+        log(f"note: --gpus {n_gpus} but WORLD_SIZE {world}; using WORLD_SIZE")
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- profiles
+def recorded_traffic(kernel_src):
+    """DRAM bytes per launch from the committed ncu summary, or None if the kernel's
+    source changed since the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "decode_gqa8b_prefix_ncu.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    mh = re.search(r"decode\.cu sha256: ([0-9a-f]{64})", text)
+    mt = re.search(r"dram bytes per launch \(read\+write\): (\d+)", text)
+    if not mh or not mt:
+        return None
+    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
+    return int(mt.group(1)) if cur == mh.group(1) else None
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    world, rank, local = dist_setup(args.gpus)
+    import paged_kv_cache_389_b200 as pa
+    from paged_kv_cache_389_b200.cache import PagedKVCache
+
+    t_setup = time.time()
+    wl = workloads.make(CONFIG_ID)
+    step = wl.steps[0]
+    S = len(step.seqs)
+    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, torch.bfloat16, "cuda",
+                         wl.free_order)
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    workloads.replay(wl, cache.manager, lambda k, v, s: pa.pa_cache_write(
+        dev(k), dev(v), torch.from_numpy(s).cuda(), cache.key_cache, cache.value_cache, cache.err_flag))
+    slots, pairs = cache.plan_append(step.seqs)
+    assert len(pairs) == 0
+    max_blocks = max(cache.manager.num_seq_blocks(s) for s in step.seqs)
+    tables_h, lens_h = cache.manager.build_tables(step.seqs, max_blocks)
+    max_ctx = int(lens_h.max())
+    # device-resident step inputs
+    q = dev(step.q)
+    k_new, v_new = dev(step.k_new), dev(step.v_new)
+    slots_d = torch.from_numpy(slots).cuda()
+    tables_d = torch.from_numpy(tables_h).cuda()
+    lens_d = torch.from_numpy(lens_h).cuda()
+    out = torch.empty_like(q)
+    ws_n = pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, max_ctx, PARTITION)
+    ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    unique_b, logical_b = step_bytes(wl, tables_h, lens_h)
+    cw_b = cache_write_bytes(wl, S)
+    log(f"rank {rank}: setup {time.time() - t_setup:.1f}s; {S} seqs, max ctx {max_ctx}, "
+        f"unique {unique_b / 1e9:.3f} GB, logical {logical_b / 1e9:.3f} GB")
+
+    def step_fn(ev_a=None, ev_b=None):
+        pa.pa_cache_write(k_new, v_new, slots_d, cache.key_cache, cache.value_cache, cache.err_flag, stream)
+        if ev_a is not None:
+            ev_a.record(stream)
+        pa.pa_decode(q, cache.key_cache, cache.value_cache, tables_d, lens_d, max_ctx, wl.scale, out,
+                     PARTITION, ws, cache.err_flag, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    for _ in range(args.warmup):
+        step_fn()
+    torch.cuda.synchronize()
+    flag = pa.pa_wait(cache.err_flag)
+    assert flag == 0, f"device error flag {flag} during warm-up"
+
+    K = args.steps
+    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(torch, local)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    h0 = time.perf_counter()
+    e0.record(stream)
+    for i in range(K):
+        step_fn(*ev_dec[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    h1 = time.perf_counter()
+    barrier(world)
+    sampler.stop()
+    ms = e0.elapsed_time(e1)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    ms_max = max_over_ranks(ms, world)
+    clocks = sampler.summary(h0, h1)
+
+    # end to end: host buffers in, result out, through the same calls
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
+        hq, hk, hv, hs = pin(q), pin(k_new), pin(v_new), pin(slots_d)
+        ht, hl = pin(tables_d), pin(lens_d)
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, ht, hl))
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k_new, hk), (v_new, hv), (slots_d, hs), (tables_d, ht), (lens_d, hl)):
+                dst.copy_(src, non_blocking=True)
+            step_fn()
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        barrier(world)
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(K):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+        e2e = {"value": round(world * (unique_b + cw_b) * K / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "ms_per_step": round(e2e_ms / K, 5),
+               "seq_steps_per_s": round(world * S * K / (e2e_ms * 1e-3), 1),
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+    flag = pa.pa_wait(cache.err_flag)
+    assert flag == 0, f"device error flag {flag}"
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, cache, step, tables_h, lens_h, budget_s=args.cpu_seconds)
+
+    if rank == 0:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+        peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
+        achieved = unique_b / (dec_ms * 1e-3) / 1e9
+        value = world * (unique_b + cw_b) * K / (ms_max * 1e-3) / 1e9
+        line = {
+            "metric": "paged-decode KV GB/s (unique algorithmic bytes) on B200",
+            "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(ms_max / K, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAME, "num_seqs": S, "num_q_heads": wl.num_q_heads,
+                       "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
+                       "prefix_tokens": 512, "group_size": 16, "max_context": max_ctx,
+                       "mean_context": float(np.mean(lens_h)), "partition_size": PARTITION,
+                       "parallelism": f"dp{world} (sequences sharded, no exchange)",
+                       "l2": "inputs larger than L2 (126 MB); no flush"},
+            "seq_steps_per_s": round(world * S * K / (ms_max * 1e-3), 1),
+            "pct_of_8tbs": round(100 * value / world / 8000, 2),
+            "pct_of_measured_hbm": round(100 * value / world / peak, 2),
+            "logical_gbs": round(world * (logical_b + cw_b) * K / (ms_max * 1e-3) / 1e9, 2),
+            "bytes_per_step": {"decode_unique": unique_b, "decode_logical": logical_b, "cache_write": cw_b},
+            "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel + lse reduce)",
+                         "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4),
+                         "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if peaks else "fallback",
+                         "traffic": recorded_traffic(os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", "decode.cu")),
+                         "decode_ms": round(dec_ms, 5)},
+            "e2e": e2e,
+            "gpu_launches": K * 3,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------- CPU oracle
+def _oracle_pools(wl):
+    import oracle
+    from oracle.block_model import BlockManagerModel
+    model = BlockManagerModel(wl.num_blocks, wl.block_size, wl.free_order.tolist())
+    kc = np.full(wl.cache_shape(), 0x7FC0, wl.np_dtype)
+    vc = np.full(wl.cache_shape(), 0x7FC0, wl.np_dtype)
+    workloads.replay(wl, model, lambda k, v, s: oracle.cache_write(k, v, s, kc, vc))
+    step = wl.steps[0]
+    slots = np.array([model.append_slot(s)[0] for s in step.seqs], np.int64)
+    return model, kc, vc, slots
+
+
+def _time_oracle_steps(wl, model, kc, vc, slots, n_seqs, reps):
+    """Time `reps` oracle steps (cache write of the new tokens + decode) over the first
+    n_seqs sequences; returns (seconds per step, unique bytes per step)."""
+    import oracle
+    step = wl.steps[0]
+    seqs = step.seqs[:n_seqs]
+    mb = max(len(model.block_table(s)) for s in seqs)
+    t, l = model.build_tables(seqs, mb)
+    ub, _ = step_bytes(wl, t, l)
+    cw = cache_write_bytes(wl, n_seqs)
+    q = np.ascontiguousarray(step.q[:n_seqs])
+    k, v = np.ascontiguousarray(step.k_new[:n_seqs]), np.ascontiguousarray(step.v_new[:n_seqs])
+    sl = slots[:n_seqs]
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        oracle.cache_write(k, v, sl, kc, vc)
+        oracle.decode(q, kc, vc, t, l, wl.scale)
+    return (time.perf_counter() - t0) / reps, ub + cw
+
+
+def cpu_baseline(wl, cache, step, tables_h, lens_h, budget_s=15.0):
+    import oracle
+    model, kc, vc, slots = _oracle_pools(wl)
+    S = len(step.seqs)
+    per, b = _time_oracle_steps(wl, model, kc, vc, slots, S, 1)
+    reps = max(1, min(int(budget_s / max(per, 1e-3)), 20))
+    per, b = _time_oracle_steps(wl, model, kc, vc, slots, S, reps)
+    return {"value": round(b / per / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds_per_step": round(per, 4),
+            "sample": f"full step ({S} sequences: cache write + decode), {reps} rep(s), fp64 C + OpenMP",
+            "cpu": _cpu_model()}
+
+
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args):
+    """The oracle as it stands, timed on the host cores, on this workload."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    wl = workloads.make(CONFIG_ID)
+    model, kc, vc, slots = _oracle_pools(wl)
+    S = len(wl.steps[0].seqs)
+    one, _ = _time_oracle_steps(wl, model, kc, vc, slots, 1, 1)
+    budget = 150.0 / max(1, args.steps + args.warmup)          # seconds of oracle work per step
+    n = int(max(1, min(S, budget / max(one, 1e-4))))
+    for _ in range(args.warmup):
+        _time_oracle_steps(wl, model, kc, vc, slots, n, 1)
+    t0 = time.perf_counter()
+    total_b = 0
+    for _ in range(args.steps):
+        _, b = _time_oracle_steps(wl, model, kc, vc, slots, n, 1)
+        total_b += b
+    el = time.perf_counter() - t0
+    value = total_b / el / 1e9
+    line = {
+        "impl": "reference", "metric": "paged-decode KV GB/s (unique algorithmic bytes) on B200",
+        "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "num_seqs": S, "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": f"first {n} of {S} sequences per step "
+                                                     "(cache write + decode), fp64 C + OpenMP",
+                         "cpu": _cpu_model()},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

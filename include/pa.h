@@ -1,0 +1,196 @@
+/*
+ * pa.h -- C ABI of the B200 (sm_100a) paged-KV-cache attention library.
+ *
+ * The KV cache of one attention layer lives in a pool of fixed-size physical
+ * blocks; a per-sequence block table maps logical block j to a physical block.
+ * Sources (page title, section):
+ *   "vLLM 深度拆解：当大模型推理学会「分页注意力」" (chenxutan.com), 1.1 and 2.1:
+ *       K and V of every past token are kept and attended to; they are split
+ *       into fixed 16-token blocks placed anywhere in the pool; a block table
+ *       maps logical to physical blocks.  2.3: decode is memory-bandwidth bound,
+ *       prefill compute bound.  3.1: every step writes the new token's K/V back.
+ *       3.3: shared prefix blocks, copy on write.  5.1: chunked prefill.
+ *   devpress.csdn.net/amd vLLM v0.6.x teardown, section 核心代码拆解: tensor
+ *       layouts (below), the physical block looked up through the table, the
+ *       score scaled by `scale`, softmax and a V-weighted sum.  Section
+ *       关键设计二: copy-on-write copies a whole shared block into a new one.
+ *
+ * Layouts (all row-major, all device pointers 16-byte aligned):
+ *   key_cache, value_cache  [num_blocks, num_kv_heads, block_size, head_dim]
+ *   query, out (decode)     [num_seqs, num_q_heads, head_dim]
+ *   query, out (prefill)    [num_seqs, max_chunk, num_q_heads, head_dim]
+ *   block_tables            int32 [num_seqs, max_blocks_per_seq]
+ *   context_lens            int32 [num_seqs]
+ *   slot_mapping            int64 [num_tokens]; slot = block * block_size + offset
+ * Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ * Supported: dtype PA_F32 or PA_BF16 (cache, query, key/value and out share it),
+ * head_dim 64 or 128, block_size 16, num_q_heads / num_kv_heads in {1,2,4,8}.
+ *
+ * Conventions:
+ *   - Ownership: the caller owns every buffer, the decode workspace included.
+ *     The library allocates no device memory.
+ *   - Asynchrony: each call validates its arguments on the host and enqueues its
+ *     kernels on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     PA_OK means "validated and launched", not "finished".
+ *   - Host validation errors (PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED) launch
+ *     nothing.  A CUDA launch failure returns PA_ERR_CUDA.
+ *   - Device-side index faults (a table entry outside the pool, a slot outside
+ *     the pool, a context longer than its table, a copy pair outside the pool)
+ *     never trap: the kernel ORs a PA_DEVERR_* bit into *err_flag (when
+ *     err_flag is not NULL), skips the offending element and carries on.  The
+ *     affected outputs are then unspecified.  Read the flag with pa_wait().
+ *   - Every wait inside a kernel is bounded; a wait that runs out sets
+ *     PA_DEVERR_TIMEOUT and the kernel returns early.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Exported entry points (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define PA_API __attribute__((visibility("default")))
+#else
+#define PA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum pa_status {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer, ... */
+    PA_ERR_UNSUPPORTED = 2,   /* valid but not built: dtype, head_dim, group size, ... */
+    PA_ERR_OOM = 3,           /* block pool exhausted (host block manager) */
+    PA_ERR_DEVICE_INDEX = 4,  /* a kernel flagged an out-of-range index (pa_wait) */
+    PA_ERR_CUDA = 5,          /* a CUDA runtime call failed */
+    PA_ERR_TIMEOUT = 6,       /* pa_wait gave up, or a kernel's bounded wait ran out */
+    PA_ERR_NOT_FOUND = 7      /* unknown sequence id (host block manager) */
+} pa_status;
+
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+
+/* Bits a kernel ORs into *err_flag. */
+#define PA_DEVERR_BLOCK_ID 1     /* block table entry outside [0, num_blocks) */
+#define PA_DEVERR_SLOT 2         /* slot_mapping entry >= num_blocks * block_size */
+#define PA_DEVERR_CONTEXT_LEN 4  /* context_len < 0, > max_context_len or > table capacity */
+#define PA_DEVERR_PAIR 8         /* copy pair id outside [0, num_blocks) */
+#define PA_DEVERR_TIMEOUT 16     /* a bounded in-kernel wait ran out */
+#define PA_DEVERR_CHUNK 32       /* chunk_len < 0, > max_chunk or > context_len */
+
+/* The KV pool one call works on. */
+typedef struct pa_cache_desc {
+    int32_t num_blocks;
+    int32_t num_kv_heads;
+    int32_t block_size;   /* must be 16 */
+    int32_t head_dim;     /* 64 or 128 */
+    int32_t dtype;        /* pa_dtype */
+} pa_cache_desc;
+
+/* Version of this ABI (bumped on any signature or layout change). */
+PA_API int32_t pa_abi_version(void);
+
+/* Human-readable name of a status code (static storage). */
+PA_API const char *pa_status_string(pa_status status);
+
+/*
+ * KV append through a slot mapping (reshape-and-cache).
+ * For every token i < num_tokens with slot = slot_mapping[i] >= 0 and every kv
+ * head h:  key_cache[slot / block_size][h][slot % block_size][:] = key[i][h][:]
+ * and the same for value.  key/value: [num_tokens, num_kv_heads, head_dim].
+ * slot < 0 is padding (skipped).  slot >= num_blocks * block_size sets
+ * PA_DEVERR_SLOT and that token is skipped.  Two tokens with the same slot:
+ * unspecified which one lands.  num_tokens == 0 launches nothing.
+ * Source: chenxutan 3.1 (write the new token's K/V back into the cache) and 3.3
+ * (append_slot: the token goes into the current block).
+ */
+PA_API pa_status pa_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
+                         int32_t num_tokens, void *key_cache, void *value_cache,
+                         const pa_cache_desc *cache, int32_t *err_flag, void *stream);
+
+/*
+ * Copy-on-Write block copy.  For each pair p < num_pairs, (src, dst) =
+ * (src_dst_pairs[2p], src_dst_pairs[2p+1]): block dst of key_cache and of
+ * value_cache becomes a copy of block src (every kv head, slot and dim).
+ * Pairs must be independent (no dst repeated, no dst that is also a src); the
+ * host block manager only emits such pairs.  An id outside [0, num_blocks) sets
+ * PA_DEVERR_PAIR and that pair is skipped.  num_pairs == 0 launches nothing.
+ * Source: devpress teardown, 关键设计二 (allocate a new block, copy the shared
+ * one into it, drop a reference to the old one).
+ */
+PA_API pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pairs,
+                         int32_t num_pairs, const pa_cache_desc *cache, int32_t *err_flag,
+                         void *stream);
+
+/*
+ * Bytes of workspace pa_decode needs for a split (partitioned) context:
+ * partials of num_seqs * num_q_heads * ceil(max_context_len / partition_size)
+ * partitions.  Returns 0 when partition_size <= 0 (no split, no workspace).
+ */
+PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size);
+
+/*
+ * Decode attention over the paged cache, one query token per sequence:
+ *   out[s][h][:] = sum_{t < L_s} softmax_t(scale * <query[s][h], K_s[t]>) V_s[t]
+ * with L_s = context_lens[s], K_s[t] = key_cache[block_tables[s][t / 16]][h / g]
+ * [t % 16][:] (V alike) and g = num_q_heads / num_kv_heads.  L_s == 0 gives 0.
+ * Softmax is computed online in fp32 (running max and sum), products and sums in
+ * fp32; bf16 outputs are rounded to nearest even from fp32.
+ * partition_size == 0: each (sequence, kv head) is one work unit.
+ * partition_size > 0 (a multiple of 16): the context is split into partitions of
+ * that many tokens (split-K); each partition keeps its running max m_p, sum
+ * l_p and unnormalised accumulator o_p in `workspace`, and a second kernel
+ * combines them: out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p with
+ * M = max_p m_p.  Sequences with a single partition are finished by the first
+ * kernel.  workspace_bytes must be >= pa_decode_workspace_size(...) for the same
+ * num_seqs, num_q_heads, head_dim, max_context_len and partition_size.
+ * max_context_len bounds every context_lens[s] (larger sets PA_DEVERR_CONTEXT_LEN
+ * and that sequence's outputs are unspecified).  num_seqs <= 16384.
+ * Source: chenxutan 2.3 (one query token per step, bandwidth bound); devpress
+ * teardown 核心代码拆解 (table lookup per logical block, scaled scores, softmax,
+ * weighted V sum).
+ */
+PA_API pa_status pa_decode(const void *query, const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, int32_t max_blocks_per_seq,
+                    const int32_t *context_lens, int32_t max_context_len, int32_t num_seqs,
+                    int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
+                    size_t workspace_bytes, void *out, const pa_cache_desc *cache,
+                    int32_t *err_flag, void *stream);
+
+/*
+ * Causal chunked prefill against the paged cache.  Sequence s has
+ * C_s = chunk_lens[s] new query rows, the last C_s positions of its context of
+ * L_s = context_lens[s] tokens (their K/V already written with pa_cache_write).
+ * Row i < C_s sits at position p = L_s - C_s + i and
+ *   out[s][i][h][:] = sum_{t <= p} softmax_t(scale * <query[s][i][h], K_s[t]>) V_s[t].
+ * query/out: [num_seqs, max_chunk, num_q_heads, head_dim]; rows i >= C_s of out
+ * are not written.  Requires dtype PA_BF16 and head_dim 128 (tcgen05 tensor-core
+ * tiles, bf16 operands, fp32 accumulation in tensor memory).
+ * Source: chenxutan 2.3 (prefill computes a whole prompt and is compute bound)
+ * and 4.3/5.1 (long prompts are cut into chunks that run between decodes).
+ */
+PA_API pa_status pa_prefill_chunk(const void *query, const void *key_cache, const void *value_cache,
+                           const int32_t *block_tables, int32_t max_blocks_per_seq,
+                           const int32_t *context_lens, const int32_t *chunk_lens,
+                           int32_t num_seqs, int32_t max_chunk, int32_t num_q_heads, float scale,
+                           void *out, const pa_cache_desc *cache, int32_t *err_flag,
+                           void *stream);
+
+/*
+ * Wait for `stream` to finish (polling, at most timeout_ms milliseconds) and read
+ * the device error flag.  *flag_out (if not NULL) receives the flag value.
+ * Returns PA_OK, PA_ERR_DEVICE_INDEX (flag has an index bit), PA_ERR_TIMEOUT
+ * (stream still busy, or the flag has PA_DEVERR_TIMEOUT) or PA_ERR_CUDA.
+ * err_flag may be NULL (then only the wait is done).  Not for use during
+ * stream capture.
+ */
+PA_API pa_status pa_wait(void *stream, const int32_t *err_flag, int32_t timeout_ms, int32_t *flag_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

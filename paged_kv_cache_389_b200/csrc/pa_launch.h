@@ -1,0 +1,69 @@
+// Internal launch interface between the C ABI (pa_api.cu) and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "pa.h"
+
+namespace pa {
+
+inline int dtype_bytes(int32_t dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+cudaError_t launch_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
+                               int32_t num_tokens, void *key_cache, void *value_cache,
+                               const pa_cache_desc &c, int32_t *err, cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(void *key_cache, void *value_cache, const int32_t *pairs,
+                               int32_t num_pairs, const pa_cache_desc &c, int32_t *err,
+                               cudaStream_t stream);
+
+struct DecodeLaunch {
+    const void *query;
+    const void *key_cache;
+    const void *value_cache;
+    const int32_t *block_tables;
+    int32_t max_blocks_per_seq;
+    const int32_t *context_lens;
+    int32_t max_context_len;
+    int32_t num_seqs;
+    int32_t num_q_heads;
+    float scale;
+    int32_t partition_size;  // 0 = no split
+    int32_t max_partitions;  // ceil(max_context_len / partition_size) when split
+    float *ws_acc;           // [S][Hq][Pmax][D] unnormalised partial accumulators
+    float2 *ws_ml;           // [S][Hq][Pmax] (running max in log2 units, running sum)
+    void *out;
+    pa_cache_desc cache;
+    int32_t *err;
+};
+
+// Largest num_seqs a split decode supports (the per-CTA partition prefix sum
+// lives in shared memory).
+constexpr int32_t kMaxSplitSeqs = 4096;
+
+cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream);
+
+struct PrefillLaunch {
+    const void *query;
+    const void *key_cache;
+    const void *value_cache;
+    const int32_t *block_tables;
+    int32_t max_blocks_per_seq;
+    const int32_t *context_lens;
+    const int32_t *chunk_lens;
+    int32_t num_seqs;
+    int32_t max_chunk;
+    int32_t num_q_heads;
+    float scale;
+    void *out;
+    pa_cache_desc cache;
+    int32_t *err;
+};
+
+cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
+
+int num_sms(int device);
+
+}  // namespace pa

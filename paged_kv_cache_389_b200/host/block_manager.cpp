@@ -1,0 +1,213 @@
+// Host-side block allocator and block tables (see include/pa_block_manager.h for
+// the contract and the page passages it follows).
+//
+// Data structures: a LIFO free stack of block ids, a reference count per block,
+// and a hash map from sequence id to (token count, block table).  Every mutating
+// call first works out how many fresh blocks it needs and fails with PA_ERR_OOM
+// before touching anything if the free stack is too short, so a failed call
+// leaves the manager exactly as it was.
+#include <cstdint>
+#include <cstring>
+#include <new>
+#include <unordered_map>
+#include <vector>
+
+#include "pa_block_manager.h"
+
+namespace {
+
+struct Sequence {
+    int64_t tokens = 0;
+    std::vector<int32_t> blocks;  // logical block j -> physical block blocks[j]
+};
+
+}  // namespace
+
+struct pa_block_manager {
+    int32_t num_blocks = 0;
+    int32_t block_size = 0;
+    std::vector<int32_t> free_stack;  // back() is the next block handed out
+    std::vector<int32_t> refs;
+    std::unordered_map<int64_t, Sequence> seqs;
+
+    int32_t take() {
+        int32_t b = free_stack.back();
+        free_stack.pop_back();
+        refs[b] = 1;
+        return b;
+    }
+    void release(int32_t b) {
+        if (--refs[b] == 0) free_stack.push_back(b);
+    }
+    static int64_t blocks_for(int64_t tokens, int32_t bs) { return (tokens + bs - 1) / bs; }
+};
+
+extern "C" {
+
+pa_status pa_bm_create(int32_t num_blocks, int32_t block_size, const int32_t *free_order,
+                       pa_block_manager **out) {
+    if (!out || num_blocks < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    *out = nullptr;
+    pa_block_manager *bm = new (std::nothrow) pa_block_manager;
+    if (!bm) return PA_ERR_OOM;
+    bm->num_blocks = num_blocks;
+    bm->block_size = block_size;
+    bm->refs.assign(num_blocks, 0);
+    bm->free_stack.resize(num_blocks);
+    if (free_order) {
+        std::vector<char> seen(num_blocks, 0);
+        for (int32_t i = 0; i < num_blocks; ++i) {
+            int32_t b = free_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) {
+                delete bm;
+                return PA_ERR_INVALID_ARG;
+            }
+            seen[b] = 1;
+            bm->free_stack[i] = b;
+        }
+    } else {
+        for (int32_t i = 0; i < num_blocks; ++i) bm->free_stack[i] = i;
+    }
+    *out = bm;
+    return PA_OK;
+}
+
+void pa_bm_destroy(pa_block_manager *bm) { delete bm; }
+
+pa_status pa_bm_add_seq(pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+    bm->seqs.emplace(seq_id, Sequence{});
+    return PA_OK;
+}
+
+pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, int64_t *slots_out,
+                             int32_t *cow_pairs_out, int32_t cow_capacity, int32_t *num_cow_out) {
+    if (!bm || n < 0) return PA_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    Sequence &sq = it->second;
+    const int32_t bs = bm->block_size;
+    // Plan first: fresh blocks for new block boundaries, plus one copy if the
+    // first token lands in a shared, partly filled last block.
+    const bool cow = n > 0 && (sq.tokens % bs) != 0 && bm->refs[sq.blocks.back()] > 1;
+    const int64_t fresh =
+        pa_block_manager::blocks_for(sq.tokens + n, bs) - pa_block_manager::blocks_for(sq.tokens, bs);
+    if (fresh + (cow ? 1 : 0) > (int64_t)bm->free_stack.size()) return PA_ERR_OOM;
+    if (cow && cow_pairs_out && cow_capacity < 1) return PA_ERR_INVALID_ARG;
+    int32_t ncow = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        const int64_t offset = sq.tokens % bs;
+        if (offset == 0) {
+            sq.blocks.push_back(bm->take());
+        } else if (bm->refs[sq.blocks.back()] > 1) {
+            const int32_t old_block = sq.blocks.back();
+            const int32_t new_block = bm->take();
+            if (cow_pairs_out) {
+                cow_pairs_out[2 * ncow] = old_block;
+                cow_pairs_out[2 * ncow + 1] = new_block;
+            }
+            ++ncow;
+            bm->release(old_block);
+            sq.blocks.back() = new_block;
+        }
+        if (slots_out) slots_out[i] = (int64_t)sq.blocks.back() * bs + offset;
+        ++sq.tokens;
+    }
+    if (num_cow_out) *num_cow_out = ncow;
+    return PA_OK;
+}
+
+pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    auto p = bm->seqs.find(parent_id);
+    if (p == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    if (bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
+    Sequence child = p->second;  // copies token count and table
+    for (int32_t b : child.blocks) ++bm->refs[b];
+    bm->seqs.emplace(child_id, std::move(child));
+    return PA_OK;
+}
+
+pa_status pa_bm_free_seq(pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return PA_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    for (int32_t b : it->second.blocks) bm->release(b);
+    bm->seqs.erase(it);
+    return PA_OK;
+}
+
+int64_t pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : it->second.tokens;
+}
+
+int32_t pa_bm_num_seq_blocks(const pa_block_manager *bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : (int32_t)it->second.blocks.size();
+}
+
+pa_status pa_bm_block_table(const pa_block_manager *bm, int64_t seq_id, int32_t *out,
+                            int32_t capacity, int32_t *len_out) {
+    if (!bm || capacity < 0 || (capacity > 0 && !out)) return PA_ERR_INVALID_ARG;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+    const auto &b = it->second.blocks;
+    const int32_t k = (int32_t)b.size() < capacity ? (int32_t)b.size() : capacity;
+    if (k > 0) std::memcpy(out, b.data(), sizeof(int32_t) * k);
+    if (len_out) *len_out = (int32_t)b.size();
+    return PA_OK;
+}
+
+pa_status pa_bm_build_tables(const pa_block_manager *bm, const int64_t *seq_ids, int32_t n,
+                             int32_t max_blocks, int32_t *tables_out, int32_t *lens_out) {
+    if (!bm || n < 0 || max_blocks < 0 || (n > 0 && (!seq_ids || !tables_out)))
+        return PA_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+        if ((int64_t)it->second.blocks.size() > max_blocks) return PA_ERR_INVALID_ARG;
+    }
+    for (int32_t i = 0; i < n; ++i) {
+        const Sequence &sq = bm->seqs.find(seq_ids[i])->second;
+        int32_t *row = tables_out + (int64_t)i * max_blocks;
+        const int32_t k = (int32_t)sq.blocks.size();
+        if (k > 0) std::memcpy(row, sq.blocks.data(), sizeof(int32_t) * k);
+        for (int32_t j = k; j < max_blocks; ++j) row[j] = -1;
+        if (lens_out) lens_out[i] = (int32_t)sq.tokens;
+    }
+    return PA_OK;
+}
+
+int32_t pa_bm_refcount(const pa_block_manager *bm, int32_t block) {
+    if (!bm || block < 0 || block >= bm->num_blocks) return -1;
+    return bm->refs[block];
+}
+
+int32_t pa_bm_num_free(const pa_block_manager *bm) {
+    return bm ? (int32_t)bm->free_stack.size() : -1;
+}
+
+int32_t pa_bm_num_blocks(const pa_block_manager *bm) { return bm ? bm->num_blocks : -1; }
+
+int32_t pa_bm_free_stack(const pa_block_manager *bm, int32_t *out, int32_t capacity) {
+    if (!bm) return -1;
+    const int32_t k = (int32_t)bm->free_stack.size();
+    if (out) {
+        const int32_t m = k < capacity ? k : capacity;
+        if (m > 0) std::memcpy(out, bm->free_stack.data(), sizeof(int32_t) * m);
+    }
+    return k;
+}
+
+int64_t pa_bm_tokens_stored(const pa_block_manager *bm) {
+    if (!bm) return -1;
+    int64_t total = 0;
+    for (const auto &kv : bm->seqs) total += kv.second.tokens;
+    return total;
+}
+
+}  // extern "C"

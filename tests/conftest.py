@@ -17,3 +17,21 @@ def oracle_lib():
     import oracle
     oracle._load()
     return oracle
+
+
+def build_library():
+    """Compile libpa_b200.so if stale, loading the build script by path (importing the
+    package itself needs the library to exist already)."""
+    import importlib.util
+    path = os.path.join(ROOT, "paged_kv_cache_389_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("pa_b200_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod.build()
+
+
+@pytest.fixture(scope="session")
+def pa():
+    build_library()
+    import paged_kv_cache_389_b200 as pa
+    return pa

@@ -1,0 +1,89 @@
+"""The C-ABI library loads, exports every function its headers declare, and its
+host-side validation rejects bad arguments before launching anything (these
+paths make no CUDA call, so they run without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in ("pa.h", "pa_block_manager.h"):
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^PA_API\s+[^(]*?\b(pa_[a-z_0-9]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_headers_declare_the_four_calls():
+    names = declared_functions()
+    for n in ("pa_cache_write", "pa_copy_blocks", "pa_decode", "pa_prefill_chunk"):
+        assert n in names
+    assert len(names) >= 20
+
+
+def test_every_declared_symbol_is_exported(pa):
+    lib = C.CDLL(pa.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_only_the_abi_is_exported(pa):
+    """Internal kernels and helpers are hidden; the dynamic symbol table holds the ABI."""
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", pa.LIB_PATH], capture_output=True, text=True).stdout
+    ours = sorted({l.split()[-1] for l in out.splitlines() if " T " in l and l.split()[-1].startswith("pa_")})
+    assert ours == declared_functions()
+
+
+def test_version_and_status_strings(pa):
+    assert pa.abi_version() == 1
+    assert pa.status_string(pa.PA_OK) == "ok"
+    assert "out of" in pa.status_string(pa.PA_ERR_OOM)
+    assert pa.status_string(99) == "unknown status"
+
+
+def desc(nb=8, hkv=2, bs=16, d=128, dt=1):
+    from paged_kv_cache_389_b200 import CacheDesc
+    return CacheDesc(nb, hkv, bs, d, dt)
+
+
+def test_host_validation_launches_nothing(pa):
+    L = pa._lib
+    p16 = C.c_void_p(0x10000)   # fake, never dereferenced: validation fails first
+    d = desc()
+    # unsupported block size / head dim / dtype
+    assert L.pa_cache_write(p16, p16, p16, 1, p16, p16, C.byref(desc(bs=32)), None, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_cache_write(p16, p16, p16, 1, p16, p16, C.byref(desc(d=96)), None, None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_cache_write(p16, p16, p16, 1, p16, p16, C.byref(desc(dt=7)), None, None) == pa.PA_ERR_UNSUPPORTED
+    # null / misaligned pointers, negative counts
+    assert L.pa_cache_write(None, p16, p16, 1, p16, p16, C.byref(d), None, None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_cache_write(C.c_void_p(0x10008), p16, p16, 1, p16, p16, C.byref(d), None, None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_cache_write(p16, p16, p16, -1, p16, p16, C.byref(d), None, None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_cache_write(None, None, None, 0, None, None, C.byref(d), None, None) == pa.PA_OK   # empty: no launch
+    assert L.pa_copy_blocks(p16, p16, p16, -2, C.byref(d), None, None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_copy_blocks(None, None, None, 0, C.byref(d), None, None) == pa.PA_OK
+    # decode: group size, partition multiple, workspace, context vs table capacity
+    args = lambda hq, part, ws, wsb, maxctx=100, mb=8: (p16, p16, p16, p16, mb, p16, maxctx, 4, hq, 0.1, part,
+                                                        ws, wsb, p16, C.byref(d), None, None)
+    assert L.pa_decode(*args(3, 0, None, 0)) == pa.PA_ERR_INVALID_ARG           # 3 % 2 != 0
+    assert L.pa_decode(*args(32, 0, None, 0)) == pa.PA_ERR_UNSUPPORTED          # group 16
+    assert L.pa_decode(*args(4, 24, None, 0)) == pa.PA_ERR_INVALID_ARG          # not a multiple of 16
+    assert L.pa_decode(*args(4, 32, None, 0)) == pa.PA_ERR_INVALID_ARG          # split needs workspace
+    need = pa.pa_decode_workspace_size(4, 4, 128, 100, 32)
+    assert L.pa_decode(*args(4, 32, p16, need - 1)) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_decode(*args(4, 0, None, 0, maxctx=129, mb=8)) == pa.PA_ERR_INVALID_ARG
+    # prefill needs bf16 / head_dim 128
+    assert L.pa_prefill_chunk(p16, p16, p16, p16, 8, p16, p16, 2, 4, 4, 0.1, p16, C.byref(desc(dt=0)),
+                              None, None) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_workspace_size_formula(pa):
+    # rows = S * Hq * ceil(maxctx / part); each row: head_dim fp32 partials + (m, l)
+    assert pa.pa_decode_workspace_size(8, 64, 128, 32768, 512) == 8 * 64 * 64 * (128 * 4 + 8)
+    assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == 3 * 4 * 4 * (64 * 4 + 8)
+    assert pa.pa_decode_workspace_size(3, 4, 64, 100, 0) == 0

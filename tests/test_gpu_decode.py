@@ -1,0 +1,204 @@
+"""GPU parity: cache write, copy-on-write block copy and decode attention (unsplit
+and split-K) against the CPU oracle, on every workload, through the C ABI.
+
+Bit-exact: pools after every cache write / block copy, block tables, slot mappings.
+Attention: fp32 max |err| <= 1e-5; bf16 |err| <= 1.5e-2 + 1e-2 |ref| per element.
+"""
+import copy
+
+import numpy as np
+import pytest
+
+import workloads
+from gpu_harness import TwoSided, check_close, to_dev, to_host, torch_mod
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _lib(pa):
+    torch = torch_mod()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    return pa
+
+
+def partitions_for(wl):
+    return (0, 16, 32) if wl.config_id == 1 else (0, 512, 256)
+
+
+def run_workload(cid, mini, full_every=1, sample=64):
+    wl = workloads.make(cid, mini=mini)
+    ts = TwoSided(wl)
+    assert ts.pools_equal(), "cache write of the set-up tokens is not bit-exact"
+    assert ts.err_flag() == 0
+    rng = np.random.default_rng(cid)
+    for i, step in enumerate(wl.steps):
+        ts.append_step(step)
+        if i in (0, 1, len(wl.steps) - 1):
+            assert ts.pools_equal(), f"step {i}: pools differ after copy-on-write + cache write"
+        S = len(step.seqs)
+        full = (i % full_every == 0) or i == len(wl.steps) - 1
+        rows = None if full or S <= sample else np.sort(rng.choice(S, sample, replace=False))
+        ref = ts.oracle_decode(step, rows)
+        for part in partitions_for(wl):
+            got = ts.gpu_decode(step, part)
+            if rows is not None:
+                got = got[rows]
+            check_close(got, ref, wl.dtype, f"config {cid} step {i} partition {part}")
+    assert ts.err_flag() == 0
+    return ts
+
+
+def test_tiny_fp32():
+    run_workload(1, False)
+
+
+@pytest.mark.parametrize("cid", [2, 3, 4, 5])
+def test_mini_workloads(cid):
+    run_workload(cid, True)
+
+
+def test_mha_7b():
+    run_workload(2, False)
+
+
+def test_gqa_prefix_sharing():
+    run_workload(3, False)
+
+
+def test_parallel_sampling_fork_cow():
+    ts = run_workload(4, False, full_every=5, sample=64)
+    assert ts.model.num_free() == ts.gpu.manager.num_free()
+
+
+def test_long_context_decode():
+    run_workload(5, False)
+
+
+def test_copy_on_write_pairs_in_first_step_only():
+    wl = workloads.make(4, mini=True)
+    ts = TwoSided(wl)
+    ts.append_step(wl.steps[0])
+    assert len(ts.last_pairs) == 3 * (len(wl.steps[0].seqs) // 4)
+    ts.append_step(wl.steps[1])
+    assert len(ts.last_pairs) == 0
+    assert ts.pools_equal()
+
+
+def _permuted(wl, seed):
+    wl2 = copy.copy(wl)
+    wl2.free_order = np.random.default_rng(seed).permutation(wl.num_blocks).astype(np.int32)
+    return wl2
+
+
+@pytest.mark.parametrize("part", [0, 256])
+def test_physical_placement_is_bitwise_invisible(part):
+    """Same logical data in two differently shuffled pools: identical GPU outputs,
+    since every reduction runs in logical-block order."""
+    wl = workloads.make(3, mini=True)
+    outs = []
+    for seed in (1, 2):
+        w = _permuted(wl, seed)
+        ts = TwoSided(w)
+        ts.append_step(w.steps[0])
+        outs.append(ts.gpu_decode(w.steps[0], part))
+    assert outs[0].tobytes() == outs[1].tobytes()
+
+
+def _custom(lens, hq, hkv, d, dtype, seed=5, extra_blocks=4):
+    rng = np.random.default_rng(seed)
+    need = sum(-(-L // 16) for L in lens) + extra_blocks
+    wl = workloads.Workload(0, "custom", dtype, need, hq, hkv, d, 1.0 / np.sqrt(d),
+                            rng.permutation(need).astype(np.int32))
+    for s, L in enumerate(lens):
+        wl.ops.append(("add", s))
+        if L:
+            wl.ops.append(("append", s, workloads.normal(rng, (L, hkv, d), dtype),
+                           workloads.normal(rng, (L, hkv, d), dtype)))
+    q = workloads.normal(rng, (len(lens), hq, d), dtype)
+    wl.steps.append(workloads.Step(list(range(len(lens))), None, None, q))
+    return wl
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 128), ("f32", 64)])
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_edge_lengths_all_variants(dtype, d, g):
+    """Empty context, a single token, block and partition boundaries +-1, ragged tails."""
+    lens = [0, 1, 15, 16, 17, 31, 33, 255, 256, 257, 511, 512, 513, 700]
+    wl = _custom(lens, 2 * g, 2, d, dtype)
+    ts = TwoSided(wl)
+    step = wl.steps[0]
+    ref = ts.oracle_decode(step)
+    assert np.array_equal(ref[0], np.zeros_like(ref[0]))
+    for part in (0, 16, 256):
+        got = ts.gpu_decode(step, part)
+        assert np.array_equal(got[0], np.zeros_like(got[0])), "empty context must give 0"
+        check_close(got, ref, dtype, f"{dtype} d{d} g{g} part {part}")
+    assert ts.err_flag() == 0
+
+
+def test_gqa_equals_repeated_mha():
+    wl = _custom([40, 300, 129], 8, 2, 128, "bf16")
+    ts = TwoSided(wl)
+    out_gqa = ts.gpu_decode(wl.steps[0], 0)
+    # same data with kv heads repeated 4x: an MHA pool
+    kc = np.repeat(ts.kc, 4, axis=1)
+    vc = np.repeat(ts.vc, 4, axis=1)
+    torch = torch_mod()
+    import paged_kv_cache_389_b200 as pa
+    t, l = ts.tables(wl.steps[0].seqs)
+    kd, vd = to_dev(kc), to_dev(vc)
+    q = to_dev(wl.steps[0].q)
+    out = torch.empty_like(q)
+    pa.pa_decode(q, kd, vd, torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), int(l.max()),
+                 wl.scale, out)
+    check_close(to_host(out), np.asarray(workloads.bf16_bits_to_f32(out_gqa), np.float64), "bf16", "gqa vs mha")
+
+
+def test_many_sequences_split_limit():
+    """4096 short sequences with split-K (the largest batch the split path takes)."""
+    rng = np.random.default_rng(9)
+    lens = rng.integers(1, 80, size=4096).tolist()
+    wl = _custom(lens, 4, 1, 64, "bf16")
+    ts = TwoSided(wl)
+    ref = ts.oracle_decode(wl.steps[0])
+    check_close(ts.gpu_decode(wl.steps[0], 32), ref, "bf16", "4096 seqs split")
+    check_close(ts.gpu_decode(wl.steps[0], 0), ref, "bf16", "4096 seqs")
+
+
+def test_device_index_errors_are_flagged_not_fatal():
+    torch = torch_mod()
+    import paged_kv_cache_389_b200 as pa
+    wl = _custom([40, 20], 4, 4, 128, "bf16")
+    ts = TwoSided(wl)
+    g = ts.gpu
+    step = wl.steps[0]
+    t, l = ts.tables(step.seqs)
+    # table entry outside the pool
+    bad = t.copy()
+    bad[0, 1] = wl.num_blocks + 3
+    g.err_flag.zero_()
+    ts.gpu_decode(step, 0, tables=bad, lens=l)
+    assert pa.pa_wait(g.err_flag) & pa.PA_DEVERR_BLOCK_ID
+    # context longer than max_context_len
+    g.err_flag.zero_()
+    ts.gpu_decode(step, 0, tables=t, lens=l, max_context=30)
+    assert pa.pa_wait(g.err_flag) & pa.PA_DEVERR_CONTEXT_LEN
+    # slot outside the pool; negative slot is padding (no flag, nothing written)
+    g.err_flag.zero_()
+    k = torch.zeros((2, 4, 128), dtype=torch.bfloat16, device="cuda")
+    before = to_host(g.key_cache).tobytes()
+    pa.pa_cache_write(k, k, torch.tensor([-1, wl.num_blocks * 16], dtype=torch.int64, device="cuda"),
+                      g.key_cache, g.value_cache, g.err_flag)
+    assert pa.pa_wait(g.err_flag) == pa.PA_DEVERR_SLOT
+    assert to_host(g.key_cache).tobytes() == before
+    # copy pair outside the pool
+    g.err_flag.zero_()
+    pa.pa_copy_blocks(g.key_cache, g.value_cache,
+                      torch.tensor([[0, wl.num_blocks]], dtype=torch.int32, device="cuda"), g.err_flag)
+    assert pa.pa_wait(g.err_flag) == pa.PA_DEVERR_PAIR
+    assert to_host(g.key_cache).tobytes() == before
+    # the context is still healthy: a clean decode matches the oracle
+    g.err_flag.zero_()
+    check_close(ts.gpu_decode(step, 0), ts.oracle_decode(step), "bf16", "after flagged errors")
+    assert pa.pa_wait(g.err_flag) == 0
