@@ -14,26 +14,36 @@
 //    per unit.  The grid is persistent (one CTA per SM); CTA c takes units
 //    c, c + gridDim, ...  Units are ordered "first partition of every sequence,
 //    kv head innermost" then "remaining partitions, sequence-major": the first
-//    512 tokens of sibling sequences that share prefix blocks are read by CTAs
+//    partition of sibling sequences that share prefix blocks is read by CTAs
 //    running at the same time, so the shared blocks are served from L2.
-//  * Warp 8 is the producer: it reads block-table entries (32 per warp load)
-//    and issues 1-D bulk async copies (TMA engine, cp.async.bulk) of each
-//    4 KB (block, kv head) slab of K and of V into a ring of shared-memory
-//    stages, completion tracked by mbarriers.  No register staging, no
-//    address-generation cost on the consumer warps.
-//  * Warps 0..7 are consumers.  Consumer w takes logical blocks w, w+8, ... of
-//    the unit.  QK: 8 lanes per token (16-byte conflict-free smem reads), packed
-//    fp32 FMAs (FFMA2), a transposing shuffle reduction that leaves each lane
-//    with one head's score.  Online softmax in fp32 (running max m, running
-//    sum l, log2 domain: q is pre-scaled by scale*log2(e)).  PV: each lane owns
-//    D/32 output dims of every head, FFMA2 again.  At the end of a unit the 8
-//    warps' (m, l, acc) are merged through shared memory.
+//  * Each of the CTA's 8 warps takes logical blocks w, w+8, ... of a unit and
+//    streams them itself: the (block, kv head) slabs of K and V (4 KB each in
+//    bf16) are fetched with 16-byte cp.async, all 32 lanes issuing, into a
+//    two-stage per-warp ring, the next block (across unit boundaries) always in
+//    flight while the current one is computed.  Measured on B200: random 4 KB
+//    slabs stream at ~6.6-7 TB/s this way, while bulk copies issued by a single
+//    thread per SM cap near 0.9 TB/s (each copy costs the issuing thread
+//    ~0.65 us), so there is no producer warp.  Each warp keeps its own
+//    online-softmax state (running max m, running sum l, unnormalised
+//    accumulator); the 8 states are merged through shared memory per unit.
+//  * bf16: QK and PV run on warp-level tensor-core tiles (mma.sync m16n8k16, bf16
+//    operands, fp32 accumulation).  QK puts the block's 16 tokens in M and the g
+//    heads in N (S^T = K Q^T); PV computes O^T = V^T P^T with head_dim in M, so no
+//    tile rows are padding.  movmatrix turns S^T's fragments into P^T's operand
+//    fragments in registers.  Slab rows are stored with an XOR swizzle of their
+//    16-byte chunks so the ldmatrix reads are bank-conflict free.  A CUDA-core
+//    version of this path (packed fp32 FMAs, shuffle reductions) measured issue
+//    bound: 63 warp instructions per (token, kv head) against ~6 here.
+//  * fp32: CUDA-core path (tensor cores would round fp32 inputs to tf32): 8 lanes
+//    per token for QK with a transposing shuffle reduction, packed FFMA2 for QK
+//    and PV.
 //  * Split-K (partition_size > 0): a sequence with several partitions writes
 //    (m, l, acc) per partition to the workspace and reduce_kernel combines them;
 //    single-partition sequences are finished directly.
-//  * Every mbarrier wait is bounded (pa_common.cuh); on a timeout the CTA sets
-//    an abort flag, stops issuing, drains its in-flight copies and returns.
+//  * No kernel here spins: cp.async completion is waited for with wait_group and
+//    the only barriers are CTA-wide ones every warp reaches.
 #include <cfloat>
+#include <cstring>
 
 #include "pa_common.cuh"
 #include "pa_launch.h"
@@ -44,6 +54,8 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
 
 template <typename T>
 struct ElemBytes;
@@ -57,43 +69,23 @@ struct ElemBytes<__nv_bfloat16> {
 };
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
-constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Shared-memory carve-up (byte offsets from the dynamic shared memory base).
 template <typename T, int D, int G>
-struct Cfg {
+struct Layout {
     static constexpr int kElem = ElemBytes<T>::value;
     static constexpr int kRowBytes = D * kElem;                 // one token of one head
     static constexpr int kSlabBytes = kBlockSize * kRowBytes;   // one (block, kv head) slab
     static constexpr int kStageBytes = 2 * kSlabBytes;          // K slab + V slab
-    static constexpr int kConsumerWarps = 8;
-    static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kStages = cmin(16, (128 * 1024) / kStageBytes);
-    // QK: 8 lanes per token; each lane reads kQkChunks 16-byte chunks of a row.
-    static constexpr int kQkChunks = kRowBytes / 128;
-    static constexpr int kEpc = 16 / kElem;                     // elements per 16-byte chunk
-    static constexpr int kQkPairs = kQkChunks * kEpc / 2;       // float2 of q per head per lane
-    // PV: each lane owns kDpl consecutive dims of every head.
-    static constexpr int kDpl = D / 32;
-    static constexpr int kPvPairs = kDpl / 2;
-    static constexpr int kPvBytes = kDpl * kElem;
-    static constexpr int kLogG = ilog2(G);
-    static constexpr int kDupMask = (8 >> kLogG) - 1;           // lanes holding the same score
-    static_assert(kRowBytes % 128 == 0, "a row must split into 8 lanes of 16-byte chunks");
-    static_assert(G == 1 || G == 2 || G == 4 || G == 8, "group size");
-
-    // shared-memory carve-up (byte offsets)
+    static constexpr int kStagesPerWarp = kStageBytes <= 8192 ? 2 : 1;
     static constexpr size_t kOffRing = 0;
-    static constexpr size_t kOffQ = kOffRing + (size_t)kStages * kStageBytes;
-    static constexpr size_t kOffP = align_up(kOffQ + 2ull * G * kRowBytes, 16);
-    static constexpr size_t kPWarpFloats = 16 * G + G;          // p[16][G] then alpha[G]
+    static constexpr size_t kOffP = kOffRing + (size_t)kWarps * kStagesPerWarp * kStageBytes;
+    static constexpr size_t kPWarpFloats = 16 * G + G;          // fp32 path: p[16][G], alpha[G]
     static constexpr size_t kOffMacc =
-        align_up(kOffP + (size_t)kConsumerWarps * kPWarpFloats * 4, 16);
-    static constexpr size_t kOffMml = kOffMacc + 2ull * kConsumerWarps * G * D * 4;
-    static constexpr size_t kOffBar = align_up(kOffMml + 2ull * kConsumerWarps * G * 8, 8);
-    static constexpr size_t kOffSlotOk = kOffBar + (2ull * kStages + 4) * 8;
-    static constexpr size_t kOffAbort = kOffSlotOk + (size_t)kStages * 4;
-    static constexpr size_t kOffCum = align_up(kOffAbort + 4, 16);
+        align_up(kOffP + (sizeof(T) == 4 ? (size_t)kWarps * kPWarpFloats * 4 : 64), 16);
+    static constexpr size_t kOffMml = kOffMacc + 2ull * kWarps * G * D * 4;
+    static constexpr size_t kOffCum = align_up(kOffMml + 2ull * kWarps * G * 8, 16);
     static constexpr size_t smem_bytes(int cum_entries) { return kOffCum + (size_t)cum_entries * 4; }
 };
 
@@ -118,12 +110,13 @@ struct Params {
     float scale_log2;
 };
 
-// Context length of sequence s, or -1 when it is outside [0, max_context] or
-// longer than its table.
-__device__ __forceinline__ int checked_len(const Params &p, int s) {
-    const int L = __ldg(p.lens + s);
+// Context length, or -1 when outside [0, max_context] or longer than its table.
+__device__ __forceinline__ int check_len(const Params &p, int L) {
     if (L < 0 || L > p.max_context || (int64_t)L > (int64_t)p.max_blocks * kBlockSize) return -1;
     return L;
+}
+__device__ __forceinline__ int checked_len(const Params &p, int s) {
+    return check_len(p, __ldg(p.lens + s));
 }
 
 __device__ __forceinline__ int num_parts(const Params &p, int L) {
@@ -151,53 +144,251 @@ __device__ __forceinline__ Unit unit_of(int64_t u, int64_t units_first, int hkv,
     return Unit{lo, 1 + e - cum[lo], h};
 }
 
-// Token range [t0, t0 + nt) of a unit.
-__device__ __forceinline__ void unit_range(const Params &p, const Unit &un, int L, int &t0,
-                                           int &nt) {
+// What one warp needs to know about a unit.  `tab` holds, in lane i, the table
+// entry of the unit's logical block i (for i < 32).
+struct WarpUnit {
+    Unit un;
+    int L;    // validated context length (0 when invalid)
+    int t0;   // first token of the partition
+    int nt;   // tokens in the partition
+    int nb;   // blocks in the partition
+    int tab;
+    const int32_t *trow;
+};
+
+__device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t units_first,
+                                          const int *cum, WarpUnit &w, int lane, bool flagger) {
+    w.un = unit_of(u, units_first, p.num_kv_heads, cum, p.num_seqs);
+    const int b0 = p.part_tokens > 0 ? w.un.part * (p.part_tokens / kBlockSize) : 0;
+    w.trow = p.tables + (int64_t)w.un.s * p.max_blocks + b0;
+    // both loads issued before either value is needed
+    const int raw = __ldg(p.lens + w.un.s);
+    w.tab = lane < p.max_blocks - b0 ? __ldg(w.trow + lane) : -1;
+    int L = check_len(p, raw);
+    if (L < 0) {
+        if (flagger && lane == 0 && w.un.part == 0 && w.un.h == 0) flag_error(p.err, PA_DEVERR_CONTEXT_LEN);
+        L = 0;
+    }
+    w.L = L;
     if (p.part_tokens <= 0) {
-        t0 = 0;
-        nt = L;
+        w.t0 = 0;
+        w.nt = L;
     } else {
-        t0 = un.part * p.part_tokens;
-        const int t1 = min(L, t0 + p.part_tokens);
-        nt = max(0, t1 - t0);
+        w.t0 = w.un.part * p.part_tokens;
+        w.nt = max(0, min(L, w.t0 + p.part_tokens) - w.t0);
+    }
+    w.nb = (w.nt + kBlockSize - 1) / kBlockSize;
+}
+
+// Barrier-free prologue: cum[s] = sum_{s' < s} (parts(s') - 1) (exclusive scan,
+// one chunk of sequences per thread).  Ends with __syncthreads.
+__device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (p.part_tokens > 0) {
+        const int S = p.num_seqs;
+        const int per = (S + kThreads - 1) / kThreads;
+        const int beg = min(S, (int)threadIdx.x * per), end = min(S, beg + per);
+        int local = 0;
+        for (int s = beg; s < end; ++s) {
+            const int L = checked_len(p, s);
+            local += num_parts(p, L < 0 ? 0 : L) - 1;
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) scratch[warp] = incl;
+        __syncthreads();
+        int off = 0;
+        for (int w = 0; w < warp; ++w) off += scratch[w];
+        int run = off + incl - local;
+        for (int s = beg; s < end; ++s) {
+            cum[s] = run;
+            const int L = checked_len(p, s);
+            run += num_parts(p, L < 0 ? 0 : L) - 1;
+        }
+        if ((int)threadIdx.x == kThreads - 1) cum[S] = run;
+    }
+    __syncthreads();
+}
+
+// Issue the cp.async copies of one (block, kv head) slab pair into a stage.
+// bf16 rows are 2*D bytes; chunk c of row r goes to chunk position
+// (c & ~7) | ((c ^ r) & 7), which keeps 8 consecutive rows of any column in 8
+// different bank groups.  fp32 rows keep their natural order.
+template <typename T, int D, int G>
+__device__ __forceinline__ void issue_slabs(const Params &p, uint32_t stage, int blk, int h,
+                                            int lane) {
+    using Lay = Layout<T, D, G>;
+    constexpr int kChunksPerRow = Lay::kRowBytes / 16;
+    constexpr int kChunks = Lay::kSlabBytes / 16;
+    const int64_t off = ((int64_t)blk * p.num_kv_heads + h) * Lay::kSlabBytes;
+    const unsigned char *ks = p.kc + off;
+    const unsigned char *vs = p.vc + off;
+#pragma unroll
+    for (int i = lane; i < kChunks; i += 32) {
+        const int r = i / kChunksPerRow, c = i % kChunksPerRow;
+        const int pc = sizeof(T) == 2 ? ((c & ~7) | ((c ^ r) & 7)) : c;
+        const uint32_t d = stage + r * Lay::kRowBytes + pc * 16;
+        cp_async16(d, ks + i * 16);
+        cp_async16(d + Lay::kSlabBytes, vs + i * 16);
     }
 }
 
 template <typename T>
-__device__ __forceinline__ void unpack16(const uint4 &r, float2 *f);
+__device__ __forceinline__ void store_out(void *out, int64_t idx, float v);
 template <>
-__device__ __forceinline__ void unpack16<__nv_bfloat16>(const uint4 &r, float2 *f) {
-    f[0] = bf16x2_to_float2(r.x);
-    f[1] = bf16x2_to_float2(r.y);
-    f[2] = bf16x2_to_float2(r.z);
-    f[3] = bf16x2_to_float2(r.w);
+__device__ __forceinline__ void store_out<float>(void *out, int64_t idx, float v) {
+    static_cast<float *>(out)[idx] = v;
 }
 template <>
-__device__ __forceinline__ void unpack16<float>(const uint4 &r, float2 *f) {
-    f[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
-    f[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+__device__ __forceinline__ void store_out<__nv_bfloat16>(void *out, int64_t idx, float v) {
+    static_cast<__nv_bfloat16 *>(out)[idx] = __float2bfloat16_rn(v);
 }
 
-// Load kBytes (4, 8 or 16) of one row for the PV step and widen to float2 pairs.
-template <typename T, int kBytes>
-__device__ __forceinline__ void load_pv(const unsigned char *src, float2 *f) {
-    if constexpr (kBytes == 16) {
-        const uint4 r = *reinterpret_cast<const uint4 *>(src);
-        unpack16<T>(r, f);
-    } else if constexpr (kBytes == 8) {
-        const uint2 r = *reinterpret_cast<const uint2 *>(src);
-        if constexpr (sizeof(T) == 2) {
-            f[0] = bf16x2_to_float2(r.x);
-            f[1] = bf16x2_to_float2(r.y);
-        } else {
-            f[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+// After the warps' states of a unit are in macc/mml: combine them and write the
+// output (single partition) or the partition's (m, l, acc) to the workspace.
+template <typename T, int D, int G>
+__device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, const float *uacc,
+                                            const float2 *uml) {
+    const bool single = num_parts(p, w.L) == 1;
+    const int64_t head0 = (int64_t)w.un.s * p.num_q_heads + (int64_t)w.un.h * G;
+    for (int e = threadIdx.x; e < G * D; e += kThreads) {
+        const int h = e / D, dd = e - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) M = fmaxf(M, uml[k * G + h].x);
+        float lsum = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int k = 0; k < kWarps; ++k) {
+                const float2 ml = uml[k * G + h];
+                if (ml.x != -INFINITY) {
+                    const float f = fast_exp2(ml.x - M);
+                    lsum = fmaf(ml.y, f, lsum);
+                    o = fmaf(uacc[(k * G + h) * D + dd], f, o);
+                }
+            }
         }
-    } else {
-        static_assert(kBytes == 4 && sizeof(T) == 2, "4-byte PV loads are bf16 pairs");
-        f[0] = bf16x2_to_float2(*reinterpret_cast<const uint32_t *>(src));
+        if (single) {
+            store_out<T>(p.out, (head0 + h) * D + dd, lsum > 0.f ? o / lsum : 0.f);
+        } else {
+            const int64_t row = (head0 + h) * p.max_parts + w.un.part;
+            p.ws_acc[row * D + dd] = o;
+            if (dd == 0) p.ws_ml[row] = make_float2(M, lsum);
+        }
     }
 }
+
+// ------------------------------------------------------------- bf16 block
+// Per-warp state of the tensor-core path.  m, l: online-softmax state of this
+// thread's two head columns 2*(lane%4) and 2*(lane%4)+1; o: O^T accumulator
+// fragments (rows = head dims, cols = heads); qb: Q^T operand fragments.
+template <int D>
+struct MmaState {
+    float m[2], l[2];
+    float o[D / 16][4];
+    uint32_t qb[D / 16][2];
+};
+
+// One 16-token block on tensor-core tiles.  kb: shared address of the K slab
+// (V slab follows), rows of 2*D bytes with swizzled 16-byte chunks.
+template <int D>
+__device__ __forceinline__ void mma_block(uint32_t kb, unsigned char *vgen, int ntok,
+                                          MmaState<D> &st, float sl2, int lane) {
+    constexpr int KS = D / 16;
+    constexpr int kRow = 2 * D;
+    const uint32_t vb = kb + kBlockSize * kRow;
+    const int mat = lane >> 3, r8 = lane & 7;
+    auto addr = [&](uint32_t base, int row, int chunk) {
+        return base + row * kRow + ((((chunk & ~7) | ((chunk ^ row) & 7))) << 4);
+    };
+    // S^T = K Q^T: rows = tokens, cols = heads (two accumulators halve the chain)
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    const int krow = ((mat & 1) << 3) + r8;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(a, addr(kb, krow, kk * 2 + (mat >> 1)));
+        if (kk & 1) mma_bf16_16816(sb, a, st.qb[kk][0], st.qb[kk][1]);
+        else mma_bf16_16816(sa, a, st.qb[kk][0], st.qb[kk][1]);
+    }
+    float s[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s[k] = (sa[k] + sb[k]) * sl2;
+    const int t0 = lane >> 2;
+    if (t0 >= ntok) s[0] = s[1] = -INFINITY;
+    if (t0 + 8 >= ntok) s[2] = s[3] = -INFINITY;
+    // online softmax per head column over the block's tokens
+    float c0 = fmaxf(s[0], s[2]), c1 = fmaxf(s[1], s[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        c0 = fmaxf(c0, __shfl_xor_sync(kFull, c0, off));
+        c1 = fmaxf(c1, __shfl_xor_sync(kFull, c1, off));
+    }
+    const float mn0 = fmaxf(st.m[0], c0), mn1 = fmaxf(st.m[1], c1);
+    const float al0 = fast_exp2(st.m[0] - mn0), al1 = fast_exp2(st.m[1] - mn1);
+    const float p0 = fast_exp2(s[0] - mn0), p1 = fast_exp2(s[1] - mn1);
+    const float p2 = fast_exp2(s[2] - mn0), p3 = fast_exp2(s[3] - mn1);
+    float r0 = p0 + p2, r1 = p1 + p3;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        r0 += __shfl_xor_sync(kFull, r0, off);
+        r1 += __shfl_xor_sync(kFull, r1, off);
+    }
+    st.l[0] = st.l[0] * al0 + r0;
+    st.l[1] = st.l[1] * al1 + r1;
+    st.m[0] = mn0;
+    st.m[1] = mn1;
+    if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            st.o[mt][0] *= al0;
+            st.o[mt][1] *= al1;
+            st.o[mt][2] *= al0;
+            st.o[mt][3] *= al1;
+        }
+    }
+    // P^T operand fragments: rows 0-7 / 8-15 of S^T, transposed in registers
+    const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
+    if (ntok < kBlockSize) {
+        // zero the V rows past the context: 0 * (NaN or Inf) would poison the sums
+        for (int idx = lane; idx < (kBlockSize - ntok) * (kRow / 16); idx += 32)
+            *reinterpret_cast<uint4 *>(vgen + (ntok + idx / (kRow / 16)) * kRow + (idx % (kRow / 16)) * 16) =
+                make_uint4(0, 0, 0, 0);
+        __syncwarp();
+    }
+    // O^T += V^T P^T: rows = head dims, cols = heads
+    const int vrow = ((mat >> 1) << 3) + r8;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_trans(a, addr(vb, vrow, mt * 2 + (mat & 1)));
+        mma_bf16_16816(st.o[mt], a, pb0, pb1);
+    }
+}
+
+// ------------------------------------------------------------- fp32 block
+template <int D, int G>
+struct F32Cfg {
+    static constexpr int kRowBytes = D * 4;
+    static constexpr int kQkChunks = kRowBytes / 128;   // 16-byte chunks per lane (8 lanes/token)
+    static constexpr int kQkPairs = kQkChunks * 2;      // float2 of q per head per lane
+    static constexpr int kDpl = D / 32;                 // PV dims per lane
+    static constexpr int kPvPairs = kDpl / 2;
+    static constexpr int kLogG = ilog2(G);
+    static constexpr int kDupMask = (8 >> kLogG) - 1;  // lanes holding the same score
+};
+
+template <int D, int G>
+struct F32State {
+    float m, l;
+    float2 acc[G][F32Cfg<D, G>::kPvPairs];
+    float2 qreg[G][F32Cfg<D, G>::kQkPairs];
+};
 
 // Transposing reduction over the 8 lanes of one token (lanes differing in bits
 // 0..2).  Lane holds N partial sums (one per head); each level halves the set,
@@ -224,15 +415,10 @@ __device__ __forceinline__ float reduce8(float *w, int part) {
     }
 }
 
-// One 16-token block for one consumer warp: QK, online-softmax update, PV.
-template <typename T, int D, int G>
-__device__ __forceinline__ void process_block(const unsigned char *kb, const unsigned char *vb,
-                                              int ntok,
-                                              const float2 (&qreg)[G][Cfg<T, D, G>::kQkPairs],
-                                              float &m, float &l,
-                                              float2 (&acc)[G][Cfg<T, D, G>::kPvPairs],
-                                              float *pw, int lane) {
-    using C = Cfg<T, D, G>;
+template <int D, int G>
+__device__ __forceinline__ void f32_block(const unsigned char *kb, const unsigned char *vb, int ntok,
+                                          F32State<D, G> &st, float *pw, int lane) {
+    using C = F32Cfg<D, G>;
     const int tq = lane >> 3, part = lane & 7;
     const int hd = part >> (3 - C::kLogG);
     float sc[4];
@@ -244,15 +430,12 @@ __device__ __forceinline__ void process_block(const unsigned char *kb, const uns
         for (int h = 0; h < G; ++h) a[h] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int i = 0; i < C::kQkChunks; ++i) {
-            const uint4 raw =
-                *reinterpret_cast<const uint4 *>(kb + t * C::kRowBytes + (part + 8 * i) * 16);
-            float2 kv[C::kEpc / 2];
-            unpack16<T>(raw, kv);
+            const float4 kv = *reinterpret_cast<const float4 *>(kb + t * C::kRowBytes + (part + 8 * i) * 16);
 #pragma unroll
-            for (int h = 0; h < G; ++h)
-#pragma unroll
-                for (int k = 0; k < C::kEpc / 2; ++k)
-                    a[h] = ffma2(qreg[h][i * (C::kEpc / 2) + k], kv[k], a[h]);
+            for (int h = 0; h < G; ++h) {
+                a[h] = ffma2(st.qreg[h][2 * i], make_float2(kv.x, kv.y), a[h]);
+                a[h] = ffma2(st.qreg[h][2 * i + 1], make_float2(kv.z, kv.w), a[h]);
+            }
         }
         float v[G];
 #pragma unroll
@@ -260,12 +443,11 @@ __device__ __forceinline__ void process_block(const unsigned char *kb, const uns
         const float s = reduce8<G, 2>(v, part);
         sc[r] = t < ntok ? s : -INFINITY;
     }
-    // online softmax for head hd over the block's 16 tokens
     float bm = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
     bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 8));
     bm = fmaxf(bm, __shfl_xor_sync(kFull, bm, 16));
-    const float m_new = fmaxf(m, bm);
-    const float alpha = fast_exp2(m - m_new);
+    const float m_new = fmaxf(st.m, bm);
+    const float alpha = fast_exp2(st.m - m_new);
     float ps = 0.f;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -274,308 +456,221 @@ __device__ __forceinline__ void process_block(const unsigned char *kb, const uns
     }
     ps += __shfl_xor_sync(kFull, ps, 8);
     ps += __shfl_xor_sync(kFull, ps, 16);
-    l = l * alpha + ps;
-    m = m_new;
+    st.l = st.l * alpha + ps;
+    st.m = m_new;
     if ((part & C::kDupMask) == 0) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) pw[(tq + 4 * r) * G + hd] = sc[r];
         if (tq == 0) pw[16 * G + hd] = alpha;
     }
     __syncwarp();
-    // PV
 #pragma unroll
     for (int h = 0; h < G; ++h) {
         const float al = pw[16 * G + h];
 #pragma unroll
         for (int k = 0; k < C::kPvPairs; ++k) {
-            acc[h][k].x *= al;
-            acc[h][k].y *= al;
+            st.acc[h][k].x *= al;
+            st.acc[h][k].y *= al;
         }
     }
-    const unsigned char *vrow = vb + lane * C::kPvBytes;
+    const unsigned char *vrow = vb + lane * C::kDpl * 4;
 #pragma unroll
     for (int t = 0; t < kBlockSize; ++t) {
         if (t < ntok) {
             float2 vv[C::kPvPairs];
-            load_pv<T, C::kPvBytes>(vrow + t * C::kRowBytes, vv);
-            float pt[G];
-            if constexpr (G >= 4) {
-#pragma unroll
-                for (int h = 0; h < G; h += 4) {
-                    const float4 p4 = *reinterpret_cast<const float4 *>(pw + t * G + h);
-                    pt[h] = p4.x; pt[h + 1] = p4.y; pt[h + 2] = p4.z; pt[h + 3] = p4.w;
-                }
+            if constexpr (C::kPvPairs == 2) {
+                const float4 x = *reinterpret_cast<const float4 *>(vrow + t * C::kRowBytes);
+                vv[0] = make_float2(x.x, x.y);
+                vv[1] = make_float2(x.z, x.w);
             } else {
-#pragma unroll
-                for (int h = 0; h < G; ++h) pt[h] = pw[t * G + h];
+                vv[0] = *reinterpret_cast<const float2 *>(vrow + t * C::kRowBytes);
             }
 #pragma unroll
-            for (int h = 0; h < G; ++h)
+            for (int h = 0; h < G; ++h) {
+                const float pt = pw[t * G + h];
 #pragma unroll
                 for (int k = 0; k < C::kPvPairs; ++k)
-                    acc[h][k] = ffma2(make_float2(pt[h], pt[h]), vv[k], acc[h][k]);
+                    st.acc[h][k] = ffma2(make_float2(pt, pt), vv[k], st.acc[h][k]);
+            }
         }
     }
     __syncwarp();  // pw is rewritten by the next block
 }
 
-template <typename T>
-__device__ __forceinline__ void store_out(void *out, int64_t idx, float v);
-template <>
-__device__ __forceinline__ void store_out<float>(void *out, int64_t idx, float v) {
-    static_cast<float *>(out)[idx] = v;
-}
-template <>
-__device__ __forceinline__ void store_out<__nv_bfloat16>(void *out, int64_t idx, float v) {
-    static_cast<__nv_bfloat16 *>(out)[idx] = __float2bfloat16_rn(v);
-}
-
+// ------------------------------------------------------------- the kernel
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(Cfg<T, D, G>::kThreads, 1) decode_kernel(const Params p) {
-    using C = Cfg<T, D, G>;
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
+    using Lay = Layout<T, D, G>;
+    constexpr bool kMma = sizeof(T) == 2;
+    constexpr int NS = Lay::kStagesPerWarp;
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *ring = smem + C::kOffRing;
-    unsigned char *qbuf = smem + C::kOffQ;
-    float *pbuf = reinterpret_cast<float *>(smem + C::kOffP);
-    float *macc = reinterpret_cast<float *>(smem + C::kOffMacc);
-    float2 *mml = reinterpret_cast<float2 *>(smem + C::kOffMml);
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
-    uint64_t *empty = full + C::kStages;
-    uint64_t *qfull = empty + C::kStages;  // [2]
-    uint64_t *qempty = qfull + 2;          // [2]
-    int *slot_ok = reinterpret_cast<int *>(smem + C::kOffSlotOk);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kOffAbort);
-    int *cum = reinterpret_cast<int *>(smem + C::kOffCum);
+    float *pbuf = reinterpret_cast<float *>(smem + Lay::kOffP);
+    float *macc = reinterpret_cast<float *>(smem + Lay::kOffMacc);
+    float2 *mml = reinterpret_cast<float2 *>(smem + Lay::kOffMml);
+    int *cum = reinterpret_cast<int *>(smem + Lay::kOffCum);
 
+    prologue(p, cum, reinterpret_cast<int *>(macc));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.num_seqs, hkv = p.num_kv_heads;
-    const bool split = p.part_tokens > 0;
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < C::kStages; ++i) {
-            mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&qfull[b], 1);
-            mbar_init(&qempty[b], C::kConsumerWarps);
-        }
-        *abort_flag = 0;
-        mbar_init_fence();
-    }
-    // cum[s] = sum_{s' < s} (parts(s') - 1): exclusive scan, one chunk per thread.
-    if (split) {
-        const int nthr = C::kThreads;
-        const int per = (S + nthr - 1) / nthr;
-        const int beg = min(S, (int)threadIdx.x * per), end = min(S, beg + per);
-        int local = 0;
-        for (int s = beg; s < end; ++s) {
-            const int L = checked_len(p, s);
-            local += num_parts(p, L < 0 ? 0 : L) - 1;
-        }
-        // scan the per-thread totals: warp inclusive scan, then across warps
-        int incl = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += y;
-        }
-        int *wsum = reinterpret_cast<int *>(pbuf);  // scratch before pbuf's first use
-        if (lane == 31) wsum[warp] = incl;
-        __syncthreads();
-        int off = 0;
-        for (int w = 0; w < warp; ++w) off += wsum[w];
-        int run = off + incl - local;
-        for (int s = beg; s < end; ++s) {
-            cum[s] = run;
-            const int L = checked_len(p, s);
-            run += num_parts(p, L < 0 ? 0 : L) - 1;
-        }
-        if ((int)threadIdx.x == nthr - 1) cum[S] = run;
-    }
-    __syncthreads();
-
     const int64_t units_first = (int64_t)S * hkv;
-    const int64_t total = units_first + (split ? (int64_t)cum[S] * hkv : 0);
-    const int hq_total = p.num_q_heads;
+    const int64_t total = units_first + (p.part_tokens > 0 ? (int64_t)cum[S] * hkv : 0);
+    unsigned char *wring = smem + Lay::kOffRing + (size_t)warp * NS * Lay::kStageBytes;
+    const uint32_t wring_s = smem_u32(wring);
+    float *pw = pbuf + warp * Lay::kPWarpFloats;
+    const int q4 = lane & 3, dr = lane >> 2;
 
-    if (warp == C::kConsumerWarps) {
-        // ------------------------------------------------------------ producer
-        int64_t gq = 0, issued = 0;
-        int uc = 0, q_issued = 0;
-        for (int64_t u = blockIdx.x; u < total; u += gridDim.x, ++uc) {
-            const Unit un = unit_of(u, units_first, hkv, cum, S);
-            int L = checked_len(p, un.s);
-            if (L < 0) {
-                if (lane == 0 && un.part == 0 && un.h == 0) flag_error(p.err, PA_DEVERR_CONTEXT_LEN);
-                L = 0;
-            }
-            int t0, nt;
-            unit_range(p, un, L, t0, nt);
-            const int nb = (nt + kBlockSize - 1) / kBlockSize;
-            const int b = uc & 1;
-            if (lane == 0 && !*abort_flag) {
-                bool ok = true;
-                if (uc >= 2) ok = mbar_wait_bounded(&qempty[b], ((uc >> 1) - 1) & 1, abort_flag, p.err);
-                if (ok) {
-                    const uint32_t qbytes = G * C::kRowBytes;
-                    mbar_arrive_expect_tx(&qfull[b], qbytes);
-                    bulk_g2s(qbuf + b * qbytes,
-                             p.q + ((int64_t)un.s * hq_total + (int64_t)un.h * G) * C::kRowBytes,
-                             qbytes, &qfull[b]);
-                    q_issued = uc + 1;
-                }
-            }
-            const int32_t *trow = p.tables + (int64_t)un.s * p.max_blocks + t0 / kBlockSize;
-            for (int jc = 0; jc < nb; jc += 32) {
-                const int j = jc + lane;
-                const int phys = j < nb ? __ldg(trow + j) : 0;
-                const int cnt = min(32, nb - jc);
-                for (int jj = 0; jj < cnt; ++jj, ++gq) {
-                    const int blk = __shfl_sync(kFull, phys, jj);
-                    if (lane == 0 && !*abort_flag) {
-                        const int slot = (int)(gq % C::kStages);
-                        if (gq >= C::kStages &&
-                            !mbar_wait_bounded(&empty[slot], (uint32_t)((gq / C::kStages - 1) & 1),
-                                               abort_flag, p.err))
-                            continue;
-                        const bool ok = blk >= 0 && blk < p.num_blocks;
-                        slot_ok[slot] = ok;
-                        if (ok) {
-                            const int64_t off = ((int64_t)blk * hkv + un.h) * C::kSlabBytes;
-                            unsigned char *dst = ring + (size_t)slot * C::kStageBytes;
-                            mbar_arrive_expect_tx(&full[slot], 2 * C::kSlabBytes);
-                            bulk_g2s(dst, p.kc + off, C::kSlabBytes, &full[slot]);
-                            bulk_g2s(dst + C::kSlabBytes, p.vc + off, C::kSlabBytes, &full[slot]);
-                        } else {
-                            flag_error(p.err, PA_DEVERR_BLOCK_ID);
-                            mbar_arrive(&full[slot]);
-                        }
-                        issued = gq + 1;
-                    }
-                }
-            }
-        }
-        // After an abort, wait for copies that may still be landing in our smem.
-        if (lane == 0 && *abort_flag) {
-            for (int64_t g = issued > C::kStages ? issued - C::kStages : 0; g < issued; ++g)
-                mbar_wait_drain(&full[g % C::kStages], (uint32_t)((g / C::kStages) & 1));
-            for (int k = q_issued > 2 ? q_issued - 2 : 0; k < q_issued; ++k)
-                mbar_wait_drain(&qfull[k & 1], (uint32_t)((k >> 1) & 1));
-        }
-        return;
-    }
+    // table entry of logical block j of a unit (the first 32 come from registers)
+    auto phys_of = [&](const WarpUnit &w, int j) {
+        const int v = __shfl_sync(kFull, w.tab, j & 31);
+        return j < 32 ? v : __ldg(w.trow + j);
+    };
+    // issue one block into stage `stg`; returns whether the block id was valid
+    auto issue = [&](const WarpUnit &w, int j, int stg) {
+        const int blk = phys_of(w, j);
+        const bool ok = blk >= 0 && blk < p.num_blocks;
+        if (ok) issue_slabs<T, D, G>(p, wring_s + stg * Lay::kStageBytes, blk, w.un.h, lane);
+        else if (lane == 0) flag_error(p.err, PA_DEVERR_BLOCK_ID);
+        cp_async_commit();
+        return ok;
+    };
 
-    // -------------------------------------------------------------- consumers
-    float *pw = pbuf + warp * C::kPWarpFloats;
-    const int tq = lane >> 3, part = lane & 7;
-    const int hd = part >> (3 - C::kLogG);
-    int64_t gq = 0;
+    WarpUnit cur, nxt;
+    int64_t u = blockIdx.x;
+    if (u >= total) return;
+    load_unit(p, u, units_first, cum, cur, lane, warp == 0);
+    bool have_nxt = u + gridDim.x < total;
+    if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
+    int stg = 0;
+    bool pre = false, pre_ok = false;  // cur's first block for this warp already in flight?
     int uc = 0;
-    for (int64_t u = blockIdx.x; u < total; u += gridDim.x, ++uc) {
-        const Unit un = unit_of(u, units_first, hkv, cum, S);
-        int L = checked_len(p, un.s);
-        if (L < 0) L = 0;
-        int t0, nt;
-        unit_range(p, un, L, t0, nt);
-        const int nb = (nt + kBlockSize - 1) / kBlockSize;
-        const int b = uc & 1;
-
-        bool live = !*abort_flag;
-        if (live) live = mbar_wait_bounded(&qfull[b], (uint32_t)((uc >> 1) & 1), abort_flag, p.err);
-        live = __all_sync(kFull, live);
-        float2 qreg[G][C::kQkPairs];
-        if (live) {
-            const unsigned char *qs = qbuf + b * G * C::kRowBytes;
+    for (;; ++uc) {
+        // ---- q operands of this unit (tiny, L2 resident)
+        MmaState<D> ms;
+        F32State<D, G> fs;
+        const unsigned char *qg =
+            p.q + ((int64_t)cur.un.s * p.num_q_heads + (int64_t)cur.un.h * G) * Lay::kRowBytes;
+        if constexpr (kMma) {
+            const bool hv = dr < G;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int d0 = kk * 16 + 2 * q4;
+                ms.qb[kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qg + dr * Lay::kRowBytes + d0 * 2)) : 0u;
+                ms.qb[kk][1] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qg + dr * Lay::kRowBytes + (d0 + 8) * 2)) : 0u;
+            }
+            ms.m[0] = ms.m[1] = -INFINITY;
+            ms.l[0] = ms.l[1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) ms.o[mt][0] = ms.o[mt][1] = ms.o[mt][2] = ms.o[mt][3] = 0.f;
+        } else {
+            using C = F32Cfg<D, G>;
+            const int part = lane & 7;
 #pragma unroll
             for (int h = 0; h < G; ++h)
 #pragma unroll
                 for (int i = 0; i < C::kQkChunks; ++i) {
-                    const uint4 raw =
-                        *reinterpret_cast<const uint4 *>(qs + h * C::kRowBytes + (part + 8 * i) * 16);
-                    float2 f[C::kEpc / 2];
-                    unpack16<T>(raw, f);
-#pragma unroll
-                    for (int k = 0; k < C::kEpc / 2; ++k)
-                        qreg[h][i * (C::kEpc / 2) + k] =
-                            make_float2(f[k].x * p.scale_log2, f[k].y * p.scale_log2);
+                    const float4 x = __ldg(reinterpret_cast<const float4 *>(qg + h * C::kRowBytes + (part + 8 * i) * 16));
+                    fs.qreg[h][2 * i] = make_float2(x.x * p.scale_log2, x.y * p.scale_log2);
+                    fs.qreg[h][2 * i + 1] = make_float2(x.z * p.scale_log2, x.w * p.scale_log2);
                 }
+            fs.m = -INFINITY;
+            fs.l = 0.f;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int k = 0; k < C::kPvPairs; ++k) fs.acc[h][k] = make_float2(0.f, 0.f);
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&qempty[b]);
 
-        float m = -INFINITY, l = 0.f;
-        float2 acc[G][C::kPvPairs];
-#pragma unroll
-        for (int h = 0; h < G; ++h)
-#pragma unroll
-            for (int k = 0; k < C::kPvPairs; ++k) acc[h][k] = make_float2(0.f, 0.f);
-
-        for (int j = warp; j < nb; j += C::kConsumerWarps) {
-            const int64_t g = gq + j;
-            const int slot = (int)(g % C::kStages);
-            if (live)
-                live = mbar_wait_bounded(&full[slot], (uint32_t)((g / C::kStages) & 1), abort_flag,
-                                         p.err);
-            live = __all_sync(kFull, live);
-            if (live && slot_ok[slot]) {
-                const int ntok = min(kBlockSize, nt - j * kBlockSize);
-                const unsigned char *kb = ring + (size_t)slot * C::kStageBytes;
-                process_block<T, D, G>(kb, kb + C::kSlabBytes, ntok, qreg, m, l, acc, pw, lane);
+        // ---- this warp's blocks of the unit, one always in flight ahead
+        bool cur_ok = pre_ok;
+        if (cur.nb > warp && !pre) cur_ok = issue(cur, warp, stg);
+        bool next_pre = false, next_ok = false;
+        for (int j = warp; j < cur.nb; j += kWarps) {
+            bool ok_next = false;
+            if constexpr (NS == 2) {
+                if (j + kWarps < cur.nb) {
+                    ok_next = issue(cur, j + kWarps, stg ^ 1);
+                } else if (have_nxt && nxt.nb > warp) {
+                    next_ok = issue(nxt, warp, stg ^ 1);
+                    next_pre = true;
+                } else {
+                    cp_async_commit();
+                }
+                cp_async_wait<1>();
+            } else {
+                cp_async_wait<0>();
             }
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[slot]);
+            if (cur_ok) {
+                const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
+                if constexpr (kMma)
+                    mma_block<D>(wring_s + stg * Lay::kStageBytes,
+                                 wring + stg * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
+                                 p.scale_log2, lane);
+                else
+                    f32_block<D, G>(wring + stg * Lay::kStageBytes,
+                                    wring + stg * Lay::kStageBytes + Lay::kSlabBytes, ntok, fs, pw, lane);
+            }
+            __syncwarp();
+            if constexpr (NS == 2) {
+                stg ^= 1;
+                cur_ok = ok_next;
+            } else if (j + kWarps < cur.nb) {
+                cur_ok = issue(cur, j + kWarps, stg);
+            }
         }
-        gq += nb;
+        if constexpr (NS == 1) {
+            if (have_nxt && nxt.nb > warp) {  // single stage: next unit's first block now
+                next_ok = issue(nxt, warp, stg);
+                next_pre = true;
+            }
+        }
 
-        // merge the consumer warps' partial states for this unit
-        float *wacc = macc + ((size_t)b * C::kConsumerWarps + warp) * G * D;
-        float2 *wml = mml + ((size_t)b * C::kConsumerWarps + warp) * G;
+        // ---- merge the warps' states for this unit
+        const int b = uc & 1;
+        float *wacc = macc + ((size_t)b * kWarps + warp) * G * D;
+        float2 *wml = mml + ((size_t)b * kWarps + warp) * G;
+        if constexpr (kMma) {
 #pragma unroll
-        for (int h = 0; h < G; ++h)
+            for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
-            for (int k = 0; k < C::kPvPairs; ++k)
-                *reinterpret_cast<float2 *>(wacc + h * D + lane * C::kDpl + 2 * k) = acc[h][k];
-        if (tq == 0 && (part & C::kDupMask) == 0) wml[hd] = make_float2(m, l);
-        named_barrier(1, C::kConsumerWarps * 32);
-        if (*abort_flag) continue;
-
-        const float2 *uml = mml + (size_t)b * C::kConsumerWarps * G;
-        const float *uacc = macc + (size_t)b * C::kConsumerWarps * G * D;
-        const bool single = num_parts(p, L) == 1;
-        const int64_t head0 = (int64_t)un.s * hq_total + (int64_t)un.h * G;
-        for (int e = threadIdx.x; e < G * D; e += C::kConsumerWarps * 32) {
-            const int h = e / D, dd = e - h * D;
-            float M = -INFINITY;
-#pragma unroll
-            for (int w = 0; w < C::kConsumerWarps; ++w) M = fmaxf(M, uml[w * G + h].x);
-            float lsum = 0.f, o = 0.f;
-            if (M != -INFINITY) {
-#pragma unroll
-                for (int w = 0; w < C::kConsumerWarps; ++w) {
-                    const float2 ml = uml[w * G + h];
-                    if (ml.x != -INFINITY) {
-                        const float f = fast_exp2(ml.x - M);
-                        lsum = fmaf(ml.y, f, lsum);
-                        o = fmaf(uacc[(w * G + h) * D + dd], f, o);
-                    }
+                for (int half = 0; half < 2; ++half) {
+                    const int d = mt * 16 + dr + 8 * half;
+                    if (2 * q4 < G) wacc[(2 * q4) * D + d] = ms.o[mt][2 * half];
+                    if (2 * q4 + 1 < G) wacc[(2 * q4 + 1) * D + d] = ms.o[mt][2 * half + 1];
                 }
+            if (dr == 0) {
+                if (2 * q4 < G) wml[2 * q4] = make_float2(ms.m[0], ms.l[0]);
+                if (2 * q4 + 1 < G) wml[2 * q4 + 1] = make_float2(ms.m[1], ms.l[1]);
             }
-            if (single) {
-                store_out<T>(p.out, (head0 + h) * D + dd, lsum > 0.f ? o / lsum : 0.f);
-            } else {
-                const int64_t row = (head0 + h) * p.max_parts + un.part;
-                p.ws_acc[row * D + dd] = o;
-                if (dd == 0) p.ws_ml[row] = make_float2(M, lsum);
-            }
+        } else {
+            using C = F32Cfg<D, G>;
+            const int tq = lane >> 3, part = lane & 7;
+#pragma unroll
+            for (int h = 0; h < G; ++h)
+#pragma unroll
+                for (int k = 0; k < C::kPvPairs; ++k)
+                    *reinterpret_cast<float2 *>(wacc + h * D + lane * C::kDpl + 2 * k) = fs.acc[h][k];
+            if (tq == 0 && (part & C::kDupMask) == 0) wml[part >> (3 - C::kLogG)] = make_float2(fs.m, fs.l);
         }
+        __syncthreads();
+        finish_unit<T, D, G>(p, cur, macc + (size_t)b * kWarps * G * D, mml + (size_t)b * kWarps * G);
+
+        // ---- advance
+        u += gridDim.x;
+        if (!have_nxt) break;
+        cur = nxt;
+        pre = next_pre;
+        pre_ok = next_ok;
+        have_nxt = u + gridDim.x < total;
+        if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
     }
+    cp_async_wait<0>();
 }
 
 // Combine split-K partials: one warp per (sequence, query head) with more than
 // one partition.  M = max_p m_p; out = sum_p 2^(m_p-M) acc_p / sum_p 2^(m_p-M) l_p.
 template <typename T, int D>
-__global__ void __launch_bounds__(128) reduce_kernel(const Params p) {
+__global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Params p) {
     constexpr int kDpl = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -615,20 +710,20 @@ __global__ void __launch_bounds__(128) reduce_kernel(const Params p) {
 
 template <typename T, int D, int G>
 cudaError_t launch_t(const DecodeLaunch &a, const Params &prm, cudaStream_t stream) {
-    using C = Cfg<T, D, G>;
+    using Lay = Layout<T, D, G>;
     const bool split = prm.part_tokens > 0;
-    const size_t smem = C::smem_bytes(split ? a.num_seqs + 1 : 0);
+    const size_t smem = Lay::smem_bytes(split ? a.num_seqs + 1 : 0);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    static_assert(C::smem_bytes(kMaxSplitSeqs + 1) <= 232448, "decode smem over the sm_100 limit");
+    static_assert(Lay::smem_bytes(kMaxSplitSeqs + 1) <= 232448, "decode smem over the sm_100 limit");
     e = cudaFuncSetAttribute(decode_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)C::smem_bytes(kMaxSplitSeqs + 1));
+                             (int)Lay::smem_bytes(kMaxSplitSeqs + 1));
     if (e != cudaSuccess) return e;
     int64_t grid = num_sms(dev);
     if (!split) grid = std::min<int64_t>(grid, (int64_t)a.num_seqs * a.cache.num_kv_heads);
     if (grid < 1) grid = 1;
-    decode_kernel<T, D, G><<<(unsigned)grid, C::kThreads, smem, stream>>>(prm);
+    decode_kernel<T, D, G><<<(unsigned)grid, kThreads, smem, stream>>>(prm);
     e = cudaGetLastError();
     if (e != cudaSuccess || !split) return e;
     const int64_t warps = (int64_t)a.num_seqs * a.num_q_heads;
@@ -651,6 +746,7 @@ cudaError_t launch_g(const DecodeLaunch &a, const Params &prm, cudaStream_t stre
 
 cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
     Params prm;
+    std::memset(&prm, 0, sizeof(prm));
     prm.q = static_cast<const unsigned char *>(a.query);
     prm.kc = static_cast<const unsigned char *>(a.key_cache);
     prm.vc = static_cast<const unsigned char *>(a.value_cache);
