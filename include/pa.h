@@ -161,6 +161,33 @@ PA_API pa_status pa_decode(const void *query, const void *key_cache, const void 
                     int32_t *err_flag, void *stream);
 
 /*
+ * pa_decode with its split-K scratch taken from a fixed array inside the library
+ * instead of a caller-provided workspace.  The pages have no counterpart: this
+ * exists for callers that cannot allocate device memory -- code running inside an
+ * allocator's callbacks, in a process whose device memory is owned and capped by
+ * another framework, or in a plugin handed only the step's tensors.  Arguments and
+ * results are those of pa_decode without workspace/workspace_bytes.
+ * Limit: pa_decode_workspace_size(num_seqs, num_q_heads, head_dim,
+ * max_context_len, partition_size) must be <= PA_DECODE_STATIC_SCRATCH_BYTES
+ * (32 MiB), else PA_ERR_UNSUPPORTED and nothing is launched.  Every GPU that loads
+ * the library holds that array until the process exits.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make it before any stream capture.  No allocation happens.
+ * All calls share the one array and it keeps the last call's contents; nothing in
+ * it needs to start at zero.  Calls whose kernels overlap on the GPU (different
+ * streams, no ordering between them) race on the array and give wrong results:
+ * order them on one stream or with events.
+ */
+#define PA_DECODE_STATIC_SCRATCH_BYTES (32u << 20)
+PA_API pa_status pa_decode_static_scratch(const void *query, const void *key_cache,
+                                          const void *value_cache, const int32_t *block_tables,
+                                          int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                          int32_t max_context_len, int32_t num_seqs,
+                                          int32_t num_q_heads, float scale, int32_t partition_size,
+                                          void *out, const pa_cache_desc *cache, int32_t *err_flag,
+                                          void *stream);
+
+/*
  * Causal chunked prefill against the paged cache.  Sequence s has
  * C_s = chunk_lens[s] new query rows, the last C_s positions of its context of
  * L_s = context_lens[s] tokens (their K/V already written with pa_cache_write).
