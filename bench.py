@@ -5,7 +5,7 @@ sequences in 16 groups of 16 sharing a 512-token prefix (32 shared blocks), priv
 lognormal suffixes (median 600, cap 8192), 32 query / 8 kv heads, head_dim 128,
 block_size 16.  One step = the whole decode hot path for one batch:
 pa_cache_write of the 256 new tokens' K/V through their slot mapping, then
-pa_decode over every sequence (split-K partitions of 512 tokens + LSE reduce).
+pa_decode over every sequence (split-K partitions of 1024 tokens + LSE reduce).
 
 Timed region: K steps after W warm-up steps, CUDA events on the launching stream,
 barrier + synchronize on both sides, max over ranks.  The step's inputs (1.1 GB of
@@ -37,7 +37,7 @@ sys.path.insert(0, ROOT)
 
 import workloads  # noqa: E402
 
-PARTITION = 512
+PARTITION = 1024
 CONFIG_ID = 3
 WORKLOAD_NAME = "llama3-8b-gqa-prefix-sharing-decode"
 

@@ -19,7 +19,7 @@
 //  * Each of the CTA's 8 warps takes logical blocks w, w+8, ... of a unit and
 //    streams them itself: the (block, kv head) slabs of K and V (4 KB each in
 //    bf16) are fetched with 16-byte cp.async, all 32 lanes issuing, into a
-//    two-stage per-warp ring, the next block (across unit boundaries) always in
+//    per-warp ring of stages, the next block (across unit boundaries) always in
 //    flight while the current one is computed.  Measured on B200: random 4 KB
 //    slabs stream at ~6.6-7 TB/s this way, while bulk copies issued by a single
 //    thread per SM cap near 0.9 TB/s (each copy costs the issuing thread
@@ -72,20 +72,31 @@ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Shared-memory carve-up (byte offsets from the dynamic shared memory base).
+// Each warp owns kStagesPerWarp ring stages (K slab + V slab each): two, or one
+// when a stage is too large (fp32, head_dim 128).  The merge buffers are
+// double-buffered when they fit, else single-buffered (one more CTA barrier per
+// unit).
 template <typename T, int D, int G>
 struct Layout {
     static constexpr int kElem = ElemBytes<T>::value;
     static constexpr int kRowBytes = D * kElem;                 // one token of one head
     static constexpr int kSlabBytes = kBlockSize * kRowBytes;   // one (block, kv head) slab
     static constexpr int kStageBytes = 2 * kSlabBytes;          // K slab + V slab
-    static constexpr int kStagesPerWarp = kStageBytes <= 8192 ? 2 : 1;
+    static constexpr size_t kLimit = 232448;                    // sm_100 max dynamic smem per CTA
+    static constexpr size_t kPBytes = sizeof(T) == 4 ? (size_t)kWarps * (16 * G + G) * 4 : 64;
+    static constexpr size_t kMergeBytes = (size_t)kWarps * G * (D * 4 + 8);
+    static constexpr size_t kFixed = kPBytes + 16 + (size_t)(kMaxSplitSeqs + 1) * 4 + 64;
+    static constexpr int stages_fit(int bufs) {
+        return (int)((kLimit - kFixed - bufs * kMergeBytes) / ((size_t)kWarps * kStageBytes));
+    }
+    static constexpr int kStagesPerWarp = stages_fit(2) >= 2 ? 2 : 1;
+    static constexpr int kMergeBufs = stages_fit(2) >= kStagesPerWarp ? 2 : 1;
+    static constexpr size_t kPWarpFloats = 16 * G + G;          // fp32 path: p[16][G], alpha[G]
     static constexpr size_t kOffRing = 0;
     static constexpr size_t kOffP = kOffRing + (size_t)kWarps * kStagesPerWarp * kStageBytes;
-    static constexpr size_t kPWarpFloats = 16 * G + G;          // fp32 path: p[16][G], alpha[G]
-    static constexpr size_t kOffMacc =
-        align_up(kOffP + (sizeof(T) == 4 ? (size_t)kWarps * kPWarpFloats * 4 : 64), 16);
-    static constexpr size_t kOffMml = kOffMacc + 2ull * kWarps * G * D * 4;
-    static constexpr size_t kOffCum = align_up(kOffMml + 2ull * kWarps * G * 8, 16);
+    static constexpr size_t kOffMacc = align_up(kOffP + kPBytes, 16);
+    static constexpr size_t kOffMml = kOffMacc + (size_t)kMergeBufs * kWarps * G * D * 4;
+    static constexpr size_t kOffCum = align_up(kOffMml + (size_t)kMergeBufs * kWarps * G * 8, 16);
     static constexpr size_t smem_bytes(int cum_entries) { return kOffCum + (size_t)cum_entries * 4; }
 };
 
@@ -498,6 +509,19 @@ __device__ __forceinline__ void f32_block(const unsigned char *kb, const unsigne
 }
 
 // ------------------------------------------------------------- the kernel
+// cp.async.wait_group with a run-time count (at most 3 groups pending here).
+__device__ __forceinline__ void cp_async_wait_dyn(int pending) {
+    if (pending <= 0) cp_async_wait<0>();
+    else if (pending == 1) cp_async_wait<1>();
+    else if (pending == 2) cp_async_wait<2>();
+    else cp_async_wait<3>();
+}
+
+// Blocks of the warp's work, one after another: blocks w, w+8, ... of the current
+// unit, then of the next one.  Each is fetched with cp.async up to NS items before
+// it is computed.  (An extra prefetch.global.L2 a few items further ahead measured
+// slower on B200 at every distance tried, as did a third stage per warp.)
+
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
     using Lay = Layout<T, D, G>;
@@ -519,31 +543,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     float *pw = pbuf + warp * Lay::kPWarpFloats;
     const int q4 = lane & 3, dr = lane >> 2;
 
-    // table entry of logical block j of a unit (the first 32 come from registers)
-    auto phys_of = [&](const WarpUnit &w, int j) {
-        const int v = __shfl_sync(kFull, w.tab, j & 31);
-        return j < 32 ? v : __ldg(w.trow + j);
-    };
-    // issue one block into stage `stg`; returns whether the block id was valid
-    auto issue = [&](const WarpUnit &w, int j, int stg) {
-        const int blk = phys_of(w, j);
-        const bool ok = blk >= 0 && blk < p.num_blocks;
-        if (ok) issue_slabs<T, D, G>(p, wring_s + stg * Lay::kStageBytes, blk, w.un.h, lane);
-        else if (lane == 0) flag_error(p.err, PA_DEVERR_BLOCK_ID);
-        cp_async_commit();
-        return ok;
-    };
-
     WarpUnit cur, nxt;
     int64_t u = blockIdx.x;
     if (u >= total) return;
     load_unit(p, u, units_first, cum, cur, lane, warp == 0);
     bool have_nxt = u + gridDim.x < total;
     if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
-    int stg = 0;
-    bool pre = false, pre_ok = false;  // cur's first block for this warp already in flight?
-    int uc = 0;
-    for (;; ++uc) {
+
+    // table entry of logical block j of a unit (the first 32 come from registers)
+    auto phys_of = [&](const WarpUnit &w, int j) {
+        const int v = __shfl_sync(kFull, w.tab, j & 31);
+        return j < 32 ? v : __ldg(w.trow + j);
+    };
+    // normalise a cursor (iu: 0 = cur, 1 = nxt) onto an existing item, skipping
+    // `steps` items; false when it runs past the next unit
+    auto walk = [&](int &iu, int &ij, int steps) {
+        for (;;) {
+            if (iu > 1 || (iu == 1 && !have_nxt)) return false;
+            const WarpUnit &w = iu ? nxt : cur;
+            if (ij >= w.nb) {
+                ++iu;
+                ij = warp;
+                continue;
+            }
+            if (steps == 0) return true;
+            ij += kWarps;
+            --steps;
+        }
+    };
+    int iss_u = 0, iss_j = warp;  // next item to fetch
+    int n_iss = 0, n_cmp = 0;     // items fetched / computed so far
+    uint32_t okmask = 0;          // per stage: block id was valid
+    auto fetch_one = [&]() {
+        if (!walk(iss_u, iss_j, 0)) return false;
+        const WarpUnit &w = iss_u ? nxt : cur;
+        const int stage = n_iss % NS;
+        const int blk = phys_of(w, iss_j);
+        const bool ok = blk >= 0 && blk < p.num_blocks;
+        if (ok) issue_slabs<T, D, G>(p, wring_s + stage * Lay::kStageBytes, blk, w.un.h, lane);
+        else if (lane == 0) flag_error(p.err, PA_DEVERR_BLOCK_ID);
+        cp_async_commit();
+        okmask = (okmask & ~(1u << stage)) | ((ok ? 1u : 0u) << stage);
+        iss_j += kWarps;
+        ++n_iss;
+        return true;
+    };
+
+    for (int uc = 0;; ++uc) {
         // ---- q operands of this unit (tiny, L2 resident)
         MmaState<D> ms;
         F32State<D, G> fs;
@@ -580,53 +626,32 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 for (int k = 0; k < C::kPvPairs; ++k) fs.acc[h][k] = make_float2(0.f, 0.f);
         }
 
-        // ---- this warp's blocks of the unit, one always in flight ahead
-        bool cur_ok = pre_ok;
-        if (cur.nb > warp && !pre) cur_ok = issue(cur, warp, stg);
-        bool next_pre = false, next_ok = false;
+        // ---- this warp's blocks of the unit, up to NS fetched ahead
         for (int j = warp; j < cur.nb; j += kWarps) {
-            bool ok_next = false;
-            if constexpr (NS == 2) {
-                if (j + kWarps < cur.nb) {
-                    ok_next = issue(cur, j + kWarps, stg ^ 1);
-                } else if (have_nxt && nxt.nb > warp) {
-                    next_ok = issue(nxt, warp, stg ^ 1);
-                    next_pre = true;
-                } else {
-                    cp_async_commit();
-                }
-                cp_async_wait<1>();
-            } else {
-                cp_async_wait<0>();
+            while (n_iss - n_cmp < NS && fetch_one()) {
             }
+            cp_async_wait_dyn(n_iss - n_cmp - 1);
             __syncwarp();
-            if (cur_ok) {
+            const int stage = n_cmp % NS;
+            if ((okmask >> stage) & 1u) {
                 const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
                 if constexpr (kMma)
-                    mma_block<D>(wring_s + stg * Lay::kStageBytes,
-                                 wring + stg * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
+                    mma_block<D>(wring_s + stage * Lay::kStageBytes,
+                                 wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
                                  p.scale_log2, lane);
                 else
-                    f32_block<D, G>(wring + stg * Lay::kStageBytes,
-                                    wring + stg * Lay::kStageBytes + Lay::kSlabBytes, ntok, fs, pw, lane);
+                    f32_block<D, G>(wring + stage * Lay::kStageBytes,
+                                    wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, fs, pw, lane);
             }
-            __syncwarp();
-            if constexpr (NS == 2) {
-                stg ^= 1;
-                cur_ok = ok_next;
-            } else if (j + kWarps < cur.nb) {
-                cur_ok = issue(cur, j + kWarps, stg);
-            }
+            __syncwarp();  // the stage may be refilled by the next fetch
+            ++n_cmp;
         }
-        if constexpr (NS == 1) {
-            if (have_nxt && nxt.nb > warp) {  // single stage: next unit's first block now
-                next_ok = issue(nxt, warp, stg);
-                next_pre = true;
-            }
+        // keep the pipeline full across the merge
+        while (n_iss - n_cmp < NS && fetch_one()) {
         }
 
         // ---- merge the warps' states for this unit
-        const int b = uc & 1;
+        const int b = Lay::kMergeBufs == 2 ? (uc & 1) : 0;
         float *wacc = macc + ((size_t)b * kWarps + warp) * G * D;
         float2 *wml = mml + ((size_t)b * kWarps + warp) * G;
         if constexpr (kMma) {
@@ -654,13 +679,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         __syncthreads();
         finish_unit<T, D, G>(p, cur, macc + (size_t)b * kWarps * G * D, mml + (size_t)b * kWarps * G);
+        if constexpr (Lay::kMergeBufs == 1) __syncthreads();  // buffer is rewritten next unit
 
-        // ---- advance
+        // ---- advance: the fetch cursor moves down one unit with the window
         u += gridDim.x;
         if (!have_nxt) break;
+        walk(iss_u, iss_j, 0);
         cur = nxt;
-        pre = next_pre;
-        pre_ok = next_ok;
+        iss_u = iss_u > 0 ? iss_u - 1 : 0;
         have_nxt = u + gridDim.x < total;
         if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
     }
