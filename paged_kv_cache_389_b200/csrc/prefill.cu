@@ -1,9 +1,452 @@
-// Chunked-prefill attention against the paged cache (tcgen05 tensor-core path).
+// Chunked-prefill attention against the paged KV cache on 5th-generation tensor
+// cores (tcgen05.mma, accumulators in tensor memory).
+//
+// What is computed (include/pa.h): sequence s has C_s query rows, the last C_s
+// positions of its L_s-token context; row i sits at position p = L_s - C_s + i
+// and attends to keys 0..p (causal), K/V read through the block table.
+// Sources: "vLLM 深度拆解" (chenxutan) 2.3 (prefill processes a whole prompt and is
+// compute bound) and 4.3/5.1 (long prompts are cut into chunks interleaved with
+// decode); devpress vLLM v0.6.x teardown, 核心代码拆解 (paged K/V via the table).
+//
+// Tile: one CTA computes a 128-row query tile of one (sequence, kv head): the g
+// query heads of that kv head are packed into the rows (row = chunk row * g +
+// head), so every K/V byte staged in shared memory serves all g heads.  The CTA
+// walks the keys in tiles of 128 (8 blocks of 16) up to the tile's last position.
+//   S   = Q K^T      tcgen05.mma kind::f16, M=128, N=128 keys, K=16 x 8, -> TMEM
+//   P   = softmax    online, fp32, one query row per thread (tcgen05.ld from TMEM)
+//   O  += P V        tcgen05.mma, A = P (bf16, smem), B = V (MN-major), -> TMEM
+// Warp roles: warps 0-3 load (16-byte cp.async into 128-byte-swizzled layouts:
+// Q and K K-major, V MN-major, the canonical layouts the MMA descriptors name),
+// warps 4-7 run the softmax (TMEM lanes 0..127), warp 8 owns the tensor memory
+// and issues the MMAs from one thread.  K/V tiles are double-buffered; the
+// stages are handed over with mbarriers; every wait is bounded and an abort
+// still frees the tensor memory.
+#include <cstring>
+
 #include "pa_common.cuh"
 #include "pa_launch.h"
 
 namespace pa {
+namespace {
 
-cudaError_t launch_prefill(const PrefillLaunch &, cudaStream_t) { return cudaErrorNotSupported; }
+constexpr unsigned kFull = 0xffffffffu;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kD = 128;              // head_dim (bf16 only)
+constexpr int kTileM = 128;          // query rows per CTA
+constexpr int kTileN = 128;          // keys per KV tile
+constexpr int kThreads = 9 * 32;     // 4 load warps, 4 softmax warps, 1 MMA warp
+constexpr int kMmaWarp = 8;
+constexpr uint32_t kTmemCols = 256;  // S: columns 0..127, O: 128..255
+
+// shared memory (offsets from a 1024-byte aligned base)
+constexpr uint32_t kHalf = kTileM * 128;           // one 64-column half of a 128-row tile
+constexpr uint32_t kTileBytes = 2 * kHalf;         // 32 KB
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kOffQ + kTileBytes;     // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTileBytes; // 2 stages
+constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffP + kTileBytes;
+constexpr uint32_t kOffTab = kOffBar + 16 * 8;     // 8 table entries per stage
+constexpr uint32_t kOffMisc = kOffTab + 2 * 8 * 4;
+constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
+
+struct Params {
+    const unsigned char *q;
+    const unsigned char *kc;
+    const unsigned char *vc;
+    const int32_t *tables;
+    const int32_t *lens;
+    const int32_t *chunks;
+    unsigned char *out;
+    int32_t *err;
+    int32_t max_blocks;
+    int32_t num_seqs;
+    int32_t max_chunk;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t num_blocks;
+    float scale_log2;
+};
+
+// ---- tcgen05 wrappers --------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t cols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(cols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: 128-byte swizzle, start/LBO/SBO in 16-byte units,
+// descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+    return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
+           ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M=128, N=128.
+constexpr uint32_t idesc_bf16(bool b_mn_major) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(kTileN >> 3) << 17) |
+           ((uint32_t)(kTileM >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk c (0..15) of row r in a 128-row tile stored as
+// two 64-column halves of 128-byte rows with the 128-byte swizzle.
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return (uint32_t)((c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Bounded mbarrier wait honouring the CTA abort flag (pa_common.cuh).
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *err) {
+    return mbar_wait_bounded(bar, parity, abort, err);
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    const uint32_t sbase = smem_u32(smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+    uint64_t *q_full = bars + 0;
+    uint64_t *kv_full = bars + 1;   // [2]
+    uint64_t *kv_empty = bars + 3;  // [2]
+    uint64_t *s_full = bars + 5;
+    uint64_t *p_full = bars + 6;
+    uint64_t *pv_done = bars + 7;
+    uint64_t *mma_idle = bars + 8;
+    int *tab = reinterpret_cast<int *>(smem + kOffTab);  // [2][8]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+
+    constexpr int kRowsPerTile = kTileM / G;  // chunk rows per query tile
+    const int s = blockIdx.z, h = blockIdx.y;
+    const int i0 = blockIdx.x * kRowsPerTile;
+    const int L = __ldg(p.lens + s), C = __ldg(p.chunks + s);
+    // validate once; an invalid sequence is skipped (flagged by its first tile)
+    if (C < 0 || C > p.max_chunk || C > L || (int64_t)L > (int64_t)p.max_blocks * kBlockSize) {
+        if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) flag_error(p.err, PA_DEVERR_CHUNK);
+        return;
+    }
+    if (i0 >= C) return;
+    const int start = L - C;
+    const int last_row = min(C, i0 + kRowsPerTile) - 1;
+    const int ntiles = (start + last_row + 1 + kTileN - 1) / kTileN;  // keys 0..start+last_row
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 128);
+        mbar_init(&kv_full[0], 128);
+        mbar_init(&kv_full[1], 128);
+        mbar_init(&kv_empty[0], 1);
+        mbar_init(&kv_empty[1], 1);
+        mbar_init(s_full, 1);
+        mbar_init(p_full, 128);
+        mbar_init(pv_done, 1);
+        mbar_init(mma_idle, 1);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
+    if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tS = tmem, tO = tmem + 128;
+    const int64_t head_stride = (int64_t)kD * 2;  // bytes per (row, head)
+
+    if (warp < 4) {
+        // ------------------------------------------------------------ loaders
+        const int t = threadIdx.x;  // 0..127
+        // Q tile: row m = (chunk row, head) pair; 16 chunks of 16 bytes per row
+        for (int idx = t; idx < kTileM * 16; idx += 128) {
+            const int m = idx >> 4, c = idx & 15;
+            const int i = i0 + m / G, hq = h * G + m % G;
+            const uint32_t dst = sbase + kOffQ + swz(m, c);
+            if (i < C)
+                cp_async16(dst, p.q + (((int64_t)s * p.max_chunk + i) * p.num_q_heads + hq) * head_stride + c * 16);
+            else
+                *reinterpret_cast<uint4 *>(smem + kOffQ + swz(m, c)) = make_uint4(0, 0, 0, 0);
+        }
+        cp_async_commit();
+        cp_async_wait<0>();
+        fence_proxy_async_smem();
+        mbar_arrive(q_full);
+        const int32_t *trow = p.tables + (int64_t)s * p.max_blocks;
+        volatile int *go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
+        for (int j = 0; j < ntiles; ++j) {
+            const int st = j & 1;
+            // one thread waits for the stage; the decision reaches all loaders
+            // through shared memory behind the barrier, so they break together
+            if (t == 0) *go = (j < 2 || wait_bar(&kv_empty[st], ((j >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
+            // table entries of the tile's 8 blocks (-1: past the context)
+            if (t < 8) {
+                const int b = j * 8 + t;
+                int e = -1;
+                if (b * kBlockSize < L) {
+                    e = __ldg(trow + b);
+                    if (e < 0 || e >= p.num_blocks) {
+                        flag_error(p.err, PA_DEVERR_BLOCK_ID);
+                        e = -1;
+                    }
+                }
+                tab[st * 8 + t] = e;
+            }
+            named_barrier(1, 128);
+            if (!*go) break;
+            const uint32_t kst = sbase + kOffK + st * kTileBytes, vst = sbase + kOffV + st * kTileBytes;
+            unsigned char *kgen = smem + kOffK + st * kTileBytes, *vgen = smem + kOffV + st * kTileBytes;
+            for (int idx = t; idx < kTileN * 16; idx += 128) {
+                const int n = idx >> 4, c = idx & 15;
+                const int key = j * kTileN + n;
+                const int blk = tab[st * 8 + (n >> 4)];
+                const uint32_t off = swz(n, c);
+                if (blk >= 0 && key < L) {
+                    const int64_t src = (((int64_t)blk * p.num_kv_heads + h) * kBlockSize + (n & 15)) * head_stride + c * 16;
+                    cp_async16(kst + off, p.kc + src);
+                    cp_async16(vst + off, p.vc + src);
+                } else {  // past the context or a bad id: zeros (0 * garbage must not reach the sums)
+                    *reinterpret_cast<uint4 *>(kgen + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(vgen + off) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            cp_async_commit();
+            cp_async_wait<0>();
+            fence_proxy_async_smem();
+            mbar_arrive(&kv_full[st]);
+            named_barrier(1, 128);  // tab[st] and *go are rewritten next iteration
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
+            bool ok = wait_bar(q_full, 0, abort_flag, p.err);
+            for (int j = 0; ok && j < ntiles; ++j) {
+                const int st = j & 1;
+                if (!wait_bar(&kv_full[st], (j >> 1) & 1, abort_flag, p.err)) break;
+                tc_fence_after();
+                const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32 + (kk >> 2) * kHalf;
+                    tc_mma(tS, smem_desc(qa + koff, 16, 1024), smem_desc(ka + koff, 16, 1024), kIdQK, kk > 0);
+                }
+                tc_commit(s_full);
+                if (!wait_bar(p_full, j & 1, abort_flag, p.err)) break;
+                tc_fence_after();
+                const uint32_t pa_ = sbase + kOffP, va = sbase + kOffV + st * kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk) {
+                    const uint32_t poff = (kk & 3) * 32 + (kk >> 2) * kHalf;
+                    tc_mma(tO, smem_desc(pa_ + poff, 16, 1024), smem_desc(va + kk * 2048, kHalf, 1024), kIdPV,
+                           j > 0 || kk > 0);
+                }
+                tc_commit(pv_done);
+                tc_commit(&kv_empty[st]);
+            }
+            // everything issued has completed once this arrives
+            tc_commit(mma_idle);
+            mbar_wait_drain(mma_idle, 0);
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int r = (warp - 4) * 32 + lane;        // query row = TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+        const int i = i0 + r / G;
+        const int pos = start + i;                   // last key this row may see
+        const bool row_ok = i < C;
+        float m = -INFINITY, l = 0.f;
+        bool live = true;
+        for (int j = 0; j < ntiles; ++j) {
+            live = live && wait_bar(s_full, j & 1, abort_flag, p.err);
+            live = __all_sync(kFull, live);
+            if (!live) break;
+            tc_fence_after();
+            // pass 1: row max of the scaled, masked scores (32 columns at a time)
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tmem_ld32(tS + lane_off + c * 32, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int key = j * kTileN + c * 32 + k;
+                    if (row_ok && key <= pos) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                }
+            }
+            const float m_new = fmaxf(m, mx);
+            const float m_use = m_new == -INFINITY ? 0.f : m_new;
+            const float alpha = fast_exp2(m - m_use);
+            if (j > 0) {
+                // P and O are still in use by the previous tile's PV
+                live = wait_bar(pv_done, (j - 1) & 1, abort_flag, p.err);
+                live = __all_sync(kFull, live);
+                if (!live) break;
+                tc_fence_after();
+                if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float ov[32];
+                        tmem_ld32(tO + lane_off + c * 32, ov);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int k = 0; k < 32; ++k) ov[k] *= alpha;
+                        tmem_st32(tO + lane_off + c * 32, ov);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // pass 2: P = 2^(s - m) as bf16 into the K-major swizzled A-operand tile
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float sv[32];
+                tmem_ld32(tS + lane_off + c * 32, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 32; ++k) {
+                    const int key = j * kTileN + c * 32 + k;
+                    sv[k] = (row_ok && key <= pos) ? fast_exp2(sv[k] * p.scale_log2 - m_use) : 0.f;
+                    rs += sv[k];
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float *x = &sv[q * 8];
+                    const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                    *reinterpret_cast<uint4 *>(smem + kOffP + swz(r, c * 4 + q)) = w;
+                }
+            }
+            l = l * alpha + rs;
+            m = m_new;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(p_full);
+        }
+        if (live) live = wait_bar(pv_done, (ntiles - 1) & 1, abort_flag, p.err);
+        live = __all_sync(kFull, live);
+        if (live) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            unsigned char *dst = p.out + (((int64_t)s * p.max_chunk + i) * p.num_q_heads + h * G + r % G) * head_stride;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float ov[32];
+                tmem_ld32(tO + lane_off + c * 32, ov);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int k = 0; k < 32; k += 8) {
+                        const uint4 w = make_uint4(pack_bf16x2(ov[k] * inv, ov[k + 1] * inv),
+                                                   pack_bf16x2(ov[k + 2] * inv, ov[k + 3] * inv),
+                                                   pack_bf16x2(ov[k + 4] * inv, ov[k + 5] * inv),
+                                                   pack_bf16x2(ov[k + 6] * inv, ov[k + 7] * inv));
+                        *reinterpret_cast<uint4 *>(dst + (c * 32 + k) * 2) = w;
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+template <int G>
+cudaError_t launch_g(const PrefillLaunch &a, const Params &prm, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    constexpr int rows = kTileM / G;
+    dim3 grid((unsigned)((a.max_chunk + rows - 1) / rows), (unsigned)a.cache.num_kv_heads, (unsigned)a.num_seqs);
+    prefill_kernel<G><<<grid, kThreads, kSmemBytes, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
+    static_assert(kSmemBytes <= 232448, "prefill smem over the sm_100 limit");
+    if (a.cache.dtype != PA_BF16 || a.cache.head_dim != kD) return cudaErrorNotSupported;
+    if (a.num_seqs > 65535) return cudaErrorNotSupported;
+    Params prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.q = static_cast<const unsigned char *>(a.query);
+    prm.kc = static_cast<const unsigned char *>(a.key_cache);
+    prm.vc = static_cast<const unsigned char *>(a.value_cache);
+    prm.tables = a.block_tables;
+    prm.lens = a.context_lens;
+    prm.chunks = a.chunk_lens;
+    prm.out = static_cast<unsigned char *>(a.out);
+    prm.err = a.err;
+    prm.max_blocks = a.max_blocks_per_seq;
+    prm.num_seqs = a.num_seqs;
+    prm.max_chunk = a.max_chunk;
+    prm.num_q_heads = a.num_q_heads;
+    prm.num_kv_heads = a.cache.num_kv_heads;
+    prm.num_blocks = a.cache.num_blocks;
+    prm.scale_log2 = a.scale * kLog2e;
+    switch (a.num_q_heads / a.cache.num_kv_heads) {
+        case 1: return launch_g<1>(a, prm, stream);
+        case 2: return launch_g<2>(a, prm, stream);
+        case 4: return launch_g<4>(a, prm, stream);
+        case 8: return launch_g<8>(a, prm, stream);
+        default: return cudaErrorNotSupported;
+    }
+}
 
 }  // namespace pa

@@ -1,0 +1,109 @@
+"""GPU parity of the tcgen05 chunked-prefill kernel against the CPU oracle.
+
+Row i of a chunk of C_s rows sits at position L_s - C_s + i and attends causally to
+keys 0..that position through the block table.  bf16 tolerance per element:
+|gpu - oracle| <= 1.5e-2 + 1e-2 |oracle|.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from gpu_harness import TwoSided, check_close, to_dev, to_host, torch_mod
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _lib(pa):
+    return pa
+
+
+def gpu_prefill(ts, q_np, chunk_lens, tables, lens):
+    torch = torch_mod()
+    q = to_dev(q_np)
+    out = torch.full_like(q, float("nan"))
+    ts.pa.pa_prefill_chunk(q, ts.gpu.key_cache, ts.gpu.value_cache, torch.from_numpy(tables).cuda(),
+                           torch.from_numpy(lens).cuda(), torch.from_numpy(np.asarray(chunk_lens, np.int32)).cuda(),
+                           ts.wl.scale, out, ts.gpu.err_flag)
+    return to_host(out)
+
+
+def rows_mask(chunk_lens, mc):
+    m = np.zeros((len(chunk_lens), mc), bool)
+    for s, c in enumerate(chunk_lens):
+        m[s, :c] = True
+    return m
+
+
+def test_long_context_chunk_mini():
+    wl = workloads.make(5, mini=True)
+    ts = TwoSided(wl)
+    pf = wl.prefill
+    t, l = ts.tables(pf.seqs)
+    ch = [pf.chunk] * len(pf.seqs)
+    got = gpu_prefill(ts, pf.q, ch, t, l)
+    ref = oracle.prefill(pf.q, ts.kc, ts.vc, t, l, np.array(ch, np.int32), wl.scale)
+    check_close(got, ref, "bf16", "prefill mini")
+    assert ts.err_flag() == 0
+
+
+def _custom(lens, hq, hkv, seed=3, extra=5):
+    rng = np.random.default_rng(seed)
+    need = sum(-(-L // 16) for L in lens) + extra
+    wl = workloads.Workload(0, "custom", "bf16", need, hq, hkv, 128, 1.0 / np.sqrt(128),
+                            rng.permutation(need).astype(np.int32))
+    for s, L in enumerate(lens):
+        wl.ops.append(("add", s))
+        wl.ops.append(("append", s, workloads.normal(rng, (L, hkv, 128), "bf16"),
+                       workloads.normal(rng, (L, hkv, 128), "bf16")))
+    return wl, rng
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_ragged_chunks_all_group_sizes(g):
+    """Chunks of 1 row, a whole prompt, lengths off tile and block boundaries, an empty chunk."""
+    lens = [1, 37, 300, 129, 16, 600]
+    chunks = [1, 37, 130, 0, 16, 257]
+    wl, rng = _custom(lens, 2 * g, 2)
+    ts = TwoSided(wl)
+    t, l = ts.tables(list(range(len(lens))))
+    mc = max(chunks)
+    q = workloads.normal(rng, (len(lens), mc, 2 * g, 128), "bf16")
+    got = gpu_prefill(ts, q, chunks, t, l)
+    ref = oracle.prefill(q, ts.kc, ts.vc, t, l, np.array(chunks, np.int32), wl.scale)
+    mask = rows_mask(chunks, mc)
+    check_close(got[mask], ref[mask], "bf16", f"prefill g={g}")
+    assert np.isnan(workloads.bf16_bits_to_f32(got[~mask])).all(), "rows past the chunk must not be written"
+    assert ts.err_flag() == 0
+
+
+def test_single_row_chunk_equals_decode():
+    wl, rng = _custom([777, 65, 2049], 32, 8, seed=9)
+    ts = TwoSided(wl)
+    t, l = ts.tables([0, 1, 2])
+    q1 = workloads.normal(rng, (3, 1, 32, 128), "bf16")
+    pre = gpu_prefill(ts, q1, [1, 1, 1], t, l)
+    step = workloads.Step([0, 1, 2], None, None, np.ascontiguousarray(q1[:, 0]))
+    dec = ts.gpu_decode(step, 0)
+    check_close(pre[:, 0], workloads.bf16_bits_to_f32(dec).astype(np.float64), "bf16", "1-row chunk vs decode")
+
+
+def test_long_context_chunk_full_sampled_rows():
+    """8 x 32768 tokens, 512-row chunk, 64/8 heads: every output checked for finiteness,
+    sampled rows (first, last and random) against the oracle."""
+    wl = workloads.make(5)
+    ts = TwoSided(wl)
+    pf = wl.prefill
+    t, l = ts.tables(pf.seqs)
+    ch = [pf.chunk] * len(pf.seqs)
+    got = gpu_prefill(ts, pf.q, ch, t, l)
+    assert np.isfinite(workloads.bf16_bits_to_f32(got)).all()
+    rng = np.random.default_rng(5)
+    mask = np.zeros((len(pf.seqs), pf.chunk), bool)
+    mask[:, [0, 1, pf.chunk - 2, pf.chunk - 1]] = True
+    for s in range(len(pf.seqs)):
+        mask[s, rng.choice(pf.chunk, 8, replace=False)] = True
+    ref = oracle.prefill(pf.q, ts.kc, ts.vc, t, l, np.array(ch, np.int32), wl.scale, row_mask=mask)
+    check_close(got[mask], ref[mask], "bf16", "prefill full (sampled rows)")
+    assert ts.err_flag() == 0
