@@ -166,11 +166,8 @@ def barrier(world):
 def max_over_ranks(x, world):
     if world == 1:
         return x
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from paged_kv_cache_389_b200.dist import max_over_ranks as _max
+    return _max(x, device="cuda")
 
 
 # ----------------------------------------------------------------- profiles
@@ -296,9 +293,17 @@ def run_ours(args):
     flag = pa.pa_wait(cache.err_flag)
     assert flag == 0, f"device error flag {flag}"
 
+    rows = None
+    if rank == 0 and world == 1 and not args.no_rows:
+        peaks0 = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+        del cache, ws, out, q, k_new, v_new, tables_d, lens_d, slots_d
+        torch.cuda.empty_cache()
+        rows = run_rows(args.row_reps, peaks0)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(wl, cache, step, tables_h, lens_h, budget_s=args.cpu_seconds)
+        cpu = cpu_baseline(wl, None, step, tables_h, lens_h, budget_s=args.cpu_seconds)
 
     if rank == 0:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
@@ -332,11 +337,178 @@ def run_ours(args):
             "gpu_launches": K * 3,
             "clocks": clocks,
             "cpu_baseline": cpu,
+            "rows": rows,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------- per-row figures
+def _setup(wl):
+    import torch
+    import paged_kv_cache_389_b200 as pa
+    from paged_kv_cache_389_b200.cache import PagedKVCache
+    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, torch.bfloat16, "cuda", wl.free_order)
+    dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
+    workloads.replay(wl, cache.manager, lambda k, v, s: pa.pa_cache_write(
+        dev(k), dev(v), torch.from_numpy(s).cuda(), cache.key_cache, cache.value_cache, cache.err_flag))
+    return cache, dev
+
+
+def _time(fn, reps, warm=3, graph=False):
+    """Mean device ms of fn() over reps (CUDA events on the current stream).  With
+    graph=True the reps are captured into one CUDA graph first, so microsecond
+    kernels are timed on the device rather than at Python's launch rate."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    if g is not None:
+        g.replay()
+    else:
+        for _ in range(reps):
+            fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def run_rows(reps, peaks):
+    """Each hot-path row on its own workload; device time, inputs resident in HBM."""
+    import torch
+    import paged_kv_cache_389_b200 as pa
+    hbm = float(peaks["hbm_gbs"]) if peaks else 6650.0
+    tf_burst = float(peaks["bf16_tflops"]) if peaks else 1590.0
+    rows = {}
+
+    def dec_entry(name, cache, q, td, ld, maxc, scale, part, bytes_u, bytes_l, nseq):
+        out = torch.empty_like(q)
+        n = pa.pa_decode_workspace_size(q.shape[0], q.shape[1], q.shape[2], maxc, part) if part else 0
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+        ms = _time(lambda: pa.pa_decode(q, cache.key_cache, cache.value_cache, td, ld, maxc, scale, out,
+                                        part, ws, cache.err_flag), reps)
+        rows[name] = {"ms": round(ms, 5), "unique_gbs": round(bytes_u / ms / 1e6, 1),
+                      "logical_gbs": round(bytes_l / ms / 1e6, 1), "frac_of_measured_hbm": round(bytes_u / ms / 1e6 / hbm, 4),
+                      "seq_steps_per_s": round(nseq / ms * 1e3, 1), "partition_size": part}
+
+    # -- MHA-7B decode (64 seqs, 32/32 heads): unsplit and split-K
+    wl = workloads.make(2)
+    cache, dev = _setup(wl)
+    st = wl.steps[0]
+    cache.append(st.seqs, dev(st.k_new), dev(st.v_new))
+    mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+    t, l = cache.manager.build_tables(st.seqs, mb)
+    ub, lb = step_bytes(wl, t, l)
+    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+    for part in (0, 1024):
+        dec_entry(f"a3_decode_mha7b_p{part}", cache, q, td, ld, int(l.max()), wl.scale, part, ub, lb, len(st.seqs))
+    del cache
+    torch.cuda.empty_cache()
+
+    # -- parallel sampling: 128 parents x 4 children, 16 steps of copy-on-write + cache write + decode
+    wl = workloads.make(4)
+    cache, dev = _setup(wl)
+    S = len(wl.steps[0].seqs)
+    part = 1024
+    ev = []
+    host_s = 0.0
+    total_pairs = 0
+    ub_sum = 0
+    pairs1 = None
+    for st in wl.steps:
+        h0 = time.perf_counter()
+        slots, pairs = cache.plan_append(st.seqs)
+        mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+        t, l = cache.manager.build_tables(st.seqs, mb)
+        host_s += time.perf_counter() - h0
+        ub, _ = step_bytes(wl, t, l)
+        ub_sum += ub
+        total_pairs += len(pairs)
+        td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+        kn, vn = dev(st.k_new), dev(st.v_new)
+        sl = torch.from_numpy(slots).cuda()
+        pr = torch.from_numpy(pairs).cuda() if len(pairs) else None
+        if pairs1 is None and pr is not None:
+            pairs1 = pr
+        out = torch.empty_like(q)
+        maxc = int(l.max())
+        n = pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, maxc, part)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        e[0].record()
+        if pr is not None:
+            pa.pa_copy_blocks(cache.key_cache, cache.value_cache, pr, cache.err_flag)
+        e[1].record()
+        pa.pa_cache_write(kn, vn, sl, cache.key_cache, cache.value_cache, cache.err_flag)
+        e[2].record()
+        pa.pa_decode(q, cache.key_cache, cache.value_cache, td, ld, maxc, wl.scale, out, part, ws, cache.err_flag)
+        e[3].record()
+        ev.append((e, len(pairs)))
+    torch.cuda.synchronize()
+    assert pa.pa_wait(cache.err_flag) == 0
+    copy_ms = sum(e[0].elapsed_time(e[1]) for e, _ in ev)
+    cw_ms = sum(e[1].elapsed_time(e[2]) for e, _ in ev)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e, _ in ev)
+    blk_bytes = wl.num_kv_heads * 16 * wl.head_dim * 2 * 2          # K + V of one block
+    e1, np1 = ev[0]
+    c1 = e1[0].elapsed_time(e1[1])
+    rows["fork_cow_16_steps"] = {"seq_steps_per_s_device": round(S * len(wl.steps) / ((copy_ms + cw_ms + dec_ms) * 1e-3), 1),
+                                 "device_ms_total": round(copy_ms + cw_ms + dec_ms, 4), "host_plan_ms_total": round(1e3 * host_s, 3),
+                                 "decode_ms_total": round(dec_ms, 4), "decode_unique_gbs": round(ub_sum / dec_ms / 1e6, 1),
+                                 "cache_write_ms_total": round(cw_ms, 4), "copy_blocks_ms_total": round(copy_ms, 4),
+                                 "copy_pairs_total": total_pairs}
+    rows["a2_copy_blocks_step1"] = {"pairs": np1, "ms_first_launch": round(c1, 5),
+                                    "gbs_first_launch": round(np1 * blk_bytes * 2 / c1 / 1e6, 1)}   # read + write
+    if pairs1 is not None:   # same pairs again (the pool is not used afterwards)
+        ms = _time(lambda: pa.pa_copy_blocks(cache.key_cache, cache.value_cache, pairs1, cache.err_flag), reps, graph=True)
+        rows["a2_copy_blocks_step1"].update({"ms": round(ms, 5), "gbs": round(np1 * blk_bytes * 2 / ms / 1e6, 1)})
+    # steady-state copy of the same 384 pairs (idempotent), and the 512-token cache write
+    st = wl.steps[-1]
+    kn, vn = dev(st.k_new), dev(st.v_new)
+    slots = torch.from_numpy(np.array([cache.manager.block_table(s)[-1] * 16 for s in st.seqs], np.int64)).cuda()
+    ms = _time(lambda: pa.pa_cache_write(kn, vn, slots, cache.key_cache, cache.value_cache, cache.err_flag), reps,
+               graph=True)
+    rows["a1_cache_write_512tok"] = {"ms": round(ms, 5), "gbs": round(cache_write_bytes(wl, S) / ms / 1e6, 1)}
+    del cache
+    torch.cuda.empty_cache()
+
+    # -- long context: split-K decode + tcgen05 prefill chunk
+    wl = workloads.make(5)
+    cache, dev = _setup(wl)
+    st = wl.steps[0]
+    mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+    t, l = cache.manager.build_tables(st.seqs, mb)
+    ub, lb = step_bytes(wl, t, l)
+    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+    for part in (512, 2048):
+        dec_entry(f"a4_decode_long_p{part}", cache, q, td, ld, int(l.max()), wl.scale, part, ub, lb, len(st.seqs))
+    pf = wl.prefill
+    qp = dev(pf.q)
+    outp = torch.empty_like(qp)
+    ch = torch.full((len(pf.seqs),), pf.chunk, dtype=torch.int32, device="cuda")
+    ms = _time(lambda: pa.pa_prefill_chunk(qp, cache.key_cache, cache.value_cache, td, ld, ch, wl.scale, outp,
+                                           cache.err_flag), max(3, reps // 10))
+    keys = sum(int(L) - pf.chunk + i + 1 for L in l for i in range(pf.chunk))
+    flops = 4.0 * wl.num_q_heads * wl.head_dim * keys
+    rows["a5_prefill_chunk_long"] = {"ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1),
+                                     "frac_of_measured_bf16": round(flops / ms / 1e9 / tf_burst, 4),
+                                     "flops": flops, "rows": len(pf.seqs) * pf.chunk}
+    assert pa.pa_wait(cache.err_flag) == 0
+    del cache
+    torch.cuda.empty_cache()
+    return rows
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -442,6 +614,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row figures of the other workloads")
+    ap.add_argument("--row-reps", type=int, default=50)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
