@@ -5,7 +5,8 @@ sequences in 16 groups of 16 sharing a 512-token prefix (32 shared blocks), priv
 lognormal suffixes (median 600, cap 8192), 32 query / 8 kv heads, head_dim 128,
 block_size 16.  One step = the whole decode hot path for one batch:
 pa_cache_write of the 256 new tokens' K/V through their slot mapping, then
-pa_decode over every sequence (split-K partitions of 1024 tokens + LSE reduce).
+pa_decode over every sequence (split-K partitions of 512 tokens; sibling runs
+that share whole partitions read them once as a group; LSE reduce).
 
 Timed region: K steps after W warm-up steps, CUDA events on the launching stream,
 barrier + synchronize on both sides, max over ranks.  The step's inputs (1.1 GB of
@@ -37,7 +38,7 @@ sys.path.insert(0, ROOT)
 
 import workloads  # noqa: E402
 
-PARTITION = 1024
+PARTITION = 512
 CONFIG_ID = 3
 WORKLOAD_NAME = "llama3-8b-gqa-prefix-sharing-decode"
 
@@ -214,7 +215,8 @@ def run_ours(args):
     tables_d = torch.from_numpy(tables_h).cuda()
     lens_d = torch.from_numpy(lens_h).cuda()
     out = torch.empty_like(q)
-    ws_n = pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, max_ctx, PARTITION)
+    part = args.partition
+    ws_n = pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, max_ctx, part)
     ws = torch.empty(max(ws_n, 16), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
     unique_b, logical_b = step_bytes(wl, tables_h, lens_h)
@@ -227,7 +229,7 @@ def run_ours(args):
         if ev_a is not None:
             ev_a.record(stream)
         pa.pa_decode(q, cache.key_cache, cache.value_cache, tables_d, lens_d, max_ctx, wl.scale, out,
-                     PARTITION, ws, cache.err_flag, stream)
+                     part, ws, cache.err_flag, stream)
         if ev_b is not None:
             ev_b.record(stream)
 
@@ -299,7 +301,7 @@ def run_ours(args):
             if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
         del cache, ws, out, q, k_new, v_new, tables_d, lens_d, slots_d
         torch.cuda.empty_cache()
-        rows = run_rows(args.row_reps, peaks0)
+        rows = run_rows(args.row_reps, peaks0, args.partition)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -319,7 +321,7 @@ def run_ours(args):
             "config": {"workload": WORKLOAD_NAME, "num_seqs": S, "num_q_heads": wl.num_q_heads,
                        "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
                        "prefix_tokens": 512, "group_size": 16, "max_context": max_ctx,
-                       "mean_context": float(np.mean(lens_h)), "partition_size": PARTITION,
+                       "mean_context": float(np.mean(lens_h)), "partition_size": part,
                        "parallelism": f"dp{world} (sequences sharded, no exchange)",
                        "l2": "inputs larger than L2 (126 MB); no flush"},
             "seq_steps_per_s": round(world * S * K / (ms_max * 1e-3), 1),
@@ -334,7 +336,7 @@ def run_ours(args):
                          "traffic": recorded_traffic(os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", "decode.cu")),
                          "decode_ms": round(dec_ms, 5)},
             "e2e": e2e,
-            "gpu_launches": K * 3,
+            "gpu_launches": K * (1 + pa.pa_decode_launches(S, wl.head_dim, pa.PA_BF16, part)),
             "clocks": clocks,
             "cpu_baseline": cpu,
             "rows": rows,
@@ -385,7 +387,7 @@ def _time(fn, reps, warm=3, graph=False):
     return a.elapsed_time(b) / reps
 
 
-def run_rows(reps, peaks):
+def run_rows(reps, peaks, partition=PARTITION):
     """Each hot-path row on its own workload; device time, inputs resident in HBM."""
     import torch
     import paged_kv_cache_389_b200 as pa
@@ -421,7 +423,7 @@ def run_rows(reps, peaks):
     wl = workloads.make(4)
     cache, dev = _setup(wl)
     S = len(wl.steps[0].seqs)
-    part = 1024
+    part = partition
     ev = []
     host_s = 0.0
     total_pairs = 0
@@ -616,6 +618,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row figures of the other workloads")
     ap.add_argument("--row-reps", type=int, default=50)
+    ap.add_argument("--partition", type=int, default=PARTITION,
+                    help="split-K partition size in tokens (multiple of 16) of the timed decode")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -127,10 +127,23 @@ PA_API pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_
 /*
  * Bytes of workspace pa_decode needs for a split (partitioned) context:
  * partials of num_seqs * num_q_heads * ceil(max_context_len / partition_size)
- * partitions.  Returns 0 when partition_size <= 0 (no split, no workspace).
+ * partitions (head_dim fp32 accumulators plus a running max and sum each), then
+ * the shared-prefix group area (a shared-block count, a first-partition index
+ * and a 16-byte group record per sequence, and a count word).  Returns 0 when partition_size <= 0
+ * (no split, no workspace).
  */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
                                 int32_t max_context_len, int32_t partition_size);
+
+/*
+ * Number of kernels one pa_decode call with these arguments launches on its
+ * stream (for launch accounting and graph planning): 1 unsplit; 2 split (the
+ * partition kernel and the combine); 5 split with dtype PA_BF16, head_dim 128 and
+ * num_seqs <= 4096 (two shared-prefix detection kernels and the group kernel
+ * run first).  0 when num_seqs <= 0.  Pure host function.
+ */
+PA_API int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype,
+                                  int32_t partition_size);
 
 /*
  * Decode attention over the paged cache, one query token per sequence:
@@ -145,7 +158,13 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
  * l_p and unnormalised accumulator o_p in `workspace`, and a second kernel
  * combines them: out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p with
  * M = max_p m_p.  Sequences with a single partition are finished by the first
- * kernel.  workspace_bytes must be >= pa_decode_workspace_size(...) for the same
+ * kernel.  With a split, bf16 caches, head_dim 128 and num_seqs <= 4096, runs of
+ * adjacent sequences whose block tables begin with the same block ids (forked
+ * siblings, a common prompt) read the partitions that lie wholly inside those
+ * shared blocks once for the whole run, with all its queries against each K/V
+ * tile; the result is the same sum, and the shared blocks cross the memory bus
+ * once instead of once per sibling (devpress teardown, 关键设计二: siblings point
+ * at the same physical blocks).  workspace_bytes must be >= pa_decode_workspace_size(...) for the same
  * num_seqs, num_q_heads, head_dim, max_context_len and partition_size.
  * max_context_len bounds every context_lens[s] (larger sets PA_DEVERR_CONTEXT_LEN
  * and that sequence's outputs are unspecified).  num_seqs <= 16384.

@@ -47,6 +47,7 @@ def _load():
         "pa_cache_write": (C.c_int, [vp, vp, vp, i32, vp, vp, desc, vp, vp]),
         "pa_copy_blocks": (C.c_int, [vp, vp, vp, i32, desc, vp, vp]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32]),
+        "pa_decode_launches": (i32, [i32, i32, i32, i32]),
         "pa_decode": (C.c_int, [vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, i32, vp, sz, vp, desc,
                                 vp, vp]),
         "pa_prefill_chunk": (C.c_int, [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, f32, vp, desc,
@@ -79,7 +80,7 @@ _lib = _load()
 
 EXPORTED = (
     "pa_abi_version", "pa_status_string", "pa_cache_write", "pa_copy_blocks",
-    "pa_decode_workspace_size", "pa_decode", "pa_prefill_chunk", "pa_wait",
+    "pa_decode_workspace_size", "pa_decode_launches", "pa_decode", "pa_prefill_chunk", "pa_wait",
 )
 
 
@@ -162,6 +163,11 @@ def pa_copy_blocks(key_cache, value_cache, src_dst_pairs, err_flag=None, stream=
 def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size) -> int:
     return int(_lib.pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len,
                                              partition_size))
+
+
+def pa_decode_launches(num_seqs, head_dim, dtype, partition_size) -> int:
+    """Kernels one pa_decode call launches; dtype PA_F32 / PA_BF16."""
+    return int(_lib.pa_decode_launches(num_seqs, head_dim, dtype, partition_size))
 
 
 def pa_decode(query, key_cache, value_cache, block_tables, context_lens, max_context_len, scale,

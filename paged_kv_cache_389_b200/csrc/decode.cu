@@ -43,6 +43,7 @@
 //  * No kernel here spins: cp.async completion is waited for with wait_group and
 //    the only barriers are CTA-wide ones every warp reaches.
 #include <cfloat>
+#include <climits>
 #include <cstring>
 
 #include "pa_common.cuh"
@@ -119,6 +120,12 @@ struct Params {
     int32_t part_tokens;  // 0 = whole context is one unit
     int32_t max_parts;
     float scale_log2;
+    // shared-prefix groups (split contexts only; nullptr = none): first_p[s] is the
+    // number of leading partitions of s computed by group_decode_kernel
+    const int32_t *first_p;
+    const int4 *groups;     // (first seq, members, shared partitions, units before)
+    const int32_t *meta;    // [0] groups, [1] group units
+    int32_t max_members;    // sequences per group: query rows members x g <= 128
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -139,12 +146,20 @@ struct Unit {
     int s, part, h;
 };
 
-// Unit u -> (sequence, partition, kv head).  Units [0, S*Hkv) are partition 0
-// of every sequence, kv head innermost; after them come partitions >= 1,
-// sequence-major, using cum[s] = sum_{s' < s} (parts(s') - 1).
-__device__ __forceinline__ Unit unit_of(int64_t u, int64_t units_first, int hkv, const int *cum,
-                                        int S) {
-    if (u < units_first) return Unit{(int)(u / hkv), 0, (int)(u % hkv)};
+__device__ __forceinline__ int first_part(const Params &p, int s) {
+    return p.first_p ? __ldg(p.first_p + s) : 0;
+}
+
+// Unit u -> (sequence, partition, kv head).  Units [0, S*Hkv) are the first
+// partition f(s) of every sequence not covered by a group unit (f = first_part),
+// kv head innermost; after them come partitions > f(s), sequence-major, using
+// cum[s] = sum_{s' < s} (parts(s') - f(s') - 1)^+.
+__device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t units_first, int hkv,
+                                        const int *cum, int S) {
+    if (u < units_first) {
+        const int s = (int)(u / hkv);
+        return Unit{s, first_part(p, s), (int)(u % hkv)};
+    }
     const int64_t v = u - units_first;
     const int e = (int)(v / hkv), h = (int)(v % hkv);
     int lo = 0, hi = S;  // cum[lo] <= e < cum[hi]
@@ -152,7 +167,7 @@ __device__ __forceinline__ Unit unit_of(int64_t u, int64_t units_first, int hkv,
         const int mid = (lo + hi) >> 1;
         if (cum[mid] <= e) lo = mid; else hi = mid;
     }
-    return Unit{lo, 1 + e - cum[lo], h};
+    return Unit{lo, first_part(p, lo) + 1 + e - cum[lo], h};
 }
 
 // What one warp needs to know about a unit.  `tab` holds, in lane i, the table
@@ -165,11 +180,12 @@ struct WarpUnit {
     int nb;   // blocks in the partition
     int tab;
     const int32_t *trow;
+    bool skip;  // partition past the end (every partition was covered by a group unit)
 };
 
 __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t units_first,
                                           const int *cum, WarpUnit &w, int lane, bool flagger) {
-    w.un = unit_of(u, units_first, p.num_kv_heads, cum, p.num_seqs);
+    w.un = unit_of(p, u, units_first, p.num_kv_heads, cum, p.num_seqs);
     const int b0 = p.part_tokens > 0 ? w.un.part * (p.part_tokens / kBlockSize) : 0;
     w.trow = p.tables + (int64_t)w.un.s * p.max_blocks + b0;
     // both loads issued before either value is needed
@@ -188,11 +204,13 @@ __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t un
         w.t0 = w.un.part * p.part_tokens;
         w.nt = max(0, min(L, w.t0 + p.part_tokens) - w.t0);
     }
+    w.skip = w.un.part >= num_parts(p, L);
+    if (w.skip) w.nt = 0;
     w.nb = (w.nt + kBlockSize - 1) / kBlockSize;
 }
 
-// Barrier-free prologue: cum[s] = sum_{s' < s} (parts(s') - 1) (exclusive scan,
-// one chunk of sequences per thread).  Ends with __syncthreads.
+// Prologue: cum[s] = sum_{s' < s} (parts(s') - first_part(s') - 1)^+ (exclusive
+// scan, one chunk of sequences per thread).  Ends with __syncthreads.
 __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (p.part_tokens > 0) {
@@ -202,7 +220,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
         int local = 0;
         for (int s = beg; s < end; ++s) {
             const int L = checked_len(p, s);
-            local += num_parts(p, L < 0 ? 0 : L) - 1;
+            local += max(0, num_parts(p, L < 0 ? 0 : L) - first_part(p, s) - 1);
         }
         int incl = local;
 #pragma unroll
@@ -218,7 +236,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
         for (int s = beg; s < end; ++s) {
             cum[s] = run;
             const int L = checked_len(p, s);
-            run += num_parts(p, L < 0 ? 0 : L) - 1;
+            run += max(0, num_parts(p, L < 0 ? 0 : L) - first_part(p, s) - 1);
         }
         if ((int)threadIdx.x == kThreads - 1) cum[S] = run;
     }
@@ -264,7 +282,8 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(void *out, int64_t idx,
 template <typename T, int D, int G>
 __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, const float *uacc,
                                             const float2 *uml) {
-    const bool single = num_parts(p, w.L) == 1;
+    if (w.skip) return;
+    const bool single = num_parts(p, w.L) == 1 && first_part(p, w.un.s) == 0;
     const int64_t head0 = (int64_t)w.un.s * p.num_q_heads + (int64_t)w.un.h * G;
     for (int e = threadIdx.x; e < G * D; e += kThreads) {
         const int h = e / D, dd = e - h * D;
@@ -693,6 +712,154 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     cp_async_wait<0>();
 }
 
+// ------------------------------------------------------------- shared prefixes
+// Sequences next to each other in the batch whose tables start with the same
+// physical blocks (forks, a shared system prompt: chenxutan 2.1 / 3.3, devpress
+// 关键设计二) read those blocks once: the shared leading partitions are computed
+// by group units whose query columns are members x heads, and the per-sequence
+// kernel starts after them.  Results are unchanged -- the same partials land in
+// the same workspace slots and the LSE reduce combines them.
+//
+// Detection takes two launches: group_lcp_kernel (a warp per sequence) counts the
+// leading full blocks each sequence shares with its predecessor; group_form_kernel
+// (one CTA) cuts the batch into chunks and lists them.  The group units -- a
+// dense (members x g) x partition x head_dim attention tile each -- run on the
+// tcgen05 tile kernel of prefill.cu (launch_group_tiles).
+
+constexpr int kLcpWarps = 8;
+constexpr int kDetectThreads = 1024;
+constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
+constexpr int kMaxGroupParts = (1 << 23) - 1;
+
+// lcp[s] = leading entries of s's table equal to those of s-1, counted over the
+// blocks both contexts fill completely (0 for s = 0).  128 entries per round.
+__global__ void __launch_bounds__(kLcpWarps * 32) group_lcp_kernel(const __grid_constant__ Params p,
+                                                                   int32_t *lcp) {
+    const int lane = threadIdx.x & 31;
+    const int nw = gridDim.x * kLcpWarps;
+    for (int s = blockIdx.x * kLcpWarps + (threadIdx.x >> 5); s < p.num_seqs; s += nw) {
+        int n = 0;
+        if (s > 0) {
+            const int La = checked_len(p, s), Lb = checked_len(p, s - 1);
+            n = min(max(La, 0), max(Lb, 0)) / kBlockSize;
+        }
+        const int32_t *ta = p.tables + (int64_t)s * p.max_blocks;
+        const int32_t *tb = ta - p.max_blocks;  // read only when n > 0, i.e. s > 0
+        int res = n;
+        for (int c0 = 0; c0 < n; c0 += 128) {
+            int a[4], b[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = c0 + 32 * k + lane;
+                a[k] = i < n ? __ldg(ta + i) : 0;
+                b[k] = i < n ? __ldg(tb + i) : 0;
+            }
+            int mis = n;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = c0 + 32 * k + lane;
+                if (i < n && a[k] != b[k]) mis = min(mis, i);
+            }
+            mis = __reduce_min_sync(kFull, mis);
+            if (mis < n) {
+                res = mis;
+                break;
+            }
+        }
+        if (lane == 0) lcp[s] = res;
+    }
+}
+
+// Block-wide exclusive scan (sum, or max when kMax) of one int per thread.
+template <bool kMax>
+__device__ __forceinline__ int block_exclusive_scan(int x, int identity, int *wbuf) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int inc = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc = kMax ? max(inc, y) : inc + y;
+    }
+    if (lane == 31) wbuf[warp] = inc;
+    __syncthreads();
+    int off = identity;
+    for (int w = 0; w < warp; ++w) off = kMax ? max(off, wbuf[w]) : off + wbuf[w];
+    int exc = __shfl_up_sync(kFull, inc, 1);
+    if (lane == 0) exc = identity;
+    __syncthreads();  // wbuf is reused by the next scan
+    return kMax ? max(off, exc) : off + exc;
+}
+
+// One CTA.  A run is a maximal stretch of sequences each sharing at least one
+// whole partition with its predecessor; runs are cut into chunks of at most
+// max_members sequences counted from the run's start.  A chunk of n >= 2
+// sequences shares min(lcp over its members after the first) blocks, i.e. np
+// whole partitions; it becomes one group with np x num_kv_heads units.
+// first_p[s] = np of s's chunk (0 for a chunk of one).
+__global__ void __launch_bounds__(kDetectThreads) group_form_kernel(const __grid_constant__ Params p,
+                                                                    const int32_t *lcp_g, int32_t *first_p,
+                                                                    int4 *groups, int32_t *meta) {
+    __shared__ int lcp[kMaxGroupSeqs];
+    __shared__ int info[kMaxGroupSeqs];  // at a chunk head: np << 8 | members (members <= 128); else -1
+    __shared__ int wbuf[kDetectThreads / 32];
+    constexpr int kPer = kMaxGroupSeqs / kDetectThreads;
+    const int S = p.num_seqs, tid = threadIdx.x;
+    const int bpp = p.part_tokens / kBlockSize, M = p.max_members;
+    const int s0 = tid * kPer;
+    // run starts: max-scan of (run head ? s : -1)
+    int lv[kPer], mx = -1;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int s = s0 + k;
+        lv[k] = s < S ? __ldg(lcp_g + s) : 0;
+        if (s < S && (s == 0 || lv[k] < bpp)) mx = s;
+    }
+    int rs = block_exclusive_scan<true>(mx, -1, wbuf);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int s = s0 + k;
+        if (s >= S) break;
+        if (s == 0 || lv[k] < bpp) rs = s;
+        lcp[s] = lv[k];
+        info[s] = (s - rs) % M == 0 ? 0 : -1;  // chunk heads marked 0 for now
+    }
+    __syncthreads();
+    // each chunk head measures its chunk
+    int chunks = 0, units = 0;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int s = s0 + k;
+        if (s >= S || info[s] < 0) continue;
+        int e = s + 1, mn = INT_MAX;
+        while (e < S && info[e] < 0) mn = min(mn, lcp[e++]);
+        const int n = e - s;
+        const int np = n > 1 ? min(mn / bpp, kMaxGroupParts) : 0;
+        info[s] = (np << 8) | n;  // stays >= 0: other threads only test the sign
+        if (np > 0) {
+            ++chunks;
+            units += np * p.num_kv_heads;
+        }
+    }
+    int oc = block_exclusive_scan<false>(chunks, 0, wbuf);
+    int ou = block_exclusive_scan<false>(units, 0, wbuf);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+        const int s = s0 + k;
+        if (s >= S || info[s] < 0) continue;
+        const int n = info[s] & 255, np = info[s] >> 8;
+        for (int m = s; m < s + n; ++m) first_p[m] = np;
+        if (np > 0) {
+            groups[oc++] = make_int4(s, n, np, ou);
+            ou += np * p.num_kv_heads;
+        }
+    }
+    if (tid == kDetectThreads - 1) {
+        meta[0] = oc;
+        meta[1] = ou;
+    }
+}
+
+
 // Combine split-K partials: one warp per (sequence, query head) with more than
 // one partition.  M = max_p m_p; out = sum_p 2^(m_p-M) acc_p / sum_p 2^(m_p-M) l_p.
 template <typename T, int D>
@@ -705,7 +872,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
     int L = checked_len(p, s);
     if (L < 0) L = 0;
     const int n = num_parts(p, L);
-    if (n <= 1) return;
+    if (n <= 1 && first_part(p, s) == 0) return;  // finished by the decode kernel
     const float2 *ml = p.ws_ml + wid * p.max_parts;
     const float *acc = p.ws_acc + wid * p.max_parts * D + lane * kDpl;
     float M = -INFINITY;
@@ -735,7 +902,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_t(const DecodeLaunch &a, const Params &prm, cudaStream_t stream) {
+cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
     using Lay = Layout<T, D, G>;
     const bool split = prm.part_tokens > 0;
     const size_t smem = Lay::smem_bytes(split ? a.num_seqs + 1 : 0);
@@ -746,7 +913,47 @@ cudaError_t launch_t(const DecodeLaunch &a, const Params &prm, cudaStream_t stre
     e = cudaFuncSetAttribute(decode_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)Lay::smem_bytes(kMaxSplitSeqs + 1));
     if (e != cudaSuccess) return e;
-    int64_t grid = num_sms(dev);
+    const int sms = num_sms(dev);
+    // shared-prefix groups: bf16, head_dim 128, split contexts
+    if constexpr (sizeof(T) == 2 && D == 128) {
+        if (split && a.ws_group && a.num_seqs <= kMaxGroupSeqs) {
+            unsigned char *g = static_cast<unsigned char *>(a.ws_group);
+            // group area: lcp[S], first_p[S] (each 16-byte padded), groups[S], meta
+            const size_t sa = ((size_t)a.num_seqs * 4 + 15) / 16 * 16;
+            int32_t *lcp = reinterpret_cast<int32_t *>(g);
+            prm.first_p = reinterpret_cast<int32_t *>(g + sa);
+            prm.groups = reinterpret_cast<int4 *>(g + 2 * sa);
+            prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
+            prm.max_members = 128 / G;
+            const int lcp_grid = (int)std::min<int64_t>(((int64_t)a.num_seqs + kLcpWarps - 1) / kLcpWarps,
+                                                        (int64_t)sms * 4);
+            group_lcp_kernel<<<std::max(lcp_grid, 1), kLcpWarps * 32, 0, stream>>>(prm, lcp);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            group_form_kernel<<<1, kDetectThreads, 0, stream>>>(prm, lcp, const_cast<int32_t *>(prm.first_p),
+                                                                const_cast<int4 *>(prm.groups),
+                                                                const_cast<int32_t *>(prm.meta));
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            GroupTileLaunch gl;
+            gl.query = a.query;
+            gl.key_cache = a.key_cache;
+            gl.value_cache = a.value_cache;
+            gl.block_tables = a.block_tables;
+            gl.max_blocks_per_seq = a.max_blocks_per_seq;
+            gl.groups = prm.groups;
+            gl.meta = prm.meta;
+            gl.ws_acc = prm.ws_acc;
+            gl.ws_ml = prm.ws_ml;
+            gl.num_q_heads = a.num_q_heads;
+            gl.num_kv_heads = a.cache.num_kv_heads;
+            gl.num_blocks = a.cache.num_blocks;
+            gl.partition_size = a.partition_size;
+            gl.max_partitions = a.max_partitions;
+            gl.scale = a.scale;
+            gl.err = a.err;
+            if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
+        }
+    }
+    int64_t grid = sms;
     if (!split) grid = std::min<int64_t>(grid, (int64_t)a.num_seqs * a.cache.num_kv_heads);
     if (grid < 1) grid = 1;
     decode_kernel<T, D, G><<<(unsigned)grid, kThreads, smem, stream>>>(prm);
@@ -758,7 +965,7 @@ cudaError_t launch_t(const DecodeLaunch &a, const Params &prm, cudaStream_t stre
 }
 
 template <typename T, int D>
-cudaError_t launch_g(const DecodeLaunch &a, const Params &prm, cudaStream_t stream) {
+cudaError_t launch_g(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
     switch (a.num_q_heads / a.cache.num_kv_heads) {
         case 1: return launch_t<T, D, 1>(a, prm, stream);
         case 2: return launch_t<T, D, 2>(a, prm, stream);
@@ -800,3 +1007,4 @@ cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
 }
 
 }  // namespace pa
+

@@ -98,7 +98,19 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
         return 0;
     const int64_t parts = ((int64_t)max_context_len + partition_size - 1) / partition_size;
     const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
-    return (size_t)(rows * head_dim * 4 + rows * 8);
+    // partials (fp32 acc, then (m, l)), then the shared-prefix group bookkeeping:
+    // shared-block count and first partition per sequence (each 16-byte padded),
+    // group list (16 bytes each), 16 bytes of counters
+    const int64_t partials = rows * head_dim * 4 + rows * 8;
+    const int64_t group = 2 * (((int64_t)num_seqs * 4 + 15) / 16 * 16) + (int64_t)num_seqs * 16 + 16;
+    return (size_t)((partials + 15) / 16 * 16 + group);
+}
+
+int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype, int32_t partition_size) {
+    if (num_seqs <= 0) return 0;
+    if (partition_size <= 0) return 1;
+    const bool grouped = dtype == PA_BF16 && head_dim == 128 && num_seqs <= kMaxSplitSeqs;
+    return grouped ? 5 : 2;
 }
 
 pa_status pa_decode(const void *query, const void *key_cache, const void *value_cache,
@@ -132,9 +144,9 @@ pa_status pa_decode(const void *query, const void *key_cache, const void *value_
         a.partition_size = partition_size;
         a.max_partitions = (int32_t)parts;
         a.ws_acc = static_cast<float *>(workspace);
-        a.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) +
-                                             (size_t)num_seqs * num_q_heads * parts *
-                                                 cache->head_dim * 4);
+        const size_t rows = (size_t)num_seqs * num_q_heads * parts;
+        a.ws_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + rows * cache->head_dim * 4);
+        a.ws_group = static_cast<char *>(workspace) + (rows * cache->head_dim * 4 + rows * 8 + 15) / 16 * 16;
     } else {
         // every context fits in one partition: the split would change nothing
         a.partition_size = 0;

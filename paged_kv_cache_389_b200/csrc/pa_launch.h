@@ -34,6 +34,7 @@ struct DecodeLaunch {
     int32_t max_partitions;  // ceil(max_context_len / partition_size) when split
     float *ws_acc;           // [S][Hq][Pmax][D] unnormalised partial accumulators
     float2 *ws_ml;           // [S][Hq][Pmax] (running max in log2 units, running sum)
+    void *ws_group;          // shared-prefix group bookkeeping (split contexts), or null
     void *out;
     pa_cache_desc cache;
     int32_t *err;
@@ -63,6 +64,30 @@ struct PrefillLaunch {
 };
 
 cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
+
+// Shared-prefix group units of a split bf16 / head_dim 128 decode, on the tcgen05
+// tile kernel: rows = a group's members x g query heads, keys = one partition
+// inside the blocks they share; writes that partition's split-K partials.
+// groups / meta are the decode's detection output (device memory).
+struct GroupTileLaunch {
+    const void *query;
+    const void *key_cache;
+    const void *value_cache;
+    const int32_t *block_tables;
+    int32_t max_blocks_per_seq;
+    const int4 *groups;
+    const int32_t *meta;
+    float *ws_acc;
+    float2 *ws_ml;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int32_t num_blocks;
+    int32_t partition_size;
+    int32_t max_partitions;
+    float scale;
+    int32_t *err;
+};
+cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t stream);
 
 int num_sms(int device);
 

@@ -48,7 +48,9 @@ constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffP + kTileBytes;
 constexpr uint32_t kOffTab = kOffBar + 16 * 8;     // 8 table entries per stage
 constexpr uint32_t kOffMisc = kOffTab + 2 * 8 * 4;
-constexpr size_t kSmemBytes = 1024 + kOffMisc + 16;
+constexpr uint32_t kOffGcum = kOffMisc + 16;         // group units: units before each group
+constexpr int kMaxGroups = 2048;                     // a group has >= 2 of <= 4096 sequences
+constexpr size_t kSmemBytes = 1024 + kOffGcum + kMaxGroups * 4;
 
 struct Params {
     const unsigned char *q;
@@ -66,6 +68,13 @@ struct Params {
     int32_t num_kv_heads;
     int32_t num_blocks;
     float scale_log2;
+    // shared-prefix group units of the split decode
+    const int4 *groups;    // (first seq, members, shared partitions, units before)
+    const int32_t *meta;   // [0] groups, [1] units
+    float *ws_acc;
+    float2 *ws_ml;
+    int32_t part_tokens;
+    int32_t max_parts;
 };
 
 // ---- tcgen05 wrappers --------------------------------------------------------
@@ -151,8 +160,59 @@ __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatil
     return mbar_wait_bounded(bar, parity, abort, err);
 }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_constant__ Params p) {
+// One 128-row query tile against a run of keys.  Row r (0..127) holds query head
+// h*G + r%G of row group r/G; row groups are q_row_stride bytes apart.  Keys are
+// 0..nkeys-1 through the table entries starting at trow; row r may see keys
+// 0..lim0 + lim_step*(r/G) (lim_step 1: causal prefill; 0: every key).
+struct Job {
+    const unsigned char *q;  // query row group 0, head h*G
+    int64_t q_row_stride;
+    int nrows;               // rows r < nrows are real (the rest are zero)
+    const int32_t *trow;
+    int nkeys;
+    int lim0, lim_step;
+    int ntiles;
+    int h;
+    // output: prefill -> normalised bf16 rows at out (same strides as q);
+    // group -> fp32 partials of workspace row (first + r/G)*Hq + h*G + r%G, slot part
+    unsigned char *out;
+    int first, part;
+};
+
+template <int G, bool kGroup>
+__device__ __forceinline__ Job group_job(const Params &p, const int *gcum, int ngroups, int u) {
+    Job jb;
+    int lo = 0, hi = ngroups;  // gcum[lo] <= u < gcum[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (gcum[mid] <= u) lo = mid; else hi = mid;
+    }
+    const int4 gr = __ldg(&p.groups[lo]);  // (first seq, members, shared partitions, units before)
+    const int r = u - gr.w;
+    jb.h = r % p.num_kv_heads;
+    jb.part = r / p.num_kv_heads;
+    jb.first = gr.x;
+    const int64_t hs = (int64_t)kD * 2;
+    jb.q_row_stride = (int64_t)p.num_q_heads * hs;
+    jb.q = p.q + (int64_t)gr.x * jb.q_row_stride + (int64_t)jb.h * G * hs;
+    jb.nrows = gr.y * G;
+    jb.trow = p.tables + (int64_t)gr.x * p.max_blocks + (int64_t)jb.part * (p.part_tokens / kBlockSize);
+    jb.nkeys = p.part_tokens;
+    jb.lim0 = p.part_tokens - 1;
+    jb.lim_step = 0;
+    jb.ntiles = (p.part_tokens + kTileN - 1) / kTileN;
+    jb.out = nullptr;
+    return jb;
+}
+
+// Prefill: one CTA per (query tile, kv head, sequence).  Shared-prefix groups of
+// the split decode (kGroup): a persistent CTA loops over the group units (group,
+// partition, kv head) listed by the decode's detection kernels; the rows are the
+// members' queries, the keys one partition lying inside the blocks all members
+// share, and the result is the partition's (m, l, unnormalised O) in the split-K
+// workspace -- the same partial the per-sequence decode kernel writes.
+template <int G, bool kGroup>
+__global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_constant__ Params p) {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const uint32_t sbase = smem_u32(smem);
@@ -167,20 +227,43 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
     int *tab = reinterpret_cast<int *>(smem + kOffTab);  // [2][8]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+    volatile int *go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
+    int *gcum = reinterpret_cast<int *>(smem + kOffGcum);
+    const int64_t hs = (int64_t)kD * 2;  // bytes per (row, head)
 
-    constexpr int kRowsPerTile = kTileM / G;  // chunk rows per query tile
-    const int s = blockIdx.z, h = blockIdx.y;
-    const int i0 = blockIdx.x * kRowsPerTile;
-    const int L = __ldg(p.lens + s), C = __ldg(p.chunks + s);
-    // validate once; an invalid sequence is skipped (flagged by its first tile)
-    if (C < 0 || C > p.max_chunk || C > L || (int64_t)L > (int64_t)p.max_blocks * kBlockSize) {
-        if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) flag_error(p.err, PA_DEVERR_CHUNK);
-        return;
+    // ---- the work of this CTA
+    int u0 = 0, nunits = 1, ngroups = 0;
+    Job jb;
+    if constexpr (kGroup) {
+        nunits = __ldg(p.meta + 1);
+        ngroups = __ldg(p.meta);
+        u0 = blockIdx.x;
+        if (u0 >= nunits) return;
+    } else {
+        constexpr int kRowsPerTile = kTileM / G;
+        const int s = blockIdx.z, h = blockIdx.y;
+        const int i0 = blockIdx.x * kRowsPerTile;
+        const int L = __ldg(p.lens + s), C = __ldg(p.chunks + s);
+        // validate once; an invalid sequence is skipped (flagged by its first tile)
+        if (C < 0 || C > p.max_chunk || C > L || (int64_t)L > (int64_t)p.max_blocks * kBlockSize) {
+            if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) flag_error(p.err, PA_DEVERR_CHUNK);
+            return;
+        }
+        if (i0 >= C) return;
+        const int start = L - C;
+        const int last_row = min(C, i0 + kRowsPerTile) - 1;
+        jb.h = h;
+        jb.q_row_stride = (int64_t)p.num_q_heads * hs;
+        jb.q = p.q + ((int64_t)s * p.max_chunk + i0) * jb.q_row_stride + (int64_t)h * G * hs;
+        jb.out = p.out + ((int64_t)s * p.max_chunk + i0) * jb.q_row_stride + (int64_t)h * G * hs;
+        jb.nrows = (last_row - i0 + 1) * G;
+        jb.trow = p.tables + (int64_t)s * p.max_blocks;
+        jb.nkeys = L;
+        jb.lim0 = start + i0;
+        jb.lim_step = 1;
+        jb.ntiles = (start + last_row + 1 + kTileN - 1) / kTileN;  // keys 0..start+last_row
+        jb.first = jb.part = 0;
     }
-    if (i0 >= C) return;
-    const int start = L - C;
-    const int last_row = min(C, i0 + kRowsPerTile) - 1;
-    const int ntiles = (start + last_row + 1 + kTileN - 1) / kTileN;  // keys 0..start+last_row
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -196,207 +279,243 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
         *abort_flag = 0;
         mbar_init_fence();
     }
+    if constexpr (kGroup) {
+        for (int k = threadIdx.x; k < ngroups; k += kThreads) gcum[k] = __ldg(&p.groups[k].w);
+    }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t tS = tmem, tO = tmem + 128;
-    const int64_t head_stride = (int64_t)kD * 2;  // bytes per (row, head)
 
-    if (warp < 4) {
-        // ------------------------------------------------------------ loaders
-        const int t = threadIdx.x;  // 0..127
-        // Q tile: row m = (chunk row, head) pair; 16 chunks of 16 bytes per row
-        for (int idx = t; idx < kTileM * 16; idx += 128) {
-            const int m = idx >> 4, c = idx & 15;
-            const int i = i0 + m / G, hq = h * G + m % G;
-            const uint32_t dst = sbase + kOffQ + swz(m, c);
-            if (i < C)
-                cp_async16(dst, p.q + (((int64_t)s * p.max_chunk + i) * p.num_q_heads + hq) * head_stride + c * 16);
-            else
-                *reinterpret_cast<uint4 *>(smem + kOffQ + swz(m, c)) = make_uint4(0, 0, 0, 0);
-        }
-        cp_async_commit();
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(q_full);
-        const int32_t *trow = p.tables + (int64_t)s * p.max_blocks;
-        volatile int *go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
-        for (int j = 0; j < ntiles; ++j) {
-            const int st = j & 1;
-            // one thread waits for the stage; the decision reaches all loaders
-            // through shared memory behind the barrier, so they break together
-            if (t == 0) *go = (j < 2 || wait_bar(&kv_empty[st], ((j >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
-            // table entries of the tile's 8 blocks (-1: past the context)
-            if (t < 8) {
-                const int b = j * 8 + t;
-                int e = -1;
-                if (b * kBlockSize < L) {
-                    e = __ldg(trow + b);
-                    if (e < 0 || e >= p.num_blocks) {
-                        flag_error(p.err, PA_DEVERR_BLOCK_ID);
-                        e = -1;
-                    }
-                }
-                tab[st * 8 + t] = e;
-            }
-            named_barrier(1, 128);
-            if (!*go) break;
-            const uint32_t kst = sbase + kOffK + st * kTileBytes, vst = sbase + kOffV + st * kTileBytes;
-            unsigned char *kgen = smem + kOffK + st * kTileBytes, *vgen = smem + kOffV + st * kTileBytes;
-            for (int idx = t; idx < kTileN * 16; idx += 128) {
-                const int n = idx >> 4, c = idx & 15;
-                const int key = j * kTileN + n;
-                const int blk = tab[st * 8 + (n >> 4)];
-                const uint32_t off = swz(n, c);
-                if (blk >= 0 && key < L) {
-                    const int64_t src = (((int64_t)blk * p.num_kv_heads + h) * kBlockSize + (n & 15)) * head_stride + c * 16;
-                    cp_async16(kst + off, p.kc + src);
-                    cp_async16(vst + off, p.vc + src);
-                } else {  // past the context or a bad id: zeros (0 * garbage must not reach the sums)
-                    *reinterpret_cast<uint4 *>(kgen + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(vgen + off) = make_uint4(0, 0, 0, 0);
-                }
+    // Barrier phases run on across units: tile jt = tbase + j of the CTA uses
+    // stage jt & 1; q_full and mma_idle complete once per unit.
+    int tbase = 0, nu = 0;
+    for (int u = u0; u < nunits; u += (kGroup ? gridDim.x : 1), ++nu) {
+        if constexpr (kGroup) jb = group_job<G, kGroup>(p, gcum, ngroups, u);
+        if (warp < 4) {
+            // -------------------------------------------------------- loaders
+            const int t = threadIdx.x;  // 0..127
+            // Q tile: row r = (row group r / G, head r % G); 16 chunks of 16 bytes per row
+            for (int idx = t; idx < kTileM * 16; idx += 128) {
+                const int r = idx >> 4, c = idx & 15;
+                const uint32_t dst = sbase + kOffQ + swz(r, c);
+                if (r < jb.nrows)
+                    cp_async16(dst, jb.q + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs + c * 16);
+                else
+                    *reinterpret_cast<uint4 *>(smem + kOffQ + swz(r, c)) = make_uint4(0, 0, 0, 0);
             }
             cp_async_commit();
-            cp_async_wait<0>();
-            fence_proxy_async_smem();
-            mbar_arrive(&kv_full[st]);
-            named_barrier(1, 128);  // tab[st] and *go are rewritten next iteration
-        }
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
-            bool ok = wait_bar(q_full, 0, abort_flag, p.err);
-            for (int j = 0; ok && j < ntiles; ++j) {
-                const int st = j & 1;
-                if (!wait_bar(&kv_full[st], (j >> 1) & 1, abort_flag, p.err)) break;
-                tc_fence_after();
-                const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < kD / 16; ++kk) {
-                    const uint32_t koff = (kk & 3) * 32 + (kk >> 2) * kHalf;
-                    tc_mma(tS, smem_desc(qa + koff, 16, 1024), smem_desc(ka + koff, 16, 1024), kIdQK, kk > 0);
+            bool q_sent = false;
+            for (int j = 0; j < jb.ntiles; ++j) {
+                const int jt = tbase + j, st = jt & 1;
+                // one thread waits for the stage; the decision reaches all loaders
+                // through shared memory behind the barrier, so they break together
+                if (t == 0) *go = (jt < 2 || wait_bar(&kv_empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
+                // table entries of the tile's 8 blocks (-1: past the keys)
+                if (t < 8) {
+                    const int b = j * 8 + t;
+                    int e = -1;
+                    if (b * kBlockSize < jb.nkeys) {
+                        e = __ldg(jb.trow + b);
+                        if (e < 0 || e >= p.num_blocks) {
+                            flag_error(p.err, PA_DEVERR_BLOCK_ID);
+                            e = -1;
+                        }
+                    }
+                    tab[st * 8 + t] = e;
                 }
-                tc_commit(s_full);
-                if (!wait_bar(p_full, j & 1, abort_flag, p.err)) break;
-                tc_fence_after();
-                const uint32_t pa_ = sbase + kOffP, va = sbase + kOffV + st * kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk) {
-                    const uint32_t poff = (kk & 3) * 32 + (kk >> 2) * kHalf;
-                    tc_mma(tO, smem_desc(pa_ + poff, 16, 1024), smem_desc(va + kk * 2048, kHalf, 1024), kIdPV,
-                           j > 0 || kk > 0);
+                named_barrier(1, 128);
+                if (!*go) break;
+                const uint32_t kst = sbase + kOffK + st * kTileBytes, vst = sbase + kOffV + st * kTileBytes;
+                unsigned char *kgen = smem + kOffK + st * kTileBytes, *vgen = smem + kOffV + st * kTileBytes;
+                for (int idx = t; idx < kTileN * 16; idx += 128) {
+                    const int n = idx >> 4, c = idx & 15;
+                    const int key = j * kTileN + n;
+                    const int blk = tab[st * 8 + (n >> 4)];
+                    const uint32_t off = swz(n, c);
+                    if (blk >= 0 && key < jb.nkeys) {
+                        const int64_t src = (((int64_t)blk * p.num_kv_heads + jb.h) * kBlockSize + (n & 15)) * hs + c * 16;
+                        cp_async16(kst + off, p.kc + src);
+                        cp_async16(vst + off, p.vc + src);
+                    } else {  // past the keys or a bad id: zeros (0 * garbage must not reach the sums)
+                        *reinterpret_cast<uint4 *>(kgen + off) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(vgen + off) = make_uint4(0, 0, 0, 0);
+                    }
                 }
-                tc_commit(pv_done);
-                tc_commit(&kv_empty[st]);
+                cp_async_commit();
+                if (!q_sent) {  // the Q copies overlap the first K/V tile's
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(q_full);
+                    q_sent = true;
+                }
+                cp_async_wait<0>();
+                fence_proxy_async_smem();
+                mbar_arrive(&kv_full[st]);
+                named_barrier(1, 128);  // tab[st] and *go are rewritten next iteration
             }
-            // everything issued has completed once this arrives
-            tc_commit(mma_idle);
-            mbar_wait_drain(mma_idle, 0);
-        }
-        __syncwarp();
-    } else {
-        // ------------------------------------------------------------ softmax
-        const int r = (warp - 4) * 32 + lane;        // query row = TMEM lane
-        const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-        const int i = i0 + r / G;
-        const int pos = start + i;                   // last key this row may see
-        const bool row_ok = i < C;
-        float m = -INFINITY, l = 0.f;
-        bool live = true;
-        for (int j = 0; j < ntiles; ++j) {
-            live = live && wait_bar(s_full, j & 1, abort_flag, p.err);
-            live = __all_sync(kFull, live);
-            if (!live) break;
-            tc_fence_after();
-            // pass 1: row max of the scaled, masked scores (32 columns at a time)
-            float mx = -INFINITY;
+            cp_async_wait<0>();  // nothing may land after an abort
+        } else if (warp == kMmaWarp) {
+            // -------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
+                bool ok = wait_bar(q_full, nu & 1, abort_flag, p.err);
+                for (int j = 0; ok && j < jb.ntiles; ++j) {
+                    const int jt = tbase + j, st = jt & 1;
+                    if (!wait_bar(&kv_full[st], (jt >> 1) & 1, abort_flag, p.err)) break;
+                    tc_fence_after();
+                    const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTileBytes;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tmem_ld32(tS + lane_off + c * 32, sv);
-                tmem_wait_ld();
+                    for (int kk = 0; kk < kD / 16; ++kk) {
+                        const uint32_t koff = (kk & 3) * 32 + (kk >> 2) * kHalf;
+                        tc_mma(tS, smem_desc(qa + koff, 16, 1024), smem_desc(ka + koff, 16, 1024), kIdQK, kk > 0);
+                    }
+                    tc_commit(s_full);
+                    if (!wait_bar(p_full, jt & 1, abort_flag, p.err)) break;
+                    tc_fence_after();
+                    const uint32_t pa_ = sbase + kOffP, va = sbase + kOffV + st * kTileBytes;
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int key = j * kTileN + c * 32 + k;
-                    if (row_ok && key <= pos) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                    for (int kk = 0; kk < kTileN / 16; ++kk) {
+                        const uint32_t poff = (kk & 3) * 32 + (kk >> 2) * kHalf;
+                        tc_mma(tO, smem_desc(pa_ + poff, 16, 1024), smem_desc(va + kk * 2048, kHalf, 1024), kIdPV,
+                               j > 0 || kk > 0);
+                    }
+                    tc_commit(pv_done);
+                    tc_commit(&kv_empty[st]);
+                }
+                // everything issued has completed once this arrives
+                tc_commit(mma_idle);
+                if (!mbar_wait_drain(mma_idle, nu & 1)) {
+                    *abort_flag = 1;
+                    flag_error(p.err, PA_DEVERR_TIMEOUT);
                 }
             }
-            const float m_new = fmaxf(m, mx);
-            const float m_use = m_new == -INFINITY ? 0.f : m_new;
-            const float alpha = fast_exp2(m - m_use);
-            if (j > 0) {
-                // P and O are still in use by the previous tile's PV
-                live = wait_bar(pv_done, (j - 1) & 1, abort_flag, p.err);
+            __syncwarp();
+        } else {
+            // -------------------------------------------------------- softmax
+            const int r = (warp - 4) * 32 + lane;        // query row = TMEM lane
+            const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+            const bool row_ok = r < jb.nrows;
+            const int lim = jb.lim0 + jb.lim_step * (r / G);  // last key this row may see
+            float m = -INFINITY, l = 0.f;
+            bool live = true;
+            for (int j = 0; j < jb.ntiles; ++j) {
+                const int jt = tbase + j;
+                live = live && wait_bar(s_full, jt & 1, abort_flag, p.err);
                 live = __all_sync(kFull, live);
                 if (!live) break;
                 tc_fence_after();
-                if (__any_sync(kFull, alpha != 1.f)) {
+                // pass 1: row max of the scaled, masked scores (32 columns at a time)
+                float mx = -INFINITY;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float sv[32];
+                    tmem_ld32(tS + lane_off + c * 32, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int key = j * kTileN + c * 32 + k;
+                        if (row_ok && key <= lim) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                    }
+                }
+                const float m_new = fmaxf(m, mx);
+                const float m_use = m_new == -INFINITY ? 0.f : m_new;
+                const float alpha = fast_exp2(m - m_use);
+                if (j > 0) {
+                    // P and O are still in use by the previous tile's PV
+                    live = wait_bar(pv_done, (jt - 1) & 1, abort_flag, p.err);
+                    live = __all_sync(kFull, live);
+                    if (!live) break;
+                    tc_fence_after();
+                    if (__any_sync(kFull, alpha != 1.f)) {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            float ov[32];
+                            tmem_ld32(tO + lane_off + c * 32, ov);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) ov[k] *= alpha;
+                            tmem_st32(tO + lane_off + c * 32, ov);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+                // pass 2: P = 2^(s - m) as bf16 into the K-major swizzled A-operand tile
+                float rs = 0.f;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float sv[32];
+                    tmem_ld32(tS + lane_off + c * 32, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        const int key = j * kTileN + c * 32 + k;
+                        sv[k] = (row_ok && key <= lim) ? fast_exp2(sv[k] * p.scale_log2 - m_use) : 0.f;
+                        rs += sv[k];
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const float *x = &sv[q * 8];
+                        const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                                   pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                        *reinterpret_cast<uint4 *>(smem + kOffP + swz(r, c * 4 + q)) = w;
+                    }
+                }
+                l = l * alpha + rs;
+                m = m_new;
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (live) live = wait_bar(pv_done, (tbase + jb.ntiles - 1) & 1, abort_flag, p.err);
+            live = __all_sync(kFull, live);
+            if (live) {
+                tc_fence_after();
+                if constexpr (kGroup) {
+                    const int64_t wrow = ((int64_t)(jb.first + r / G) * p.num_q_heads + jb.h * G + r % G) * p.max_parts + jb.part;
+                    float *dst = p.ws_acc + wrow * kD;
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         float ov[32];
                         tmem_ld32(tO + lane_off + c * 32, ov);
                         tmem_wait_ld();
+                        if (row_ok) {
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) ov[k] *= alpha;
-                        tmem_st32(tO + lane_off + c * 32, ov);
+                            for (int k = 0; k < 32; k += 4)
+                                *reinterpret_cast<float4 *>(dst + c * 32 + k) = make_float4(ov[k], ov[k + 1], ov[k + 2], ov[k + 3]);
+                        }
                     }
-                    tmem_wait_st();
-                }
-            }
-            // pass 2: P = 2^(s - m) as bf16 into the K-major swizzled A-operand tile
-            float rs = 0.f;
+                    if (row_ok) p.ws_ml[wrow] = make_float2(m, l);
+                } else {
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    unsigned char *dst = jb.out + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float sv[32];
-                tmem_ld32(tS + lane_off + c * 32, sv);
-                tmem_wait_ld();
+                    for (int c = 0; c < 4; ++c) {
+                        float ov[32];
+                        tmem_ld32(tO + lane_off + c * 32, ov);
+                        tmem_wait_ld();
+                        if (row_ok) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) {
-                    const int key = j * kTileN + c * 32 + k;
-                    sv[k] = (row_ok && key <= pos) ? fast_exp2(sv[k] * p.scale_log2 - m_use) : 0.f;
-                    rs += sv[k];
-                }
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float *x = &sv[q * 8];
-                    const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-                    *reinterpret_cast<uint4 *>(smem + kOffP + swz(r, c * 4 + q)) = w;
-                }
-            }
-            l = l * alpha + rs;
-            m = m_new;
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(p_full);
-        }
-        if (live) live = wait_bar(pv_done, (ntiles - 1) & 1, abort_flag, p.err);
-        live = __all_sync(kFull, live);
-        if (live) {
-            tc_fence_after();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            unsigned char *dst = p.out + (((int64_t)s * p.max_chunk + i) * p.num_q_heads + h * G + r % G) * head_stride;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float ov[32];
-                tmem_ld32(tO + lane_off + c * 32, ov);
-                tmem_wait_ld();
-                if (row_ok) {
-#pragma unroll
-                    for (int k = 0; k < 32; k += 8) {
-                        const uint4 w = make_uint4(pack_bf16x2(ov[k] * inv, ov[k + 1] * inv),
-                                                   pack_bf16x2(ov[k + 2] * inv, ov[k + 3] * inv),
-                                                   pack_bf16x2(ov[k + 4] * inv, ov[k + 5] * inv),
-                                                   pack_bf16x2(ov[k + 6] * inv, ov[k + 7] * inv));
-                        *reinterpret_cast<uint4 *>(dst + (c * 32 + k) * 2) = w;
+                            for (int k = 0; k < 32; k += 8) {
+                                const uint4 w = make_uint4(pack_bf16x2(ov[k] * inv, ov[k + 1] * inv),
+                                                           pack_bf16x2(ov[k + 2] * inv, ov[k + 3] * inv),
+                                                           pack_bf16x2(ov[k + 4] * inv, ov[k + 5] * inv),
+                                                           pack_bf16x2(ov[k + 6] * inv, ov[k + 7] * inv));
+                                *reinterpret_cast<uint4 *>(dst + (c * 32 + k) * 2) = w;
+                            }
+                        }
                     }
                 }
             }
         }
+        tbase += jb.ntiles;
+        // the unit is finished by every role before Q, P and TMEM are reused
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (*abort_flag) break;
     }
     tc_fence_before();
     __syncthreads();
@@ -408,12 +527,21 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(const __grid_const
 
 template <int G>
 cudaError_t launch_g(const PrefillLaunch &a, const Params &prm, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     constexpr int rows = kTileM / G;
     dim3 grid((unsigned)((a.max_chunk + rows - 1) / rows), (unsigned)a.cache.num_kv_heads, (unsigned)a.num_seqs);
-    prefill_kernel<G><<<grid, kThreads, kSmemBytes, stream>>>(prm);
+    attn_tile_kernel<G, false><<<grid, kThreads, kSmemBytes, stream>>>(prm);
+    return cudaGetLastError();
+}
+
+template <int G>
+cudaError_t launch_group_g(const Params &prm, int sms, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attn_tile_kernel<G, true><<<(unsigned)sms, kThreads, kSmemBytes, stream>>>(prm);
     return cudaGetLastError();
 }
 
@@ -445,6 +573,34 @@ cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
         case 2: return launch_g<2>(a, prm, stream);
         case 4: return launch_g<4>(a, prm, stream);
         case 8: return launch_g<8>(a, prm, stream);
+        default: return cudaErrorNotSupported;
+    }
+}
+
+cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t stream) {
+    Params prm;
+    std::memset(&prm, 0, sizeof(prm));
+    prm.q = static_cast<const unsigned char *>(a.query);
+    prm.kc = static_cast<const unsigned char *>(a.key_cache);
+    prm.vc = static_cast<const unsigned char *>(a.value_cache);
+    prm.tables = a.block_tables;
+    prm.err = a.err;
+    prm.max_blocks = a.max_blocks_per_seq;
+    prm.num_q_heads = a.num_q_heads;
+    prm.num_kv_heads = a.num_kv_heads;
+    prm.num_blocks = a.num_blocks;
+    prm.scale_log2 = a.scale * kLog2e;
+    prm.groups = a.groups;
+    prm.meta = a.meta;
+    prm.ws_acc = a.ws_acc;
+    prm.ws_ml = a.ws_ml;
+    prm.part_tokens = a.partition_size;
+    prm.max_parts = a.max_partitions;
+    switch (a.num_q_heads / a.num_kv_heads) {
+        case 1: return launch_group_g<1>(prm, sms, stream);
+        case 2: return launch_group_g<2>(prm, sms, stream);
+        case 4: return launch_group_g<4>(prm, sms, stream);
+        case 8: return launch_group_g<8>(prm, sms, stream);
         default: return cudaErrorNotSupported;
     }
 }

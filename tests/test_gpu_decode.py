@@ -202,3 +202,77 @@ def test_device_index_errors_are_flagged_not_fatal():
     g.err_flag.zero_()
     check_close(ts.gpu_decode(step, 0), ts.oracle_decode(step), "bf16", "after flagged errors")
     assert pa.pa_wait(g.err_flag) == 0
+
+
+def _grouped_workload(g=4):
+    """Sibling structures the shared-prefix grouping must get right (g query heads
+    per kv head; a group takes at most 64 / g sequences)."""
+    rng = np.random.default_rng(21)
+    hkv, d = 4, 128
+    hq = g * hkv
+    # (parent tokens, [suffix lengths]) per family; forked parents end on a block
+    # boundary so that no sibling's first append needs a copy
+    spec = []
+    spec.append((1104, [int(x) for x in rng.integers(0, 300, size=20)]))   # 20 siblings: chunks of 16 + 4
+    spec.append((608, [5, 77, 130]))             # shares 38 full blocks
+    spec.append((400, [3, 9, 27, 81, 1, 0]))     # 6 siblings
+    spec.append((208, [40, 41]))                 # shares less than one 256-token partition
+    spec.append((512, [0, 0]))                   # members entirely inside the shared prefix
+    spec.append((333, []))                       # singleton (parent kept, partly filled last block)
+    nb = 20 + sum(-(-(pt + max(sx, default=0) + 2) // 16) * (len(sx) + 1) for pt, sx in spec)
+    wl = workloads.Workload(0, "groups", "bf16", nb, hq, hkv, d, 1.0 / np.sqrt(d),
+                            rng.permutation(nb).astype(np.int32))
+    seq = 0
+    seqs = []
+    for pt, sx in spec:
+        parent = 1000 + seq
+        wl.ops.append(("add", parent))
+        wl.ops.append(("append", parent, workloads.normal(rng, (pt, hkv, d), "bf16"),
+                       workloads.normal(rng, (pt, hkv, d), "bf16")))
+        if not sx:
+            seqs.append(parent)
+            continue
+        kids = []
+        for _ in sx:
+            wl.ops.append(("fork", parent, seq))
+            kids.append(seq)
+            seq += 1
+        wl.ops.append(("free", parent))
+        for kid, n in zip(kids, sx):
+            if n:
+                wl.ops.append(("append", kid, workloads.normal(rng, (n, hkv, d), "bf16"),
+                               workloads.normal(rng, (n, hkv, d), "bf16")))
+        seqs.extend(kids)
+    # a sequence that reuses family 0's prefix but is not next to it: not grouped, still correct
+    wl.ops.append(("fork", 0, 5000))
+    seqs.append(5000)
+    S = len(seqs)
+    wl.steps.append(workloads.Step(seqs, workloads.normal(rng, (S, hkv, d), "bf16"),
+                                   workloads.normal(rng, (S, hkv, d), "bf16"),
+                                   workloads.normal(rng, (S, hq, d), "bf16")))
+    return wl
+
+
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_shared_prefix_groups_match_oracle(g):
+    wl = _grouped_workload(g)
+    ts = TwoSided(wl)
+    step = wl.steps[0]
+    ts.append_step(step)
+    assert ts.pools_equal()
+    ref = ts.oracle_decode(step)
+    for part in (0, 48, 256, 512, 1024):
+        check_close(ts.gpu_decode(step, part), ref, "bf16", f"g{g} grouped decode partition {part}")
+    # members whose whole context lies inside the shared blocks: every partition
+    # comes from the group units (contexts cut back to 1024 and 512 tokens)
+    t, l = ts.tables(step.seqs)
+    l2 = l.copy()
+    l2[:4] = 1024
+    fam = [i for i, L in enumerate(l) if L == 513]
+    assert len(fam) == 2
+    l2[fam] = 512
+    ref2 = ts.oracle_decode(step, tables=t, lens=l2)
+    for part in (48, 256, 512, 1024):
+        got = ts.gpu_decode(step, part, tables=t, lens=l2, max_context=int(l.max()))
+        check_close(got, ref2, "bf16", f"g{g} fully shared members, partition {part}")
+    assert ts.err_flag() == 0
