@@ -128,8 +128,8 @@ PA_API pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_
  * Bytes of workspace pa_decode needs for a split (partitioned) context:
  * partials of num_seqs * num_q_heads * ceil(max_context_len / partition_size)
  * partitions (head_dim fp32 accumulators plus a running max and sum each), then
- * the shared-prefix group area (a shared-block count, a first-partition index
- * and a 16-byte group record per sequence, and a count word).  Returns 0 when partition_size <= 0
+ * the shared-prefix group area (a first-partition index and a 16-byte group
+ * record per sequence, and a count word).  Returns 0 when partition_size <= 0
  * (no split, no workspace).
  */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,
@@ -138,9 +138,9 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
 /*
  * Number of kernels one pa_decode call with these arguments launches on its
  * stream (for launch accounting and graph planning): 1 unsplit; 2 split (the
- * partition kernel and the combine); 5 split with dtype PA_BF16, head_dim 128 and
- * num_seqs <= 4096 (two shared-prefix detection kernels and the group kernel
- * run first).  0 when num_seqs <= 0.  Pure host function.
+ * partition kernel and the combine); 4 split with dtype PA_BF16, head_dim 128 and
+ * num_seqs <= 4096 (the shared-prefix detection kernel and the group kernel run
+ * first).  0 when num_seqs <= 0.  Pure host function.
  */
 PA_API int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype,
                                   int32_t partition_size);

@@ -74,9 +74,8 @@ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Shared-memory carve-up (byte offsets from the dynamic shared memory base).
 // Each warp owns kStagesPerWarp ring stages (K slab + V slab each): two, or one
-// when a stage is too large (fp32, head_dim 128).  The merge buffers are
-// double-buffered when they fit, else single-buffered (one more CTA barrier per
-// unit).
+// when a stage is too large (fp32, head_dim 128).  Two merge slots let the
+// merge of a unit run while the next unit streams (mbarrier hand-over).
 template <typename T, int D, int G>
 struct Layout {
     static constexpr int kElem = ElemBytes<T>::value;
@@ -86,7 +85,7 @@ struct Layout {
     static constexpr size_t kLimit = 232448;                    // sm_100 max dynamic smem per CTA
     static constexpr size_t kPBytes = sizeof(T) == 4 ? (size_t)kWarps * (16 * G + G) * 4 : 64;
     static constexpr size_t kMergeBytes = (size_t)kWarps * G * (D * 4 + 8);
-    static constexpr size_t kFixed = kPBytes + 16 + (size_t)(kMaxSplitSeqs + 1) * 4 + 64;
+    static constexpr size_t kFixed = kPBytes + 16 + 48 + (size_t)(kMaxSplitSeqs + 1) * 4 + 64;
     static constexpr int stages_fit(int bufs) {
         return (int)((kLimit - kFixed - bufs * kMergeBytes) / ((size_t)kWarps * kStageBytes));
     }
@@ -97,7 +96,8 @@ struct Layout {
     static constexpr size_t kOffP = kOffRing + (size_t)kWarps * kStagesPerWarp * kStageBytes;
     static constexpr size_t kOffMacc = align_up(kOffP + kPBytes, 16);
     static constexpr size_t kOffMml = kOffMacc + (size_t)kMergeBufs * kWarps * G * D * 4;
-    static constexpr size_t kOffCum = align_up(kOffMml + (size_t)kMergeBufs * kWarps * G * 8, 16);
+    static constexpr size_t kOffBar = align_up(kOffMml + (size_t)kMergeBufs * kWarps * G * 8, 16);
+    static constexpr size_t kOffCum = kOffBar + 48;  // 4 mbarriers + abort word
     static constexpr size_t smem_bytes(int cum_entries) { return kOffCum + (size_t)cum_entries * 4; }
 };
 
@@ -144,6 +144,7 @@ __device__ __forceinline__ int num_parts(const Params &p, int L) {
 
 struct Unit {
     int s, part, h;
+    int fp;  // first_part(s): partitions of s computed by group units
 };
 
 __device__ __forceinline__ int first_part(const Params &p, int s) {
@@ -158,7 +159,8 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t unit
                                         const int *cum, int S) {
     if (u < units_first) {
         const int s = (int)(u / hkv);
-        return Unit{s, first_part(p, s), (int)(u % hkv)};
+        const int fp = first_part(p, s);
+        return Unit{s, fp, (int)(u % hkv), fp};
     }
     const int64_t v = u - units_first;
     const int e = (int)(v / hkv), h = (int)(v % hkv);
@@ -167,7 +169,8 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t unit
         const int mid = (lo + hi) >> 1;
         if (cum[mid] <= e) lo = mid; else hi = mid;
     }
-    return Unit{lo, first_part(p, lo) + 1 + e - cum[lo], h};
+    const int fp = first_part(p, lo);
+    return Unit{lo, fp + 1 + e - cum[lo], h, fp};
 }
 
 // What one warp needs to know about a unit.  `tab` holds, in lane i, the table
@@ -283,7 +286,7 @@ template <typename T, int D, int G>
 __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, const float *uacc,
                                             const float2 *uml) {
     if (w.skip) return;
-    const bool single = num_parts(p, w.L) == 1 && first_part(p, w.un.s) == 0;
+    const bool single = num_parts(p, w.L) == 1 && w.un.fp == 0;
     const int64_t head0 = (int64_t)w.un.s * p.num_q_heads + (int64_t)w.un.h * G;
     for (int e = threadIdx.x; e < G * D; e += kThreads) {
         const int h = e / D, dd = e - h * D;
@@ -303,7 +306,7 @@ __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, 
             }
         }
         if (single) {
-            store_out<T>(p.out, (head0 + h) * D + dd, lsum > 0.f ? o / lsum : 0.f);
+            store_out<T>(p.out, (head0 + h) * D + dd, lsum > 0.f ? o * (1.f / lsum) : 0.f);
         } else {
             const int64_t row = (head0 + h) * p.max_parts + w.un.part;
             p.ws_acc[row * D + dd] = o;
@@ -552,6 +555,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     float2 *mml = reinterpret_cast<float2 *>(smem + Lay::kOffMml);
     int *cum = reinterpret_cast<int *>(smem + Lay::kOffCum);
 
+    static_assert(Lay::kMergeBufs == 2, "the deferred merge needs two slots");
+    // merge slot hand-over: full[b] when all warps wrote their state of the
+    // slot's unit, freed[b] when all warps finished their share of its merge
+    uint64_t *mfull = reinterpret_cast<uint64_t *>(smem + Lay::kOffBar);
+    uint64_t *mfreed = mfull + 2;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + Lay::kOffBar + 32);
+    if (threadIdx.x == 0) {
+        mbar_init(&mfull[0], kWarps);
+        mbar_init(&mfull[1], kWarps);
+        mbar_init(&mfreed[0], kWarps);
+        mbar_init(&mfreed[1], kWarps);
+        *abort_flag = 0;
+        mbar_init_fence();
+    }
     prologue(p, cum, reinterpret_cast<int *>(macc));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.num_seqs, hkv = p.num_kv_heads;
@@ -608,7 +625,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         return true;
     };
 
-    for (int uc = 0;; ++uc) {
+    WarpUnit prv;            // unit whose merge is still to be finished
+    bool dead = false;       // a hand-over wait timed out
+    int uc = 0;
+    for (;; ++uc) {
         // ---- q operands of this unit (tiny, L2 resident)
         MmaState<D> ms;
         F32State<D, G> fs;
@@ -669,8 +689,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         while (n_iss - n_cmp < NS && fetch_one()) {
         }
 
-        // ---- merge the warps' states for this unit
-        const int b = Lay::kMergeBufs == 2 ? (uc & 1) : 0;
+        // ---- this warp's state into merge slot uc & 1, once the slot's previous
+        // unit (uc - 2) has been merged by every warp
+        const int b = uc & 1;
+        if (uc >= 2 && !mbar_wait_bounded(&mfreed[b], ((uc - 2) >> 1) & 1, abort_flag, p.err)) {
+            dead = true;
+            break;
+        }
         float *wacc = macc + ((size_t)b * kWarps + warp) * G * D;
         float2 *wml = mml + ((size_t)b * kWarps + warp) * G;
         if constexpr (kMma) {
@@ -696,9 +721,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                     *reinterpret_cast<float2 *>(wacc + h * D + lane * C::kDpl + 2 * k) = fs.acc[h][k];
             if (tq == 0 && (part & C::kDupMask) == 0) wml[part >> (3 - C::kLogG)] = make_float2(fs.m, fs.l);
         }
-        __syncthreads();
-        finish_unit<T, D, G>(p, cur, macc + (size_t)b * kWarps * G * D, mml + (size_t)b * kWarps * G);
-        if constexpr (Lay::kMergeBufs == 1) __syncthreads();  // buffer is rewritten next unit
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&mfull[b]);
+        // ---- this warp's share of the previous unit's merge (its states are
+        // all in by now unless a warp is a whole unit behind)
+        if (uc >= 1) {
+            const int pb = b ^ 1;
+            if (!mbar_wait_bounded(&mfull[pb], ((uc - 1) >> 1) & 1, abort_flag, p.err)) {
+                dead = true;
+                break;
+            }
+            finish_unit<T, D, G>(p, prv, macc + (size_t)pb * kWarps * G * D, mml + (size_t)pb * kWarps * G);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mfreed[pb]);
+        }
+        prv = cur;
 
         // ---- advance: the fetch cursor moves down one unit with the window
         u += gridDim.x;
@@ -709,6 +746,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         have_nxt = u + gridDim.x < total;
         if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
     }
+    // the last unit's merge
+    if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err))
+        finish_unit<T, D, G>(p, prv, macc + (size_t)(uc & 1) * kWarps * G * D, mml + (size_t)(uc & 1) * kWarps * G);
     cp_async_wait<0>();
 }
 
@@ -720,53 +760,66 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 // kernel starts after them.  Results are unchanged -- the same partials land in
 // the same workspace slots and the LSE reduce combines them.
 //
-// Detection takes two launches: group_lcp_kernel (a warp per sequence) counts the
-// leading full blocks each sequence shares with its predecessor; group_form_kernel
-// (one CTA) cuts the batch into chunks and lists them.  The group units -- a
-// dense (members x g) x partition x head_dim attention tile each -- run on the
-// tcgen05 tile kernel of prefill.cu (launch_group_tiles).
+// Detection is one single-CTA kernel: each sequence's count of leading full
+// blocks shared with its predecessor, then the cut of the batch into groups.
+// The group units -- a dense (members x g) x partition x head_dim attention
+// tile each -- run on the tcgen05 tile kernel of prefill.cu (launch_group_tiles).
 
-constexpr int kLcpWarps = 8;
 constexpr int kDetectThreads = 1024;
 constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
 constexpr int kMaxGroupParts = (1 << 23) - 1;
+constexpr int kLcpBatch = 8;         // sequences a warp compares at once
 
 // lcp[s] = leading entries of s's table equal to those of s-1, counted over the
-// blocks both contexts fill completely (0 for s = 0).  128 entries per round.
-__global__ void __launch_bounds__(kLcpWarps * 32) group_lcp_kernel(const __grid_constant__ Params p,
-                                                                   int32_t *lcp) {
-    const int lane = threadIdx.x & 31;
-    const int nw = gridDim.x * kLcpWarps;
-    for (int s = blockIdx.x * kLcpWarps + (threadIdx.x >> 5); s < p.num_seqs; s += nw) {
-        int n = 0;
-        if (s > 0) {
-            const int La = checked_len(p, s), Lb = checked_len(p, s - 1);
-            n = min(max(La, 0), max(Lb, 0)) / kBlockSize;
-        }
-        const int32_t *ta = p.tables + (int64_t)s * p.max_blocks;
-        const int32_t *tb = ta - p.max_blocks;  // read only when n > 0, i.e. s > 0
-        int res = n;
-        for (int c0 = 0; c0 < n; c0 += 128) {
-            int a[4], b[4];
+// blocks both contexts fill completely (0 for s = 0).  A warp takes kLcpBatch
+// sequences at a time and compares 64 entries of each per round.
+__device__ __forceinline__ void shared_prefix_lengths(const Params &p, int *lcp) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int S = p.num_seqs;
+    for (int base = warp * kLcpBatch; base < S; base += (kDetectThreads / 32) * kLcpBatch) {
+        int n[kLcpBatch], res[kLcpBatch];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = c0 + 32 * k + lane;
-                a[k] = i < n ? __ldg(ta + i) : 0;
-                b[k] = i < n ? __ldg(tb + i) : 0;
+        for (int b = 0; b < kLcpBatch; ++b) {
+            const int s = base + b;
+            n[b] = 0;
+            if (s > 0 && s < S) {
+                const int La = checked_len(p, s), Lb = checked_len(p, s - 1);
+                n[b] = min(max(La, 0), max(Lb, 0)) / kBlockSize;
             }
-            int mis = n;
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = c0 + 32 * k + lane;
-                if (i < n && a[k] != b[k]) mis = min(mis, i);
-            }
-            mis = __reduce_min_sync(kFull, mis);
-            if (mis < n) {
-                res = mis;
-                break;
-            }
+            res[b] = n[b];  // == n: no difference found yet
         }
-        if (lane == 0) lcp[s] = res;
+        for (int c0 = 0;; c0 += 64) {
+            int va[kLcpBatch][2], vb[kLcpBatch][2];
+#pragma unroll
+            for (int b = 0; b < kLcpBatch; ++b) {
+                const int32_t *ta = p.tables + (int64_t)(base + b) * p.max_blocks;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int i = c0 + 32 * k + lane;
+                    const bool act = res[b] == n[b] && i < n[b];  // implies 0 < s < S
+                    va[b][k] = act ? __ldg(ta + i) : 0;
+                    vb[b][k] = act ? __ldg(ta - p.max_blocks + i) : 0;
+                }
+            }
+            bool more = false;
+#pragma unroll
+            for (int b = 0; b < kLcpBatch; ++b) {
+                if (res[b] != n[b] || c0 >= n[b]) continue;  // warp-uniform
+                int mis = n[b];
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int i = c0 + 32 * k + lane;
+                    if (i < n[b] && va[b][k] != vb[b][k]) mis = min(mis, i);
+                }
+                mis = __reduce_min_sync(kFull, mis);
+                if (mis < n[b]) res[b] = mis;
+                else more = more || c0 + 64 < n[b];
+            }
+            if (!more) break;
+        }
+#pragma unroll
+        for (int b = 0; b < kLcpBatch; ++b)
+            if (lane == 0 && base + b < S) lcp[base + b] = res[b];
     }
 }
 
@@ -796,9 +849,9 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int identity, int *wb
 // sequences shares min(lcp over its members after the first) blocks, i.e. np
 // whole partitions; it becomes one group with np x num_kv_heads units.
 // first_p[s] = np of s's chunk (0 for a chunk of one).
-__global__ void __launch_bounds__(kDetectThreads) group_form_kernel(const __grid_constant__ Params p,
-                                                                    const int32_t *lcp_g, int32_t *first_p,
-                                                                    int4 *groups, int32_t *meta) {
+__global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __grid_constant__ Params p,
+                                                                      int32_t *first_p, int4 *groups,
+                                                                      int32_t *meta) {
     __shared__ int lcp[kMaxGroupSeqs];
     __shared__ int info[kMaxGroupSeqs];  // at a chunk head: np << 8 | members (members <= 128); else -1
     __shared__ int wbuf[kDetectThreads / 32];
@@ -806,12 +859,14 @@ __global__ void __launch_bounds__(kDetectThreads) group_form_kernel(const __grid
     const int S = p.num_seqs, tid = threadIdx.x;
     const int bpp = p.part_tokens / kBlockSize, M = p.max_members;
     const int s0 = tid * kPer;
+    shared_prefix_lengths(p, lcp);
+    __syncthreads();
     // run starts: max-scan of (run head ? s : -1)
     int lv[kPer], mx = -1;
 #pragma unroll
     for (int k = 0; k < kPer; ++k) {
         const int s = s0 + k;
-        lv[k] = s < S ? __ldg(lcp_g + s) : 0;
+        lv[k] = s < S ? lcp[s] : 0;
         if (s < S && (s == 0 || lv[k] < bpp)) mx = s;
     }
     int rs = block_exclusive_scan<true>(mx, -1, wbuf);
@@ -820,7 +875,6 @@ __global__ void __launch_bounds__(kDetectThreads) group_form_kernel(const __grid
         const int s = s0 + k;
         if (s >= S) break;
         if (s == 0 || lv[k] < bpp) rs = s;
-        lcp[s] = lv[k];
         info[s] = (s - rs) % M == 0 ? 0 : -1;  // chunk heads marked 0 for now
     }
     __syncthreads();
@@ -918,20 +972,15 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
     if constexpr (sizeof(T) == 2 && D == 128) {
         if (split && a.ws_group && a.num_seqs <= kMaxGroupSeqs) {
             unsigned char *g = static_cast<unsigned char *>(a.ws_group);
-            // group area: lcp[S], first_p[S] (each 16-byte padded), groups[S], meta
+            // group area: first_p[S] (16-byte padded), groups[S], meta
             const size_t sa = ((size_t)a.num_seqs * 4 + 15) / 16 * 16;
-            int32_t *lcp = reinterpret_cast<int32_t *>(g);
-            prm.first_p = reinterpret_cast<int32_t *>(g + sa);
-            prm.groups = reinterpret_cast<int4 *>(g + 2 * sa);
+            prm.first_p = reinterpret_cast<int32_t *>(g);
+            prm.groups = reinterpret_cast<int4 *>(g + sa);
             prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
             prm.max_members = 128 / G;
-            const int lcp_grid = (int)std::min<int64_t>(((int64_t)a.num_seqs + kLcpWarps - 1) / kLcpWarps,
-                                                        (int64_t)sms * 4);
-            group_lcp_kernel<<<std::max(lcp_grid, 1), kLcpWarps * 32, 0, stream>>>(prm, lcp);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-            group_form_kernel<<<1, kDetectThreads, 0, stream>>>(prm, lcp, const_cast<int32_t *>(prm.first_p),
-                                                                const_cast<int4 *>(prm.groups),
-                                                                const_cast<int32_t *>(prm.meta));
+            group_detect_kernel<<<1, kDetectThreads, 0, stream>>>(prm, const_cast<int32_t *>(prm.first_p),
+                                                                  const_cast<int4 *>(prm.groups),
+                                                                  const_cast<int32_t *>(prm.meta));
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
             GroupTileLaunch gl;
             gl.query = a.query;

@@ -99,10 +99,10 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
     const int64_t parts = ((int64_t)max_context_len + partition_size - 1) / partition_size;
     const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
     // partials (fp32 acc, then (m, l)), then the shared-prefix group bookkeeping:
-    // shared-block count and first partition per sequence (each 16-byte padded),
-    // group list (16 bytes each), 16 bytes of counters
+    // first partition per sequence (16-byte padded), group list (16 bytes each),
+    // 16 bytes of counters
     const int64_t partials = rows * head_dim * 4 + rows * 8;
-    const int64_t group = 2 * (((int64_t)num_seqs * 4 + 15) / 16 * 16) + (int64_t)num_seqs * 16 + 16;
+    const int64_t group = ((int64_t)num_seqs * 4 + 15) / 16 * 16 + (int64_t)num_seqs * 16 + 16;
     return (size_t)((partials + 15) / 16 * 16 + group);
 }
 
@@ -110,7 +110,7 @@ int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype, in
     if (num_seqs <= 0) return 0;
     if (partition_size <= 0) return 1;
     const bool grouped = dtype == PA_BF16 && head_dim == 128 && num_seqs <= kMaxSplitSeqs;
-    return grouped ? 5 : 2;
+    return grouped ? 4 : 2;
 }
 
 pa_status pa_decode(const void *query, const void *key_cache, const void *value_cache,

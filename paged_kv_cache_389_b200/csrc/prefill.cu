@@ -17,10 +17,11 @@
 //   O  += P V        tcgen05.mma, A = P (bf16, smem), B = V (MN-major), -> TMEM
 // Warp roles: warps 0-3 load (16-byte cp.async into 128-byte-swizzled layouts:
 // Q and K K-major, V MN-major, the canonical layouts the MMA descriptors name),
-// warps 4-7 run the softmax (TMEM lanes 0..127), warp 8 owns the tensor memory
-// and issues the MMAs from one thread.  K/V tiles are double-buffered; the
-// stages are handed over with mbarriers; every wait is bounded and an abort
-// still frees the tensor memory.
+// warps 4-11 run the softmax (warp w: TMEM lanes 32*(w%4)..+31, one 64-column
+// half of the tile), warp 12 owns the tensor memory and issues the MMAs from one
+// thread.  K/V tiles are double-buffered and loaded two deep; the stages are
+// handed over with mbarriers; every wait is bounded and an abort still frees
+// the tensor memory.
 #include <cstring>
 
 #include "pa_common.cuh"
@@ -34,8 +35,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kD = 128;              // head_dim (bf16 only)
 constexpr int kTileM = 128;          // query rows per CTA
 constexpr int kTileN = 128;          // keys per KV tile
-constexpr int kThreads = 9 * 32;     // 4 load warps, 4 softmax warps, 1 MMA warp
-constexpr int kMmaWarp = 8;
+constexpr int kThreads = 13 * 32;    // 4 load warps, 8 softmax warps, 1 MMA warp
+constexpr int kMmaWarp = 12;
+constexpr int kSoftmaxThreads = 256;
 constexpr uint32_t kTmemCols = 256;  // S: columns 0..127, O: 128..255
 
 // shared memory (offsets from a 1024-byte aligned base)
@@ -48,7 +50,9 @@ constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffP + kTileBytes;
 constexpr uint32_t kOffTab = kOffBar + 16 * 8;     // 8 table entries per stage
 constexpr uint32_t kOffMisc = kOffTab + 2 * 8 * 4;
-constexpr uint32_t kOffGcum = kOffMisc + 16;         // group units: units before each group
+constexpr uint32_t kOffRed = kOffMisc + 16;          // row-max halves [2 tiles][2 halves][128 rows]
+constexpr uint32_t kOffLsum = kOffRed + 2 * 2 * 128 * 4;  // row-sum halves [2][128]
+constexpr uint32_t kOffGcum = kOffLsum + 2 * 128 * 4;  // group units: units before each group
 constexpr int kMaxGroups = 2048;                     // a group has >= 2 of <= 4096 sequences
 constexpr size_t kSmemBytes = 1024 + kOffGcum + kMaxGroups * 4;
 
@@ -224,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     uint64_t *p_full = bars + 6;
     uint64_t *pv_done = bars + 7;
     uint64_t *mma_idle = bars + 8;
+    uint64_t *red_full = bars + 9;  // [2]
+    uint64_t *l_full = bars + 11;
     int *tab = reinterpret_cast<int *>(smem + kOffTab);  // [2][8]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
@@ -273,9 +279,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
         mbar_init(&kv_empty[0], 1);
         mbar_init(&kv_empty[1], 1);
         mbar_init(s_full, 1);
-        mbar_init(p_full, 128);
+        mbar_init(p_full, kSoftmaxThreads);
         mbar_init(pv_done, 1);
         mbar_init(mma_idle, 1);
+        mbar_init(&red_full[0], kSoftmaxThreads);
+        mbar_init(&red_full[1], kSoftmaxThreads);
+        mbar_init(l_full, kSoftmaxThreads);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -307,11 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     *reinterpret_cast<uint4 *>(smem + kOffQ + swz(r, c)) = make_uint4(0, 0, 0, 0);
             }
             cp_async_commit();
-            bool q_sent = false;
-            for (int j = 0; j < jb.ntiles; ++j) {
+            // Tile j's copies are issued into stage (tbase+j) & 1 once the MMA has
+            // released that stage; tile j+1 is issued before tile j is waited
+            // for, so two tiles are in flight.  The decision to go on reaches
+            // all loaders through shared memory behind a barrier.
+            auto issue_tile = [&](int j) -> bool {
                 const int jt = tbase + j, st = jt & 1;
-                // one thread waits for the stage; the decision reaches all loaders
-                // through shared memory behind the barrier, so they break together
                 if (t == 0) *go = (jt < 2 || wait_bar(&kv_empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
                 // table entries of the tile's 8 blocks (-1: past the keys)
                 if (t < 8) {
@@ -327,34 +337,38 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     tab[st * 8 + t] = e;
                 }
                 named_barrier(1, 128);
-                if (!*go) break;
-                const uint32_t kst = sbase + kOffK + st * kTileBytes, vst = sbase + kOffV + st * kTileBytes;
-                unsigned char *kgen = smem + kOffK + st * kTileBytes, *vgen = smem + kOffV + st * kTileBytes;
-                for (int idx = t; idx < kTileN * 16; idx += 128) {
-                    const int n = idx >> 4, c = idx & 15;
-                    const int key = j * kTileN + n;
-                    const int blk = tab[st * 8 + (n >> 4)];
-                    const uint32_t off = swz(n, c);
-                    if (blk >= 0 && key < jb.nkeys) {
-                        const int64_t src = (((int64_t)blk * p.num_kv_heads + jb.h) * kBlockSize + (n & 15)) * hs + c * 16;
-                        cp_async16(kst + off, p.kc + src);
-                        cp_async16(vst + off, p.vc + src);
-                    } else {  // past the keys or a bad id: zeros (0 * garbage must not reach the sums)
-                        *reinterpret_cast<uint4 *>(kgen + off) = make_uint4(0, 0, 0, 0);
-                        *reinterpret_cast<uint4 *>(vgen + off) = make_uint4(0, 0, 0, 0);
+                const bool ok = *go != 0;
+                if (ok) {
+                    const uint32_t kst = sbase + kOffK + st * kTileBytes, vst = sbase + kOffV + st * kTileBytes;
+                    unsigned char *kgen = smem + kOffK + st * kTileBytes, *vgen = smem + kOffV + st * kTileBytes;
+                    for (int idx = t; idx < kTileN * 16; idx += 128) {
+                        const int n = idx >> 4, c = idx & 15;
+                        const int key = j * kTileN + n;
+                        const int blk = tab[st * 8 + (n >> 4)];
+                        const uint32_t off = swz(n, c);
+                        if (blk >= 0 && key < jb.nkeys) {
+                            const int64_t src = (((int64_t)blk * p.num_kv_heads + jb.h) * kBlockSize + (n & 15)) * hs + c * 16;
+                            cp_async16(kst + off, p.kc + src);
+                            cp_async16(vst + off, p.vc + src);
+                        } else {  // past the keys or a bad id: zeros (0 * garbage must not reach the sums)
+                            *reinterpret_cast<uint4 *>(kgen + off) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(vgen + off) = make_uint4(0, 0, 0, 0);
+                        }
                     }
                 }
                 cp_async_commit();
-                if (!q_sent) {  // the Q copies overlap the first K/V tile's
-                    cp_async_wait<1>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(q_full);
-                    q_sent = true;
-                }
-                cp_async_wait<0>();
+                named_barrier(1, 128);  // tab and *go are rewritten by the next issue
+                return ok;
+            };
+            bool ok = jb.ntiles > 0 && issue_tile(0);
+            for (int j = 0; ok && j < jb.ntiles; ++j) {
+                const bool more = j + 1 < jb.ntiles;
+                if (more && !issue_tile(j + 1)) break;
+                // groups so far: Q, tiles 0..j (+ j+1): all but the newest are done
+                if (more) cp_async_wait<1>(); else cp_async_wait<0>();
                 fence_proxy_async_smem();
-                mbar_arrive(&kv_full[st]);
-                named_barrier(1, 128);  // tab[st] and *go are rewritten next iteration
+                if (j == 0) mbar_arrive(q_full);
+                mbar_arrive(&kv_full[(tbase + j) & 1]);
             }
             cp_async_wait<0>();  // nothing may land after an abort
         } else if (warp == kMmaWarp) {
@@ -395,31 +409,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             __syncwarp();
         } else {
             // -------------------------------------------------------- softmax
-            const int r = (warp - 4) * 32 + lane;        // query row = TMEM lane
-            const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+            // Warp w owns TMEM lane quadrant w % 4 (rows 32*(w%4)..+31) and column
+            // half hf of S, O and P.  The two halves of a row trade their partial
+            // maxima through shared memory each tile (bounded mbarrier) and add
+            // their partial sums at the end.
+            const int qd = warp & 3, hf = (warp - 4) >> 2;
+            const int r = qd * 32 + lane;                // query row = TMEM lane
+            const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+            const uint32_t cS = tS + lane_off + hf * 64, cO = tO + lane_off + hf * 64;
+            float *red = reinterpret_cast<float *>(smem + kOffRed);    // [2][2][128]
+            float *lsum = reinterpret_cast<float *>(smem + kOffLsum);  // [2][128]
             const bool row_ok = r < jb.nrows;
-            const int lim = jb.lim0 + jb.lim_step * (r / G);  // last key this row may see
+            const bool warp_rows = __any_sync(kFull, row_ok);         // any real row in this warp
+            const int lim = jb.lim0 + jb.lim_step * (r / G);          // last key this row may see
             float m = -INFINITY, l = 0.f;
             bool live = true;
             for (int j = 0; j < jb.ntiles; ++j) {
                 const int jt = tbase + j;
+                const int key0 = j * kTileN + hf * 64;                // first key of this half
+                // the whole half is visible to every row of the warp: no per-key test
+                const bool open = __all_sync(kFull, row_ok && lim >= key0 + 63);
                 live = live && wait_bar(s_full, jt & 1, abort_flag, p.err);
                 live = __all_sync(kFull, live);
                 if (!live) break;
                 tc_fence_after();
-                // pass 1: row max of the scaled, masked scores (32 columns at a time)
+                // pass 1: partial row max of the scaled, masked scores
                 float mx = -INFINITY;
+                if (warp_rows) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float sv[32];
-                    tmem_ld32(tS + lane_off + c * 32, sv);
-                    tmem_wait_ld();
+                    for (int c = 0; c < 2; ++c) {
+                        float sv[32];
+                        tmem_ld32(cS + c * 32, sv);
+                        tmem_wait_ld();
+                        if (open) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int key = j * kTileN + c * 32 + k;
-                        if (row_ok && key <= lim) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 32; ++k)
+                                if (row_ok && key0 + c * 32 + k <= lim) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                        }
                     }
                 }
+                float *rb = red + (jt & 1) * 256;
+                rb[hf * 128 + r] = mx;
+                mbar_arrive(&red_full[jt & 1]);
+                live = wait_bar(&red_full[jt & 1], (jt >> 1) & 1, abort_flag, p.err);
+                live = __all_sync(kFull, live);
+                if (!live) break;
+                mx = fmaxf(rb[r], rb[128 + r]);
                 const float m_new = fmaxf(m, mx);
                 const float m_use = m_new == -INFINITY ? 0.f : m_new;
                 const float alpha = fast_exp2(m - m_use);
@@ -429,38 +467,47 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     live = __all_sync(kFull, live);
                     if (!live) break;
                     tc_fence_after();
-                    if (__any_sync(kFull, alpha != 1.f)) {
+                    if (warp_rows && __any_sync(kFull, alpha != 1.f)) {
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
+                        for (int c = 0; c < 2; ++c) {
                             float ov[32];
-                            tmem_ld32(tO + lane_off + c * 32, ov);
+                            tmem_ld32(cO + c * 32, ov);
                             tmem_wait_ld();
 #pragma unroll
                             for (int k = 0; k < 32; ++k) ov[k] *= alpha;
-                            tmem_st32(tO + lane_off + c * 32, ov);
+                            tmem_st32(cO + c * 32, ov);
                         }
                         tmem_wait_st();
                     }
                 }
-                // pass 2: P = 2^(s - m) as bf16 into the K-major swizzled A-operand tile
+                // pass 2: P = 2^(s - m) as bf16 into this half of the K-major swizzled A tile
                 float rs = 0.f;
+                if (warp_rows) {
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float sv[32];
-                    tmem_ld32(tS + lane_off + c * 32, sv);
-                    tmem_wait_ld();
+                    for (int c = 0; c < 2; ++c) {
+                        float sv[32];
+                        tmem_ld32(cS + c * 32, sv);
+                        tmem_wait_ld();
+                        if (open) {
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) {
-                        const int key = j * kTileN + c * 32 + k;
-                        sv[k] = (row_ok && key <= lim) ? fast_exp2(sv[k] * p.scale_log2 - m_use) : 0.f;
-                        rs += sv[k];
-                    }
+                            for (int k = 0; k < 32; ++k) {
+                                sv[k] = fast_exp2(sv[k] * p.scale_log2 - m_use);
+                                rs += sv[k];
+                            }
+                        } else {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const float *x = &sv[q * 8];
-                        const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                                                   pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-                        *reinterpret_cast<uint4 *>(smem + kOffP + swz(r, c * 4 + q)) = w;
+                            for (int k = 0; k < 32; ++k) {
+                                sv[k] = (row_ok && key0 + c * 32 + k <= lim) ? fast_exp2(sv[k] * p.scale_log2 - m_use) : 0.f;
+                                rs += sv[k];
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float *x = &sv[q * 8];
+                            const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                                       pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+                            *reinterpret_cast<uint4 *>(smem + kOffP + swz(r, hf * 8 + c * 4 + q)) = w;
+                        }
                     }
                 }
                 l = l * alpha + rs;
@@ -472,14 +519,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             if (live) live = wait_bar(pv_done, (tbase + jb.ntiles - 1) & 1, abort_flag, p.err);
             live = __all_sync(kFull, live);
             if (live) {
+                lsum[hf * 128 + r] = l;
+                mbar_arrive(l_full);
+                live = wait_bar(l_full, nu & 1, abort_flag, p.err);
+                live = __all_sync(kFull, live);
+            }
+            if (live && warp_rows) {
                 tc_fence_after();
+                const float lt = lsum[r] + lsum[128 + r];
                 if constexpr (kGroup) {
                     const int64_t wrow = ((int64_t)(jb.first + r / G) * p.num_q_heads + jb.h * G + r % G) * p.max_parts + jb.part;
-                    float *dst = p.ws_acc + wrow * kD;
+                    float *dst = p.ws_acc + wrow * kD + hf * 64;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         float ov[32];
-                        tmem_ld32(tO + lane_off + c * 32, ov);
+                        tmem_ld32(cO + c * 32, ov);
                         tmem_wait_ld();
                         if (row_ok) {
 #pragma unroll
@@ -487,14 +541,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                                 *reinterpret_cast<float4 *>(dst + c * 32 + k) = make_float4(ov[k], ov[k + 1], ov[k + 2], ov[k + 3]);
                         }
                     }
-                    if (row_ok) p.ws_ml[wrow] = make_float2(m, l);
+                    if (row_ok && hf == 0) p.ws_ml[wrow] = make_float2(m, lt);
                 } else {
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
-                    unsigned char *dst = jb.out + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs;
+                    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+                    unsigned char *dst = jb.out + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs + hf * 128;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         float ov[32];
-                        tmem_ld32(tO + lane_off + c * 32, ov);
+                        tmem_ld32(cO + c * 32, ov);
                         tmem_wait_ld();
                         if (row_ok) {
 #pragma unroll

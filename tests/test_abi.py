@@ -84,18 +84,18 @@ def test_host_validation_launches_nothing(pa):
 
 def test_workspace_size_formula(pa):
     # partials: rows = S * Hq * ceil(maxctx / part), each head_dim fp32 + (m, l);
-    # then the shared-prefix group area: S int32 shared-block counts and S int32
-    # first partitions (each 16-byte padded), S int4 group records, 16 count bytes.
+    # then the shared-prefix group area: S int32 first partitions (16-byte
+    # padded), S int4 group records, 16 count bytes.
     def a16(x):
         return (x + 15) // 16 * 16
 
     def expect(S, hq, d, ctx, part):
         rows = S * hq * (-(-ctx // part))
-        return a16(rows * (d * 4 + 8)) + 2 * a16(S * 4) + S * 16 + 16
+        return a16(rows * (d * 4 + 8)) + a16(S * 4) + S * 16 + 16
 
     assert pa.pa_decode_workspace_size(8, 64, 128, 32768, 512) == expect(8, 64, 128, 32768, 512)
     assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == expect(3, 4, 64, 100, 32)
-    assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == 3 * 4 * 4 * (64 * 4 + 8) + 32 + 48 + 16
+    assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == 3 * 4 * 4 * (64 * 4 + 8) + 16 + 48 + 16
     assert pa.pa_decode_workspace_size(3, 4, 64, 100, 0) == 0
 
 
@@ -104,5 +104,5 @@ def test_decode_launch_count(pa):
     assert pa.pa_decode_launches(8, 128, pa.PA_BF16, 0) == 1
     assert pa.pa_decode_launches(8, 128, pa.PA_F32, 512) == 2
     assert pa.pa_decode_launches(8, 64, pa.PA_BF16, 512) == 2
-    assert pa.pa_decode_launches(4096, 128, pa.PA_BF16, 512) == 5
+    assert pa.pa_decode_launches(4096, 128, pa.PA_BF16, 512) == 4
 
