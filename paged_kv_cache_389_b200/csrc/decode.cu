@@ -531,14 +531,6 @@ __device__ __forceinline__ void f32_block(const unsigned char *kb, const unsigne
 }
 
 // ------------------------------------------------------------- the kernel
-// cp.async.wait_group with a run-time count (at most 3 groups pending here).
-__device__ __forceinline__ void cp_async_wait_dyn(int pending) {
-    if (pending <= 0) cp_async_wait<0>();
-    else if (pending == 1) cp_async_wait<1>();
-    else if (pending == 2) cp_async_wait<2>();
-    else cp_async_wait<3>();
-}
-
 // Blocks of the warp's work, one after another: blocks w, w+8, ... of the current
 // unit, then of the next one.  Each is fetched with cp.async up to NS items before
 // it is computed.  (An extra prefetch.global.L2 a few items further ahead measured
@@ -556,6 +548,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     int *cum = reinterpret_cast<int *>(smem + Lay::kOffCum);
 
     static_assert(Lay::kMergeBufs == 2, "the deferred merge needs two slots");
+    // The combine may start launching now; it waits for this grid to finish.
+    // When launched behind the group tiles, this grid reads only what the
+    // detection wrote (complete before the tiles let it start) and writes other
+    // partitions; it waits for the tiles only before exiting, so that its
+    // completion implies theirs.
+    grid_dep_launch();
     // merge slot hand-over: full[b] when all warps wrote their state of the
     // slot's unit, freed[b] when all warps finished their share of its merge
     uint64_t *mfull = reinterpret_cast<uint64_t *>(smem + Lay::kOffBar);
@@ -581,7 +579,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
     WarpUnit cur, nxt;
     int64_t u = blockIdx.x;
-    if (u >= total) return;
+    if (u >= total) {
+        grid_dep_wait();
+        return;
+    }
     load_unit(p, u, units_first, cum, cur, lane, warp == 0);
     bool have_nxt = u + gridDim.x < total;
     if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
@@ -750,6 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err))
         finish_unit<T, D, G>(p, prv, macc + (size_t)(uc & 1) * kWarps * G * D, mml + (size_t)(uc & 1) * kWarps * G);
     cp_async_wait<0>();
+    grid_dep_wait();
 }
 
 // ------------------------------------------------------------- shared prefixes
@@ -855,6 +857,7 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     __shared__ int lcp[kMaxGroupSeqs];
     __shared__ int info[kMaxGroupSeqs];  // at a chunk head: np << 8 | members (members <= 128); else -1
     __shared__ int wbuf[kDetectThreads / 32];
+    grid_dep_launch();  // the group tiles set up while this runs, then wait for it
     constexpr int kPer = kMaxGroupSeqs / kDetectThreads;
     const int S = p.num_seqs, tid = threadIdx.x;
     const int bpp = p.part_tokens / kBlockSize, M = p.max_members;
@@ -918,6 +921,7 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
 // one partition.  M = max_p m_p; out = sum_p 2^(m_p-M) acc_p / sum_p 2^(m_p-M) l_p.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Params p) {
+    grid_dep_wait();  // every partial is written
     constexpr int kDpl = D / 32;
     const int lane = threadIdx.x & 31;
     const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
@@ -968,7 +972,10 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
                              (int)Lay::smem_bytes(kMaxSplitSeqs + 1));
     if (e != cudaSuccess) return e;
     const int sms = num_sms(dev);
-    // shared-prefix groups: bf16, head_dim 128, split contexts
+    // shared-prefix groups: bf16, head_dim 128, split contexts.  Detection, the
+    // group tiles, this kernel and the combine follow one another with
+    // programmatic dependent launch (see the kernels for where each waits).
+    bool grouped = false;
     if constexpr (sizeof(T) == 2 && D == 128) {
         if (split && a.ws_group && a.num_seqs <= kMaxGroupSeqs) {
             unsigned char *g = static_cast<unsigned char *>(a.ws_group);
@@ -1000,17 +1007,23 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             gl.scale = a.scale;
             gl.err = a.err;
             if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
+            grouped = true;
         }
     }
     int64_t grid = sms;
     if (!split) grid = std::min<int64_t>(grid, (int64_t)a.num_seqs * a.cache.num_kv_heads);
     if (grid < 1) grid = 1;
-    decode_kernel<T, D, G><<<(unsigned)grid, kThreads, smem, stream>>>(prm);
-    e = cudaGetLastError();
+    if (grouped) {
+        e = launch_after(decode_kernel<T, D, G>, dim3((unsigned)grid), dim3(kThreads), smem, stream,
+                         static_cast<const Params &>(prm));
+    } else {
+        decode_kernel<T, D, G><<<(unsigned)grid, kThreads, smem, stream>>>(prm);
+        e = cudaGetLastError();
+    }
     if (e != cudaSuccess || !split) return e;
     const int64_t warps = (int64_t)a.num_seqs * a.num_q_heads;
-    reduce_kernel<T, D><<<(unsigned)((warps + 3) / 4), 128, 0, stream>>>(prm);
-    return cudaGetLastError();
+    return launch_after(reduce_kernel<T, D>, dim3((unsigned)((warps + 3) / 4)), dim3(128), 0, stream,
+                        static_cast<const Params &>(prm));
 }
 
 template <typename T, int D>

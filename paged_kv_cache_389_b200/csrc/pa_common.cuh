@@ -198,5 +198,21 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// ---- programmatic dependent launch ---------------------------------------------
+// grid_dep_wait: block until the grid this one was launched behind (with the
+// programmatic-serialization attribute) has completed and its writes are
+// visible; a no-op for an ordinary launch.  grid_dep_launch: let the next grid
+// on the stream start launching (it still waits where it calls grid_dep_wait).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Wait until at most `pending` (0..3; larger counts wait for 3) of this
+// thread's most recent commit groups are still in flight.
+__device__ __forceinline__ void cp_async_wait_dyn(int pending) {
+    if (pending <= 0) cp_async_wait<0>();
+    else if (pending == 1) cp_async_wait<1>();
+    else if (pending == 2) cp_async_wait<2>();
+    else cp_async_wait<3>();
+}
 
 }  // namespace pa

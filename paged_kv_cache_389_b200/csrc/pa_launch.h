@@ -11,6 +11,25 @@ namespace pa {
 
 inline int dtype_bytes(int32_t dtype) { return dtype == PA_F32 ? 4 : 2; }
 
+// Launch `kern` behind the previous grid on `stream` with programmatic stream
+// serialization: it may start before that grid ends and must call grid_dep_wait
+// (pa_common.cuh) before reading what that grid writes.
+template <typename... Args>
+cudaError_t launch_after(void (*kern)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         const Args &...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 cudaError_t launch_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
                                int32_t num_tokens, void *key_cache, void *value_cache,
                                const pa_cache_desc &c, int32_t *err, cudaStream_t stream);

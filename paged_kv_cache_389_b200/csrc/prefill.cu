@@ -241,6 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     int u0 = 0, nunits = 1, ngroups = 0;
     Job jb;
     if constexpr (kGroup) {
+        // launched behind the detection kernel: its group list must be complete;
+        // then the per-sequence decode may start (it reads only detection output)
+        grid_dep_wait();
+        grid_dep_launch();
         nunits = __ldg(p.meta + 1);
         ngroups = __ldg(p.meta);
         u0 = blockIdx.x;
@@ -595,8 +599,8 @@ cudaError_t launch_group_g(const Params &prm, int sms, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    attn_tile_kernel<G, true><<<(unsigned)sms, kThreads, kSmemBytes, stream>>>(prm);
-    return cudaGetLastError();
+    return launch_after(attn_tile_kernel<G, true>, dim3((unsigned)sms), dim3(kThreads), kSmemBytes, stream,
+                        static_cast<const Params &>(prm));
 }
 
 }  // namespace
