@@ -172,19 +172,22 @@ def max_over_ranks(x, world):
 
 
 # ----------------------------------------------------------------- profiles
-def recorded_traffic(kernel_src):
-    """DRAM bytes per launch from the committed ncu summary, or None if the kernel's
-    source changed since the counters were taken."""
+def recorded_traffic():
+    """DRAM bytes of one pa_decode call (all its kernels) from the committed ncu
+    summary, or None if a kernel source changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "decode_gqa8b_prefix_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    mh = re.search(r"decode\.cu sha256: ([0-9a-f]{64})", text)
-    mt = re.search(r"dram bytes per launch \(read\+write\): (\d+)", text)
-    if not mh or not mt:
+    mt = re.search(r"dram bytes per pa_decode call \(read\+write\): (\d+)", text)
+    if not mt:
         return None
-    cur = hashlib.sha256(open(kernel_src, "rb").read()).hexdigest()
-    return int(mt.group(1)) if cur == mh.group(1) else None
+    for name in ("decode.cu", "prefill.cu"):
+        mh = re.search(name.replace(".", r"\.") + r" sha256: ([0-9a-f]{64})", text)
+        src = os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", name)
+        if not mh or hashlib.sha256(open(src, "rb").read()).hexdigest() != mh.group(1):
+            return None
+    return int(mt.group(1))
 
 
 # ----------------------------------------------------------------- our arm
@@ -329,11 +332,11 @@ def run_ours(args):
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "logical_gbs": round(world * (logical_b + cw_b) * K / (ms_max * 1e-3) / 1e9, 2),
             "bytes_per_step": {"decode_unique": unique_b, "decode_logical": logical_b, "cache_write": cw_b},
-            "roofline": {"bound": "hbm", "kernel": "pa_decode (decode_kernel + lse reduce)",
+            "roofline": {"bound": "hbm", "kernel": "pa_decode call (group detection + tcgen05 group tiles + decode_kernel + lse reduce)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if peaks else "fallback",
-                         "traffic": recorded_traffic(os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", "decode.cu")),
+                         "traffic": recorded_traffic(),
                          "decode_ms": round(dec_ms, 5)},
             "e2e": e2e,
             "gpu_launches": K * (1 + pa.pa_decode_launches(S, wl.head_dim, pa.PA_BF16, part)),
