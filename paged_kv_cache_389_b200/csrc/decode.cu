@@ -119,6 +119,7 @@ struct Params {
     int32_t num_blocks;
     int32_t part_tokens;  // 0 = whole context is one unit
     int32_t max_parts;
+    int32_t seq_tokens;   // split: tokens per per-sequence unit (a multiple of part_tokens)
     float scale_log2;
     // shared-prefix groups (split contexts only; nullptr = none): first_p[s] is the
     // number of leading partitions of s computed by group_decode_kernel
@@ -137,9 +138,14 @@ __device__ __forceinline__ int checked_len(const Params &p, int s) {
     return check_len(p, __ldg(p.lens + s));
 }
 
-__device__ __forceinline__ int num_parts(const Params &p, int L) {
-    if (p.part_tokens <= 0 || L <= 0) return 1;
-    return (L + p.part_tokens - 1) / p.part_tokens;
+// Split contexts: the first fp partitions of part_tokens (shared-prefix group
+// units) are followed by per-sequence units of seq_tokens each; unit k writes
+// workspace slot fp + k.  Returns the number of per-sequence units (1 unsplit).
+__device__ __forceinline__ int seq_units(const Params &p, int L, int fp) {
+    if (p.part_tokens <= 0) return 1;
+    const int rem = L - fp * p.part_tokens;
+    if (fp == 0 && rem <= 0) return 1;  // empty context: one unit, finished as 0
+    return rem > 0 ? (rem + p.seq_tokens - 1) / p.seq_tokens : 0;
 }
 
 struct Unit {
@@ -151,10 +157,10 @@ __device__ __forceinline__ int first_part(const Params &p, int s) {
     return p.first_p ? __ldg(p.first_p + s) : 0;
 }
 
-// Unit u -> (sequence, partition, kv head).  Units [0, S*Hkv) are the first
-// partition f(s) of every sequence not covered by a group unit (f = first_part),
-// kv head innermost; after them come partitions > f(s), sequence-major, using
-// cum[s] = sum_{s' < s} (parts(s') - f(s') - 1)^+.
+// Unit u -> (sequence, slot, kv head).  Units [0, S*Hkv) are the first
+// per-sequence unit (slot f(s), f = first_part) of every sequence, kv head
+// innermost; after them come the further units (slots > f(s)), sequence-major,
+// using cum[s] = sum_{s' < s} (seq_units(s') - 1)^+.
 __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t units_first, int hkv,
                                         const int *cum, int S) {
     if (u < units_first) {
@@ -189,7 +195,9 @@ struct WarpUnit {
 __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t units_first,
                                           const int *cum, WarpUnit &w, int lane, bool flagger) {
     w.un = unit_of(p, u, units_first, p.num_kv_heads, cum, p.num_seqs);
-    const int b0 = p.part_tokens > 0 ? w.un.part * (p.part_tokens / kBlockSize) : 0;
+    const int k = w.un.part - w.un.fp;  // per-sequence unit index
+    const int t_first = p.part_tokens > 0 ? w.un.fp * p.part_tokens + k * p.seq_tokens : 0;
+    const int b0 = t_first / kBlockSize;
     w.trow = p.tables + (int64_t)w.un.s * p.max_blocks + b0;
     // both loads issued before either value is needed
     const int raw = __ldg(p.lens + w.un.s);
@@ -204,15 +212,15 @@ __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t un
         w.t0 = 0;
         w.nt = L;
     } else {
-        w.t0 = w.un.part * p.part_tokens;
-        w.nt = max(0, min(L, w.t0 + p.part_tokens) - w.t0);
+        w.t0 = t_first;
+        w.nt = max(0, min(L, w.t0 + p.seq_tokens) - w.t0);
     }
-    w.skip = w.un.part >= num_parts(p, L);
+    w.skip = k >= seq_units(p, L, w.un.fp);
     if (w.skip) w.nt = 0;
     w.nb = (w.nt + kBlockSize - 1) / kBlockSize;
 }
 
-// Prologue: cum[s] = sum_{s' < s} (parts(s') - first_part(s') - 1)^+ (exclusive
+// Prologue: cum[s] = sum_{s' < s} (seq_units(s') - 1)^+ (exclusive
 // scan, one chunk of sequences per thread).  Ends with __syncthreads.
 __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -223,7 +231,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
         int local = 0;
         for (int s = beg; s < end; ++s) {
             const int L = checked_len(p, s);
-            local += max(0, num_parts(p, L < 0 ? 0 : L) - first_part(p, s) - 1);
+            local += max(0, seq_units(p, L < 0 ? 0 : L, first_part(p, s)) - 1);
         }
         int incl = local;
 #pragma unroll
@@ -239,7 +247,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
         for (int s = beg; s < end; ++s) {
             cum[s] = run;
             const int L = checked_len(p, s);
-            run += max(0, num_parts(p, L < 0 ? 0 : L) - first_part(p, s) - 1);
+            run += max(0, seq_units(p, L < 0 ? 0 : L, first_part(p, s)) - 1);
         }
         if ((int)threadIdx.x == kThreads - 1) cum[S] = run;
     }
@@ -286,7 +294,7 @@ template <typename T, int D, int G>
 __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, const float *uacc,
                                             const float2 *uml) {
     if (w.skip) return;
-    const bool single = num_parts(p, w.L) == 1 && w.un.fp == 0;
+    const bool single = w.un.fp == 0 && seq_units(p, w.L, 0) == 1;
     const int64_t head0 = (int64_t)w.un.s * p.num_q_heads + (int64_t)w.un.h * G;
     for (int e = threadIdx.x; e < G * D; e += kThreads) {
         const int h = e / D, dd = e - h * D;
@@ -825,84 +833,71 @@ __device__ __forceinline__ void shared_prefix_lengths(const Params &p, int *lcp)
     }
 }
 
-// Block-wide exclusive scan (sum, or max when kMax) of one int per thread.
+// Warp-wide exclusive scan (sum, or max when kMax) of one int per lane.
 template <bool kMax>
-__device__ __forceinline__ int block_exclusive_scan(int x, int identity, int *wbuf) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ int warp_exclusive_scan(int x, int identity) {
+    const int lane = threadIdx.x & 31;
     int inc = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(kFull, inc, o);
         if (lane >= o) inc = kMax ? max(inc, y) : inc + y;
     }
-    if (lane == 31) wbuf[warp] = inc;
-    __syncthreads();
-    int off = identity;
-    for (int w = 0; w < warp; ++w) off = kMax ? max(off, wbuf[w]) : off + wbuf[w];
-    int exc = __shfl_up_sync(kFull, inc, 1);
-    if (lane == 0) exc = identity;
-    __syncthreads();  // wbuf is reused by the next scan
-    return kMax ? max(off, exc) : off + exc;
+    const int exc = __shfl_up_sync(kFull, inc, 1);
+    return lane == 0 ? identity : exc;
 }
 
-// One CTA.  A run is a maximal stretch of sequences each sharing at least one
-// whole partition with its predecessor; runs are cut into chunks of at most
-// max_members sequences counted from the run's start.  A chunk of n >= 2
-// sequences shares min(lcp over its members after the first) blocks, i.e. np
-// whole partitions; it becomes one group with np x num_kv_heads units.
-// first_p[s] = np of s's chunk (0 for a chunk of one).
+// One CTA: all warps compare tables, then warp 0 forms the groups.  A run is a
+// maximal stretch of sequences each sharing at least one whole partition with
+// its predecessor; runs are cut into chunks of at most max_members sequences
+// counted from the run's start.  A chunk of n >= 2 sequences shares min(lcp over
+// its members after the first) blocks, i.e. np whole partitions; it becomes one
+// group with np x num_kv_heads units.  first_p[s] = np of s's chunk (0 for a
+// chunk of one).
 __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __grid_constant__ Params p,
                                                                       int32_t *first_p, int4 *groups,
                                                                       int32_t *meta) {
     __shared__ int lcp[kMaxGroupSeqs];
     __shared__ int info[kMaxGroupSeqs];  // at a chunk head: np << 8 | members (members <= 128); else -1
-    __shared__ int wbuf[kDetectThreads / 32];
     grid_dep_launch();  // the group tiles set up while this runs, then wait for it
-    constexpr int kPer = kMaxGroupSeqs / kDetectThreads;
-    const int S = p.num_seqs, tid = threadIdx.x;
-    const int bpp = p.part_tokens / kBlockSize, M = p.max_members;
-    const int s0 = tid * kPer;
+    const int S = p.num_seqs;
     shared_prefix_lengths(p, lcp);
     __syncthreads();
+    if (threadIdx.x >= 32) return;
+    // warp 0: lane owns sequences [s0, s1)
+    const int lane = threadIdx.x;
+    const int bpp = p.part_tokens / kBlockSize;
+    const int M = p.max_members;  // 128 / g: a power of two
+    const int per = (S + 31) / 32, s0 = min(S, lane * per), s1 = min(S, s0 + per);
     // run starts: max-scan of (run head ? s : -1)
-    int lv[kPer], mx = -1;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        const int s = s0 + k;
-        lv[k] = s < S ? lcp[s] : 0;
-        if (s < S && (s == 0 || lv[k] < bpp)) mx = s;
+    int mx = -1;
+    for (int s = s0; s < s1; ++s)
+        if (s == 0 || lcp[s] < bpp) mx = s;
+    int rs = warp_exclusive_scan<true>(mx, -1);
+    for (int s = s0; s < s1; ++s) {
+        if (s == 0 || lcp[s] < bpp) rs = s;
+        info[s] = ((s - rs) & (M - 1)) == 0 ? 0 : -1;  // chunk heads marked 0 for now
     }
-    int rs = block_exclusive_scan<true>(mx, -1, wbuf);
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        const int s = s0 + k;
-        if (s >= S) break;
-        if (s == 0 || lv[k] < bpp) rs = s;
-        info[s] = (s - rs) % M == 0 ? 0 : -1;  // chunk heads marked 0 for now
-    }
-    __syncthreads();
+    __syncwarp();
     // each chunk head measures its chunk
     int chunks = 0, units = 0;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        const int s = s0 + k;
-        if (s >= S || info[s] < 0) continue;
+    for (int s = s0; s < s1; ++s) {
+        if (info[s] < 0) continue;
         int e = s + 1, mn = INT_MAX;
         while (e < S && info[e] < 0) mn = min(mn, lcp[e++]);
         const int n = e - s;
         const int np = n > 1 ? min(mn / bpp, kMaxGroupParts) : 0;
-        info[s] = (np << 8) | n;  // stays >= 0: other threads only test the sign
+        info[s] = (np << 8) | n;  // stays >= 0: other lanes only test the sign
         if (np > 0) {
             ++chunks;
             units += np * p.num_kv_heads;
         }
     }
-    int oc = block_exclusive_scan<false>(chunks, 0, wbuf);
-    int ou = block_exclusive_scan<false>(units, 0, wbuf);
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-        const int s = s0 + k;
-        if (s >= S || info[s] < 0) continue;
+    __syncwarp();
+    int oc = warp_exclusive_scan<false>(chunks, 0);
+    int ou = warp_exclusive_scan<false>(units, 0);
+    for (int s = s0; s < s1; ++s) {
+        if (info[s] < 0) continue;
         const int n = info[s] & 255, np = info[s] >> 8;
         for (int m = s; m < s + n; ++m) first_p[m] = np;
         if (np > 0) {
@@ -910,12 +905,11 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
             ou += np * p.num_kv_heads;
         }
     }
-    if (tid == kDetectThreads - 1) {
+    if (lane == 31) {  // its running counts end at the totals
         meta[0] = oc;
         meta[1] = ou;
     }
 }
-
 
 // Combine split-K partials: one warp per (sequence, query head) with more than
 // one partition.  M = max_p m_p; out = sum_p 2^(m_p-M) acc_p / sum_p 2^(m_p-M) l_p.
@@ -929,8 +923,9 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
     const int s = (int)(wid / p.num_q_heads);
     int L = checked_len(p, s);
     if (L < 0) L = 0;
-    const int n = num_parts(p, L);
-    if (n <= 1 && first_part(p, s) == 0) return;  // finished by the decode kernel
+    const int fp = first_part(p, s);
+    const int n = fp + seq_units(p, L, fp);  // slots written
+    if (fp == 0 && n <= 1) return;            // finished by the decode kernel
     const float2 *ml = p.ws_ml + wid * p.max_parts;
     const float *acc = p.ws_acc + wid * p.max_parts * D + lane * kDpl;
     float M = -INFINITY;
@@ -972,6 +967,14 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
                              (int)Lay::smem_bytes(kMaxSplitSeqs + 1));
     if (e != cudaSuccess) return e;
     const int sms = num_sms(dev);
+    // Per-sequence units after the group-covered partitions span several
+    // partitions, so that the per-unit merge is amortised: 1024 tokens, or 2048
+    // when there are few (sequence, kv head) pairs to spread over the SMs
+    // (measured on B200: 512-token units cost 4-16% against these).
+    if (split) {
+        const int want = (int64_t)a.num_seqs * a.cache.num_kv_heads < 4LL * sms ? 2048 : 1024;
+        prm.seq_tokens = prm.part_tokens * std::max(1, want / prm.part_tokens);
+    }
     // shared-prefix groups: bf16, head_dim 128, split contexts.  Detection, the
     // group tiles, this kernel and the combine follow one another with
     // programmatic dependent launch (see the kernels for where each waits).
@@ -1059,6 +1062,7 @@ cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
     prm.num_blocks = a.cache.num_blocks;
     prm.part_tokens = a.partition_size;
     prm.max_parts = a.max_partitions;
+    prm.seq_tokens = a.partition_size;  // launch_t may widen it
     prm.scale_log2 = a.scale * kLog2e;
     const bool bf16 = a.cache.dtype == PA_BF16;
     if (a.cache.head_dim == 128)

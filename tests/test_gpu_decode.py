@@ -123,8 +123,9 @@ def _custom(lens, hq, hkv, d, dtype, seed=5, extra_blocks=4):
 @pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 128), ("f32", 64)])
 @pytest.mark.parametrize("g", [1, 2, 4, 8])
 def test_edge_lengths_all_variants(dtype, d, g):
-    """Empty context, a single token, block and partition boundaries +-1, ragged tails."""
-    lens = [0, 1, 15, 16, 17, 31, 33, 255, 256, 257, 511, 512, 513, 700]
+    """Empty context, a single token, block and partition boundaries +-1, ragged tails,
+    and lengths around the per-sequence unit sizes (1024, 2048 tokens)."""
+    lens = [0, 1, 15, 16, 17, 31, 33, 255, 256, 257, 511, 512, 513, 700, 1023, 1024, 1025, 2047, 2049, 3001]
     wl = _custom(lens, 2 * g, 2, d, dtype)
     ts = TwoSided(wl)
     step = wl.steps[0]
