@@ -159,7 +159,7 @@ PA_API int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dt
  * combines them: out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p with
  * M = max_p m_p.  Sequences with a single partition are finished by the first
  * kernel.  With a split, bf16 caches, head_dim 128 and num_seqs <= 4096, runs of
- * adjacent sequences whose block tables begin with the same block ids (forked
+ * at least 4 adjacent sequences whose block tables begin with the same block ids (forked
  * siblings, a common prompt) read the partitions that lie wholly inside those
  * shared blocks once for the whole run, with all its queries against each K/V
  * tile; the result is the same sum, and the shared blocks cross the memory bus

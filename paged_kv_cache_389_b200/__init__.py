@@ -234,7 +234,7 @@ class BlockManager:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h:
+        if h and _lib is not None:  # at interpreter exit the module globals may be gone
             _lib.pa_bm_destroy(h)
             self._h = None
 

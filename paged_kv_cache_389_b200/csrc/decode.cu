@@ -139,8 +139,9 @@ __device__ __forceinline__ int checked_len(const Params &p, int s) {
 }
 
 // Split contexts: the first fp partitions of part_tokens (shared-prefix group
-// units) are followed by per-sequence units of seq_tokens each; unit k writes
-// workspace slot fp + k.  Returns the number of per-sequence units (1 unsplit).
+// units, one partial per partition in slots 0..fp-1) are followed by
+// per-sequence units of seq_tokens each; unit k writes slot fp + k.  Returns the
+// number of per-sequence units (1 unsplit).
 __device__ __forceinline__ int seq_units(const Params &p, int L, int fp) {
     if (p.part_tokens <= 0) return 1;
     const int rem = L - fp * p.part_tokens;
@@ -149,9 +150,11 @@ __device__ __forceinline__ int seq_units(const Params &p, int L, int fp) {
 }
 
 struct Unit {
-    int s, part, h;
-    int fp;  // first_part(s): partitions of s computed by group units
+    int s, part, h;  // part: the workspace slot the unit writes
+    int fp;          // first_part(s): partitions of s computed by group units
 };
+
+__device__ __forceinline__ int slot_base(int fp) { return fp; }
 
 __device__ __forceinline__ int first_part(const Params &p, int s) {
     return p.first_p ? __ldg(p.first_p + s) : 0;
@@ -166,7 +169,7 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t unit
     if (u < units_first) {
         const int s = (int)(u / hkv);
         const int fp = first_part(p, s);
-        return Unit{s, fp, (int)(u % hkv), fp};
+        return Unit{s, slot_base(fp), (int)(u % hkv), fp};
     }
     const int64_t v = u - units_first;
     const int e = (int)(v / hkv), h = (int)(v % hkv);
@@ -176,7 +179,7 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t unit
         if (cum[mid] <= e) lo = mid; else hi = mid;
     }
     const int fp = first_part(p, lo);
-    return Unit{lo, fp + 1 + e - cum[lo], h, fp};
+    return Unit{lo, slot_base(fp) + 1 + e - cum[lo], h, fp};
 }
 
 // What one warp needs to know about a unit.  `tab` holds, in lane i, the table
@@ -195,7 +198,7 @@ struct WarpUnit {
 __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t units_first,
                                           const int *cum, WarpUnit &w, int lane, bool flagger) {
     w.un = unit_of(p, u, units_first, p.num_kv_heads, cum, p.num_seqs);
-    const int k = w.un.part - w.un.fp;  // per-sequence unit index
+    const int k = w.un.part - slot_base(w.un.fp);  // per-sequence unit index
     const int t_first = p.part_tokens > 0 ? w.un.fp * p.part_tokens + k * p.seq_tokens : 0;
     const int b0 = t_first / kBlockSize;
     w.trow = p.tables + (int64_t)w.un.s * p.max_blocks + b0;
@@ -766,18 +769,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 // Sequences next to each other in the batch whose tables start with the same
 // physical blocks (forks, a shared system prompt: chenxutan 2.1 / 3.3, devpress
 // 关键设计二) read those blocks once: the shared leading partitions are computed
-// by group units whose query columns are members x heads, and the per-sequence
-// kernel starts after them.  Results are unchanged -- the same partials land in
-// the same workspace slots and the LSE reduce combines them.
+// by group units (group, partition, kv head) whose query rows are members x
+// heads, and the per-sequence kernel starts after them.  The result is the same
+// sum -- the group partials land in slots 0..fp-1 of every member, the
+// per-sequence units in the slots after them, and the LSE reduce combines them.
 //
 // Detection is one single-CTA kernel: each sequence's count of leading full
 // blocks shared with its predecessor, then the cut of the batch into groups.
 // The group units -- a dense (members x g) x partition x head_dim attention
-// tile each -- run on the tcgen05 tile kernel of prefill.cu (launch_group_tiles).
+// each -- run on the tcgen05 tile kernel of prefill.cu (launch_group_tiles).
 
 constexpr int kDetectThreads = 1024;
 constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
 constexpr int kMaxGroupParts = (1 << 23) - 1;
+// A group unit costs its SM a roughly fixed ~17 us for a 512-token partition
+// (four key tiles through the tensor-core tile kernel), while each member that
+// reads the partition itself costs ~5 us of SM time, so tiny groups do not pay.
+// Measured on B200 with 4-sibling groups (parallel sampling): 498 us per call
+// grouped against 515 us without.
+constexpr int kMinGroupMembers = 4;
 constexpr int kLcpBatch = 8;         // sequences a warp compares at once
 
 // lcp[s] = leading entries of s's table equal to those of s-1, counted over the
@@ -850,10 +860,10 @@ __device__ __forceinline__ int warp_exclusive_scan(int x, int identity) {
 // One CTA: all warps compare tables, then warp 0 forms the groups.  A run is a
 // maximal stretch of sequences each sharing at least one whole partition with
 // its predecessor; runs are cut into chunks of at most max_members sequences
-// counted from the run's start.  A chunk of n >= 2 sequences shares min(lcp over
-// its members after the first) blocks, i.e. np whole partitions; it becomes one
-// group with np x num_kv_heads units.  first_p[s] = np of s's chunk (0 for a
-// chunk of one).
+// counted from the run's start.  A chunk of n >= kMinGroupMembers sequences
+// shares min(lcp over its members after the first) blocks, i.e. np whole
+// partitions; it becomes one group with np x num_kv_heads units.  first_p[s] =
+// np of s's chunk (0 for a smaller chunk).
 __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __grid_constant__ Params p,
                                                                       int32_t *first_p, int4 *groups,
                                                                       int32_t *meta) {
@@ -886,7 +896,7 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         int e = s + 1, mn = INT_MAX;
         while (e < S && info[e] < 0) mn = min(mn, lcp[e++]);
         const int n = e - s;
-        const int np = n > 1 ? min(mn / bpp, kMaxGroupParts) : 0;
+        const int np = n >= kMinGroupMembers ? min(mn / bpp, kMaxGroupParts) : 0;
         info[s] = (np << 8) | n;  // stays >= 0: other lanes only test the sign
         if (np > 0) {
             ++chunks;
@@ -924,8 +934,8 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
     int L = checked_len(p, s);
     if (L < 0) L = 0;
     const int fp = first_part(p, s);
-    const int n = fp + seq_units(p, L, fp);  // slots written
-    if (fp == 0 && n <= 1) return;            // finished by the decode kernel
+    const int n = slot_base(fp) + seq_units(p, L, fp);  // slots written
+    if (fp == 0 && n <= 1) return;                       // finished by the decode kernel
     const float2 *ml = p.ws_ml + wid * p.max_parts;
     const float *acc = p.ws_acc + wid * p.max_parts * D + lane * kDpl;
     float M = -INFINITY;

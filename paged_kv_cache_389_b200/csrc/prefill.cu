@@ -19,8 +19,9 @@
 // Q and K K-major, V MN-major, the canonical layouts the MMA descriptors name),
 // warps 4-11 run the softmax (warp w: TMEM lanes 32*(w%4)..+31, one 64-column
 // half of the tile), warp 12 owns the tensor memory and issues the MMAs from one
-// thread.  K/V tiles are double-buffered and loaded two deep; the stages are
-// handed over with mbarriers; every wait is bounded and an abort still frees
+// thread.  K and V tiles have separate two-stage rings and loader warps (0-1: Q
+// and K, 2-3: V), so a K stage is refilled as soon as its QK is done; the stages
+// are handed over with mbarriers; every wait is bounded and an abort still frees
 // the tensor memory.
 #include <cstring>
 
@@ -48,12 +49,12 @@ constexpr uint32_t kOffK = kOffQ + kTileBytes;     // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kTileBytes; // 2 stages
 constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
 constexpr uint32_t kOffBar = kOffP + kTileBytes;
-constexpr uint32_t kOffTab = kOffBar + 16 * 8;     // 8 table entries per stage
-constexpr uint32_t kOffMisc = kOffTab + 2 * 8 * 4;
+constexpr uint32_t kOffTab = kOffBar + 24 * 8;     // 24 mbarriers
+constexpr uint32_t kOffMisc = kOffTab + 2 * 2 * 8 * 4;  // [K, V loader][2 stages][8 table entries]
 constexpr uint32_t kOffRed = kOffMisc + 16;          // row-max halves [2 tiles][2 halves][128 rows]
 constexpr uint32_t kOffLsum = kOffRed + 2 * 2 * 128 * 4;  // row-sum halves [2][128]
 constexpr uint32_t kOffGcum = kOffLsum + 2 * 128 * 4;  // group units: units before each group
-constexpr int kMaxGroups = 2048;                     // a group has >= 2 of <= 4096 sequences
+constexpr int kMaxGroups = 2048;                     // a group has >= 2 (in fact >= 4) of <= 4096 sequences
 constexpr size_t kSmemBytes = 1024 + kOffGcum + kMaxGroups * 4;
 
 struct Params {
@@ -194,7 +195,7 @@ __device__ __forceinline__ Job group_job(const Params &p, const int *gcum, int n
     const int4 gr = __ldg(&p.groups[lo]);  // (first seq, members, shared partitions, units before)
     const int r = u - gr.w;
     jb.h = r % p.num_kv_heads;
-    jb.part = r / p.num_kv_heads;
+    jb.part = r / p.num_kv_heads;  // partition = workspace slot
     jb.first = gr.x;
     const int64_t hs = (int64_t)kD * 2;
     jb.q_row_stride = (int64_t)p.num_q_heads * hs;
@@ -211,10 +212,12 @@ __device__ __forceinline__ Job group_job(const Params &p, const int *gcum, int n
 
 // Prefill: one CTA per (query tile, kv head, sequence).  Shared-prefix groups of
 // the split decode (kGroup): a persistent CTA loops over the group units (group,
-// partition, kv head) listed by the decode's detection kernels; the rows are the
+// partition, kv head) listed by the decode's detection kernel; the rows are the
 // members' queries, the keys one partition lying inside the blocks all members
-// share, and the result is the partition's (m, l, unnormalised O) in the split-K
-// workspace -- the same partial the per-sequence decode kernel writes.
+// share, and the result is the partition's (m, l, unnormalised O) in workspace
+// slot p of every member -- the same partial the per-sequence kernel would write.
+// (Units spanning all of a group's partitions were measured: they balance worse
+// over the SMs and were slower.)
 template <int G, bool kGroup>
 __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_constant__ Params p) {
     extern __shared__ unsigned char smem_raw[];
@@ -222,18 +225,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     const uint32_t sbase = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
     uint64_t *q_full = bars + 0;
-    uint64_t *kv_full = bars + 1;   // [2]
-    uint64_t *kv_empty = bars + 3;  // [2]
-    uint64_t *s_full = bars + 5;
-    uint64_t *p_full = bars + 6;
-    uint64_t *pv_done = bars + 7;
-    uint64_t *mma_idle = bars + 8;
-    uint64_t *red_full = bars + 9;  // [2]
-    uint64_t *l_full = bars + 11;
-    int *tab = reinterpret_cast<int *>(smem + kOffTab);  // [2][8]
+    uint64_t *k_full = bars + 1;    // [2] K tile landed
+    uint64_t *k_empty = bars + 3;   // [2] its QK is done: the K stage may be refilled
+    uint64_t *v_full = bars + 5;    // [2] V tile landed
+    uint64_t *v_empty = bars + 7;   // [2] its PV is done: the V stage may be refilled
+    uint64_t *s_full = bars + 9;
+    uint64_t *p_full = bars + 10;
+    uint64_t *pv_done = bars + 11;
+    uint64_t *mma_idle = bars + 12;
+    uint64_t *red_full = bars + 13;  // [2]
+    uint64_t *l_full = bars + 15;
+    uint64_t *q_empty = bars + 16;  // a unit's last QK is done: Q may be rewritten
+    uint64_t *o_free = bars + 17;   // the softmax warps have read a unit's O
+    int *tab = reinterpret_cast<int *>(smem + kOffTab);  // [K, V loader][2][8]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
-    volatile int *go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);
+    volatile int *go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);  // [K, V loader]
     int *gcum = reinterpret_cast<int *>(smem + kOffGcum);
     const int64_t hs = (int64_t)kD * 2;  // bytes per (row, head)
 
@@ -277,15 +284,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 128);
-        mbar_init(&kv_full[0], 128);
-        mbar_init(&kv_full[1], 128);
-        mbar_init(&kv_empty[0], 1);
-        mbar_init(&kv_empty[1], 1);
+        mbar_init(q_full, 64);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&k_full[i], 64);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 64);
+            mbar_init(&v_empty[i], 1);
+        }
         mbar_init(s_full, 1);
         mbar_init(p_full, kSoftmaxThreads);
         mbar_init(pv_done, 1);
         mbar_init(mma_idle, 1);
+        mbar_init(q_empty, 1);
+        mbar_init(o_free, kSoftmaxThreads);
         mbar_init(&red_full[0], kSoftmaxThreads);
         mbar_init(&red_full[1], kSoftmaxThreads);
         mbar_init(l_full, kSoftmaxThreads);
@@ -303,76 +314,100 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     const uint32_t tS = tmem, tO = tmem + 128;
 
     // Barrier phases run on across units: tile jt = tbase + j of the CTA uses
-    // stage jt & 1; q_full and mma_idle complete once per unit.
+    // stage jt & 1; q_full, q_empty, l_full and o_free complete once per unit.
+    // Units follow one another without a CTA barrier: the loader streams the
+    // next unit's Q (after q_empty) and K/V tiles while the current one is
+    // still being computed, and the MMA starts the next unit's PV only after
+    // o_free.  Every wait is bounded; after an abort the remaining units fall
+    // through their (failing) waits.
     int tbase = 0, nu = 0;
     for (int u = u0; u < nunits; u += (kGroup ? gridDim.x : 1), ++nu) {
         if constexpr (kGroup) jb = group_job<G, kGroup>(p, gcum, ngroups, u);
         if (warp < 4) {
             // -------------------------------------------------------- loaders
-            const int t = threadIdx.x;  // 0..127
-            // Q tile: row r = (row group r / G, head r % G); 16 chunks of 16 bytes per row
-            for (int idx = t; idx < kTileM * 16; idx += 128) {
-                const int r = idx >> 4, c = idx & 15;
-                const uint32_t dst = sbase + kOffQ + swz(r, c);
-                if (r < jb.nrows)
-                    cp_async16(dst, jb.q + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs + c * 16);
-                else
-                    *reinterpret_cast<uint4 *>(smem + kOffQ + swz(r, c)) = make_uint4(0, 0, 0, 0);
+            // Warps 0-1 stream Q and K, warps 2-3 stream V, each group through
+            // its own two-stage ring, two tiles deep.  A K stage comes back as
+            // soon as its QK is done, so K runs ahead of V.  Within a group one
+            // thread waits and the decision reaches the others through shared
+            // memory behind the group's named barrier.
+            const bool is_k = warp < 2;
+            const int t = threadIdx.x & 63;
+            const int gbar = is_k ? 1 : 2;
+            volatile int *gw = go + (is_k ? 0 : 1);
+            int *gtab = tab + (is_k ? 0 : 16);
+            uint64_t *full = is_k ? k_full : v_full;
+            uint64_t *empty = is_k ? k_empty : v_empty;
+            const uint32_t ring_s = sbase + (is_k ? kOffK : kOffV);
+            unsigned char *ring = smem + (is_k ? kOffK : kOffV);
+            const unsigned char *src0 = is_k ? p.kc : p.vc;
+            bool q_ok = true;
+            if (is_k) {
+                // the previous unit's QK must be done with Q
+                if (t == 0) *gw = (nu == 0 || wait_bar(q_empty, (nu - 1) & 1, abort_flag, p.err)) ? 1 : 0;
+                named_barrier(gbar, 64);
+                q_ok = *gw != 0;
+                named_barrier(gbar, 64);  // *gw is rewritten by the first tile issue
+                // Q tile: row r = (row group r / G, head r % G); 16 chunks of 16 bytes per row
+                for (int idx = t; q_ok && idx < kTileM * 16; idx += 64) {
+                    const int r = idx >> 4, c = idx & 15;
+                    const uint32_t dst = sbase + kOffQ + swz(r, c);
+                    if (r < jb.nrows)
+                        cp_async16(dst, jb.q + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs + c * 16);
+                    else
+                        *reinterpret_cast<uint4 *>(smem + kOffQ + swz(r, c)) = make_uint4(0, 0, 0, 0);
+                }
+                cp_async_commit();
             }
-            cp_async_commit();
-            // Tile j's copies are issued into stage (tbase+j) & 1 once the MMA has
-            // released that stage; tile j+1 is issued before tile j is waited
-            // for, so two tiles are in flight.  The decision to go on reaches
-            // all loaders through shared memory behind a barrier.
+            // table entry of block t of tile j (threads t < 8; -1: past the keys),
+            // loaded one tile ahead so its latency hides behind the current tile
+            auto table_entry = [&](int j) -> int {
+                const int b = j * 8 + t;
+                return (t < 8 && b * kBlockSize < jb.nkeys) ? __ldg(jb.trow + b) : -1;
+            };
+            int next_e = table_entry(0);
             auto issue_tile = [&](int j) -> bool {
                 const int jt = tbase + j, st = jt & 1;
-                if (t == 0) *go = (jt < 2 || wait_bar(&kv_empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
-                // table entries of the tile's 8 blocks (-1: past the keys)
+                if (t == 0) *gw = (jt < 2 || wait_bar(&empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
                 if (t < 8) {
-                    const int b = j * 8 + t;
-                    int e = -1;
-                    if (b * kBlockSize < jb.nkeys) {
-                        e = __ldg(jb.trow + b);
-                        if (e < 0 || e >= p.num_blocks) {
-                            flag_error(p.err, PA_DEVERR_BLOCK_ID);
-                            e = -1;
-                        }
+                    int e = next_e;
+                    if (j * 8 + t < (jb.nkeys + kBlockSize - 1) / kBlockSize && (e < 0 || e >= p.num_blocks)) {
+                        flag_error(p.err, PA_DEVERR_BLOCK_ID);
+                        e = -1;
                     }
-                    tab[st * 8 + t] = e;
+                    gtab[st * 8 + t] = e;
+                    next_e = table_entry(j + 1);
                 }
-                named_barrier(1, 128);
-                const bool ok = *go != 0;
+                named_barrier(gbar, 64);
+                const bool ok = *gw != 0;
                 if (ok) {
-                    const uint32_t kst = sbase + kOffK + st * kTileBytes, vst = sbase + kOffV + st * kTileBytes;
-                    unsigned char *kgen = smem + kOffK + st * kTileBytes, *vgen = smem + kOffV + st * kTileBytes;
-                    for (int idx = t; idx < kTileN * 16; idx += 128) {
+                    const uint32_t dst0 = ring_s + st * kTileBytes;
+                    unsigned char *gen0 = ring + st * kTileBytes;
+                    for (int idx = t; idx < kTileN * 16; idx += 64) {
                         const int n = idx >> 4, c = idx & 15;
                         const int key = j * kTileN + n;
-                        const int blk = tab[st * 8 + (n >> 4)];
+                        const int blk = gtab[st * 8 + (n >> 4)];
                         const uint32_t off = swz(n, c);
                         if (blk >= 0 && key < jb.nkeys) {
                             const int64_t src = (((int64_t)blk * p.num_kv_heads + jb.h) * kBlockSize + (n & 15)) * hs + c * 16;
-                            cp_async16(kst + off, p.kc + src);
-                            cp_async16(vst + off, p.vc + src);
+                            cp_async16(dst0 + off, src0 + src);
                         } else {  // past the keys or a bad id: zeros (0 * garbage must not reach the sums)
-                            *reinterpret_cast<uint4 *>(kgen + off) = make_uint4(0, 0, 0, 0);
-                            *reinterpret_cast<uint4 *>(vgen + off) = make_uint4(0, 0, 0, 0);
+                            *reinterpret_cast<uint4 *>(gen0 + off) = make_uint4(0, 0, 0, 0);
                         }
                     }
                 }
                 cp_async_commit();
-                named_barrier(1, 128);  // tab and *go are rewritten by the next issue
+                named_barrier(gbar, 64);  // gtab and *gw are rewritten by the next issue
                 return ok;
             };
-            bool ok = jb.ntiles > 0 && issue_tile(0);
+            bool ok = q_ok && jb.ntiles > 0 && issue_tile(0);
             for (int j = 0; ok && j < jb.ntiles; ++j) {
                 const bool more = j + 1 < jb.ntiles;
                 if (more && !issue_tile(j + 1)) break;
-                // groups so far: Q, tiles 0..j (+ j+1): all but the newest are done
+                // copy groups so far: (Q,) tiles 0..j (+ j+1): all but the newest are done
                 if (more) cp_async_wait<1>(); else cp_async_wait<0>();
                 fence_proxy_async_smem();
-                if (j == 0) mbar_arrive(q_full);
-                mbar_arrive(&kv_full[(tbase + j) & 1]);
+                if (is_k && j == 0) mbar_arrive(q_full);
+                mbar_arrive(&full[(tbase + j) & 1]);
             }
             cp_async_wait<0>();  // nothing may land after an abort
         } else if (warp == kMmaWarp) {
@@ -382,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 bool ok = wait_bar(q_full, nu & 1, abort_flag, p.err);
                 for (int j = 0; ok && j < jb.ntiles; ++j) {
                     const int jt = tbase + j, st = jt & 1;
-                    if (!wait_bar(&kv_full[st], (jt >> 1) & 1, abort_flag, p.err)) break;
+                    if (!wait_bar(&k_full[st], (jt >> 1) & 1, abort_flag, p.err)) break;
                     tc_fence_after();
                     const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTileBytes;
 #pragma unroll
@@ -391,7 +426,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                         tc_mma(tS, smem_desc(qa + koff, 16, 1024), smem_desc(ka + koff, 16, 1024), kIdQK, kk > 0);
                     }
                     tc_commit(s_full);
+                    tc_commit(&k_empty[st]);
+                    if (j == jb.ntiles - 1) tc_commit(q_empty);
                     if (!wait_bar(p_full, jt & 1, abort_flag, p.err)) break;
+                    // the first PV overwrites O: the previous unit's O must have been read
+                    if (j == 0 && nu > 0 && !wait_bar(o_free, (nu - 1) & 1, abort_flag, p.err)) break;
+                    if (!wait_bar(&v_full[st], (jt >> 1) & 1, abort_flag, p.err)) break;
                     tc_fence_after();
                     const uint32_t pa_ = sbase + kOffP, va = sbase + kOffV + st * kTileBytes;
 #pragma unroll
@@ -401,13 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                                j > 0 || kk > 0);
                     }
                     tc_commit(pv_done);
-                    tc_commit(&kv_empty[st]);
-                }
-                // everything issued has completed once this arrives
-                tc_commit(mma_idle);
-                if (!mbar_wait_drain(mma_idle, nu & 1)) {
-                    *abort_flag = 1;
-                    flag_error(p.err, PA_DEVERR_TIMEOUT);
+                    tc_commit(&v_empty[st]);
                 }
             }
             __syncwarp();
@@ -567,13 +601,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     }
                 }
             }
+            // this unit's O has been read (or was never needed): the MMA may
+            // overwrite it with the next unit's first PV
+            if (live) {
+                tc_fence_before();
+                mbar_arrive(o_free);
+            }
         }
         tbase += jb.ntiles;
-        // the unit is finished by every role before Q, P and TMEM are reused
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (*abort_flag) break;
+    }
+    if (warp == kMmaWarp && lane == 0) {
+        // everything issued has completed once this arrives
+        tc_commit(mma_idle);
+        if (!mbar_wait_drain(mma_idle, 0)) {
+            *abort_flag = 1;
+            flag_error(p.err, PA_DEVERR_TIMEOUT);
+        }
     }
     tc_fence_before();
     __syncthreads();

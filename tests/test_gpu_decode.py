@@ -212,21 +212,22 @@ def _grouped_workload(g=4):
     hkv, d = 4, 128
     hq = g * hkv
     # (parent tokens, [suffix lengths]) per family; forked parents end on a block
-    # boundary so that no sibling's first append needs a copy
+    # boundary so that no sibling's first append needs a copy.  A group needs at
+    # least 4 members and takes at most 128 / g.
     spec = []
-    spec.append((1104, [int(x) for x in rng.integers(0, 300, size=20)]))   # 20 siblings: chunks of 16 + 4
-    spec.append((608, [5, 77, 130]))             # shares 38 full blocks
-    spec.append((400, [3, 9, 27, 81, 1, 0]))     # 6 siblings
-    spec.append((208, [40, 41]))                 # shares less than one 256-token partition
-    spec.append((512, [0, 0]))                   # members entirely inside the shared prefix
+    spec.append((1104, [int(x) for x in rng.integers(0, 300, size=20)]))   # 20 siblings
+    spec.append((608, [5, 77, 130, 3, 9, 27, 81, 1, 40]))   # 9 siblings sharing 38 full blocks
+    spec.append((208, [40, 41, 0, 7, 13, 90, 5, 60]))        # shares 13 blocks: < one 256-token partition
+    spec.append((512, [0] * 8))                  # members entirely inside the shared prefix
     spec.append((333, []))                       # singleton (parent kept, partly filled last block)
+    spec.append((400, [3, 9, 27]))               # 3 siblings: too few to group
     nb = 20 + sum(-(-(pt + max(sx, default=0) + 2) // 16) * (len(sx) + 1) for pt, sx in spec)
     wl = workloads.Workload(0, "groups", "bf16", nb, hq, hkv, d, 1.0 / np.sqrt(d),
                             rng.permutation(nb).astype(np.int32))
     seq = 0
     seqs = []
-    for pt, sx in spec:
-        parent = 1000 + seq
+    for fi, (pt, sx) in enumerate(spec):
+        parent = 1000 + fi
         wl.ops.append(("add", parent))
         wl.ops.append(("append", parent, workloads.normal(rng, (pt, hkv, d), "bf16"),
                        workloads.normal(rng, (pt, hkv, d), "bf16")))
@@ -270,7 +271,7 @@ def test_shared_prefix_groups_match_oracle(g):
     l2 = l.copy()
     l2[:4] = 1024
     fam = [i for i, L in enumerate(l) if L == 513]
-    assert len(fam) == 2
+    assert len(fam) == 8
     l2[fam] = 512
     ref2 = ts.oracle_decode(step, tables=t, lens=l2)
     for part in (48, 256, 512, 1024):
