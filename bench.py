@@ -3,10 +3,11 @@
 Workload (default): Llama-3-8B-shaped GQA decode with prefix sharing, bf16 -- 256
 sequences in 16 groups of 16 sharing a 512-token prefix (32 shared blocks), private
 lognormal suffixes (median 600, cap 8192), 32 query / 8 kv heads, head_dim 128,
-block_size 16.  One step = the whole decode hot path for one batch:
-pa_cache_write of the 256 new tokens' K/V through their slot mapping, then
-pa_decode over every sequence (split-K partitions of 512 tokens; sibling runs
-that share whole partitions read them once as a group; LSE reduce).
+block_size 16.  One step = the whole decode hot path for one batch: the 256 new
+tokens' K/V written through their slot mapping, then decode attention over every
+sequence (split-K partitions of 512 tokens; sibling runs that share whole
+partitions read them once as a group; LSE reduce) -- one pa_append_decode call.
+The same step as two calls (pa_cache_write, pa_decode) is timed as well.
 
 Timed region: K steps after W warm-up steps, CUDA events on the launching stream,
 barrier + synchronize on both sides, max over ranks.  The step's inputs (1.1 GB of
@@ -173,16 +174,16 @@ def max_over_ranks(x, world):
 
 # ----------------------------------------------------------------- profiles
 def recorded_traffic():
-    """DRAM bytes of one pa_decode call (all its kernels) from the committed ncu
-    summary, or None if a kernel source changed since the counters were taken."""
+    """DRAM bytes of one pa_append_decode call (all its kernels) from the committed
+    ncu summary, or None if a kernel source changed since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "decode_gqa8b_prefix_ncu.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    mt = re.search(r"dram bytes per pa_decode call \(read\+write\): (\d+)", text)
+    mt = re.search(r"dram bytes per pa_append_decode call \(read\+write\): (\d+)", text)
     if not mt:
         return None
-    for name in ("decode.cu", "prefill.cu"):
+    for name in ("cache_ops.cu", "decode.cu", "prefill.cu"):
         mh = re.search(name.replace(".", r"\.") + r" sha256: ([0-9a-f]{64})", text)
         src = os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", name)
         if not mh or hashlib.sha256(open(src, "rb").read()).hexdigest() != mh.group(1):
@@ -227,7 +228,18 @@ def run_ours(args):
     log(f"rank {rank}: setup {time.time() - t_setup:.1f}s; {S} seqs, max ctx {max_ctx}, "
         f"unique {unique_b / 1e9:.3f} GB, logical {logical_b / 1e9:.3f} GB")
 
+    # one step = write the new tokens' K/V, then decode every sequence: one
+    # pa_append_decode call (the write and the decode kernels chained)
     def step_fn(ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record(stream)
+        pa.pa_append_decode(k_new, v_new, slots_d, q, cache.key_cache, cache.value_cache, tables_d, lens_d,
+                            max_ctx, wl.scale, out, part, ws, cache.err_flag, stream)
+        if ev_b is not None:
+            ev_b.record(stream)
+
+    # the same step as two calls, pa_cache_write then pa_decode (the decode bracketed)
+    def two_calls_fn(ev_a=None, ev_b=None):
         pa.pa_cache_write(k_new, v_new, slots_d, cache.key_cache, cache.value_cache, cache.err_flag, stream)
         if ev_a is not None:
             ev_a.record(stream)
@@ -259,9 +271,26 @@ def run_ours(args):
     barrier(world)
     sampler.stop()
     ms = e0.elapsed_time(e1)
-    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
     ms_max = max_over_ranks(ms, world)
     clocks = sampler.summary(h0, h1)
+
+    # the same step as two calls, for comparison: whole step and the decode call alone
+    for _ in range(3):
+        two_calls_fn()
+    nf = min(K, 500)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nf)]
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    f0.record(stream)
+    for i in range(nf):
+        two_calls_fn(*ev2[i])
+    f1.record(stream)
+    torch.cuda.synchronize()
+    two_ms = max_over_ranks(f0.elapsed_time(f1) / nf, world)
+    dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev2]))
+    assert pa.pa_wait(cache.err_flag) == 0
 
     # end to end: host buffers in, result out, through the same calls
     e2e = None
@@ -314,7 +343,7 @@ def run_ours(args):
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
             if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
         peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
-        achieved = unique_b / (dec_ms * 1e-3) / 1e9
+        achieved = (unique_b + cw_b) / (call_ms * 1e-3) / 1e9
         value = world * (unique_b + cw_b) * K / (ms_max * 1e-3) / 1e9
         line = {
             "metric": "paged-decode KV GB/s (unique algorithmic bytes) on B200",
@@ -332,12 +361,16 @@ def run_ours(args):
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "logical_gbs": round(world * (logical_b + cw_b) * K / (ms_max * 1e-3) / 1e9, 2),
             "bytes_per_step": {"decode_unique": unique_b, "decode_logical": logical_b, "cache_write": cw_b},
-            "roofline": {"bound": "hbm", "kernel": "pa_decode call (group detection + tcgen05 group tiles + decode_kernel + lse reduce)",
+            "roofline": {"bound": "hbm", "kernel": "pa_append_decode call (cache write + group detection + tcgen05 group tiles + decode_kernel + lse reduce)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if peaks else "fallback",
                          "traffic": recorded_traffic(),
-                         "decode_ms": round(dec_ms, 5)},
+                         "call_ms": round(call_ms, 5)},
+            "two_calls": {"ms_per_step": round(two_ms, 5),
+                          "value": round(world * (unique_b + cw_b) / (two_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                          "pa_decode_ms": round(dec_ms, 5),
+                          "pa_decode_gbs": round(unique_b / (dec_ms * 1e-3) / 1e9, 1), "steps": nf},
             "e2e": e2e,
             "gpu_launches": K * (1 + pa.pa_decode_launches(S, wl.head_dim, pa.PA_BF16, part)),
             "clocks": clocks,
@@ -486,6 +519,32 @@ def run_rows(reps, peaks, partition=PARTITION):
     ms = _time(lambda: pa.pa_cache_write(kn, vn, slots, cache.key_cache, cache.value_cache, cache.err_flag), reps,
                graph=True)
     rows["a1_cache_write_512tok"] = {"ms": round(ms, 5), "gbs": round(cache_write_bytes(wl, S) / ms / 1e6, 1)}
+    del cache
+    torch.cuda.empty_cache()
+
+    # -- speculative verify on the prefix-sharing workload: every sequence appends 4
+    #    draft tokens; the 4 new positions attend causally (a 4-row chunk)
+    wl = workloads.make(CONFIG_ID)
+    cache, dev = _setup(wl)
+    seqs = wl.steps[0].seqs
+    S, kdraft = len(seqs), 4
+    rng = np.random.default_rng(7)
+    kd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
+    vd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
+    cache.append(seqs, kd, vd, counts=[kdraft] * S)
+    mb = max(cache.manager.num_seq_blocks(s) for s in seqs)
+    t, l = cache.manager.build_tables(seqs, mb)
+    td, ld = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda()
+    qv = dev(workloads.normal(rng, (S, kdraft, wl.num_q_heads, wl.head_dim), "bf16"))
+    outv = torch.empty_like(qv)
+    chv = torch.full((S,), kdraft, dtype=torch.int32, device="cuda")
+    ms = _time(lambda: pa.pa_prefill_chunk(qv, cache.key_cache, cache.value_cache, td, ld, chv, wl.scale, outv,
+                                           cache.err_flag), reps)
+    ub, lb = step_bytes(wl, t, l)
+    rows["a6_spec_verify_k4"] = {"ms": round(ms, 5), "verified_tokens_per_s": round(S * kdraft / ms * 1e3, 1),
+                                 "kv_logical_gbs": round(lb / ms / 1e6, 1), "kv_unique_gbs": round(ub / ms / 1e6, 1),
+                                 "draft_tokens": kdraft, "num_seqs": S}
+    assert pa.pa_wait(cache.err_flag) == 0
     del cache
     torch.cuda.empty_cache()
 

@@ -180,6 +180,27 @@ PA_API pa_status pa_decode(const void *query, const void *key_cache, const void 
                     int32_t *err_flag, void *stream);
 
 /*
+ * One decode step in one call: pa_cache_write(key, value, slot_mapping,
+ * num_tokens, ...) followed by pa_decode(...) on the same stream, with the same
+ * results (the same kernels run).  The write and the decode's shared-prefix
+ * detection run side by side and the decode kernels start without a launch gap
+ * (programmatic dependent launch); everything that reads the cache still waits
+ * for the write.  Copy-on-write pairs must be applied (pa_copy_blocks) before.
+ * Both sets of arguments are validated before anything is launched; argument
+ * meaning and errors are those of the two calls.  num_tokens == 0 skips the write.
+ * Source: chenxutan 3.1 (each step writes the new token's K/V back into the
+ * cache, then attends over it).
+ */
+PA_API pa_status pa_append_decode(const void *key, const void *value, const int64_t *slot_mapping,
+                                  int32_t num_tokens, const void *query, void *key_cache,
+                                  void *value_cache, const int32_t *block_tables,
+                                  int32_t max_blocks_per_seq, const int32_t *context_lens,
+                                  int32_t max_context_len, int32_t num_seqs, int32_t num_q_heads,
+                                  float scale, int32_t partition_size, void *workspace,
+                                  size_t workspace_bytes, void *out, const pa_cache_desc *cache,
+                                  int32_t *err_flag, void *stream);
+
+/*
  * pa_decode with its split-K scratch taken from a fixed array inside the library
  * instead of a caller-provided workspace.  The pages have no counterpart: this
  * exists for callers that cannot allocate device memory -- code running inside an
@@ -215,6 +236,10 @@ PA_API pa_status pa_decode_static_scratch(const void *query, const void *key_cac
  * query/out: [num_seqs, max_chunk, num_q_heads, head_dim]; rows i >= C_s of out
  * are not written.  Requires dtype PA_BF16 and head_dim 128 (tcgen05 tensor-core
  * tiles, bf16 operands, fp32 accumulation in tensor memory).
+ * A speculative-decoding verify step is the same operation: each sequence appends
+ * its k_s draft tokens (pa_cache_write), then the k_s new positions attend
+ * causally with chunk_lens[s] = k_s (chenxutan 5.4, speculative decoding: the
+ * target model checks several proposed tokens in one pass).
  * Source: chenxutan 2.3 (prefill computes a whole prompt and is compute bound)
  * and 4.3/5.1 (long prompts are cut into chunks that run between decodes).
  */

@@ -50,6 +50,8 @@ def _load():
         "pa_decode_launches": (i32, [i32, i32, i32, i32]),
         "pa_decode": (C.c_int, [vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, i32, vp, sz, vp, desc,
                                 vp, vp]),
+        "pa_append_decode": (C.c_int, [vp, vp, vp, i32, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, i32,
+                                       vp, sz, vp, desc, vp, vp]),
         "pa_prefill_chunk": (C.c_int, [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, f32, vp, desc,
                                        vp, vp]),
         "pa_wait": (C.c_int, [vp, vp, i32, C.POINTER(i32)]),
@@ -80,7 +82,8 @@ _lib = _load()
 
 EXPORTED = (
     "pa_abi_version", "pa_status_string", "pa_cache_write", "pa_copy_blocks",
-    "pa_decode_workspace_size", "pa_decode_launches", "pa_decode", "pa_prefill_chunk", "pa_wait",
+    "pa_decode_workspace_size", "pa_decode_launches", "pa_decode", "pa_append_decode", "pa_prefill_chunk",
+    "pa_wait",
 )
 
 
@@ -185,6 +188,28 @@ def pa_decode(query, key_cache, value_cache, block_tables, context_lens, max_con
                           block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, hq,
                           float(scale), int(partition_size), _ptr(workspace), ws_bytes, _ptr(out),
                           C.byref(d), _ptr(err_flag), _stream(stream)), "pa_decode")
+
+
+def pa_append_decode(key, value, slot_mapping, query, key_cache, value_cache, block_tables, context_lens,
+                     max_context_len, scale, out, partition_size=0, workspace=None, err_flag=None,
+                     stream=None):
+    """pa_cache_write(key, value, slot_mapping, ...) then pa_decode(...) in one call."""
+    torch = _torch()
+    _same_pool(key_cache, value_cache)
+    assert key.shape == value.shape and key.dim() == 3 and key.shape[1:] == (key_cache.shape[1], key_cache.shape[3])
+    assert key.dtype == key_cache.dtype == value.dtype and slot_mapping.dtype == torch.int64
+    assert slot_mapping.shape == (key.shape[0],)
+    S, hq, dd = query.shape
+    assert out.shape == query.shape and out.dtype == query.dtype == key_cache.dtype
+    assert block_tables.dtype == torch.int32 and block_tables.dim() == 2 and block_tables.shape[0] == S
+    assert context_lens.dtype == torch.int32 and context_lens.shape == (S,)
+    d = cache_desc(key_cache)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.pa_append_decode(_ptr(key), _ptr(value), _ptr(slot_mapping), key.shape[0], _ptr(query),
+                                 _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), block_tables.shape[1],
+                                 _ptr(context_lens), int(max_context_len), S, hq, float(scale),
+                                 int(partition_size), _ptr(workspace), ws_bytes, _ptr(out), C.byref(d),
+                                 _ptr(err_flag), _stream(stream)), "pa_append_decode")
 
 
 def pa_prefill_chunk(query, key_cache, value_cache, block_tables, context_lens, chunk_lens, scale,

@@ -16,6 +16,9 @@ __global__ void __launch_bounds__(256) cache_write_kernel(
     const int64_t *__restrict__ slot_mapping, int32_t num_tokens, uint4 *__restrict__ key_cache,
     uint4 *__restrict__ value_cache, int32_t num_kv_heads, int32_t chunks_per_row,
     int64_t num_slots, int32_t *err) {
+    // a decode launched behind this write (pa_append_decode) may start launching;
+    // whatever of it reads the cache waits for this grid to finish
+    grid_dep_launch();
     const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t per_token = (int64_t)num_kv_heads * chunks_per_row;
     const int64_t token = idx / per_token;

@@ -127,6 +127,7 @@ struct Params {
     const int4 *groups;     // (first seq, members, shared partitions, units before)
     const int32_t *meta;    // [0] groups, [1] group units
     int32_t max_members;    // sequences per group: query rows members x g <= 128
+    int32_t wait_first;     // launched right behind a cache write: wait for it first
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -563,8 +564,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     // When launched behind the group tiles, this grid reads only what the
     // detection wrote (complete before the tiles let it start) and writes other
     // partitions; it waits for the tiles only before exiting, so that its
-    // completion implies theirs.
+    // completion implies theirs.  Launched right behind a cache write instead
+    // (pa_append_decode without groups), it waits for the write first.
     grid_dep_launch();
+    if (p.wait_first) grid_dep_wait();
     // merge slot hand-over: full[b] when all warps wrote their state of the
     // slot's unit, freed[b] when all warps finished their share of its merge
     uint64_t *mfull = reinterpret_cast<uint64_t *>(smem + Lay::kOffBar);
@@ -873,6 +876,10 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     const int S = p.num_seqs;
     shared_prefix_lengths(p, lcp);
     __syncthreads();
+    // Behind a cache write (pa_append_decode) this kernel neither reads nor writes
+    // the cache, so it runs alongside the write, but it finishes only after it:
+    // the group tiles wait for this kernel and so see the new tokens' K/V.
+    grid_dep_wait();
     if (threadIdx.x >= 32) return;
     // warp 0: lane owns sequences [s0, s1)
     const int lane = threadIdx.x;
@@ -998,10 +1005,17 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             prm.groups = reinterpret_cast<int4 *>(g + sa);
             prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
             prm.max_members = 128 / G;
-            group_detect_kernel<<<1, kDetectThreads, 0, stream>>>(prm, const_cast<int32_t *>(prm.first_p),
-                                                                  const_cast<int4 *>(prm.groups),
-                                                                  const_cast<int32_t *>(prm.meta));
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if (a.after_write) {
+                e = launch_after(group_detect_kernel, dim3(1), dim3(kDetectThreads), 0, stream,
+                                 static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_p),
+                                 const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta));
+            } else {
+                group_detect_kernel<<<1, kDetectThreads, 0, stream>>>(prm, const_cast<int32_t *>(prm.first_p),
+                                                                      const_cast<int4 *>(prm.groups),
+                                                                      const_cast<int32_t *>(prm.meta));
+                e = cudaGetLastError();
+            }
+            if (e != cudaSuccess) return e;
             GroupTileLaunch gl;
             gl.query = a.query;
             gl.key_cache = a.key_cache;
@@ -1026,7 +1040,8 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
     int64_t grid = sms;
     if (!split) grid = std::min<int64_t>(grid, (int64_t)a.num_seqs * a.cache.num_kv_heads);
     if (grid < 1) grid = 1;
-    if (grouped) {
+    prm.wait_first = (!grouped && a.after_write) ? 1 : 0;
+    if (grouped || a.after_write) {
         e = launch_after(decode_kernel<T, D, G>, dim3((unsigned)grid), dim3(kThreads), smem, stream,
                          static_cast<const Params &>(prm));
     } else {

@@ -64,9 +64,10 @@ const char *pa_status_string(pa_status s) {
     return "unknown status";
 }
 
-pa_status pa_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
-                         int32_t num_tokens, void *key_cache, void *value_cache,
-                         const pa_cache_desc *cache, int32_t *err_flag, void *stream) {
+namespace {
+pa_status check_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
+                            int32_t num_tokens, const void *key_cache, const void *value_cache,
+                            const pa_cache_desc *cache) {
     pa_status st = check_cache(cache);
     if (st != PA_OK) return st;
     if (num_tokens < 0) return PA_ERR_INVALID_ARG;
@@ -74,6 +75,15 @@ pa_status pa_cache_write(const void *key, const void *value, const int64_t *slot
     if (!key || !value || !slot_mapping || !key_cache || !value_cache) return PA_ERR_INVALID_ARG;
     if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
         return PA_ERR_INVALID_ARG;
+    return PA_OK;
+}
+}  // namespace
+
+pa_status pa_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
+                         int32_t num_tokens, void *key_cache, void *value_cache,
+                         const pa_cache_desc *cache, int32_t *err_flag, void *stream) {
+    const pa_status st = check_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache, cache);
+    if (st != PA_OK || num_tokens == 0) return st;
     return from_cuda(launch_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache,
                                         *cache, err_flag, static_cast<cudaStream_t>(stream)));
 }
@@ -113,12 +123,14 @@ int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype, in
     return grouped ? 4 : 2;
 }
 
-pa_status pa_decode(const void *query, const void *key_cache, const void *value_cache,
-                    const int32_t *block_tables, int32_t max_blocks_per_seq,
-                    const int32_t *context_lens, int32_t max_context_len, int32_t num_seqs,
-                    int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
-                    size_t workspace_bytes, void *out, const pa_cache_desc *cache,
-                    int32_t *err_flag, void *stream) {
+namespace {
+// Validate pa_decode's arguments and fill the launch record; launches nothing.
+pa_status prepare_decode(const void *query, const void *key_cache, const void *value_cache,
+                         const int32_t *block_tables, int32_t max_blocks_per_seq,
+                         const int32_t *context_lens, int32_t max_context_len, int32_t num_seqs,
+                         int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
+                         size_t workspace_bytes, void *out, const pa_cache_desc *cache,
+                         int32_t *err_flag, DecodeLaunch &a) {
     pa_status st = check_cache(cache);
     if (st != PA_OK) return st;
     st = check_group(num_q_heads, cache->num_kv_heads);
@@ -134,7 +146,7 @@ pa_status pa_decode(const void *query, const void *key_cache, const void *value_
         return PA_ERR_INVALID_ARG;
     if ((int64_t)max_context_len > (int64_t)max_blocks_per_seq * kBlockSize)
         return PA_ERR_INVALID_ARG;
-    DecodeLaunch a{};
+    a = DecodeLaunch{};
     if (partition_size > 0 && max_context_len > partition_size) {
         if (num_seqs > kMaxSplitSeqs) return PA_ERR_UNSUPPORTED;
         const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, cache->head_dim,
@@ -165,7 +177,48 @@ pa_status pa_decode(const void *query, const void *key_cache, const void *value_
     a.out = out;
     a.cache = *cache;
     a.err = err_flag;
+    return PA_OK;
+}
+
+}  // namespace
+
+pa_status pa_decode(const void *query, const void *key_cache, const void *value_cache,
+                    const int32_t *block_tables, int32_t max_blocks_per_seq,
+                    const int32_t *context_lens, int32_t max_context_len, int32_t num_seqs,
+                    int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
+                    size_t workspace_bytes, void *out, const pa_cache_desc *cache,
+                    int32_t *err_flag, void *stream) {
+    DecodeLaunch a;
+    const pa_status st = prepare_decode(query, key_cache, value_cache, block_tables, max_blocks_per_seq,
+                                        context_lens, max_context_len, num_seqs, num_q_heads, scale,
+                                        partition_size, workspace, workspace_bytes, out, cache, err_flag, a);
+    if (st != PA_OK || num_seqs == 0) return st;
     return from_cuda(launch_decode(a, static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_append_decode(const void *key, const void *value, const int64_t *slot_mapping,
+                           int32_t num_tokens, const void *query, void *key_cache, void *value_cache,
+                           const int32_t *block_tables, int32_t max_blocks_per_seq,
+                           const int32_t *context_lens, int32_t max_context_len, int32_t num_seqs,
+                           int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
+                           size_t workspace_bytes, void *out, const pa_cache_desc *cache,
+                           int32_t *err_flag, void *stream) {
+    pa_status st = check_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache, cache);
+    if (st != PA_OK) return st;
+    DecodeLaunch a;
+    st = prepare_decode(query, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens,
+                        max_context_len, num_seqs, num_q_heads, scale, partition_size, workspace,
+                        workspace_bytes, out, cache, err_flag, a);
+    if (st != PA_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (num_tokens > 0) {
+        st = from_cuda(launch_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache, *cache,
+                                          err_flag, s));
+        if (st != PA_OK) return st;
+        a.after_write = true;  // the decode chain starts behind the write
+    }
+    if (num_seqs == 0) return PA_OK;
+    return from_cuda(launch_decode(a, s));
 }
 
 pa_status pa_prefill_chunk(const void *query, const void *key_cache, const void *value_cache,

@@ -57,6 +57,7 @@ struct DecodeLaunch {
     void *out;
     pa_cache_desc cache;
     int32_t *err;
+    bool after_write;  // launched behind a cache write on the same stream (pa_append_decode)
 };
 
 // Largest num_seqs a split decode supports (the per-CTA partition prefix sum

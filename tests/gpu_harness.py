@@ -128,6 +128,40 @@ class TwoSided:
                           self.gpu.key_cache, self.gpu.value_cache, self.gpu.err_flag)
         self.last_pairs = np.array(pairs_o, np.int32).reshape(-1, 2)
 
+    def append_decode_step(self, step, partition_size=0):
+        """The step's copy-on-write and cache write on both sides, then the GPU side's
+        write + decode as one pa_append_decode call.  Returns the GPU output."""
+        torch = torch_mod()
+        pa = self.pa
+        slots_o, pairs_o = [], []
+        for s in step.seqs:
+            sl, pr = self.model.append_slot(s)
+            slots_o.append(sl)
+            if pr is not None:
+                pairs_o.append(pr)
+        slots_g, pairs_g = self.gpu.plan_append(step.seqs)
+        assert slots_g.tolist() == slots_o and [tuple(p) for p in pairs_g.tolist()] == pairs_o
+        if pairs_o:
+            oracle.copy_blocks(self.kc, self.vc, np.array(pairs_o, np.int32))
+            pa.pa_copy_blocks(self.gpu.key_cache, self.gpu.value_cache,
+                              torch.from_numpy(pairs_g).cuda(), self.gpu.err_flag)
+        sl = np.array(slots_o, np.int64)
+        oracle.cache_write(step.k_new, step.v_new, sl, self.kc, self.vc)
+        t, l = self.tables(step.seqs)
+        q = to_dev(step.q)
+        out = torch.empty_like(q)
+        maxc = max(int(l.max(initial=1)), 1)
+        ws = None
+        if partition_size:
+            n = pa.pa_decode_workspace_size(len(step.seqs), q.shape[1], q.shape[2], maxc, partition_size)
+            ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+        pa.pa_append_decode(to_dev(step.k_new), to_dev(step.v_new), torch.from_numpy(sl).cuda(), q,
+                            self.gpu.key_cache, self.gpu.value_cache, torch.from_numpy(t).cuda(),
+                            torch.from_numpy(l).cuda(), maxc, self.wl.scale, out, partition_size, ws,
+                            self.gpu.err_flag)
+        self.last_pairs = np.array(pairs_o, np.int32).reshape(-1, 2)
+        return to_host(out)
+
     def gpu_decode(self, step, partition_size=0, tables=None, lens=None, max_context=None):
         torch = torch_mod()
         t, l = self.tables(step.seqs) if tables is None else (tables, lens)

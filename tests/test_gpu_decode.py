@@ -278,3 +278,27 @@ def test_shared_prefix_groups_match_oracle(g):
         got = ts.gpu_decode(step, part, tables=t, lens=l2, max_context=int(l.max()))
         check_close(got, ref2, "bf16", f"g{g} fully shared members, partition {part}")
     assert ts.err_flag() == 0
+
+
+@pytest.mark.parametrize("cid,part", [(1, 0), (1, 16), (2, 256), (3, 0), (3, 256), (4, 256)])
+def test_append_decode_one_call(cid, part):
+    """pa_append_decode (cache write + decode in one call, chained launches) gives the
+    oracle's result for every step and leaves the pools bit-identical to the oracle's."""
+    wl = workloads.make(cid, mini=cid != 1)
+    ts = TwoSided(wl)
+    for i, step in enumerate(wl.steps[:3]):
+        got = ts.append_decode_step(step, part)
+        assert ts.pools_equal(), f"config {cid} step {i}: pools differ"
+        check_close(got, ts.oracle_decode(step), wl.dtype, f"append+decode config {cid} step {i} partition {part}")
+    assert ts.err_flag() == 0
+
+
+def test_append_decode_matches_two_calls_bitwise():
+    """Same kernels, same order of arithmetic: one call and two calls agree bit for bit."""
+    wl = workloads.make(3, mini=True)
+    a, b = TwoSided(wl), TwoSided(wl)
+    step = wl.steps[0]
+    got = a.append_decode_step(step, 256)
+    b.append_step(step)
+    ref = b.gpu_decode(step, 256)
+    assert got.tobytes() == ref.tobytes()

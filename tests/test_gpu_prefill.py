@@ -107,3 +107,38 @@ def test_long_context_chunk_full_sampled_rows():
     ref = oracle.prefill(pf.q, ts.kc, ts.vc, t, l, np.array(ch, np.int32), wl.scale, row_mask=mask)
     check_close(got[mask], ref[mask], "bf16", "prefill full (sampled rows)")
     assert ts.err_flag() == 0
+
+
+@pytest.mark.parametrize("hq,hkv", [(32, 8), (16, 16), (64, 8)])
+def test_speculative_verify_chunks(hq, hkv):
+    """Speculative-decoding verify: every sequence appends k_s in [1, 8] draft tokens and
+    the k_s new positions attend causally to the paged cache -- a k_s-row chunk.  Shapes of
+    the prefix-sharing workload (siblings sharing prefix blocks), ragged k_s."""
+    rng = np.random.default_rng(17)
+    d, S, prefix = 128, 12, 96
+    ks = rng.integers(1, 9, size=S).tolist()
+    suffix = rng.integers(1, 200, size=S).tolist()
+    need = 3 * (prefix // 16) + sum(-(-(prefix + x + k) // 16) for x, k in zip(suffix, ks)) + 8
+    wl = workloads.Workload(0, "verify", "bf16", need, hq, hkv, d, 1.0 / np.sqrt(d),
+                            rng.permutation(need).astype(np.int32))
+    for grp in range(3):                       # 3 parents x 4 forked siblings
+        parent = 100 + grp
+        wl.ops.append(("add", parent))
+        wl.ops.append(("append", parent, workloads.normal(rng, (prefix, hkv, d), "bf16"),
+                       workloads.normal(rng, (prefix, hkv, d), "bf16")))
+        for c in range(4):
+            wl.ops.append(("fork", parent, grp * 4 + c))
+        wl.ops.append(("free", parent))
+    for s in range(S):                         # private suffix, then the k_s draft tokens
+        n = suffix[s] + ks[s]
+        wl.ops.append(("append", s, workloads.normal(rng, (n, hkv, d), "bf16"),
+                       workloads.normal(rng, (n, hkv, d), "bf16")))
+    ts = TwoSided(wl)
+    assert ts.pools_equal()
+    t, l = ts.tables(list(range(S)))
+    q = workloads.normal(rng, (S, 8, hq, d), "bf16")
+    got = gpu_prefill(ts, q, ks, t, l)
+    ref = oracle.prefill(q, ts.kc, ts.vc, t, l, np.array(ks, np.int32), wl.scale)
+    mask = rows_mask(ks, 8)
+    check_close(got[mask], ref[mask], "bf16", f"verify {hq}/{hkv}")
+    assert ts.err_flag() == 0
