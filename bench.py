@@ -548,6 +548,23 @@ def run_rows(reps, peaks, partition=PARTITION):
     del cache
     torch.cuda.empty_cache()
 
+    # -- automatic prefix caching (host): 256 prompts = a shared 512-token system
+    #    prompt + a private lognormal tail, created from their token ids
+    bm = pa.BlockManager(32768, 16)
+    prng = np.random.default_rng(11)
+    system = prng.integers(0, 32000, size=512).tolist()
+    tails = np.clip(np.rint(600 * np.exp(prng.standard_normal(256))), 1, 8192).astype(int)
+    prompts = [system + prng.integers(0, 32000, size=int(n)).tolist() for n in tails]
+    h0 = time.perf_counter()
+    hit = sum(bm.add_seq_tokens(i, pr)[0] for i, pr in enumerate(prompts))
+    host_s = time.perf_counter() - h0
+    total = sum(len(pr) for pr in prompts)
+    rows["a7_prefix_cache_host"] = {"prompts": len(prompts), "prompt_tokens": total, "cached_tokens": int(hit),
+                                    "hit_fraction": round(hit / total, 4), "kv_writes_saved_bytes":
+                                    int(hit) * 8 * 128 * 2 * 2,
+                                    "host_us_per_prompt": round(1e6 * host_s / len(prompts), 2)}
+    del bm
+
     # -- long context: split-K decode + tcgen05 prefill chunk
     wl = workloads.make(5)
     cache, dev = _setup(wl)

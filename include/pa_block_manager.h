@@ -27,6 +27,28 @@
  *     reaches zero onto the free stack;
  *   - an operation that would run out of blocks fails with PA_ERR_OOM and
  *     changes nothing.
+ *
+ * Automatic prefix caching (chenxutan "vLLM 深度拆解" 5.2: prompts that share a
+ * prefix -- a system prompt, RAG context -- reuse its KV instead of computing it
+ * again, without the caller naming the prefix).  The pages give no mechanism;
+ * the reading taken:
+ *   - only sequences created from their prompt's token ids (pa_bm_add_seq_tokens)
+ *     take part; a full block of such a prompt is indexed by the key (parent
+ *     physical block, the parent's generation, its block_size token ids), where
+ *     the parent is the previous block of the same prompt (-1 for the first) and
+ *     a block's generation counts how often it has been handed out -- so a key
+ *     identifies the whole prefix up to and including the block, and a block that
+ *     was reclaimed and reused never matches its old children's keys;
+ *   - a new prompt reuses the longest run of leading full blocks found in the
+ *     index (counts go up by one) and allocates the rest as appends would; its
+ *     own full blocks are indexed;
+ *   - an indexed block whose count drops to zero is not freed but becomes
+ *     evictable (still indexed, reusable by a later prompt); free_seq puts a
+ *     sequence's evictable blocks last-block first; allocation takes the free
+ *     stack first, then reclaims the least recently evictable block (removing it
+ *     from the index);
+ *   - blocks filled by later appends are not indexed (their token ids are not
+ *     known here).
  */
 #ifndef PA_BLOCK_MANAGER_H_
 #define PA_BLOCK_MANAGER_H_
@@ -82,7 +104,8 @@ PA_API pa_status pa_bm_block_table(const pa_block_manager *bm, int64_t seq_id, i
 PA_API pa_status pa_bm_build_tables(const pa_block_manager *bm, const int64_t *seq_ids, int32_t n,
                              int32_t max_blocks, int32_t *tables_out, int32_t *lens_out);
 
-/* Reference count of a block (-1 if out of range), free-block count, pool size. */
+/* Reference count of a block (-1 if out of range), free-stack length (evictable
+ * blocks are counted by pa_bm_num_evictable), pool size. */
 PA_API int32_t pa_bm_refcount(const pa_block_manager *bm, int32_t block);
 PA_API int32_t pa_bm_num_free(const pa_block_manager *bm);
 PA_API int32_t pa_bm_num_blocks(const pa_block_manager *bm);
@@ -93,6 +116,25 @@ PA_API int32_t pa_bm_free_stack(const pa_block_manager *bm, int32_t *out, int32_
 
 /* Tokens stored over all live sequences (for utilisation statistics). */
 PA_API int64_t pa_bm_tokens_stored(const pa_block_manager *bm);
+
+/* Register sequence seq_id holding the n prompt tokens whose ids are tokens[0..n).
+ * The longest run of leading full blocks already in the prefix index is reused;
+ * *num_cached_out (nullable) receives the number of tokens it covers (a multiple
+ * of block_size) -- their K/V are already in the cache.  slots_out (nullable,
+ * n - *num_cached_out entries) receives the slots of the remaining tokens, in
+ * order, for pa_cache_write.  Full blocks of the prompt are entered in the index.
+ * PA_ERR_INVALID_ARG if seq_id exists; PA_ERR_OOM (nothing changed) if too few
+ * blocks are free or evictable. */
+PA_API pa_status pa_bm_add_seq_tokens(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens,
+                                      int32_t n, int64_t *slots_out, int32_t *num_cached_out);
+
+/* Indexed blocks with count zero (reclaimable), and all indexed blocks. */
+PA_API int32_t pa_bm_num_evictable(const pa_block_manager *bm);
+PA_API int32_t pa_bm_num_cached(const pa_block_manager *bm);
+
+/* Copy the evictable list, next reclaimed first, into out (at most capacity
+ * entries); returns its length (-1 if bm is NULL). */
+PA_API int32_t pa_bm_evictable(const pa_block_manager *bm, int32_t *out, int32_t capacity);
 
 #ifdef __cplusplus
 }

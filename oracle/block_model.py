@@ -35,6 +35,16 @@ silent or buggy are marked READING):
   reaches zero is pushed on the free stack at that moment.
 * Out of memory leaves every structure unchanged (devpress "关键设计一" raises
   before touching the table).
+* Automatic prefix caching -- chenxutan 5.2 (prompts sharing a prefix reuse its
+  KV; automatic).  READING (the pages give no mechanism): a sequence created from
+  its prompt's token ids (``add_seq_tokens``) reuses the longest run of leading
+  full blocks whose exact key is known, key = (parent block, the parent's
+  generation, the block's token ids), parent = the prompt's previous block (-1
+  for the first), generation = how often the block has been allocated.  Its own
+  full blocks are entered under their keys.  A keyed block reaching count zero
+  becomes evictable instead of free (a freed sequence's such blocks from the last
+  to the first); allocation uses the free stack first, then reclaims the
+  earliest evictable block and forgets its key.  Appended blocks get no key.
 """
 from __future__ import annotations
 
@@ -58,19 +68,36 @@ class BlockManagerModel:
         self.ref = [0] * self.num_blocks
         self.tables: dict[int, list[int]] = {}
         self.ntok: dict[int, int] = {}
+        self.gen = [0] * self.num_blocks          # times each block was allocated
+        self.key: dict[int, tuple] = {}            # keyed block -> its key
+        self.index: dict[tuple, int] = {}          # key -> block
+        self.evictable_list: list[int] = []        # front = next reclaimed
 
     # -- allocator -----------------------------------------------------------
     def _allocate(self) -> int:
-        if not self.free_stack:
+        if self.free_stack:
+            b = self.free_stack.pop()
+        elif self.evictable_list:
+            b = self.evictable_list.pop(0)
+            del self.index[self.key.pop(b)]
+        else:
             raise OutOfBlocks("no free blocks")
-        b = self.free_stack.pop()
         self.ref[b] = 1
+        self.gen[b] += 1
         return b
 
-    def _drop(self, b: int) -> None:
+    def _drop(self, b: int) -> bool:
+        """Drop a reference; True when a keyed block reached zero (the caller
+        makes it evictable)."""
         self.ref[b] -= 1
         if self.ref[b] == 0:
+            if b in self.key:
+                return True
             self.free_stack.append(b)
+        return False
+
+    def _available(self) -> int:
+        return len(self.free_stack) + len(self.evictable_list)
 
     def num_free(self) -> int:
         return len(self.free_stack)
@@ -101,7 +128,7 @@ class BlockManagerModel:
         """Append n tokens; return (slots list, list of (src, dst) copy pairs)."""
         if seq not in self.tables:
             raise KeyError(f"no sequence {seq}")
-        if self._blocks_needed(seq, n) > len(self.free_stack):
+        if self._blocks_needed(seq, n) > self._available():
             raise OutOfBlocks(f"sequence {seq} needs more blocks than are free")
         B = self.block_size
         table = self.tables[seq]
@@ -114,7 +141,8 @@ class BlockManagerModel:
                 old = table[-1]
                 new = self._allocate()
                 pairs.append((old, new))
-                self._drop(old)
+                if self._drop(old):
+                    self.evictable_list.append(old)
                 table[-1] = new
             slots.append(table[-1] * B + k % B)
             self.ntok[seq] = k + 1
@@ -133,9 +161,57 @@ class BlockManagerModel:
     def free(self, seq: int) -> None:
         if seq not in self.tables:
             raise KeyError(f"no sequence {seq}")
-        for b in self.tables.pop(seq):
-            self._drop(b)
+        reached_zero = [b for b in self.tables.pop(seq) if self._drop(b)]
+        self.evictable_list.extend(reversed(reached_zero))
         del self.ntok[seq]
+
+    def add_seq_tokens(self, seq: int, tokens):
+        """Create a sequence from its prompt token ids; return (tokens whose K/V are
+        cached already, slots of the remaining tokens)."""
+        if seq in self.tables:
+            raise KeyError(f"sequence {seq} exists")
+        B = self.block_size
+        tokens = [int(t) for t in tokens]
+        n = len(tokens)
+        hits, parent, pgen = [], -1, 0
+        for j in range(n // B):
+            b = self.index.get((parent, pgen, tuple(tokens[j * B:(j + 1) * B])))
+            if b is None:
+                break
+            hits.append(b)
+            parent, pgen = b, self.gen[b]
+        need = -(-n // B) - len(hits)
+        if need > self._available() - sum(1 for b in hits if b in self.evictable_list):
+            raise OutOfBlocks(f"sequence {seq} needs more blocks than are free")
+        for b in hits:
+            if b in self.evictable_list:
+                self.evictable_list.remove(b)
+            self.ref[b] += 1
+        table = list(hits)
+        slots = []
+        for i in range(len(hits) * B, n):
+            off = i % B
+            if off == 0:
+                table.append(self._allocate())
+            slots.append(table[-1] * B + off)
+            if off == B - 1:
+                j = i // B
+                par = table[j - 1] if j > 0 else -1
+                k = (par, self.gen[par] if par >= 0 else 0, tuple(tokens[j * B:(j + 1) * B]))
+                self.index[k] = table[j]
+                self.key[table[j]] = k
+        self.tables[seq] = table
+        self.ntok[seq] = n
+        return len(hits) * B, slots
+
+    def num_evictable(self) -> int:
+        return len(self.evictable_list)
+
+    def num_cached(self) -> int:
+        return len(self.index)
+
+    def evictable(self) -> list[int]:
+        return list(self.evictable_list)
 
     def block_table(self, seq: int) -> list[int]:
         return list(self.tables[seq])

@@ -70,6 +70,10 @@ def _load():
         "pa_bm_num_blocks": (i32, [vp]),
         "pa_bm_free_stack": (i32, [vp, vp, i32]),
         "pa_bm_tokens_stored": (i64, [vp]),
+        "pa_bm_add_seq_tokens": (C.c_int, [vp, i64, vp, i32, vp, C.POINTER(i32)]),
+        "pa_bm_num_evictable": (i32, [vp]),
+        "pa_bm_num_cached": (i32, [vp]),
+        "pa_bm_evictable": (i32, [vp, vp, i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -334,3 +338,27 @@ class BlockManager:
 
     def tokens_stored(self) -> int:
         return int(_lib.pa_bm_tokens_stored(self._h))
+
+    def add_seq_tokens(self, seq: int, tokens):
+        """Create a sequence from its prompt token ids with automatic prefix caching.
+        Returns (number of leading tokens whose K/V are already cached, int64 slots
+        of the remaining tokens)."""
+        toks = np.ascontiguousarray(tokens, dtype=np.int32)
+        slots = np.empty(max(len(toks), 1), dtype=np.int64)
+        ncached = C.c_int32(0)
+        self._st(_lib.pa_bm_add_seq_tokens(self._h, int(seq), toks.ctypes.data_as(C.c_void_p), len(toks),
+                                           slots.ctypes.data_as(C.c_void_p), C.byref(ncached)),
+                 f"add_seq_tokens({seq}, {len(toks)})")
+        return int(ncached.value), slots[:len(toks) - ncached.value].copy()
+
+    def num_evictable(self) -> int:
+        return int(_lib.pa_bm_num_evictable(self._h))
+
+    def num_cached(self) -> int:
+        return int(_lib.pa_bm_num_cached(self._h))
+
+    def evictable(self) -> list:
+        n = _lib.pa_bm_evictable(self._h, None, 0)
+        out = np.empty(max(n, 1), dtype=np.int32)
+        _lib.pa_bm_evictable(self._h, out.ctypes.data_as(C.c_void_p), n)
+        return out[:n].tolist()

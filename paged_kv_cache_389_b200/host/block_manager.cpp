@@ -4,10 +4,19 @@
 // Data structures: a LIFO free stack of block ids, a reference count per block,
 // and a hash map from sequence id to (token count, block table).  Every mutating
 // call first works out how many fresh blocks it needs and fails with PA_ERR_OOM
-// before touching anything if the free stack is too short, so a failed call
-// leaves the manager exactly as it was.
+// before touching anything if too few can be had, so a failed call leaves the
+// manager exactly as it was.
+//
+// Automatic prefix caching (sequences created from prompt tokens): a full prompt
+// block is indexed by (parent block, parent's generation, its 16 token ids); a
+// block's generation counts how often it was handed out, so a key never matches
+// a block that has since been reused.  Cached blocks whose count drops to zero
+// stay indexed on an evictable list (least recently freed first, and a freed
+// sequence's blocks tail first) and are reclaimed only when the free stack is
+// empty.
 #include <cstdint>
 #include <cstring>
+#include <list>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -21,6 +30,30 @@ struct Sequence {
     std::vector<int32_t> blocks;  // logical block j -> physical block blocks[j]
 };
 
+struct CacheKey {
+    int32_t parent = -1;     // physical block before this one in the prompt (-1: first)
+    uint32_t parent_gen = 0;
+    std::vector<int32_t> tokens;
+    bool operator==(const CacheKey &o) const {
+        return parent == o.parent && parent_gen == o.parent_gen && tokens == o.tokens;
+    }
+};
+
+uint64_t key_hash(const CacheKey &k) {
+    // FNV-1a over the key's 32-bit words
+    uint64_t h = 1469598103934665603ull;
+    auto mix = [&](uint32_t w) {
+        for (int i = 0; i < 4; ++i) {
+            h ^= (w >> (8 * i)) & 0xffu;
+            h *= 1099511628211ull;
+        }
+    };
+    mix((uint32_t)k.parent);
+    mix(k.parent_gen);
+    for (int32_t t : k.tokens) mix((uint32_t)t);
+    return h;
+}
+
 }  // namespace
 
 struct pa_block_manager {
@@ -28,16 +61,72 @@ struct pa_block_manager {
     int32_t block_size = 0;
     std::vector<int32_t> free_stack;  // back() is the next block handed out
     std::vector<int32_t> refs;
+    std::vector<uint32_t> gen;        // times each block was handed out
     std::unordered_map<int64_t, Sequence> seqs;
+    // prefix cache
+    std::vector<char> cached;                      // block is in the index
+    std::vector<CacheKey> keys;                    // its key while cached
+    std::unordered_multimap<uint64_t, int32_t> index;
+    std::list<int32_t> evictable;                  // cached, count 0; front = next reclaimed
+    std::vector<std::list<int32_t>::iterator> evict_pos;
+    std::vector<char> on_evictable;
 
+    int32_t available() const { return (int32_t)(free_stack.size() + evictable.size()); }
+
+    void uncache(int32_t b) {
+        auto range = index.equal_range(key_hash(keys[b]));
+        for (auto it = range.first; it != range.second; ++it)
+            if (it->second == b) {
+                index.erase(it);
+                break;
+            }
+        cached[b] = 0;
+        keys[b] = CacheKey{};
+    }
     int32_t take() {
-        int32_t b = free_stack.back();
-        free_stack.pop_back();
+        int32_t b;
+        if (!free_stack.empty()) {
+            b = free_stack.back();
+            free_stack.pop_back();
+        } else {  // reclaim the least recently freed cached block
+            b = evictable.front();
+            evictable.pop_front();
+            on_evictable[b] = 0;
+            uncache(b);
+        }
         refs[b] = 1;
+        ++gen[b];
         return b;
     }
-    void release(int32_t b) {
-        if (--refs[b] == 0) free_stack.push_back(b);
+    // drop a reference; a block reaching zero goes to the free stack, or (cached)
+    // is returned for the caller to put on the evictable list
+    bool release(int32_t b) {
+        if (--refs[b] != 0) return false;
+        if (cached[b]) return true;
+        free_stack.push_back(b);
+        return false;
+    }
+    void make_evictable(int32_t b) {
+        evict_pos[b] = evictable.insert(evictable.end(), b);
+        on_evictable[b] = 1;
+    }
+    void revive(int32_t b) {  // a hit on a cached block
+        if (on_evictable[b]) {
+            evictable.erase(evict_pos[b]);
+            on_evictable[b] = 0;
+        }
+        ++refs[b];
+    }
+    int32_t lookup(const CacheKey &k) const {
+        auto range = index.equal_range(key_hash(k));
+        for (auto it = range.first; it != range.second; ++it)
+            if (keys[it->second] == k) return it->second;
+        return -1;
+    }
+    void insert(int32_t b, CacheKey k) {
+        index.emplace(key_hash(k), b);
+        keys[b] = std::move(k);
+        cached[b] = 1;
     }
     static int64_t blocks_for(int64_t tokens, int32_t bs) { return (tokens + bs - 1) / bs; }
 };
@@ -53,6 +142,11 @@ pa_status pa_bm_create(int32_t num_blocks, int32_t block_size, const int32_t *fr
     bm->num_blocks = num_blocks;
     bm->block_size = block_size;
     bm->refs.assign(num_blocks, 0);
+    bm->gen.assign(num_blocks, 0);
+    bm->cached.assign(num_blocks, 0);
+    bm->keys.resize(num_blocks);
+    bm->evict_pos.resize(num_blocks);
+    bm->on_evictable.assign(num_blocks, 0);
     bm->free_stack.resize(num_blocks);
     if (free_order) {
         std::vector<char> seen(num_blocks, 0);
@@ -81,6 +175,49 @@ pa_status pa_bm_add_seq(pa_block_manager *bm, int64_t seq_id) {
     return PA_OK;
 }
 
+pa_status pa_bm_add_seq_tokens(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens, int32_t n,
+                               int64_t *slots_out, int32_t *num_cached_out) {
+    if (!bm || n < 0 || (n > 0 && !tokens)) return PA_ERR_INVALID_ARG;
+    if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+    const int32_t bs = bm->block_size;
+    // Plan: the longest run of leading full blocks already cached.
+    std::vector<int32_t> hits;
+    int32_t parent = -1;
+    uint32_t pgen = 0;
+    int32_t hits_evictable = 0;
+    for (int64_t j = 0; j < n / bs; ++j) {
+        CacheKey k{parent, pgen, std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)};
+        const int32_t b = bm->lookup(k);
+        if (b < 0) break;
+        hits.push_back(b);
+        hits_evictable += bm->on_evictable[b] ? 1 : 0;
+        parent = b;
+        pgen = bm->gen[b];
+    }
+    const int64_t need = pa_block_manager::blocks_for(n, bs) - (int64_t)hits.size();
+    if (need > (int64_t)bm->available() - hits_evictable) return PA_ERR_OOM;
+    // Commit: reuse the hits, allocate the rest, index each new full block.
+    for (int32_t b : hits) bm->revive(b);
+    Sequence sq;
+    sq.blocks = hits;
+    int64_t k_out = 0;
+    for (int64_t i = (int64_t)hits.size() * bs; i < n; ++i) {
+        const int64_t offset = i % bs;
+        if (offset == 0) sq.blocks.push_back(bm->take());
+        if (slots_out) slots_out[k_out++] = (int64_t)sq.blocks.back() * bs + offset;
+        if (offset == bs - 1) {
+            const int64_t j = i / bs;
+            const int32_t par = j > 0 ? sq.blocks[j - 1] : -1;
+            bm->insert(sq.blocks[j], CacheKey{par, par >= 0 ? bm->gen[par] : 0u,
+                                              std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)});
+        }
+    }
+    sq.tokens = n;
+    bm->seqs.emplace(seq_id, std::move(sq));
+    if (num_cached_out) *num_cached_out = (int32_t)hits.size() * bs;
+    return PA_OK;
+}
+
 pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, int64_t *slots_out,
                              int32_t *cow_pairs_out, int32_t cow_capacity, int32_t *num_cow_out) {
     if (!bm || n < 0) return PA_ERR_INVALID_ARG;
@@ -93,7 +230,7 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, in
     const bool cow = n > 0 && (sq.tokens % bs) != 0 && bm->refs[sq.blocks.back()] > 1;
     const int64_t fresh =
         pa_block_manager::blocks_for(sq.tokens + n, bs) - pa_block_manager::blocks_for(sq.tokens, bs);
-    if (fresh + (cow ? 1 : 0) > (int64_t)bm->free_stack.size()) return PA_ERR_OOM;
+    if (fresh + (cow ? 1 : 0) > (int64_t)bm->available()) return PA_ERR_OOM;
     if (cow && cow_pairs_out && cow_capacity < 1) return PA_ERR_INVALID_ARG;
     int32_t ncow = 0;
     for (int32_t i = 0; i < n; ++i) {
@@ -108,7 +245,7 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, in
                 cow_pairs_out[2 * ncow + 1] = new_block;
             }
             ++ncow;
-            bm->release(old_block);
+            if (bm->release(old_block)) bm->make_evictable(old_block);
             sq.blocks.back() = new_block;
         }
         if (slots_out) slots_out[i] = (int64_t)sq.blocks.back() * bs + offset;
@@ -133,7 +270,12 @@ pa_status pa_bm_free_seq(pa_block_manager *bm, int64_t seq_id) {
     if (!bm) return PA_ERR_INVALID_ARG;
     auto it = bm->seqs.find(seq_id);
     if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
-    for (int32_t b : it->second.blocks) bm->release(b);
+    // references drop in logical order; cached blocks reaching zero become
+    // evictable from the last to the first, so a prefix's tail goes before its head
+    std::vector<int32_t> to_evictable;
+    for (int32_t b : it->second.blocks)
+        if (bm->release(b)) to_evictable.push_back(b);
+    for (auto r = to_evictable.rbegin(); r != to_evictable.rend(); ++r) bm->make_evictable(*r);
     bm->seqs.erase(it);
     return PA_OK;
 }
@@ -192,6 +334,22 @@ int32_t pa_bm_num_free(const pa_block_manager *bm) {
 }
 
 int32_t pa_bm_num_blocks(const pa_block_manager *bm) { return bm ? bm->num_blocks : -1; }
+
+int32_t pa_bm_num_evictable(const pa_block_manager *bm) {
+    return bm ? (int32_t)bm->evictable.size() : -1;
+}
+
+int32_t pa_bm_num_cached(const pa_block_manager *bm) { return bm ? (int32_t)bm->index.size() : -1; }
+
+int32_t pa_bm_evictable(const pa_block_manager *bm, int32_t *out, int32_t capacity) {
+    if (!bm) return -1;
+    int32_t k = 0;
+    for (int32_t b : bm->evictable) {
+        if (out && k < capacity) out[k] = b;
+        ++k;
+    }
+    return k;
+}
 
 int32_t pa_bm_free_stack(const pa_block_manager *bm, int32_t *out, int32_t capacity) {
     if (!bm) return -1;

@@ -302,3 +302,86 @@ def test_append_decode_matches_two_calls_bitwise():
     b.append_step(step)
     ref = b.gpu_decode(step, 256)
     assert got.tobytes() == ref.tobytes()
+
+
+def test_prefix_cached_prompts_decode_as_if_written_in_full():
+    """Automatic prefix caching on the hot path: prompts sharing a system prompt are
+    created from their token ids, only the tokens not found in the cache get their K/V
+    written, and decode through the shared blocks matches (a) the oracle over the same
+    pool and (b) a dense reference over each prompt's own K/V.  A token's K/V depend only
+    on the prompt up to it, as a model's would."""
+    import zlib
+    import oracle
+    from oracle.block_model import BlockManagerModel
+    from paged_kv_cache_389_b200.cache import PagedKVCache
+    torch = torch_mod()
+    import paged_kv_cache_389_b200 as pa
+    rng = np.random.default_rng(31)
+    hq, hkv, d, nb = 32, 8, 128, 96
+    scale = 1.0 / np.sqrt(d)
+
+    def kv_of(prompt, p):
+        g = np.random.default_rng(zlib.crc32(np.asarray(prompt[:p + 1], np.int32).tobytes()))
+        return workloads.normal(g, (2, hkv, d), "bf16")
+
+    system = rng.integers(0, 1000, size=80).tolist()            # five full blocks
+    prompts = [system + rng.integers(0, 1000, size=int(n)).tolist() for n in (3, 17, 40, 0, 25)]
+    prompts += [system[:48] + rng.integers(0, 1000, size=9).tolist()]   # shares three blocks
+    free_order = rng.permutation(nb).astype(np.int32)
+    gpu = PagedKVCache(nb, hkv, d, torch.bfloat16, "cuda", free_order)
+    model = BlockManagerModel(nb, 16, free_order.tolist())
+    kc = np.full((nb, hkv, 16, d), 0x7FC0, np.uint16)           # NaN-filled like the GPU pools
+    vc = kc.copy()
+    cached = []
+    order = list(range(len(prompts)))
+    for i in order:
+        n_g, slots_g = gpu.manager.add_seq_tokens(i, prompts[i])
+        n_m, slots_m = model.add_seq_tokens(i, prompts[i])
+        assert n_g == n_m and slots_g.tolist() == list(slots_m)
+        cached.append(n_m)
+        new = [kv_of(prompts[i], p) for p in range(n_m, len(prompts[i]))]
+        if new:
+            k = np.stack([x[0] for x in new])
+            v = np.stack([x[1] for x in new])
+            sl = np.asarray(slots_m, np.int64)
+            oracle.cache_write(k, v, sl, kc, vc)
+            pa.pa_cache_write(to_dev(k), to_dev(v), torch.from_numpy(sl).cuda(), gpu.key_cache,
+                              gpu.value_cache, gpu.err_flag)
+        if i == 2:                                               # free one prompt midway
+            gpu.manager.free(1)
+            model.free(1)
+    assert cached[1:] == [80, 80, 80, 80, 48] and cached[0] == 0
+    live = [i for i in order if i != 1]
+    assert to_host(gpu.key_cache).tobytes() == kc.tobytes()
+    t, l = model.build_tables(live, max(len(model.block_table(i)) for i in live))
+    q = workloads.normal(rng, (len(live), hq, d), "bf16")
+    ref = oracle.decode(q, kc, vc, t, l, scale)
+    # dense reference over each prompt's own K/V
+    g = hq // hkv
+    for row, i in enumerate(live):
+        kv = np.stack([kv_of(prompts[i], p) for p in range(len(prompts[i]))])   # [L, 2, hkv, d]
+        K = workloads.bf16_bits_to_f32(kv[:, 0]).astype(np.float64)
+        V = workloads.bf16_bits_to_f32(kv[:, 1]).astype(np.float64)
+        Q = workloads.bf16_bits_to_f32(q[row]).astype(np.float64)
+        for h in range(hq):
+            sc = K[:, h // g] @ Q[h] * scale
+            w = np.exp(sc - sc.max())
+            dense = (w[:, None] * V[:, h // g]).sum(0) / w.sum()
+            assert np.allclose(ref[row, h], dense, rtol=1e-9, atol=1e-9)
+    for part in (0, 32):
+        got = ts_free_decode(pa, torch, q, gpu, t, l, scale, part)
+        check_close(got, ref, "bf16", f"prefix-cached decode partition {part}")
+    assert pa.pa_wait(gpu.err_flag) == 0
+
+
+def ts_free_decode(pa, torch, q_np, gpu, t, l, scale, part):
+    q = to_dev(q_np)
+    out = torch.empty_like(q)
+    maxc = int(l.max())
+    ws = None
+    if part:
+        n = pa.pa_decode_workspace_size(q.shape[0], q.shape[1], q.shape[2], maxc, part)
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    pa.pa_decode(q, gpu.key_cache, gpu.value_cache, torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(),
+                 maxc, scale, out, part, ws, gpu.err_flag)
+    return to_host(out)
