@@ -39,6 +39,13 @@ def _load():
         lib.oracle_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i64]
         for f in ("oracle_decode", "oracle_prefill", "oracle_cache_write", "oracle_copy_blocks"):
             getattr(lib, f).restype = C.c_int
+        lib.oracle_e4m3_encode.argtypes = [vp, i64, C.c_float, vp]
+        lib.oracle_e4m3_decode.argtypes = [vp, i64, vp]
+        lib.oracle_cache_write_fp8.argtypes = [vp, vp, vp, i32, vp, vp, i32, i32, i32, i32, C.c_float, C.c_float]
+        lib.oracle_cache_write_fp8.restype = C.c_int
+        lib.oracle_decode_fp8.argtypes = [vp, vp, vp, i32, i32, i32, i32, vp, i32, vp, i32, i32, dbl, dbl,
+                                          dbl, vp]
+        lib.oracle_decode_fp8.restype = C.c_int
         lib.oracle_num_threads.restype = C.c_int
         lib.oracle_set_num_threads.argtypes = [C.c_int]
         _lib = lib
@@ -135,3 +142,50 @@ def copy_blocks(k_cache, v_cache, pairs):
 
 def lib_path() -> str:
     return os.path.abspath(_build.LIB)
+
+
+# ---- FP8 (e4m3) KV cache -----------------------------------------------------
+def e4m3_encode(x, scale=1.0):
+    """uint8 e4m3 codes of float32(x) / float32(scale): nearest, ties to even,
+    saturated to +-448, NaN -> 0x7F."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _load().oracle_e4m3_encode(_ptr(x), x.size, float(np.float32(scale)), _ptr(out))
+    return out
+
+
+def e4m3_decode(codes):
+    """Exact float64 values of uint8 e4m3 codes."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    out = np.empty(c.shape, np.float64)
+    _load().oracle_e4m3_decode(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def cache_write_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale):
+    """Append bf16 K/V [T, Hkv, d] into uint8 e4m3 pools [NB, Hkv, 16, d]."""
+    assert k.dtype == v.dtype == np.uint16 and k_cache.dtype == v_cache.dtype == np.uint8
+    nb, nkv, bs, d = k_cache.shape
+    sl = np.ascontiguousarray(slot_mapping, dtype=np.int64)
+    st = _load().oracle_cache_write_fp8(_ptr(np.ascontiguousarray(k)), _ptr(np.ascontiguousarray(v)), _ptr(sl),
+                                        len(sl), _ptr(k_cache), _ptr(v_cache), nb, nkv, bs, d,
+                                        float(np.float32(k_scale)), float(np.float32(v_scale)))
+    if st != 0:
+        raise IndexError("slot beyond the pool")
+
+
+def decode_fp8(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale, v_scale):
+    """Decode attention over e4m3 pools: bf16 q [S, Hq, d] -> float64 [S, Hq, d]."""
+    assert q.dtype == np.uint16 and k_cache.dtype == np.uint8
+    nb, nkv, bs, d = k_cache.shape
+    S, hq, _ = q.shape
+    t = np.ascontiguousarray(block_tables, dtype=np.int32)
+    l = np.ascontiguousarray(context_lens, dtype=np.int32)
+    out = np.zeros((S, hq, d), np.float64)
+    st = _load().oracle_decode_fp8(_ptr(np.ascontiguousarray(q)), _ptr(k_cache), _ptr(v_cache), nb, nkv, bs, d,
+                                   _ptr(t), t.shape[1], _ptr(l), S, hq, float(scale),
+                                   float(np.float32(k_scale)), float(np.float32(v_scale)), _ptr(out))
+    if st != 0:
+        raise ValueError(f"oracle_decode_fp8 failed ({st})")
+    return out
+

@@ -20,6 +20,8 @@
  *        block looked up through the table; score scaled by `scale`; softmax and
  *        a V-weighted sum "as in standard attention"), section "关键设计二"
  *        (Copy-on-Write copies a whole block from the shared one to a new one).
+ *   [P1] 5.3 and the [P3] architecture figure -- an FP8 KV cache; the e4m3
+ *        reading and its scale convention are stated above e4m3_value() below.
  *
  * Arithmetic: every element is widened exactly to double (bf16 is the upper half
  * of an IEEE binary32, so widening is exact) and all sums, the max, exp and the
@@ -38,12 +40,61 @@
 
 #define ORACLE_F32 0
 #define ORACLE_BF16 1
+#define ORACLE_FP8 2   /* e4m3 code; widen() gives its value, unscaled */
+
+/*
+ * FP8 KV cache.  The pages name FP8 without a format (chenxutan 5.3: FP8 is nearly
+ * lossless and cuts memory and bandwidth; the devpress teardown's architecture
+ * figure lists FP8/INT8 quantisation in the kernel layer).  Reading taken: the
+ * E4M3 format of the OCP 8-bit floating point specification with one scale per
+ * tensor -- sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent 0 holds
+ * the subnormals m * 2^-9; no infinities; S.1111.111 is NaN, so the largest
+ * finite value is S.1111.110 = 448.
+ */
+static double e4m3_value(uint8_t c)
+{
+    const int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    const double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return sgn ? -v : v;
+}
+
+/* Nearest e4m3 code to x, ties to even mantissa, magnitudes beyond the largest
+ * finite value (and infinities) saturated to +-448, NaN to 0x7F. */
+static uint8_t e4m3_encode(float x)
+{
+    if (isnan(x))
+        return 0x7F;
+    const uint8_t sgn = signbit(x) ? 0x80 : 0x00;
+    const double a = fabs((double)x);
+    if (a >= 448.0)
+        return sgn | 0x7E;
+    if (a < ldexp(1.0, -6)) {                 /* subnormal range: a multiple of 2^-9 */
+        const double m = nearbyint(a * 512.0); /* round to nearest, ties to even; 8 -> 2^-6 */
+        return sgn | (uint8_t)m;
+    }
+    int e2;
+    const double f = frexp(a, &e2);            /* a = f * 2^e2, f in [0.5, 1) */
+    int ex = e2 - 1;                           /* a = (1 + frac) * 2^ex */
+    double mq = nearbyint((2.0 * f - 1.0) * 8.0);
+    if (mq == 8.0) {
+        ex += 1;
+        mq = 0.0;
+    }
+    const int biased = ex + 7;
+    if (biased > 15 || (biased == 15 && mq == 7.0))
+        return sgn | 0x7E;
+    return sgn | (uint8_t)((biased << 3) | (int)mq);
+}
 
 /* Exact widening of one stored element to double. */
 static double widen(const void *base, int64_t idx, int dtype)
 {
     if (dtype == ORACLE_F32)
         return (double)((const float *)base)[idx];
+    if (dtype == ORACLE_FP8)
+        return e4m3_value(((const uint8_t *)base)[idx]);
     uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 16;
     float f;
     memcpy(&f, &bits, sizeof f);
@@ -303,3 +354,105 @@ void oracle_set_num_threads(int n)
     (void)n;
 #endif
 }
+
+/* out[i] = the e4m3 code of the binary32 quotient x[i] / scale (fp32 division). */
+void oracle_e4m3_encode(const float *x, int64_t n, float scale, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const float t = x[i] / scale;
+        out[i] = e4m3_encode(t);
+    }
+}
+
+/* out[i] = exact value of code c[i]. */
+void oracle_e4m3_decode(const uint8_t *c, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = e4m3_value(c[i]);
+}
+
+/*
+ * KV append into FP8 pools: key/value [num_tokens, num_kv_heads, head_dim] bf16;
+ * each element x is stored as the e4m3 code of fl32(x) / k_scale (v_scale for V)
+ * in pools of one byte per element, laid out as for oracle_cache_write.
+ * Returns 0, or -1 if a slot is beyond the pool (nothing after it is written).
+ */
+int oracle_cache_write_fp8(const void *key, const void *value, const int64_t *slot_mapping,
+                           int32_t num_tokens, uint8_t *key_cache, uint8_t *value_cache,
+                           int32_t num_blocks, int32_t num_kv_heads, int32_t block_size,
+                           int32_t head_dim, float k_scale, float v_scale)
+{
+    for (int32_t i = 0; i < num_tokens; ++i) {
+        const int64_t slot = slot_mapping[i];
+        if (slot < 0)
+            continue;
+        if (slot >= (int64_t)num_blocks * block_size)
+            return -1;
+        const int64_t blk = slot / block_size, off = slot % block_size;
+        for (int32_t h = 0; h < num_kv_heads; ++h) {
+            const int64_t dst = pool_offset(blk, h, off, num_kv_heads, block_size, head_dim);
+            const int64_t src = ((int64_t)i * num_kv_heads + h) * head_dim;
+            for (int32_t k = 0; k < head_dim; ++k) {
+                const float kx = (float)widen(key, src + k, ORACLE_BF16);
+                const float vx = (float)widen(value, src + k, ORACLE_BF16);
+                key_cache[dst + k] = e4m3_encode(kx / k_scale);
+                value_cache[dst + k] = e4m3_encode(vx / v_scale);
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * Decode attention over FP8 pools: as oracle_decode with bf16 queries, each
+ * cached key element taken as its code's value times k_scale and each value
+ * element times v_scale (products exact in double).
+ */
+int oracle_decode_fp8(const void *query, const uint8_t *key_cache, const uint8_t *value_cache,
+                      int32_t num_blocks, int32_t num_kv_heads, int32_t block_size, int32_t head_dim,
+                      const int32_t *block_tables, int32_t max_blocks_per_seq,
+                      const int32_t *context_lens, int32_t num_seqs, int32_t num_q_heads, double scale,
+                      double k_scale, double v_scale, double *out)
+{
+    const int64_t d = head_dim, nkv = num_kv_heads, bs = block_size;
+    const int64_t group = num_q_heads / num_kv_heads;
+    for (int32_t s = 0; s < num_seqs; ++s)
+        if (context_lens[s] < 0 || context_lens[s] > (int64_t)max_blocks_per_seq * bs)
+            return -2;
+    int status = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int32_t s = 0; s < num_seqs; ++s) {
+        for (int32_t h = 0; h < num_q_heads; ++h) {
+            const int64_t len = context_lens[s];
+            double *kd = malloc(sizeof(double) * (size_t)(len * d + 1));
+            double *vd = malloc(sizeof(double) * (size_t)(len * d + 1));
+            double *x = malloc(sizeof(double) * (size_t)(len + 1));
+            double *qd = malloc(sizeof(double) * (size_t)d);
+            if (!kd || !vd || !x || !qd) {
+#pragma omp atomic write
+                status = -3;
+            } else {
+                const int32_t *table = block_tables + (int64_t)s * max_blocks_per_seq;
+                if (gather_kv(key_cache, value_cache, ORACLE_FP8, num_blocks, nkv, bs, d, table, len,
+                              h / group, kd, vd) != 0) {
+#pragma omp atomic write
+                    status = -1;
+                } else {
+                    for (int64_t i = 0; i < len * d; ++i) {
+                        kd[i] *= k_scale;
+                        vd[i] *= v_scale;
+                    }
+                    for (int64_t i = 0; i < d; ++i)
+                        qd[i] = widen(query, ((int64_t)s * num_q_heads + h) * d + i, ORACLE_BF16);
+                    attend(qd, kd, vd, len, d, scale, x, out + ((int64_t)s * num_q_heads + h) * d);
+                }
+            }
+            free(kd);
+            free(vd);
+            free(x);
+            free(qd);
+        }
+    }
+    return status;
+}
+
