@@ -25,6 +25,14 @@
  * Query head h reads kv head h / (num_q_heads / num_kv_heads).
  * Supported: dtype PA_F32 or PA_BF16 (cache, query, key/value and out share it),
  * head_dim 64 or 128, block_size 16, num_q_heads / num_kv_heads in {1,2,4,8}.
+ * FP8 KV cache (chenxutan 5.3: FP8 KV is close to lossless and halves the bytes;
+ * the devpress teardown's architecture figure puts FP8/INT8 quantisation in the
+ * kernel layer): dtype PA_FP8_E4M3 stores the pools as one-byte e4m3 codes (OCP
+ * 8-bit floating point: bias 7, largest finite 448, S.1111.111 NaN) with one
+ * float scale per pool, code = e4m3(fp32(x) / scale) rounded to nearest even and
+ * saturated to +-448, value = e4m3 * scale.  key/value inputs, query and out are
+ * then bf16.  pa_cache_write, pa_copy_blocks, pa_decode and pa_append_decode take
+ * it with head_dim 128; pa_prefill_chunk returns PA_ERR_UNSUPPORTED.
  *
  * Conventions:
  *   - Ownership: the caller owns every buffer, the decode workspace included.
@@ -70,7 +78,7 @@ typedef enum pa_status {
     PA_ERR_NOT_FOUND = 7      /* unknown sequence id (host block manager) */
 } pa_status;
 
-typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1 } pa_dtype;
+typedef enum pa_dtype { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
 
 /* Bits a kernel ORs into *err_flag. */
 #define PA_DEVERR_BLOCK_ID 1     /* block table entry outside [0, num_blocks) */
@@ -87,6 +95,8 @@ typedef struct pa_cache_desc {
     int32_t block_size;   /* must be 16 */
     int32_t head_dim;     /* 64 or 128 */
     int32_t dtype;        /* pa_dtype */
+    float k_scale;        /* PA_FP8_E4M3: dequantisation scale of the key pool (finite, > 0) */
+    float v_scale;        /* PA_FP8_E4M3: the same for the value pool; both ignored otherwise */
 } pa_cache_desc;
 
 /* Version of this ABI (bumped on any signature or layout change). */
@@ -103,6 +113,8 @@ PA_API const char *pa_status_string(pa_status status);
  * slot < 0 is padding (skipped).  slot >= num_blocks * block_size sets
  * PA_DEVERR_SLOT and that token is skipped.  Two tokens with the same slot:
  * unspecified which one lands.  num_tokens == 0 launches nothing.
+ * PA_FP8_E4M3 pools: key/value are bf16 and each element is stored as
+ * e4m3(fp32(x) / k_scale) (v_scale for value), nearest even, saturated.
  * Source: chenxutan 3.1 (write the new token's K/V back into the cache) and 3.3
  * (append_slot: the token goes into the current block).
  */

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libpa_b200.so")
 
 PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_OOM = 0, 1, 2, 3
 PA_ERR_DEVICE_INDEX, PA_ERR_CUDA, PA_ERR_TIMEOUT, PA_ERR_NOT_FOUND = 4, 5, 6, 7
-PA_F32, PA_BF16 = 0, 1
+PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 PA_DEVERR_BLOCK_ID, PA_DEVERR_SLOT, PA_DEVERR_CONTEXT_LEN = 1, 2, 4
 PA_DEVERR_PAIR, PA_DEVERR_TIMEOUT, PA_DEVERR_CHUNK = 8, 16, 32
 BLOCK_SIZE = 16
@@ -32,7 +32,8 @@ class PAError(RuntimeError):
 
 class CacheDesc(C.Structure):
     _fields_ = [("num_blocks", C.c_int32), ("num_kv_heads", C.c_int32), ("block_size", C.c_int32),
-                ("head_dim", C.c_int32), ("dtype", C.c_int32)]
+                ("head_dim", C.c_int32), ("dtype", C.c_int32), ("k_scale", C.c_float),
+                ("v_scale", C.c_float)]
 
 
 def _load():
@@ -116,13 +117,22 @@ def _dtype_code(t) -> int:
         return PA_BF16
     if t.dtype == torch.float32:
         return PA_F32
+    if t.dtype == torch.float8_e4m3fn:
+        return PA_FP8_E4M3
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def cache_desc(key_cache) -> CacheDesc:
-    """Descriptor of a pool tensor [num_blocks, num_kv_heads, block_size, head_dim]."""
+def io_dtype(key_cache):
+    """dtype of queries, outputs and appended K/V for a pool: bf16 for an fp8 pool."""
+    torch = _torch()
+    return torch.bfloat16 if key_cache.dtype == torch.float8_e4m3fn else key_cache.dtype
+
+
+def cache_desc(key_cache, k_scale=1.0, v_scale=1.0) -> CacheDesc:
+    """Descriptor of a pool tensor [num_blocks, num_kv_heads, block_size, head_dim]; the
+    scales matter for torch.float8_e4m3fn pools only."""
     nb, hkv, bs, d = key_cache.shape
-    return CacheDesc(nb, hkv, bs, d, _dtype_code(key_cache))
+    return CacheDesc(nb, hkv, bs, d, _dtype_code(key_cache), float(k_scale), float(v_scale))
 
 
 def _ptr(t):
@@ -143,14 +153,16 @@ def _same_pool(key_cache, value_cache):
     assert key_cache.is_cuda and value_cache.is_cuda
 
 
-def pa_cache_write(key, value, slot_mapping, key_cache, value_cache, err_flag=None, stream=None):
-    """Scatter key/value [T, Hkv, d] into the pools at slot_mapping (int64 [T])."""
+def pa_cache_write(key, value, slot_mapping, key_cache, value_cache, err_flag=None, stream=None,
+                   k_scale=1.0, v_scale=1.0):
+    """Scatter key/value [T, Hkv, d] into the pools at slot_mapping (int64 [T]); fp8 pools
+    store e4m3(x / k_scale) and e4m3(x / v_scale)."""
     torch = _torch()
     _same_pool(key_cache, value_cache)
     assert key.shape == value.shape and key.dim() == 3 and key.shape[1:] == (key_cache.shape[1], key_cache.shape[3])
-    assert key.dtype == key_cache.dtype == value.dtype and slot_mapping.dtype == torch.int64
+    assert key.dtype == io_dtype(key_cache) == value.dtype and slot_mapping.dtype == torch.int64
     assert slot_mapping.shape == (key.shape[0],)
-    d = cache_desc(key_cache)
+    d = cache_desc(key_cache, k_scale, v_scale)
     _check(_lib.pa_cache_write(_ptr(key), _ptr(value), _ptr(slot_mapping), key.shape[0],
                                _ptr(key_cache), _ptr(value_cache), C.byref(d), _ptr(err_flag),
                                _stream(stream)), "pa_cache_write")
@@ -162,6 +174,8 @@ def pa_copy_blocks(key_cache, value_cache, src_dst_pairs, err_flag=None, stream=
     _same_pool(key_cache, value_cache)
     assert src_dst_pairs.dtype == torch.int32 and src_dst_pairs.dim() == 2 and src_dst_pairs.shape[1] == 2
     d = cache_desc(key_cache)
+    if d.dtype == PA_FP8_E4M3:
+        d.k_scale = d.v_scale = 1.0       # a byte copy: the scales are not used
     _check(_lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(src_dst_pairs),
                                src_dst_pairs.shape[0], C.byref(d), _ptr(err_flag), _stream(stream)),
            "pa_copy_blocks")
@@ -173,20 +187,20 @@ def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, p
 
 
 def pa_decode_launches(num_seqs, head_dim, dtype, partition_size) -> int:
-    """Kernels one pa_decode call launches; dtype PA_F32 / PA_BF16."""
+    """Kernels one pa_decode call launches; dtype PA_F32 / PA_BF16 / PA_FP8_E4M3."""
     return int(_lib.pa_decode_launches(num_seqs, head_dim, dtype, partition_size))
 
 
 def pa_decode(query, key_cache, value_cache, block_tables, context_lens, max_context_len, scale,
-              out, partition_size=0, workspace=None, err_flag=None, stream=None):
+              out, partition_size=0, workspace=None, err_flag=None, stream=None, k_scale=1.0, v_scale=1.0):
     """Decode attention; query/out [S, Hq, d]; tables int32 [S, max_blocks]; lens int32 [S]."""
     torch = _torch()
     _same_pool(key_cache, value_cache)
     S, hq, dd = query.shape
-    assert out.shape == query.shape and out.dtype == query.dtype == key_cache.dtype
+    assert out.shape == query.shape and out.dtype == query.dtype == io_dtype(key_cache)
     assert block_tables.dtype == torch.int32 and block_tables.dim() == 2 and block_tables.shape[0] == S
     assert context_lens.dtype == torch.int32 and context_lens.shape == (S,)
-    d = cache_desc(key_cache)
+    d = cache_desc(key_cache, k_scale, v_scale)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.pa_decode(_ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
                           block_tables.shape[1], _ptr(context_lens), int(max_context_len), S, hq,
@@ -196,18 +210,18 @@ def pa_decode(query, key_cache, value_cache, block_tables, context_lens, max_con
 
 def pa_append_decode(key, value, slot_mapping, query, key_cache, value_cache, block_tables, context_lens,
                      max_context_len, scale, out, partition_size=0, workspace=None, err_flag=None,
-                     stream=None):
+                     stream=None, k_scale=1.0, v_scale=1.0):
     """pa_cache_write(key, value, slot_mapping, ...) then pa_decode(...) in one call."""
     torch = _torch()
     _same_pool(key_cache, value_cache)
     assert key.shape == value.shape and key.dim() == 3 and key.shape[1:] == (key_cache.shape[1], key_cache.shape[3])
-    assert key.dtype == key_cache.dtype == value.dtype and slot_mapping.dtype == torch.int64
+    assert key.dtype == io_dtype(key_cache) == value.dtype and slot_mapping.dtype == torch.int64
     assert slot_mapping.shape == (key.shape[0],)
     S, hq, dd = query.shape
-    assert out.shape == query.shape and out.dtype == query.dtype == key_cache.dtype
+    assert out.shape == query.shape and out.dtype == query.dtype == io_dtype(key_cache)
     assert block_tables.dtype == torch.int32 and block_tables.dim() == 2 and block_tables.shape[0] == S
     assert context_lens.dtype == torch.int32 and context_lens.shape == (S,)
-    d = cache_desc(key_cache)
+    d = cache_desc(key_cache, k_scale, v_scale)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.pa_append_decode(_ptr(key), _ptr(value), _ptr(slot_mapping), key.shape[0], _ptr(query),
                                  _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), block_tables.shape[1],

@@ -23,15 +23,23 @@ def _torch():
 
 class PagedKVCache:
     def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, dtype, device="cuda",
-                 free_order=None, fill_nan: bool = True):
+                 free_order=None, fill_nan: bool = True, k_scale: float = 1.0, v_scale: float = 1.0):
+        """dtype torch.float32, torch.bfloat16 or torch.float8_e4m3fn; an fp8 pool stores
+        e4m3(x / k_scale) and e4m3(x / v_scale) and takes bf16 queries and K/V."""
         torch = _torch()
         self.num_blocks, self.num_kv_heads, self.head_dim = num_blocks, num_kv_heads, head_dim
         self.dtype, self.device = dtype, torch.device(device)
+        self.k_scale, self.v_scale = float(k_scale), float(v_scale)
         shape = (num_blocks, num_kv_heads, BLOCK_SIZE, head_dim)
-        fill = float("nan") if fill_nan else 0.0
         # NaN in every slot nothing has written: a stray read poisons the output
-        self.key_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
-        self.value_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
+        if dtype == torch.float8_e4m3fn:
+            code = 0x7F if fill_nan else 0x00          # e4m3 NaN / +0
+            self.key_cache = torch.full(shape, code, dtype=torch.uint8, device=self.device).view(dtype)
+            self.value_cache = torch.full(shape, code, dtype=torch.uint8, device=self.device).view(dtype)
+        else:
+            fill = float("nan") if fill_nan else 0.0
+            self.key_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
+            self.value_cache = torch.full(shape, fill, dtype=dtype, device=self.device)
         self.manager = BlockManager(num_blocks, BLOCK_SIZE, free_order)
         self.err_flag = torch.zeros(1, dtype=torch.int32, device=self.device)
 
@@ -67,7 +75,7 @@ class PagedKVCache:
                            self.err_flag, stream)
         if len(slots):
             pa_cache_write(k, v, torch.as_tensor(slots, device=self.device), self.key_cache,
-                           self.value_cache, self.err_flag, stream)
+                           self.value_cache, self.err_flag, stream, self.k_scale, self.v_scale)
 
     def append(self, seqs, k, v, counts=None, stream=None):
         slots, pairs = self.plan_append(seqs, counts)
@@ -92,7 +100,7 @@ class PagedKVCache:
             ws = pa_decode_workspace_size(len(seqs), q.shape[1], q.shape[2], max_len, partition_size)
             workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=self.device)
         pa_decode(q, self.key_cache, self.value_cache, tables, lens, max_len, scale, out,
-                  partition_size, workspace, self.err_flag, stream)
+                  partition_size, workspace, self.err_flag, stream, self.k_scale, self.v_scale)
         return out
 
     def prefill(self, q, seqs, chunk_lens, scale, out=None, max_blocks=None, stream=None):

@@ -34,6 +34,12 @@
 //    16-byte chunks so the ldmatrix reads are bank-conflict free.  A CUDA-core
 //    version of this path (packed fp32 FMAs, shuffle reductions) measured issue
 //    bound: 63 warp instructions per (token, kv head) against ~6 here.
+//  * fp8 (e4m3 codes, head_dim 128): the slabs are 2 KB, half of bf16.  Each
+//    thread reads whole 16-byte chunks of them and turns the codes into f16
+//    (exact: e4m3 is a subset of f16) right before f16 tensor-core tiles; the
+//    query goes to f16 once per unit.  k_scale is folded into the softmax scale,
+//    v_scale into the merge.  Four stages per warp keep as many bytes in flight
+//    as bf16's two.
 //  * fp32: CUDA-core path (tensor cores would round fp32 inputs to tf32): 8 lanes
 //    per token for QK with a transposing shuffle reduction, packed FFMA2 for QK
 //    and PV.
@@ -45,6 +51,9 @@
 #include <cfloat>
 #include <climits>
 #include <cstring>
+#include <type_traits>
+
+#include <cuda_fp8.h>
 
 #include "pa_common.cuh"
 #include "pa_launch.h"
@@ -68,6 +77,19 @@ template <>
 struct ElemBytes<__nv_bfloat16> {
     static constexpr int value = 2;
 };
+// One e4m3 code of an FP8 pool (queries and outputs are bf16 then).
+struct e4m3_t {
+    unsigned char bits;
+};
+template <>
+struct ElemBytes<e4m3_t> {
+    static constexpr int value = 1;
+};
+template <typename T>
+constexpr bool kIsFp8 = std::is_same<T, e4m3_t>::value;
+// element type of queries and outputs
+template <typename T>
+using IoT = typename std::conditional<kIsFp8<T>, __nv_bfloat16, T>::type;
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -80,6 +102,7 @@ template <typename T, int D, int G>
 struct Layout {
     static constexpr int kElem = ElemBytes<T>::value;
     static constexpr int kRowBytes = D * kElem;                 // one token of one head
+    static constexpr int kQRowBytes = D * (int)sizeof(IoT<T>);  // one query head
     static constexpr int kSlabBytes = kBlockSize * kRowBytes;   // one (block, kv head) slab
     static constexpr int kStageBytes = 2 * kSlabBytes;          // K slab + V slab
     static constexpr size_t kLimit = 232448;                    // sm_100 max dynamic smem per CTA
@@ -89,7 +112,8 @@ struct Layout {
     static constexpr int stages_fit(int bufs) {
         return (int)((kLimit - kFixed - bufs * kMergeBytes) / ((size_t)kWarps * kStageBytes));
     }
-    static constexpr int kStagesPerWarp = stages_fit(2) >= 2 ? 2 : 1;
+    static constexpr int kWantStages = kIsFp8<T> ? 4 : 2;
+    static constexpr int kStagesPerWarp = stages_fit(2) >= kWantStages ? kWantStages : (stages_fit(2) >= 2 ? 2 : 1);
     static constexpr int kMergeBufs = stages_fit(2) >= kStagesPerWarp ? 2 : 1;
     static constexpr size_t kPWarpFloats = 16 * G + G;          // fp32 path: p[16][G], alpha[G]
     static constexpr size_t kOffRing = 0;
@@ -128,6 +152,7 @@ struct Params {
     const int32_t *meta;    // [0] groups, [1] group units
     int32_t max_members;    // sequences per group: query rows members x g <= 128
     int32_t wait_first;     // launched right behind a cache write: wait for it first
+    float v_scale;          // fp8 pools: value dequantisation scale (1 otherwise)
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -259,7 +284,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
 }
 
 // Issue the cp.async copies of one (block, kv head) slab pair into a stage.
-// bf16 rows are 2*D bytes; chunk c of row r goes to chunk position
+// bf16 rows are 2*D bytes (fp8: D); chunk c of row r goes to chunk position
 // (c & ~7) | ((c ^ r) & 7), which keeps 8 consecutive rows of any column in 8
 // different bank groups.  fp32 rows keep their natural order.
 template <typename T, int D, int G>
@@ -274,7 +299,7 @@ __device__ __forceinline__ void issue_slabs(const Params &p, uint32_t stage, int
 #pragma unroll
     for (int i = lane; i < kChunks; i += 32) {
         const int r = i / kChunksPerRow, c = i % kChunksPerRow;
-        const int pc = sizeof(T) == 2 ? ((c & ~7) | ((c ^ r) & 7)) : c;
+        const int pc = sizeof(T) <= 2 ? ((c & ~7) | ((c ^ r) & 7)) : c;
         const uint32_t d = stage + r * Lay::kRowBytes + pc * 16;
         cp_async16(d, ks + i * 16);
         cp_async16(d + Lay::kSlabBytes, vs + i * 16);
@@ -317,8 +342,9 @@ __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, 
                 }
             }
         }
+        if constexpr (kIsFp8<T>) o *= p.v_scale;
         if (single) {
-            store_out<T>(p.out, (head0 + h) * D + dd, lsum > 0.f ? o * (1.f / lsum) : 0.f);
+            store_out<IoT<T>>(p.out, (head0 + h) * D + dd, lsum > 0.f ? o * (1.f / lsum) : 0.f);
         } else {
             const int64_t row = (head0 + h) * p.max_parts + w.un.part;
             p.ws_acc[row * D + dd] = o;
@@ -337,6 +363,52 @@ struct MmaState {
     float o[D / 16][4];
     uint32_t qb[D / 16][2];
 };
+
+// Online-softmax step of one 16-token block.  s: the block's scores in log2
+// units as S^T fragments (tokens lane/4 and lane/4 + 8, head columns 2(lane%4)
+// and 2(lane%4)+1).  Masks tokens at or past ntok, updates m and l, rescales
+// the O^T accumulators and leaves the unnormalised probabilities in s.
+template <int D>
+__device__ __forceinline__ void softmax_block(float (&s)[4], int ntok, MmaState<D> &st, int lane) {
+    constexpr int KS = D / 16;
+    const int t0 = lane >> 2;
+    if (t0 >= ntok) s[0] = s[1] = -INFINITY;
+    if (t0 + 8 >= ntok) s[2] = s[3] = -INFINITY;
+    // online softmax per head column over the block's tokens
+    float c0 = fmaxf(s[0], s[2]), c1 = fmaxf(s[1], s[3]);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        c0 = fmaxf(c0, __shfl_xor_sync(kFull, c0, off));
+        c1 = fmaxf(c1, __shfl_xor_sync(kFull, c1, off));
+    }
+    const float mn0 = fmaxf(st.m[0], c0), mn1 = fmaxf(st.m[1], c1);
+    const float al0 = fast_exp2(st.m[0] - mn0), al1 = fast_exp2(st.m[1] - mn1);
+    const float p0 = fast_exp2(s[0] - mn0), p1 = fast_exp2(s[1] - mn1);
+    const float p2 = fast_exp2(s[2] - mn0), p3 = fast_exp2(s[3] - mn1);
+    s[0] = p0;
+    s[1] = p1;
+    s[2] = p2;
+    s[3] = p3;
+    float r0 = p0 + p2, r1 = p1 + p3;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        r0 += __shfl_xor_sync(kFull, r0, off);
+        r1 += __shfl_xor_sync(kFull, r1, off);
+    }
+    st.l[0] = st.l[0] * al0 + r0;
+    st.l[1] = st.l[1] * al1 + r1;
+    st.m[0] = mn0;
+    st.m[1] = mn1;
+    if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+            st.o[mt][0] *= al0;
+            st.o[mt][1] *= al1;
+            st.o[mt][2] *= al0;
+            st.o[mt][3] *= al1;
+        }
+    }
+}
 
 // One 16-token block on tensor-core tiles.  kb: shared address of the K slab
 // (V slab follows), rows of 2*D bytes with swizzled 16-byte chunks.
@@ -363,39 +435,8 @@ __device__ __forceinline__ void mma_block(uint32_t kb, unsigned char *vgen, int 
     float s[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) s[k] = (sa[k] + sb[k]) * sl2;
-    const int t0 = lane >> 2;
-    if (t0 >= ntok) s[0] = s[1] = -INFINITY;
-    if (t0 + 8 >= ntok) s[2] = s[3] = -INFINITY;
-    // online softmax per head column over the block's tokens
-    float c0 = fmaxf(s[0], s[2]), c1 = fmaxf(s[1], s[3]);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        c0 = fmaxf(c0, __shfl_xor_sync(kFull, c0, off));
-        c1 = fmaxf(c1, __shfl_xor_sync(kFull, c1, off));
-    }
-    const float mn0 = fmaxf(st.m[0], c0), mn1 = fmaxf(st.m[1], c1);
-    const float al0 = fast_exp2(st.m[0] - mn0), al1 = fast_exp2(st.m[1] - mn1);
-    const float p0 = fast_exp2(s[0] - mn0), p1 = fast_exp2(s[1] - mn1);
-    const float p2 = fast_exp2(s[2] - mn0), p3 = fast_exp2(s[3] - mn1);
-    float r0 = p0 + p2, r1 = p1 + p3;
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        r0 += __shfl_xor_sync(kFull, r0, off);
-        r1 += __shfl_xor_sync(kFull, r1, off);
-    }
-    st.l[0] = st.l[0] * al0 + r0;
-    st.l[1] = st.l[1] * al1 + r1;
-    st.m[0] = mn0;
-    st.m[1] = mn1;
-    if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-            st.o[mt][0] *= al0;
-            st.o[mt][1] *= al1;
-            st.o[mt][2] *= al0;
-            st.o[mt][3] *= al1;
-        }
-    }
+    softmax_block<D>(s, ntok, st, lane);
+    const float p0 = s[0], p1 = s[1], p2 = s[2], p3 = s[3];
     // P^T operand fragments: rows 0-7 / 8-15 of S^T, transposed in registers
     const uint32_t pb0 = movmatrix_trans(pack_bf16x2(p0, p1));
     const uint32_t pb1 = movmatrix_trans(pack_bf16x2(p2, p3));
@@ -413,6 +454,84 @@ __device__ __forceinline__ void mma_block(uint32_t kb, unsigned char *vgen, int 
         uint32_t a[4];
         ldsm_x4_trans(a, addr(vb, vrow, mt * 2 + (mat & 1)));
         mma_bf16_16816(st.o[mt], a, pb0, pb1);
+    }
+}
+
+// ------------------------------------------------------------- fp8 block
+// Two e4m3 codes (bits 0-7, 8-15) -> f16x2 (exact), low code in the low half.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
+    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+}
+
+// One 16-token block of an fp8 pool on f16 tensor-core tiles.  kb: the K slab
+// (V slab follows), rows of D = 128 bytes, 16-byte chunk c of row r stored at
+// chunk position c ^ (r & 7).  Head dims are laid on the mma slots so that each
+// thread reads whole chunks, conflict free:
+//   S^T = K Q^T: at k step kk = 4j + i, thread (g, t) = (lane/4, lane%4) holds
+//     dims 32t + 16j + 4i + {0,1} in k slots 2t, 2t+1 and + {2,3} in 2t+8, 2t+9
+//     (its query fragments follow the same map);
+//   O^T = V^T P^T: accumulator row g of m tile mt is dim 16g + 2mt, row g + 8 is
+//     dim 16g + 2mt + 1, so thread (g, t) reads chunk g of token rows 2t, 2t+1,
+//     2t+8, 2t+9.
+template <int D>
+__device__ __forceinline__ void mma_block_fp8(const unsigned char *kb, unsigned char *vb, int ntok,
+                                              MmaState<D> &st, float sl2, int lane) {
+    static_assert(D == 128, "the fp8 fragment map assumes 128-byte rows");
+    const int g = lane >> 2, t = lane & 3;
+    auto chunk = [&](const unsigned char *base, int row, int c) {
+        return *reinterpret_cast<const uint4 *>(base + row * D + ((c ^ (row & 7)) << 4));
+    };
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint4 lo = chunk(kb, g, 2 * t + j), hi = chunk(kb, g + 8, 2 * t + j);
+        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int kk = 4 * j + i;
+            uint32_t a[4];
+            a[0] = e4m3x2_to_f16x2(wl[i]);
+            a[1] = e4m3x2_to_f16x2(wh[i]);
+            a[2] = e4m3x2_to_f16x2(wl[i] >> 16);
+            a[3] = e4m3x2_to_f16x2(wh[i] >> 16);
+            if (kk & 1) mma_f16_16816(sb, a, st.qb[kk][0], st.qb[kk][1]);
+            else mma_f16_16816(sa, a, st.qb[kk][0], st.qb[kk][1]);
+        }
+    }
+    float s[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s[k] = (sa[k] + sb[k]) * sl2;
+    softmax_block<D>(s, ntok, st, lane);
+    const uint32_t pb0 = movmatrix_trans(pack_f16x2(s[0], s[1]));
+    const uint32_t pb1 = movmatrix_trans(pack_f16x2(s[2], s[3]));
+    if (ntok < kBlockSize) {
+        // codes past the context may be NaN: zero those V rows
+        for (int idx = lane; idx < (kBlockSize - ntok) * (D / 16); idx += 32)
+            *reinterpret_cast<uint4 *>(vb + (ntok + idx / (D / 16)) * D + (idx % (D / 16)) * 16) =
+                make_uint4(0, 0, 0, 0);
+        __syncwarp();
+    }
+    const uint4 v0 = chunk(vb, 2 * t, g), v1 = chunk(vb, 2 * t + 1, g);
+    const uint4 v2 = chunk(vb, 2 * t + 8, g), v3 = chunk(vb, 2 * t + 9, g);
+    const uint32_t r0[4] = {v0.x, v0.y, v0.z, v0.w}, r1[4] = {v1.x, v1.y, v1.z, v1.w};
+    const uint32_t r2[4] = {v2.x, v2.y, v2.z, v2.w}, r3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        // interleave token pairs: (2t, 2t+1) and (2t+8, 2t+9) of dims 4w+{0,1} and 4w+{2,3}
+        const uint32_t e01 = __byte_perm(r0[w], r1[w], 0x5140), f01 = __byte_perm(r0[w], r1[w], 0x7362);
+        const uint32_t e23 = __byte_perm(r2[w], r3[w], 0x5140), f23 = __byte_perm(r2[w], r3[w], 0x7362);
+        uint32_t a[4];
+        a[0] = e4m3x2_to_f16x2(e01);
+        a[1] = e4m3x2_to_f16x2(e01 >> 16);
+        a[2] = e4m3x2_to_f16x2(e23);
+        a[3] = e4m3x2_to_f16x2(e23 >> 16);
+        mma_f16_16816(st.o[2 * w], a, pb0, pb1);
+        a[0] = e4m3x2_to_f16x2(f01);
+        a[1] = e4m3x2_to_f16x2(f01 >> 16);
+        a[2] = e4m3x2_to_f16x2(f23);
+        a[3] = e4m3x2_to_f16x2(f23 >> 16);
+        mma_f16_16816(st.o[2 * w + 1], a, pb0, pb1);
     }
 }
 
@@ -551,7 +670,8 @@ __device__ __forceinline__ void f32_block(const unsigned char *kb, const unsigne
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ Params p) {
     using Lay = Layout<T, D, G>;
-    constexpr bool kMma = sizeof(T) == 2;
+    constexpr bool kFp8 = kIsFp8<T>;
+    constexpr bool kMma = sizeof(T) <= 2;  // bf16 and fp8 run on tensor-core tiles
     constexpr int NS = Lay::kStagesPerWarp;
     extern __shared__ __align__(128) unsigned char smem[];
     float *pbuf = reinterpret_cast<float *>(smem + Lay::kOffP);
@@ -648,14 +768,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         MmaState<D> ms;
         F32State<D, G> fs;
         const unsigned char *qg =
-            p.q + ((int64_t)cur.un.s * p.num_q_heads + (int64_t)cur.un.h * G) * Lay::kRowBytes;
-        if constexpr (kMma) {
+            p.q + ((int64_t)cur.un.s * p.num_q_heads + (int64_t)cur.un.h * G) * Lay::kQRowBytes;
+        if constexpr (kFp8) {
+            // bf16 -> f16 in the k-slot map of mma_block_fp8; clamped to the f16 range
+            const bool hv = dr < G;
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int d0 = 32 * q4 + 16 * j + 4 * i;
+                    uint2 x = make_uint2(0u, 0u);
+                    if (hv) x = __ldg(reinterpret_cast<const uint2 *>(qg + dr * Lay::kQRowBytes + d0 * 2));
+                    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.x));
+                    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.y));
+                    auto c = [](float v) { return fminf(fmaxf(v, -65504.f), 65504.f); };
+                    ms.qb[4 * j + i][0] = pack_f16x2(c(a.x), c(a.y));
+                    ms.qb[4 * j + i][1] = pack_f16x2(c(b.x), c(b.y));
+                }
+            ms.m[0] = ms.m[1] = -INFINITY;
+            ms.l[0] = ms.l[1] = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) ms.o[mt][0] = ms.o[mt][1] = ms.o[mt][2] = ms.o[mt][3] = 0.f;
+        } else if constexpr (kMma) {
             const bool hv = dr < G;
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const int d0 = kk * 16 + 2 * q4;
-                ms.qb[kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qg + dr * Lay::kRowBytes + d0 * 2)) : 0u;
-                ms.qb[kk][1] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qg + dr * Lay::kRowBytes + (d0 + 8) * 2)) : 0u;
+                ms.qb[kk][0] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qg + dr * Lay::kQRowBytes + d0 * 2)) : 0u;
+                ms.qb[kk][1] = hv ? __ldg(reinterpret_cast<const uint32_t *>(qg + dr * Lay::kQRowBytes + (d0 + 8) * 2)) : 0u;
             }
             ms.m[0] = ms.m[1] = -INFINITY;
             ms.l[0] = ms.l[1] = 0.f;
@@ -689,7 +829,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int stage = n_cmp % NS;
             if ((okmask >> stage) & 1u) {
                 const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
-                if constexpr (kMma)
+                if constexpr (kFp8)
+                    mma_block_fp8<D>(wring + stage * Lay::kStageBytes,
+                                     wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
+                                     p.scale_log2, lane);
+                else if constexpr (kMma)
                     mma_block<D>(wring_s + stage * Lay::kStageBytes,
                                  wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
                                  p.scale_log2, lane);
@@ -718,7 +862,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    const int d = mt * 16 + dr + 8 * half;
+                    // accumulator row dr + 8 half of tile mt (fp8: the dim map of mma_block_fp8)
+                    const int d = kFp8 ? 16 * dr + 2 * mt + half : mt * 16 + dr + 8 * half;
                     if (2 * q4 < G) wacc[(2 * q4) * D + d] = ms.o[mt][2 * half];
                     if (2 * q4 + 1 < G) wacc[(2 * q4 + 1) * D + d] = ms.o[mt][2 * half + 1];
                 }
@@ -968,7 +1113,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
     }
     const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll
-    for (int k = 0; k < kDpl; ++k) store_out<T>(p.out, wid * D + lane * kDpl + k, o[k] * inv);
+    for (int k = 0; k < kDpl; ++k) store_out<IoT<T>>(p.out, wid * D + lane * kDpl + k, o[k] * inv);
 }
 
 template <typename T, int D, int G>
@@ -1089,6 +1234,13 @@ cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
     prm.max_parts = a.max_partitions;
     prm.seq_tokens = a.partition_size;  // launch_t may widen it
     prm.scale_log2 = a.scale * kLog2e;
+    prm.v_scale = 1.f;
+    if (a.cache.dtype == PA_FP8_E4M3) {
+        if (a.cache.head_dim != 128) return cudaErrorInvalidValue;
+        prm.scale_log2 = a.scale * a.cache.k_scale * kLog2e;
+        prm.v_scale = a.cache.v_scale;
+        return launch_g<e4m3_t, 128>(a, prm, stream);
+    }
     const bool bf16 = a.cache.dtype == PA_BF16;
     if (a.cache.head_dim == 128)
         return bf16 ? launch_g<__nv_bfloat16, 128>(a, prm, stream) : launch_g<float, 128>(a, prm, stream);

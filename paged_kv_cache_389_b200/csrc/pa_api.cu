@@ -1,6 +1,7 @@
 // C ABI entry points (include/pa.h): host-side validation, then kernel launch.
 // No device memory is allocated here; every buffer belongs to the caller.
 #include <chrono>
+#include <cmath>
 #include <cstdint>
 #include <thread>
 
@@ -28,6 +29,13 @@ pa_status check_cache(const pa_cache_desc *c) {
     if (c->num_blocks < 0 || c->num_kv_heads <= 0) return PA_ERR_INVALID_ARG;
     if (c->block_size != kBlockSize) return PA_ERR_UNSUPPORTED;
     if (c->head_dim != 64 && c->head_dim != 128) return PA_ERR_UNSUPPORTED;
+    if (c->dtype == PA_FP8_E4M3) {
+        if (!(c->k_scale > 0.f) || !(c->v_scale > 0.f) || !std::isfinite(c->k_scale) ||
+            !std::isfinite(c->v_scale))
+            return PA_ERR_INVALID_ARG;
+        if (c->head_dim != 128) return PA_ERR_UNSUPPORTED;
+        return PA_OK;
+    }
     if (c->dtype != PA_F32 && c->dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
     return PA_OK;
 }
@@ -48,7 +56,7 @@ using namespace pa;
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 1; }
+int32_t pa_abi_version(void) { return 2; }
 
 const char *pa_status_string(pa_status s) {
     switch (s) {

@@ -9,7 +9,7 @@
 
 namespace pa {
 
-inline int dtype_bytes(int32_t dtype) { return dtype == PA_F32 ? 4 : 2; }
+inline int dtype_bytes(int32_t dtype) { return dtype == PA_F32 ? 4 : dtype == PA_FP8_E4M3 ? 1 : 2; }
 
 // Launch `kern` behind the previous grid on `stream` with programmatic stream
 // serialization: it may start before that grid ends and must call grid_dep_wait

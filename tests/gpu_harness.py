@@ -33,6 +33,8 @@ def to_dev(a):
 
 def to_host(t):
     torch = torch_mod()
+    if t.dtype == torch.float8_e4m3fn:
+        return t.contiguous().view(torch.uint8).cpu().numpy()
     if t.dtype == torch.bfloat16:
         return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
     return t.contiguous().cpu().numpy()
@@ -65,28 +67,44 @@ def check_close(got, ref, dtype: str, what: str = ""):
 class TwoSided:
     """A workload set up on the oracle and on the GPU, stepped in lockstep."""
 
-    def __init__(self, wl: workloads.Workload):
+    def __init__(self, wl: workloads.Workload, fp8_scales=None):
+        """fp8_scales = (k_scale, v_scale): a bf16 workload stored in e4m3 pools."""
         torch = torch_mod()
         import paged_kv_cache_389_b200 as pa
         from paged_kv_cache_389_b200.cache import PagedKVCache
         self.pa, self.wl = pa, wl
+        self.fp8 = fp8_scales is not None
+        ks, vs = fp8_scales if self.fp8 else (1.0, 1.0)
+        self.ks, self.vs = ks, vs
         # oracle side
         self.model = BlockManagerModel(wl.num_blocks, wl.block_size, wl.free_order.tolist())
-        fill = BF16_NAN if wl.dtype == "bf16" else np.nan
-        self.kc = np.full(wl.cache_shape(), fill, wl.np_dtype)
-        self.vc = np.full(wl.cache_shape(), fill, wl.np_dtype)
-        workloads.replay(wl, self.model, lambda k, v, s: oracle.cache_write(k, v, s, self.kc, self.vc))
+        if self.fp8:
+            assert wl.dtype == "bf16"
+            self.kc = np.full(wl.cache_shape(), 0x7F, np.uint8)     # e4m3 NaN
+            self.vc = self.kc.copy()
+        else:
+            fill = BF16_NAN if wl.dtype == "bf16" else np.nan
+            self.kc = np.full(wl.cache_shape(), fill, wl.np_dtype)
+            self.vc = np.full(wl.cache_shape(), fill, wl.np_dtype)
+        workloads.replay(wl, self.model, self._oracle_write)
         # GPU side
-        tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
-        self.gpu = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, tdt, "cuda", wl.free_order)
+        tdt = torch.float8_e4m3fn if self.fp8 else torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        self.gpu = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, tdt, "cuda", wl.free_order,
+                                k_scale=ks, v_scale=vs)
         g = self.gpu
 
         def write(k, v, slots):
             pa.pa_cache_write(to_dev(k), to_dev(v), torch.from_numpy(slots).cuda(), g.key_cache,
-                              g.value_cache, g.err_flag)
+                              g.value_cache, g.err_flag, k_scale=ks, v_scale=vs)
         workloads.replay(wl, g.manager, write)
         self.step_index = 0
         self.last_pairs = np.zeros((0, 2), np.int32)
+
+    def _oracle_write(self, k, v, slots):
+        if self.fp8:
+            oracle.cache_write_fp8(k, v, slots, self.kc, self.vc, self.ks, self.vs)
+        else:
+            oracle.cache_write(k, v, slots, self.kc, self.vc)
 
     # -- comparisons -------------------------------------------------------
     def pools_equal(self):
@@ -123,9 +141,10 @@ class TwoSided:
             pa.pa_copy_blocks(self.gpu.key_cache, self.gpu.value_cache,
                               torch.from_numpy(pairs_g).cuda(), self.gpu.err_flag)
         sl = np.array(slots_o, np.int64)
-        oracle.cache_write(step.k_new, step.v_new, sl, self.kc, self.vc)
+        self._oracle_write(step.k_new, step.v_new, sl)
         pa.pa_cache_write(to_dev(step.k_new), to_dev(step.v_new), torch.from_numpy(sl).cuda(),
-                          self.gpu.key_cache, self.gpu.value_cache, self.gpu.err_flag)
+                          self.gpu.key_cache, self.gpu.value_cache, self.gpu.err_flag,
+                          k_scale=self.ks, v_scale=self.vs)
         self.last_pairs = np.array(pairs_o, np.int32).reshape(-1, 2)
 
     def append_decode_step(self, step, partition_size=0):
@@ -146,7 +165,7 @@ class TwoSided:
             pa.pa_copy_blocks(self.gpu.key_cache, self.gpu.value_cache,
                               torch.from_numpy(pairs_g).cuda(), self.gpu.err_flag)
         sl = np.array(slots_o, np.int64)
-        oracle.cache_write(step.k_new, step.v_new, sl, self.kc, self.vc)
+        self._oracle_write(step.k_new, step.v_new, sl)
         t, l = self.tables(step.seqs)
         q = to_dev(step.q)
         out = torch.empty_like(q)
@@ -158,7 +177,7 @@ class TwoSided:
         pa.pa_append_decode(to_dev(step.k_new), to_dev(step.v_new), torch.from_numpy(sl).cuda(), q,
                             self.gpu.key_cache, self.gpu.value_cache, torch.from_numpy(t).cuda(),
                             torch.from_numpy(l).cuda(), maxc, self.wl.scale, out, partition_size, ws,
-                            self.gpu.err_flag)
+                            self.gpu.err_flag, k_scale=self.ks, v_scale=self.vs)
         self.last_pairs = np.array(pairs_o, np.int32).reshape(-1, 2)
         return to_host(out)
 
@@ -175,13 +194,17 @@ class TwoSided:
             ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
         self.pa.pa_decode(q, self.gpu.key_cache, self.gpu.value_cache, torch.from_numpy(t).cuda(),
                           torch.from_numpy(l).cuda(), maxc, self.wl.scale, out, partition_size, ws,
-                          self.gpu.err_flag)
+                          self.gpu.err_flag, k_scale=self.ks, v_scale=self.vs)
         return to_host(out)
 
     def oracle_decode(self, step, rows=None, tables=None, lens=None):
         t, l = self.tables(step.seqs) if tables is None else (tables, lens)
-        if rows is None:
-            return oracle.decode(step.q, self.kc, self.vc, t, l, self.wl.scale)
-        rows = np.asarray(rows)
-        return oracle.decode(np.ascontiguousarray(step.q[rows]), self.kc, self.vc,
-                             np.ascontiguousarray(t[rows]), np.ascontiguousarray(l[rows]), self.wl.scale)
+        if rows is not None:
+            rows = np.asarray(rows)
+            q, t, l = (np.ascontiguousarray(step.q[rows]), np.ascontiguousarray(t[rows]),
+                       np.ascontiguousarray(l[rows]))
+        else:
+            q = step.q
+        if self.fp8:
+            return oracle.decode_fp8(q, self.kc, self.vc, t, l, self.wl.scale, self.ks, self.vs)
+        return oracle.decode(q, self.kc, self.vc, t, l, self.wl.scale)

@@ -41,15 +41,15 @@ def test_only_the_abi_is_exported(pa):
 
 
 def test_version_and_status_strings(pa):
-    assert pa.abi_version() == 1
+    assert pa.abi_version() == 2
     assert pa.status_string(pa.PA_OK) == "ok"
     assert "out of" in pa.status_string(pa.PA_ERR_OOM)
     assert pa.status_string(99) == "unknown status"
 
 
-def desc(nb=8, hkv=2, bs=16, d=128, dt=1):
+def desc(nb=8, hkv=2, bs=16, d=128, dt=1, ks=1.0, vs=1.0):
     from paged_kv_cache_389_b200 import CacheDesc
-    return CacheDesc(nb, hkv, bs, d, dt)
+    return CacheDesc(nb, hkv, bs, d, dt, ks, vs)
 
 
 def test_host_validation_launches_nothing(pa):
@@ -80,6 +80,19 @@ def test_host_validation_launches_nothing(pa):
     # prefill needs bf16 / head_dim 128
     assert L.pa_prefill_chunk(p16, p16, p16, p16, 8, p16, p16, 2, 4, 4, 0.1, p16, C.byref(desc(dt=0)),
                               None, None) == pa.PA_ERR_UNSUPPORTED
+    # fp8 pools: head_dim 128 only, finite positive scales, no prefill
+    f8 = pa.PA_FP8_E4M3
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert L.pa_cache_write(p16, p16, p16, 1, p16, p16, C.byref(desc(dt=f8, ks=bad)), None,
+                                None) == pa.PA_ERR_INVALID_ARG
+        assert L.pa_cache_write(p16, p16, p16, 1, p16, p16, C.byref(desc(dt=f8, vs=bad)), None,
+                                None) == pa.PA_ERR_INVALID_ARG
+    assert L.pa_cache_write(p16, p16, p16, 1, p16, p16, C.byref(desc(dt=f8, d=64)), None,
+                            None) == pa.PA_ERR_UNSUPPORTED
+    assert L.pa_cache_write(None, None, None, 0, None, None, C.byref(desc(dt=f8, ks=0.5)), None,
+                            None) == pa.PA_OK
+    assert L.pa_prefill_chunk(p16, p16, p16, p16, 8, p16, p16, 2, 4, 4, 0.1, p16, C.byref(desc(dt=f8)),
+                              None, None) == pa.PA_ERR_UNSUPPORTED
 
 
 def test_workspace_size_formula(pa):
@@ -105,4 +118,6 @@ def test_decode_launch_count(pa):
     assert pa.pa_decode_launches(8, 128, pa.PA_F32, 512) == 2
     assert pa.pa_decode_launches(8, 64, pa.PA_BF16, 512) == 2
     assert pa.pa_decode_launches(4096, 128, pa.PA_BF16, 512) == 4
+    assert pa.pa_decode_launches(4096, 128, pa.PA_FP8_E4M3, 512) == 2   # no shared-prefix groups
+    assert pa.pa_decode_launches(8, 128, pa.PA_FP8_E4M3, 0) == 1
 
