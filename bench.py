@@ -41,6 +41,9 @@ import workloads  # noqa: E402
 
 PARTITION = 512
 CONFIG_ID = 3
+# FP8 pools: one scale per pool, amax / 448 with amax = 6 (K) and 5 (V) for the
+# synthetic N(0, 1) keys and values
+FP8_SCALES = (6.0 / 448, 5.0 / 448)
 WORKLOAD_NAME = "llama3-8b-gqa-prefix-sharing-decode"
 
 
@@ -49,12 +52,13 @@ def log(*a):
 
 
 # ----------------------------------------------------------------- accounting
-def step_bytes(wl, tables, lens):
+def step_bytes(wl, tables, lens, kv_elem=None):
     """Algorithmic bytes of one decode launch: K+V of every token attended, q in,
     out written.  'unique' counts each (physical block, token slot) once -- the
-    HBM floor when siblings share prefix blocks; 'logical' counts per sequence."""
+    HBM floor when siblings share prefix blocks; 'logical' counts per sequence.
+    kv_elem: bytes per cached element (1 for an fp8 pool; default the workload's)."""
     e = wl.elem_bytes
-    row = wl.num_kv_heads * wl.head_dim * e * 2          # K + V of one token, all kv heads
+    row = wl.num_kv_heads * wl.head_dim * (kv_elem or e) * 2   # K + V of one token, all kv heads
     qo = len(lens) * wl.num_q_heads * wl.head_dim * e * 2
     used = {}
     for s, L in enumerate(lens):
@@ -66,8 +70,9 @@ def step_bytes(wl, tables, lens):
     return unique, logical
 
 
-def cache_write_bytes(wl, ntok):
-    return ntok * wl.num_kv_heads * wl.head_dim * wl.elem_bytes * 2 * 2   # K,V read + write
+def cache_write_bytes(wl, ntok, kv_elem=None):
+    # K,V read (workload dtype) + written (pool dtype)
+    return ntok * wl.num_kv_heads * wl.head_dim * 2 * (wl.elem_bytes + (kv_elem or wl.elem_bytes))
 
 
 # ----------------------------------------------------------------- clocks
@@ -384,14 +389,20 @@ def run_ours(args):
 
 
 # ----------------------------------------------------------------- per-row figures
-def _setup(wl):
+def _setup(wl, fp8=None):
+    """The workload's pool (bf16, or e4m3 with fp8 = (k_scale, v_scale)) filled by
+    replaying its set-up writes through pa_cache_write."""
     import torch
     import paged_kv_cache_389_b200 as pa
     from paged_kv_cache_389_b200.cache import PagedKVCache
-    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, torch.bfloat16, "cuda", wl.free_order)
+    ks, vs = fp8 if fp8 else (1.0, 1.0)
+    dt = torch.float8_e4m3fn if fp8 else torch.bfloat16
+    cache = PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_dim, dt, "cuda", wl.free_order,
+                         k_scale=ks, v_scale=vs)
     dev = lambda a: torch.from_numpy(a.view(np.int16)).cuda().view(torch.bfloat16)
     workloads.replay(wl, cache.manager, lambda k, v, s: pa.pa_cache_write(
-        dev(k), dev(v), torch.from_numpy(s).cuda(), cache.key_cache, cache.value_cache, cache.err_flag))
+        dev(k), dev(v), torch.from_numpy(s).cuda(), cache.key_cache, cache.value_cache, cache.err_flag,
+        k_scale=ks, v_scale=vs))
     return cache, dev
 
 
@@ -436,7 +447,7 @@ def run_rows(reps, peaks, partition=PARTITION):
         n = pa.pa_decode_workspace_size(q.shape[0], q.shape[1], q.shape[2], maxc, part) if part else 0
         ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
         ms = _time(lambda: pa.pa_decode(q, cache.key_cache, cache.value_cache, td, ld, maxc, scale, out,
-                                        part, ws, cache.err_flag), reps)
+                                        part, ws, cache.err_flag, None, cache.k_scale, cache.v_scale), reps)
         rows[name] = {"ms": round(ms, 5), "unique_gbs": round(bytes_u / ms / 1e6, 1),
                       "logical_gbs": round(bytes_l / ms / 1e6, 1), "frac_of_measured_hbm": round(bytes_u / ms / 1e6 / hbm, 4),
                       "seq_steps_per_s": round(nseq / ms * 1e3, 1), "partition_size": part}
@@ -544,6 +555,36 @@ def run_rows(reps, peaks, partition=PARTITION):
     rows["a6_spec_verify_k4"] = {"ms": round(ms, 5), "verified_tokens_per_s": round(S * kdraft / ms * 1e3, 1),
                                  "kv_logical_gbs": round(lb / ms / 1e6, 1), "kv_unique_gbs": round(ub / ms / 1e6, 1),
                                  "draft_tokens": kdraft, "num_seqs": S}
+    assert pa.pa_wait(cache.err_flag) == 0
+    del cache
+    torch.cuda.empty_cache()
+
+    # -- FP8 (e4m3) pools on the same workload: the headline step (cache write +
+    #    decode in one pa_append_decode call) and the decode alone; half the K/V bytes
+    wl = workloads.make(CONFIG_ID)
+    cache, dev = _setup(wl, fp8=FP8_SCALES)
+    st = wl.steps[0]
+    slots, pairs = cache.plan_append(st.seqs)
+    assert len(pairs) == 0
+    mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+    t, l = cache.manager.build_tables(st.seqs, mb)
+    ub, lb = step_bytes(wl, t, l, kv_elem=1)
+    cwb = cache_write_bytes(wl, len(st.seqs), kv_elem=1)
+    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+    kn, vn, sl = dev(st.k_new), dev(st.v_new), torch.from_numpy(slots).cuda()
+    maxc = int(l.max())
+    n = pa.pa_decode_workspace_size(len(st.seqs), wl.num_q_heads, wl.head_dim, maxc, partition)
+    ws8 = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+    out8 = torch.empty_like(q)
+    ms = _time(lambda: pa.pa_append_decode(kn, vn, sl, q, cache.key_cache, cache.value_cache, td, ld, maxc,
+                                           wl.scale, out8, partition, ws8, cache.err_flag, None,
+                                           cache.k_scale, cache.v_scale), reps)
+    rows["a8_fp8_append_decode"] = {"ms": round(ms, 5), "unique_gbs": round((ub + cwb) / ms / 1e6, 1),
+                                    "frac_of_measured_hbm": round((ub + cwb) / ms / 1e6 / hbm, 4),
+                                    "seq_steps_per_s": round(len(st.seqs) / ms * 1e3, 1),
+                                    "kv_bytes_per_element": 1, "partition_size": partition,
+                                    "k_scale": cache.k_scale, "v_scale": cache.v_scale}
+    dec_entry("a8_fp8_decode", cache, q, td, ld, maxc, wl.scale, partition, ub, lb, len(st.seqs))
     assert pa.pa_wait(cache.err_flag) == 0
     del cache
     torch.cuda.empty_cache()
