@@ -458,10 +458,13 @@ __device__ __forceinline__ void mma_block(uint32_t kb, unsigned char *vgen, int 
 }
 
 // ------------------------------------------------------------- fp8 block
-// Two e4m3 codes (bits 0-7, 8-15) -> f16x2 (exact), low code in the low half.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(two & 0xffffu), __NV_E4M3);
-    return (uint32_t)h.x | ((uint32_t)h.y << 16);
+// Four e4m3 codes (bytes 0..3 of w) -> two f16x2 registers (exact): lo holds
+// bytes 0, 1 and hi bytes 2, 3, the lower byte in the lower half of each.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // One 16-token block of an fp8 pool on f16 tensor-core tiles.  kb: the K slab
@@ -491,10 +494,8 @@ __device__ __forceinline__ void mma_block_fp8(const unsigned char *kb, unsigned 
         for (int i = 0; i < 4; ++i) {
             const int kk = 4 * j + i;
             uint32_t a[4];
-            a[0] = e4m3x2_to_f16x2(wl[i]);
-            a[1] = e4m3x2_to_f16x2(wh[i]);
-            a[2] = e4m3x2_to_f16x2(wl[i] >> 16);
-            a[3] = e4m3x2_to_f16x2(wh[i] >> 16);
+            e4m3x4_to_f16x2x2(wl[i], a[0], a[2]);
+            e4m3x4_to_f16x2x2(wh[i], a[1], a[3]);
             if (kk & 1) mma_f16_16816(sb, a, st.qb[kk][0], st.qb[kk][1]);
             else mma_f16_16816(sa, a, st.qb[kk][0], st.qb[kk][1]);
         }
@@ -522,15 +523,11 @@ __device__ __forceinline__ void mma_block_fp8(const unsigned char *kb, unsigned 
         const uint32_t e01 = __byte_perm(r0[w], r1[w], 0x5140), f01 = __byte_perm(r0[w], r1[w], 0x7362);
         const uint32_t e23 = __byte_perm(r2[w], r3[w], 0x5140), f23 = __byte_perm(r2[w], r3[w], 0x7362);
         uint32_t a[4];
-        a[0] = e4m3x2_to_f16x2(e01);
-        a[1] = e4m3x2_to_f16x2(e01 >> 16);
-        a[2] = e4m3x2_to_f16x2(e23);
-        a[3] = e4m3x2_to_f16x2(e23 >> 16);
+        e4m3x4_to_f16x2x2(e01, a[0], a[1]);
+        e4m3x4_to_f16x2x2(e23, a[2], a[3]);
         mma_f16_16816(st.o[2 * w], a, pb0, pb1);
-        a[0] = e4m3x2_to_f16x2(f01);
-        a[1] = e4m3x2_to_f16x2(f01 >> 16);
-        a[2] = e4m3x2_to_f16x2(f23);
-        a[3] = e4m3x2_to_f16x2(f23 >> 16);
+        e4m3x4_to_f16x2x2(f01, a[0], a[1]);
+        e4m3x4_to_f16x2x2(f23, a[2], a[3]);
         mma_f16_16816(st.o[2 * w + 1], a, pb0, pb1);
     }
 }
