@@ -364,18 +364,25 @@ struct MmaState {
     uint32_t qb[D / 16][2];
 };
 
-// Online-softmax step of one 16-token block.  s: the block's scores in log2
+// Online-softmax step over NT 16-token tiles.  s[i]: tile i's scores in log2
 // units as S^T fragments (tokens lane/4 and lane/4 + 8, head columns 2(lane%4)
-// and 2(lane%4)+1).  Masks tokens at or past ntok, updates m and l, rescales
-// the O^T accumulators and leaves the unnormalised probabilities in s.
-template <int D>
-__device__ __forceinline__ void softmax_block(float (&s)[4], int ntok, MmaState<D> &st, int lane) {
+// and 2(lane%4)+1).  Masks tokens at or past ntok[i] (ntok 0: the whole tile),
+// updates m and l, rescales the O^T accumulators and leaves the unnormalised
+// probabilities in s.  At least one tile must hold a token.
+template <int D, int NT>
+__device__ __forceinline__ void softmax_tiles(float (&s)[NT][4], const int (&ntok)[NT], MmaState<D> &st,
+                                              int lane) {
     constexpr int KS = D / 16;
     const int t0 = lane >> 2;
-    if (t0 >= ntok) s[0] = s[1] = -INFINITY;
-    if (t0 + 8 >= ntok) s[2] = s[3] = -INFINITY;
-    // online softmax per head column over the block's tokens
-    float c0 = fmaxf(s[0], s[2]), c1 = fmaxf(s[1], s[3]);
+    float c0 = -INFINITY, c1 = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        if (t0 >= ntok[i]) s[i][0] = s[i][1] = -INFINITY;
+        if (t0 + 8 >= ntok[i]) s[i][2] = s[i][3] = -INFINITY;
+        c0 = fmaxf(c0, fmaxf(s[i][0], s[i][2]));
+        c1 = fmaxf(c1, fmaxf(s[i][1], s[i][3]));
+    }
+    // online softmax per head column over the tiles' tokens
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
         c0 = fmaxf(c0, __shfl_xor_sync(kFull, c0, off));
@@ -383,13 +390,16 @@ __device__ __forceinline__ void softmax_block(float (&s)[4], int ntok, MmaState<
     }
     const float mn0 = fmaxf(st.m[0], c0), mn1 = fmaxf(st.m[1], c1);
     const float al0 = fast_exp2(st.m[0] - mn0), al1 = fast_exp2(st.m[1] - mn1);
-    const float p0 = fast_exp2(s[0] - mn0), p1 = fast_exp2(s[1] - mn1);
-    const float p2 = fast_exp2(s[2] - mn0), p3 = fast_exp2(s[3] - mn1);
-    s[0] = p0;
-    s[1] = p1;
-    s[2] = p2;
-    s[3] = p3;
-    float r0 = p0 + p2, r1 = p1 + p3;
+    float r0 = 0.f, r1 = 0.f;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+        s[i][0] = fast_exp2(s[i][0] - mn0);
+        s[i][1] = fast_exp2(s[i][1] - mn1);
+        s[i][2] = fast_exp2(s[i][2] - mn0);
+        s[i][3] = fast_exp2(s[i][3] - mn1);
+        r0 += s[i][0] + s[i][2];
+        r1 += s[i][1] + s[i][3];
+    }
 #pragma unroll
     for (int off = 4; off < 32; off <<= 1) {
         r0 += __shfl_xor_sync(kFull, r0, off);
@@ -408,6 +418,15 @@ __device__ __forceinline__ void softmax_block(float (&s)[4], int ntok, MmaState<
             st.o[mt][3] *= al1;
         }
     }
+}
+
+template <int D>
+__device__ __forceinline__ void softmax_block(float (&s)[4], int ntok, MmaState<D> &st, int lane) {
+    float t[1][4] = {{s[0], s[1], s[2], s[3]}};
+    const int n[1] = {ntok};
+    softmax_tiles<D, 1>(t, n, st, lane);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) s[k] = t[0][k];
 }
 
 // One 16-token block on tensor-core tiles.  kb: shared address of the K slab
@@ -467,68 +486,86 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t &lo, uint
         : "r"(w));
 }
 
-// One 16-token block of an fp8 pool on f16 tensor-core tiles.  kb: the K slab
-// (V slab follows), rows of D = 128 bytes, 16-byte chunk c of row r stored at
-// chunk position c ^ (r & 7).  Head dims are laid on the mma slots so that each
-// thread reads whole chunks, conflict free:
+// NT (1 or 2) 16-token blocks of an fp8 pool on f16 tensor-core tiles, with one
+// softmax step for all of them: two blocks per step interleave their QK chains
+// and halve the shuffle reductions per token.  kb[i]: block i's stage (K slab,
+// V slab behind it), rows of D = 128 bytes, 16-byte chunk c of row r stored at
+// chunk position c ^ (r & 7); ntok[i]: its tokens (0: skip the block).  Head
+// dims are laid on the mma slots so that each thread reads whole chunks,
+// conflict free:
 //   S^T = K Q^T: at k step kk = 4j + i, thread (g, t) = (lane/4, lane%4) holds
 //     dims 32t + 16j + 4i + {0,1} in k slots 2t, 2t+1 and + {2,3} in 2t+8, 2t+9
 //     (its query fragments follow the same map);
 //   O^T = V^T P^T: accumulator row g of m tile mt is dim 16g + 2mt, row g + 8 is
 //     dim 16g + 2mt + 1, so thread (g, t) reads chunk g of token rows 2t, 2t+1,
 //     2t+8, 2t+9.
-template <int D>
-__device__ __forceinline__ void mma_block_fp8(const unsigned char *kb, unsigned char *vb, int ntok,
+template <int D, int NT>
+__device__ __forceinline__ void mma_tiles_fp8(unsigned char *const (&kb)[NT], const int (&ntok)[NT],
                                               MmaState<D> &st, float sl2, int lane) {
     static_assert(D == 128, "the fp8 fragment map assumes 128-byte rows");
+    constexpr int kSlab = kBlockSize * D;
     const int g = lane >> 2, t = lane & 3;
     auto chunk = [&](const unsigned char *base, int row, int c) {
         return *reinterpret_cast<const uint4 *>(base + row * D + ((c ^ (row & 7)) << 4));
     };
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    float s[NT][4];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const uint4 lo = chunk(kb, g, 2 * t + j), hi = chunk(kb, g + 8, 2 * t + j);
-        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+    for (int b = 0; b < NT; ++b) {
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int kk = 4 * j + i;
-            uint32_t a[4];
-            e4m3x4_to_f16x2x2(wl[i], a[0], a[2]);
-            e4m3x4_to_f16x2x2(wh[i], a[1], a[3]);
-            if (kk & 1) mma_f16_16816(sb, a, st.qb[kk][0], st.qb[kk][1]);
-            else mma_f16_16816(sa, a, st.qb[kk][0], st.qb[kk][1]);
+        for (int j = 0; j < 2; ++j) {
+            const uint4 lo = chunk(kb[b], g, 2 * t + j), hi = chunk(kb[b], g + 8, 2 * t + j);
+            const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int kk = 4 * j + i;
+                uint32_t a[4];
+                e4m3x4_to_f16x2x2(wl[i], a[0], a[2]);
+                e4m3x4_to_f16x2x2(wh[i], a[1], a[3]);
+                if (kk & 1) mma_f16_16816(sb, a, st.qb[kk][0], st.qb[kk][1]);
+                else mma_f16_16816(sa, a, st.qb[kk][0], st.qb[kk][1]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s[b][k] = (sa[k] + sb[k]) * sl2;
+    }
+    softmax_tiles<D, NT>(s, ntok, st, lane);
+    uint32_t pb0[NT], pb1[NT];
+    bool zero = false;
+#pragma unroll
+    for (int b = 0; b < NT; ++b) {
+        pb0[b] = movmatrix_trans(pack_f16x2(s[b][0], s[b][1]));
+        pb1[b] = movmatrix_trans(pack_f16x2(s[b][2], s[b][3]));
+        if (ntok[b] < kBlockSize) {
+            // codes past the context (or of a skipped block) may be NaN: zero those V rows
+            unsigned char *vb = kb[b] + kSlab;
+            for (int idx = lane; idx < (kBlockSize - ntok[b]) * (D / 16); idx += 32)
+                *reinterpret_cast<uint4 *>(vb + (ntok[b] + idx / (D / 16)) * D + (idx % (D / 16)) * 16) =
+                    make_uint4(0, 0, 0, 0);
+            zero = true;
         }
     }
-    float s[4];
+    if (zero) __syncwarp();
 #pragma unroll
-    for (int k = 0; k < 4; ++k) s[k] = (sa[k] + sb[k]) * sl2;
-    softmax_block<D>(s, ntok, st, lane);
-    const uint32_t pb0 = movmatrix_trans(pack_f16x2(s[0], s[1]));
-    const uint32_t pb1 = movmatrix_trans(pack_f16x2(s[2], s[3]));
-    if (ntok < kBlockSize) {
-        // codes past the context may be NaN: zero those V rows
-        for (int idx = lane; idx < (kBlockSize - ntok) * (D / 16); idx += 32)
-            *reinterpret_cast<uint4 *>(vb + (ntok + idx / (D / 16)) * D + (idx % (D / 16)) * 16) =
-                make_uint4(0, 0, 0, 0);
-        __syncwarp();
-    }
-    const uint4 v0 = chunk(vb, 2 * t, g), v1 = chunk(vb, 2 * t + 1, g);
-    const uint4 v2 = chunk(vb, 2 * t + 8, g), v3 = chunk(vb, 2 * t + 9, g);
-    const uint32_t r0[4] = {v0.x, v0.y, v0.z, v0.w}, r1[4] = {v1.x, v1.y, v1.z, v1.w};
-    const uint32_t r2[4] = {v2.x, v2.y, v2.z, v2.w}, r3[4] = {v3.x, v3.y, v3.z, v3.w};
+    for (int b = 0; b < NT; ++b) {
+        const unsigned char *vb = kb[b] + kSlab;
+        const uint4 v0 = chunk(vb, 2 * t, g), v1 = chunk(vb, 2 * t + 1, g);
+        const uint4 v2 = chunk(vb, 2 * t + 8, g), v3 = chunk(vb, 2 * t + 9, g);
+        const uint32_t r0[4] = {v0.x, v0.y, v0.z, v0.w}, r1[4] = {v1.x, v1.y, v1.z, v1.w};
+        const uint32_t r2[4] = {v2.x, v2.y, v2.z, v2.w}, r3[4] = {v3.x, v3.y, v3.z, v3.w};
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        // interleave token pairs: (2t, 2t+1) and (2t+8, 2t+9) of dims 4w+{0,1} and 4w+{2,3}
-        const uint32_t e01 = __byte_perm(r0[w], r1[w], 0x5140), f01 = __byte_perm(r0[w], r1[w], 0x7362);
-        const uint32_t e23 = __byte_perm(r2[w], r3[w], 0x5140), f23 = __byte_perm(r2[w], r3[w], 0x7362);
-        uint32_t a[4];
-        e4m3x4_to_f16x2x2(e01, a[0], a[1]);
-        e4m3x4_to_f16x2x2(e23, a[2], a[3]);
-        mma_f16_16816(st.o[2 * w], a, pb0, pb1);
-        e4m3x4_to_f16x2x2(f01, a[0], a[1]);
-        e4m3x4_to_f16x2x2(f23, a[2], a[3]);
-        mma_f16_16816(st.o[2 * w + 1], a, pb0, pb1);
+        for (int w = 0; w < 4; ++w) {
+            // interleave token pairs (2t, 2t+1) and (2t+8, 2t+9) of dims 4w+{0,1}, 4w+{2,3}
+            const uint32_t e01 = __byte_perm(r0[w], r1[w], 0x5140), f01 = __byte_perm(r0[w], r1[w], 0x7362);
+            const uint32_t e23 = __byte_perm(r2[w], r3[w], 0x5140), f23 = __byte_perm(r2[w], r3[w], 0x7362);
+            uint32_t a[4];
+            e4m3x4_to_f16x2x2(e01, a[0], a[1]);
+            e4m3x4_to_f16x2x2(e23, a[2], a[3]);
+            mma_f16_16816(st.o[2 * w], a, pb0[b], pb1[b]);
+            e4m3x4_to_f16x2x2(f01, a[0], a[1]);
+            e4m3x4_to_f16x2x2(f23, a[2], a[3]);
+            mma_f16_16816(st.o[2 * w + 1], a, pb0[b], pb1[b]);
+        }
     }
 }
 
@@ -817,7 +854,34 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 for (int k = 0; k < C::kPvPairs; ++k) fs.acc[h][k] = make_float2(0.f, 0.f);
         }
 
-        // ---- this warp's blocks of the unit, up to NS fetched ahead
+        // ---- this warp's blocks of the unit, up to NS fetched ahead (fp8: two
+        // blocks per step, the pair's stages both landed before it is computed)
+        if constexpr (kFp8) {
+            static_assert(NS >= 2, "paired fp8 blocks need two stages");
+            for (int j = warp; j < cur.nb; j += 2 * kWarps) {
+                const bool two = j + kWarps < cur.nb;
+                while (n_iss - n_cmp < NS && fetch_one()) {
+                }
+                cp_async_wait_dyn(n_iss - n_cmp - (two ? 2 : 1));
+                __syncwarp();
+                const int s0 = n_cmp % NS, s1 = (n_cmp + 1) % NS;
+                const bool ok0 = (okmask >> s0) & 1u, ok1 = two && ((okmask >> s1) & 1u);
+                const int nt0 = ok0 ? min(kBlockSize, cur.nt - j * kBlockSize) : 0;
+                if (two) {
+                    if (ok0 || ok1) {
+                        unsigned char *const kb2[2] = {wring + s0 * Lay::kStageBytes, wring + s1 * Lay::kStageBytes};
+                        const int n2[2] = {nt0, ok1 ? min(kBlockSize, cur.nt - (j + kWarps) * kBlockSize) : 0};
+                        mma_tiles_fp8<D, 2>(kb2, n2, ms, p.scale_log2, lane);
+                    }
+                } else if (ok0) {
+                    unsigned char *const kb1[1] = {wring + s0 * Lay::kStageBytes};
+                    const int n1[1] = {nt0};
+                    mma_tiles_fp8<D, 1>(kb1, n1, ms, p.scale_log2, lane);
+                }
+                __syncwarp();  // the stages may be refilled by the next fetch
+                n_cmp += two ? 2 : 1;
+            }
+        } else
         for (int j = warp; j < cur.nb; j += kWarps) {
             while (n_iss - n_cmp < NS && fetch_one()) {
             }
@@ -826,11 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int stage = n_cmp % NS;
             if ((okmask >> stage) & 1u) {
                 const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
-                if constexpr (kFp8)
-                    mma_block_fp8<D>(wring + stage * Lay::kStageBytes,
-                                     wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
-                                     p.scale_log2, lane);
-                else if constexpr (kMma)
+                if constexpr (kMma)
                     mma_block<D>(wring_s + stage * Lay::kStageBytes,
                                  wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
                                  p.scale_log2, lane);
