@@ -334,8 +334,7 @@ def run_ours(args):
 
     rows = None
     if rank == 0 and world == 1 and not args.no_rows:
-        peaks0 = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
-            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+        peaks0 = load_peaks()
         del cache, ws, out, q, k_new, v_new, tables_d, lens_d, slots_d
         torch.cuda.empty_cache()
         rows = run_rows(args.row_reps, peaks0, args.partition)
@@ -345,8 +344,7 @@ def run_ours(args):
         cpu = cpu_baseline(wl, None, step, tables_h, lens_h, budget_s=args.cpu_seconds)
 
     if rank == 0:
-        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
-            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+        peaks = load_peaks()
         peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
         achieved = (unique_b + cw_b) / (call_ms * 1e-3) / 1e9
         value = world * (unique_b + cw_b) * K / (ms_max * 1e-3) / 1e9
@@ -389,6 +387,11 @@ def run_ours(args):
 
 
 # ----------------------------------------------------------------- per-row figures
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    return json.load(open(path)) if os.path.exists(path) else None
+
+
 def _setup(wl, fp8=None):
     """The workload's pool (bf16, or e4m3 with fp8 = (k_scale, v_scale)) filled by
     replaying its set-up writes through pa_cache_write."""
@@ -434,8 +437,16 @@ def _time(fn, reps, warm=3, graph=False):
     return a.elapsed_time(b) / reps
 
 
-def run_rows(reps, peaks, partition=PARTITION):
-    """Each hot-path row on its own workload; device time, inputs resident in HBM."""
+ROW_GROUPS = ("mha7b", "fork", "spec", "fp8", "prefix", "long")
+
+
+def run_rows(reps, peaks, partition=PARTITION, groups=None):
+    """Each hot-path row on its own workload; device time, inputs resident in HBM.
+    groups: the row groups to run (default all of ROW_GROUPS)."""
+    groups = set(ROW_GROUPS) if not groups else groups
+    unknown = groups - set(ROW_GROUPS)
+    if unknown:
+        raise ValueError(f"unknown row groups {sorted(unknown)}; known: {ROW_GROUPS}")
     import torch
     import paged_kv_cache_389_b200 as pa
     hbm = float(peaks["hbm_gbs"]) if peaks else 6650.0
@@ -452,184 +463,191 @@ def run_rows(reps, peaks, partition=PARTITION):
                       "logical_gbs": round(bytes_l / ms / 1e6, 1), "frac_of_measured_hbm": round(bytes_u / ms / 1e6 / hbm, 4),
                       "seq_steps_per_s": round(nseq / ms * 1e3, 1), "partition_size": part}
 
-    # -- MHA-7B decode (64 seqs, 32/32 heads): unsplit and split-K
-    wl = workloads.make(2)
-    cache, dev = _setup(wl)
-    st = wl.steps[0]
-    cache.append(st.seqs, dev(st.k_new), dev(st.v_new))
-    mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
-    t, l = cache.manager.build_tables(st.seqs, mb)
-    ub, lb = step_bytes(wl, t, l)
-    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
-    for part in (0, 1024):
-        dec_entry(f"a3_decode_mha7b_p{part}", cache, q, td, ld, int(l.max()), wl.scale, part, ub, lb, len(st.seqs))
-    del cache
-    torch.cuda.empty_cache()
-
-    # -- parallel sampling: 128 parents x 4 children, 16 steps of copy-on-write + cache write + decode
-    wl = workloads.make(4)
-    cache, dev = _setup(wl)
-    S = len(wl.steps[0].seqs)
-    part = partition
-    ev = []
-    host_s = 0.0
-    total_pairs = 0
-    ub_sum = 0
-    pairs1 = None
-    for st in wl.steps:
-        h0 = time.perf_counter()
-        slots, pairs = cache.plan_append(st.seqs)
+    if "mha7b" in groups:
+        # -- MHA-7B decode (64 seqs, 32/32 heads): unsplit and split-K
+        wl = workloads.make(2)
+        cache, dev = _setup(wl)
+        st = wl.steps[0]
+        cache.append(st.seqs, dev(st.k_new), dev(st.v_new))
         mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
         t, l = cache.manager.build_tables(st.seqs, mb)
-        host_s += time.perf_counter() - h0
-        ub, _ = step_bytes(wl, t, l)
-        ub_sum += ub
-        total_pairs += len(pairs)
+        ub, lb = step_bytes(wl, t, l)
         td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+        for part in (0, 1024):
+            dec_entry(f"a3_decode_mha7b_p{part}", cache, q, td, ld, int(l.max()), wl.scale, part, ub, lb, len(st.seqs))
+        del cache
+        torch.cuda.empty_cache()
+
+    if "fork" in groups:
+        # -- parallel sampling: 128 parents x 4 children, 16 steps of copy-on-write + cache write + decode
+        wl = workloads.make(4)
+        cache, dev = _setup(wl)
+        S = len(wl.steps[0].seqs)
+        part = partition
+        ev = []
+        host_s = 0.0
+        total_pairs = 0
+        ub_sum = 0
+        pairs1 = None
+        for st in wl.steps:
+            h0 = time.perf_counter()
+            slots, pairs = cache.plan_append(st.seqs)
+            mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+            t, l = cache.manager.build_tables(st.seqs, mb)
+            host_s += time.perf_counter() - h0
+            ub, _ = step_bytes(wl, t, l)
+            ub_sum += ub
+            total_pairs += len(pairs)
+            td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+            kn, vn = dev(st.k_new), dev(st.v_new)
+            sl = torch.from_numpy(slots).cuda()
+            pr = torch.from_numpy(pairs).cuda() if len(pairs) else None
+            if pairs1 is None and pr is not None:
+                pairs1 = pr
+            out = torch.empty_like(q)
+            maxc = int(l.max())
+            n = pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, maxc, part)
+            ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record()
+            if pr is not None:
+                pa.pa_copy_blocks(cache.key_cache, cache.value_cache, pr, cache.err_flag)
+            e[1].record()
+            pa.pa_cache_write(kn, vn, sl, cache.key_cache, cache.value_cache, cache.err_flag)
+            e[2].record()
+            pa.pa_decode(q, cache.key_cache, cache.value_cache, td, ld, maxc, wl.scale, out, part, ws, cache.err_flag)
+            e[3].record()
+            ev.append((e, len(pairs)))
+        torch.cuda.synchronize()
+        assert pa.pa_wait(cache.err_flag) == 0
+        copy_ms = sum(e[0].elapsed_time(e[1]) for e, _ in ev)
+        cw_ms = sum(e[1].elapsed_time(e[2]) for e, _ in ev)
+        dec_ms = sum(e[2].elapsed_time(e[3]) for e, _ in ev)
+        blk_bytes = wl.num_kv_heads * 16 * wl.head_dim * 2 * 2          # K + V of one block
+        e1, np1 = ev[0]
+        c1 = e1[0].elapsed_time(e1[1])
+        rows["fork_cow_16_steps"] = {"seq_steps_per_s_device": round(S * len(wl.steps) / ((copy_ms + cw_ms + dec_ms) * 1e-3), 1),
+                                     "device_ms_total": round(copy_ms + cw_ms + dec_ms, 4), "host_plan_ms_total": round(1e3 * host_s, 3),
+                                     "decode_ms_total": round(dec_ms, 4), "decode_unique_gbs": round(ub_sum / dec_ms / 1e6, 1),
+                                     "cache_write_ms_total": round(cw_ms, 4), "copy_blocks_ms_total": round(copy_ms, 4),
+                                     "copy_pairs_total": total_pairs}
+        rows["a2_copy_blocks_step1"] = {"pairs": np1, "ms_first_launch": round(c1, 5),
+                                        "gbs_first_launch": round(np1 * blk_bytes * 2 / c1 / 1e6, 1)}   # read + write
+        if pairs1 is not None:   # same pairs again (the pool is not used afterwards)
+            ms = _time(lambda: pa.pa_copy_blocks(cache.key_cache, cache.value_cache, pairs1, cache.err_flag), reps, graph=True)
+            rows["a2_copy_blocks_step1"].update({"ms": round(ms, 5), "gbs": round(np1 * blk_bytes * 2 / ms / 1e6, 1)})
+        # steady-state copy of the same 384 pairs (idempotent), and the 512-token cache write
+        st = wl.steps[-1]
         kn, vn = dev(st.k_new), dev(st.v_new)
-        sl = torch.from_numpy(slots).cuda()
-        pr = torch.from_numpy(pairs).cuda() if len(pairs) else None
-        if pairs1 is None and pr is not None:
-            pairs1 = pr
-        out = torch.empty_like(q)
+        slots = torch.from_numpy(np.array([cache.manager.block_table(s)[-1] * 16 for s in st.seqs], np.int64)).cuda()
+        ms = _time(lambda: pa.pa_cache_write(kn, vn, slots, cache.key_cache, cache.value_cache, cache.err_flag), reps,
+                   graph=True)
+        rows["a1_cache_write_512tok"] = {"ms": round(ms, 5), "gbs": round(cache_write_bytes(wl, S) / ms / 1e6, 1)}
+        del cache
+        torch.cuda.empty_cache()
+
+    if "spec" in groups:
+        # -- speculative verify on the prefix-sharing workload: every sequence appends 4
+        #    draft tokens; the 4 new positions attend causally (a 4-row chunk)
+        wl = workloads.make(CONFIG_ID)
+        cache, dev = _setup(wl)
+        seqs = wl.steps[0].seqs
+        S, kdraft = len(seqs), 4
+        rng = np.random.default_rng(7)
+        kd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
+        vd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
+        cache.append(seqs, kd, vd, counts=[kdraft] * S)
+        mb = max(cache.manager.num_seq_blocks(s) for s in seqs)
+        t, l = cache.manager.build_tables(seqs, mb)
+        td, ld = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda()
+        qv = dev(workloads.normal(rng, (S, kdraft, wl.num_q_heads, wl.head_dim), "bf16"))
+        outv = torch.empty_like(qv)
+        chv = torch.full((S,), kdraft, dtype=torch.int32, device="cuda")
+        ms = _time(lambda: pa.pa_prefill_chunk(qv, cache.key_cache, cache.value_cache, td, ld, chv, wl.scale, outv,
+                                               cache.err_flag), reps)
+        ub, lb = step_bytes(wl, t, l)
+        rows["a6_spec_verify_k4"] = {"ms": round(ms, 5), "verified_tokens_per_s": round(S * kdraft / ms * 1e3, 1),
+                                     "kv_logical_gbs": round(lb / ms / 1e6, 1), "kv_unique_gbs": round(ub / ms / 1e6, 1),
+                                     "draft_tokens": kdraft, "num_seqs": S}
+        assert pa.pa_wait(cache.err_flag) == 0
+        del cache
+        torch.cuda.empty_cache()
+
+    if "fp8" in groups:
+        # -- FP8 (e4m3) pools on the same workload: the headline step (cache write +
+        #    decode in one pa_append_decode call) and the decode alone; half the K/V bytes
+        wl = workloads.make(CONFIG_ID)
+        cache, dev = _setup(wl, fp8=FP8_SCALES)
+        st = wl.steps[0]
+        slots, pairs = cache.plan_append(st.seqs)
+        assert len(pairs) == 0
+        mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+        t, l = cache.manager.build_tables(st.seqs, mb)
+        ub, lb = step_bytes(wl, t, l, kv_elem=1)
+        cwb = cache_write_bytes(wl, len(st.seqs), kv_elem=1)
+        td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+        kn, vn, sl = dev(st.k_new), dev(st.v_new), torch.from_numpy(slots).cuda()
         maxc = int(l.max())
-        n = pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, maxc, part)
-        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-        e[0].record()
-        if pr is not None:
-            pa.pa_copy_blocks(cache.key_cache, cache.value_cache, pr, cache.err_flag)
-        e[1].record()
-        pa.pa_cache_write(kn, vn, sl, cache.key_cache, cache.value_cache, cache.err_flag)
-        e[2].record()
-        pa.pa_decode(q, cache.key_cache, cache.value_cache, td, ld, maxc, wl.scale, out, part, ws, cache.err_flag)
-        e[3].record()
-        ev.append((e, len(pairs)))
-    torch.cuda.synchronize()
-    assert pa.pa_wait(cache.err_flag) == 0
-    copy_ms = sum(e[0].elapsed_time(e[1]) for e, _ in ev)
-    cw_ms = sum(e[1].elapsed_time(e[2]) for e, _ in ev)
-    dec_ms = sum(e[2].elapsed_time(e[3]) for e, _ in ev)
-    blk_bytes = wl.num_kv_heads * 16 * wl.head_dim * 2 * 2          # K + V of one block
-    e1, np1 = ev[0]
-    c1 = e1[0].elapsed_time(e1[1])
-    rows["fork_cow_16_steps"] = {"seq_steps_per_s_device": round(S * len(wl.steps) / ((copy_ms + cw_ms + dec_ms) * 1e-3), 1),
-                                 "device_ms_total": round(copy_ms + cw_ms + dec_ms, 4), "host_plan_ms_total": round(1e3 * host_s, 3),
-                                 "decode_ms_total": round(dec_ms, 4), "decode_unique_gbs": round(ub_sum / dec_ms / 1e6, 1),
-                                 "cache_write_ms_total": round(cw_ms, 4), "copy_blocks_ms_total": round(copy_ms, 4),
-                                 "copy_pairs_total": total_pairs}
-    rows["a2_copy_blocks_step1"] = {"pairs": np1, "ms_first_launch": round(c1, 5),
-                                    "gbs_first_launch": round(np1 * blk_bytes * 2 / c1 / 1e6, 1)}   # read + write
-    if pairs1 is not None:   # same pairs again (the pool is not used afterwards)
-        ms = _time(lambda: pa.pa_copy_blocks(cache.key_cache, cache.value_cache, pairs1, cache.err_flag), reps, graph=True)
-        rows["a2_copy_blocks_step1"].update({"ms": round(ms, 5), "gbs": round(np1 * blk_bytes * 2 / ms / 1e6, 1)})
-    # steady-state copy of the same 384 pairs (idempotent), and the 512-token cache write
-    st = wl.steps[-1]
-    kn, vn = dev(st.k_new), dev(st.v_new)
-    slots = torch.from_numpy(np.array([cache.manager.block_table(s)[-1] * 16 for s in st.seqs], np.int64)).cuda()
-    ms = _time(lambda: pa.pa_cache_write(kn, vn, slots, cache.key_cache, cache.value_cache, cache.err_flag), reps,
-               graph=True)
-    rows["a1_cache_write_512tok"] = {"ms": round(ms, 5), "gbs": round(cache_write_bytes(wl, S) / ms / 1e6, 1)}
-    del cache
-    torch.cuda.empty_cache()
+        n = pa.pa_decode_workspace_size(len(st.seqs), wl.num_q_heads, wl.head_dim, maxc, partition)
+        ws8 = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+        out8 = torch.empty_like(q)
+        ms = _time(lambda: pa.pa_append_decode(kn, vn, sl, q, cache.key_cache, cache.value_cache, td, ld, maxc,
+                                               wl.scale, out8, partition, ws8, cache.err_flag, None,
+                                               cache.k_scale, cache.v_scale), reps)
+        rows["a8_fp8_append_decode"] = {"ms": round(ms, 5), "unique_gbs": round((ub + cwb) / ms / 1e6, 1),
+                                        "frac_of_measured_hbm": round((ub + cwb) / ms / 1e6 / hbm, 4),
+                                        "seq_steps_per_s": round(len(st.seqs) / ms * 1e3, 1),
+                                        "kv_bytes_per_element": 1, "partition_size": partition,
+                                        "k_scale": cache.k_scale, "v_scale": cache.v_scale}
+        dec_entry("a8_fp8_decode", cache, q, td, ld, maxc, wl.scale, partition, ub, lb, len(st.seqs))
+        assert pa.pa_wait(cache.err_flag) == 0
+        del cache
+        torch.cuda.empty_cache()
 
-    # -- speculative verify on the prefix-sharing workload: every sequence appends 4
-    #    draft tokens; the 4 new positions attend causally (a 4-row chunk)
-    wl = workloads.make(CONFIG_ID)
-    cache, dev = _setup(wl)
-    seqs = wl.steps[0].seqs
-    S, kdraft = len(seqs), 4
-    rng = np.random.default_rng(7)
-    kd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
-    vd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
-    cache.append(seqs, kd, vd, counts=[kdraft] * S)
-    mb = max(cache.manager.num_seq_blocks(s) for s in seqs)
-    t, l = cache.manager.build_tables(seqs, mb)
-    td, ld = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda()
-    qv = dev(workloads.normal(rng, (S, kdraft, wl.num_q_heads, wl.head_dim), "bf16"))
-    outv = torch.empty_like(qv)
-    chv = torch.full((S,), kdraft, dtype=torch.int32, device="cuda")
-    ms = _time(lambda: pa.pa_prefill_chunk(qv, cache.key_cache, cache.value_cache, td, ld, chv, wl.scale, outv,
-                                           cache.err_flag), reps)
-    ub, lb = step_bytes(wl, t, l)
-    rows["a6_spec_verify_k4"] = {"ms": round(ms, 5), "verified_tokens_per_s": round(S * kdraft / ms * 1e3, 1),
-                                 "kv_logical_gbs": round(lb / ms / 1e6, 1), "kv_unique_gbs": round(ub / ms / 1e6, 1),
-                                 "draft_tokens": kdraft, "num_seqs": S}
-    assert pa.pa_wait(cache.err_flag) == 0
-    del cache
-    torch.cuda.empty_cache()
+    if "prefix" in groups:
+        # -- automatic prefix caching (host): 256 prompts = a shared 512-token system
+        #    prompt + a private lognormal tail, created from their token ids
+        bm = pa.BlockManager(32768, 16)
+        prng = np.random.default_rng(11)
+        system = prng.integers(0, 32000, size=512).tolist()
+        tails = np.clip(np.rint(600 * np.exp(prng.standard_normal(256))), 1, 8192).astype(int)
+        prompts = [system + prng.integers(0, 32000, size=int(n)).tolist() for n in tails]
+        h0 = time.perf_counter()
+        hit = sum(bm.add_seq_tokens(i, pr)[0] for i, pr in enumerate(prompts))
+        host_s = time.perf_counter() - h0
+        total = sum(len(pr) for pr in prompts)
+        rows["a7_prefix_cache_host"] = {"prompts": len(prompts), "prompt_tokens": total, "cached_tokens": int(hit),
+                                        "hit_fraction": round(hit / total, 4), "kv_writes_saved_bytes":
+                                        int(hit) * 8 * 128 * 2 * 2,
+                                        "host_us_per_prompt": round(1e6 * host_s / len(prompts), 2)}
+        del bm
 
-    # -- FP8 (e4m3) pools on the same workload: the headline step (cache write +
-    #    decode in one pa_append_decode call) and the decode alone; half the K/V bytes
-    wl = workloads.make(CONFIG_ID)
-    cache, dev = _setup(wl, fp8=FP8_SCALES)
-    st = wl.steps[0]
-    slots, pairs = cache.plan_append(st.seqs)
-    assert len(pairs) == 0
-    mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
-    t, l = cache.manager.build_tables(st.seqs, mb)
-    ub, lb = step_bytes(wl, t, l, kv_elem=1)
-    cwb = cache_write_bytes(wl, len(st.seqs), kv_elem=1)
-    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
-    kn, vn, sl = dev(st.k_new), dev(st.v_new), torch.from_numpy(slots).cuda()
-    maxc = int(l.max())
-    n = pa.pa_decode_workspace_size(len(st.seqs), wl.num_q_heads, wl.head_dim, maxc, partition)
-    ws8 = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
-    out8 = torch.empty_like(q)
-    ms = _time(lambda: pa.pa_append_decode(kn, vn, sl, q, cache.key_cache, cache.value_cache, td, ld, maxc,
-                                           wl.scale, out8, partition, ws8, cache.err_flag, None,
-                                           cache.k_scale, cache.v_scale), reps)
-    rows["a8_fp8_append_decode"] = {"ms": round(ms, 5), "unique_gbs": round((ub + cwb) / ms / 1e6, 1),
-                                    "frac_of_measured_hbm": round((ub + cwb) / ms / 1e6 / hbm, 4),
-                                    "seq_steps_per_s": round(len(st.seqs) / ms * 1e3, 1),
-                                    "kv_bytes_per_element": 1, "partition_size": partition,
-                                    "k_scale": cache.k_scale, "v_scale": cache.v_scale}
-    dec_entry("a8_fp8_decode", cache, q, td, ld, maxc, wl.scale, partition, ub, lb, len(st.seqs))
-    assert pa.pa_wait(cache.err_flag) == 0
-    del cache
-    torch.cuda.empty_cache()
+    if "long" in groups:
+        # -- long context: split-K decode + tcgen05 prefill chunk
+        wl = workloads.make(5)
+        cache, dev = _setup(wl)
+        st = wl.steps[0]
+        mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+        t, l = cache.manager.build_tables(st.seqs, mb)
+        ub, lb = step_bytes(wl, t, l)
+        td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+        for part in (512, 2048):
+            dec_entry(f"a4_decode_long_p{part}", cache, q, td, ld, int(l.max()), wl.scale, part, ub, lb, len(st.seqs))
+        pf = wl.prefill
+        qp = dev(pf.q)
+        outp = torch.empty_like(qp)
+        ch = torch.full((len(pf.seqs),), pf.chunk, dtype=torch.int32, device="cuda")
+        ms = _time(lambda: pa.pa_prefill_chunk(qp, cache.key_cache, cache.value_cache, td, ld, ch, wl.scale, outp,
+                                               cache.err_flag), max(3, reps // 10))
+        keys = sum(int(L) - pf.chunk + i + 1 for L in l for i in range(pf.chunk))
+        flops = 4.0 * wl.num_q_heads * wl.head_dim * keys
+        rows["a5_prefill_chunk_long"] = {"ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1),
+                                         "frac_of_measured_bf16": round(flops / ms / 1e9 / tf_burst, 4),
+                                         "flops": flops, "rows": len(pf.seqs) * pf.chunk}
+        assert pa.pa_wait(cache.err_flag) == 0
+        del cache
+        torch.cuda.empty_cache()
 
-    # -- automatic prefix caching (host): 256 prompts = a shared 512-token system
-    #    prompt + a private lognormal tail, created from their token ids
-    bm = pa.BlockManager(32768, 16)
-    prng = np.random.default_rng(11)
-    system = prng.integers(0, 32000, size=512).tolist()
-    tails = np.clip(np.rint(600 * np.exp(prng.standard_normal(256))), 1, 8192).astype(int)
-    prompts = [system + prng.integers(0, 32000, size=int(n)).tolist() for n in tails]
-    h0 = time.perf_counter()
-    hit = sum(bm.add_seq_tokens(i, pr)[0] for i, pr in enumerate(prompts))
-    host_s = time.perf_counter() - h0
-    total = sum(len(pr) for pr in prompts)
-    rows["a7_prefix_cache_host"] = {"prompts": len(prompts), "prompt_tokens": total, "cached_tokens": int(hit),
-                                    "hit_fraction": round(hit / total, 4), "kv_writes_saved_bytes":
-                                    int(hit) * 8 * 128 * 2 * 2,
-                                    "host_us_per_prompt": round(1e6 * host_s / len(prompts), 2)}
-    del bm
-
-    # -- long context: split-K decode + tcgen05 prefill chunk
-    wl = workloads.make(5)
-    cache, dev = _setup(wl)
-    st = wl.steps[0]
-    mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
-    t, l = cache.manager.build_tables(st.seqs, mb)
-    ub, lb = step_bytes(wl, t, l)
-    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
-    for part in (512, 2048):
-        dec_entry(f"a4_decode_long_p{part}", cache, q, td, ld, int(l.max()), wl.scale, part, ub, lb, len(st.seqs))
-    pf = wl.prefill
-    qp = dev(pf.q)
-    outp = torch.empty_like(qp)
-    ch = torch.full((len(pf.seqs),), pf.chunk, dtype=torch.int32, device="cuda")
-    ms = _time(lambda: pa.pa_prefill_chunk(qp, cache.key_cache, cache.value_cache, td, ld, ch, wl.scale, outp,
-                                           cache.err_flag), max(3, reps // 10))
-    keys = sum(int(L) - pf.chunk + i + 1 for L in l for i in range(pf.chunk))
-    flops = 4.0 * wl.num_q_heads * wl.head_dim * keys
-    rows["a5_prefill_chunk_long"] = {"ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1),
-                                     "frac_of_measured_bf16": round(flops / ms / 1e9 / tf_burst, 4),
-                                     "flops": flops, "rows": len(pf.seqs) * pf.chunk}
-    assert pa.pa_wait(cache.err_flag) == 0
-    del cache
-    torch.cuda.empty_cache()
     return rows
 
 
@@ -738,6 +756,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row figures of the other workloads")
     ap.add_argument("--row-reps", type=int, default=50)
+    ap.add_argument("--rows-only", default="",
+                    help="comma list of row groups (mha7b, fork, spec, fp8, prefix, long): time only "
+                         "those rows, print them as one JSON line and skip the headline step")
     ap.add_argument("--partition", type=int, default=PARTITION,
                     help="split-K partition size in tokens (multiple of 16) of the timed decode")
     args = ap.parse_args()
@@ -745,6 +766,9 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.rows_only:
+        print(json.dumps({"rows": run_rows(args.row_reps, load_peaks(), args.partition,
+                                           set(args.rows_only.split(",")))}), flush=True)
     else:
         run_ours(args)
 
