@@ -374,11 +374,14 @@ __device__ __forceinline__ void softmax_tiles(float (&s)[NT][4], const int (&nto
                                               int lane) {
     constexpr int KS = D / 16;
     const int t0 = lane >> 2;
-    float c0 = -INFINITY, c1 = -INFINITY;
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
         if (t0 >= ntok[i]) s[i][0] = s[i][1] = -INFINITY;
         if (t0 + 8 >= ntok[i]) s[i][2] = s[i][3] = -INFINITY;
+    }
+    float c0 = fmaxf(s[0][0], s[0][2]), c1 = fmaxf(s[0][1], s[0][3]);
+#pragma unroll
+    for (int i = 1; i < NT; ++i) {
         c0 = fmaxf(c0, fmaxf(s[i][0], s[i][2]));
         c1 = fmaxf(c1, fmaxf(s[i][1], s[i][3]));
     }
@@ -390,13 +393,16 @@ __device__ __forceinline__ void softmax_tiles(float (&s)[NT][4], const int (&nto
     }
     const float mn0 = fmaxf(st.m[0], c0), mn1 = fmaxf(st.m[1], c1);
     const float al0 = fast_exp2(st.m[0] - mn0), al1 = fast_exp2(st.m[1] - mn1);
-    float r0 = 0.f, r1 = 0.f;
 #pragma unroll
     for (int i = 0; i < NT; ++i) {
         s[i][0] = fast_exp2(s[i][0] - mn0);
         s[i][1] = fast_exp2(s[i][1] - mn1);
         s[i][2] = fast_exp2(s[i][2] - mn0);
         s[i][3] = fast_exp2(s[i][3] - mn1);
+    }
+    float r0 = s[0][0] + s[0][2], r1 = s[0][1] + s[0][3];
+#pragma unroll
+    for (int i = 1; i < NT; ++i) {
         r0 += s[i][0] + s[i][2];
         r1 += s[i][1] + s[i][3];
     }
