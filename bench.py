@@ -691,10 +691,22 @@ def cpu_baseline(wl, cache, step, tables_h, lens_h, budget_s=15.0):
     per, b = _time_oracle_steps(wl, model, kc, vc, slots, S, 1)
     reps = max(1, min(int(budget_s / max(per, 1e-3)), 20))
     per, b = _time_oracle_steps(wl, model, kc, vc, slots, S, reps)
-    return {"value": round(b / per / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle", "seconds_per_step": round(per, 4),
-            "sample": f"full step ({S} sequences: cache write + decode), {reps} rep(s), fp64 C + OpenMP",
-            "cpu": _cpu_model()}
+    out = {"value": round(b / per / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+           "kind": "oracle", "seconds_per_step": round(per, 4),
+           "sample": f"full step ({S} sequences: cache write + decode), {reps} rep(s), fp64 C + OpenMP",
+           "cpu": _cpu_model()}
+    # the same oracle on one thread, over the first eighth of the sequences
+    threads = oracle.num_threads()
+    n1 = max(1, S // 8)
+    oracle.set_num_threads(1)
+    try:
+        per1, b1 = _time_oracle_steps(wl, model, kc, vc, slots, n1, 1)
+    finally:
+        oracle.set_num_threads(threads)
+    out["single_thread"] = {"value": round(b1 / per1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                            "seconds_per_step": round(per1, 4),
+                            "sample": f"first {n1} of {S} sequences (cache write + decode), 1 rep"}
+    return out
 
 
 def _cpu_model():

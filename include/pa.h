@@ -137,6 +137,17 @@ PA_API pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_
                          void *stream);
 
 /*
+ * Checked mode for copy pairs (host function, host pointer): PA_OK when every id of
+ * the num_pairs (src, dst) pairs in src_dst_pairs[2 * num_pairs] lies in
+ * [0, num_blocks), src != dst, no dst repeats and no block is both a source and a
+ * destination -- the conditions under which pa_copy_blocks's result does not depend
+ * on the order its pairs run in; PA_ERR_INVALID_ARG otherwise (also for negative
+ * counts or a null pointer with num_pairs > 0).  Reads the pairs only; launches
+ * nothing.  The host block manager only emits valid pairs.
+ */
+PA_API pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs, int32_t num_pairs, int32_t num_blocks);
+
+/*
  * Bytes of workspace pa_decode needs for a split (partitioned) context:
  * partials of num_seqs * num_q_heads * ceil(max_context_len / partition_size)
  * partitions (head_dim fp32 accumulators plus a running max and sum each), then

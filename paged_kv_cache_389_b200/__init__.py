@@ -47,6 +47,7 @@ def _load():
         "pa_status_string": (C.c_char_p, [C.c_int]),
         "pa_cache_write": (C.c_int, [vp, vp, vp, i32, vp, vp, desc, vp, vp]),
         "pa_copy_blocks": (C.c_int, [vp, vp, vp, i32, desc, vp, vp]),
+        "pa_check_copy_pairs": (C.c_int, [vp, i32, i32]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32]),
         "pa_decode_launches": (i32, [i32, i32, i32, i32]),
         "pa_decode": (C.c_int, [vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, i32, vp, sz, vp, desc,
@@ -86,7 +87,7 @@ def _load():
 _lib = _load()
 
 EXPORTED = (
-    "pa_abi_version", "pa_status_string", "pa_cache_write", "pa_copy_blocks",
+    "pa_abi_version", "pa_status_string", "pa_cache_write", "pa_copy_blocks", "pa_check_copy_pairs",
     "pa_decode_workspace_size", "pa_decode_launches", "pa_decode", "pa_append_decode", "pa_prefill_chunk",
     "pa_wait",
 )
@@ -179,6 +180,13 @@ def pa_copy_blocks(key_cache, value_cache, src_dst_pairs, err_flag=None, stream=
     _check(_lib.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(src_dst_pairs),
                                src_dst_pairs.shape[0], C.byref(d), _ptr(err_flag), _stream(stream)),
            "pa_copy_blocks")
+
+
+def pa_check_copy_pairs(pairs, num_blocks) -> int:
+    """Host-side check of copy pairs (int32 [P, 2], host memory): PA_OK or PA_ERR_INVALID_ARG."""
+    arr = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+    return int(_lib.pa_check_copy_pairs(arr.ctypes.data_as(C.c_void_p) if len(arr) else None, len(arr),
+                                        int(num_blocks)))
 
 
 def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, partition_size) -> int:

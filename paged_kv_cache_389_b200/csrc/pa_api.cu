@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdint>
 #include <thread>
+#include <vector>
 
 #include "pa_common.cuh"
 #include "pa_launch.h"
@@ -94,6 +95,24 @@ pa_status pa_cache_write(const void *key, const void *value, const int64_t *slot
     if (st != PA_OK || num_tokens == 0) return st;
     return from_cuda(launch_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache,
                                         *cache, err_flag, static_cast<cudaStream_t>(stream)));
+}
+
+pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs, int32_t num_pairs, int32_t num_blocks) {
+    if (num_pairs < 0 || num_blocks < 0) return PA_ERR_INVALID_ARG;
+    if (num_pairs == 0) return PA_OK;
+    if (!src_dst_pairs) return PA_ERR_INVALID_ARG;
+    // one byte per block: bit 0 = seen as a source, bit 1 = seen as a destination
+    std::vector<unsigned char> role((size_t)num_blocks, 0);
+    for (int32_t p = 0; p < num_pairs; ++p) {
+        const int32_t src = src_dst_pairs[2 * p], dst = src_dst_pairs[2 * p + 1];
+        if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks || src == dst)
+            return PA_ERR_INVALID_ARG;
+        if ((role[(size_t)dst] & 2u) || (role[(size_t)dst] & 1u) || (role[(size_t)src] & 2u))
+            return PA_ERR_INVALID_ARG;
+        role[(size_t)src] |= 1u;
+        role[(size_t)dst] |= 2u;
+    }
+    return PA_OK;
 }
 
 pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pairs,

@@ -5,6 +5,7 @@ import ctypes as C
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -121,3 +122,35 @@ def test_decode_launch_count(pa):
     assert pa.pa_decode_launches(4096, 128, pa.PA_FP8_E4M3, 512) == 2   # no shared-prefix groups
     assert pa.pa_decode_launches(8, 128, pa.PA_FP8_E4M3, 0) == 1
 
+
+
+def test_copy_pair_checked_mode(pa):
+    """pa_check_copy_pairs accepts independent pairs (one source may feed several
+    destinations) and rejects what would make pa_copy_blocks order dependent."""
+    ok, bad = pa.PA_OK, pa.PA_ERR_INVALID_ARG
+    assert pa.pa_check_copy_pairs(np.zeros((0, 2), np.int32), 8) == ok
+    assert pa.pa_check_copy_pairs([[0, 1], [0, 2], [0, 3], [5, 4]], 8) == ok
+    assert pa.pa_check_copy_pairs([[0, 1], [2, 1]], 8) == bad          # dst repeated
+    assert pa.pa_check_copy_pairs([[0, 1], [1, 2]], 8) == bad          # dst later a src
+    assert pa.pa_check_copy_pairs([[1, 2], [0, 1]], 8) == bad          # src 1 is a later dst
+    assert pa.pa_check_copy_pairs([[3, 3]], 8) == bad                  # src == dst
+    assert pa.pa_check_copy_pairs([[0, 8]], 8) == bad                  # out of range
+    assert pa.pa_check_copy_pairs([[-1, 2]], 8) == bad
+    L = pa._lib
+    assert L.pa_check_copy_pairs(None, 1, 8) == bad
+    assert L.pa_check_copy_pairs(None, -1, 8) == bad
+
+
+def test_block_manager_pairs_pass_the_checked_mode(pa):
+    """Copy-on-write pairs emitted by the host manager for forked siblings are always
+    independent (config 4's first step: 3 copies per parent)."""
+    import workloads
+    wl = workloads.make(4, mini=True)
+    bm = pa.BlockManager(wl.num_blocks, 16, wl.free_order)
+    workloads.replay(wl, bm, lambda k, v, s: None)
+    pairs = []
+    for s in wl.steps[0].seqs:
+        _, pr = bm.append_slots(s, 1)
+        pairs.extend(tuple(p) for p in pr)
+    assert len(pairs) > 0
+    assert pa.pa_check_copy_pairs(pairs, wl.num_blocks) == pa.PA_OK
