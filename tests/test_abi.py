@@ -154,3 +154,16 @@ def test_block_manager_pairs_pass_the_checked_mode(pa):
         pairs.extend(tuple(p) for p in pr)
     assert len(pairs) > 0
     assert pa.pa_check_copy_pairs(pairs, wl.num_blocks) == pa.PA_OK
+
+
+def test_fp8_pool_descriptor(pa):
+    """A torch.float8_e4m3fn pool maps to PA_FP8_E4M3 with its scales; its queries, outputs
+    and appended K/V are bf16."""
+    import torch
+    kc = torch.empty((4, 2, 16, 128), dtype=torch.float8_e4m3fn)
+    d = pa.cache_desc(kc, 0.5, 0.25)
+    assert (d.num_blocks, d.num_kv_heads, d.block_size, d.head_dim) == (4, 2, 16, 128)
+    assert d.dtype == pa.PA_FP8_E4M3 and d.k_scale == 0.5 and d.v_scale == 0.25
+    assert pa.io_dtype(kc) == torch.bfloat16
+    assert pa.io_dtype(torch.empty(1, dtype=torch.float32)) == torch.float32
+    assert pa.cache_desc(torch.empty((4, 2, 16, 64), dtype=torch.bfloat16)).dtype == pa.PA_BF16
