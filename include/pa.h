@@ -142,8 +142,9 @@ PA_API pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_
  * [0, num_blocks), src != dst, no dst repeats and no block is both a source and a
  * destination -- the conditions under which pa_copy_blocks's result does not depend
  * on the order its pairs run in; PA_ERR_INVALID_ARG otherwise (also for negative
- * counts or a null pointer with num_pairs > 0).  Reads the pairs only; launches
- * nothing.  The host block manager only emits valid pairs.
+ * counts or a null pointer with num_pairs > 0); PA_ERR_OOM when the host scratch
+ * of num_blocks bytes cannot be allocated.  Reads the pairs only; launches nothing.
+ * The host block manager only emits valid pairs.
  */
 PA_API pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs, int32_t num_pairs, int32_t num_blocks);
 

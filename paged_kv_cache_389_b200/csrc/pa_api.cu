@@ -102,7 +102,12 @@ pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs, int32_t num_pairs, i
     if (num_pairs == 0) return PA_OK;
     if (!src_dst_pairs) return PA_ERR_INVALID_ARG;
     // one byte per block: bit 0 = seen as a source, bit 1 = seen as a destination
-    std::vector<unsigned char> role((size_t)num_blocks, 0);
+    std::vector<unsigned char> role;
+    try {
+        role.assign((size_t)num_blocks, 0);
+    } catch (...) {
+        return PA_ERR_OOM;  // no exception crosses the C boundary
+    }
     for (int32_t p = 0; p < num_pairs; ++p) {
         const int32_t src = src_dst_pairs[2 * p], dst = src_dst_pairs[2 * p + 1];
         if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks || src == dst)
