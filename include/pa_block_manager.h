@@ -4,7 +4,9 @@
  * Host code (C++), not the hot path: it decides where each token's K/V goes and
  * produces the int32 block tables, the int64 slot mappings and the (src, dst)
  * copy-on-write pairs that pa_cache_write / pa_copy_blocks / pa_decode consume.
- * All pointers here are HOST pointers.  A manager is not thread-safe.
+ * All pointers here are HOST pointers.  A manager is not thread-safe.  No C++
+ * exception crosses this boundary: a failed host allocation inside a call returns
+ * PA_ERR_OOM, after which that manager's state is unspecified (destroy it).
  *
  * Sources (page title, section):
  *   devpress.csdn.net/amd vLLM v0.6.x teardown, 关键设计一 (BlockTable,

@@ -17,6 +17,7 @@
 #include <cstdint>
 #include <cstring>
 #include <list>
+#include <memory>
 #include <new>
 #include <unordered_map>
 #include <vector>
@@ -131,153 +132,175 @@ struct pa_block_manager {
     static int64_t blocks_for(int64_t tokens, int32_t bs) { return (tokens + bs - 1) / bs; }
 };
 
+// Host allocation failures (std::bad_alloc from the containers) must not cross the
+// C boundary: they become PA_ERR_OOM, and the manager's state is then unspecified.
+template <typename F>
+pa_status guarded(F &&f) {
+    try {
+        return f();
+    } catch (const std::bad_alloc &) {
+        return PA_ERR_OOM;
+    } catch (...) {
+        return PA_ERR_INVALID_ARG;
+    }
+}
+
 extern "C" {
 
 pa_status pa_bm_create(int32_t num_blocks, int32_t block_size, const int32_t *free_order,
                        pa_block_manager **out) {
     if (!out || num_blocks < 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
     *out = nullptr;
-    pa_block_manager *bm = new (std::nothrow) pa_block_manager;
-    if (!bm) return PA_ERR_OOM;
-    bm->num_blocks = num_blocks;
-    bm->block_size = block_size;
-    bm->refs.assign(num_blocks, 0);
-    bm->gen.assign(num_blocks, 0);
-    bm->cached.assign(num_blocks, 0);
-    bm->keys.resize(num_blocks);
-    bm->evict_pos.resize(num_blocks);
-    bm->on_evictable.assign(num_blocks, 0);
-    bm->free_stack.resize(num_blocks);
-    if (free_order) {
-        std::vector<char> seen(num_blocks, 0);
-        for (int32_t i = 0; i < num_blocks; ++i) {
-            int32_t b = free_order[i];
-            if (b < 0 || b >= num_blocks || seen[b]) {
-                delete bm;
-                return PA_ERR_INVALID_ARG;
+    return guarded([&]() -> pa_status {
+        std::unique_ptr<pa_block_manager> owner(new pa_block_manager);
+        pa_block_manager *bm = owner.get();
+        bm->num_blocks = num_blocks;
+        bm->block_size = block_size;
+        bm->refs.assign(num_blocks, 0);
+        bm->gen.assign(num_blocks, 0);
+        bm->cached.assign(num_blocks, 0);
+        bm->keys.resize(num_blocks);
+        bm->evict_pos.resize(num_blocks);
+        bm->on_evictable.assign(num_blocks, 0);
+        bm->free_stack.resize(num_blocks);
+        if (free_order) {
+            std::vector<char> seen(num_blocks, 0);
+            for (int32_t i = 0; i < num_blocks; ++i) {
+                int32_t b = free_order[i];
+                if (b < 0 || b >= num_blocks || seen[b]) return PA_ERR_INVALID_ARG;
+                seen[b] = 1;
+                bm->free_stack[i] = b;
             }
-            seen[b] = 1;
-            bm->free_stack[i] = b;
+        } else {
+            for (int32_t i = 0; i < num_blocks; ++i) bm->free_stack[i] = i;
         }
-    } else {
-        for (int32_t i = 0; i < num_blocks; ++i) bm->free_stack[i] = i;
-    }
-    *out = bm;
-    return PA_OK;
+        *out = owner.release();
+        return PA_OK;
+    });
 }
 
 void pa_bm_destroy(pa_block_manager *bm) { delete bm; }
 
 pa_status pa_bm_add_seq(pa_block_manager *bm, int64_t seq_id) {
-    if (!bm) return PA_ERR_INVALID_ARG;
-    if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
-    bm->seqs.emplace(seq_id, Sequence{});
-    return PA_OK;
+    return guarded([&]() -> pa_status {
+        if (!bm) return PA_ERR_INVALID_ARG;
+        if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+        bm->seqs.emplace(seq_id, Sequence{});
+        return PA_OK;
+    });
 }
 
 pa_status pa_bm_add_seq_tokens(pa_block_manager *bm, int64_t seq_id, const int32_t *tokens, int32_t n,
                                int64_t *slots_out, int32_t *num_cached_out) {
-    if (!bm || n < 0 || (n > 0 && !tokens)) return PA_ERR_INVALID_ARG;
-    if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
-    const int32_t bs = bm->block_size;
-    // Plan: the longest run of leading full blocks already cached.
-    std::vector<int32_t> hits;
-    int32_t parent = -1;
-    uint32_t pgen = 0;
-    int32_t hits_evictable = 0;
-    for (int64_t j = 0; j < n / bs; ++j) {
-        CacheKey k{parent, pgen, std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)};
-        const int32_t b = bm->lookup(k);
-        if (b < 0) break;
-        hits.push_back(b);
-        hits_evictable += bm->on_evictable[b] ? 1 : 0;
-        parent = b;
-        pgen = bm->gen[b];
-    }
-    const int64_t need = pa_block_manager::blocks_for(n, bs) - (int64_t)hits.size();
-    if (need > (int64_t)bm->available() - hits_evictable) return PA_ERR_OOM;
-    // Commit: reuse the hits, allocate the rest, index each new full block.
-    for (int32_t b : hits) bm->revive(b);
-    Sequence sq;
-    sq.blocks = hits;
-    int64_t k_out = 0;
-    for (int64_t i = (int64_t)hits.size() * bs; i < n; ++i) {
-        const int64_t offset = i % bs;
-        if (offset == 0) sq.blocks.push_back(bm->take());
-        if (slots_out) slots_out[k_out++] = (int64_t)sq.blocks.back() * bs + offset;
-        if (offset == bs - 1) {
-            const int64_t j = i / bs;
-            const int32_t par = j > 0 ? sq.blocks[j - 1] : -1;
-            bm->insert(sq.blocks[j], CacheKey{par, par >= 0 ? bm->gen[par] : 0u,
-                                              std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)});
+    return guarded([&]() -> pa_status {
+        if (!bm || n < 0 || (n > 0 && !tokens)) return PA_ERR_INVALID_ARG;
+        if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
+        const int32_t bs = bm->block_size;
+        // Plan: the longest run of leading full blocks already cached.
+        std::vector<int32_t> hits;
+        int32_t parent = -1;
+        uint32_t pgen = 0;
+        int32_t hits_evictable = 0;
+        for (int64_t j = 0; j < n / bs; ++j) {
+            CacheKey k{parent, pgen, std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)};
+            const int32_t b = bm->lookup(k);
+            if (b < 0) break;
+            hits.push_back(b);
+            hits_evictable += bm->on_evictable[b] ? 1 : 0;
+            parent = b;
+            pgen = bm->gen[b];
         }
-    }
-    sq.tokens = n;
-    bm->seqs.emplace(seq_id, std::move(sq));
-    if (num_cached_out) *num_cached_out = (int32_t)hits.size() * bs;
-    return PA_OK;
+        const int64_t need = pa_block_manager::blocks_for(n, bs) - (int64_t)hits.size();
+        if (need > (int64_t)bm->available() - hits_evictable) return PA_ERR_OOM;
+        // Commit: reuse the hits, allocate the rest, index each new full block.
+        for (int32_t b : hits) bm->revive(b);
+        Sequence sq;
+        sq.blocks = hits;
+        int64_t k_out = 0;
+        for (int64_t i = (int64_t)hits.size() * bs; i < n; ++i) {
+            const int64_t offset = i % bs;
+            if (offset == 0) sq.blocks.push_back(bm->take());
+            if (slots_out) slots_out[k_out++] = (int64_t)sq.blocks.back() * bs + offset;
+            if (offset == bs - 1) {
+                const int64_t j = i / bs;
+                const int32_t par = j > 0 ? sq.blocks[j - 1] : -1;
+                bm->insert(sq.blocks[j], CacheKey{par, par >= 0 ? bm->gen[par] : 0u,
+                                                  std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)});
+            }
+        }
+        sq.tokens = n;
+        bm->seqs.emplace(seq_id, std::move(sq));
+        if (num_cached_out) *num_cached_out = (int32_t)hits.size() * bs;
+        return PA_OK;
+    });
 }
 
 pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, int64_t *slots_out,
                              int32_t *cow_pairs_out, int32_t cow_capacity, int32_t *num_cow_out) {
-    if (!bm || n < 0) return PA_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
-    Sequence &sq = it->second;
-    const int32_t bs = bm->block_size;
-    // Plan first: fresh blocks for new block boundaries, plus one copy if the
-    // first token lands in a shared, partly filled last block.
-    const bool cow = n > 0 && (sq.tokens % bs) != 0 && bm->refs[sq.blocks.back()] > 1;
-    const int64_t fresh =
-        pa_block_manager::blocks_for(sq.tokens + n, bs) - pa_block_manager::blocks_for(sq.tokens, bs);
-    if (fresh + (cow ? 1 : 0) > (int64_t)bm->available()) return PA_ERR_OOM;
-    if (cow && cow_pairs_out && cow_capacity < 1) return PA_ERR_INVALID_ARG;
-    int32_t ncow = 0;
-    for (int32_t i = 0; i < n; ++i) {
-        const int64_t offset = sq.tokens % bs;
-        if (offset == 0) {
-            sq.blocks.push_back(bm->take());
-        } else if (bm->refs[sq.blocks.back()] > 1) {
-            const int32_t old_block = sq.blocks.back();
-            const int32_t new_block = bm->take();
-            if (cow_pairs_out) {
-                cow_pairs_out[2 * ncow] = old_block;
-                cow_pairs_out[2 * ncow + 1] = new_block;
+    return guarded([&]() -> pa_status {
+        if (!bm || n < 0) return PA_ERR_INVALID_ARG;
+        auto it = bm->seqs.find(seq_id);
+        if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+        Sequence &sq = it->second;
+        const int32_t bs = bm->block_size;
+        // Plan first: fresh blocks for new block boundaries, plus one copy if the
+        // first token lands in a shared, partly filled last block.
+        const bool cow = n > 0 && (sq.tokens % bs) != 0 && bm->refs[sq.blocks.back()] > 1;
+        const int64_t fresh =
+            pa_block_manager::blocks_for(sq.tokens + n, bs) - pa_block_manager::blocks_for(sq.tokens, bs);
+        if (fresh + (cow ? 1 : 0) > (int64_t)bm->available()) return PA_ERR_OOM;
+        if (cow && cow_pairs_out && cow_capacity < 1) return PA_ERR_INVALID_ARG;
+        int32_t ncow = 0;
+        for (int32_t i = 0; i < n; ++i) {
+            const int64_t offset = sq.tokens % bs;
+            if (offset == 0) {
+                sq.blocks.push_back(bm->take());
+            } else if (bm->refs[sq.blocks.back()] > 1) {
+                const int32_t old_block = sq.blocks.back();
+                const int32_t new_block = bm->take();
+                if (cow_pairs_out) {
+                    cow_pairs_out[2 * ncow] = old_block;
+                    cow_pairs_out[2 * ncow + 1] = new_block;
+                }
+                ++ncow;
+                if (bm->release(old_block)) bm->make_evictable(old_block);
+                sq.blocks.back() = new_block;
             }
-            ++ncow;
-            if (bm->release(old_block)) bm->make_evictable(old_block);
-            sq.blocks.back() = new_block;
+            if (slots_out) slots_out[i] = (int64_t)sq.blocks.back() * bs + offset;
+            ++sq.tokens;
         }
-        if (slots_out) slots_out[i] = (int64_t)sq.blocks.back() * bs + offset;
-        ++sq.tokens;
-    }
-    if (num_cow_out) *num_cow_out = ncow;
-    return PA_OK;
+        if (num_cow_out) *num_cow_out = ncow;
+        return PA_OK;
+    });
 }
 
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) {
-    if (!bm) return PA_ERR_INVALID_ARG;
-    auto p = bm->seqs.find(parent_id);
-    if (p == bm->seqs.end()) return PA_ERR_NOT_FOUND;
-    if (bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
-    Sequence child = p->second;  // copies token count and table
-    for (int32_t b : child.blocks) ++bm->refs[b];
-    bm->seqs.emplace(child_id, std::move(child));
-    return PA_OK;
+    return guarded([&]() -> pa_status {
+        if (!bm) return PA_ERR_INVALID_ARG;
+        auto p = bm->seqs.find(parent_id);
+        if (p == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+        if (bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
+        Sequence child = p->second;  // copies token count and table
+        for (int32_t b : child.blocks) ++bm->refs[b];
+        bm->seqs.emplace(child_id, std::move(child));
+        return PA_OK;
+    });
 }
 
 pa_status pa_bm_free_seq(pa_block_manager *bm, int64_t seq_id) {
-    if (!bm) return PA_ERR_INVALID_ARG;
-    auto it = bm->seqs.find(seq_id);
-    if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
-    // references drop in logical order; cached blocks reaching zero become
-    // evictable from the last to the first, so a prefix's tail goes before its head
-    std::vector<int32_t> to_evictable;
-    for (int32_t b : it->second.blocks)
-        if (bm->release(b)) to_evictable.push_back(b);
-    for (auto r = to_evictable.rbegin(); r != to_evictable.rend(); ++r) bm->make_evictable(*r);
-    bm->seqs.erase(it);
-    return PA_OK;
+    return guarded([&]() -> pa_status {
+        if (!bm) return PA_ERR_INVALID_ARG;
+        auto it = bm->seqs.find(seq_id);
+        if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+        // references drop in logical order; cached blocks reaching zero become
+        // evictable from the last to the first, so a prefix's tail goes before its head
+        std::vector<int32_t> to_evictable;
+        for (int32_t b : it->second.blocks)
+            if (bm->release(b)) to_evictable.push_back(b);
+        for (auto r = to_evictable.rbegin(); r != to_evictable.rend(); ++r) bm->make_evictable(*r);
+        bm->seqs.erase(it);
+        return PA_OK;
+    });
 }
 
 int64_t pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id) {
