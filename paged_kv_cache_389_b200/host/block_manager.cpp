@@ -35,25 +35,23 @@ struct CacheKey {
     int32_t parent = -1;     // physical block before this one in the prompt (-1: first)
     uint32_t parent_gen = 0;
     std::vector<int32_t> tokens;
-    bool operator==(const CacheKey &o) const {
-        return parent == o.parent && parent_gen == o.parent_gen && tokens == o.tokens;
-    }
 };
 
-uint64_t key_hash(const CacheKey &k) {
-    // FNV-1a over the key's 32-bit words
+// FNV-1a taken over 32-bit words (one xor and one multiply per word) with a final
+// xor-shift, over (parent, parent generation, token ids).  Collisions are harmless:
+// every hit is verified against the stored key.
+uint64_t key_hash(int32_t parent, uint32_t parent_gen, const int32_t *tokens, size_t n) {
     uint64_t h = 1469598103934665603ull;
     auto mix = [&](uint32_t w) {
-        for (int i = 0; i < 4; ++i) {
-            h ^= (w >> (8 * i)) & 0xffu;
-            h *= 1099511628211ull;
-        }
+        h ^= w;
+        h *= 1099511628211ull;
     };
-    mix((uint32_t)k.parent);
-    mix(k.parent_gen);
-    for (int32_t t : k.tokens) mix((uint32_t)t);
-    return h;
+    mix((uint32_t)parent);
+    mix(parent_gen);
+    for (size_t i = 0; i < n; ++i) mix((uint32_t)tokens[i]);
+    return h ^ (h >> 29);
 }
+uint64_t key_hash(const CacheKey &k) { return key_hash(k.parent, k.parent_gen, k.tokens.data(), k.tokens.size()); }
 
 }  // namespace
 
@@ -118,10 +116,15 @@ struct pa_block_manager {
         }
         ++refs[b];
     }
-    int32_t lookup(const CacheKey &k) const {
-        auto range = index.equal_range(key_hash(k));
-        for (auto it = range.first; it != range.second; ++it)
-            if (keys[it->second] == k) return it->second;
+    // cached block whose key is (parent, parent_gen, tokens[0..block_size)), or -1
+    int32_t lookup(int32_t parent, uint32_t parent_gen, const int32_t *tokens) const {
+        auto range = index.equal_range(key_hash(parent, parent_gen, tokens, (size_t)block_size));
+        for (auto it = range.first; it != range.second; ++it) {
+            const CacheKey &k = keys[it->second];
+            if (k.parent == parent && k.parent_gen == parent_gen && k.tokens.size() == (size_t)block_size &&
+                std::memcmp(k.tokens.data(), tokens, sizeof(int32_t) * (size_t)block_size) == 0)
+                return it->second;
+        }
         return -1;
     }
     void insert(int32_t b, CacheKey k) {
@@ -202,8 +205,7 @@ pa_status pa_bm_add_seq_tokens(pa_block_manager *bm, int64_t seq_id, const int32
         uint32_t pgen = 0;
         int32_t hits_evictable = 0;
         for (int64_t j = 0; j < n / bs; ++j) {
-            CacheKey k{parent, pgen, std::vector<int32_t>(tokens + j * bs, tokens + (j + 1) * bs)};
-            const int32_t b = bm->lookup(k);
+            const int32_t b = bm->lookup(parent, pgen, tokens + j * bs);
             if (b < 0) break;
             hits.push_back(b);
             hits_evictable += bm->on_evictable[b] ? 1 : 0;
