@@ -214,7 +214,7 @@ def run_ours(args):
         dev(k), dev(v), torch.from_numpy(s).cuda(), cache.key_cache, cache.value_cache, cache.err_flag))
     slots, pairs = cache.plan_append(step.seqs)
     assert len(pairs) == 0
-    max_blocks = max(cache.manager.num_seq_blocks(s) for s in step.seqs)
+    max_blocks = cache.manager.max_seq_blocks(step.seqs)
     tables_h, lens_h = cache.manager.build_tables(step.seqs, max_blocks)
     max_ctx = int(lens_h.max())
     # device-resident step inputs
@@ -469,7 +469,7 @@ def run_rows(reps, peaks, partition=PARTITION, groups=None):
         cache, dev = _setup(wl)
         st = wl.steps[0]
         cache.append(st.seqs, dev(st.k_new), dev(st.v_new))
-        mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+        mb = cache.manager.max_seq_blocks(st.seqs)
         t, l = cache.manager.build_tables(st.seqs, mb)
         ub, lb = step_bytes(wl, t, l)
         td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
@@ -492,7 +492,7 @@ def run_rows(reps, peaks, partition=PARTITION, groups=None):
         for st in wl.steps:
             h0 = time.perf_counter()
             slots, pairs = cache.plan_append(st.seqs)
-            mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+            mb = cache.manager.max_seq_blocks(st.seqs)
             t, l = cache.manager.build_tables(st.seqs, mb)
             host_s += time.perf_counter() - h0
             ub, _ = step_bytes(wl, t, l)
@@ -557,7 +557,7 @@ def run_rows(reps, peaks, partition=PARTITION, groups=None):
         kd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
         vd = dev(workloads.normal(rng, (S * kdraft, wl.num_kv_heads, wl.head_dim), "bf16"))
         cache.append(seqs, kd, vd, counts=[kdraft] * S)
-        mb = max(cache.manager.num_seq_blocks(s) for s in seqs)
+        mb = cache.manager.max_seq_blocks(seqs)
         t, l = cache.manager.build_tables(seqs, mb)
         td, ld = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda()
         qv = dev(workloads.normal(rng, (S, kdraft, wl.num_q_heads, wl.head_dim), "bf16"))
@@ -581,7 +581,7 @@ def run_rows(reps, peaks, partition=PARTITION, groups=None):
         st = wl.steps[0]
         slots, pairs = cache.plan_append(st.seqs)
         assert len(pairs) == 0
-        mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+        mb = cache.manager.max_seq_blocks(st.seqs)
         t, l = cache.manager.build_tables(st.seqs, mb)
         ub, lb = step_bytes(wl, t, l, kv_elem=1)
         cwb = cache_write_bytes(wl, len(st.seqs), kv_elem=1)
@@ -636,7 +636,7 @@ def run_rows(reps, peaks, partition=PARTITION, groups=None):
         wl = workloads.make(5)
         cache, dev = _setup(wl)
         st = wl.steps[0]
-        mb = max(cache.manager.num_seq_blocks(s) for s in st.seqs)
+        mb = cache.manager.max_seq_blocks(st.seqs)
         t, l = cache.manager.build_tables(st.seqs, mb)
         ub, lb = step_bytes(wl, t, l)
         td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)

@@ -85,6 +85,19 @@ PA_API pa_status pa_bm_add_seq(pa_block_manager *bm, int64_t seq_id);
 PA_API pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, int64_t *slots_out,
                              int32_t *cow_pairs_out, int32_t cow_capacity, int32_t *num_cow_out);
 
+/* One step for n distinct sequences in one call: appends counts[i] >= 0 tokens
+ * (counts NULL: one each) to seq_ids[i], in the order given -- the same result as
+ * n pa_bm_append_slots calls in that order.  slots_out (nullable, sum of counts
+ * entries) receives the slots sequence by sequence; cow_pairs_out (nullable, room
+ * for 2 * cow_capacity int32) the copy pairs in order, *num_cow_out (nullable)
+ * their count.  All or nothing: PA_ERR_OOM if the pool lacks the blocks for the
+ * whole step, PA_ERR_NOT_FOUND for an unknown id, PA_ERR_INVALID_ARG for a
+ * repeated id, a negative count or more pairs than cow_capacity -- and then
+ * nothing is changed. */
+PA_API pa_status pa_bm_append_step(pa_block_manager *bm, const int64_t *seq_ids, const int32_t *counts,
+                                   int32_t n, int64_t *slots_out, int32_t *cow_pairs_out,
+                                   int32_t cow_capacity, int32_t *num_cow_out);
+
 /* Child shares all of parent's blocks (their counts go up by one). */
 PA_API pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id);
 
@@ -94,6 +107,10 @@ PA_API pa_status pa_bm_free_seq(pa_block_manager *bm, int64_t seq_id);
 /* Number of tokens / blocks of a sequence (-1 if unknown). */
 PA_API int64_t pa_bm_num_tokens(const pa_block_manager *bm, int64_t seq_id);
 PA_API int32_t pa_bm_num_seq_blocks(const pa_block_manager *bm, int64_t seq_id);
+
+/* Longest block table among n sequences: the max_blocks pa_bm_build_tables needs
+ * (0 for n == 0; -1 for an unknown id or bad arguments). */
+PA_API int32_t pa_bm_max_seq_blocks(const pa_block_manager *bm, const int64_t *seq_ids, int32_t n);
 
 /* Copy a sequence's block table (its first `capacity` entries at most) into out;
  * *len_out (nullable) gets the table length. */

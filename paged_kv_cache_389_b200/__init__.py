@@ -61,10 +61,12 @@ def _load():
         "pa_bm_destroy": (None, [vp]),
         "pa_bm_add_seq": (C.c_int, [vp, i64]),
         "pa_bm_append_slots": (C.c_int, [vp, i64, i32, vp, vp, i32, C.POINTER(i32)]),
+        "pa_bm_append_step": (C.c_int, [vp, vp, vp, i32, vp, vp, i32, C.POINTER(i32)]),
         "pa_bm_fork": (C.c_int, [vp, i64, i64]),
         "pa_bm_free_seq": (C.c_int, [vp, i64]),
         "pa_bm_num_tokens": (i64, [vp, i64]),
         "pa_bm_num_seq_blocks": (i32, [vp, i64]),
+        "pa_bm_max_seq_blocks": (i32, [vp, vp, i32]),
         "pa_bm_block_table": (C.c_int, [vp, i64, vp, i32, C.POINTER(i32)]),
         "pa_bm_build_tables": (C.c_int, [vp, vp, i32, i32, vp, vp]),
         "pa_bm_refcount": (i32, [vp, i32]),
@@ -299,6 +301,23 @@ class BlockManager:
     def add_seq(self, seq: int):
         self._st(_lib.pa_bm_add_seq(self._h, int(seq)), f"add_seq({seq})")
 
+    def append_step(self, seqs, counts=None):
+        """One step for distinct sequences in one call (all or nothing): append counts[i]
+        tokens (default 1) to seqs[i] in order.  Returns (int64 slots [sum counts],
+        int32 copy pairs [P, 2])."""
+        ids = np.ascontiguousarray(seqs, dtype=np.int64)
+        cnt = None if counts is None else np.ascontiguousarray(counts, dtype=np.int32)
+        total = len(ids) if cnt is None else int(cnt.sum())
+        slots = np.empty(max(total, 1), dtype=np.int64)
+        pairs = np.empty((max(len(ids), 1), 2), dtype=np.int32)   # at most one copy per sequence
+        ncow = C.c_int32(0)
+        self._st(_lib.pa_bm_append_step(self._h, ids.ctypes.data_as(C.c_void_p),
+                                        None if cnt is None else cnt.ctypes.data_as(C.c_void_p), len(ids),
+                                        slots.ctypes.data_as(C.c_void_p), pairs.ctypes.data_as(C.c_void_p),
+                                        len(pairs), C.byref(ncow)),
+                 f"append_step({len(ids)} sequences)")
+        return slots[:total].copy(), pairs[:ncow.value].copy()
+
     def append_slots(self, seq: int, n: int):
         """Append n tokens; return (int64 slots [n], list of (src, dst) copy pairs)."""
         slots = np.empty(int(n), dtype=np.int64)
@@ -326,6 +345,14 @@ class BlockManager:
         n = int(_lib.pa_bm_num_seq_blocks(self._h, int(seq)))
         if n < 0:
             raise KeyError(seq)
+        return n
+
+    def max_seq_blocks(self, seqs) -> int:
+        """Longest block table among seqs (one call)."""
+        ids = np.ascontiguousarray(seqs, dtype=np.int64)
+        n = int(_lib.pa_bm_max_seq_blocks(self._h, ids.ctypes.data_as(C.c_void_p) if len(ids) else None, len(ids)))
+        if n < 0:
+            raise KeyError("unknown sequence id")
         return n
 
     def block_table(self, seq: int) -> list:

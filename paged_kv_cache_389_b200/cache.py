@@ -55,17 +55,10 @@ class PagedKVCache:
 
     # -- step pieces -----------------------------------------------------------
     def plan_append(self, seqs, counts=None):
-        """Allocate slots for ``counts[i]`` new tokens of each seq (default 1).
-        Returns (int64 slots [sum counts], int32 copy pairs [P, 2]) as numpy arrays."""
-        counts = [1] * len(seqs) if counts is None else counts
-        slots, pairs = [], []
-        for s, n in zip(seqs, counts):
-            sl, pr = self.manager.append_slots(s, n)
-            slots.append(sl)
-            pairs.extend(pr)
-        slots = np.concatenate(slots) if slots else np.zeros(0, np.int64)
-        pairs = np.asarray(pairs, dtype=np.int32).reshape(-1, 2)
-        return slots, pairs
+        """Allocate slots for ``counts[i]`` new tokens of each seq (default 1), all or
+        nothing, in one call to the host manager.  Returns (int64 slots [sum counts],
+        int32 copy pairs [P, 2]) as numpy arrays."""
+        return self.manager.append_step(seqs, counts)
 
     def write(self, k, v, slots, pairs=None, stream=None):
         """Copy-on-write copies (if any), then scatter k/v [T, Hkv, d] into ``slots``."""
@@ -86,7 +79,7 @@ class PagedKVCache:
         """int32 block tables [S, max_blocks] (padded with -1) and lengths, on the device."""
         torch = _torch()
         if max_blocks is None:
-            max_blocks = max(1, max(self.manager.num_seq_blocks(s) for s in seqs))
+            max_blocks = max(1, self.manager.max_seq_blocks(seqs))
         t, lens = self.manager.build_tables(seqs, max_blocks)
         return torch.from_numpy(t).to(self.device), torch.from_numpy(lens).to(self.device), int(lens.max(initial=0))
 

@@ -14,6 +14,7 @@
 // stay indexed on an evictable list (least recently freed first, and a freed
 // sequence's blocks tail first) and are reclaimed only when the free stack is
 // empty.
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <list>
@@ -276,6 +277,73 @@ pa_status pa_bm_append_slots(pa_block_manager *bm, int64_t seq_id, int32_t n, in
     });
 }
 
+pa_status pa_bm_append_step(pa_block_manager *bm, const int64_t *seq_ids, const int32_t *counts, int32_t n,
+                            int64_t *slots_out, int32_t *cow_pairs_out, int32_t cow_capacity,
+                            int32_t *num_cow_out) {
+    return guarded([&]() -> pa_status {
+        if (!bm || n < 0 || (n > 0 && !seq_ids) || cow_capacity < 0) return PA_ERR_INVALID_ARG;
+        const int32_t bs = bm->block_size;
+        // Plan the whole step in order: fresh blocks at block boundaries, and a copy
+        // when a token goes into a partly filled last block still shared at that
+        // moment (an earlier sibling's copy in this step drops the count by one).
+        std::unordered_map<int64_t, char> seen;
+        std::unordered_map<int32_t, int32_t> dropped;  // references given up by copies so far
+        seen.reserve((size_t)n * 2);
+        int64_t need = 0, cows = 0;
+        std::vector<Sequence *> seq(n);
+        for (int32_t i = 0; i < n; ++i) {
+            const int32_t c = counts ? counts[i] : 1;
+            if (c < 0) return PA_ERR_INVALID_ARG;
+            if (!seen.emplace(seq_ids[i], 1).second) return PA_ERR_INVALID_ARG;  // one entry per sequence
+            auto it = bm->seqs.find(seq_ids[i]);
+            if (it == bm->seqs.end()) return PA_ERR_NOT_FOUND;
+            seq[i] = &it->second;
+            const Sequence &sq = it->second;
+            if (c > 0 && sq.tokens % bs != 0) {
+                const int32_t last = sq.blocks.back();
+                auto d = dropped.find(last);
+                const int32_t refs_now = bm->refs[last] - (d == dropped.end() ? 0 : d->second);
+                if (refs_now > 1) {
+                    ++need;
+                    ++cows;
+                    ++dropped[last];
+                }
+            }
+            need += pa_block_manager::blocks_for(sq.tokens + c, bs) - pa_block_manager::blocks_for(sq.tokens, bs);
+        }
+        if (cow_pairs_out && cows > cow_capacity) return PA_ERR_INVALID_ARG;
+        if (need > (int64_t)bm->available()) return PA_ERR_OOM;
+        // Commit: the same steps as pa_bm_append_slots, sequence by sequence.
+        int64_t k = 0;
+        int32_t ncow = 0;
+        for (int32_t i = 0; i < n; ++i) {
+            Sequence &sq = *seq[i];
+            const int32_t c = counts ? counts[i] : 1;
+            for (int32_t t = 0; t < c; ++t) {
+                const int64_t offset = sq.tokens % bs;
+                if (offset == 0) {
+                    sq.blocks.push_back(bm->take());
+                } else if (bm->refs[sq.blocks.back()] > 1) {
+                    const int32_t old_block = sq.blocks.back();
+                    const int32_t new_block = bm->take();
+                    if (cow_pairs_out) {
+                        cow_pairs_out[2 * ncow] = old_block;
+                        cow_pairs_out[2 * ncow + 1] = new_block;
+                    }
+                    ++ncow;
+                    if (bm->release(old_block)) bm->make_evictable(old_block);
+                    sq.blocks.back() = new_block;
+                }
+                if (slots_out) slots_out[k] = (int64_t)sq.blocks.back() * bs + offset;
+                ++k;
+                ++sq.tokens;
+            }
+        }
+        if (num_cow_out) *num_cow_out = ncow;
+        return PA_OK;
+    });
+}
+
 pa_status pa_bm_fork(pa_block_manager *bm, int64_t parent_id, int64_t child_id) {
     return guarded([&]() -> pa_status {
         if (!bm) return PA_ERR_INVALID_ARG;
@@ -315,6 +383,17 @@ int32_t pa_bm_num_seq_blocks(const pa_block_manager *bm, int64_t seq_id) {
     if (!bm) return -1;
     auto it = bm->seqs.find(seq_id);
     return it == bm->seqs.end() ? -1 : (int32_t)it->second.blocks.size();
+}
+
+int32_t pa_bm_max_seq_blocks(const pa_block_manager *bm, const int64_t *seq_ids, int32_t n) {
+    if (!bm || n < 0 || (n > 0 && !seq_ids)) return -1;
+    int32_t mx = 0;
+    for (int32_t i = 0; i < n; ++i) {
+        auto it = bm->seqs.find(seq_ids[i]);
+        if (it == bm->seqs.end()) return -1;
+        mx = std::max(mx, (int32_t)it->second.blocks.size());
+    }
+    return mx;
 }
 
 pa_status pa_bm_block_table(const pa_block_manager *bm, int64_t seq_id, int32_t *out,
