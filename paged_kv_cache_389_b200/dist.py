@@ -7,6 +7,13 @@ KV pool and block manager for its sequences.  Sequences that share prefix blocks
 (forks, a common system prompt) must stay on one rank, since a block lives in one
 rank's pool; ``shard_ranges`` cuts only between such groups.
 
+The other split is tensor-parallel (chenxutan "vLLM 深度拆解" 3.4: each layer is cut
+across cards): every rank holds all sequences but only a contiguous range of kv
+heads, with their query heads (a GQA group is never split), and the same block
+tables (each rank's manager makes the same decisions).  Each rank decodes its heads
+with no exchange; ``gather_heads`` is the one collective, an all-gather of the
+output heads for a consumer that needs all of them on every rank.
+
 One process per GPU, ``torch.distributed`` for the plumbing (NCCL on GPUs, gloo
 for the CPU tests).  Timing across ranks takes the maximum device time.
 """
@@ -72,3 +79,41 @@ def max_over_ranks(value: float, device=None) -> float:
     t = torch.tensor([float(value)], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_kv_heads(num_kv_heads: int, world: int):
+    """Contiguous [start, end) kv-head ranges, one per rank, as even as possible (the
+    first num_kv_heads % world ranks take one more).  Rank r's query heads are
+    [start * g, end * g) with g = num_q_heads / num_kv_heads."""
+    if world < 1 or num_kv_heads < world:
+        raise ValueError("need 1 <= world <= num_kv_heads")
+    base, extra = divmod(num_kv_heads, world)
+    ranges, lo = [], 0
+    for r in range(world):
+        hi = lo + base + (1 if r < extra else 0)
+        ranges.append((lo, hi))
+        lo = hi
+    return ranges
+
+
+def gather_heads(out_local, kv_ranges, group_size: int, group=None):
+    """All-gather each rank's attention output [S, (end - start) * g, d] along the head
+    axis into [S, num_kv_heads * g, d] on every rank.  Uneven shards are padded to
+    the largest for the collective and trimmed after it."""
+    import torch
+    import torch.distributed as dist
+    world = dist.get_world_size(group)
+    if len(kv_ranges) != world:
+        raise ValueError("one kv-head range per rank")
+    widths = [(hi - lo) * group_size for lo, hi in kv_ranges]
+    rank = dist.get_rank(group)
+    if out_local.shape[1] != widths[rank]:
+        raise ValueError("local output does not match this rank's heads")
+    S, _, d = out_local.shape
+    wmax = max(widths)
+    padded = out_local.new_zeros((S, wmax, d))
+    padded[:, :widths[rank]] = out_local
+    parts = [torch.empty_like(padded) for _ in range(world)]
+    dist.all_gather(parts, padded.contiguous(), group=group)
+    return torch.cat([p[:, :w] for p, w in zip(parts, widths)], dim=1)
+

@@ -1,5 +1,6 @@
-"""Multi-rank host path on CPU (gloo, world size 2): sequence sharding, timing
-reduction, reassembly of per-rank outputs, and a rank that dies.
+"""Multi-rank host path on CPU (gloo, world size 2 and 3): sequence sharding, timing
+reduction, reassembly of per-rank outputs, the tensor-parallel kv-head split with its
+output all-gather, and a rank that dies.
 
 The decode path shards by sequence with no data-path exchange; here each rank
 runs the CPU oracle on its shard and the shards must reassemble bit-exactly into
@@ -134,3 +135,76 @@ def test_rank_that_dies_is_detected_on_the_host():
             p.kill()
     assert msg != "no error"
     assert procs[1].exitcode == 3
+
+
+def test_kv_head_shards_are_contiguous_and_even():
+    from paged_kv_cache_389_b200.dist import shard_kv_heads
+    for hkv in (1, 2, 8, 32):
+        for world in range(1, hkv + 1):
+            r = shard_kv_heads(hkv, world)
+            assert r[0][0] == 0 and r[-1][1] == hkv and all(a[1] == b[0] for a, b in zip(r, r[1:]))
+            w = [hi - lo for lo, hi in r]
+            assert max(w) - min(w) <= 1 and min(w) >= 1
+    with pytest.raises(ValueError):
+        shard_kv_heads(4, 5)
+
+
+def _tp_worker(rank, world, port, q):
+    """Tensor-parallel split: this rank stores only its kv heads (same tables as every
+    other rank), decodes them with the oracle, and all-gathers the output heads."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        import oracle
+        import workloads
+        from oracle.block_model import BlockManagerModel
+        from paged_kv_cache_389_b200.dist import gather_heads, shard_kv_heads
+        wl = workloads.make(3, mini=True)
+        g = wl.num_q_heads // wl.num_kv_heads
+        lo, hi = shard_kv_heads(wl.num_kv_heads, world)[rank]
+        model = BlockManagerModel(wl.num_blocks, wl.block_size, wl.free_order.tolist())
+        shape = list(wl.cache_shape())
+        shape[1] = hi - lo
+        kc = np.zeros(shape, wl.np_dtype)
+        vc = np.zeros_like(kc)
+        workloads.replay(wl, model, lambda k, v, s: oracle.cache_write(
+            np.ascontiguousarray(k[:, lo:hi]), np.ascontiguousarray(v[:, lo:hi]), s, kc, vc))
+        step = wl.steps[0]
+        mb = max(len(model.block_table(s)) for s in step.seqs)
+        t, l = model.build_tables(step.seqs, mb)
+        mine = oracle.decode(np.ascontiguousarray(step.q[:, lo * g:hi * g]), kc, vc, t, l, wl.scale)
+        full = gather_heads(torch.from_numpy(mine), shard_kv_heads(wl.num_kv_heads, world), g)
+        q.put((rank, full.numpy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_three_gloo_ranks_split_kv_heads_and_gather():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    world = 3                                        # 8 kv heads: 3 + 3 + 2 (uneven shards)
+    procs = [ctx.Process(target=_tp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=180) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    import oracle
+    import workloads
+    from oracle.block_model import BlockManagerModel
+    wl = workloads.make(3, mini=True)
+    model = BlockManagerModel(wl.num_blocks, wl.block_size, wl.free_order.tolist())
+    kc = np.zeros(wl.cache_shape(), wl.np_dtype)
+    vc = np.zeros_like(kc)
+    workloads.replay(wl, model, lambda k, v, s: oracle.cache_write(k, v, s, kc, vc))
+    step = wl.steps[0]
+    mb = max(len(model.block_table(s)) for s in step.seqs)
+    t, l = model.build_tables(step.seqs, mb)
+    want = oracle.decode(step.q, kc, vc, t, l, wl.scale)
+    for r in range(world):                          # every rank holds the whole, bit for bit
+        assert np.array_equal(out[r], want)
