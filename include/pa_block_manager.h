@@ -155,6 +155,18 @@ PA_API int32_t pa_bm_num_cached(const pa_block_manager *bm);
  * entries); returns its length (-1 if bm is NULL). */
 PA_API int32_t pa_bm_evictable(const pa_block_manager *bm, int32_t *out, int32_t capacity);
 
+/* Snapshot of a manager's whole state (free stack, counts, generations, sequences,
+ * prefix-cache keys and the evictable order) as bytes, for checkpoints and test
+ * reproducibility; a restored manager behaves exactly as the original from then on.
+ * pa_bm_snapshot_size: the bytes needed (0 for NULL).  pa_bm_snapshot: writes them
+ * into buf; *len_out (nullable) gets the size; PA_ERR_INVALID_ARG if capacity is
+ * too small.  pa_bm_restore: a new manager from a snapshot of this format version;
+ * PA_ERR_INVALID_ARG for a truncated, foreign or out-of-range buffer (structure and
+ * bounds are checked, not that counts match the tables). */
+PA_API size_t pa_bm_snapshot_size(const pa_block_manager *bm);
+PA_API pa_status pa_bm_snapshot(const pa_block_manager *bm, void *buf, size_t capacity, size_t *len_out);
+PA_API pa_status pa_bm_restore(const void *buf, size_t len, pa_block_manager **out);
+
 #ifdef __cplusplus
 }
 #endif

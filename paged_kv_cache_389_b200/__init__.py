@@ -78,6 +78,9 @@ def _load():
         "pa_bm_num_evictable": (i32, [vp]),
         "pa_bm_num_cached": (i32, [vp]),
         "pa_bm_evictable": (i32, [vp, vp, i32]),
+        "pa_bm_snapshot_size": (sz, [vp]),
+        "pa_bm_snapshot": (C.c_int, [vp, vp, sz, C.POINTER(sz)]),
+        "pa_bm_restore": (C.c_int, [vp, sz, C.POINTER(vp)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -284,6 +287,26 @@ class BlockManager:
         self._h = h
         self.num_blocks = int(num_blocks)
         self.block_size = int(block_size)
+
+    def snapshot(self) -> bytes:
+        """The manager's whole state as bytes (pa_bm_snapshot)."""
+        n = int(_lib.pa_bm_snapshot_size(self._h))
+        buf = (C.c_ubyte * max(n, 1))()
+        got = C.c_size_t(0)
+        _check(_lib.pa_bm_snapshot(self._h, buf, n, C.byref(got)), "pa_bm_snapshot")
+        return bytes(buf[:got.value])
+
+    @classmethod
+    def restore(cls, data: bytes) -> "BlockManager":
+        """A new manager from snapshot() bytes (pa_bm_restore)."""
+        raw = bytes(data)
+        h = C.c_void_p()
+        _check(_lib.pa_bm_restore(raw, len(raw), C.byref(h)), "pa_bm_restore")
+        self = cls.__new__(cls)
+        self._h = h
+        self.num_blocks = int(_lib.pa_bm_num_blocks(h))
+        self.block_size = BLOCK_SIZE if len(raw) < 16 else int.from_bytes(raw[12:16], "little", signed=True)
+        return self
 
     def __del__(self):
         h = getattr(self, "_h", None)

@@ -473,3 +473,184 @@ int64_t pa_bm_tokens_stored(const pa_block_manager *bm) {
 }
 
 }  // extern "C"
+
+// ---- snapshot / restore ---------------------------------------------------------
+// Byte format (host byte order): "PABM", u32 version 1, i32 num_blocks, i32 block_size,
+// u32 n + i32[n] free stack (bottom first), i32[num_blocks] counts, u32[num_blocks]
+// generations, u32 n + per sequence in ascending id (i64 id, i64 tokens, u32 k, i32[k]
+// blocks), u32 n + per cached block in ascending id (i32 block, i32 parent, u32 parent
+// generation, u32 k, i32[k] tokens), u32 n + i32[n] evictable list (next reclaimed first).
+
+namespace {
+
+struct Writer {
+    unsigned char *p;
+    size_t cap, len = 0;
+    template <typename T>
+    void put(const T &v) {
+        if (p && len + sizeof(T) <= cap) std::memcpy(p + len, &v, sizeof(T));
+        len += sizeof(T);
+    }
+    void put_ids(const int32_t *v, size_t n) {
+        if (p && len + 4 * n <= cap && n) std::memcpy(p + len, v, 4 * n);
+        len += 4 * n;
+    }
+};
+
+struct Reader {
+    const unsigned char *p;
+    size_t len, at = 0;
+    bool ok = true;
+    template <typename T>
+    T get() {
+        T v{};
+        if (at + sizeof(T) > len) {
+            ok = false;
+            return v;
+        }
+        std::memcpy(&v, p + at, sizeof(T));
+        at += sizeof(T);
+        return v;
+    }
+    bool get_ids(std::vector<int32_t> &v, size_t n) {
+        if (n > (len - at) / 4) return ok = false;
+        v.resize(n);
+        if (n) std::memcpy(v.data(), p + at, 4 * n);
+        at += 4 * n;
+        return true;
+    }
+};
+
+constexpr uint32_t kSnapshotVersion = 1;
+
+size_t write_snapshot(const pa_block_manager &bm, unsigned char *buf, size_t cap) {
+    Writer w{buf, cap};
+    uint32_t magic;
+    std::memcpy(&magic, "PABM", 4);
+    w.put(magic);
+    w.put(kSnapshotVersion);
+    w.put(bm.num_blocks);
+    w.put(bm.block_size);
+    w.put((uint32_t)bm.free_stack.size());
+    w.put_ids(bm.free_stack.data(), bm.free_stack.size());
+    w.put_ids(bm.refs.data(), bm.refs.size());
+    w.put_ids(reinterpret_cast<const int32_t *>(bm.gen.data()), bm.gen.size());
+    std::vector<int64_t> ids;
+    ids.reserve(bm.seqs.size());
+    for (const auto &kv : bm.seqs) ids.push_back(kv.first);
+    std::sort(ids.begin(), ids.end());
+    w.put((uint32_t)ids.size());
+    for (int64_t id : ids) {
+        const Sequence &sq = bm.seqs.at(id);
+        w.put(id);
+        w.put(sq.tokens);
+        w.put((uint32_t)sq.blocks.size());
+        w.put_ids(sq.blocks.data(), sq.blocks.size());
+    }
+    uint32_t ncached = 0;
+    for (int32_t b = 0; b < bm.num_blocks; ++b) ncached += bm.cached[b] ? 1u : 0u;
+    w.put(ncached);
+    for (int32_t b = 0; b < bm.num_blocks; ++b) {
+        if (!bm.cached[b]) continue;
+        const CacheKey &k = bm.keys[b];
+        w.put(b);
+        w.put(k.parent);
+        w.put(k.parent_gen);
+        w.put((uint32_t)k.tokens.size());
+        w.put_ids(k.tokens.data(), k.tokens.size());
+    }
+    w.put((uint32_t)bm.evictable.size());
+    for (int32_t b : bm.evictable) w.put(b);
+    return w.len;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t pa_bm_snapshot_size(const pa_block_manager *bm) {
+    if (!bm) return 0;
+    try {
+        return write_snapshot(*bm, nullptr, 0);
+    } catch (...) {
+        return 0;
+    }
+}
+
+pa_status pa_bm_snapshot(const pa_block_manager *bm, void *buf, size_t capacity, size_t *len_out) {
+    return guarded([&]() -> pa_status {
+        if (!bm || (capacity > 0 && !buf)) return PA_ERR_INVALID_ARG;
+        const size_t need = write_snapshot(*bm, nullptr, 0);
+        if (len_out) *len_out = need;
+        if (capacity < need) return PA_ERR_INVALID_ARG;
+        write_snapshot(*bm, static_cast<unsigned char *>(buf), capacity);
+        return PA_OK;
+    });
+}
+
+pa_status pa_bm_restore(const void *buf, size_t len, pa_block_manager **out) {
+    if (!out || (len > 0 && !buf)) return PA_ERR_INVALID_ARG;
+    *out = nullptr;
+    return guarded([&]() -> pa_status {
+        Reader r{static_cast<const unsigned char *>(buf), len};
+        const uint32_t magic = r.get<uint32_t>();
+        uint32_t want_magic;
+        std::memcpy(&want_magic, "PABM", 4);
+        if (!r.ok || magic != want_magic || r.get<uint32_t>() != kSnapshotVersion) return PA_ERR_INVALID_ARG;
+        const int32_t nb = r.get<int32_t>(), bs = r.get<int32_t>();
+        if (!r.ok || nb < 0 || bs <= 0) return PA_ERR_INVALID_ARG;
+        std::unique_ptr<pa_block_manager> owner(new pa_block_manager);
+        pa_block_manager &bm = *owner;
+        bm.num_blocks = nb;
+        bm.block_size = bs;
+        auto in_pool = [&](int32_t b) { return b >= 0 && b < nb; };
+        std::vector<int32_t> tmp;
+        if (!r.get_ids(bm.free_stack, r.get<uint32_t>()) || bm.free_stack.size() > (size_t)nb) return PA_ERR_INVALID_ARG;
+        for (int32_t b : bm.free_stack)
+            if (!in_pool(b)) return PA_ERR_INVALID_ARG;
+        if (!r.get_ids(bm.refs, (size_t)nb) || !r.get_ids(tmp, (size_t)nb)) return PA_ERR_INVALID_ARG;
+        bm.gen.assign(tmp.begin(), tmp.end());
+        for (int32_t c : bm.refs)
+            if (c < 0) return PA_ERR_INVALID_ARG;
+        const uint32_t nseq = r.get<uint32_t>();
+        for (uint32_t i = 0; r.ok && i < nseq; ++i) {
+            const int64_t id = r.get<int64_t>();
+            Sequence sq;
+            sq.tokens = r.get<int64_t>();
+            if (!r.ok || !r.get_ids(sq.blocks, r.get<uint32_t>())) return PA_ERR_INVALID_ARG;
+            for (int32_t b : sq.blocks)
+                if (!in_pool(b)) return PA_ERR_INVALID_ARG;
+            if (sq.tokens < 0 || pa_block_manager::blocks_for(sq.tokens, bs) != (int64_t)sq.blocks.size())
+                return PA_ERR_INVALID_ARG;
+            if (!bm.seqs.emplace(id, std::move(sq)).second) return PA_ERR_INVALID_ARG;
+        }
+        bm.cached.assign(nb, 0);
+        bm.keys.resize(nb);
+        bm.evict_pos.resize(nb);
+        bm.on_evictable.assign(nb, 0);
+        const uint32_t ncached = r.get<uint32_t>();
+        for (uint32_t i = 0; r.ok && i < ncached; ++i) {
+            const int32_t b = r.get<int32_t>();
+            CacheKey k;
+            k.parent = r.get<int32_t>();
+            k.parent_gen = r.get<uint32_t>();
+            if (!r.ok || !r.get_ids(k.tokens, r.get<uint32_t>())) return PA_ERR_INVALID_ARG;
+            if (!in_pool(b) || bm.cached[b] || (k.parent != -1 && !in_pool(k.parent)) ||
+                k.tokens.size() != (size_t)bs)
+                return PA_ERR_INVALID_ARG;
+            bm.insert(b, std::move(k));
+        }
+        const uint32_t nev = r.get<uint32_t>();
+        for (uint32_t i = 0; r.ok && i < nev; ++i) {
+            const int32_t b = r.get<int32_t>();
+            if (!r.ok || !in_pool(b) || !bm.cached[b] || bm.on_evictable[b] || bm.refs[b] != 0)
+                return PA_ERR_INVALID_ARG;
+            bm.make_evictable(b);
+        }
+        if (!r.ok || r.at != len) return PA_ERR_INVALID_ARG;
+        *out = owner.release();
+        return PA_OK;
+    });
+}
+
+}  // extern "C"
