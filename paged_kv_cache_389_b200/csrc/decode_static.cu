@@ -15,6 +15,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "pa_trace.h"
 #include "pa_common.cuh"
 #include "pa_launch.h"
 
@@ -48,6 +49,7 @@ extern "C" pa_status pa_decode_static_scratch(
     int32_t max_blocks_per_seq, const int32_t *context_lens, int32_t max_context_len,
     int32_t num_seqs, int32_t num_q_heads, float scale, int32_t partition_size, void *out,
     const pa_cache_desc *cache, int32_t *err_flag, void *stream) {
+    const pa::NvtxRange nvtx_range("pa_decode_static_scratch");
     if (!cache || partition_size < 0) return PA_ERR_INVALID_ARG;
     const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, cache->head_dim,
                                                  max_context_len, partition_size);

@@ -6,6 +6,7 @@
 #include <thread>
 #include <vector>
 
+#include "pa_trace.h"
 #include "pa_common.cuh"
 #include "pa_launch.h"
 
@@ -91,6 +92,7 @@ pa_status check_cache_write(const void *key, const void *value, const int64_t *s
 pa_status pa_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
                          int32_t num_tokens, void *key_cache, void *value_cache,
                          const pa_cache_desc *cache, int32_t *err_flag, void *stream) {
+    const NvtxRange nvtx_range("pa_cache_write");
     const pa_status st = check_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache, cache);
     if (st != PA_OK || num_tokens == 0) return st;
     return from_cuda(launch_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache,
@@ -123,6 +125,7 @@ pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs, int32_t num_pairs, i
 pa_status pa_copy_blocks(void *key_cache, void *value_cache, const int32_t *src_dst_pairs,
                          int32_t num_pairs, const pa_cache_desc *cache, int32_t *err_flag,
                          void *stream) {
+    const NvtxRange nvtx_range("pa_copy_blocks");
     pa_status st = check_cache(cache);
     if (st != PA_OK) return st;
     if (num_pairs < 0) return PA_ERR_INVALID_ARG;
@@ -220,6 +223,7 @@ pa_status pa_decode(const void *query, const void *key_cache, const void *value_
                     int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
                     size_t workspace_bytes, void *out, const pa_cache_desc *cache,
                     int32_t *err_flag, void *stream) {
+    const NvtxRange nvtx_range("pa_decode");
     DecodeLaunch a;
     const pa_status st = prepare_decode(query, key_cache, value_cache, block_tables, max_blocks_per_seq,
                                         context_lens, max_context_len, num_seqs, num_q_heads, scale,
@@ -235,6 +239,7 @@ pa_status pa_append_decode(const void *key, const void *value, const int64_t *sl
                            int32_t num_q_heads, float scale, int32_t partition_size, void *workspace,
                            size_t workspace_bytes, void *out, const pa_cache_desc *cache,
                            int32_t *err_flag, void *stream) {
+    const NvtxRange nvtx_range("pa_append_decode");
     pa_status st = check_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache, cache);
     if (st != PA_OK) return st;
     DecodeLaunch a;
@@ -259,6 +264,7 @@ pa_status pa_prefill_chunk(const void *query, const void *key_cache, const void 
                            int32_t num_seqs, int32_t max_chunk, int32_t num_q_heads, float scale,
                            void *out, const pa_cache_desc *cache, int32_t *err_flag,
                            void *stream) {
+    const NvtxRange nvtx_range("pa_prefill_chunk");
     pa_status st = check_cache(cache);
     if (st != PA_OK) return st;
     st = check_group(num_q_heads, cache->num_kv_heads);
@@ -291,6 +297,7 @@ pa_status pa_prefill_chunk(const void *query, const void *key_cache, const void 
 }
 
 pa_status pa_wait(void *stream, const int32_t *err_flag, int32_t timeout_ms, int32_t *flag_out) {
+    const NvtxRange nvtx_range("pa_wait");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaEvent_t ev = nullptr;
     if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return PA_ERR_CUDA;
