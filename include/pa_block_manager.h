@@ -128,6 +128,7 @@ PA_API pa_status pa_bm_build_tables(const pa_block_manager *bm, const int64_t *s
 PA_API int32_t pa_bm_refcount(const pa_block_manager *bm, int32_t block);
 PA_API int32_t pa_bm_num_free(const pa_block_manager *bm);
 PA_API int32_t pa_bm_num_blocks(const pa_block_manager *bm);
+PA_API int32_t pa_bm_block_size(const pa_block_manager *bm);   /* tokens per block (-1 for NULL) */
 
 /* Copy the free stack, bottom first (the next allocation takes the last entry);
  * returns its length.  out may be NULL to query the length. */

@@ -72,6 +72,7 @@ def _load():
         "pa_bm_refcount": (i32, [vp, i32]),
         "pa_bm_num_free": (i32, [vp]),
         "pa_bm_num_blocks": (i32, [vp]),
+        "pa_bm_block_size": (i32, [vp]),
         "pa_bm_free_stack": (i32, [vp, vp, i32]),
         "pa_bm_tokens_stored": (i64, [vp]),
         "pa_bm_add_seq_tokens": (C.c_int, [vp, i64, vp, i32, vp, C.POINTER(i32)]),
@@ -305,7 +306,7 @@ class BlockManager:
         self = cls.__new__(cls)
         self._h = h
         self.num_blocks = int(_lib.pa_bm_num_blocks(h))
-        self.block_size = BLOCK_SIZE if len(raw) < 16 else int.from_bytes(raw[12:16], "little", signed=True)
+        self.block_size = int(_lib.pa_bm_block_size(h))
         return self
 
     def __del__(self):

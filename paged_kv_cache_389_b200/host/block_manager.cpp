@@ -438,6 +438,7 @@ int32_t pa_bm_num_free(const pa_block_manager *bm) {
 }
 
 int32_t pa_bm_num_blocks(const pa_block_manager *bm) { return bm ? bm->num_blocks : -1; }
+int32_t pa_bm_block_size(const pa_block_manager *bm) { return bm ? bm->block_size : -1; }
 
 int32_t pa_bm_num_evictable(const pa_block_manager *bm) {
     return bm ? (int32_t)bm->evictable.size() : -1;
