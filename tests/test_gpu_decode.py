@@ -293,6 +293,19 @@ def test_append_decode_one_call(cid, part):
     assert ts.err_flag() == 0
 
 
+def test_append_decode_full_size_in_the_timed_configuration():
+    """The benchmark's timed step itself: the GQA-8B prefix-sharing workload at full size,
+    one pa_append_decode call at 512-token partitions; pools bit-exact, rows sampled."""
+    wl = workloads.make(3)
+    ts = TwoSided(wl)
+    step = wl.steps[0]
+    got = ts.append_decode_step(step, 512)
+    assert ts.pools_equal(), "pools differ after the one-call write"
+    rows = np.sort(np.random.default_rng(7).choice(len(step.seqs), 48, replace=False))
+    check_close(got[rows], ts.oracle_decode(step, rows), "bf16", "append+decode full size, partition 512")
+    assert ts.err_flag() == 0
+
+
 def test_append_decode_matches_two_calls_bitwise():
     """Same kernels, same order of arithmetic: one call and two calls agree bit for bit."""
     wl = workloads.make(3, mini=True)
