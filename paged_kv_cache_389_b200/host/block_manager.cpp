@@ -565,6 +565,36 @@ size_t write_snapshot(const pa_block_manager &bm, unsigned char *buf, size_t cap
     return w.len;
 }
 
+// Cross-checks of a parsed snapshot, so that a restored manager can never hand a
+// block that a sequence still holds to another one:
+//  * each block's count equals the number of table entries naming it;
+//  * every block is in exactly one state: free (on the free stack once, count 0,
+//    not in the prefix index), evictable (indexed, count 0, on the evictable
+//    list), or held (count > 0).
+bool consistent(const pa_block_manager &bm) {
+    const size_t nb = (size_t)bm.num_blocks;
+    std::vector<int64_t> held(nb, 0);
+    for (const auto &kv : bm.seqs)
+        for (int32_t b : kv.second.blocks) ++held[(size_t)b];
+    std::vector<char> on_free(nb, 0);
+    for (int32_t b : bm.free_stack) {
+        if (on_free[(size_t)b]) return false;  // listed twice
+        on_free[(size_t)b] = 1;
+    }
+    for (size_t b = 0; b < nb; ++b) {
+        if (held[b] != bm.refs[b]) return false;
+        const bool is_free = on_free[b] != 0, is_evictable = bm.on_evictable[b] != 0;
+        if (bm.refs[b] > 0) {
+            if (is_free || is_evictable) return false;
+        } else if (is_free == is_evictable) {
+            return false;  // a count-0 block must be free or evictable, not both or neither
+        } else if (is_free && bm.cached[b]) {
+            return false;  // a free block is not in the prefix index
+        }
+    }
+    return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -649,6 +679,7 @@ pa_status pa_bm_restore(const void *buf, size_t len, pa_block_manager **out) {
             bm.make_evictable(b);
         }
         if (!r.ok || r.at != len) return PA_ERR_INVALID_ARG;
+        if (!consistent(bm)) return PA_ERR_INVALID_ARG;
         *out = owner.release();
         return PA_OK;
     });

@@ -112,3 +112,86 @@ def test_malformed_snapshots_are_refused(pa):
             pa.BlockManager.restore(data)
         assert e.value.status == pa.PA_ERR_INVALID_ARG
     assert pa.BlockManager.restore(good).snapshot() == good
+
+
+# ---- cross-checked restore: one malformed snapshot per consistency rule --------
+def _parse(data):
+    """Split a version-1 snapshot into its fields (layout of pa_bm_snapshot)."""
+    at = 0
+
+    def take(fmt):
+        nonlocal at
+        v = struct.unpack_from("<" + fmt, data, at)
+        at += struct.calcsize("<" + fmt)
+        return v
+
+    magic, ver, nb, bs = take("4sIii")
+    (nfree,) = take("I")
+    free = list(take(f"{nfree}i")) if nfree else []
+    refs = list(take(f"{nb}i"))
+    gen = list(take(f"{nb}I"))
+    (nseq,) = take("I")
+    seqs = []
+    for _ in range(nseq):
+        sid, tokens, n = take("qqI")
+        seqs.append([sid, tokens, list(take(f"{n}i")) if n else []])
+    (ncached,) = take("I")
+    cached = []
+    for _ in range(ncached):
+        b, parent, pgen, n = take("iiII")
+        cached.append([b, parent, pgen, list(take(f"{n}i"))])
+    (nev,) = take("I")
+    ev = list(take(f"{nev}i")) if nev else []
+    assert at == len(data)
+    return dict(head=(magic, ver, nb, bs), free=free, refs=refs, gen=gen, seqs=seqs, cached=cached, ev=ev)
+
+
+def _pack(f):
+    out = struct.pack("<4sIii", *f["head"])
+    out += struct.pack("<I", len(f["free"])) + struct.pack(f"<{len(f['free'])}i", *f["free"])
+    nb = f["head"][2]
+    out += struct.pack(f"<{nb}i", *f["refs"]) + struct.pack(f"<{nb}I", *f["gen"])
+    out += struct.pack("<I", len(f["seqs"]))
+    for sid, tokens, blocks in f["seqs"]:
+        out += struct.pack("<qqI", sid, tokens, len(blocks)) + struct.pack(f"<{len(blocks)}i", *blocks)
+    out += struct.pack("<I", len(f["cached"]))
+    for b, parent, pgen, toks in f["cached"]:
+        out += struct.pack("<iiII", b, parent, pgen, len(toks)) + struct.pack(f"<{len(toks)}i", *toks)
+    out += struct.pack("<I", len(f["ev"])) + struct.pack(f"<{len(f['ev'])}i", *f["ev"])
+    return out
+
+
+def test_inconsistent_snapshots_are_refused(pa):
+    """pa_bm_restore rebuilds every block's count from the tables and requires each
+    block to be exactly one of free, evictable or held; a snapshot that breaks this
+    would let take() hand a live block to a second sequence."""
+    import copy
+    m = pa.BlockManager(32, 16)
+    m.add_seq_tokens(0, list(range(40)))      # 3 blocks, 2 of them indexed
+    m.fork(0, 1)                              # counts 2
+    m.add_seq_tokens(2, [7] * 33)             # 3 blocks, 2 indexed
+    m.free(2)                                 # 2 evictable, 1 free
+    m.add_seq(3)
+    m.append_slots(3, 5)
+    good = m.snapshot()
+    f = _parse(good)
+    assert _pack(f) == good                   # the test's own parser round-trips
+    assert len(f["ev"]) == 2 and len(f["free"]) >= 3
+    held = f["seqs"][0][2][0]
+    cases = {}
+    g = copy.deepcopy(f); g["free"][-1] = g["free"][-2]; cases["free stack lists a block twice"] = g
+    g = copy.deepcopy(f); g["free"][-1] = held; cases["a held block on the free stack"] = g
+    g = copy.deepcopy(f); g["refs"][held] += 1; cases["count above the tables holding it"] = g
+    g = copy.deepcopy(f); g["refs"][held] -= 1; cases["count below the tables holding it"] = g
+    g = copy.deepcopy(f); g["free"].pop(0); cases["a count-0 block neither free nor evictable"] = g
+    g = copy.deepcopy(f); g["ev"].pop(0); cases["an indexed count-0 block off the evictable list"] = g
+    g = copy.deepcopy(f); g["free"].append(g["ev"][0]); cases["an evictable block also free"] = g
+    g = copy.deepcopy(f)
+    ev0 = g["ev"].pop(0)
+    g["free"].append(ev0)
+    cases["an indexed block on the free stack"] = g
+    for what, bad in cases.items():
+        with pytest.raises(pa.PAError) as e:
+            pa.BlockManager.restore(_pack(bad))
+        assert e.value.status == pa.PA_ERR_INVALID_ARG, what
+    assert pa.BlockManager.restore(good).snapshot() == good
