@@ -237,6 +237,9 @@ PA_API pa_status pa_append_decode(const void *key, const void *value, const int6
  * the library holds that array until the process exits.
  * The first call on a device looks up the array's device address (with that
  * device current); make it before any stream capture.  No allocation happens.
+ * The address is kept for the life of the process: after cudaDeviceReset (or
+ * anything else that destroys the device's primary context) the process must be
+ * restarted before this entry point is called again on that device.
  * All calls share the one array and it keeps the last call's contents; nothing in
  * it needs to start at zero.  Calls whose kernels overlap on the GPU (different
  * streams, no ordering between them) race on the array and give wrong results:
@@ -283,6 +286,20 @@ PA_API pa_status pa_prefill_chunk(const void *query, const void *key_cache, cons
  * stream capture.
  */
 PA_API pa_status pa_wait(void *stream, const int32_t *err_flag, int32_t timeout_ms, int32_t *flag_out);
+
+/*
+ * Bound, in nanoseconds, of every wait inside the kernels launched from now on by
+ * this process (mbarrier hand-overs between the warps of a CTA); 0 restores the
+ * default of one second.  Returns the previous bound.  A wait that runs out sets
+ * PA_DEVERR_TIMEOUT in *err_flag, and the kernel stops its work, waits (with the
+ * default bound) for the copies and tensor-core operations it has in flight,
+ * releases its tensor memory and returns; the outputs of that call are then
+ * unspecified and later calls are unaffected.  It exists to exercise that path:
+ * a bound of a few nanoseconds makes ordinary waits run out.  Not a per-call or
+ * per-thread setting: it applies to launches from every host thread.
+ * Source: none on the pages (failure handling of this library).
+ */
+PA_API uint64_t pa_set_wait_timeout_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

@@ -57,6 +57,7 @@ def _load():
         "pa_prefill_chunk": (C.c_int, [vp, vp, vp, vp, i32, vp, vp, i32, i32, i32, f32, vp, desc,
                                        vp, vp]),
         "pa_wait": (C.c_int, [vp, vp, i32, C.POINTER(i32)]),
+        "pa_set_wait_timeout_ns": (C.c_uint64, [C.c_uint64]),
         "pa_bm_create": (C.c_int, [i32, i32, vp, C.POINTER(vp)]),
         "pa_bm_destroy": (None, [vp]),
         "pa_bm_add_seq": (C.c_int, [vp, i64]),
@@ -95,7 +96,7 @@ _lib = _load()
 EXPORTED = (
     "pa_abi_version", "pa_status_string", "pa_cache_write", "pa_copy_blocks", "pa_check_copy_pairs",
     "pa_decode_workspace_size", "pa_decode_launches", "pa_decode", "pa_append_decode", "pa_prefill_chunk",
-    "pa_wait",
+    "pa_wait", "pa_set_wait_timeout_ns",
 )
 
 
@@ -267,6 +268,12 @@ def pa_wait(err_flag=None, stream=None, timeout_ms: int = 10000) -> int:
     if st not in (PA_OK, PA_ERR_DEVICE_INDEX, PA_ERR_TIMEOUT) or (st == PA_ERR_TIMEOUT and flag.value == 0):
         raise PAError(st, "pa_wait")
     return int(flag.value)
+
+
+def pa_set_wait_timeout_ns(ns: int) -> int:
+    """Bound of every in-kernel wait of later launches (0: the 1 s default); returns the
+    previous bound."""
+    return int(_lib.pa_set_wait_timeout_ns(int(ns)))
 
 
 # ------------------------------------------------------------------ host manager

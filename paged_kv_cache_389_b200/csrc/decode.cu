@@ -153,6 +153,7 @@ struct Params {
     int32_t max_members;    // sequences per group: query rows members x g <= 128
     int32_t wait_first;     // launched right behind a cache write: wait for it first
     float v_scale;          // fp8 pools: value dequantisation scale (1 otherwise)
+    unsigned long long wait_ns;  // bound of every in-kernel wait
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -914,7 +915,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // ---- this warp's state into merge slot uc & 1, once the slot's previous
         // unit (uc - 2) has been merged by every warp
         const int b = uc & 1;
-        if (uc >= 2 && !mbar_wait_bounded(&mfreed[b], ((uc - 2) >> 1) & 1, abort_flag, p.err)) {
+        if (uc >= 2 && !mbar_wait_bounded(&mfreed[b], ((uc - 2) >> 1) & 1, abort_flag, p.err, p.wait_ns)) {
             dead = true;
             break;
         }
@@ -950,7 +951,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // all in by now unless a warp is a whole unit behind)
         if (uc >= 1) {
             const int pb = b ^ 1;
-            if (!mbar_wait_bounded(&mfull[pb], ((uc - 1) >> 1) & 1, abort_flag, p.err)) {
+            if (!mbar_wait_bounded(&mfull[pb], ((uc - 1) >> 1) & 1, abort_flag, p.err, p.wait_ns)) {
                 dead = true;
                 break;
             }
@@ -970,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
     }
     // the last unit's merge
-    if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err))
+    if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err, p.wait_ns))
         finish_unit<T, D, G>(p, prv, macc + (size_t)(uc & 1) * kWarps * G * D, mml + (size_t)(uc & 1) * kWarps * G);
     cp_async_wait<0>();
     grid_dep_wait();
@@ -1298,6 +1299,7 @@ cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
     prm.seq_tokens = a.partition_size;  // launch_t may widen it
     prm.scale_log2 = a.scale * kLog2e;
     prm.v_scale = 1.f;
+    prm.wait_ns = wait_limit_ns();
     if (a.cache.dtype == PA_FP8_E4M3) {
         if (a.cache.head_dim != 128) return cudaErrorInvalidValue;
         prm.scale_log2 = a.scale * a.cache.k_scale * kLog2e;

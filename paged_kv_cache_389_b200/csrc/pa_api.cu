@@ -1,5 +1,6 @@
 // C ABI entry points (include/pa.h): host-side validation, then kernel launch.
 // No device memory is allocated here; every buffer belongs to the caller.
+#include <atomic>
 #include <chrono>
 #include <cmath>
 #include <cstdint>
@@ -21,6 +22,12 @@ int num_sms(int device) {
     if (device >= 0 && device < 64) cached[device] = n;
     return n;
 }
+
+namespace {
+std::atomic<unsigned long long> g_wait_limit_ns{kWaitTimeoutNs};
+}  // namespace
+
+unsigned long long wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 namespace {
 
@@ -59,6 +66,11 @@ using namespace pa;
 extern "C" {
 
 int32_t pa_abi_version(void) { return 2; }
+
+uint64_t pa_set_wait_timeout_ns(uint64_t ns) {
+    if (ns == 0) ns = kWaitTimeoutNs;
+    return g_wait_limit_ns.exchange(ns);
+}
 
 const char *pa_status_string(pa_status s) {
     switch (s) {

@@ -1,6 +1,6 @@
-// Device helpers shared by the sm_100a kernels: mbarriers, 1-D bulk async copies
-// (the TMA engine's untiled cp.async.bulk), bounded waits, packed fp32 math and
-// the device error flag.  Written for sm_100a only.
+// Device helpers shared by the sm_100a kernels: mbarriers, bounded waits,
+// cp.async, warp-level tensor-core tiles, packed fp32 math and the device
+// error flag.  Written for sm_100a only.
 #pragma once
 
 #include <cstdint>
@@ -12,7 +12,7 @@
 namespace pa {
 
 constexpr int kBlockSize = 16;                        // tokens per KV block
-constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // 1 s for any in-kernel wait
+constexpr unsigned long long kWaitTimeoutNs = 1000000000ull;  // default bound of an in-kernel wait (1 s)
 
 __device__ __forceinline__ void flag_error(int32_t *err, int bits) {
     if (err) atomicOr(err, bits);
@@ -61,17 +61,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Gives up (returns false)
-// when *abort becomes non-zero or after kWaitTimeoutNs; on a timeout it raises
-// *abort and PA_DEVERR_TIMEOUT so every other warp of the CTA stops waiting too.
+// when *abort becomes non-zero or after limit_ns (the launch's wait bound,
+// kWaitTimeoutNs unless pa_set_wait_timeout_ns changed it); on a timeout it
+// raises *abort and PA_DEVERR_TIMEOUT so every other warp of the CTA stops
+// waiting too.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  volatile int *abort, int32_t *err) {
+                                                  volatile int *abort, int32_t *err,
+                                                  unsigned long long limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if ((it & 7u) == 0) {
             if (*abort) return false;
-            if (global_ns() - t0 > kWaitTimeoutNs) {
+            if (global_ns() - t0 > limit_ns) {
                 *abort = 1;
                 flag_error(err, PA_DEVERR_TIMEOUT);
                 return false;
@@ -80,24 +83,14 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     }
 }
 
-// Bounded wait that ignores *abort (used to drain copies still in flight).
+// Bounded wait that ignores *abort (used to drain copies still in flight); its
+// bound is always kWaitTimeoutNs, whatever the launch's wait bound.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity) {
     const unsigned long long t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (global_ns() - t0 > kWaitTimeoutNs) return false;
     }
     return true;
-}
-
-// ---- 1-D bulk copy global -> shared (TMA engine, no tensor map) -------------
-// dst and src 16-byte aligned, bytes a multiple of 16; completion is signalled
-// as transaction bytes on `bar`.
-__device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
-                                         uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(smem_u32(dst_smem)), "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
 }
 
 // Named barrier over `threads` threads (a multiple of 32) with id >= 1.
@@ -113,12 +106,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
-// Exact bf16 -> fp32 widening of the two halves of a packed pair (low half is
-// the element at the lower address).
-__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
-    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
     return __ffma2_rn(a, b, c);  // sm_100 packed fp32 FMA
 }
@@ -126,22 +113,6 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
 }  // namespace pa
 
 namespace pa {
-
-// ---- tiled tensor TMA (2-D), warp-level tensor-core tiles ------------------
-// 2-D tiled TMA load of one box at (x = column element, y = row) into shared
-// memory; x * element size must be a multiple of 16 bytes.
-__device__ __forceinline__ void tma_load_2d(void *dst_smem, const void *tmap, int32_t x, int32_t y,
-                                            uint64_t *bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst_smem)),
-        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_tmap(const void *tmap) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
-}
 
 // Order this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA) accesses of the same bytes.

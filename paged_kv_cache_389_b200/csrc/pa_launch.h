@@ -111,4 +111,8 @@ cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t s
 
 int num_sms(int device);
 
+// Bound of every in-kernel wait for launches made from now on, in ns
+// (pa_set_wait_timeout_ns; kWaitTimeoutNs by default).
+unsigned long long wait_limit_ns();
+
 }  // namespace pa

@@ -80,6 +80,7 @@ struct Params {
     float2 *ws_ml;
     int32_t part_tokens;
     int32_t max_parts;
+    unsigned long long wait_ns;  // bound of every in-kernel wait
 };
 
 // ---- tcgen05 wrappers --------------------------------------------------------
@@ -161,8 +162,9 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 }
 
 // Bounded mbarrier wait honouring the CTA abort flag (pa_common.cuh).
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *err) {
-    return mbar_wait_bounded(bar, parity, abort, err);
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *err,
+                                         unsigned long long limit_ns) {
+    return mbar_wait_bounded(bar, parity, abort, err, limit_ns);
 }
 
 // One 128-row query tile against a run of keys.  Row r (0..127) holds query head
@@ -343,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             bool q_ok = true;
             if (is_k) {
                 // the previous unit's QK must be done with Q
-                if (t == 0) *gw = (nu == 0 || wait_bar(q_empty, (nu - 1) & 1, abort_flag, p.err)) ? 1 : 0;
+                if (t == 0) *gw = (nu == 0 || wait_bar(q_empty, (nu - 1) & 1, abort_flag, p.err, p.wait_ns)) ? 1 : 0;
                 named_barrier(gbar, 64);
                 q_ok = *gw != 0;
                 named_barrier(gbar, 64);  // *gw is rewritten by the first tile issue
@@ -367,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             int next_e = table_entry(0);
             auto issue_tile = [&](int j) -> bool {
                 const int jt = tbase + j, st = jt & 1;
-                if (t == 0) *gw = (jt < 2 || wait_bar(&empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err)) ? 1 : 0;
+                if (t == 0) *gw = (jt < 2 || wait_bar(&empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err, p.wait_ns)) ? 1 : 0;
                 if (t < 8) {
                     int e = next_e;
                     if (j * 8 + t < (jb.nkeys + kBlockSize - 1) / kBlockSize && (e < 0 || e >= p.num_blocks)) {
@@ -414,10 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             // -------------------------------------------------------- MMA issuer
             if (lane == 0) {
                 constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
-                bool ok = wait_bar(q_full, nu & 1, abort_flag, p.err);
+                bool ok = wait_bar(q_full, nu & 1, abort_flag, p.err, p.wait_ns);
                 for (int j = 0; ok && j < jb.ntiles; ++j) {
                     const int jt = tbase + j, st = jt & 1;
-                    if (!wait_bar(&k_full[st], (jt >> 1) & 1, abort_flag, p.err)) break;
+                    if (!wait_bar(&k_full[st], (jt >> 1) & 1, abort_flag, p.err, p.wait_ns)) break;
                     tc_fence_after();
                     const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTileBytes;
 #pragma unroll
@@ -428,10 +430,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     tc_commit(s_full);
                     tc_commit(&k_empty[st]);
                     if (j == jb.ntiles - 1) tc_commit(q_empty);
-                    if (!wait_bar(p_full, jt & 1, abort_flag, p.err)) break;
+                    if (!wait_bar(p_full, jt & 1, abort_flag, p.err, p.wait_ns)) break;
                     // the first PV overwrites O: the previous unit's O must have been read
-                    if (j == 0 && nu > 0 && !wait_bar(o_free, (nu - 1) & 1, abort_flag, p.err)) break;
-                    if (!wait_bar(&v_full[st], (jt >> 1) & 1, abort_flag, p.err)) break;
+                    if (j == 0 && nu > 0 && !wait_bar(o_free, (nu - 1) & 1, abort_flag, p.err, p.wait_ns)) break;
+                    if (!wait_bar(&v_full[st], (jt >> 1) & 1, abort_flag, p.err, p.wait_ns)) break;
                     tc_fence_after();
                     const uint32_t pa_ = sbase + kOffP, va = sbase + kOffV + st * kTileBytes;
 #pragma unroll
@@ -467,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 const int key0 = j * kTileN + hf * 64;                // first key of this half
                 // the whole half is visible to every row of the warp: no per-key test
                 const bool open = __all_sync(kFull, row_ok && lim >= key0 + 63);
-                live = live && wait_bar(s_full, jt & 1, abort_flag, p.err);
+                live = live && wait_bar(s_full, jt & 1, abort_flag, p.err, p.wait_ns);
                 live = __all_sync(kFull, live);
                 if (!live) break;
                 tc_fence_after();
@@ -492,7 +494,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 float *rb = red + (jt & 1) * 256;
                 rb[hf * 128 + r] = mx;
                 mbar_arrive(&red_full[jt & 1]);
-                live = wait_bar(&red_full[jt & 1], (jt >> 1) & 1, abort_flag, p.err);
+                live = wait_bar(&red_full[jt & 1], (jt >> 1) & 1, abort_flag, p.err, p.wait_ns);
                 live = __all_sync(kFull, live);
                 if (!live) break;
                 mx = fmaxf(rb[r], rb[128 + r]);
@@ -501,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 const float alpha = fast_exp2(m - m_use);
                 if (j > 0) {
                     // P and O are still in use by the previous tile's PV
-                    live = wait_bar(pv_done, (jt - 1) & 1, abort_flag, p.err);
+                    live = wait_bar(pv_done, (jt - 1) & 1, abort_flag, p.err, p.wait_ns);
                     live = __all_sync(kFull, live);
                     if (!live) break;
                     tc_fence_after();
@@ -554,12 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 tc_fence_before();
                 mbar_arrive(p_full);
             }
-            if (live) live = wait_bar(pv_done, (tbase + jb.ntiles - 1) & 1, abort_flag, p.err);
+            if (live) live = wait_bar(pv_done, (tbase + jb.ntiles - 1) & 1, abort_flag, p.err, p.wait_ns);
             live = __all_sync(kFull, live);
             if (live) {
                 lsum[hf * 128 + r] = l;
                 mbar_arrive(l_full);
-                live = wait_bar(l_full, nu & 1, abort_flag, p.err);
+                live = wait_bar(l_full, nu & 1, abort_flag, p.err, p.wait_ns);
                 live = __all_sync(kFull, live);
             }
             if (live && warp_rows) {
@@ -669,6 +671,7 @@ cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
     prm.num_kv_heads = a.cache.num_kv_heads;
     prm.num_blocks = a.cache.num_blocks;
     prm.scale_log2 = a.scale * kLog2e;
+    prm.wait_ns = wait_limit_ns();
     switch (a.num_q_heads / a.cache.num_kv_heads) {
         case 1: return launch_g<1>(a, prm, stream);
         case 2: return launch_g<2>(a, prm, stream);
@@ -697,6 +700,7 @@ cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t s
     prm.ws_ml = a.ws_ml;
     prm.part_tokens = a.partition_size;
     prm.max_parts = a.max_partitions;
+    prm.wait_ns = wait_limit_ns();
     switch (a.num_q_heads / a.num_kv_heads) {
         case 1: return launch_group_g<1>(prm, sms, stream);
         case 2: return launch_group_g<2>(prm, sms, stream);

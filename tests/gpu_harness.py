@@ -114,6 +114,9 @@ class TwoSided:
     def err_flag(self):
         return self.pa.pa_wait(self.gpu.err_flag)
 
+    def clear_err(self):
+        self.gpu.err_flag.zero_()
+
     def tables(self, seqs):
         mb = max(1, max(len(self.model.block_table(s)) for s in seqs))
         t_o, l_o = self.model.build_tables(seqs, mb)

@@ -53,6 +53,16 @@ def desc(nb=8, hkv=2, bs=16, d=128, dt=1, ks=1.0, vs=1.0):
     return CacheDesc(nb, hkv, bs, d, dt, ks, vs)
 
 
+def _gpu_visible():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+@pytest.mark.skipif(_gpu_visible(), reason="passes placeholder device addresses: run only where no GPU is "
+                    "reachable, so a regressed check can never launch on them")
 def test_host_validation_launches_nothing(pa):
     L = pa._lib
     p16 = C.c_void_p(0x10000)   # fake, never dereferenced: validation fails first

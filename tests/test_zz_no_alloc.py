@@ -63,9 +63,26 @@ def test_static_scratch_matches_caller_workspace(pa, cid, part):
 
 
 def test_static_scratch_rejects_requests_beyond_its_array(pa):
+    """A request whose partials would not fit in the array is refused before any
+    launch.  Every buffer is a real device allocation of the size the arguments
+    declare, and every context is empty, so even if the size check ever regressed
+    the launched kernels would stay inside these buffers (an fp32 pool takes no
+    shared-prefix path and an empty context writes no partial)."""
+    torch = torch_mod()
     fn = _entry(pa)
-    desc = pa.CacheDesc(16, 8, 16, 128, pa.PA_BF16)
-    fake = C.c_void_p(0x10000)   # never dereferenced: the size check fails first
-    # 4096 seqs x 64 heads x 4 partitions x 520 B = 545 MB > 32 MiB
-    st = fn(fake, fake, fake, fake, 8, fake, 2048, 4096, 64, 0.1, 512, fake, C.byref(desc), None, None)
+    S, hkv, d, maxc, part, mb = 4096, 8, 64, 2048, 16, 128
+    need = pa.pa_decode_workspace_size(S, hkv, d, maxc, part)
+    assert need > (32 << 20)                      # 4096 x 8 x 128 partitions x 264 B
+    kc = torch.zeros((16, hkv, 16, d), dtype=torch.float32, device="cuda")
+    vc = torch.zeros_like(kc)
+    q = torch.zeros((S, hkv, d), dtype=torch.float32, device="cuda")
+    out = torch.zeros_like(q)
+    tables = torch.zeros((S, mb), dtype=torch.int32, device="cuda")
+    lens = torch.zeros(S, dtype=torch.int32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    desc = pa.cache_desc(kc)
+    st = fn(_ptr(q), _ptr(kc), _ptr(vc), _ptr(tables), mb, _ptr(lens), maxc, S, hkv, 0.125, part,
+            _ptr(out), C.byref(desc), _ptr(err), C.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == pa.PA_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
