@@ -208,3 +208,96 @@ def test_three_gloo_ranks_split_kv_heads_and_gather():
     want = oracle.decode(step.q, kc, vc, t, l, wl.scale)
     for r in range(world):                          # every rank holds the whole, bit for bit
         assert np.array_equal(out[r], want)
+
+
+def _shard_ops(wl, keep):
+    """The workload's allocator operations for the sequences in ``keep`` and every
+    parent they were forked from (a group stays on one rank with its parent)."""
+    parent = {}
+    for op in wl.ops:
+        if op[0] == "fork":
+            parent[op[2]] = op[1]
+    mine = set(keep)
+    for s in list(keep):
+        while s in parent:
+            s = parent[s]
+            mine.add(s)
+    return [op for op in wl.ops if op[1] in mine]
+
+
+def _manager_worker(rank, world, port, q):
+    """Each rank owns a pool and the library's C++ block manager for its shard only,
+    and a Python model of the same shard: tables, lengths, slots and copy-on-write
+    pairs of every step must agree bit for bit (the host side of the sharded path)."""
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=30))
+    try:
+        import workloads
+        from oracle.block_model import BlockManagerModel
+        import paged_kv_cache_389_b200 as pa
+        wl = workloads.make(4, mini=True)             # parents forked into 4 children each
+        seqs = wl.steps[0].seqs
+        groups = [s // 4 for s in seqs]
+        n = {}
+        for op in wl.ops:
+            if op[0] == "add":
+                n[op[1]] = 0
+            elif op[0] == "append":
+                n[op[1]] += op[2].shape[0]
+            elif op[0] == "fork":
+                n[op[2]] = n[op[1]]
+        lo, hi = shard_ranges([n[s] for s in seqs], world, groups)[rank]
+        mine = seqs[lo:hi]
+        ops = _shard_ops(wl, mine)
+        cpp = pa.BlockManager(wl.num_blocks, wl.block_size, wl.free_order)
+        model = BlockManagerModel(wl.num_blocks, wl.block_size, wl.free_order.tolist())
+        shard = workloads.Workload(wl.config_id, wl.name, wl.dtype, wl.num_blocks, wl.num_q_heads,
+                                   wl.num_kv_heads, wl.head_dim, wl.scale, wl.free_order)
+        shard.ops = ops
+        workloads.replay(shard, cpp, lambda k, v, s: None)
+        workloads.replay(shard, model, lambda k, v, s: None)
+        steps = []
+        for st in wl.steps:
+            part = [s for s in st.seqs if s in set(mine)]
+            if not part:
+                continue
+            slots_c, pairs_c = cpp.append_step(part, [1] * len(part))
+            slots_m, pairs_m = [], []
+            for s in part:
+                sl, pr = model.append_slot(s)
+                slots_m.append(sl)
+                if pr is not None:
+                    pairs_m.append(pr)
+            mb = max(len(model.block_table(s)) for s in part)
+            tc, lc = cpp.build_tables(part, mb)
+            tm, lm = model.build_tables(part, mb)
+            steps.append((slots_c.tolist() == slots_m,
+                          [tuple(p) for p in pairs_c.tolist()] == pairs_m,
+                          np.array_equal(tc, tm) and np.array_equal(lc, lm), len(part), len(pairs_m)))
+        got = [None] * world
+        dist.all_gather_object(got, (lo, hi, steps))
+        q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_run_the_block_manager_on_their_shards():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_manager_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=180) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ranges = sorted((lo, hi) for lo, hi, _ in out[0])
+    assert ranges[0][0] == 0 and ranges[0][1] == ranges[1][0] and ranges[1][0] > 0
+    for lo, hi, steps in out[0]:
+        assert steps, "every rank ran steps"
+        for slots_ok, pairs_ok, tables_ok, n, _ in steps:
+            assert slots_ok and pairs_ok and tables_ok and n == hi - lo
+        assert sum(st[4] for st in steps) > 0, "the shard's first step copies shared last blocks"
