@@ -108,7 +108,7 @@ struct Layout {
     static constexpr size_t kLimit = 232448;                    // sm_100 max dynamic smem per CTA
     static constexpr size_t kPBytes = sizeof(T) == 4 ? (size_t)kWarps * (16 * G + G) * 4 : 64;
     static constexpr size_t kMergeBytes = (size_t)kWarps * G * (D * 4 + 8);
-    static constexpr size_t kFixed = kPBytes + 16 + 48 + (size_t)(kMaxSplitSeqs + 1) * 4 + 64;
+    static constexpr size_t kFixed = kPBytes + 16 + 48 + 96 + (size_t)(kMaxSplitSeqs + 1) * 4 + 64;
     static constexpr int stages_fit(int bufs) {
         return (int)((kLimit - kFixed - bufs * kMergeBytes) / ((size_t)kWarps * kStageBytes));
     }
@@ -121,7 +121,8 @@ struct Layout {
     static constexpr size_t kOffMacc = align_up(kOffP + kPBytes, 16);
     static constexpr size_t kOffMml = kOffMacc + (size_t)kMergeBufs * kWarps * G * D * 4;
     static constexpr size_t kOffBar = align_up(kOffMml + (size_t)kMergeBufs * kWarps * G * 8, 16);
-    static constexpr size_t kOffCum = kOffBar + 48;  // 4 mbarriers + abort word
+    static constexpr size_t kOffRingIds = kOffBar + 48;  // after 4 mbarriers + abort word
+    static constexpr size_t kOffCum = kOffRingIds + 96;    // unit-id ring: ids, tags, claims [8] each
     static constexpr size_t smem_bytes(int cum_entries) { return kOffCum + (size_t)cum_entries * 4; }
 };
 
@@ -154,6 +155,8 @@ struct Params {
     int32_t wait_first;     // launched right behind a cache write: wait for it first
     float v_scale;          // fp8 pools: value dequantisation scale (1 otherwise)
     unsigned long long wait_ns;  // bound of every in-kernel wait
+    int32_t *work_ctr;      // units handed out beyond the first gridDim.x (zeroed by the
+                            // detection kernel of this call), or nullptr: static order
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -742,6 +745,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         *abort_flag = 0;
         mbar_init_fence();
     }
+    // This CTA's units, in order: unit 0 is blockIdx.x.  With a work counter,
+    // unit k >= 1 is gridDim.x + a value drawn from it, so CTAs that start early
+    // (beside the group tiles) or get short units take more of them; without one
+    // it is blockIdx.x + k * gridDim.x.  Ids are drawn two units ahead, in order,
+    // by the first warp to start a unit, and published in a ring of 8 slots.
+    volatile int *ring_id = reinterpret_cast<volatile int *>(smem + Lay::kOffRingIds);
+    volatile int *ring_tag = ring_id + 8;      // unit index whose id the slot holds
+    int *ring_claim = const_cast<int *>(ring_id) + 16;  // unit index last claimed for the slot
+    const bool dyn = p.work_ctr != nullptr;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 8; ++i) {
+            ring_tag[i] = -1;
+            ring_claim[i] = i - 8;
+        }
+        ring_tag[0] = ring_claim[0] = 0;
+        if (dyn) {
+            const int v = (int)gridDim.x + atomicAdd(p.work_ctr, 2);
+            ring_id[1] = v;
+            ring_id[2] = v + 1;
+            ring_tag[1] = ring_claim[1] = 1;
+            ring_tag[2] = ring_claim[2] = 2;
+        }
+    }
     prologue(p, cum, reinterpret_cast<int *>(macc));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.num_seqs, hkv = p.num_kv_heads;
@@ -752,15 +778,54 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     float *pw = pbuf + warp * Lay::kPWarpFloats;
     const int q4 = lane & 3, dr = lane >> 2;
 
+    // id of this CTA's unit k (whole warp; bounded wait for a dynamic id; INT64_MAX
+    // ends the work)
+    auto unit_id = [&](int k) -> int64_t {
+        if (k == 0) return blockIdx.x;
+        if (!dyn) return (int64_t)blockIdx.x + (int64_t)k * gridDim.x;
+        int v = INT_MAX;
+        if (lane == 0) {
+            const unsigned long long t0 = global_ns();
+            bool ok = true;
+            while (ring_tag[k & 7] != k) {
+                if (*abort_flag || global_ns() - t0 > p.wait_ns) {
+                    if (!*abort_flag) flag_error(p.err, PA_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                    ok = false;
+                    break;
+                }
+            }
+            __threadfence_block();
+            if (ok) v = ring_id[k & 7];
+        }
+        v = __shfl_sync(kFull, v, 0);
+        return v == INT_MAX ? INT64_MAX : (int64_t)v;
+    };
+    // at the start of unit k: the first warp there draws the id of unit k + 2,
+    // after the id of unit k + 1 is out, so that a CTA's ids only grow
+    auto claim_ahead = [&](int k) {
+        if (!dyn || lane != 0 || k < 1) return;
+        const int k2 = k + 2, sl = k2 & 7;
+        if (atomicCAS(&ring_claim[sl], k2 - 8, k2) != k2 - 8) return;
+        const unsigned long long t0 = global_ns();
+        while (ring_tag[(k2 - 1) & 7] != k2 - 1) {
+            if (*abort_flag || global_ns() - t0 > p.wait_ns) break;
+        }
+        ring_id[sl] = (int)gridDim.x + atomicAdd(p.work_ctr, 1);
+        __threadfence_block();
+        ring_tag[sl] = k2;
+    };
+
     WarpUnit cur, nxt;
-    int64_t u = blockIdx.x;
+    int64_t u = unit_id(0);
     if (u >= total) {
         grid_dep_wait();
         return;
     }
     load_unit(p, u, units_first, cum, cur, lane, warp == 0);
-    bool have_nxt = u + gridDim.x < total;
-    if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
+    int64_t u_nxt = unit_id(1);
+    bool have_nxt = u_nxt < total;
+    if (have_nxt) load_unit(p, u_nxt, units_first, cum, nxt, lane, warp == 0);
 
     // table entry of logical block j of a unit (the first 32 come from registers)
     auto phys_of = [&](const WarpUnit &w, int j) {
@@ -805,6 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     bool dead = false;       // a hand-over wait timed out
     int uc = 0;
     for (;; ++uc) {
+        claim_ahead(uc);
         // ---- q operands of this unit (tiny, L2 resident)
         MmaState<D> ms;
         F32State<D, G> fs;
@@ -962,13 +1028,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         prv = cur;
 
         // ---- advance: the fetch cursor moves down one unit with the window
-        u += gridDim.x;
         if (!have_nxt) break;
         walk(iss_u, iss_j, 0);
         cur = nxt;
         iss_u = iss_u > 0 ? iss_u - 1 : 0;
-        have_nxt = u + gridDim.x < total;
-        if (have_nxt) load_unit(p, u + gridDim.x, units_first, cum, nxt, lane, warp == 0);
+        u_nxt = unit_id(uc + 2);
+        have_nxt = u_nxt < total;
+        if (have_nxt) load_unit(p, u_nxt, units_first, cum, nxt, lane, warp == 0);
     }
     // the last unit's merge
     if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err, p.wait_ns))
@@ -1134,6 +1200,7 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     if (lane == 31) {  // its running counts end at the totals
         meta[0] = oc;
         meta[1] = ou;
+        meta[2] = 0;   // the per-sequence kernel's work counter
     }
 }
 
@@ -1227,6 +1294,7 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             if (e != cudaSuccess) return e;
             GroupTileLaunch gl;
             gl.query = a.query;
+            gl.num_seqs = a.num_seqs;
             gl.key_cache = a.key_cache;
             gl.value_cache = a.value_cache;
             gl.block_tables = a.block_tables;
@@ -1244,6 +1312,7 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             gl.err = a.err;
             if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
             grouped = true;
+            prm.work_ctr = const_cast<int32_t *>(prm.meta) + 2;
         }
     }
     int64_t grid = sms;

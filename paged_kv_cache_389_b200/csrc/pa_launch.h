@@ -90,7 +90,8 @@ cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
 // inside the blocks they share; writes that partition's split-K partials.
 // groups / meta are the decode's detection output (device memory).
 struct GroupTileLaunch {
-    const void *query;
+    const void *query;       // [num_seqs, num_q_heads, 128] bf16
+    int32_t num_seqs;
     const void *key_cache;
     const void *value_cache;
     const int32_t *block_tables;

@@ -1,5 +1,6 @@
-// Chunked-prefill attention against the paged KV cache on 5th-generation tensor
-// cores (tcgen05.mma, accumulators in tensor memory).
+// Attention tiles on 5th-generation tensor cores (tcgen05.mma, accumulators and
+// probabilities in tensor memory, operands staged by TMA): the chunked prefill,
+// and the shared-prefix group units of the split decode.
 //
 // What is computed (include/pa.h): sequence s has C_s query rows, the last C_s
 // positions of its L_s-token context; row i sits at position p = L_s - C_s + i
@@ -8,22 +9,35 @@
 // compute bound) and 4.3/5.1 (long prompts are cut into chunks interleaved with
 // decode); devpress vLLM v0.6.x teardown, 核心代码拆解 (paged K/V via the table).
 //
-// Tile: one CTA computes a 128-row query tile of one (sequence, kv head): the g
-// query heads of that kv head are packed into the rows (row = chunk row * g +
-// head), so every K/V byte staged in shared memory serves all g heads.  The CTA
-// walks the keys in tiles of 128 (8 blocks of 16) up to the tile's last position.
-//   S   = Q K^T      tcgen05.mma kind::f16, M=128, N=128 keys, K=16 x 8, -> TMEM
-//   P   = softmax    online, fp32, one query row per thread (tcgen05.ld from TMEM)
-//   O  += P V        tcgen05.mma, A = P (bf16, smem), B = V (MN-major), -> TMEM
-// Warp roles: warps 0-3 load (16-byte cp.async into 128-byte-swizzled layouts:
-// Q and K K-major, V MN-major, the canonical layouts the MMA descriptors name),
-// warps 4-11 run the softmax (warp w: TMEM lanes 32*(w%4)..+31, one 64-column
-// half of the tile), warp 12 owns the tensor memory and issues the MMAs from one
-// thread.  K and V tiles have separate two-stage rings and loader warps (0-1: Q
-// and K, 2-3: V), so a K stage is refilled as soon as its QK is done; the stages
-// are handed over with mbarriers; every wait is bounded and an abort still frees
-// the tensor memory.
+// Rows: the g query heads of one kv head are packed into the rows of a tile
+// (row = chunk row * g + head), so every K/V byte staged in shared memory serves
+// all g of them.  A persistent CTA runs two row streams over 128-key tiles:
+//   S_t = Q_t K^T   tcgen05.mma kind::f16, M = 128, N = 128, K = 16 x 8 -> tensor memory
+//   P_t = softmax   online, fp32, one row per thread (tcgen05.ld), written back as
+//                   bf16 over the first 64 columns of S_t (tcgen05.st)
+//   O_t += P_t V    tcgen05.mma with A = P_t read from tensor memory, B = V (MN-major)
+// A job is either two 128-row query tiles sharing every K/V tile (stream t owns
+// tile t), or one query tile whose key tiles alternate between the streams (each
+// keeps its own running max, sum and O; the two are merged at the end).  Either
+// way one stream's softmax runs while the tensor core computes the other's
+// products.  The MMA issue order per key tile is PV_t(previous tile of t), then
+// QK_t(this tile): S_t being full therefore also means O_t is not being written.
+// Tensor memory (512 columns): S0 | S1 | O0 | O1.  The reference point of P and O
+// (a running row maximum) moves only when a row's maximum rises by more than 2^8,
+// so O is rescaled rarely; the merge and the final division use the same point.
+// Warp roles: 0-3 softmax of stream 0, 4-7 softmax of stream 1 (warp w reads
+// tensor-memory lanes 32 (w % 4) .. + 31), 8 issues the MMAs from one thread and
+// owns the tensor memory, 9 loads (10 and 11 only complete the third warpgroup): Q and K/V tiles by TMA (128-byte swizzle, the
+// canonical layouts the MMA descriptors name) through a ring of 32 KB stages
+// holding K(0), V(0), K(1), V(1), ...; one TMA box per (16-token block, 64-column
+// half).  Every wait is bounded; an abort drains the copies and MMAs in flight
+// and still frees the tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "pa_common.cuh"
 #include "pa_launch.h"
@@ -34,33 +48,50 @@ namespace {
 constexpr unsigned kFull = 0xffffffffu;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kD = 128;              // head_dim (bf16 only)
-constexpr int kTileM = 128;          // query rows per CTA
-constexpr int kTileN = 128;          // keys per KV tile
-constexpr int kThreads = 13 * 32;    // 4 load warps, 8 softmax warps, 1 MMA warp
-constexpr int kMmaWarp = 12;
+constexpr int kTileM = 128;          // query rows per stream tile
+constexpr int kTileN = 128;          // keys per K/V tile
+constexpr int kStages = 4;           // K/V ring stages
+constexpr int kThreads = 12 * 32;    // 8 softmax warps, 1 MMA warp, 1 load warp, 2 idle
+constexpr int kMmaWarp = 8, kLoadWarp = 9;
+// Registers per thread after the split (setmaxnreg, per warpgroup of 4 warps): the
+// launch gives 384 threads x 168; the softmax warpgroups take 200 (a row of S in
+// registers), the MMA / load warpgroup 96: 256 x 200 + 128 x 96 <= 384 x 168, and
+// each SM sub-partition (warps w, w + 4, w + 8) holds 2 x 200 + 96 <= 512 per lane.
+constexpr int kRegsSoftmax = 200, kRegsOther = 96;
+static_assert(256 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split over the launch's total");
 constexpr int kSoftmaxThreads = 256;
-constexpr uint32_t kTmemCols = 256;  // S: columns 0..127, O: 128..255
+constexpr uint32_t kTmemCols = 512;  // S0, S1, O0, O1
+constexpr float kRescaleLog2 = 8.f;  // the reference point moves when a row max rises by more (log2 units)
 
-// shared memory (offsets from a 1024-byte aligned base)
-constexpr uint32_t kHalf = kTileM * 128;           // one 64-column half of a 128-row tile
-constexpr uint32_t kTileBytes = 2 * kHalf;         // 32 KB
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTileBytes;     // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTileBytes; // 2 stages
-constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;
-constexpr uint32_t kOffBar = kOffP + kTileBytes;
-constexpr uint32_t kOffTab = kOffBar + 24 * 8;     // 24 mbarriers
-constexpr uint32_t kOffMisc = kOffTab + 2 * 2 * 8 * 4;  // [K, V loader][2 stages][8 table entries]
-constexpr uint32_t kOffRed = kOffMisc + 16;          // row-max halves [2 tiles][2 halves][128 rows]
-constexpr uint32_t kOffLsum = kOffRed + 2 * 2 * 128 * 4;  // row-sum halves [2][128]
-constexpr uint32_t kOffGcum = kOffLsum + 2 * 128 * 4;  // group units: units before each group
-constexpr int kMaxGroups = 2048;                     // a group has >= 2 (in fact >= 4) of <= 4096 sequences
-constexpr size_t kSmemBytes = 1024 + kOffGcum + kMaxGroups * 4;
+// shared memory (offsets from a 1024-byte aligned base inside the dynamic area)
+constexpr uint32_t kHalf = kTileM * 128;            // one 64-column half of a 128-row tile
+constexpr uint32_t kTileBytes = 2 * kHalf;          // 32 KB
+constexpr uint32_t kBlockBytes = kBlockSize * 128;  // one block's rows in one half
+constexpr uint32_t kOffQ = 0;                       // Q buffers 0 and 1
+constexpr uint32_t kOffRing = 2 * kTileBytes;
+constexpr uint32_t kOffBar = kOffRing + kStages * kTileBytes;
+// barriers
+constexpr int kBarFull = 0;                     // [kStages] stage landed: TMA bytes + the loader's 2nd arrival
+constexpr int kBarEmpty = kBarFull + kStages;   // [kStages] stage consumed (MMA commit)
+constexpr int kBarQFull = kBarEmpty + kStages;  // [2] Q buffer landed
+constexpr int kBarQEmpty = kBarQFull + 2;       // [2] last QK reading a Q buffer done
+constexpr int kBarSFull = kBarQEmpty + 2;       // [2] S_t written
+constexpr int kBarPFull = kBarSFull + 2;        // [2] P_t written (the 128 softmax threads of stream t)
+constexpr int kBarOFull = kBarPFull + 2;        // [2] last PV_t of a job done
+constexpr int kBarOFree = kBarOFull + 2;        // the job's O read by every softmax thread
+constexpr int kBarMl = kBarOFree + 1;           // both streams' (m, l) rows published
+constexpr int kBarIdle = kBarMl + 1;            // every MMA issued has completed
+constexpr int kNumBars = kBarIdle + 1;
+constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
+constexpr uint32_t kOffMl = kOffMisc + 16;             // float2 (m, l) [2 streams][128 rows]
+constexpr size_t kSmemUsed = kOffMl + 2 * 128 * 8;
+constexpr size_t kSmemBytes = kSmemUsed + 1024;       // slack to align the base
 
 struct Params {
-    const unsigned char *q;
-    const unsigned char *kc;
-    const unsigned char *vc;
+    CUtensorMap qmap;  // query rows: {head_dim, Hq, rows of Hq heads}, box {64, G, 128 / G}
+    CUtensorMap kmap;  // pool: {head_dim, 16 tokens, blocks x kv heads}, box {64, 16, 1}
+    CUtensorMap vmap;
+    const unsigned char *vc;  // value pool (rows of a partly filled last block are copied by hand)
     const int32_t *tables;
     const int32_t *lens;
     const int32_t *chunks;
@@ -72,6 +103,7 @@ struct Params {
     int32_t num_q_heads;
     int32_t num_kv_heads;
     int32_t num_blocks;
+    int32_t pairs;     // prefill: 256-row jobs per (sequence, kv head)
     float scale_log2;
     // shared-prefix group units of the split decode
     const int4 *groups;    // (first seq, members, shared partitions, units before)
@@ -83,7 +115,7 @@ struct Params {
     unsigned long long wait_ns;  // bound of every in-kernel wait
 };
 
-// ---- tcgen05 wrappers --------------------------------------------------------
+// ---- tcgen05 and TMA wrappers -------------------------------------------------
 __device__ __forceinline__ void tmem_alloc(uint32_t *dst_smem, uint32_t cols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
                  "r"(cols)
@@ -96,8 +128,9 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t cols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                       bool accumulate) {
+// D (tensor memory) (+)= A (shared-memory descriptor) * B (shared-memory descriptor)
+__device__ __forceinline__ void tc_mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
@@ -105,11 +138,23 @@ __device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t a_desc, uint64_
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
         : "memory");
 }
+// D (tensor memory) (+)= A (tensor memory: rows = lanes, K packed two bf16 per
+// column) * B (shared-memory descriptor)
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+        : "memory");
+}
 __device__ __forceinline__ void tc_commit(uint64_t *bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+// 32 lanes x 32 columns of 32 bits: thread i gets columns c..c+31 of lane base + i
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
     uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -122,502 +167,614 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
     asm volatile(
         "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
         "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-          "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-          "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-          "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-          "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-          "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
-          "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
-          "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
-          "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
-          "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
-          "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Shared-memory matrix descriptor: 128-byte swizzle, start/LBO/SBO in 16-byte units,
-// descriptor version 1 (sm_100).
+// 3-D tiled TMA load of one box into shared memory; completion as transaction
+// bytes on `bar`.  x (the innermost coordinate) is 0 or 64 here: 16-byte aligned.
+// A box reaching outside the tensor (z = -1 included) reads zeros there.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst_smem, const CUtensorMap *map, int x, int y, int z,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst_smem),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Shared-memory matrix descriptor: 128-byte swizzle, start/LBO/SBO in 16-byte
+// units, descriptor version 1 (sm_100).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
     return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)((lbo_bytes >> 4) & 0x3FFF) << 16) |
            ((uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M=128, N=128.
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 accumulator, M = 128,
+// N = 128, A K-major; B K-major (QK) or MN-major (PV).
 constexpr uint32_t idesc_bf16(bool b_mn_major) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(kTileN >> 3) << 17) |
            ((uint32_t)(kTileM >> 4) << 24);
 }
 
-// Byte offset of 16-byte chunk c (0..15) of row r in a 128-row tile stored as
-// two 64-column halves of 128-byte rows with the 128-byte swizzle.
-__device__ __forceinline__ uint32_t swz(int r, int c) {
-    return (uint32_t)((c >> 3) * kHalf + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, const Params &p) {
+    return mbar_wait_bounded(bar, parity, abort, p.err, p.wait_ns);
 }
 
-// Bounded mbarrier wait honouring the CTA abort flag (pa_common.cuh).
-__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, int32_t *err,
-                                         unsigned long long limit_ns) {
-    return mbar_wait_bounded(bar, parity, abort, err, limit_ns);
-}
-
-// One 128-row query tile against a run of keys.  Row r (0..127) holds query head
-// h*G + r%G of row group r/G; row groups are q_row_stride bytes apart.  Keys are
-// 0..nkeys-1 through the table entries starting at trow; row r may see keys
-// 0..lim0 + lim_step*(r/G) (lim_step 1: causal prefill; 0: every key).
+// One job of a CTA.  Packed row r (0..127) of query tile t holds query head
+// h*G + r%G of row group qz[t] + r/G.  two: both tiles hold rows and share every
+// key tile; otherwise one tile (t = 0) whose key tile j goes to stream j & 1.
+// Row r of tile t may see keys 0..lim0[t] + lim_step * (r / G) (all < nkeys).
 struct Job {
-    const unsigned char *q;  // query row group 0, head h*G
-    int64_t q_row_stride;
-    int nrows;               // rows r < nrows are real (the rest are zero)
+    bool two;
+    int nrows[2];
+    int qz[2];         // TMA z coordinate of the tile's first row group
+    int lim0[2];
+    int lim_step;
+    int nkeys, ntiles;
+    int h;             // kv head
     const int32_t *trow;
-    int nkeys;
-    int lim0, lim_step;
-    int ntiles;
-    int h;
-    // output: prefill -> normalised bf16 rows at out (same strides as q);
-    // group -> fp32 partials of workspace row (first + r/G)*Hq + h*G + r%G, slot part
-    unsigned char *out;
+    // output: prefill -> bf16 rows of row group out_row0 + ..; group -> fp32
+    // partials of workspace row (first + r/G)*Hq + h*G + r%G, slot part
+    int64_t out_row0;
     int first, part;
 };
 
 template <int G, bool kGroup>
-__device__ __forceinline__ Job group_job(const Params &p, const int *gcum, int ngroups, int u) {
-    Job jb;
-    int lo = 0, hi = ngroups;  // gcum[lo] <= u < gcum[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (gcum[mid] <= u) lo = mid; else hi = mid;
+__device__ __forceinline__ bool make_job(const Params &p, int u, Job &jb) {
+    if constexpr (kGroup) {
+        const int ngroups = __ldg(p.meta);
+        int lo = 0, hi = ngroups;  // groups[lo].w <= u < groups[hi].w
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (__ldg(&p.groups[mid].w) <= u) lo = mid; else hi = mid;
+        }
+        const int4 gr = __ldg(&p.groups[lo]);  // (first seq, members, shared partitions, units before)
+        const int r = u - gr.w;
+        jb.h = r % p.num_kv_heads;
+        jb.part = r / p.num_kv_heads;  // partition = workspace slot
+        jb.first = gr.x;
+        jb.two = false;
+        jb.nrows[0] = gr.y * G;
+        jb.nrows[1] = 0;
+        jb.qz[0] = jb.qz[1] = gr.x;
+        jb.trow = p.tables + (int64_t)gr.x * p.max_blocks + (int64_t)jb.part * (p.part_tokens / kBlockSize);
+        jb.nkeys = p.part_tokens;
+        jb.lim0[0] = jb.lim0[1] = p.part_tokens - 1;
+        jb.lim_step = 0;
+        jb.ntiles = (p.part_tokens + kTileN - 1) / kTileN;
+        jb.out_row0 = 0;
+        return true;
+    } else {
+        const int jp = u % p.pairs;
+        const int rem = u / p.pairs;
+        const int h = rem % p.num_kv_heads, s = rem / p.num_kv_heads;
+        const int L = __ldg(p.lens + s), C = __ldg(p.chunks + s);
+        if (C < 0 || C > p.max_chunk || C > L || (int64_t)L > (int64_t)p.max_blocks * kBlockSize) return false;
+        const int rows = C * G, r0 = jp * 2 * kTileM;
+        if (r0 >= rows) return false;
+        const int start = L - C;
+        jb.h = h;
+        jb.nrows[0] = min(kTileM, rows - r0);
+        jb.nrows[1] = min(kTileM, max(0, rows - r0 - kTileM));
+        jb.two = jb.nrows[1] > 0;
+        const int i0 = r0 / G;  // chunk row of the job's first packed row
+        jb.qz[0] = s * p.max_chunk + i0;
+        jb.qz[1] = jb.qz[0] + kTileM / G;
+        jb.lim0[0] = start + i0;
+        jb.lim0[1] = jb.two ? start + i0 + kTileM / G : jb.lim0[0];
+        jb.lim_step = 1;
+        const int last_row = (r0 + jb.nrows[0] + jb.nrows[1] - 1) / G;
+        jb.nkeys = start + last_row + 1;  // keys 0..start + last_row
+        jb.ntiles = (jb.nkeys + kTileN - 1) / kTileN;
+        jb.trow = p.tables + (int64_t)s * p.max_blocks;
+        jb.out_row0 = (int64_t)s * p.max_chunk + i0;
+        jb.first = jb.part = 0;
+        return true;
     }
-    const int4 gr = __ldg(&p.groups[lo]);  // (first seq, members, shared partitions, units before)
-    const int r = u - gr.w;
-    jb.h = r % p.num_kv_heads;
-    jb.part = r / p.num_kv_heads;  // partition = workspace slot
-    jb.first = gr.x;
-    const int64_t hs = (int64_t)kD * 2;
-    jb.q_row_stride = (int64_t)p.num_q_heads * hs;
-    jb.q = p.q + (int64_t)gr.x * jb.q_row_stride + (int64_t)jb.h * G * hs;
-    jb.nrows = gr.y * G;
-    jb.trow = p.tables + (int64_t)gr.x * p.max_blocks + (int64_t)jb.part * (p.part_tokens / kBlockSize);
-    jb.nkeys = p.part_tokens;
-    jb.lim0 = p.part_tokens - 1;
-    jb.lim_step = 0;
-    jb.ntiles = (p.part_tokens + kTileN - 1) / kTileN;
-    jb.out = nullptr;
-    return jb;
 }
 
-// Prefill: one CTA per (query tile, kv head, sequence).  Shared-prefix groups of
-// the split decode (kGroup): a persistent CTA loops over the group units (group,
-// partition, kv head) listed by the decode's detection kernel; the rows are the
-// members' queries, the keys one partition lying inside the blocks all members
-// share, and the result is the partition's (m, l, unnormalised O) in workspace
-// slot p of every member -- the same partial the per-sequence kernel would write.
-// (Units spanning all of a group's partitions were measured: they balance worse
-// over the SMs and were slower.)
+// An invalid prefill chunk is flagged once, by its sequence's first job.
+__device__ __forceinline__ void flag_bad_chunk(const Params &p, int u) {
+    if (u % p.pairs != 0 || (u / p.pairs) % p.num_kv_heads != 0) return;
+    const int s = u / p.pairs / p.num_kv_heads;
+    const int L = __ldg(p.lens + s), C = __ldg(p.chunks + s);
+    if (C < 0 || C > p.max_chunk || C > L || (int64_t)L > (int64_t)p.max_blocks * kBlockSize)
+        flag_error(p.err, PA_DEVERR_CHUNK);
+}
+
+// Streams that consume key tile j of a job (bit t = stream t).
+__device__ __forceinline__ unsigned consumers(const Job &jb, int j) { return jb.two ? 3u : (1u << (j & 1)); }
+// Does stream t take part in the job (it has at least one key tile)?
+__device__ __forceinline__ bool stream_used(const Job &jb, int t) { return jb.two || jb.ntiles > t; }
+// Q buffer of stream t: a two-tile job uses both; a one-tile job alternates
+// buffers with the job count, so the next job's Q loads during this one.
+__device__ __forceinline__ int q_buffer(const Job &jb, int t, int njob) { return jb.two ? t : (njob & 1); }
+
 template <int G, bool kGroup>
 __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_constant__ Params p) {
-    extern __shared__ unsigned char smem_raw[];
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     const uint32_t sbase = smem_u32(smem);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint64_t *q_full = bars + 0;
-    uint64_t *k_full = bars + 1;    // [2] K tile landed
-    uint64_t *k_empty = bars + 3;   // [2] its QK is done: the K stage may be refilled
-    uint64_t *v_full = bars + 5;    // [2] V tile landed
-    uint64_t *v_empty = bars + 7;   // [2] its PV is done: the V stage may be refilled
-    uint64_t *s_full = bars + 9;
-    uint64_t *p_full = bars + 10;
-    uint64_t *pv_done = bars + 11;
-    uint64_t *mma_idle = bars + 12;
-    uint64_t *red_full = bars + 13;  // [2]
-    uint64_t *l_full = bars + 15;
-    uint64_t *q_empty = bars + 16;  // a unit's last QK is done: Q may be rewritten
-    uint64_t *o_free = bars + 17;   // the softmax warps have read a unit's O
-    int *tab = reinterpret_cast<int *>(smem + kOffTab);  // [K, V loader][2][8]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
-    volatile int *go = reinterpret_cast<volatile int *>(smem + kOffMisc + 8);  // [K, V loader]
-    int *gcum = reinterpret_cast<int *>(smem + kOffGcum);
-    const int64_t hs = (int64_t)kD * 2;  // bytes per (row, head)
+    float2 *mlx = reinterpret_cast<float2 *>(smem + kOffMl);  // [2][128]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // ---- the work of this CTA
-    int u0 = 0, nunits = 1, ngroups = 0;
-    Job jb;
+    int njobs;
     if constexpr (kGroup) {
         // launched behind the detection kernel: its group list must be complete;
         // then the per-sequence decode may start (it reads only detection output)
         grid_dep_wait();
         grid_dep_launch();
-        nunits = __ldg(p.meta + 1);
-        ngroups = __ldg(p.meta);
-        u0 = blockIdx.x;
-        if (u0 >= nunits) return;
+        njobs = __ldg(p.meta + 1);
     } else {
-        constexpr int kRowsPerTile = kTileM / G;
-        const int s = blockIdx.z, h = blockIdx.y;
-        const int i0 = blockIdx.x * kRowsPerTile;
-        const int L = __ldg(p.lens + s), C = __ldg(p.chunks + s);
-        // validate once; an invalid sequence is skipped (flagged by its first tile)
-        if (C < 0 || C > p.max_chunk || C > L || (int64_t)L > (int64_t)p.max_blocks * kBlockSize) {
-            if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) flag_error(p.err, PA_DEVERR_CHUNK);
-            return;
-        }
-        if (i0 >= C) return;
-        const int start = L - C;
-        const int last_row = min(C, i0 + kRowsPerTile) - 1;
-        jb.h = h;
-        jb.q_row_stride = (int64_t)p.num_q_heads * hs;
-        jb.q = p.q + ((int64_t)s * p.max_chunk + i0) * jb.q_row_stride + (int64_t)h * G * hs;
-        jb.out = p.out + ((int64_t)s * p.max_chunk + i0) * jb.q_row_stride + (int64_t)h * G * hs;
-        jb.nrows = (last_row - i0 + 1) * G;
-        jb.trow = p.tables + (int64_t)s * p.max_blocks;
-        jb.nkeys = L;
-        jb.lim0 = start + i0;
-        jb.lim_step = 1;
-        jb.ntiles = (start + last_row + 1 + kTileN - 1) / kTileN;  // keys 0..start+last_row
-        jb.first = jb.part = 0;
+        njobs = p.num_seqs * p.num_kv_heads * p.pairs;
     }
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if ((int)blockIdx.x >= njobs) return;
     if (threadIdx.x == 0) {
-        mbar_init(q_full, 64);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&k_full[i], 64);
-            mbar_init(&k_empty[i], 1);
-            mbar_init(&v_full[i], 64);
-            mbar_init(&v_empty[i], 1);
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bars[kBarFull + i], 2);
+            mbar_init(&bars[kBarEmpty + i], 1);
         }
-        mbar_init(s_full, 1);
-        mbar_init(p_full, kSoftmaxThreads);
-        mbar_init(pv_done, 1);
-        mbar_init(mma_idle, 1);
-        mbar_init(q_empty, 1);
-        mbar_init(o_free, kSoftmaxThreads);
-        mbar_init(&red_full[0], kSoftmaxThreads);
-        mbar_init(&red_full[1], kSoftmaxThreads);
-        mbar_init(l_full, kSoftmaxThreads);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars[kBarQFull + t], 1);
+            mbar_init(&bars[kBarQEmpty + t], 1);
+            mbar_init(&bars[kBarSFull + t], 1);
+            mbar_init(&bars[kBarPFull + t], kSoftmaxThreads / 2);
+            mbar_init(&bars[kBarOFull + t], 1);
+        }
+        mbar_init(&bars[kBarOFree], kSoftmaxThreads);
+        mbar_init(&bars[kBarMl], kSoftmaxThreads);
+        mbar_init(&bars[kBarIdle], 1);
         *abort_flag = 0;
         mbar_init_fence();
     }
-    if constexpr (kGroup) {
-        for (int k = threadIdx.x; k < ngroups; k += kThreads) gcum[k] = __ldg(&p.groups[k].w);
+    if (warp == kLoadWarp && lane == 0) {
+        prefetch_tensormap(&p.qmap);
+        prefetch_tensormap(&p.kmap);
+        prefetch_tensormap(&p.vmap);
     }
     if (warp == kMmaWarp) tmem_alloc(tmem_slot, kTmemCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem, tO = tmem + 128;
 
-    // Barrier phases run on across units: tile jt = tbase + j of the CTA uses
-    // stage jt & 1; q_full, q_empty, l_full and o_free complete once per unit.
-    // Units follow one another without a CTA barrier: the loader streams the
-    // next unit's Q (after q_empty) and K/V tiles while the current one is
-    // still being computed, and the MMA starts the next unit's PV only after
-    // o_free.  Every wait is bounded; after an abort the remaining units fall
-    // through their (failing) waits.
-    int tbase = 0, nu = 0;
-    for (int u = u0; u < nunits; u += (kGroup ? gridDim.x : 1), ++nu) {
-        if constexpr (kGroup) jb = group_job<G, kGroup>(p, gcum, ngroups, u);
-        if (warp < 4) {
-            // -------------------------------------------------------- loaders
-            // Warps 0-1 stream Q and K, warps 2-3 stream V, each group through
-            // its own two-stage ring, two tiles deep.  A K stage comes back as
-            // soon as its QK is done, so K runs ahead of V.  Within a group one
-            // thread waits and the decision reaches the others through shared
-            // memory behind the group's named barrier.
-            const bool is_k = warp < 2;
-            const int t = threadIdx.x & 63;
-            const int gbar = is_k ? 1 : 2;
-            volatile int *gw = go + (is_k ? 0 : 1);
-            int *gtab = tab + (is_k ? 0 : 16);
-            uint64_t *full = is_k ? k_full : v_full;
-            uint64_t *empty = is_k ? k_empty : v_empty;
-            const uint32_t ring_s = sbase + (is_k ? kOffK : kOffV);
-            unsigned char *ring = smem + (is_k ? kOffK : kOffV);
-            const unsigned char *src0 = is_k ? p.kc : p.vc;
-            bool q_ok = true;
-            if (is_k) {
-                // the previous unit's QK must be done with Q
-                if (t == 0) *gw = (nu == 0 || wait_bar(q_empty, (nu - 1) & 1, abort_flag, p.err, p.wait_ns)) ? 1 : 0;
-                named_barrier(gbar, 64);
-                q_ok = *gw != 0;
-                named_barrier(gbar, 64);  // *gw is rewritten by the first tile issue
-                // Q tile: row r = (row group r / G, head r % G); 16 chunks of 16 bytes per row
-                for (int idx = t; q_ok && idx < kTileM * 16; idx += 64) {
-                    const int r = idx >> 4, c = idx & 15;
-                    const uint32_t dst = sbase + kOffQ + swz(r, c);
-                    if (r < jb.nrows)
-                        cp_async16(dst, jb.q + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs + c * 16);
-                    else
-                        *reinterpret_cast<uint4 *>(smem + kOffQ + swz(r, c)) = make_uint4(0, 0, 0, 0);
+    // each warpgroup sets its register count at one instruction that dominates
+    // all of its code
+    if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ loader
+        // Lane 0 issues Q and arms the barriers; lanes 0..7 each own one 16-token
+        // block of a key tile: its table entry (loaded a tile ahead) and its two
+        // TMA boxes.  A stage completes on the TMA bytes plus a second arrival of
+        // lane 0, made once the warp has filled by hand the block that holds the
+        // last keys of a job when they end inside it (V only: its rows past the
+        // keys become zeros -- 0 * (NaN or Inf) would poison the sums).
+        int it = 0;                 // K/V items issued: K(j), V(j) of each job in order
+        int qn[2] = {0, 0};         // loads issued per Q buffer
+        bool ok = true;
+        int njob = 0;
+        for (int u = blockIdx.x; ok && u < njobs; u += gridDim.x) {
+            Job jb;
+            if (!make_job<G, kGroup>(p, u, jb)) {
+                if constexpr (!kGroup) {
+                    if (lane == 0) flag_bad_chunk(p, u);
                 }
-                cp_async_commit();
+                continue;
             }
-            // table entry of block t of tile j (threads t < 8; -1: past the keys),
-            // loaded one tile ahead so its latency hides behind the current tile
-            auto table_entry = [&](int j) -> int {
-                const int b = j * 8 + t;
-                return (t < 8 && b * kBlockSize < jb.nkeys) ? __ldg(jb.trow + b) : -1;
-            };
-            int next_e = table_entry(0);
-            auto issue_tile = [&](int j) -> bool {
-                const int jt = tbase + j, st = jt & 1;
-                if (t == 0) *gw = (jt < 2 || wait_bar(&empty[st], ((jt >> 1) - 1) & 1, abort_flag, p.err, p.wait_ns)) ? 1 : 0;
-                if (t < 8) {
-                    int e = next_e;
-                    if (j * 8 + t < (jb.nkeys + kBlockSize - 1) / kBlockSize && (e < 0 || e >= p.num_blocks)) {
-                        flag_error(p.err, PA_DEVERR_BLOCK_ID);
-                        e = -1;
-                    }
-                    gtab[st * 8 + t] = e;
-                    next_e = table_entry(j + 1);
-                }
-                named_barrier(gbar, 64);
-                const bool ok = *gw != 0;
-                if (ok) {
-                    const uint32_t dst0 = ring_s + st * kTileBytes;
-                    unsigned char *gen0 = ring + st * kTileBytes;
-                    for (int idx = t; idx < kTileN * 16; idx += 64) {
-                        const int n = idx >> 4, c = idx & 15;
-                        const int key = j * kTileN + n;
-                        const int blk = gtab[st * 8 + (n >> 4)];
-                        const uint32_t off = swz(n, c);
-                        if (blk >= 0 && key < jb.nkeys) {
-                            const int64_t src = (((int64_t)blk * p.num_kv_heads + jb.h) * kBlockSize + (n & 15)) * hs + c * 16;
-                            cp_async16(dst0 + off, src0 + src);
-                        } else {  // past the keys or a bad id: zeros (0 * garbage must not reach the sums)
-                            *reinterpret_cast<uint4 *>(gen0 + off) = make_uint4(0, 0, 0, 0);
-                        }
+            // Q tiles: a buffer is rewritten once the QKs of its previous use are done
+            const int nq = jb.two ? 2 : 1;
+            for (int t = 0; ok && t < nq; ++t) {
+                const int b = q_buffer(jb, t, njob);
+                if (lane == 0) {
+                    ok = qn[b] == 0 || wait_bar(&bars[kBarQEmpty + b], (qn[b] - 1) & 1, abort_flag, p);
+                    if (ok) {
+                        mbar_arrive_expect_tx(&bars[kBarQFull + b], kTileBytes);
+                        const uint32_t dst = sbase + kOffQ + b * kTileBytes;
+                        tma_load_3d(dst, &p.qmap, 0, jb.h * G, jb.qz[t], &bars[kBarQFull + b]);
+                        tma_load_3d(dst + kHalf, &p.qmap, 64, jb.h * G, jb.qz[t], &bars[kBarQFull + b]);
                     }
                 }
-                cp_async_commit();
-                named_barrier(gbar, 64);  // gtab and *gw are rewritten by the next issue
-                return ok;
+                ok = __shfl_sync(kFull, ok, 0);
+                if (ok) ++qn[b];
+            }
+            const int nblk = (jb.nkeys + kBlockSize - 1) / kBlockSize;
+            const int tail = jb.nkeys % kBlockSize;  // tokens in a partly filled last block (0: none)
+            auto entry = [&](int j) -> int {          // this lane's block of tile j: physical id, or -1
+                const int b = j * 8 + lane;
+                if (lane >= 8 || b >= nblk) return -1;
+                const int e = __ldg(jb.trow + b);
+                if (e < 0 || e >= p.num_blocks) {
+                    flag_error(p.err, PA_DEVERR_BLOCK_ID);
+                    return -1;
+                }
+                return e;
             };
-            bool ok = q_ok && jb.ntiles > 0 && issue_tile(0);
+            int cur_e = entry(0);
             for (int j = 0; ok && j < jb.ntiles; ++j) {
-                const bool more = j + 1 < jb.ntiles;
-                if (more && !issue_tile(j + 1)) break;
-                // copy groups so far: (Q,) tiles 0..j (+ j+1): all but the newest are done
-                if (more) cp_async_wait<1>(); else cp_async_wait<0>();
-                fence_proxy_async_smem();
-                if (is_k && j == 0) mbar_arrive(q_full);
-                mbar_arrive(&full[(tbase + j) & 1]);
+                const int next_e = j + 1 < jb.ntiles ? entry(j + 1) : -1;
+                // invalid or past the keys: a coordinate outside the map reads zeros
+                const int z = cur_e >= 0 ? cur_e * p.num_kv_heads + jb.h : -1;
+                // block of this tile filled by hand (V only), or -1
+                const int hand = (tail != 0 && (jb.nkeys - 1) / kTileN == j) ? (jb.nkeys - 1) / kBlockSize - j * 8 : -1;
+                for (int kv = 0; kv < 2; ++kv) {
+                    const int st = it % kStages;
+                    const bool by_hand = kv == 1 && hand >= 0;
+                    if (lane == 0) {
+                        ok = it < kStages || wait_bar(&bars[kBarEmpty + st], ((it / kStages) - 1) & 1, abort_flag, p);
+                        if (ok) mbar_arrive_expect_tx(&bars[kBarFull + st], by_hand ? kTileBytes - 2 * kBlockBytes : kTileBytes);
+                    }
+                    ok = __shfl_sync(kFull, ok, 0);
+                    if (!ok) break;
+                    const CUtensorMap *map = kv ? &p.vmap : &p.kmap;
+                    const uint32_t dst = sbase + kOffRing + st * kTileBytes + lane * kBlockBytes;
+                    if (lane < 8 && !(by_hand && lane == hand)) {
+                        tma_load_3d(dst, map, 0, 0, z, &bars[kBarFull + st]);
+                        tma_load_3d(dst + kHalf, map, 64, 0, z, &bars[kBarFull + st]);
+                    }
+                    if (by_hand) {
+                        const int e = __shfl_sync(kFull, cur_e, hand);
+                        unsigned char *base = smem + kOffRing + st * kTileBytes + hand * kBlockBytes;
+                        const unsigned char *src =
+                            e >= 0 ? p.vc + ((int64_t)e * p.num_kv_heads + jb.h) * kBlockSize * (kD * 2) : nullptr;
+                        // 16 rows x 16 chunks of 16 bytes, stored as TMA would (128-byte swizzle)
+                        for (int idx = lane; idx < kBlockSize * 16; idx += 32) {
+                            const int rr = idx >> 4, c = idx & 15;
+                            uint4 v = make_uint4(0, 0, 0, 0);
+                            if (src && rr < tail) v = *reinterpret_cast<const uint4 *>(src + rr * (kD * 2) + c * 16);
+                            const int row = hand * kBlockSize + rr;  // row inside the 128-row tile
+                            *reinterpret_cast<uint4 *>(base - hand * kBlockBytes + (c >> 3) * kHalf + row * 128 +
+                                                       (((c & 7) ^ (row & 7)) << 4)) = v;
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                    }
+                    if (lane == 0) mbar_arrive(&bars[kBarFull + st]);
+                    ++it;
+                }
+                cur_e = next_e;
             }
-            cp_async_wait<0>();  // nothing may land after an abort
-        } else if (warp == kMmaWarp) {
-            // -------------------------------------------------------- MMA issuer
-            if (lane == 0) {
-                constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
-                bool ok = wait_bar(q_full, nu & 1, abort_flag, p.err, p.wait_ns);
+            ++njob;
+        }
+        // nothing may land after the CTA exits: wait for every stage still in flight
+        if (lane == 0) {
+            for (int k = std::max(0, it - kStages); k < it; ++k)
+                mbar_wait_drain(&bars[kBarFull + k % kStages], (k / kStages) & 1);
+            for (int b = 0; b < 2; ++b)
+                if (qn[b] > 0) mbar_wait_drain(&bars[kBarQFull + b], (qn[b] - 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
+            int it = 0;                  // K/V items consumed
+            int qn[2] = {0, 0};          // uses per Q buffer
+            int npf[2] = {0, 0};         // P_t tiles consumed
+            int njob = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; ok && u < njobs; u += gridDim.x) {
+                Job jb;
+                if (!make_job<G, kGroup>(p, u, jb)) continue;
+                const int nq = jb.two ? 2 : 1;
+                int qb[2];
+                for (int t = 0; t < 2; ++t) qb[t] = q_buffer(jb, t, njob);
+                for (int t = 0; ok && t < nq; ++t) {
+                    ok = wait_bar(&bars[kBarQFull + qb[t]], qn[qb[t]] & 1, abort_flag, p);
+                    ++qn[qb[t]];
+                }
+                if (!ok) break;
+                int pend[2] = {-1, -1};     // key tile whose PV is still to be issued, per stream
+                bool first_pv[2] = {true, true};
+                bool o_ready = njob == 0;   // the previous job's O has been read
+                const int it0 = it;
+                // PV_t of key tile jp (V item it0 + 2 jp + 1)
+                auto issue_pv = [&](int t, int jp) -> bool {
+                    if (!o_ready) {
+                        if (!wait_bar(&bars[kBarOFree], (njob - 1) & 1, abort_flag, p)) return false;
+                        o_ready = true;
+                    }
+                    if (!wait_bar(&bars[kBarPFull + t], npf[t] & 1, abort_flag, p)) return false;
+                    ++npf[t];
+                    const int iv = it0 + 2 * jp + 1, st = iv % kStages;
+                    if (!wait_bar(&bars[kBarFull + st], (iv / kStages) & 1, abort_flag, p)) return false;
+                    tc_fence_after();
+                    const uint32_t va = sbase + kOffRing + st * kTileBytes;
+                    const uint32_t tP = tmem + t * 128, tO = tmem + 256 + t * 128;
+#pragma unroll
+                    for (int kk = 0; kk < kTileN / 16; ++kk)
+                        tc_mma_ts(tO, tP + kk * 8, smem_desc(va + kk * 2048, kHalf, 1024), kIdPV,
+                                  !first_pv[t] || kk > 0);
+                    first_pv[t] = false;
+                    // V(jp) is free once its last consumer's PV is done
+                    if (!jb.two || t == 1) tc_commit(&bars[kBarEmpty + st]);
+                    return true;
+                };
                 for (int j = 0; ok && j < jb.ntiles; ++j) {
-                    const int jt = tbase + j, st = jt & 1;
-                    if (!wait_bar(&k_full[st], (jt >> 1) & 1, abort_flag, p.err, p.wait_ns)) break;
-                    tc_fence_after();
-                    const uint32_t qa = sbase + kOffQ, ka = sbase + kOffK + st * kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < kD / 16; ++kk) {
-                        const uint32_t koff = (kk & 3) * 32 + (kk >> 2) * kHalf;
-                        tc_mma(tS, smem_desc(qa + koff, 16, 1024), smem_desc(ka + koff, 16, 1024), kIdQK, kk > 0);
-                    }
-                    tc_commit(s_full);
-                    tc_commit(&k_empty[st]);
-                    if (j == jb.ntiles - 1) tc_commit(q_empty);
-                    if (!wait_bar(p_full, jt & 1, abort_flag, p.err, p.wait_ns)) break;
-                    // the first PV overwrites O: the previous unit's O must have been read
-                    if (j == 0 && nu > 0 && !wait_bar(o_free, (nu - 1) & 1, abort_flag, p.err, p.wait_ns)) break;
-                    if (!wait_bar(&v_full[st], (jt >> 1) & 1, abort_flag, p.err, p.wait_ns)) break;
-                    tc_fence_after();
-                    const uint32_t pa_ = sbase + kOffP, va = sbase + kOffV + st * kTileBytes;
-#pragma unroll
-                    for (int kk = 0; kk < kTileN / 16; ++kk) {
-                        const uint32_t poff = (kk & 3) * 32 + (kk >> 2) * kHalf;
-                        tc_mma(tO, smem_desc(pa_ + poff, 16, 1024), smem_desc(va + kk * 2048, kHalf, 1024), kIdPV,
-                               j > 0 || kk > 0);
-                    }
-                    tc_commit(pv_done);
-                    tc_commit(&v_empty[st]);
-                }
-            }
-            __syncwarp();
-        } else {
-            // -------------------------------------------------------- softmax
-            // Warp w owns TMEM lane quadrant w % 4 (rows 32*(w%4)..+31) and column
-            // half hf of S, O and P.  The two halves of a row trade their partial
-            // maxima through shared memory each tile (bounded mbarrier) and add
-            // their partial sums at the end.
-            const int qd = warp & 3, hf = (warp - 4) >> 2;
-            const int r = qd * 32 + lane;                // query row = TMEM lane
-            const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
-            const uint32_t cS = tS + lane_off + hf * 64, cO = tO + lane_off + hf * 64;
-            float *red = reinterpret_cast<float *>(smem + kOffRed);    // [2][2][128]
-            float *lsum = reinterpret_cast<float *>(smem + kOffLsum);  // [2][128]
-            const bool row_ok = r < jb.nrows;
-            const bool warp_rows = __any_sync(kFull, row_ok);         // any real row in this warp
-            const int lim = jb.lim0 + jb.lim_step * (r / G);          // last key this row may see
-            float m = -INFINITY, l = 0.f;
-            bool live = true;
-            for (int j = 0; j < jb.ntiles; ++j) {
-                const int jt = tbase + j;
-                const int key0 = j * kTileN + hf * 64;                // first key of this half
-                // the whole half is visible to every row of the warp: no per-key test
-                const bool open = __all_sync(kFull, row_ok && lim >= key0 + 63);
-                live = live && wait_bar(s_full, jt & 1, abort_flag, p.err, p.wait_ns);
-                live = __all_sync(kFull, live);
-                if (!live) break;
-                tc_fence_after();
-                // pass 1: partial row max of the scaled, masked scores
-                float mx = -INFINITY;
-                if (warp_rows) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float sv[32];
-                        tmem_ld32(cS + c * 32, sv);
-                        tmem_wait_ld();
-                        if (open) {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) mx = fmaxf(mx, sv[k] * p.scale_log2);
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k)
-                                if (row_ok && key0 + c * 32 + k <= lim) mx = fmaxf(mx, sv[k] * p.scale_log2);
+                    const int ik = it0 + 2 * j, sk = ik % kStages;
+                    const unsigned cons = consumers(jb, j);
+                    bool k_ready = false;
+                    for (int t = 0; t < 2; ++t) {
+                        if (!(cons >> t & 1u)) continue;
+                        if (pend[t] >= 0 && !issue_pv(t, pend[t])) {
+                            ok = false;
+                            break;
                         }
-                    }
-                }
-                float *rb = red + (jt & 1) * 256;
-                rb[hf * 128 + r] = mx;
-                mbar_arrive(&red_full[jt & 1]);
-                live = wait_bar(&red_full[jt & 1], (jt >> 1) & 1, abort_flag, p.err, p.wait_ns);
-                live = __all_sync(kFull, live);
-                if (!live) break;
-                mx = fmaxf(rb[r], rb[128 + r]);
-                const float m_new = fmaxf(m, mx);
-                const float m_use = m_new == -INFINITY ? 0.f : m_new;
-                const float alpha = fast_exp2(m - m_use);
-                if (j > 0) {
-                    // P and O are still in use by the previous tile's PV
-                    live = wait_bar(pv_done, (jt - 1) & 1, abort_flag, p.err, p.wait_ns);
-                    live = __all_sync(kFull, live);
-                    if (!live) break;
-                    tc_fence_after();
-                    if (warp_rows && __any_sync(kFull, alpha != 1.f)) {
-#pragma unroll
-                        for (int c = 0; c < 2; ++c) {
-                            float ov[32];
-                            tmem_ld32(cO + c * 32, ov);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) ov[k] *= alpha;
-                            tmem_st32(cO + c * 32, ov);
-                        }
-                        tmem_wait_st();
-                    }
-                }
-                // pass 2: P = 2^(s - m) as bf16 into this half of the K-major swizzled A tile
-                float rs = 0.f;
-                if (warp_rows) {
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float sv[32];
-                        tmem_ld32(cS + c * 32, sv);
-                        tmem_wait_ld();
-                        if (open) {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                sv[k] = fast_exp2(sv[k] * p.scale_log2 - m_use);
-                                rs += sv[k];
+                        if (!k_ready) {
+                            if (!wait_bar(&bars[kBarFull + sk], (ik / kStages) & 1, abort_flag, p)) {
+                                ok = false;
+                                break;
                             }
-                        } else {
-#pragma unroll
-                            for (int k = 0; k < 32; ++k) {
-                                sv[k] = (row_ok && key0 + c * 32 + k <= lim) ? fast_exp2(sv[k] * p.scale_log2 - m_use) : 0.f;
-                                rs += sv[k];
-                            }
+                            tc_fence_after();
+                            k_ready = true;
                         }
+                        const uint32_t qa = sbase + kOffQ + qb[t] * kTileBytes;
+                        const uint32_t ka = sbase + kOffRing + sk * kTileBytes;
+                        const uint32_t tS = tmem + t * 128;
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const float *x = &sv[q * 8];
-                            const uint4 w = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                                                       pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-                            *reinterpret_cast<uint4 *>(smem + kOffP + swz(r, hf * 8 + c * 4 + q)) = w;
+                        for (int kk = 0; kk < kD / 16; ++kk) {
+                            const uint32_t koff = (kk & 3) * 32 + (kk >> 2) * kHalf;
+                            tc_mma_ss(tS, smem_desc(qa + koff, 16, 1024), smem_desc(ka + koff, 16, 1024), kIdQK,
+                                      kk > 0);
                         }
+                        tc_commit(&bars[kBarSFull + t]);
+                        pend[t] = j;
+                    }
+                    if (!ok) break;
+                    tc_commit(&bars[kBarEmpty + sk]);  // K(j) is free once its QKs are done
+                    if (j == jb.ntiles - 1) {          // the job's last QKs: its Q buffers are free
+                        tc_commit(&bars[kBarQEmpty + qb[0]]);
+                        if (jb.two) tc_commit(&bars[kBarQEmpty + qb[1]]);
                     }
                 }
-                l = l * alpha + rs;
-                m = m_new;
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(p_full);
-            }
-            if (live) live = wait_bar(pv_done, (tbase + jb.ntiles - 1) & 1, abort_flag, p.err, p.wait_ns);
-            live = __all_sync(kFull, live);
-            if (live) {
-                lsum[hf * 128 + r] = l;
-                mbar_arrive(l_full);
-                live = wait_bar(l_full, nu & 1, abort_flag, p.err, p.wait_ns);
-                live = __all_sync(kFull, live);
-            }
-            if (live && warp_rows) {
-                tc_fence_after();
-                const float lt = lsum[r] + lsum[128 + r];
-                if constexpr (kGroup) {
-                    const int64_t wrow = ((int64_t)(jb.first + r / G) * p.num_q_heads + jb.h * G + r % G) * p.max_parts + jb.part;
-                    float *dst = p.ws_acc + wrow * kD + hf * 64;
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float ov[32];
-                        tmem_ld32(cO + c * 32, ov);
-                        tmem_wait_ld();
-                        if (row_ok) {
-#pragma unroll
-                            for (int k = 0; k < 32; k += 4)
-                                *reinterpret_cast<float4 *>(dst + c * 32 + k) = make_float4(ov[k], ov[k + 1], ov[k + 2], ov[k + 3]);
-                        }
+                for (int t = 0; ok && t < 2; ++t) {
+                    if (pend[t] < 0) continue;
+                    if (!issue_pv(t, pend[t])) {
+                        ok = false;
+                        break;
                     }
-                    if (row_ok && hf == 0) p.ws_ml[wrow] = make_float2(m, lt);
-                } else {
-                    const float inv = lt > 0.f ? 1.f / lt : 0.f;
-                    unsigned char *dst = jb.out + (int64_t)(r / G) * jb.q_row_stride + (int64_t)(r % G) * hs + hf * 128;
-#pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float ov[32];
-                        tmem_ld32(cO + c * 32, ov);
-                        tmem_wait_ld();
-                        if (row_ok) {
-#pragma unroll
-                            for (int k = 0; k < 32; k += 8) {
-                                const uint4 w = make_uint4(pack_bf16x2(ov[k] * inv, ov[k + 1] * inv),
-                                                           pack_bf16x2(ov[k + 2] * inv, ov[k + 3] * inv),
-                                                           pack_bf16x2(ov[k + 4] * inv, ov[k + 5] * inv),
-                                                           pack_bf16x2(ov[k + 6] * inv, ov[k + 7] * inv));
-                                *reinterpret_cast<uint4 *>(dst + (c * 32 + k) * 2) = w;
-                            }
-                        }
-                    }
+                    tc_commit(&bars[kBarOFull + t]);
                 }
+                it = it0 + 2 * jb.ntiles;
+                ++njob;
             }
-            // this unit's O has been read (or was never needed): the MMA may
-            // overwrite it with the next unit's first PV
-            if (live) {
-                tc_fence_before();
-                mbar_arrive(o_free);
+            // everything issued has completed once this arrives
+            tc_commit(&bars[kBarIdle]);
+            if (!mbar_wait_drain(&bars[kBarIdle], 0)) {
+                *abort_flag = 1;
+                flag_error(p.err, PA_DEVERR_TIMEOUT);
             }
         }
-        tbase += jb.ntiles;
+        __syncwarp();
     }
-    if (warp == kMmaWarp && lane == 0) {
-        // everything issued has completed once this arrives
-        tc_commit(mma_idle);
-        if (!mbar_wait_drain(mma_idle, 0)) {
-            *abort_flag = 1;
-            flag_error(p.err, PA_DEVERR_TIMEOUT);
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        // ------------------------------------------------------------ softmax
+        // Stream t = warp / 4; one row per thread (tensor-memory lane 32 (warp % 4) + lane).
+        const int t = warp >> 2, qd = warp & 3;
+        const int r = qd * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+        const uint32_t tS = tmem + lane_off + t * 128;
+        const float sl2 = p.scale_log2;
+        int ns = 0;             // S_t fills seen
+        int no[2] = {0, 0};     // O_t completions, both streams
+        int njob = 0;
+        bool live = true;
+        for (int u = blockIdx.x; live && u < njobs; u += gridDim.x) {
+            Job jb;
+            if (!make_job<G, kGroup>(p, u, jb)) continue;
+            const int tile = jb.two ? t : 0;  // query tile whose rows this thread's lane holds
+            const bool row_ok = r < jb.nrows[tile];
+            const bool warp_rows = __any_sync(kFull, row_ok);
+            // last key this row may see (-1: a padding row sees nothing)
+            const int lim = row_ok ? jb.lim0[tile] + jb.lim_step * (r / G) : -1;
+            float m = -INFINITY, l = 0.f;
+            bool first = true;
+            if (stream_used(jb, t)) {
+                for (int j = 0; j < jb.ntiles; ++j) {
+                    if (!(consumers(jb, j) >> t & 1u)) continue;
+                    live = live && wait_bar(&bars[kBarSFull + t], ns & 1, abort_flag, p);
+                    live = __all_sync(kFull, live);
+                    if (!live) break;
+                    ++ns;
+                    tc_fence_after();
+                    if (warp_rows) {
+                        const int key0 = j * kTileN;
+                        float sv[kTileN];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
+                        tmem_wait_ld();
+                        // every key of the tile visible to every row of the warp: no per-key test
+                        const bool open = __all_sync(kFull, lim >= key0 + kTileN - 1);
+                        // row max of the scaled visible scores
+                        float mx = -INFINITY;
+                        if (sl2 >= 0.f) {
+                            float a = -INFINITY;
+                            if (open) {
+#pragma unroll
+                                for (int k = 0; k < kTileN; ++k) a = fmaxf(a, sv[k]);
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < kTileN; ++k) a = key0 + k <= lim ? fmaxf(a, sv[k]) : a;
+                            }
+                            mx = a == -INFINITY ? -INFINITY : a * sl2;
+                        } else {
+                            float a = INFINITY;
+#pragma unroll
+                            for (int k = 0; k < kTileN; ++k) a = key0 + k <= lim ? fminf(a, sv[k]) : a;
+                            mx = a == INFINITY ? -INFINITY : a * sl2;
+                        }
+                        if (mx != mx) mx = -INFINITY;
+                        const float m_new = fmaxf(m, mx);
+                        float alpha = 1.f;
+                        bool resc = false;
+                        if (first) {
+                            m = m_new;
+                        } else if (m_new > m + kRescaleLog2) {
+                            alpha = fast_exp2(m - m_new);  // m = -inf: O holds zeros, alpha 0
+                            m = m_new;
+                            resc = true;
+                        }
+                        if (__any_sync(kFull, resc)) {
+                            // O_t is idle: its last PV completed before this S was written
+                            const uint32_t tO = tmem + lane_off + 256 + t * 128;
+#pragma unroll 1
+                            for (int c = 0; c < 8; ++c) {
+                                float ov[16];
+                                tmem_ld16(tO + c * 16, ov);
+                                tmem_wait_ld();
+                                uint32_t w[16];
+#pragma unroll
+                                for (int k = 0; k < 16; ++k) w[k] = __float_as_uint(ov[k] * alpha);
+                                tmem_st16(tO + c * 16, w);
+                            }
+                        }
+                        l *= alpha;
+                        const float m_use = m == -INFINITY ? 0.f : m;
+                        // P = 2^(s * scale - m) as bf16 pairs over columns 0..63 of S_t
+                        float2 acc = make_float2(0.f, 0.f);
+                        const float2 sc2 = make_float2(sl2, sl2), nm2 = make_float2(-m_use, -m_use);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int k = 0; k < 16; ++k) {
+                                const int e = c * 32 + 2 * k;
+                                float2 x = __ffma2_rn(make_float2(sv[e], sv[e + 1]), sc2, nm2);
+                                x.x = fast_exp2(x.x);
+                                x.y = fast_exp2(x.y);
+                                if (!open) {
+                                    if (key0 + e > lim) x.x = 0.f;
+                                    if (key0 + e + 1 > lim) x.y = 0.f;
+                                }
+                                acc = __fadd2_rn(acc, x);
+                                w[k] = pack_bf16x2(x.x, x.y);
+                            }
+                            tmem_st16(tS + c * 16, w);
+                        }
+                        l += acc.x + acc.y;
+                        tmem_wait_st();
+                    }
+                    first = false;
+                    tc_fence_before();
+                    mbar_arrive(&bars[kBarPFull + t]);
+                }
+            }
+            if (!live) break;
+            // ---- epilogue: publish this stream's (m, l), then the output rows
+            mlx[t * 128 + r] = make_float2(m, l);
+            mbar_arrive(&bars[kBarMl]);
+            live = wait_bar(&bars[kBarMl], njob & 1, abort_flag, p);
+            live = __all_sync(kFull, live);
+            const bool used1 = stream_used(jb, 1);
+            if (live) {
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    if (!stream_used(jb, s2) || (jb.two && s2 != t)) continue;
+                    live = live && wait_bar(&bars[kBarOFull + s2], no[s2] & 1, abort_flag, p);
+                }
+                live = __all_sync(kFull, live);
+            }
+            ++no[0];
+            if (used1) ++no[1];
+            if (live && warp_rows) {
+                tc_fence_after();
+                // columns of this thread: a two-tile job -> all 128 of its own tile;
+                // a one-tile job -> stream t takes columns 64t..64t+63 of the merge
+                const int c0 = jb.two ? 0 : t * 64, ncol = jb.two ? 128 : 64;
+                float f0 = 0.f, f1 = 0.f, M = -INFINITY, lt = 0.f;
+                if (jb.two) {
+                    M = m;
+                    f0 = 1.f;
+                    lt = l;
+                } else {
+                    const float2 a = mlx[r], b = used1 ? mlx[128 + r] : make_float2(-INFINITY, 0.f);
+                    M = fmaxf(a.x, b.x);
+                    if (M != -INFINITY) {
+                        f0 = a.x == -INFINITY ? 0.f : fast_exp2(a.x - M);
+                        f1 = b.x == -INFINITY ? 0.f : fast_exp2(b.x - M);
+                    }
+                    lt = a.y * f0 + b.y * f1;
+                }
+                const uint32_t tO0 = tmem + lane_off + 256 + (jb.two ? t * 128 : 0);
+                const uint32_t tO1 = tmem + lane_off + 384;
+                const bool any0 = __any_sync(kFull, f0 != 0.f);
+                const bool any1 = __any_sync(kFull, f1 != 0.f);
+                const float inv = kGroup ? 1.f : (lt > 0.f ? 1.f / lt : 0.f);
+                for (int c = c0; c < c0 + ncol; c += 32) {
+                    float o[32], o1[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) o[k] = o1[k] = 0.f;
+                    if (any0) tmem_ld32(tO0 + c, o);
+                    if (any1) tmem_ld32(tO1 + c, o1);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) {
+                        float v = f0 != 0.f ? o[k] * f0 : 0.f;
+                        if (f1 != 0.f) v = fmaf(o1[k], f1, v);
+                        o[k] = v * inv;
+                    }
+                    if (!row_ok) continue;
+                    if constexpr (kGroup) {
+                        const int64_t wrow =
+                            ((int64_t)(jb.first + r / G) * p.num_q_heads + jb.h * G + r % G) * p.max_parts + jb.part;
+                        float *dst = p.ws_acc + wrow * kD + c;
+#pragma unroll
+                        for (int k = 0; k < 32; k += 4)
+                            *reinterpret_cast<float4 *>(dst + k) = make_float4(o[k], o[k + 1], o[k + 2], o[k + 3]);
+                        if (c == c0 && t == 0) p.ws_ml[wrow] = make_float2(M, lt);
+                    } else {
+                        const int64_t hs = (int64_t)kD * 2;
+                        const int rr = (jb.two ? t * kTileM : 0) + r;  // packed row inside the job
+                        unsigned char *dst = p.out + (jb.out_row0 + rr / G) * (int64_t)p.num_q_heads * hs +
+                                             (int64_t)(jb.h * G + rr % G) * hs + c * 2;
+#pragma unroll
+                        for (int k = 0; k < 32; k += 8) {
+                            const uint4 w = make_uint4(pack_bf16x2(o[k], o[k + 1]), pack_bf16x2(o[k + 2], o[k + 3]),
+                                                       pack_bf16x2(o[k + 4], o[k + 5]), pack_bf16x2(o[k + 6], o[k + 7]));
+                            *reinterpret_cast<uint4 *>(dst + k * 2) = w;
+                        }
+                    }
+                }
+            }
+            // this job's O has been read (or was never needed): the MMA may overwrite it
+            if (live) {
+                tc_fence_before();
+                mbar_arrive(&bars[kBarOFree]);
+            }
+            ++njob;
         }
     }
     tc_fence_before();
@@ -628,37 +785,66 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     }
 }
 
-template <int G>
-cudaError_t launch_g(const PrefillLaunch &a, const Params &prm, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<G, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
-    if (e != cudaSuccess) return e;
-    constexpr int rows = kTileM / G;
-    dim3 grid((unsigned)((a.max_chunk + rows - 1) / rows), (unsigned)a.cache.num_kv_heads, (unsigned)a.num_seqs);
-    attn_tile_kernel<G, false><<<grid, kThreads, kSmemBytes, stream>>>(prm);
-    return cudaGetLastError();
+// ---- tensor maps (host) -------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
 }
 
-template <int G>
-cudaError_t launch_group_g(const Params &prm, int sms, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<G, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+// bf16 rows of 128 elements seen as {128, n1, n2} with byte strides {256,
+// stride2}, box {64, b1, b2}, 128-byte swizzle; coordinates outside read zeros.
+bool encode_map(CUtensorMap *m, const void *base, uint64_t n1, uint64_t n2, uint64_t stride2, uint32_t b1,
+                uint32_t b2) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)n1, (cuuint64_t)(n2 > 0 ? n2 : 1)};
+    const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)stride2};
+    const cuuint32_t box[3] = {64, b1, b2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// K/V pools [num_blocks, Hkv, 16, 128] as {128, 16, num_blocks * Hkv}, box {64, 16, 1}.
+bool encode_cache_maps(Params &prm, const void *kc, const void *vc) {
+    const uint64_t n2 = (uint64_t)prm.num_blocks * prm.num_kv_heads;
+    prm.vc = static_cast<const unsigned char *>(vc);
+    return encode_map(&prm.kmap, kc, kBlockSize, n2, (uint64_t)kBlockSize * kD * 2, kBlockSize, 1) &&
+           encode_map(&prm.vmap, vc, kBlockSize, n2, (uint64_t)kBlockSize * kD * 2, kBlockSize, 1);
+}
+
+template <int G, bool kGroup>
+cudaError_t launch_tiles(const Params &prm, int grid, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(attn_tile_kernel<G, kGroup>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    return launch_after(attn_tile_kernel<G, true>, dim3((unsigned)sms), dim3(kThreads), kSmemBytes, stream,
-                        static_cast<const Params &>(prm));
+    if constexpr (kGroup) {
+        return launch_after(attn_tile_kernel<G, true>, dim3((unsigned)grid), dim3(kThreads), kSmemBytes, stream,
+                            static_cast<const Params &>(prm));
+    } else {
+        attn_tile_kernel<G, false><<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(prm);
+        return cudaGetLastError();
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
-    static_assert(kSmemBytes <= 232448, "prefill smem over the sm_100 limit");
+    static_assert(kSmemBytes <= 232448, "tile kernel shared memory over the sm_100 limit");
     if (a.cache.dtype != PA_BF16 || a.cache.head_dim != kD) return cudaErrorNotSupported;
-    if (a.num_seqs > 65535) return cudaErrorNotSupported;
+    const int G = a.num_q_heads / a.cache.num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return cudaErrorNotSupported;
     Params prm;
     std::memset(&prm, 0, sizeof(prm));
-    prm.q = static_cast<const unsigned char *>(a.query);
-    prm.kc = static_cast<const unsigned char *>(a.key_cache);
-    prm.vc = static_cast<const unsigned char *>(a.value_cache);
     prm.tables = a.block_tables;
     prm.lens = a.context_lens;
     prm.chunks = a.chunk_lens;
@@ -670,23 +856,34 @@ cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream) {
     prm.num_q_heads = a.num_q_heads;
     prm.num_kv_heads = a.cache.num_kv_heads;
     prm.num_blocks = a.cache.num_blocks;
+    prm.pairs = (a.max_chunk * G + 2 * kTileM - 1) / (2 * kTileM);
     prm.scale_log2 = a.scale * kLog2e;
     prm.wait_ns = wait_limit_ns();
-    switch (a.num_q_heads / a.cache.num_kv_heads) {
-        case 1: return launch_g<1>(a, prm, stream);
-        case 2: return launch_g<2>(a, prm, stream);
-        case 4: return launch_g<4>(a, prm, stream);
-        case 8: return launch_g<8>(a, prm, stream);
-        default: return cudaErrorNotSupported;
+    const int64_t njobs = (int64_t)a.num_seqs * a.cache.num_kv_heads * prm.pairs;
+    if (njobs <= 0) return cudaSuccess;
+    if (njobs > INT32_MAX) return cudaErrorNotSupported;
+    const uint64_t qrows = (uint64_t)a.num_seqs * a.max_chunk;
+    if (!encode_map(&prm.qmap, a.query, (uint64_t)a.num_q_heads, qrows, (uint64_t)a.num_q_heads * kD * 2, G,
+                    kTileM / G) ||
+        !encode_cache_maps(prm, a.key_cache, a.value_cache))
+        return cudaErrorInvalidValue;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(njobs, num_sms(dev));
+    switch (G) {
+        case 1: return launch_tiles<1, false>(prm, grid, stream);
+        case 2: return launch_tiles<2, false>(prm, grid, stream);
+        case 4: return launch_tiles<4, false>(prm, grid, stream);
+        default: return launch_tiles<8, false>(prm, grid, stream);
     }
 }
 
 cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t stream) {
+    const int G = a.num_q_heads / a.num_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return cudaErrorNotSupported;
     Params prm;
     std::memset(&prm, 0, sizeof(prm));
-    prm.q = static_cast<const unsigned char *>(a.query);
-    prm.kc = static_cast<const unsigned char *>(a.key_cache);
-    prm.vc = static_cast<const unsigned char *>(a.value_cache);
     prm.tables = a.block_tables;
     prm.err = a.err;
     prm.max_blocks = a.max_blocks_per_seq;
@@ -701,12 +898,15 @@ cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t s
     prm.part_tokens = a.partition_size;
     prm.max_parts = a.max_partitions;
     prm.wait_ns = wait_limit_ns();
-    switch (a.num_q_heads / a.num_kv_heads) {
-        case 1: return launch_group_g<1>(prm, sms, stream);
-        case 2: return launch_group_g<2>(prm, sms, stream);
-        case 4: return launch_group_g<4>(prm, sms, stream);
-        case 8: return launch_group_g<8>(prm, sms, stream);
-        default: return cudaErrorNotSupported;
+    if (!encode_map(&prm.qmap, a.query, (uint64_t)a.num_q_heads, (uint64_t)a.num_seqs,
+                    (uint64_t)a.num_q_heads * kD * 2, G, kTileM / G) ||
+        !encode_cache_maps(prm, a.key_cache, a.value_cache))
+        return cudaErrorInvalidValue;
+    switch (G) {
+        case 1: return launch_tiles<1, true>(prm, sms, stream);
+        case 2: return launch_tiles<2, true>(prm, sms, stream);
+        case 4: return launch_tiles<4, true>(prm, sms, stream);
+        default: return launch_tiles<8, true>(prm, sms, stream);
     }
 }
 
