@@ -27,7 +27,6 @@ import hashlib
 import json
 import math
 import os
-import re
 import sys
 import threading
 import time
@@ -178,22 +177,38 @@ def max_over_ranks(x, world):
 
 
 # ----------------------------------------------------------------- profiles
-def recorded_traffic():
-    """DRAM bytes of one pa_append_decode call (all its kernels) from the committed
-    ncu summary, or None if a kernel source changed since the counters were taken."""
-    path = os.path.join(ROOT, "profiles", "decode_gqa8b_prefix_ncu.md")
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    mt = re.search(r"dram bytes per pa_append_decode call \(read\+write\): (\d+)", text)
-    if not mt:
-        return None
-    for name in ("cache_ops.cu", "decode.cu", "prefill.cu"):
-        mh = re.search(name.replace(".", r"\.") + r" sha256: ([0-9a-f]{64})", text)
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gqa8b_prefix_traffic.json")
+
+
+def kernel_sources_sha256():
+    """sha256 of every kernel source that one pa_append_decode call runs."""
+    out = {}
+    for name in ("cache_ops.cu", "decode.cu", "prefill.cu", "pa_common.cuh"):
         src = os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", name)
-        if not mh or hashlib.sha256(open(src, "rb").read()).hexdigest() != mh.group(1):
-            return None
-    return int(mt.group(1))
+        out[name] = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    return out
+
+
+def recorded_traffic():
+    """DRAM bytes (read + write) of one pa_append_decode call, all its kernels, from
+    the committed ncu record -- or None if a kernel source changed since the counters
+    were taken (the record stores the sources' sha256)."""
+    if not os.path.exists(TRAFFIC_RECORD):
+        return None
+    rec = json.load(open(TRAFFIC_RECORD))
+    if rec.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return int(rec["dram_bytes_per_call"])
+
+
+def headline_config(wl, S, max_ctx, mean_ctx, part, world):
+    """The `config` of the headline line, the same for both arms."""
+    return {"workload": WORKLOAD_NAME, "num_seqs": S, "num_q_heads": wl.num_q_heads,
+            "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
+            "prefix_tokens": 512, "group_size": 16, "max_context": int(max_ctx),
+            "mean_context": float(mean_ctx), "partition_size": int(part),
+            "parallelism": f"dp{world} (sequences sharded, no exchange)",
+            "l2": "inputs larger than L2 (126 MB); no flush"}
 
 
 # ----------------------------------------------------------------- our arm
@@ -260,7 +275,6 @@ def run_ours(args):
     assert flag == 0, f"device error flag {flag} during warm-up"
 
     K = args.steps
-    ev_dec = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(torch, local)
     sampler.start()
@@ -269,14 +283,15 @@ def run_ours(args):
     h0 = time.perf_counter()
     e0.record(stream)
     for i in range(K):
-        step_fn(*ev_dec[i])
+        step_fn()
     e1.record(stream)
     torch.cuda.synchronize()
     h1 = time.perf_counter()
     barrier(world)
     sampler.stop()
     ms = e0.elapsed_time(e1)
-    call_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_dec]))
+    # one call per step, back to back: its average duration over the timed region
+    call_ms = ms / K
     ms_max = max_over_ranks(ms, world)
     clocks = sampler.summary(h0, h1)
 
@@ -297,38 +312,97 @@ def run_ours(args):
     dec_ms = float(np.mean([a.elapsed_time(b) for a, b in ev2]))
     assert pa.pa_wait(cache.err_flag) == 0
 
-    # end to end: host buffers in, result out, through the same calls
+    # end to end: every step's inputs from pinned host memory (query, new K/V, slots,
+    # lengths; the block tables only when they change -- here once), the step, and the
+    # output read back to pinned host memory.  Host-to-device and device-to-host copies
+    # run on two streams of their own into two device buffer sets, so step i+1's inputs
+    # and step i's output cross PCIe while a step computes; events order each buffer's
+    # reuse.
     e2e = None
     if not args.no_e2e:
         pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True).copy_(t.cpu())
-        hq, hk, hv, hs = pin(q), pin(k_new), pin(v_new), pin(slots_d)
-        ht, hl = pin(tables_d), pin(lens_d)
-        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, ht, hl))
-        d2h = hout.numel() * hout.element_size()
+        hq, hk, hv, hs, hl = pin(q), pin(k_new), pin(v_new), pin(slots_d), pin(lens_d)
+        ht = pin(tables_d)
+        hout = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+        sets = [dict(q=torch.empty_like(q), k=torch.empty_like(k_new), v=torch.empty_like(v_new),
+                     s=torch.empty_like(slots_d), l=torch.empty_like(lens_d), o=torch.empty_like(out))
+                for _ in range(2)]
+        tab = torch.empty_like(tables_d)
+        h2d_stream, d2h_stream = torch.cuda.Stream(), torch.cuda.Stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]     # inputs of a set landed
+        ev_used = [torch.cuda.Event() for _ in range(2)]   # the step reading a set is done
+        ev_out = [torch.cuda.Event() for _ in range(2)]    # a set's output read back
+        h2d_step = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hs, hl))
+        d2h = hout[0].numel() * hout[0].element_size()
+        tables_bytes = ht.numel() * ht.element_size()
+        state = {"i": 0}
 
         def e2e_step():
-            for dst, src in ((q, hq), (k_new, hk), (v_new, hv), (slots_d, hs), (tables_d, ht), (lens_d, hl)):
-                dst.copy_(src, non_blocking=True)
-            step_fn()
-            hout.copy_(out, non_blocking=True)
+            i = state["i"]
+            b = i & 1
+            st = sets[b]
+            with torch.cuda.stream(h2d_stream):
+                if i == 0:
+                    tab.copy_(ht, non_blocking=True)           # tables: only when they change
+                if i >= 2:
+                    h2d_stream.wait_event(ev_used[b])          # step i-2 has read this set
+                for dst, src in ((st["q"], hq), (st["k"], hk), (st["v"], hv), (st["s"], hs), (st["l"], hl)):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[b].record(h2d_stream)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])                   # step i-2's output was read back
+            pa.pa_append_decode(st["k"], st["v"], st["s"], st["q"], cache.key_cache, cache.value_cache, tab,
+                                st["l"], max_ctx, wl.scale, st["o"], part, ws, cache.err_flag, stream)
+            ev_used[b].record(stream)
+            with torch.cuda.stream(d2h_stream):
+                d2h_stream.wait_event(ev_used[b])
+                hout[b].copy_(st["o"], non_blocking=True)
+                ev_out[b].record(d2h_stream)
+            state["i"] = i + 1
 
         for _ in range(args.warmup):
             e2e_step()
+        torch.cuda.synchronize()
+        state["i"] = 0
         barrier(world)
         torch.cuda.synchronize()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
         for _ in range(K):
             e2e_step()
+        stream.wait_event(ev_out[(K - 1) & 1])              # the last output is on the host
         f1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(f0.elapsed_time(f1), world)
+        ref = out.cpu()
+        assert torch.equal(hout[(K - 1) & 1], ref), "end-to-end output differs from the device-resident step"
         e2e = {"value": round(world * (unique_b + cw_b) * K / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                "ms_per_step": round(e2e_ms / K, 5),
                "seq_steps_per_s": round(world * S * K / (e2e_ms * 1e-3), 1),
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+               "h2d_bytes_per_step": int(h2d_step + tables_bytes / K), "d2h_bytes_per_step": int(d2h),
+               "h2d_tables_bytes_once": int(tables_bytes),
+               "overlap": "h2d and d2h streams, two device buffer sets; tables uploaded once (unchanged "
+                          "across the repeated step)"}
+
+    # the same step with L2 flushed before each call (a 2 x L2 write outside the
+    # timed events): shared prefix blocks can no longer be found in L2 from the
+    # previous step, only within the call
+    flushed = None
+    if not args.no_e2e:
+        l2 = torch.cuda.get_device_properties(local).L2_cache_size
+        scrub = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+        nfl = min(K, 100)
+        evf = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nfl)]
+        for i in range(nfl):
+            scrub.fill_(i & 0xFF)
+            step_fn(*evf[i])
+        torch.cuda.synchronize()
+        fl_ms = float(np.mean([a.elapsed_time(b) for a, b in evf]))
+        flushed = {"ms_per_call": round(fl_ms, 5), "value": round((unique_b + cw_b) / (fl_ms * 1e-3) / 1e9, 2),
+                   "unit": "GB/s", "calls": nfl, "flush_bytes": int(scrub.numel())}
+        del scrub
     flag = pa.pa_wait(cache.err_flag)
     assert flag == 0, f"device error flag {flag}"
 
@@ -338,12 +412,19 @@ def run_ours(args):
         del cache, ws, out, q, k_new, v_new, tables_d, lens_d, slots_d
         torch.cuda.empty_cache()
         rows = run_rows(args.row_reps, peaks0, args.partition)
+        if not args.no_cpu_baseline:
+            for name, cb in cpu_rows(set(ROW_GROUPS)).items():
+                rows.setdefault(name, {})["cpu_baseline"] = cb
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, None, step, tables_h, lens_h, budget_s=args.cpu_seconds)
 
     if rank == 0:
+        # kernels of one pa_append_decode call: the decode chain, plus the write's own
+        # launch unless the shared-prefix chain (4 kernels) takes the write into its first
+        n_dec = pa.pa_decode_launches(S, wl.head_dim, pa.PA_BF16, part)
+        step_launches = n_dec if n_dec == 4 else n_dec + 1
         peaks = load_peaks()
         peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
         achieved = (unique_b + cw_b) / (call_ms * 1e-3) / 1e9
@@ -353,29 +434,25 @@ def run_ours(args):
             "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": round(ms_max / K, 5), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAME, "num_seqs": S, "num_q_heads": wl.num_q_heads,
-                       "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
-                       "prefix_tokens": 512, "group_size": 16, "max_context": max_ctx,
-                       "mean_context": float(np.mean(lens_h)), "partition_size": part,
-                       "parallelism": f"dp{world} (sequences sharded, no exchange)",
-                       "l2": "inputs larger than L2 (126 MB); no flush"},
+            "config": headline_config(wl, S, max_ctx, np.mean(lens_h), part, world),
             "seq_steps_per_s": round(world * S * K / (ms_max * 1e-3), 1),
             "pct_of_8tbs": round(100 * value / world / 8000, 2),
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "logical_gbs": round(world * (logical_b + cw_b) * K / (ms_max * 1e-3) / 1e9, 2),
             "bytes_per_step": {"decode_unique": unique_b, "decode_logical": logical_b, "cache_write": cw_b},
-            "roofline": {"bound": "hbm", "kernel": "pa_append_decode call (cache write + group detection + tcgen05 group tiles + decode_kernel + lse reduce)",
+            "roofline": {"bound": "hbm", "kernel": "pa_append_decode call (cache write fused with group detection, tcgen05 group tiles, decode_kernel, lse reduce)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if peaks else "fallback",
                          "traffic": recorded_traffic(),
                          "call_ms": round(call_ms, 5)},
+            "l2_flushed": flushed,
             "two_calls": {"ms_per_step": round(two_ms, 5),
                           "value": round(world * (unique_b + cw_b) / (two_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                           "pa_decode_ms": round(dec_ms, 5),
                           "pa_decode_gbs": round(unique_b / (dec_ms * 1e-3) / 1e9, 1), "steps": nf},
             "e2e": e2e,
-            "gpu_launches": K * (1 + pa.pa_decode_launches(S, wl.head_dim, pa.PA_BF16, part)),
+            "gpu_launches": K * step_launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
             "rows": rows,
@@ -440,6 +517,36 @@ def _time(fn, reps, warm=3, graph=False):
 ROW_GROUPS = ("mha7b", "fork", "spec", "fp8", "prefix", "long")
 
 
+def _warm_kernels():
+    """One small call of each kernel family before any row is timed, so no row pays
+    for loading the library's kernels (the fork row times single launches)."""
+    import torch
+    import paged_kv_cache_389_b200 as pa
+    wl = workloads.make(3, mini=True)
+    cache, dev = _setup(wl)
+    st = wl.steps[0]
+    slots, _ = cache.plan_append(st.seqs)
+    mb = cache.manager.max_seq_blocks(st.seqs)
+    t, l = cache.manager.build_tables(st.seqs, mb)
+    td, ld, q = torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(), dev(st.q)
+    out = torch.empty_like(q)
+    for part in (0, 64, 512):
+        n = pa.pa_decode_workspace_size(len(st.seqs), wl.num_q_heads, wl.head_dim, int(l.max()), part) if part else 0
+        ws = torch.empty(max(n, 16), dtype=torch.uint8, device="cuda")
+        pa.pa_append_decode(dev(st.k_new), dev(st.v_new), torch.from_numpy(slots).cuda(), q, cache.key_cache,
+                            cache.value_cache, td, ld, int(l.max()), wl.scale, out, part, ws, cache.err_flag)
+    qp = dev(np.zeros((len(st.seqs), 4, wl.num_q_heads, wl.head_dim), np.uint16))
+    pa.pa_prefill_chunk(qp, cache.key_cache, cache.value_cache, td, ld,
+                        torch.full((len(st.seqs),), 4, dtype=torch.int32, device="cuda"), wl.scale,
+                        torch.empty_like(qp), cache.err_flag)
+    # a block copy into the pool's last block (the pool is dropped right after)
+    pa.pa_copy_blocks(cache.key_cache, cache.value_cache,
+                      torch.tensor([[0, wl.num_blocks - 1]], dtype=torch.int32, device="cuda"), cache.err_flag)
+    torch.cuda.synchronize()
+    del cache
+    torch.cuda.empty_cache()
+
+
 def run_rows(reps, peaks, partition=PARTITION, groups=None):
     """Each hot-path row on its own workload; device time, inputs resident in HBM.
     groups: the row groups to run (default all of ROW_GROUPS)."""
@@ -452,6 +559,7 @@ def run_rows(reps, peaks, partition=PARTITION, groups=None):
     hbm = float(peaks["hbm_gbs"]) if peaks else 6650.0
     tf_burst = float(peaks["bf16_tflops"]) if peaks else 1590.0
     rows = {}
+    _warm_kernels()
 
     def dec_entry(name, cache, q, td, ld, maxc, scale, part, bytes_u, bytes_l, nseq):
         out = torch.empty_like(q)
@@ -718,6 +826,116 @@ def cpu_baseline(wl, cache, step, tables_h, lens_h, budget_s=15.0):
     return out
 
 
+def _oracle_setup(wl):
+    """The oracle's pools and block model after the workload's set-up operations."""
+    import oracle
+    from oracle.block_model import BlockManagerModel
+    model = BlockManagerModel(wl.num_blocks, wl.block_size, wl.free_order.tolist())
+    fill = np.nan if wl.dtype == "f32" else 0x7FC0
+    kc = np.full(wl.cache_shape(), fill, wl.np_dtype)
+    vc = np.full(wl.cache_shape(), fill, wl.np_dtype)
+    workloads.replay(wl, model, lambda k, v, sl: oracle.cache_write(k, v, sl, kc, vc))
+    return model, kc, vc
+
+
+def _oracle_step(wl, model, kc, vc, step):
+    """One step of the hot path on the oracle: copy-on-write pairs, the new tokens'
+    cache write, decode of every sequence.  Returns (tables, lens) of the decode."""
+    import oracle
+    slots, pairs = [], []
+    for sq in step.seqs:
+        sl, pr = model.append_slot(sq)
+        slots.append(sl)
+        if pr is not None:
+            pairs.append(pr)
+    if pairs:
+        oracle.copy_blocks(kc, vc, np.array(pairs, np.int32))
+    oracle.cache_write(step.k_new, step.v_new, np.array(slots, np.int64), kc, vc)
+    mb = max(len(model.block_table(sq)) for sq in step.seqs)
+    t, l = model.build_tables(step.seqs, mb)
+    oracle.decode(step.q, kc, vc, t, l, wl.scale)
+    return t, l
+
+
+def cpu_rows(groups, budget_s=12.0):
+    """The oracle, as it stands, timed on the host cores for the rows' workloads
+    (a baseline, not a target): config 1 and 2 steps, config 4's fork / copy-on-write
+    steps (all 16 when they fit the budget, else the first ones), config 5's decode in
+    full and its prefill chunk on one sequence scaled x8.  Returns {row: cpu_baseline}."""
+    import oracle
+    cores, cpu = oracle.num_threads(), _cpu_model()
+    out = {}
+
+    def entry(value, unit, secs, sample):
+        return {"value": round(value, 4), "unit": unit, "cores": cores, "kind": "oracle",
+                "seconds": round(secs, 3), "sample": sample, "cpu": cpu}
+
+    wl = workloads.make(1)
+    model, kc, vc = _oracle_setup(wl)
+    t0 = time.perf_counter()
+    t, l = _oracle_step(wl, model, kc, vc, wl.steps[0])
+    el = time.perf_counter() - t0
+    ub, _ = step_bytes(wl, t, l)
+    out["c1_tiny_fp32"] = entry((ub + cache_write_bytes(wl, len(l))) / el / 1e9, "GB/s", el,
+                                "config 1: the whole step (4 sequences, cache write + decode)")
+    if "mha7b" in groups:
+        wl = workloads.make(2)
+        model, kc, vc = _oracle_setup(wl)
+        t0 = time.perf_counter()
+        t, l = _oracle_step(wl, model, kc, vc, wl.steps[0])
+        el = time.perf_counter() - t0
+        ub, _ = step_bytes(wl, t, l)
+        e = entry((ub + cache_write_bytes(wl, len(l))) / el / 1e9, "GB/s", el,
+                  "config 2: the whole step (64 sequences, cache write + decode, unsplit)")
+        out["a3_decode_mha7b_p0"] = out["a3_decode_mha7b_p1024"] = e
+    if "fork" in groups:
+        wl = workloads.make(4)
+        model, kc, vc = _oracle_setup(wl)
+        n = done = 0
+        ub_sum = 0
+        t0 = time.perf_counter()
+        for st in wl.steps:
+            t, l = _oracle_step(wl, model, kc, vc, st)
+            ub_sum += step_bytes(wl, t, l)[0]
+            n += len(st.seqs)
+            done += 1
+            if time.perf_counter() - t0 > budget_s:
+                break
+        el = time.perf_counter() - t0
+        out["fork_cow_16_steps"] = entry(n / el, "seq_steps/s", el,
+                                         f"config 4: the first {done} of {len(wl.steps)} steps (copy-on-write, "
+                                         f"cache write, decode of 512 sequences)")
+        out["fork_cow_16_steps"]["decode_unique_gbs"] = round(ub_sum / el / 1e9, 4)
+    if "long" in groups:
+        wl = workloads.make(5)
+        model, kc, vc = _oracle_setup(wl)
+        st = wl.steps[0]
+        mb = max(len(model.block_table(sq)) for sq in st.seqs)
+        t, l = model.build_tables(st.seqs, mb)
+        t0 = time.perf_counter()
+        oracle.decode(st.q, kc, vc, t, l, wl.scale)
+        el = time.perf_counter() - t0
+        ub, _ = step_bytes(wl, t, l)
+        e = entry(ub / el / 1e9, "GB/s", el, "config 5: decode of all 8 x 32768-token sequences")
+        out["a4_decode_long_p512"] = out["a4_decode_long_p2048"] = e
+        pf = wl.prefill
+        rows = np.arange(0, pf.chunk, pf.chunk // 64)          # 64 rows of sequence 0, evenly spread
+        mask = np.zeros((len(pf.seqs), pf.chunk), bool)
+        mask[0, rows] = True
+        ch = np.full(len(pf.seqs), pf.chunk, np.int32)
+        t0 = time.perf_counter()
+        oracle.prefill(pf.q, kc, vc, t, l, ch, wl.scale, row_mask=mask)
+        el = time.perf_counter() - t0
+        keys = sum(int(l[0]) - pf.chunk + int(i) + 1 for i in rows)
+        flops = 4.0 * wl.num_q_heads * wl.head_dim * keys
+        scale_up = len(pf.seqs) * pf.chunk / len(rows)
+        out["a5_prefill_chunk_long"] = entry(flops / el / 1e12, "TFLOP/s", el * scale_up,
+                                             f"config 5: {len(rows)} of the 512 chunk rows of sequence 0 (all "
+                                             f"heads) timed; seconds = the timed ones x {scale_up:.0f} for all 8 "
+                                             "sequences' rows")
+    return out
+
+
 def _cpu_model():
     try:
         for line in open("/proc/cpuinfo"):
@@ -738,6 +956,7 @@ def run_reference(args):
     wl = workloads.make(CONFIG_ID)
     model, kc, vc, slots = _oracle_pools(wl)
     S = len(wl.steps[0].seqs)
+    _, lens_all = model.build_tables(wl.steps[0].seqs, max(len(model.block_table(s)) for s in wl.steps[0].seqs))
     one, _ = _time_oracle_steps(wl, model, kc, vc, slots, 1, 1)
     budget = 150.0 / max(1, args.steps + args.warmup)          # seconds of oracle work per step
     n = int(max(1, min(S, budget / max(one, 1e-4))))
@@ -755,8 +974,7 @@ def run_reference(args):
         "value": round(value, 4), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAME, "num_seqs": S, "num_q_heads": wl.num_q_heads,
-                   "num_kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16},
+        "config": headline_config(wl, S, int(lens_all.max()), np.mean(lens_all), args.partition, world),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": f"first {n} of {S} sequences per step "
                                                      "(cache write + decode), fp64 C + OpenMP",
@@ -788,8 +1006,12 @@ def main():
     if args.impl == "reference":
         run_reference(args)
     elif args.rows_only:
-        print(json.dumps({"rows": run_rows(args.row_reps, load_peaks(), args.partition,
-                                           set(args.rows_only.split(",")))}), flush=True)
+        groups = set(args.rows_only.split(","))
+        rows = run_rows(args.row_reps, load_peaks(), args.partition, groups)
+        if not args.no_cpu_baseline:
+            for name, cb in cpu_rows(groups).items():
+                rows.setdefault(name, {})["cpu_baseline"] = cb
+        print(json.dumps({"rows": rows}), flush=True)
     else:
         run_ours(args)
 

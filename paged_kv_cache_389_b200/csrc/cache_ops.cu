@@ -7,6 +7,7 @@
 // copies a whole shared block into a freshly allocated one.
 #include <cuda_fp8.h>
 
+#include "cache_write.cuh"
 #include "pa_common.cuh"
 #include "pa_launch.h"
 
@@ -21,23 +22,8 @@ __global__ void __launch_bounds__(256) cache_write_kernel(
     // a decode launched behind this write (pa_append_decode) may start launching;
     // whatever of it reads the cache waits for this grid to finish
     grid_dep_launch();
-    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t per_token = (int64_t)num_kv_heads * chunks_per_row;
-    const int64_t token = idx / per_token;
-    if (token >= num_tokens) return;
-    const int64_t slot = slot_mapping[token];
-    if (slot < 0) return;  // padding
-    if (slot >= num_slots) {
-        if (idx % per_token == 0) flag_error(err, PA_DEVERR_SLOT);
-        return;
-    }
-    const int64_t rem = idx - token * per_token;      // (head, chunk) inside the token
-    const int64_t head = rem / chunks_per_row;
-    const int64_t chunk = rem - head * chunks_per_row;
-    const int64_t block = slot / kBlockSize, offset = slot % kBlockSize;
-    const int64_t dst = ((block * num_kv_heads + head) * kBlockSize + offset) * chunks_per_row + chunk;
-    key_cache[dst] = key[idx];
-    value_cache[dst] = value[idx];
+    write_chunk((int64_t)blockIdx.x * blockDim.x + threadIdx.x, key, value, slot_mapping, num_tokens, key_cache,
+                value_cache, num_kv_heads, chunks_per_row, num_slots, err);
 }
 
 // FP8 pools: one thread per 8 elements (16 bytes of bf16 in, 8 bytes of e4m3

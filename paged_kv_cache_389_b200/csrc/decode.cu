@@ -55,6 +55,7 @@
 
 #include <cuda_fp8.h>
 
+#include "cache_write.cuh"
 #include "pa_common.cuh"
 #include "pa_launch.h"
 
@@ -184,7 +185,10 @@ struct Unit {
     int fp;          // first_part(s): partitions of s computed by group units
 };
 
-__device__ __forceinline__ int slot_base(int fp) { return fp; }
+// Workspace slot of a sequence's first per-sequence unit: its shared leading
+// partitions (fp of them) are computed together by one group unit per kv head,
+// which writes one partial into slot 0.
+__device__ __forceinline__ int slot_base(int fp) { return fp > 0 ? 1 : 0; }
 
 __device__ __forceinline__ int first_part(const Params &p, int s) {
     return p.first_p ? __ldg(p.first_p + s) : 0;
@@ -801,8 +805,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         v = __shfl_sync(kFull, v, 0);
         return v == INT_MAX ? INT64_MAX : (int64_t)v;
     };
-    // at the start of unit k: the first warp there draws the id of unit k + 2,
-    // after the id of unit k + 1 is out, so that a CTA's ids only grow
+    // near the end of unit k (the first warp to finish its share of it): draw the
+    // id of unit k + 2, after the id of unit k + 1 is out, so that a CTA's ids only
+    // grow; drawn this late, a CTA holds at most one unit beyond the one it works on
     auto claim_ahead = [&](int k) {
         if (!dyn || lane != 0 || k < 1) return;
         const int k2 = k + 2, sl = k2 & 7;
@@ -870,7 +875,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     bool dead = false;       // a hand-over wait timed out
     int uc = 0;
     for (;; ++uc) {
-        claim_ahead(uc);
         // ---- q operands of this unit (tiny, L2 resident)
         MmaState<D> ms;
         F32State<D, G> fs;
@@ -977,6 +981,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         // keep the pipeline full across the merge
         while (n_iss - n_cmp < NS && fetch_one()) {
         }
+        claim_ahead(uc);
 
         // ---- this warp's state into merge slot uc & 1, once the slot's previous
         // unit (uc - 2) has been merged by every warp
@@ -1047,10 +1052,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 // Sequences next to each other in the batch whose tables start with the same
 // physical blocks (forks, a shared system prompt: chenxutan 2.1 / 3.3, devpress
 // 关键设计二) read those blocks once: the shared leading partitions are computed
-// by group units (group, partition, kv head) whose query rows are members x
-// heads, and the per-sequence kernel starts after them.  The result is the same
-// sum -- the group partials land in slots 0..fp-1 of every member, the
-// per-sequence units in the slots after them, and the LSE reduce combines them.
+// by group units (group, kv head) whose query rows are members x heads and whose
+// keys are all the group's shared partitions, and the per-sequence kernel starts
+// after them.  The result is the same sum -- the group partial lands in slot 0
+// of every member, the per-sequence units in the slots after it, and the LSE
+// reduce combines them.
 //
 // Detection is one single-CTA kernel: each sequence's count of leading full
 // blocks shared with its predecessor, then the cut of the batch into groups.
@@ -1060,11 +1066,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 constexpr int kDetectThreads = 1024;
 constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
 constexpr int kMaxGroupParts = (1 << 23) - 1;
-// A group unit costs its SM a roughly fixed ~17 us for a 512-token partition
-// (four key tiles through the tensor-core tile kernel), while each member that
-// reads the partition itself costs ~5 us of SM time, so tiny groups do not pay.
-// Measured on B200 with 4-sibling groups (parallel sampling): 498 us per call
-// grouped against 515 us without.
+// Groups of fewer members do not pay for the group unit's fixed cost (its rows
+// pad a 128-row tensor-core tile).
 constexpr int kMinGroupMembers = 4;
 constexpr int kLcpBatch = 8;         // sequences a warp compares at once
 
@@ -1075,28 +1078,43 @@ __device__ __forceinline__ void shared_prefix_lengths(const Params &p, int *lcp)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int S = p.num_seqs;
     for (int base = warp * kLcpBatch; base < S; base += (kDetectThreads / 32) * kLcpBatch) {
-        int n[kLcpBatch], res[kLcpBatch];
+        int n[kLcpBatch], res[kLcpBatch], la[kLcpBatch], lb[kLcpBatch];
+        int va[kLcpBatch][2], vb[kLcpBatch][2];
+        // the first 64 entries of both tables are loaded together with the
+        // lengths (not behind them): one memory round trip for most pairs
 #pragma unroll
         for (int b = 0; b < kLcpBatch; ++b) {
             const int s = base + b;
-            n[b] = 0;
-            if (s > 0 && s < S) {
-                const int La = checked_len(p, s), Lb = checked_len(p, s - 1);
-                n[b] = min(max(La, 0), max(Lb, 0)) / kBlockSize;
+            const bool pair = s > 0 && s < S;
+            la[b] = pair ? __ldg(p.lens + s) : 0;
+            lb[b] = pair ? __ldg(p.lens + s - 1) : 0;
+            const int32_t *ta = p.tables + (int64_t)s * p.max_blocks;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int i = 32 * k + lane;
+                const bool act = pair && i < p.max_blocks;
+                va[b][k] = act ? __ldg(ta + i) : 0;
+                vb[b][k] = act ? __ldg(ta - p.max_blocks + i) : 0;
             }
+        }
+#pragma unroll
+        for (int b = 0; b < kLcpBatch; ++b) {
+            const int La = check_len(p, la[b]), Lb = check_len(p, lb[b]);
+            n[b] = (base + b > 0 && base + b < S) ? min(max(La, 0), max(Lb, 0)) / kBlockSize : 0;
             res[b] = n[b];  // == n: no difference found yet
         }
         for (int c0 = 0;; c0 += 64) {
-            int va[kLcpBatch][2], vb[kLcpBatch][2];
+            if (c0 > 0) {
 #pragma unroll
-            for (int b = 0; b < kLcpBatch; ++b) {
-                const int32_t *ta = p.tables + (int64_t)(base + b) * p.max_blocks;
+                for (int b = 0; b < kLcpBatch; ++b) {
+                    const int32_t *ta = p.tables + (int64_t)(base + b) * p.max_blocks;
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int i = c0 + 32 * k + lane;
-                    const bool act = res[b] == n[b] && i < n[b];  // implies 0 < s < S
-                    va[b][k] = act ? __ldg(ta + i) : 0;
-                    vb[b][k] = act ? __ldg(ta - p.max_blocks + i) : 0;
+                    for (int k = 0; k < 2; ++k) {
+                        const int i = c0 + 32 * k + lane;
+                        const bool act = res[b] == n[b] && i < n[b];  // implies 0 < s < S
+                        va[b][k] = act ? __ldg(ta + i) : 0;
+                        vb[b][k] = act ? __ldg(ta - p.max_blocks + i) : 0;
+                    }
                 }
             }
             bool more = false;
@@ -1140,14 +1158,38 @@ __device__ __forceinline__ int warp_exclusive_scan(int x, int identity) {
 // its predecessor; runs are cut into chunks of at most max_members sequences
 // counted from the run's start.  A chunk of n >= kMinGroupMembers sequences
 // shares min(lcp over its members after the first) blocks, i.e. np whole
-// partitions; it becomes one group with np x num_kv_heads units.  first_p[s] =
-// np of s's chunk (0 for a smaller chunk).
+// partitions; it becomes one group with num_kv_heads units.  first_p[s] = np of
+// s's chunk (0 for a smaller chunk).
+// The one-call step's cache write, done by blocks 1.. of the detection grid.
+struct StepWriteArgs {
+    const uint4 *key;
+    const uint4 *value;
+    const int64_t *slot_mapping;
+    int32_t num_tokens;
+    uint4 *key_cache;
+    uint4 *value_cache;
+    int32_t num_kv_heads;
+    int32_t chunks_per_row;
+    int64_t num_slots;
+    int64_t chunks;  // num_tokens * num_kv_heads * chunks_per_row (0: no write)
+};
+
 __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __grid_constant__ Params p,
                                                                       int32_t *first_p, int4 *groups,
-                                                                      int32_t *meta) {
+                                                                      int32_t *meta,
+                                                                      const __grid_constant__ StepWriteArgs w) {
     __shared__ int lcp[kMaxGroupSeqs];
-    __shared__ int info[kMaxGroupSeqs];  // at a chunk head: np << 8 | members (members <= 128); else -1
+    __shared__ int info[kMaxGroupSeqs];  // at a chunk head: its size, then np << 8 | size (size <= 128)
     grid_dep_launch();  // the group tiles set up while this runs, then wait for it
+    if (blockIdx.x > 0) {
+        // the step's new K/V (pa_append_decode): the tiles and the decode wait for
+        // this whole grid, so they see it; detection reads no cache bytes
+        for (int64_t i = (int64_t)(blockIdx.x - 1) * kDetectThreads + threadIdx.x; i < w.chunks;
+             i += (int64_t)(gridDim.x - 1) * kDetectThreads)
+            write_chunk(i, w.key, w.value, w.slot_mapping, w.num_tokens, w.key_cache, w.value_cache,
+                        w.num_kv_heads, w.chunks_per_row, w.num_slots, p.err);
+        return;
+    }
     const int S = p.num_seqs;
     shared_prefix_lengths(p, lcp);
     __syncthreads();
@@ -1155,52 +1197,79 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     // the cache, so it runs alongside the write, but it finishes only after it:
     // the group tiles wait for this kernel and so see the new tokens' K/V.
     grid_dep_wait();
-    if (threadIdx.x >= 32) return;
-    // warp 0: lane owns sequences [s0, s1)
-    const int lane = threadIdx.x;
+    // Every thread owns a contiguous run of at most 4 sequences [s0, s1).
+    __shared__ int wtot[kDetectThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int bpp = p.part_tokens / kBlockSize;
     const int M = p.max_members;  // 128 / g: a power of two
-    const int per = (S + 31) / 32, s0 = min(S, lane * per), s1 = min(S, s0 + per);
-    // run starts: max-scan of (run head ? s : -1)
+    const int per = (S + kDetectThreads - 1) / kDetectThreads;
+    const int s0 = min(S, (int)threadIdx.x * per), s1 = min(S, s0 + per);
+    // block-wide exclusive scan of one value per thread (sum, or max when kMax)
+    auto block_scan = [&](int x, int identity, bool is_max) -> int {
+        const int wex = is_max ? warp_exclusive_scan<true>(x, identity) : warp_exclusive_scan<false>(x, identity);
+        const int winc = is_max ? max(wex, x) : wex + x;
+        if (lane == 31) wtot[warp] = winc;
+        __syncthreads();
+        if (warp == 0) {
+            const int v = wtot[lane];
+            const int e = is_max ? warp_exclusive_scan<true>(v, identity) : warp_exclusive_scan<false>(v, identity);
+            __syncwarp();
+            wtot[lane] = e;
+        }
+        __syncthreads();
+        const int r = is_max ? max(wtot[warp], wex) : wtot[warp] + wex;
+        __syncthreads();  // wtot is reused by the next scan
+        return r;
+    };
+    // run starts (a sequence sharing less than one whole partition with its
+    // predecessor), then each sequence's run start rs by a max-scan
     int mx = -1;
     for (int s = s0; s < s1; ++s)
         if (s == 0 || lcp[s] < bpp) mx = s;
-    int rs = warp_exclusive_scan<true>(mx, -1);
+    int rs = block_scan(mx, -1, true);
+    int head_of[4];
     for (int s = s0; s < s1; ++s) {
         if (s == 0 || lcp[s] < bpp) rs = s;
-        info[s] = ((s - rs) & (M - 1)) == 0 ? 0 : -1;  // chunk heads marked 0 for now
+        head_of[s - s0] = rs + ((s - rs) & ~(M - 1));  // chunks of M counted from the run's start
     }
-    __syncwarp();
-    // each chunk head measures its chunk
-    int chunks = 0, units = 0;
+    // chunk heads collect their size and the smallest shared length of the
+    // members after them (a head's own lcp is no longer needed)
+    for (int s = s0; s < s1; ++s)
+        if (head_of[s - s0] == s) {
+            info[s] = 0;
+            lcp[s] = INT_MAX;
+        }
+    __syncthreads();
     for (int s = s0; s < s1; ++s) {
-        if (info[s] < 0) continue;
-        int e = s + 1, mn = INT_MAX;
-        while (e < S && info[e] < 0) mn = min(mn, lcp[e++]);
-        const int n = e - s;
+        const int hd = head_of[s - s0];
+        atomicAdd(&info[hd], 1);
+        if (hd != s) atomicMin(&lcp[hd], lcp[s]);
+    }
+    __syncthreads();
+    int heads = 0;  // this thread's groups
+    for (int s = s0; s < s1; ++s) {
+        if (head_of[s - s0] != s) continue;
+        const int n = info[s], mn = lcp[s];
         const int np = n >= kMinGroupMembers ? min(mn / bpp, kMaxGroupParts) : 0;
-        info[s] = (np << 8) | n;  // stays >= 0: other lanes only test the sign
-        if (np > 0) {
-            ++chunks;
-            units += np * p.num_kv_heads;
-        }
+        info[s] = (np << 8) | n;
+        if (np > 0) ++heads;
     }
-    __syncwarp();
-    int oc = warp_exclusive_scan<false>(chunks, 0);
-    int ou = warp_exclusive_scan<false>(units, 0);
+    const int g0 = block_scan(heads, 0, false);  // (the scan's barriers publish info)
+    for (int s = s0; s < s1; ++s) first_p[s] = info[head_of[s - s0]] >> 8;
+    int g = g0;
     for (int s = s0; s < s1; ++s) {
-        if (info[s] < 0) continue;
+        if (head_of[s - s0] != s) continue;
         const int n = info[s] & 255, np = info[s] >> 8;
-        for (int m = s; m < s + n; ++m) first_p[m] = np;
         if (np > 0) {
-            groups[oc++] = make_int4(s, n, np, ou);
-            ou += np * p.num_kv_heads;
+            groups[g] = make_int4(s, n, np, g * p.num_kv_heads);
+            ++g;
         }
     }
-    if (lane == 31) {  // its running counts end at the totals
-        meta[0] = oc;
-        meta[1] = ou;
+    if (threadIdx.x == kDetectThreads - 1) {  // its running count ends at the total
+        meta[0] = g;
+        meta[1] = g * p.num_kv_heads;
         meta[2] = 0;   // the per-sequence kernel's work counter
+        meta[3] = 0;   // the group tiles' work counter
     }
 }
 
@@ -1281,14 +1350,33 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             prm.groups = reinterpret_cast<int4 *>(g + sa);
             prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
             prm.max_members = 128 / G;
+            StepWriteArgs wa;
+            std::memset(&wa, 0, sizeof(wa));
+            unsigned write_blocks = 0;
+            if (a.write && a.write->num_tokens > 0) {
+                const StepWrite &sw = *a.write;
+                wa.key = static_cast<const uint4 *>(sw.key);
+                wa.value = static_cast<const uint4 *>(sw.value);
+                wa.slot_mapping = sw.slot_mapping;
+                wa.num_tokens = sw.num_tokens;
+                wa.key_cache = static_cast<uint4 *>(sw.key_cache);
+                wa.value_cache = static_cast<uint4 *>(sw.value_cache);
+                wa.num_kv_heads = a.cache.num_kv_heads;
+                wa.chunks_per_row = a.cache.head_dim * (int)sizeof(T) / 16;
+                wa.num_slots = (int64_t)a.cache.num_blocks * kBlockSize;
+                wa.chunks = (int64_t)sw.num_tokens * wa.num_kv_heads * wa.chunks_per_row;
+                write_blocks = (unsigned)std::min<int64_t>((wa.chunks + kDetectThreads - 1) / kDetectThreads,
+                                                           4 * sms);
+            }
             if (a.after_write) {
-                e = launch_after(group_detect_kernel, dim3(1), dim3(kDetectThreads), 0, stream,
+                e = launch_after(group_detect_kernel, dim3(1 + write_blocks), dim3(kDetectThreads), 0, stream,
                                  static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_p),
-                                 const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta));
+                                 const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta),
+                                 static_cast<const StepWriteArgs &>(wa));
             } else {
-                group_detect_kernel<<<1, kDetectThreads, 0, stream>>>(prm, const_cast<int32_t *>(prm.first_p),
-                                                                      const_cast<int4 *>(prm.groups),
-                                                                      const_cast<int32_t *>(prm.meta));
+                group_detect_kernel<<<1 + write_blocks, kDetectThreads, 0, stream>>>(
+                    prm, const_cast<int32_t *>(prm.first_p), const_cast<int4 *>(prm.groups),
+                    const_cast<int32_t *>(prm.meta), wa);
                 e = cudaGetLastError();
             }
             if (e != cudaSuccess) return e;
@@ -1344,6 +1432,24 @@ cudaError_t launch_g(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
 }
 
 }  // namespace
+
+cudaError_t launch_append_decode(const StepWrite &w, DecodeLaunch a, cudaStream_t stream) {
+    // the shared-prefix path (bf16, head_dim 128, split contexts) starts with the
+    // detection kernel, whose grid takes the write along
+    const bool grouped = a.cache.dtype == PA_BF16 && a.cache.head_dim == 128 && a.partition_size > 0 &&
+                         a.ws_group && a.num_seqs <= kMaxGroupSeqs;
+    if (w.num_tokens > 0) {
+        if (grouped) {
+            a.write = &w;
+        } else {
+            const cudaError_t e = launch_cache_write(w.key, w.value, w.slot_mapping, w.num_tokens, w.key_cache,
+                                                     w.value_cache, a.cache, a.err, stream);
+            if (e != cudaSuccess) return e;
+            a.after_write = true;  // the decode chain starts behind the write
+        }
+    }
+    return launch_decode(a, stream);
+}
 
 cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream) {
     Params prm;

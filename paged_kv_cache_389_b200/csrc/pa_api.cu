@@ -260,14 +260,13 @@ pa_status pa_append_decode(const void *key, const void *value, const int64_t *sl
                         workspace_bytes, out, cache, err_flag, a);
     if (st != PA_OK) return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (num_tokens > 0) {
-        st = from_cuda(launch_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache, *cache,
-                                          err_flag, s));
-        if (st != PA_OK) return st;
-        a.after_write = true;  // the decode chain starts behind the write
+    if (num_seqs == 0) {
+        if (num_tokens == 0) return PA_OK;
+        return from_cuda(launch_cache_write(key, value, slot_mapping, num_tokens, key_cache, value_cache,
+                                            *cache, err_flag, s));
     }
-    if (num_seqs == 0) return PA_OK;
-    return from_cuda(launch_decode(a, s));
+    const StepWrite w{key, value, slot_mapping, num_tokens, key_cache, value_cache};
+    return from_cuda(launch_append_decode(w, a, s));
 }
 
 pa_status pa_prefill_chunk(const void *query, const void *key_cache, const void *value_cache,

@@ -58,6 +58,17 @@ struct DecodeLaunch {
     pa_cache_desc cache;
     int32_t *err;
     bool after_write;  // launched behind a cache write on the same stream (pa_append_decode)
+    const struct StepWrite *write;  // the step's write, done inside the first decode kernel (or null)
+};
+
+// The new tokens' cache write of a one-call step (pa_append_decode).
+struct StepWrite {
+    const void *key;
+    const void *value;
+    const int64_t *slot_mapping;
+    int32_t num_tokens;
+    void *key_cache;
+    void *value_cache;
 };
 
 // Largest num_seqs a split decode supports (the per-CTA partition prefix sum
@@ -65,6 +76,11 @@ struct DecodeLaunch {
 constexpr int32_t kMaxSplitSeqs = 4096;
 
 cudaError_t launch_decode(const DecodeLaunch &a, cudaStream_t stream);
+
+// The one-call step: the write, then the decode chain.  When the decode takes the
+// shared-prefix path the write runs inside the detection kernel's grid (no
+// launch of its own); otherwise it is launch_cache_write followed by launch_decode.
+cudaError_t launch_append_decode(const StepWrite &w, DecodeLaunch a, cudaStream_t stream);
 
 struct PrefillLaunch {
     const void *query;
@@ -86,9 +102,9 @@ struct PrefillLaunch {
 cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
 
 // Shared-prefix group units of a split bf16 / head_dim 128 decode, on the tcgen05
-// tile kernel: rows = a group's members x g query heads, keys = one partition
-// inside the blocks they share; writes that partition's split-K partials.
-// groups / meta are the decode's detection output (device memory).
+// tile kernel: one unit per (group, kv head), rows = the group's members x g query
+// heads, keys = every partition the members share; it writes one partial (slot 0
+// of each member).  groups / meta are the decode's detection output (device memory).
 struct GroupTileLaunch {
     const void *query;       // [num_seqs, num_q_heads, 128] bf16
     int32_t num_seqs;

@@ -27,15 +27,18 @@
 // so O is rescaled rarely; the merge and the final division use the same point.
 // Warp roles: 0-3 softmax of stream 0, 4-7 softmax of stream 1 (warp w reads
 // tensor-memory lanes 32 (w % 4) .. + 31), 8 issues the MMAs from one thread and
-// owns the tensor memory, 9 loads (10 and 11 only complete the third warpgroup): Q and K/V tiles by TMA (128-byte swizzle, the
-// canonical layouts the MMA descriptors name) through a ring of 32 KB stages
-// holding K(0), V(0), K(1), V(1), ...; one TMA box per (16-token block, 64-column
-// half).  Every wait is bounded; an abort drains the copies and MMAs in flight
+// owns the tensor memory, 9 loads Q and K tiles, 10 loads V tiles (11 only
+// completes the third warpgroup): TMA with the 128-byte swizzle (the canonical
+// layouts the MMA descriptors name) into separate two-stage K and V rings of
+// 32 KB stages, one TMA box per (16-token block, 64-column half).  With rings and
+// warps of their own, K loads run ahead of the V stages that PVs still hold.
+// Every wait is bounded; an abort drains the copies and MMAs in flight
 // and still frees the tensor memory.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <climits>
 #include <cstring>
 #include <mutex>
 
@@ -50,9 +53,10 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kD = 128;              // head_dim (bf16 only)
 constexpr int kTileM = 128;          // query rows per stream tile
 constexpr int kTileN = 128;          // keys per K/V tile
-constexpr int kStages = 4;           // K/V ring stages
-constexpr int kThreads = 12 * 32;    // 8 softmax warps, 1 MMA warp, 1 load warp, 2 idle
-constexpr int kMmaWarp = 8, kLoadWarp = 9;
+constexpr int kKStages = 2;          // K tile ring
+constexpr int kVStages = 2;          // V tile ring
+constexpr int kThreads = 12 * 32;    // 8 softmax warps, 1 MMA warp, 2 load warps, 1 idle
+constexpr int kMmaWarp = 8, kLoadWarp = 9, kVLoadWarp = 10;
 // Registers per thread after the split (setmaxnreg, per warpgroup of 4 warps): the
 // launch gives 384 threads x 168; the softmax warpgroups take 200 (a row of S in
 // registers), the MMA / load warpgroup 96: 256 x 200 + 128 x 96 <= 384 x 168, and
@@ -69,11 +73,14 @@ constexpr uint32_t kTileBytes = 2 * kHalf;          // 32 KB
 constexpr uint32_t kBlockBytes = kBlockSize * 128;  // one block's rows in one half
 constexpr uint32_t kOffQ = 0;                       // Q buffers 0 and 1
 constexpr uint32_t kOffRing = 2 * kTileBytes;
-constexpr uint32_t kOffBar = kOffRing + kStages * kTileBytes;
+constexpr uint32_t kOffVRing = kOffRing + kKStages * kTileBytes;
+constexpr uint32_t kOffBar = kOffVRing + kVStages * kTileBytes;
 // barriers
-constexpr int kBarFull = 0;                     // [kStages] stage landed: TMA bytes + the loader's 2nd arrival
-constexpr int kBarEmpty = kBarFull + kStages;   // [kStages] stage consumed (MMA commit)
-constexpr int kBarQFull = kBarEmpty + kStages;  // [2] Q buffer landed
+constexpr int kBarKFull = 0;                      // [kKStages] K stage landed (TMA bytes)
+constexpr int kBarKEmpty = kBarKFull + kKStages;  // [kKStages] its QKs done (MMA commit)
+constexpr int kBarVFull = kBarKEmpty + kKStages;  // [kVStages] V stage landed: TMA bytes + the V loader's 2nd arrival
+constexpr int kBarVEmpty = kBarVFull + kVStages;  // [kVStages] its PVs done (MMA commit)
+constexpr int kBarQFull = kBarVEmpty + kVStages;  // [2] Q buffer landed
 constexpr int kBarQEmpty = kBarQFull + 2;       // [2] last QK reading a Q buffer done
 constexpr int kBarSFull = kBarQEmpty + 2;       // [2] S_t written
 constexpr int kBarPFull = kBarSFull + 2;        // [2] P_t written (the 128 softmax threads of stream t)
@@ -84,7 +91,14 @@ constexpr int kBarIdle = kBarMl + 1;            // every MMA issued has complete
 constexpr int kNumBars = kBarIdle + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
 constexpr uint32_t kOffMl = kOffMisc + 16;             // float2 (m, l) [2 streams][128 rows]
-constexpr size_t kSmemUsed = kOffMl + 2 * 128 * 8;
+constexpr uint32_t kOffJobs = kOffMl + 2 * 128 * 8;  // job ids [8] and tags [8] (group units)
+constexpr uint32_t kOffGroups = (kOffJobs + 64 + 15) / 16 * 16;  // int4 group records (group units)
+constexpr int kMaxGroups = 1024;                      // >= 4 members each, <= 4096 sequences
+constexpr size_t kSmemUsed = kOffGroups + kMaxGroups * 16;
+static_assert(kOffQ % 1024 == 0 && kOffRing % 1024 == 0 && kOffVRing % 1024 == 0 && kTileBytes % 1024 == 0,
+              "swizzled tiles: 1024-byte aligned");
+static_assert(kOffBar % 8 == 0 && kOffMisc % 4 == 0 && kOffMl % 8 == 0 && kOffJobs % 4 == 0 && kOffGroups % 16 == 0,
+              "shared-memory fields aligned to their types");
 constexpr size_t kSmemBytes = kSmemUsed + 1024;       // slack to align the base
 
 struct Params {
@@ -249,29 +263,28 @@ struct Job {
     int first, part;
 };
 
+// sgroups / ngroups: the group records, copied to shared memory (group units).
 template <int G, bool kGroup>
-__device__ __forceinline__ bool make_job(const Params &p, int u, Job &jb) {
+__device__ __forceinline__ bool make_job(const Params &p, int u, Job &jb, const int4 *sgroups, int ngroups) {
     if constexpr (kGroup) {
-        const int ngroups = __ldg(p.meta);
         int lo = 0, hi = ngroups;  // groups[lo].w <= u < groups[hi].w
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (__ldg(&p.groups[mid].w) <= u) lo = mid; else hi = mid;
+            if (sgroups[mid].w <= u) lo = mid; else hi = mid;
         }
-        const int4 gr = __ldg(&p.groups[lo]);  // (first seq, members, shared partitions, units before)
-        const int r = u - gr.w;
-        jb.h = r % p.num_kv_heads;
-        jb.part = r / p.num_kv_heads;  // partition = workspace slot
+        const int4 gr = sgroups[lo];  // (first seq, members, shared partitions, units before)
+        jb.h = u - gr.w;               // one unit per kv head
+        jb.part = 0;                   // workspace slot 0 holds the shared partitions' partial
         jb.first = gr.x;
         jb.two = false;
         jb.nrows[0] = gr.y * G;
         jb.nrows[1] = 0;
         jb.qz[0] = jb.qz[1] = gr.x;
-        jb.trow = p.tables + (int64_t)gr.x * p.max_blocks + (int64_t)jb.part * (p.part_tokens / kBlockSize);
-        jb.nkeys = p.part_tokens;
-        jb.lim0[0] = jb.lim0[1] = p.part_tokens - 1;
+        jb.trow = p.tables + (int64_t)gr.x * p.max_blocks;
+        jb.nkeys = gr.z * p.part_tokens;
+        jb.lim0[0] = jb.lim0[1] = jb.nkeys - 1;
         jb.lim_step = 0;
-        jb.ntiles = (p.part_tokens + kTileN - 1) / kTileN;
+        jb.ntiles = (jb.nkeys + kTileN - 1) / kTileN;
         jb.out_row0 = 0;
         return true;
     } else {
@@ -331,21 +344,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     float2 *mlx = reinterpret_cast<float2 *>(smem + kOffMl);  // [2][128]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    int njobs;
+    int njobs, ngroups = 0;
+    int4 *sgroups = reinterpret_cast<int4 *>(smem + kOffGroups);
+    // Group units are handed out dynamically: unit 0 of a CTA is blockIdx.x, the
+    // next ones gridDim.x + values drawn from a counter (zeroed by the detection
+    // kernel).  The loader draws them and publishes job k's id in slot k & 7;
+    // the MMA and softmax warps read it there.  Prefill jobs are static.
+    volatile int *job_id = reinterpret_cast<volatile int *>(smem + kOffJobs);
+    volatile int *job_tag = job_id + 8;
     if constexpr (kGroup) {
         // launched behind the detection kernel: its group list must be complete;
         // then the per-sequence decode may start (it reads only detection output)
         grid_dep_wait();
         grid_dep_launch();
         njobs = __ldg(p.meta + 1);
+        ngroups = min(__ldg(p.meta), kMaxGroups);
     } else {
         njobs = p.num_seqs * p.num_kv_heads * p.pairs;
     }
     if ((int)blockIdx.x >= njobs) return;
+    if constexpr (kGroup) {
+        for (int i = threadIdx.x; i < ngroups; i += kThreads) sgroups[i] = __ldg(&p.groups[i]);
+    }
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bars[kBarFull + i], 2);
-            mbar_init(&bars[kBarEmpty + i], 1);
+        for (int i = 0; i < 8; ++i) job_tag[i] = -1;
+        for (int i = 0; i < kKStages; ++i) {
+            mbar_init(&bars[kBarKFull + i], 1);
+            mbar_init(&bars[kBarKEmpty + i], 1);
+        }
+        for (int i = 0; i < kVStages; ++i) {
+            mbar_init(&bars[kBarVFull + i], 2);
+            mbar_init(&bars[kBarVEmpty + i], 1);
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&bars[kBarQFull + t], 1);
@@ -370,34 +399,83 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // id of this CTA's job k as read by the calling thread (INT_MAX: none / gave up)
+    auto job_of_thread = [&](int k) -> int {
+        if constexpr (!kGroup) {
+            return (int)blockIdx.x + k * (int)gridDim.x;
+        } else {
+            const unsigned long long t0 = global_ns();
+            while (job_tag[k & 7] != k) {
+                if (*abort_flag || global_ns() - t0 > p.wait_ns) {
+                    if (!*abort_flag) flag_error(p.err, PA_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                    return INT_MAX;
+                }
+            }
+            __threadfence_block();
+            return job_id[k & 7];
+        }
+    };
+    // the same for a whole warp: lane 0 reads, the others take its value
+    auto job_of_warp = [&](int k) -> int {
+        int v = 0;
+        if (lane == 0) v = job_of_thread(k);
+        return __shfl_sync(kFull, v, 0);
+    };
 
     // each warpgroup sets its register count at one instruction that dominates
     // all of its code
     if (warp >= 8) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
-    if (warp == kLoadWarp) {
-        // ------------------------------------------------------------ loader
-        // Lane 0 issues Q and arms the barriers; lanes 0..7 each own one 16-token
-        // block of a key tile: its table entry (loaded a tile ahead) and its two
-        // TMA boxes.  A stage completes on the TMA bytes plus a second arrival of
+    if (warp == kLoadWarp || warp == kVLoadWarp) {
+        // ------------------------------------------------------------ loaders
+        // Warp 9 loads Q and the K tiles and hands out the group units' ids; warp
+        // 10 loads the V tiles.  Lane 0 issues Q and arms the barriers; lanes 0..15
+        // each issue one of a key tile's 16 TMA boxes (block lane / 2, 64-column
+        // half lane % 2): a TMA instruction holds its issuing thread for a while,
+        // so the boxes of a tile go out from 16 threads at once.  A V stage completes on the TMA bytes plus a second arrival of
         // lane 0, made once the warp has filled by hand the block that holds the
-        // last keys of a job when they end inside it (V only: its rows past the
-        // keys become zeros -- 0 * (NaN or Inf) would poison the sums).
-        int it = 0;                 // K/V items issued: K(j), V(j) of each job in order
-        int qn[2] = {0, 0};         // loads issued per Q buffer
+        // last keys of a job when they end inside it (its rows past the keys become
+        // zeros: 0 * (NaN or Inf) would poison the sums).
+        const bool is_v = warp == kVLoadWarp;
+        const int nst = is_v ? kVStages : kKStages;
+        uint64_t *full = &bars[is_v ? kBarVFull : kBarKFull];
+        uint64_t *empty = &bars[is_v ? kBarVEmpty : kBarKEmpty];
+        const uint32_t ring = sbase + (is_v ? kOffVRing : kOffRing);
+        const CUtensorMap *map = is_v ? &p.vmap : &p.kmap;
+        int it = 0;                 // tiles issued into this warp's ring (jobs in order)
+        int qn[2] = {0, 0};         // loads issued per Q buffer (warp 9)
         bool ok = true;
         int njob = 0;
-        for (int u = blockIdx.x; ok && u < njobs; u += gridDim.x) {
-            Job jb;
-            if (!make_job<G, kGroup>(p, u, jb)) {
-                if constexpr (!kGroup) {
-                    if (lane == 0) flag_bad_chunk(p, u);
+        int u = blockIdx.x;
+        for (int k = 0; ok; ++k) {
+            int u_next = u + (int)gridDim.x;
+            if constexpr (kGroup) {
+                if (is_v) {
+                    u = job_of_warp(k);
+                } else if (lane == 0) {  // publish job k (an id >= njobs ends the list)
+                    job_id[k & 7] = u;
+                    __threadfence_block();
+                    job_tag[k & 7] = k;
                 }
+            }
+            if (u >= njobs) break;
+            // the next job's id (drawn now, read at the end of this one)
+            if constexpr (kGroup) {
+                if (!is_v && lane == 0) u_next = (int)gridDim.x + atomicAdd(const_cast<int32_t *>(p.meta) + 3, 1);
+            }
+            Job jb;
+            const bool have = make_job<G, kGroup>(p, u, jb, sgroups, ngroups);
+            if (!have) {
+                if constexpr (!kGroup) {
+                    if (lane == 0 && !is_v) flag_bad_chunk(p, u);
+                }
+                u = kGroup ? __shfl_sync(kFull, u_next, 0) : u_next;
                 continue;
             }
             // Q tiles: a buffer is rewritten once the QKs of its previous use are done
             const int nq = jb.two ? 2 : 1;
-            for (int t = 0; ok && t < nq; ++t) {
+            for (int t = 0; !is_v && ok && t < nq; ++t) {
                 const int b = q_buffer(jb, t, njob);
                 if (lane == 0) {
                     ok = qn[b] == 0 || wait_bar(&bars[kBarQEmpty + b], (qn[b] - 1) & 1, abort_flag, p);
@@ -413,66 +491,70 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             }
             const int nblk = (jb.nkeys + kBlockSize - 1) / kBlockSize;
             const int tail = jb.nkeys % kBlockSize;  // tokens in a partly filled last block (0: none)
-            auto entry = [&](int j) -> int {          // this lane's block of tile j: physical id, or -1
-                const int b = j * 8 + lane;
-                if (lane >= 8 || b >= nblk) return -1;
+            // table entries 32 at a time (four key tiles), one group ahead: lane i
+            // holds block 32 q + i of group q (-1: past the keys or invalid; flagged
+            // by the K loader)
+            auto entries = [&](int q) -> int {
+                const int b = q * 32 + lane;
+                if (b >= nblk) return -1;
                 const int e = __ldg(jb.trow + b);
                 if (e < 0 || e >= p.num_blocks) {
-                    flag_error(p.err, PA_DEVERR_BLOCK_ID);
+                    if (!is_v) flag_error(p.err, PA_DEVERR_BLOCK_ID);
                     return -1;
                 }
                 return e;
             };
-            int cur_e = entry(0);
+            int ent = entries(0);
+            int ent_next = jb.ntiles > 4 ? entries(1) : -1;
             for (int j = 0; ok && j < jb.ntiles; ++j) {
-                const int next_e = j + 1 < jb.ntiles ? entry(j + 1) : -1;
+                if (j > 0 && (j & 3) == 0) {
+                    ent = ent_next;
+                    ent_next = j + 4 < jb.ntiles ? entries((j >> 2) + 1) : -1;
+                }
+                // the block of tile j whose box this lane issues (lanes 0..15)
+                const int cur_e = __shfl_sync(kFull, ent, ((j & 3) << 3) | ((lane >> 1) & 7));
                 // invalid or past the keys: a coordinate outside the map reads zeros
                 const int z = cur_e >= 0 ? cur_e * p.num_kv_heads + jb.h : -1;
-                // block of this tile filled by hand (V only), or -1
-                const int hand = (tail != 0 && (jb.nkeys - 1) / kTileN == j) ? (jb.nkeys - 1) / kBlockSize - j * 8 : -1;
-                for (int kv = 0; kv < 2; ++kv) {
-                    const int st = it % kStages;
-                    const bool by_hand = kv == 1 && hand >= 0;
-                    if (lane == 0) {
-                        ok = it < kStages || wait_bar(&bars[kBarEmpty + st], ((it / kStages) - 1) & 1, abort_flag, p);
-                        if (ok) mbar_arrive_expect_tx(&bars[kBarFull + st], by_hand ? kTileBytes - 2 * kBlockBytes : kTileBytes);
-                    }
-                    ok = __shfl_sync(kFull, ok, 0);
-                    if (!ok) break;
-                    const CUtensorMap *map = kv ? &p.vmap : &p.kmap;
-                    const uint32_t dst = sbase + kOffRing + st * kTileBytes + lane * kBlockBytes;
-                    if (lane < 8 && !(by_hand && lane == hand)) {
-                        tma_load_3d(dst, map, 0, 0, z, &bars[kBarFull + st]);
-                        tma_load_3d(dst + kHalf, map, 64, 0, z, &bars[kBarFull + st]);
-                    }
-                    if (by_hand) {
-                        const int e = __shfl_sync(kFull, cur_e, hand);
-                        unsigned char *base = smem + kOffRing + st * kTileBytes + hand * kBlockBytes;
-                        const unsigned char *src =
-                            e >= 0 ? p.vc + ((int64_t)e * p.num_kv_heads + jb.h) * kBlockSize * (kD * 2) : nullptr;
-                        // 16 rows x 16 chunks of 16 bytes, stored as TMA would (128-byte swizzle)
-                        for (int idx = lane; idx < kBlockSize * 16; idx += 32) {
-                            const int rr = idx >> 4, c = idx & 15;
-                            uint4 v = make_uint4(0, 0, 0, 0);
-                            if (src && rr < tail) v = *reinterpret_cast<const uint4 *>(src + rr * (kD * 2) + c * 16);
-                            const int row = hand * kBlockSize + rr;  // row inside the 128-row tile
-                            *reinterpret_cast<uint4 *>(base - hand * kBlockBytes + (c >> 3) * kHalf + row * 128 +
-                                                       (((c & 7) ^ (row & 7)) << 4)) = v;
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                    }
-                    if (lane == 0) mbar_arrive(&bars[kBarFull + st]);
-                    ++it;
+                // block of this V tile filled by hand, or -1
+                const int hand = (is_v && tail != 0 && (jb.nkeys - 1) / kTileN == j)
+                                     ? (jb.nkeys - 1) / kBlockSize - j * 8 : -1;
+                const int st = it % nst;
+                if (lane == 0) {
+                    ok = it < nst || wait_bar(&empty[st], ((it / nst) - 1) & 1, abort_flag, p);
+                    if (ok) mbar_arrive_expect_tx(&full[st], hand >= 0 ? kTileBytes - 2 * kBlockBytes : kTileBytes);
                 }
-                cur_e = next_e;
+                ok = __shfl_sync(kFull, ok, 0);
+                if (!ok) break;
+                if (lane < 16 && (lane >> 1) != hand) {
+                    const int hf = lane & 1;
+                    tma_load_3d(ring + st * kTileBytes + hf * kHalf + (lane >> 1) * kBlockBytes, map, hf * 64, 0, z,
+                                &full[st]);
+                }
+                if (hand >= 0) {
+                    const int e = __shfl_sync(kFull, cur_e, 2 * hand);
+                    unsigned char *base = smem + (is_v ? kOffVRing : kOffRing) + st * kTileBytes;
+                    const unsigned char *src =
+                        e >= 0 ? p.vc + ((int64_t)e * p.num_kv_heads + jb.h) * kBlockSize * (kD * 2) : nullptr;
+                    // 16 rows x 16 chunks of 16 bytes, stored as TMA would (128-byte swizzle)
+                    for (int idx = lane; idx < kBlockSize * 16; idx += 32) {
+                        const int rr = idx >> 4, c = idx & 15;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (src && rr < tail) v = *reinterpret_cast<const uint4 *>(src + rr * (kD * 2) + c * 16);
+                        const int row = hand * kBlockSize + rr;  // row inside the 128-row tile
+                        *reinterpret_cast<uint4 *>(base + (c >> 3) * kHalf + row * 128 + (((c & 7) ^ (row & 7)) << 4)) = v;
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                if (is_v && lane == 0) mbar_arrive(&full[st]);
+                ++it;
             }
             ++njob;
+            u = kGroup ? (is_v ? u : __shfl_sync(kFull, u_next, 0)) : u_next;
         }
         // nothing may land after the CTA exits: wait for every stage still in flight
         if (lane == 0) {
-            for (int k = std::max(0, it - kStages); k < it; ++k)
-                mbar_wait_drain(&bars[kBarFull + k % kStages], (k / kStages) & 1);
+            for (int k = std::max(0, it - nst); k < it; ++k) mbar_wait_drain(&full[k % nst], (k / nst) & 1);
             for (int b = 0; b < 2; ++b)
                 if (qn[b] > 0) mbar_wait_drain(&bars[kBarQFull + b], (qn[b] - 1) & 1);
         }
@@ -481,14 +563,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdQK = idesc_bf16(false), kIdPV = idesc_bf16(true);
-            int it = 0;                  // K/V items consumed
+            int itk = 0, itv = 0;        // K and V tiles consumed
             int qn[2] = {0, 0};          // uses per Q buffer
             int npf[2] = {0, 0};         // P_t tiles consumed
             int njob = 0;
             bool ok = true;
-            for (int u = blockIdx.x; ok && u < njobs; u += gridDim.x) {
+            for (int k = 0; ok; ++k) {
+                const int u = job_of_thread(k);  // this MMA thread runs alone
+                if (u >= njobs) break;
                 Job jb;
-                if (!make_job<G, kGroup>(p, u, jb)) continue;
+                if (!make_job<G, kGroup>(p, u, jb, sgroups, ngroups)) continue;
                 const int nq = jb.two ? 2 : 1;
                 int qb[2];
                 for (int t = 0; t < 2; ++t) qb[t] = q_buffer(jb, t, njob);
@@ -500,8 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 int pend[2] = {-1, -1};     // key tile whose PV is still to be issued, per stream
                 bool first_pv[2] = {true, true};
                 bool o_ready = njob == 0;   // the previous job's O has been read
-                const int it0 = it;
-                // PV_t of key tile jp (V item it0 + 2 jp + 1)
+                const int itk0 = itk, itv0 = itv;
+                // PV_t of key tile jp
                 auto issue_pv = [&](int t, int jp) -> bool {
                     if (!o_ready) {
                         if (!wait_bar(&bars[kBarOFree], (njob - 1) & 1, abort_flag, p)) return false;
@@ -509,10 +593,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     }
                     if (!wait_bar(&bars[kBarPFull + t], npf[t] & 1, abort_flag, p)) return false;
                     ++npf[t];
-                    const int iv = it0 + 2 * jp + 1, st = iv % kStages;
-                    if (!wait_bar(&bars[kBarFull + st], (iv / kStages) & 1, abort_flag, p)) return false;
+                    const int iv = itv0 + jp, st = iv % kVStages;
+                    if (!wait_bar(&bars[kBarVFull + st], (iv / kVStages) & 1, abort_flag, p)) return false;
                     tc_fence_after();
-                    const uint32_t va = sbase + kOffRing + st * kTileBytes;
+                    const uint32_t va = sbase + kOffVRing + st * kTileBytes;
                     const uint32_t tP = tmem + t * 128, tO = tmem + 256 + t * 128;
 #pragma unroll
                     for (int kk = 0; kk < kTileN / 16; ++kk)
@@ -520,11 +604,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                                   !first_pv[t] || kk > 0);
                     first_pv[t] = false;
                     // V(jp) is free once its last consumer's PV is done
-                    if (!jb.two || t == 1) tc_commit(&bars[kBarEmpty + st]);
+                    if (!jb.two || t == 1) tc_commit(&bars[kBarVEmpty + st]);
                     return true;
                 };
                 for (int j = 0; ok && j < jb.ntiles; ++j) {
-                    const int ik = it0 + 2 * j, sk = ik % kStages;
+                    const int ik = itk0 + j, sk = ik % kKStages;
                     const unsigned cons = consumers(jb, j);
                     bool k_ready = false;
                     for (int t = 0; t < 2; ++t) {
@@ -534,7 +618,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                             break;
                         }
                         if (!k_ready) {
-                            if (!wait_bar(&bars[kBarFull + sk], (ik / kStages) & 1, abort_flag, p)) {
+                            if (!wait_bar(&bars[kBarKFull + sk], (ik / kKStages) & 1, abort_flag, p)) {
                                 ok = false;
                                 break;
                             }
@@ -554,7 +638,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                         pend[t] = j;
                     }
                     if (!ok) break;
-                    tc_commit(&bars[kBarEmpty + sk]);  // K(j) is free once its QKs are done
+                    tc_commit(&bars[kBarKEmpty + sk]);  // K(j) is free once its QKs are done
                     if (j == jb.ntiles - 1) {          // the job's last QKs: its Q buffers are free
                         tc_commit(&bars[kBarQEmpty + qb[0]]);
                         if (jb.two) tc_commit(&bars[kBarQEmpty + qb[1]]);
@@ -568,7 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                     }
                     tc_commit(&bars[kBarOFull + t]);
                 }
-                it = it0 + 2 * jb.ntiles;
+                itk = itk0 + jb.ntiles;
+                itv = itv0 + jb.ntiles;
                 ++njob;
             }
             // everything issued has completed once this arrives
@@ -593,9 +678,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
         int no[2] = {0, 0};     // O_t completions, both streams
         int njob = 0;
         bool live = true;
-        for (int u = blockIdx.x; live && u < njobs; u += gridDim.x) {
+        for (int k = 0; live; ++k) {
+            const int u = job_of_warp(k);
+            if (u >= njobs) break;
             Job jb;
-            if (!make_job<G, kGroup>(p, u, jb)) continue;
+            if (!make_job<G, kGroup>(p, u, jb, sgroups, ngroups)) continue;
             const int tile = jb.two ? t : 0;  // query tile whose rows this thread's lane holds
             const bool row_ok = r < jb.nrows[tile];
             const bool warp_rows = __any_sync(kFull, row_ok);

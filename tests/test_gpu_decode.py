@@ -398,3 +398,73 @@ def ts_free_decode(pa, torch, q_np, gpu, t, l, scale, part):
     pa.pa_decode(q, gpu.key_cache, gpu.value_cache, torch.from_numpy(t).cuda(), torch.from_numpy(l).cuda(),
                  maxc, scale, out, part, ws, gpu.err_flag)
     return to_host(out)
+
+
+def _expected_groups(tables, lens, part, g, hkv, min_members=4):
+    """The shared-prefix grouping rule, written out on the host: lcp[s] = leading
+    full blocks of s's table equal to those of s - 1; a run is a stretch of
+    sequences each sharing >= one whole partition with its predecessor; runs are
+    cut into chunks of 128 / g counted from the run's start; a chunk of >= 4
+    sequences shares min(lcp over its members after the first) // blocks per
+    partition whole partitions (np) and is a group when np > 0."""
+    S = len(lens)
+    bpp = part // 16
+    M = 128 // g
+    lcp = [0] * S
+    for s in range(1, S):
+        n = min(int(lens[s]), int(lens[s - 1])) // 16
+        k = 0
+        while k < n and tables[s, k] == tables[s - 1, k]:
+            k += 1
+        lcp[s] = k
+    first_p, groups = [0] * S, []
+    rs = 0
+    heads = {}
+    for s in range(S):
+        if s == 0 or lcp[s] < bpp:
+            rs = s
+        heads.setdefault(rs + ((s - rs) // M) * M, []).append(s)
+    for hd in sorted(heads):
+        members = heads[hd]
+        n = len(members)
+        np_ = min(lcp[m] for m in members[1:]) // bpp if n >= min_members else 0
+        for m in members:
+            first_p[m] = np_
+        if np_ > 0:
+            groups.append((hd, n, np_, len(groups) * hkv))
+    return first_p, groups
+
+
+@pytest.mark.parametrize("cid,part", [(3, 512), (4, 512), (3, 64)])
+def test_group_detection_matches_the_rule(cid, part):
+    """The detection kernel's output in the workspace (first shared partitions per
+    sequence, the group list, the counts) equals the grouping rule computed on the
+    host from the same tables."""
+    torch = torch_mod()
+    wl = workloads.make(cid, mini=(part == 64))
+    ts = TwoSided(wl)
+    step = wl.steps[0]
+    ts.append_step(step)
+    t, l = ts.tables(step.seqs)
+    S = len(step.seqs)
+    maxc = int(l.max())
+    n = ts.pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, maxc, part)
+    ws = torch.zeros(n, dtype=torch.uint8, device="cuda")
+    out = torch.empty((S, wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    ts.pa.pa_decode(to_dev(step.q), ts.gpu.key_cache, ts.gpu.value_cache, torch.from_numpy(t).cuda(),
+                    torch.from_numpy(l).cuda(), maxc, wl.scale, out, part, ws, ts.gpu.err_flag)
+    assert ts.err_flag() == 0
+    parts = -(-maxc // part)
+    rows = S * wl.num_q_heads * parts
+    at = -(-(rows * wl.head_dim * 4 + rows * 8) // 16) * 16
+    raw = ws.cpu().numpy()
+    first_p = raw[at:at + 4 * S].view(np.int32)
+    gat = at + -(-4 * S // 16) * 16
+    meta = raw[gat + 16 * S:gat + 16 * S + 16].view(np.int32)
+    want_fp, want_groups = _expected_groups(t, l, part, wl.num_q_heads // wl.num_kv_heads, wl.num_kv_heads)
+    assert first_p.tolist() == want_fp
+    assert meta[0] == len(want_groups) and meta[1] == len(want_groups) * wl.num_kv_heads
+    got_groups = raw[gat:gat + 16 * len(want_groups)].view(np.int32).reshape(-1, 4)
+    assert [tuple(int(x) for x in r) for r in got_groups] == want_groups
+    if cid == 3:
+        assert len(want_groups) > 0
