@@ -151,13 +151,14 @@ struct Params {
     // number of leading partitions of s computed by group_decode_kernel
     const int32_t *first_p;
     const int4 *groups;     // (first seq, members, shared partitions, units before)
-    const int32_t *meta;    // [0] groups, [1] group units
+    const int32_t *meta;    // [0] groups, [1] group units, [2] / [3] work counters, [4] tile CTAs
     int32_t max_members;    // sequences per group: query rows members x g <= 128
     int32_t wait_first;     // launched right behind a cache write: wait for it first
     float v_scale;          // fp8 pools: value dequantisation scale (1 otherwise)
     unsigned long long wait_ns;  // bound of every in-kernel wait
     int32_t *work_ctr;      // units handed out beyond the first gridDim.x (zeroed by the
                             // detection kernel of this call), or nullptr: static order
+    int32_t num_sms;        // SMs of the device (the detection kernel splits them)
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -1255,7 +1256,30 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         if (np > 0) ++heads;
     }
     const int g0 = block_scan(heads, 0, false);  // (the scan's barriers publish info)
-    for (int s = s0; s < s1; ++s) first_p[s] = info[head_of[s - s0]] >> 8;
+    // work estimate in (token, kv head) units: the group units' keys (measured on
+    // B200 to cost about 1.5 times a per-sequence key, their rows padding a
+    // 128-row tensor-core tile) against the per-sequence kernel's keys
+    __shared__ unsigned long long work[2];
+    if (threadIdx.x == 0) work[0] = work[1] = 0ull;
+    __syncthreads();
+    unsigned long long tw = 0, dw = 0;
+    for (int s = s0; s < s1; ++s) {
+        const int np = info[head_of[s - s0]] >> 8;
+        first_p[s] = np;
+        const int L = max(checked_len(p, s), 0);
+        dw += (unsigned long long)max(0, L - np * p.part_tokens);
+        if (head_of[s - s0] == s) tw += (unsigned long long)np * p.part_tokens;
+    }
+    // one shared-memory atomic per warp (1,024 on one word would serialise)
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        tw += __shfl_xor_sync(kFull, tw, o);
+        dw += __shfl_xor_sync(kFull, dw, o);
+    }
+    if (lane == 0) {
+        atomicAdd(&work[0], tw);
+        atomicAdd(&work[1], dw);
+    }
     int g = g0;
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
@@ -1265,11 +1289,22 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
             ++g;
         }
     }
+    __syncthreads();
     if (threadIdx.x == kDetectThreads - 1) {  // its running count ends at the total
         meta[0] = g;
         meta[1] = g * p.num_kv_heads;
         meta[2] = 0;   // the per-sequence kernel's work counter
         meta[3] = 0;   // the group tiles' work counter
+        // SMs for the group tiles, in proportion to their share of the work (the
+        // per-sequence kernel takes the rest), so that the two kernels end
+        // together; at least one per 2 group units (up to half the SMs), since a
+        // short unit's time is mostly latency
+        const double t = 1.5 * (double)work[0], d = (double)work[1];
+        const int sms = max(1, p.num_sms);
+        const int units = g * p.num_kv_heads;
+        int want = (int)ceil(sms * t / (t + d + 1.0));
+        want = max(want, min(sms / 2, (units + 1) / 2));
+        meta[4] = g == 0 ? 0 : min(sms, max(1, want));
     }
 }
 
@@ -1329,6 +1364,7 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
                              (int)Lay::smem_bytes(kMaxSplitSeqs + 1));
     if (e != cudaSuccess) return e;
     const int sms = num_sms(dev);
+    prm.num_sms = sms;
     // Per-sequence units after the group-covered partitions span several
     // partitions, so that the per-unit merge is amortised: 1024 tokens, or 2048
     // when there are few (sequence, kv head) pairs to spread over the SMs
@@ -1398,6 +1434,9 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             gl.max_partitions = a.max_partitions;
             gl.scale = a.scale;
             gl.err = a.err;
+            // The detection kernel picks how many SMs take the group units (ids drawn
+            // from a counter); the tile CTAs beyond that exit at once, and the
+            // per-sequence kernel starts on those SMs instead of waiting for them.
             if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
             grouped = true;
             prm.work_ctr = const_cast<int32_t *>(prm.meta) + 2;

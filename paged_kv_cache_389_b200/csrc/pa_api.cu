@@ -157,9 +157,9 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
     const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
     // partials (fp32 acc, then (m, l)), then the shared-prefix group bookkeeping:
     // first partition per sequence (16-byte padded), group list (16 bytes each),
-    // 16 bytes of counters
+    // 32 bytes of counts and counters
     const int64_t partials = rows * head_dim * 4 + rows * 8;
-    const int64_t group = ((int64_t)num_seqs * 4 + 15) / 16 * 16 + (int64_t)num_seqs * 16 + 16;
+    const int64_t group = ((int64_t)num_seqs * 4 + 15) / 16 * 16 + (int64_t)num_seqs * 16 + 32;
     return (size_t)((partials + 15) / 16 * 16 + group);
 }
 

@@ -91,8 +91,8 @@ constexpr int kBarIdle = kBarMl + 1;            // every MMA issued has complete
 constexpr int kNumBars = kBarIdle + 1;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem slot, abort flag
 constexpr uint32_t kOffMl = kOffMisc + 16;             // float2 (m, l) [2 streams][128 rows]
-constexpr uint32_t kOffJobs = kOffMl + 2 * 128 * 8;  // job ids [8] and tags [8] (group units)
-constexpr uint32_t kOffGroups = (kOffJobs + 64 + 15) / 16 * 16;  // int4 group records (group units)
+constexpr uint32_t kOffJobs = kOffMl + 2 * 128 * 8;  // job records [8] (int4) and tags [8] (group units)
+constexpr uint32_t kOffGroups = (kOffJobs + 8 * 16 + 8 * 4 + 15) / 16 * 16;  // int4 group records
 constexpr int kMaxGroups = 1024;                      // >= 4 members each, <= 4096 sequences
 constexpr size_t kSmemUsed = kOffGroups + kMaxGroups * 16;
 static_assert(kOffQ % 1024 == 0 && kOffRing % 1024 == 0 && kOffVRing % 1024 == 0 && kTileBytes % 1024 == 0,
@@ -121,7 +121,7 @@ struct Params {
     float scale_log2;
     // shared-prefix group units of the split decode
     const int4 *groups;    // (first seq, members, shared partitions, units before)
-    const int32_t *meta;   // [0] groups, [1] units
+    const int32_t *meta;   // [0] groups, [1] units, [3] work counter, [4] CTAs that take units
     float *ws_acc;
     float2 *ws_ml;
     int32_t part_tokens;
@@ -181,16 +181,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-          "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-          "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float *v) {
     uint32_t r[16];
     asm volatile(
@@ -240,6 +230,13 @@ constexpr uint32_t idesc_bf16(bool b_mn_major) {
            ((uint32_t)(kTileM >> 4) << 24);
 }
 
+// max of three (the sm_100 three-input max)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *abort, const Params &p) {
     return mbar_wait_bounded(bar, parity, abort, p.err, p.wait_ns);
 }
@@ -263,17 +260,25 @@ struct Job {
     int first, part;
 };
 
-// sgroups / ngroups: the group records, copied to shared memory (group units).
+// Group unit u's record (first seq, members, shared partitions, kv head), from
+// the group list copied to shared memory.
+__device__ __forceinline__ int4 group_record(int u, const int4 *sgroups, int ngroups) {
+    int lo = 0, hi = ngroups;  // groups[lo].w <= u < groups[hi].w
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (sgroups[mid].w <= u) lo = mid; else hi = mid;
+    }
+    const int4 gr = sgroups[lo];  // (first seq, members, shared partitions, units before)
+    return make_int4(gr.x, gr.y, gr.z, u - gr.w);
+}
+
+// The job: a group unit from its record (u unused), a prefill job from its index u
+// (rec unused).  False: a prefill job with no rows, or an invalid chunk.
 template <int G, bool kGroup>
-__device__ __forceinline__ bool make_job(const Params &p, int u, Job &jb, const int4 *sgroups, int ngroups) {
+__device__ __forceinline__ bool make_job(const Params &p, int u, int4 rec, Job &jb) {
     if constexpr (kGroup) {
-        int lo = 0, hi = ngroups;  // groups[lo].w <= u < groups[hi].w
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (sgroups[mid].w <= u) lo = mid; else hi = mid;
-        }
-        const int4 gr = sgroups[lo];  // (first seq, members, shared partitions, units before)
-        jb.h = u - gr.w;               // one unit per kv head
+        const int4 gr = rec;
+        jb.h = gr.w;                   // one unit per kv head
         jb.part = 0;                   // workspace slot 0 holds the shared partitions' partial
         jb.first = gr.x;
         jb.two = false;
@@ -344,27 +349,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     float2 *mlx = reinterpret_cast<float2 *>(smem + kOffMl);  // [2][128]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    int njobs, ngroups = 0;
     int4 *sgroups = reinterpret_cast<int4 *>(smem + kOffGroups);
     // Group units are handed out dynamically: unit 0 of a CTA is blockIdx.x, the
     // next ones gridDim.x + values drawn from a counter (zeroed by the detection
-    // kernel).  The loader draws them and publishes job k's id in slot k & 7;
-    // the MMA and softmax warps read it there.  Prefill jobs are static.
-    volatile int *job_id = reinterpret_cast<volatile int *>(smem + kOffJobs);
-    volatile int *job_tag = job_id + 8;
-    if constexpr (kGroup) {
-        // launched behind the detection kernel: its group list must be complete;
-        // then the per-sequence decode may start (it reads only detection output)
-        grid_dep_wait();
-        grid_dep_launch();
-        njobs = __ldg(p.meta + 1);
-        ngroups = min(__ldg(p.meta), kMaxGroups);
-    } else {
+    // kernel).  The K loader (warp 9), the only warp that waits for the detection
+    // kernel, draws them and publishes job k's record (first seq, members, shared
+    // partitions, kv head; members 0 = no more jobs) in slot k & 7; the other
+    // warps read it there.  So the set-up below (barriers, tensor memory,
+    // register split) overlaps the detection kernel.  Prefill jobs are static.
+    volatile int *job_rec = reinterpret_cast<volatile int *>(smem + kOffJobs);  // [8][4]
+    volatile int *job_tag = job_rec + 32;
+    int njobs = 0;
+    if constexpr (!kGroup) {
         njobs = p.num_seqs * p.num_kv_heads * p.pairs;
-    }
-    if ((int)blockIdx.x >= njobs) return;
-    if constexpr (kGroup) {
-        for (int i = threadIdx.x; i < ngroups; i += kThreads) sgroups[i] = __ldg(&p.groups[i]);
+        if ((int)blockIdx.x >= njobs) return;
     }
     if (threadIdx.x == 0) {
         for (int i = 0; i < 8; ++i) job_tag[i] = -1;
@@ -399,28 +397,60 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // id of this CTA's job k as read by the calling thread (INT_MAX: none / gave up)
-    auto job_of_thread = [&](int k) -> int {
+    // This CTA's job k as seen by the calling thread: 1 = jb filled, 0 = a prefill
+    // job with nothing to do, -1 = no more jobs (or the wait gave up).
+    auto job_of_thread = [&](int k, Job &jb) -> int {
         if constexpr (!kGroup) {
-            return (int)blockIdx.x + k * (int)gridDim.x;
+            const int u = (int)blockIdx.x + k * (int)gridDim.x;
+            if (u >= njobs) return -1;
+            return make_job<G, false>(p, u, make_int4(0, 0, 0, 0), jb) ? 1 : 0;
         } else {
             const unsigned long long t0 = global_ns();
             while (job_tag[k & 7] != k) {
                 if (*abort_flag || global_ns() - t0 > p.wait_ns) {
                     if (!*abort_flag) flag_error(p.err, PA_DEVERR_TIMEOUT);
                     *abort_flag = 1;
-                    return INT_MAX;
+                    return -1;
                 }
             }
             __threadfence_block();
-            return job_id[k & 7];
+            const int4 rec = make_int4(job_rec[(k & 7) * 4], job_rec[(k & 7) * 4 + 1], job_rec[(k & 7) * 4 + 2],
+                                       job_rec[(k & 7) * 4 + 3]);
+            if (rec.y <= 0) return -1;
+            make_job<G, true>(p, 0, rec, jb);
+            return 1;
         }
     };
-    // the same for a whole warp: lane 0 reads, the others take its value
-    auto job_of_warp = [&](int k) -> int {
-        int v = 0;
-        if (lane == 0) v = job_of_thread(k);
-        return __shfl_sync(kFull, v, 0);
+    // the same for a whole warp: lane 0 reads the record, the others take it
+    auto job_of_warp = [&](int k, Job &jb) -> int {
+        if constexpr (!kGroup) {
+            return job_of_thread(k, jb);
+        } else {
+            int4 rec = make_int4(0, -1, 0, 0);
+            if (lane == 0) {
+                const unsigned long long t0 = global_ns();
+                bool okw = true;
+                while (job_tag[k & 7] != k) {
+                    if (*abort_flag || global_ns() - t0 > p.wait_ns) {
+                        if (!*abort_flag) flag_error(p.err, PA_DEVERR_TIMEOUT);
+                        *abort_flag = 1;
+                        okw = false;
+                        break;
+                    }
+                }
+                __threadfence_block();
+                if (okw)
+                    rec = make_int4(job_rec[(k & 7) * 4], job_rec[(k & 7) * 4 + 1], job_rec[(k & 7) * 4 + 2],
+                                    job_rec[(k & 7) * 4 + 3]);
+            }
+            rec.x = __shfl_sync(kFull, rec.x, 0);
+            rec.y = __shfl_sync(kFull, rec.y, 0);
+            rec.z = __shfl_sync(kFull, rec.z, 0);
+            rec.w = __shfl_sync(kFull, rec.w, 0);
+            if (rec.y <= 0) return -1;
+            make_job<G, true>(p, 0, rec, jb);
+            return 1;
+        }
     };
 
     // each warpgroup sets its register count at one instruction that dominates
@@ -447,31 +477,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
         int qn[2] = {0, 0};         // loads issued per Q buffer (warp 9)
         bool ok = true;
         int njob = 0;
+        int ngroups = 0, active = (int)gridDim.x;
+        if constexpr (kGroup) {
+            if (!is_v) {
+                // launched behind the detection kernel: its group list must be
+                // complete; then the per-sequence decode may start (it reads only
+                // detection output)
+                grid_dep_wait();
+                grid_dep_launch();
+                njobs = __ldg(p.meta + 1);
+                ngroups = min(__ldg(p.meta), kMaxGroups);
+                active = min((int)gridDim.x, __ldg(p.meta + 4));
+                for (int i = lane; i < ngroups; i += 32) sgroups[i] = __ldg(&p.groups[i]);
+                __syncwarp();
+            }
+        }
         int u = blockIdx.x;
         for (int k = 0; ok; ++k) {
-            int u_next = u + (int)gridDim.x;
-            if constexpr (kGroup) {
-                if (is_v) {
-                    u = job_of_warp(k);
-                } else if (lane == 0) {  // publish job k (an id >= njobs ends the list)
-                    job_id[k & 7] = u;
-                    __threadfence_block();
-                    job_tag[k & 7] = k;
-                }
-            }
-            if (u >= njobs) break;
-            // the next job's id (drawn now, read at the end of this one)
-            if constexpr (kGroup) {
-                if (!is_v && lane == 0) u_next = (int)gridDim.x + atomicAdd(const_cast<int32_t *>(p.meta) + 3, 1);
-            }
+            int u_next = 0;
             Job jb;
-            const bool have = make_job<G, kGroup>(p, u, jb, sgroups, ngroups);
-            if (!have) {
-                if constexpr (!kGroup) {
-                    if (lane == 0 && !is_v) flag_bad_chunk(p, u);
+            if constexpr (kGroup) {
+                if (!is_v) {
+                    // publish job k (members 0: no more jobs); CTAs past the number
+                    // the detection kernel chose take none and leave their SM
+                    if (k == 0 && (int)blockIdx.x >= active) u = njobs;
+                    const int4 rec = u < njobs ? group_record(u, sgroups, ngroups) : make_int4(0, 0, 0, 0);
+                    if (lane == 0) {
+                        job_rec[(k & 7) * 4] = rec.x;
+                        job_rec[(k & 7) * 4 + 1] = rec.y;
+                        job_rec[(k & 7) * 4 + 2] = rec.z;
+                        job_rec[(k & 7) * 4 + 3] = rec.w;
+                        __threadfence_block();
+                        job_tag[k & 7] = k;
+                    }
+                    if (u >= njobs) break;
+                    // the next job's id (drawn now, read at the end of this one)
+                    if (lane == 0) u_next = active + atomicAdd(const_cast<int32_t *>(p.meta) + 3, 1);
+                    make_job<G, true>(p, 0, rec, jb);
+                } else if (job_of_warp(k, jb) < 0) {
+                    break;
                 }
-                u = kGroup ? __shfl_sync(kFull, u_next, 0) : u_next;
-                continue;
+            } else {
+                const int have = job_of_warp(k, jb);
+                if (have < 0) break;
+                if (have == 0) {
+                    if (lane == 0 && !is_v) flag_bad_chunk(p, (int)blockIdx.x + k * (int)gridDim.x);
+                    continue;
+                }
             }
             // Q tiles: a buffer is rewritten once the QKs of its previous use are done
             const int nq = jb.two ? 2 : 1;
@@ -550,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                 ++it;
             }
             ++njob;
-            u = kGroup ? (is_v ? u : __shfl_sync(kFull, u_next, 0)) : u_next;
+            if constexpr (kGroup) u = __shfl_sync(kFull, u_next, 0);
         }
         // nothing may land after the CTA exits: wait for every stage still in flight
         if (lane == 0) {
@@ -569,10 +621,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
             int njob = 0;
             bool ok = true;
             for (int k = 0; ok; ++k) {
-                const int u = job_of_thread(k);  // this MMA thread runs alone
-                if (u >= njobs) break;
                 Job jb;
-                if (!make_job<G, kGroup>(p, u, jb, sgroups, ngroups)) continue;
+                const int have = job_of_thread(k, jb);  // this MMA thread runs alone
+                if (have < 0) break;
+                if (have == 0) continue;
                 const int nq = jb.two ? 2 : 1;
                 int qb[2];
                 for (int t = 0; t < 2; ++t) qb[t] = q_buffer(jb, t, njob);
@@ -679,15 +731,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
         int njob = 0;
         bool live = true;
         for (int k = 0; live; ++k) {
-            const int u = job_of_warp(k);
-            if (u >= njobs) break;
             Job jb;
-            if (!make_job<G, kGroup>(p, u, jb, sgroups, ngroups)) continue;
+            const int have = job_of_warp(k, jb);
+            if (have < 0) break;
+            if (have == 0) continue;
             const int tile = jb.two ? t : 0;  // query tile whose rows this thread's lane holds
             const bool row_ok = r < jb.nrows[tile];
             const bool warp_rows = __any_sync(kFull, row_ok);
-            // last key this row may see (-1: a padding row sees nothing)
-            const int lim = row_ok ? jb.lim0[tile] + jb.lim_step * (r / G) : -1;
+            // last key this row may see; a padding row (never written out) is left
+            // unmasked, so that it does not force the masked path on its warp
+            const int lim = row_ok ? jb.lim0[tile] + jb.lim_step * (r / G) : INT_MAX;
             float m = -INFINITY, l = 0.f;
             bool first = true;
             if (stream_used(jb, t)) {
@@ -712,8 +765,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                             float a = -INFINITY;
                             if (open) {
 #pragma unroll
-                                for (int k = 0; k < kTileN; ++k) a = fmaxf(a, sv[k]);
-                            } else {
+                                for (int k = 0; k < kTileN; k += 2) a = fmax3(a, sv[k], sv[k + 1]);
+                            } else {  // a causal edge or the keys' end
 #pragma unroll
                                 for (int k = 0; k < kTileN; ++k) a = key0 + k <= lim ? fmaxf(a, sv[k]) : a;
                             }
@@ -730,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tile_kernel(const __grid_con
                         bool resc = false;
                         if (first) {
                             m = m_new;
-                        } else if (m_new > m + kRescaleLog2) {
+                        } else if (row_ok && m_new > m + kRescaleLog2) {
                             alpha = fast_exp2(m - m_new);  // m = -inf: O holds zeros, alpha 0
                             m = m_new;
                             resc = true;

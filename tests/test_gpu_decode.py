@@ -460,11 +460,16 @@ def test_group_detection_matches_the_rule(cid, part):
     raw = ws.cpu().numpy()
     first_p = raw[at:at + 4 * S].view(np.int32)
     gat = at + -(-4 * S // 16) * 16
-    meta = raw[gat + 16 * S:gat + 16 * S + 16].view(np.int32)
+    meta = raw[gat + 16 * S:gat + 16 * S + 32].view(np.int32)
     want_fp, want_groups = _expected_groups(t, l, part, wl.num_q_heads // wl.num_kv_heads, wl.num_kv_heads)
     assert first_p.tolist() == want_fp
     assert meta[0] == len(want_groups) and meta[1] == len(want_groups) * wl.num_kv_heads
     got_groups = raw[gat:gat + 16 * len(want_groups)].view(np.int32).reshape(-1, 4)
     assert [tuple(int(x) for x in r) for r in got_groups] == want_groups
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    if want_groups:   # SMs the detection kernel gave the group tiles
+        assert 1 <= meta[4] <= sms
+    else:
+        assert meta[4] == 0
     if cid == 3:
         assert len(want_groups) > 0
