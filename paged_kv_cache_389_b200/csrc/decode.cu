@@ -11,11 +11,15 @@
 // Design (B200, HBM bound):
 //  * Work unit = (sequence, kv head, partition of the context).  One CTA serves
 //    all g = Hq/Hkv query heads of its kv head, so every K/V byte is read once
-//    per unit.  The grid is persistent (one CTA per SM); CTA c takes units
-//    c, c + gridDim, ...  Units are ordered "first partition of every sequence,
-//    kv head innermost" then "remaining partitions, sequence-major": the first
-//    partition of sibling sequences that share prefix blocks is read by CTAs
-//    running at the same time, so the shared blocks are served from L2.
+//    per unit.  The grid is persistent (one CTA per SM).  CTA c's first unit
+//    is c; after it, CTA c takes c + gridDim, ... or, when a work counter is
+//    given (the shared-prefix path), draws unit ids from it, so CTAs that start
+//    early or get short units take more.  Units are ordered "further partitions
+//    of long sequences, sequence-major, kv head innermost" then "first
+//    partition of every sequence, kv head innermost": the further partitions
+//    are all full length, and the first partitions (often shorter) even out
+//    the CTAs' finish; sibling sequences' first partitions are read by CTAs
+//    running at the same time, so blocks they share come from L2.
 //  * Each of the CTA's 8 warps takes logical blocks w, w+8, ... of a unit and
 //    streams them itself: the (block, kv head) slabs of K and V (4 KB each in
 //    bf16) are fetched with 16-byte cp.async, all 32 lanes issuing, into a
@@ -25,7 +29,10 @@
 //    thread per SM cap near 0.9 TB/s (each copy costs the issuing thread
 //    ~0.65 us), so there is no producer warp.  Each warp keeps its own
 //    online-softmax state (running max m, running sum l, unnormalised
-//    accumulator); the 8 states are merged through shared memory per unit.
+//    accumulator).  The 8 states of a unit are merged without a CTA barrier:
+//    each warp leaves its state in one of two merge slots and arrives on an
+//    mbarrier, streams the next unit, then merges its 1/8 share of the
+//    previous one.
 //  * bf16: QK and PV run on warp-level tensor-core tiles (mma.sync m16n8k16, bf16
 //    operands, fp32 accumulation).  QK puts the block's 16 tokens in M and the g
 //    heads in N (S^T = K Q^T); PV computes O^T = V^T P^T with head_dim in M, so no
@@ -46,8 +53,9 @@
 //  * Split-K (partition_size > 0): a sequence with several partitions writes
 //    (m, l, acc) per partition to the workspace and reduce_kernel combines them;
 //    single-partition sequences are finished directly.
-//  * No kernel here spins: cp.async completion is waited for with wait_group and
-//    the only barriers are CTA-wide ones every warp reaches.
+//  * Every wait that depends on another warp or kernel (the merge slots' mbarrier,
+//    the ring of unit ids) is bounded by %globaltimer; on a timeout the CTA sets
+//    PA_DEVERR_TIMEOUT, raises its abort flag and every warp leaves its loop.
 #include <cfloat>
 #include <climits>
 #include <cstring>
@@ -195,18 +203,21 @@ __device__ __forceinline__ int first_part(const Params &p, int s) {
     return p.first_p ? __ldg(p.first_p + s) : 0;
 }
 
-// Unit u -> (sequence, slot, kv head).  Units [0, S*Hkv) are the first
-// per-sequence unit (slot f(s), f = first_part) of every sequence, kv head
-// innermost; after them come the further units (slots > f(s)), sequence-major,
-// using cum[s] = sum_{s' < s} (seq_units(s') - 1)^+.
-__device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t units_first, int hkv,
+// Unit u -> (sequence, slot, kv head).  Units [0, n_extra) are the further
+// units of long sequences (slots after their first unit's), sequence-major, kv
+// head innermost, using cum[s] = sum_{s' < s} (seq_units(s') - 1)^+; after them
+// comes the first per-sequence unit of every sequence (slot slot_base(fp)).  The
+// further units are all full-length, so putting them first leaves the shorter
+// first units for the end of the queue, where they even out the CTAs' finish.
+__device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t n_extra, int hkv,
                                         const int *cum, int S) {
-    if (u < units_first) {
-        const int s = (int)(u / hkv);
+    if (u >= n_extra) {
+        const int64_t f = u - n_extra;
+        const int s = (int)(f / hkv);
         const int fp = first_part(p, s);
-        return Unit{s, slot_base(fp), (int)(u % hkv), fp};
+        return Unit{s, slot_base(fp), (int)(f % hkv), fp};
     }
-    const int64_t v = u - units_first;
+    const int64_t v = u;
     const int e = (int)(v / hkv), h = (int)(v % hkv);
     int lo = 0, hi = S;  // cum[lo] <= e < cum[hi]
     while (hi - lo > 1) {
@@ -230,9 +241,9 @@ struct WarpUnit {
     bool skip;  // partition past the end (every partition was covered by a group unit)
 };
 
-__device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t units_first,
+__device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t n_extra,
                                           const int *cum, WarpUnit &w, int lane, bool flagger) {
-    w.un = unit_of(p, u, units_first, p.num_kv_heads, cum, p.num_seqs);
+    w.un = unit_of(p, u, n_extra, p.num_kv_heads, cum, p.num_seqs);
     const int k = w.un.part - slot_base(w.un.fp);  // per-sequence unit index
     const int t_first = p.part_tokens > 0 ? w.un.fp * p.part_tokens + k * p.seq_tokens : 0;
     const int b0 = t_first / kBlockSize;
@@ -776,8 +787,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     prologue(p, cum, reinterpret_cast<int *>(macc));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.num_seqs, hkv = p.num_kv_heads;
-    const int64_t units_first = (int64_t)S * hkv;
-    const int64_t total = units_first + (p.part_tokens > 0 ? (int64_t)cum[S] * hkv : 0);
+    const int64_t n_extra = p.part_tokens > 0 ? (int64_t)cum[S] * hkv : 0;
+    const int64_t total = (int64_t)S * hkv + n_extra;
     unsigned char *wring = smem + Lay::kOffRing + (size_t)warp * NS * Lay::kStageBytes;
     const uint32_t wring_s = smem_u32(wring);
     float *pw = pbuf + warp * Lay::kPWarpFloats;
@@ -828,10 +839,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         grid_dep_wait();
         return;
     }
-    load_unit(p, u, units_first, cum, cur, lane, warp == 0);
+    load_unit(p, u, n_extra, cum, cur, lane, warp == 0);
     int64_t u_nxt = unit_id(1);
     bool have_nxt = u_nxt < total;
-    if (have_nxt) load_unit(p, u_nxt, units_first, cum, nxt, lane, warp == 0);
+    if (have_nxt) load_unit(p, u_nxt, n_extra, cum, nxt, lane, warp == 0);
 
     // table entry of logical block j of a unit (the first 32 come from registers)
     auto phys_of = [&](const WarpUnit &w, int j) {
@@ -1040,7 +1051,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         iss_u = iss_u > 0 ? iss_u - 1 : 0;
         u_nxt = unit_id(uc + 2);
         have_nxt = u_nxt < total;
-        if (have_nxt) load_unit(p, u_nxt, units_first, cum, nxt, lane, warp == 0);
+        if (have_nxt) load_unit(p, u_nxt, n_extra, cum, nxt, lane, warp == 0);
     }
     // the last unit's merge
     if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err, p.wait_ns))
@@ -1310,30 +1321,67 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
 
 // Combine split-K partials: one warp per (sequence, query head) with more than
 // one partition.  M = max_p m_p; out = sum_p 2^(m_p-M) acc_p / sum_p 2^(m_p-M) l_p.
+// The first kPre slots are loaded together with the length that says how many
+// slots there are (slots past it are ignored), so most rows take one memory
+// round trip after the decode ends.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Params p) {
     grid_dep_wait();  // every partial is written
     constexpr int kDpl = D / 32;
+    constexpr int kPre = 4;
     const int lane = threadIdx.x & 31;
     const int64_t wid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
     if (wid >= (int64_t)p.num_seqs * p.num_q_heads) return;
     const int s = (int)(wid / p.num_q_heads);
+    const float2 *ml = p.ws_ml + wid * p.max_parts;
+    const float *acc = p.ws_acc + wid * p.max_parts * D + lane * kDpl;
+    float2 mlp[kPre];
+    float ap[kPre][kDpl];
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) {
+        const bool in = i < p.max_parts;  // inside the workspace row (maybe unwritten)
+        mlp[i] = in ? ml[i] : make_float2(-INFINITY, 0.f);
+#pragma unroll
+        for (int k = 0; k < kDpl; ++k) ap[i][k] = 0.f;
+        if (in) {
+            if constexpr (kDpl == 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(acc + (int64_t)i * D);
+                ap[i][0] = a.x; ap[i][1] = a.y; ap[i][2] = a.z; ap[i][3] = a.w;
+            } else {
+                const float2 a = *reinterpret_cast<const float2 *>(acc + (int64_t)i * D);
+                ap[i][0] = a.x; ap[i][1] = a.y;
+            }
+        }
+    }
     int L = checked_len(p, s);
     if (L < 0) L = 0;
     const int fp = first_part(p, s);
     const int n = slot_base(fp) + seq_units(p, L, fp);  // slots written
     if (fp == 0 && n <= 1) return;                       // finished by the decode kernel
-    const float2 *ml = p.ws_ml + wid * p.max_parts;
-    const float *acc = p.ws_acc + wid * p.max_parts * D + lane * kDpl;
     float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[i].x);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    for (int i = 0; i < kPre; ++i)
+        if (i < n) M = fmaxf(M, mlp[i].x);
+    if (n > kPre) {
+        float Mr = -INFINITY;
+        for (int i = kPre + lane; i < n; i += 32) Mr = fmaxf(Mr, ml[i].x);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Mr = fmaxf(Mr, __shfl_xor_sync(kFull, Mr, o));
+        M = fmaxf(M, Mr);
+    }
     float lsum = 0.f, o[kDpl];
 #pragma unroll
     for (int k = 0; k < kDpl; ++k) o[k] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kPre; ++i) {
+        if (i >= n) break;
+        const float f = fast_exp2(mlp[i].x - M);
+        lsum = fmaf(mlp[i].y, f, lsum);
+#pragma unroll
+        for (int k = 0; k < kDpl; ++k) o[k] = fmaf(ap[i][k], f, o[k]);
+    }
 #pragma unroll 4
-    for (int i = 0; i < n; ++i) {
+    for (int i = kPre; i < n; ++i) {
         const float2 mi = ml[i];
         const float f = fast_exp2(mi.x - M);
         lsum = fmaf(mi.y, f, lsum);
