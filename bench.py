@@ -422,9 +422,9 @@ def run_ours(args):
 
     if rank == 0:
         # kernels of one pa_append_decode call: the decode chain, plus the write's own
-        # launch unless the shared-prefix chain (4 kernels) takes the write into its first
+        # launch unless the shared-prefix chain (5 kernels) takes the write into its first
         n_dec = pa.pa_decode_launches(S, wl.head_dim, pa.PA_BF16, part)
-        step_launches = n_dec if n_dec == 4 else n_dec + 1
+        step_launches = n_dec if n_dec == 5 else n_dec + 1
         peaks = load_peaks()
         peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
         achieved = (unique_b + cw_b) / (call_ms * 1e-3) / 1e9

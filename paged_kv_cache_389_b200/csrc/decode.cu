@@ -101,14 +101,22 @@ template <typename T>
 using IoT = typename std::conditional<kIsFp8<T>, __nv_bfloat16, T>::type;
 
 constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// Query rows of one unit of the group-rows mode (decode_kernel<T, D, kRowTile>):
+// the members x g query heads of a small sibling group, two 8-column tensor-core
+// tiles.
+constexpr int kRowTile = 16;
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Shared-memory carve-up (byte offsets from the dynamic shared memory base).
 // Each warp owns kStagesPerWarp ring stages (K slab + V slab each): two, or one
 // when a stage is too large (fp32, head_dim 128).  Two merge slots let the
-// merge of a unit run while the next unit streams (mbarrier hand-over).
+// merge of a unit run while the next unit streams (mbarrier hand-over).  The
+// group-rows mode (G == kRowTile: 16 rows per warp state) has room for one merge
+// slot only and keeps no per-sequence prefix sums.
 template <typename T, int D, int G>
 struct Layout {
+    static constexpr bool kRows = G == kRowTile;
     static constexpr int kElem = ElemBytes<T>::value;
     static constexpr int kRowBytes = D * kElem;                 // one token of one head
     static constexpr int kQRowBytes = D * (int)sizeof(IoT<T>);  // one query head
@@ -117,13 +125,14 @@ struct Layout {
     static constexpr size_t kLimit = 232448;                    // sm_100 max dynamic smem per CTA
     static constexpr size_t kPBytes = sizeof(T) == 4 ? (size_t)kWarps * (16 * G + G) * 4 : 64;
     static constexpr size_t kMergeBytes = (size_t)kWarps * G * (D * 4 + 8);
-    static constexpr size_t kFixed = kPBytes + 16 + 48 + 96 + (size_t)(kMaxSplitSeqs + 1) * 4 + 64;
+    static constexpr size_t kFixed = kPBytes + 16 + 48 + 96 + (kRows ? 0 : (size_t)(kMaxSplitSeqs + 1) * 4) + 64;
     static constexpr int stages_fit(int bufs) {
         return (int)((kLimit - kFixed - bufs * kMergeBytes) / ((size_t)kWarps * kStageBytes));
     }
     static constexpr int kWantStages = kIsFp8<T> ? 4 : 2;
-    static constexpr int kStagesPerWarp = stages_fit(2) >= kWantStages ? kWantStages : (stages_fit(2) >= 2 ? 2 : 1);
-    static constexpr int kMergeBufs = stages_fit(2) >= kStagesPerWarp ? 2 : 1;
+    static constexpr int kStagesPerWarp =
+        kRows ? kWantStages : (stages_fit(2) >= kWantStages ? kWantStages : (stages_fit(2) >= 2 ? 2 : 1));
+    static constexpr int kMergeBufs = kRows ? 1 : (stages_fit(2) >= kStagesPerWarp ? 2 : 1);
     static constexpr size_t kPWarpFloats = 16 * G + G;          // fp32 path: p[16][G], alpha[G]
     static constexpr size_t kOffRing = 0;
     static constexpr size_t kOffP = kOffRing + (size_t)kWarps * kStagesPerWarp * kStageBytes;
@@ -155,12 +164,16 @@ struct Params {
     int32_t max_parts;
     int32_t seq_tokens;   // split: tokens per per-sequence unit (a multiple of part_tokens)
     float scale_log2;
-    // shared-prefix groups (split contexts only; nullptr = none): first_p[s] is the
-    // number of leading partitions of s computed by group_decode_kernel
-    const int32_t *first_p;
-    const int4 *groups;     // (first seq, members, shared partitions, units before)
-    const int32_t *meta;    // [0] groups, [1] group units, [2] / [3] work counters, [4] tile CTAs
-    int32_t max_members;    // sequences per group: query rows members x g <= 128
+    // shared-prefix groups (split contexts only; nullptr = none): first_t[s] is the
+    // number of leading tokens of s computed by its group's unit (a multiple of 16,
+    // at least part_tokens; 0 outside a group)
+    const int32_t *first_t;
+    const int4 *groups;     // (first seq, members, shared tokens, units before)
+    const int32_t *meta;    // [0] tile groups, [1] their units, [2] / [3] work counters of the
+                            // per-sequence and tile kernels, [4] tile CTAs, [5] row groups,
+                            // [6] group-rows work counter, [7] group-rows CTAs
+    int32_t max_members;    // sequences per tile group: query rows members x g <= 128
+    int32_t tile_groups;    // detection may form tile groups (bf16 pools); else row groups only
     int32_t wait_first;     // launched right behind a cache write: wait for it first
     float v_scale;          // fp8 pools: value dequantisation scale (1 otherwise)
     unsigned long long wait_ns;  // bound of every in-kernel wait
@@ -178,35 +191,36 @@ __device__ __forceinline__ int checked_len(const Params &p, int s) {
     return check_len(p, __ldg(p.lens + s));
 }
 
-// Split contexts: the first fp partitions of part_tokens (shared-prefix group
-// units, one partial per partition in slots 0..fp-1) are followed by
-// per-sequence units of seq_tokens each; unit k writes slot fp + k.  Returns the
-// number of per-sequence units (1 unsplit).
-__device__ __forceinline__ int seq_units(const Params &p, int L, int fp) {
+// Split contexts: the first ft tokens (shared with the other members of a
+// group; one partial in slot 0, written by the group's unit) are followed by
+// per-sequence units of seq_tokens each; unit k writes slot slot_base(ft) + k.
+// Returns the number of per-sequence units (1 unsplit).  With ft >= part_tokens
+// and seq_tokens >= part_tokens the slots never exceed ceil(L / part_tokens).
+__device__ __forceinline__ int seq_units(const Params &p, int L, int ft) {
     if (p.part_tokens <= 0) return 1;
-    const int rem = L - fp * p.part_tokens;
-    if (fp == 0 && rem <= 0) return 1;  // empty context: one unit, finished as 0
+    const int rem = L - ft;
+    if (ft == 0 && rem <= 0) return 1;  // empty context: one unit, finished as 0
     return rem > 0 ? (rem + p.seq_tokens - 1) / p.seq_tokens : 0;
 }
 
 struct Unit {
     int s, part, h;  // part: the workspace slot the unit writes
-    int fp;          // first_part(s): partitions of s computed by group units
+    int ft;          // first_tok(s): leading tokens of s computed by its group's unit
 };
 
 // Workspace slot of a sequence's first per-sequence unit: its shared leading
-// partitions (fp of them) are computed together by one group unit per kv head,
-// which writes one partial into slot 0.
-__device__ __forceinline__ int slot_base(int fp) { return fp > 0 ? 1 : 0; }
+// tokens are computed together by one group unit per kv head, which writes one
+// partial into slot 0.
+__device__ __forceinline__ int slot_base(int ft) { return ft > 0 ? 1 : 0; }
 
-__device__ __forceinline__ int first_part(const Params &p, int s) {
-    return p.first_p ? __ldg(p.first_p + s) : 0;
+__device__ __forceinline__ int first_tok(const Params &p, int s) {
+    return p.first_t ? __ldg(p.first_t + s) : 0;
 }
 
 // Unit u -> (sequence, slot, kv head).  Units [0, n_extra) are the further
 // units of long sequences (slots after their first unit's), sequence-major, kv
 // head innermost, using cum[s] = sum_{s' < s} (seq_units(s') - 1)^+; after them
-// comes the first per-sequence unit of every sequence (slot slot_base(fp)).  The
+// comes the first per-sequence unit of every sequence (slot slot_base(ft)).  The
 // further units are all full-length, so putting them first leaves the shorter
 // first units for the end of the queue, where they even out the CTAs' finish.
 __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t n_extra, int hkv,
@@ -214,8 +228,8 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t n_ex
     if (u >= n_extra) {
         const int64_t f = u - n_extra;
         const int s = (int)(f / hkv);
-        const int fp = first_part(p, s);
-        return Unit{s, slot_base(fp), (int)(f % hkv), fp};
+        const int ft = first_tok(p, s);
+        return Unit{s, slot_base(ft), (int)(f % hkv), ft};
     }
     const int64_t v = u;
     const int e = (int)(v / hkv), h = (int)(v % hkv);
@@ -224,8 +238,8 @@ __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t n_ex
         const int mid = (lo + hi) >> 1;
         if (cum[mid] <= e) lo = mid; else hi = mid;
     }
-    const int fp = first_part(p, lo);
-    return Unit{lo, slot_base(fp) + 1 + e - cum[lo], h, fp};
+    const int ft = first_tok(p, lo);
+    return Unit{lo, slot_base(ft) + 1 + e - cum[lo], h, ft};
 }
 
 // What one warp needs to know about a unit.  `tab` holds, in lane i, the table
@@ -239,13 +253,31 @@ struct WarpUnit {
     int tab;
     const int32_t *trow;
     bool skip;  // partition past the end (every partition was covered by a group unit)
+    int nrow;   // group-rows mode: query rows in use (members x g)
 };
+
+// Group-rows mode: unit v = (row group v / Hkv, kv head v % Hkv).  Its keys are
+// the group's shared tokens (whole blocks of the first member's table); its rows
+// are members x g query heads, member-major.
+__device__ __forceinline__ void load_unit_rows(const Params &p, int64_t v, int gbase, WarpUnit &w, int lane) {
+    const int hkv = p.num_kv_heads;
+    const int4 gr = __ldg(p.groups + gbase + (int)(v / hkv));  // (first seq, members, shared tokens, -)
+    w.un = Unit{gr.x, 0, (int)(v % hkv), gr.z};
+    w.L = gr.z;
+    w.t0 = 0;
+    w.nt = gr.z;
+    w.nb = gr.z / kBlockSize;
+    w.trow = p.tables + (int64_t)gr.x * p.max_blocks;
+    w.tab = lane < p.max_blocks ? __ldg(w.trow + lane) : -1;
+    w.skip = false;
+    w.nrow = gr.y * (p.num_q_heads / hkv);
+}
 
 __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t n_extra,
                                           const int *cum, WarpUnit &w, int lane, bool flagger) {
     w.un = unit_of(p, u, n_extra, p.num_kv_heads, cum, p.num_seqs);
-    const int k = w.un.part - slot_base(w.un.fp);  // per-sequence unit index
-    const int t_first = p.part_tokens > 0 ? w.un.fp * p.part_tokens + k * p.seq_tokens : 0;
+    const int k = w.un.part - slot_base(w.un.ft);  // per-sequence unit index
+    const int t_first = p.part_tokens > 0 ? w.un.ft + k * p.seq_tokens : 0;
     const int b0 = t_first / kBlockSize;
     w.trow = p.tables + (int64_t)w.un.s * p.max_blocks + b0;
     // both loads issued before either value is needed
@@ -264,7 +296,7 @@ __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t n_
         w.t0 = t_first;
         w.nt = max(0, min(L, w.t0 + p.seq_tokens) - w.t0);
     }
-    w.skip = k >= seq_units(p, L, w.un.fp);
+    w.skip = k >= seq_units(p, L, w.un.ft);
     if (w.skip) w.nt = 0;
     w.nb = (w.nt + kBlockSize - 1) / kBlockSize;
 }
@@ -280,7 +312,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
         int local = 0;
         for (int s = beg; s < end; ++s) {
             const int L = checked_len(p, s);
-            local += max(0, seq_units(p, L < 0 ? 0 : L, first_part(p, s)) - 1);
+            local += max(0, seq_units(p, L < 0 ? 0 : L, first_tok(p, s)) - 1);
         }
         int incl = local;
 #pragma unroll
@@ -296,7 +328,7 @@ __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch
         for (int s = beg; s < end; ++s) {
             cum[s] = run;
             const int L = checked_len(p, s);
-            run += max(0, seq_units(p, L < 0 ? 0 : L, first_part(p, s)) - 1);
+            run += max(0, seq_units(p, L < 0 ? 0 : L, first_tok(p, s)) - 1);
         }
         if ((int)threadIdx.x == kThreads - 1) cum[S] = run;
     }
@@ -343,7 +375,7 @@ template <typename T, int D, int G>
 __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, const float *uacc,
                                             const float2 *uml) {
     if (w.skip) return;
-    const bool single = w.un.fp == 0 && seq_units(p, w.L, 0) == 1;
+    const bool single = w.un.ft == 0 && seq_units(p, w.L, 0) == 1;
     const int64_t head0 = (int64_t)w.un.s * p.num_q_heads + (int64_t)w.un.h * G;
     for (int e = threadIdx.x; e < G * D; e += kThreads) {
         const int h = e / D, dd = e - h * D;
@@ -370,6 +402,38 @@ __device__ __forceinline__ void finish_unit(const Params &p, const WarpUnit &w, 
             p.ws_acc[row * D + dd] = o;
             if (dd == 0) p.ws_ml[row] = make_float2(M, lsum);
         }
+    }
+}
+
+// Group-rows mode: combine the warps' states of a unit (rows r < w.nrow) and
+// write the partial of its shared tokens into workspace slot 0 of every member:
+// row r is query head h g + r % g of sequence first + r / g.
+template <typename T, int D>
+__device__ __forceinline__ void finish_unit_rows(const Params &p, const WarpUnit &w, const float *uacc,
+                                                 const float2 *uml) {
+    const int g = p.num_q_heads / p.num_kv_heads;
+    for (int e = threadIdx.x; e < kRowTile * D; e += kThreads) {
+        const int r = e / D, dd = e - r * D;
+        if (r >= w.nrow) break;  // rows only grow with e
+        float M = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < kWarps; ++k) M = fmaxf(M, uml[k * kRowTile + r].x);
+        float lsum = 0.f, o = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int k = 0; k < kWarps; ++k) {
+                const float2 ml = uml[k * kRowTile + r];
+                if (ml.x != -INFINITY) {
+                    const float f = fast_exp2(ml.x - M);
+                    lsum = fmaf(ml.y, f, lsum);
+                    o = fmaf(uacc[(k * kRowTile + r) * D + dd], f, o);
+                }
+            }
+        }
+        if constexpr (kIsFp8<T>) o *= p.v_scale;
+        const int64_t row = ((int64_t)(w.un.s + r / g) * p.num_q_heads + (int64_t)w.un.h * g + r % g) * p.max_parts;
+        p.ws_acc[row * D + dd] = o;
+        if (dd == 0) p.ws_ml[row] = make_float2(M, lsum);
     }
 }
 
@@ -502,6 +566,123 @@ __device__ __forceinline__ void mma_block(uint32_t kb, unsigned char *vgen, int 
     }
 }
 
+// Group-rows mode: the state of 16 query rows, two 8-column tiles (n = 0, 1).
+// m, l: columns 2(lane%4), 2(lane%4)+1 of tile 0, then of tile 1; o: O^T
+// accumulators per (head-dim tile, column tile); qb: Q^T operand fragments.
+template <int D>
+struct MmaRows {
+    float m[4], l[4];
+    float o[D / 16][2][4];
+    uint32_t qb[D / 16][2][2];
+};
+
+// Group-rows mode: one online-softmax step per column over one 16-token block.
+// s[n]: column tile n's scores in log2 units as S^T fragments (tokens lane/4 and
+// lane/4 + 8, columns 2(lane%4) and 2(lane%4)+1).  Masks tokens at or past ntok
+// (>= 1), updates m and l, rescales the O^T accumulators and leaves the
+// unnormalised probabilities in s.
+template <int D>
+__device__ __forceinline__ void softmax_rows(float (&s)[2][4], int ntok, MmaRows<D> &st, int lane) {
+    constexpr int KS = D / 16;
+    const int t0 = lane >> 2;
+    float c[4], al[4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        if (t0 >= ntok) s[n][0] = s[n][1] = -INFINITY;
+        if (t0 + 8 >= ntok) s[n][2] = s[n][3] = -INFINITY;
+        c[2 * n] = fmaxf(s[n][0], s[n][2]);
+        c[2 * n + 1] = fmaxf(s[n][1], s[n][3]);
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = fmaxf(c[i], __shfl_xor_sync(kFull, c[i], off));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float mn = fmaxf(st.m[i], c[i]);
+        al[i] = fast_exp2(st.m[i] - mn);
+        st.m[i] = mn;
+    }
+    float r[4];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        s[n][0] = fast_exp2(s[n][0] - st.m[2 * n]);
+        s[n][1] = fast_exp2(s[n][1] - st.m[2 * n + 1]);
+        s[n][2] = fast_exp2(s[n][2] - st.m[2 * n]);
+        s[n][3] = fast_exp2(s[n][3] - st.m[2 * n + 1]);
+        r[2 * n] = s[n][0] + s[n][2];
+        r[2 * n + 1] = s[n][1] + s[n][3];
+    }
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) r[i] += __shfl_xor_sync(kFull, r[i], off);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st.l[i] = st.l[i] * al[i] + r[i];
+    if (__any_sync(kFull, al[0] != 1.f || al[1] != 1.f || al[2] != 1.f || al[3] != 1.f)) {
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt)
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                st.o[mt][n][0] *= al[2 * n];
+                st.o[mt][n][1] *= al[2 * n + 1];
+                st.o[mt][n][2] *= al[2 * n];
+                st.o[mt][n][3] *= al[2 * n + 1];
+            }
+    }
+}
+
+// One 16-token block against 16 query rows: S^T = K Q^T as two 16 x 8 tiles
+// sharing every K fragment, one online-softmax step per column, then
+// O^T += V^T P^T with every V fragment feeding both column tiles.
+template <int D>
+__device__ __forceinline__ void mma_block_rows(uint32_t kb, unsigned char *vgen, int ntok, MmaRows<D> &st,
+                                               float sl2, int lane) {
+    constexpr int KS = D / 16;
+    constexpr int kRow = 2 * D;
+    const uint32_t vb = kb + kBlockSize * kRow;
+    const int mat = lane >> 3, r8 = lane & 7;
+    auto addr = [&](uint32_t base, int row, int chunk) {
+        return base + row * kRow + ((((chunk & ~7) | ((chunk ^ row) & 7))) << 4);
+    };
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const int krow = ((mat & 1) << 3) + r8;
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+        uint32_t a[4];
+        ldsm_x4(a, addr(kb, krow, kk * 2 + (mat >> 1)));
+        mma_bf16_16816(s[0], a, st.qb[kk][0][0], st.qb[kk][0][1]);
+        mma_bf16_16816(s[1], a, st.qb[kk][1][0], st.qb[kk][1][1]);
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s[n][k] *= sl2;
+    softmax_rows<D>(s, ntok, st, lane);
+    // P^T operand fragments of both column tiles, transposed in registers
+    uint32_t pb[2][2];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        pb[n][0] = movmatrix_trans(pack_bf16x2(s[n][0], s[n][1]));
+        pb[n][1] = movmatrix_trans(pack_bf16x2(s[n][2], s[n][3]));
+    }
+    if (ntok < kBlockSize) {
+        // zero the V rows past the keys: 0 * (NaN or Inf) would poison the sums
+        for (int idx = lane; idx < (kBlockSize - ntok) * (kRow / 16); idx += 32)
+            *reinterpret_cast<uint4 *>(vgen + (ntok + idx / (kRow / 16)) * kRow + (idx % (kRow / 16)) * 16) =
+                make_uint4(0, 0, 0, 0);
+        __syncwarp();
+    }
+    const int vrow = ((mat >> 1) << 3) + r8;
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) {
+        uint32_t a[4];
+        ldsm_x4_trans(a, addr(vb, vrow, mt * 2 + (mat & 1)));
+        mma_bf16_16816(st.o[mt][0], a, pb[0][0], pb[0][1]);
+        mma_bf16_16816(st.o[mt][1], a, pb[1][0], pb[1][1]);
+    }
+}
+
 // ------------------------------------------------------------- fp8 block
 // Four e4m3 codes (bytes 0..3 of w) -> two f16x2 registers (exact): lo holds
 // bytes 0, 1 and hi bytes 2, 3, the lower byte in the lower half of each.
@@ -592,6 +773,72 @@ __device__ __forceinline__ void mma_tiles_fp8(unsigned char *const (&kb)[NT], co
             e4m3x4_to_f16x2x2(f23, a[2], a[3]);
             mma_f16_16816(st.o[2 * w + 1], a, pb0[b], pb1[b]);
         }
+    }
+}
+
+// Group-rows mode on an fp8 pool: one 16-token block against 16 query rows, with
+// the dim maps of mma_tiles_fp8 (each converted K or V fragment feeds both column
+// tiles).  kb: the block's stage (K slab, V slab behind it).
+template <int D>
+__device__ __forceinline__ void mma_block_rows_fp8(unsigned char *kb, int ntok, MmaRows<D> &st, float sl2,
+                                                   int lane) {
+    static_assert(D == 128, "the fp8 fragment map assumes 128-byte rows");
+    constexpr int kSlab = kBlockSize * D;
+    const int g = lane >> 2, t = lane & 3;
+    auto chunk = [&](const unsigned char *base, int row, int c) {
+        return *reinterpret_cast<const uint4 *>(base + row * D + ((c ^ (row & 7)) << 4));
+    };
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const uint4 lo = chunk(kb, g, 2 * t + j), hi = chunk(kb, g + 8, 2 * t + j);
+        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int kk = 4 * j + i;
+            uint32_t a[4];
+            e4m3x4_to_f16x2x2(wl[i], a[0], a[2]);
+            e4m3x4_to_f16x2x2(wh[i], a[1], a[3]);
+            mma_f16_16816(s[0], a, st.qb[kk][0][0], st.qb[kk][0][1]);
+            mma_f16_16816(s[1], a, st.qb[kk][1][0], st.qb[kk][1][1]);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) s[n][k] *= sl2;
+    softmax_rows<D>(s, ntok, st, lane);
+    uint32_t pb[2][2];
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+        pb[n][0] = movmatrix_trans(pack_f16x2(s[n][0], s[n][1]));
+        pb[n][1] = movmatrix_trans(pack_f16x2(s[n][2], s[n][3]));
+    }
+    unsigned char *vb = kb + kSlab;
+    if (ntok < kBlockSize) {
+        // codes past the keys may be NaN: zero those V rows
+        for (int idx = lane; idx < (kBlockSize - ntok) * (D / 16); idx += 32)
+            *reinterpret_cast<uint4 *>(vb + (ntok + idx / (D / 16)) * D + (idx % (D / 16)) * 16) =
+                make_uint4(0, 0, 0, 0);
+        __syncwarp();
+    }
+    const uint4 v0 = chunk(vb, 2 * t, g), v1 = chunk(vb, 2 * t + 1, g);
+    const uint4 v2 = chunk(vb, 2 * t + 8, g), v3 = chunk(vb, 2 * t + 9, g);
+    const uint32_t r0[4] = {v0.x, v0.y, v0.z, v0.w}, r1[4] = {v1.x, v1.y, v1.z, v1.w};
+    const uint32_t r2[4] = {v2.x, v2.y, v2.z, v2.w}, r3[4] = {v3.x, v3.y, v3.z, v3.w};
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const uint32_t e01 = __byte_perm(r0[w], r1[w], 0x5140), f01 = __byte_perm(r0[w], r1[w], 0x7362);
+        const uint32_t e23 = __byte_perm(r2[w], r3[w], 0x5140), f23 = __byte_perm(r2[w], r3[w], 0x7362);
+        uint32_t a[4];
+        e4m3x4_to_f16x2x2(e01, a[0], a[1]);
+        e4m3x4_to_f16x2x2(e23, a[2], a[3]);
+        mma_f16_16816(st.o[2 * w][0], a, pb[0][0], pb[0][1]);
+        mma_f16_16816(st.o[2 * w][1], a, pb[1][0], pb[1][1]);
+        e4m3x4_to_f16x2x2(f01, a[0], a[1]);
+        e4m3x4_to_f16x2x2(f23, a[2], a[3]);
+        mma_f16_16816(st.o[2 * w + 1][0], a, pb[0][0], pb[0][1]);
+        mma_f16_16816(st.o[2 * w + 1][1], a, pb[1][0], pb[1][1]);
     }
 }
 
@@ -739,15 +986,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     float2 *mml = reinterpret_cast<float2 *>(smem + Lay::kOffMml);
     int *cum = reinterpret_cast<int *>(smem + Lay::kOffCum);
 
-    static_assert(Lay::kMergeBufs == 2, "the deferred merge needs two slots");
+    constexpr bool kRows = Lay::kRows;
+    static_assert(Lay::kMergeBufs == 2 || kRows, "the deferred merge needs two slots");
+    static_assert(!kRows || kMma, "group-rows mode runs on tensor-core tiles");
     // The combine may start launching now; it waits for this grid to finish.
     // When launched behind the group tiles, this grid reads only what the
     // detection wrote (complete before the tiles let it start) and writes other
     // partitions; it waits for the tiles only before exiting, so that its
     // completion implies theirs.  Launched right behind a cache write instead
     // (pa_append_decode without groups), it waits for the write first.
-    grid_dep_launch();
-    if (p.wait_first) grid_dep_wait();
+    if (kRows && p.wait_first) {
+        // group-rows mode right behind the detection (no tile kernel between): the
+        // next kernel reads the detection output, so it may launch only after it
+        grid_dep_wait();
+        grid_dep_launch();
+    } else {
+        grid_dep_launch();
+        if (p.wait_first) grid_dep_wait();
+    }
+    // Group-rows mode: the detection kernel chose how many CTAs take row-group
+    // units (ids from the counter meta[6]); the others leave their SM at once.
+    // CTA 0 always stays until the previous kernel of the call has finished, so
+    // that this grid's completion implies it (the next kernel waits for this grid).
+    int dyn_base = (int)gridDim.x;
+    if constexpr (kRows) {
+        dyn_base = min((int)gridDim.x, __ldg(p.meta + 7));
+        if ((int)blockIdx.x >= dyn_base) {
+            if (blockIdx.x == 0) grid_dep_wait();
+            return;
+        }
+    }
     // merge slot hand-over: full[b] when all warps wrote their state of the
     // slot's unit, freed[b] when all warps finished their share of its merge
     uint64_t *mfull = reinterpret_cast<uint64_t *>(smem + Lay::kOffBar);
@@ -777,18 +1045,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         ring_tag[0] = ring_claim[0] = 0;
         if (dyn) {
-            const int v = (int)gridDim.x + atomicAdd(p.work_ctr, 2);
+            const int v = dyn_base + atomicAdd(p.work_ctr, 2);
             ring_id[1] = v;
             ring_id[2] = v + 1;
             ring_tag[1] = ring_claim[1] = 1;
             ring_tag[2] = ring_claim[2] = 2;
         }
     }
-    prologue(p, cum, reinterpret_cast<int *>(macc));
+    if constexpr (kRows) __syncthreads();  // barriers and ring initialised
+    else prologue(p, cum, reinterpret_cast<int *>(macc));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = p.num_seqs, hkv = p.num_kv_heads;
-    const int64_t n_extra = p.part_tokens > 0 ? (int64_t)cum[S] * hkv : 0;
-    const int64_t total = (int64_t)S * hkv + n_extra;
+    const int64_t n_extra = !kRows && p.part_tokens > 0 ? (int64_t)cum[S] * hkv : 0;
+    const int gbase = kRows ? __ldg(p.meta) : 0;  // row groups follow the tile groups
+    const int64_t total = kRows ? (int64_t)__ldg(p.meta + 5) * hkv : (int64_t)S * hkv + n_extra;
+    auto load_any = [&](int64_t u, WarpUnit &w) {
+        if constexpr (kRows) load_unit_rows(p, u, gbase, w, lane);
+        else load_unit(p, u, n_extra, cum, w, lane, warp == 0);
+    };
     unsigned char *wring = smem + Lay::kOffRing + (size_t)warp * NS * Lay::kStageBytes;
     const uint32_t wring_s = smem_u32(wring);
     float *pw = pbuf + warp * Lay::kPWarpFloats;
@@ -828,7 +1102,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         while (ring_tag[(k2 - 1) & 7] != k2 - 1) {
             if (*abort_flag || global_ns() - t0 > p.wait_ns) break;
         }
-        ring_id[sl] = (int)gridDim.x + atomicAdd(p.work_ctr, 1);
+        ring_id[sl] = dyn_base + atomicAdd(p.work_ctr, 1);
         __threadfence_block();
         ring_tag[sl] = k2;
     };
@@ -839,10 +1113,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         grid_dep_wait();
         return;
     }
-    load_unit(p, u, n_extra, cum, cur, lane, warp == 0);
+    load_any(u, cur);
     int64_t u_nxt = unit_id(1);
     bool have_nxt = u_nxt < total;
-    if (have_nxt) load_unit(p, u_nxt, n_extra, cum, nxt, lane, warp == 0);
+    if (have_nxt) load_any(u_nxt, nxt);
 
     // table entry of logical block j of a unit (the first 32 come from registers)
     auto phys_of = [&](const WarpUnit &w, int j) {
@@ -889,10 +1163,54 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     for (;; ++uc) {
         // ---- q operands of this unit (tiny, L2 resident)
         MmaState<D> ms;
-        F32State<D, G> fs;
+        MmaRows<D> mr;
+        F32State<D, (G > 8 ? 8 : G)> fs;
         const unsigned char *qg =
             p.q + ((int64_t)cur.un.s * p.num_q_heads + (int64_t)cur.un.h * G) * Lay::kQRowBytes;
-        if constexpr (kFp8) {
+        if constexpr (kRows) {
+            // row r = 8 n + lane / 4 of column tile n: head h g + r % g of member r / g
+            const int g = p.num_q_heads / hkv;
+#pragma unroll
+            for (int n = 0; n < 2; ++n) {
+                const int r = 8 * n + dr;
+                const bool rv = r < cur.nrow;
+                const unsigned char *qr =
+                    p.q + ((int64_t)(cur.un.s + r / g) * p.num_q_heads + (int64_t)cur.un.h * g + r % g) *
+                              Lay::kQRowBytes;
+                if constexpr (kFp8) {
+                    // bf16 -> f16 in the k-slot map of mma_tiles_fp8, clamped to the f16 range
+#pragma unroll
+                    for (int j = 0; j < 2; ++j)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int d0 = 32 * q4 + 16 * j + 4 * i;
+                            uint2 x = make_uint2(0u, 0u);
+                            if (rv) x = __ldg(reinterpret_cast<const uint2 *>(qr + d0 * 2));
+                            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.x));
+                            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.y));
+                            auto c = [](float v) { return fminf(fmaxf(v, -65504.f), 65504.f); };
+                            mr.qb[4 * j + i][n][0] = pack_f16x2(c(a.x), c(a.y));
+                            mr.qb[4 * j + i][n][1] = pack_f16x2(c(b.x), c(b.y));
+                        }
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const int d0 = kk * 16 + 2 * q4;
+                        mr.qb[kk][n][0] = rv ? __ldg(reinterpret_cast<const uint32_t *>(qr + d0 * 2)) : 0u;
+                        mr.qb[kk][n][1] = rv ? __ldg(reinterpret_cast<const uint32_t *>(qr + (d0 + 8) * 2)) : 0u;
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                mr.m[i] = -INFINITY;
+                mr.l[i] = 0.f;
+            }
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+                for (int n = 0; n < 2; ++n) mr.o[mt][n][0] = mr.o[mt][n][1] = mr.o[mt][n][2] = mr.o[mt][n][3] = 0.f;
+        } else if constexpr (kFp8) {
             // bf16 -> f16 in the k-slot map of mma_block_fp8; clamped to the f16 range
             const bool hv = dr < G;
 #pragma unroll
@@ -945,7 +1263,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
         // ---- this warp's blocks of the unit, up to NS fetched ahead (fp8: two
         // blocks per step, the pair's stages both landed before it is computed)
-        if constexpr (kFp8) {
+        if constexpr (kFp8 && !kRows) {
             static_assert(NS >= 2, "paired fp8 blocks need two stages");
             for (int j = warp; j < cur.nb; j += 2 * kWarps) {
                 const bool two = j + kWarps < cur.nb;
@@ -979,7 +1297,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int stage = n_cmp % NS;
             if ((okmask >> stage) & 1u) {
                 const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
-                if constexpr (kMma)
+                if constexpr (kRows && kFp8)
+                    mma_block_rows_fp8<D>(wring + stage * Lay::kStageBytes, ntok, mr, p.scale_log2, lane);
+                else if constexpr (kRows)
+                    mma_block_rows<D>(wring_s + stage * Lay::kStageBytes,
+                                      wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, mr,
+                                      p.scale_log2, lane);
+                else if constexpr (kMma)
                     mma_block<D>(wring_s + stage * Lay::kStageBytes,
                                  wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
                                  p.scale_log2, lane);
@@ -995,6 +1319,45 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         }
         claim_ahead(uc);
 
+        if constexpr (kRows) {
+            // ---- one merge slot: this warp's state goes in once every warp has
+            // finished its share of the previous unit's merge; then all warps meet
+            // and each merges its share of this unit
+            if (uc >= 1 && !mbar_wait_bounded(&mfreed[0], (uc - 1) & 1, abort_flag, p.err, p.wait_ns)) {
+                dead = true;
+                break;
+            }
+            float *wacc = macc + (size_t)warp * kRowTile * D;
+            float2 *wml = mml + (size_t)warp * kRowTile;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    // accumulator row dr + 8 half of tile mt (fp8: the dim map of mma_tiles_fp8)
+                    const int d = kFp8 ? 16 * dr + 2 * mt + half : mt * 16 + dr + 8 * half;
+#pragma unroll
+                    for (int n = 0; n < 2; ++n) {
+                        wacc[(8 * n + 2 * q4) * D + d] = mr.o[mt][n][2 * half];
+                        wacc[(8 * n + 2 * q4 + 1) * D + d] = mr.o[mt][n][2 * half + 1];
+                    }
+                }
+            if (dr == 0) {
+#pragma unroll
+                for (int n = 0; n < 2; ++n) {
+                    wml[8 * n + 2 * q4] = make_float2(mr.m[2 * n], mr.l[2 * n]);
+                    wml[8 * n + 2 * q4 + 1] = make_float2(mr.m[2 * n + 1], mr.l[2 * n + 1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mfull[0]);
+            if (!mbar_wait_bounded(&mfull[0], uc & 1, abort_flag, p.err, p.wait_ns)) {
+                dead = true;
+                break;
+            }
+            finish_unit_rows<T, D>(p, cur, macc, mml);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mfreed[0]);
+        } else {
         // ---- this warp's state into merge slot uc & 1, once the slot's previous
         // unit (uc - 2) has been merged by every warp
         const int b = uc & 1;
@@ -1042,6 +1405,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             __syncwarp();
             if (lane == 0) mbar_arrive(&mfreed[pb]);
         }
+        }
         prv = cur;
 
         // ---- advance: the fetch cursor moves down one unit with the window
@@ -1051,10 +1415,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         iss_u = iss_u > 0 ? iss_u - 1 : 0;
         u_nxt = unit_id(uc + 2);
         have_nxt = u_nxt < total;
-        if (have_nxt) load_unit(p, u_nxt, n_extra, cum, nxt, lane, warp == 0);
+        if (have_nxt) load_any(u_nxt, nxt);
     }
-    // the last unit's merge
-    if (!dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err, p.wait_ns))
+    // the last unit's merge (group-rows mode: done in the loop)
+    if (!kRows && !dead && mbar_wait_bounded(&mfull[uc & 1], (uc >> 1) & 1, abort_flag, p.err, p.wait_ns))
         finish_unit<T, D, G>(p, prv, macc + (size_t)(uc & 1) * kWarps * G * D, mml + (size_t)(uc & 1) * kWarps * G);
     cp_async_wait<0>();
     grid_dep_wait();
@@ -1063,21 +1427,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 // ------------------------------------------------------------- shared prefixes
 // Sequences next to each other in the batch whose tables start with the same
 // physical blocks (forks, a shared system prompt: chenxutan 2.1 / 3.3, devpress
-// 关键设计二) read those blocks once: the shared leading partitions are computed
+// 关键设计二) read those blocks once: the shared leading full blocks are computed
 // by group units (group, kv head) whose query rows are members x heads and whose
-// keys are all the group's shared partitions, and the per-sequence kernel starts
-// after them.  The result is the same sum -- the group partial lands in slot 0
-// of every member, the per-sequence units in the slots after it, and the LSE
+// keys are all the group's shared tokens, and the per-sequence units start after
+// them.  The result is the same sum -- the group partial lands in slot 0 of
+// every member, the per-sequence units in the slots after it, and the LSE
 // reduce combines them.
 //
-// Detection is one single-CTA kernel: each sequence's count of leading full
-// blocks shared with its predecessor, then the cut of the batch into groups.
-// The group units -- a dense (members x g) x partition x head_dim attention
-// each -- run on the tcgen05 tile kernel of prefill.cu (launch_group_tiles).
+// Detection (block 0 of group_detect_kernel): each sequence's count of leading
+// full blocks shared with its predecessor, then the cut of the batch into
+// groups.  The group units -- a dense (members x g) x shared tokens x head_dim
+// attention each -- run on the tcgen05 tile kernel of prefill.cu
+// (launch_group_tiles).
 
 constexpr int kDetectThreads = 1024;
 constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
-constexpr int kMaxGroupParts = (1 << 23) - 1;
+constexpr int kMaxGroupBlocks = (1 << 22) - 1;  // fits info's packing (nb << 9)
 // Groups of fewer members do not pay for the group unit's fixed cost (its rows
 // pad a 128-row tensor-core tile).
 constexpr int kMinGroupMembers = 4;
@@ -1165,13 +1530,17 @@ __device__ __forceinline__ int warp_exclusive_scan(int x, int identity) {
     return lane == 0 ? identity : exc;
 }
 
-// One CTA: all warps compare tables, then warp 0 forms the groups.  A run is a
-// maximal stretch of sequences each sharing at least one whole partition with
-// its predecessor; runs are cut into chunks of at most max_members sequences
-// counted from the run's start.  A chunk of n >= kMinGroupMembers sequences
-// shares min(lcp over its members after the first) blocks, i.e. np whole
-// partitions; it becomes one group with num_kv_heads units.  first_p[s] = np of
-// s's chunk (0 for a smaller chunk).
+// Block 0: all warps compare tables, then the groups are formed block-parallel.
+// A run is a maximal stretch of sequences each sharing at least part_tokens
+// tokens of full blocks with its predecessor.  A run of n sequences with
+// n x g <= 16 query rows stays whole; a longer run is cut into chunks of
+// max_members (128 / g) sequences counted from its start (kRowTile / g without
+// tile groups).  A chunk shares its nb = min(lcp over its members after the
+// first) leading blocks; it becomes a row group when 2 <= n and n x g <= 16
+// (one group-rows unit per kv head, on decode_kernel<T, D, kRowTile>), else a
+// tile group when n >= kMinGroupMembers (one tcgen05 tile unit per kv head);
+// each unit covers the 16 nb shared tokens.  first_t[s] = 16 nb of s's group (0
+// outside one).
 // The one-call step's cache write, done by blocks 1.. of the detection grid.
 struct StepWriteArgs {
     const uint4 *key;
@@ -1187,11 +1556,12 @@ struct StepWriteArgs {
 };
 
 __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __grid_constant__ Params p,
-                                                                      int32_t *first_p, int4 *groups,
+                                                                      int32_t *first_t, int4 *groups,
                                                                       int32_t *meta,
                                                                       const __grid_constant__ StepWriteArgs w) {
     __shared__ int lcp[kMaxGroupSeqs];
-    __shared__ int info[kMaxGroupSeqs];  // at a chunk head: its size, then np << 8 | size (size <= 128)
+    __shared__ int info[kMaxGroupSeqs];  // run sizes, then at a chunk head: its size, then
+                                         // nb << 9 | row group << 8 | size (size <= 128)
     grid_dep_launch();  // the group tiles set up while this runs, then wait for it
     if (blockIdx.x > 0) {
         // the step's new K/V (pa_append_decode): the tiles and the decode wait for
@@ -1233,17 +1603,31 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         __syncthreads();  // wtot is reused by the next scan
         return r;
     };
-    // run starts (a sequence sharing less than one whole partition with its
-    // predecessor), then each sequence's run start rs by a max-scan
+    // run starts (a sequence sharing fewer than part_tokens tokens of full blocks
+    // with its predecessor), then each sequence's run start rs by a max-scan
     int mx = -1;
     for (int s = s0; s < s1; ++s)
         if (s == 0 || lcp[s] < bpp) mx = s;
     int rs = block_scan(mx, -1, true);
-    int head_of[4];
+    int rs_of[4], head_of[4];
     for (int s = s0; s < s1; ++s) {
         if (s == 0 || lcp[s] < bpp) rs = s;
-        head_of[s - s0] = rs + ((s - rs) & ~(M - 1));  // chunks of M counted from the run's start
+        rs_of[s - s0] = rs;
+        if (rs == s) info[s] = 0;
     }
+    __syncthreads();
+    for (int s = s0; s < s1; ++s) atomicAdd(&info[rs_of[s - s0]], 1);  // run sizes
+    __syncthreads();
+    // A run whose rows (members x g) fit one group-rows unit stays whole; a longer
+    // one is cut, from its start, into chunks of M (tile groups) or, without tile
+    // groups, of kRowTile / g members.
+    const int g = p.num_q_heads / p.num_kv_heads;
+    const int chunk = p.tile_groups ? M : kRowTile / g;  // powers of two
+    for (int s = s0; s < s1; ++s) {
+        const int r0 = rs_of[s - s0];
+        head_of[s - s0] = info[r0] * g <= kRowTile ? r0 : r0 + ((s - r0) & ~(chunk - 1));
+    }
+    __syncthreads();  // run sizes read; info is reused below
     // chunk heads collect their size and the smallest shared length of the
     // members after them (a head's own lcp is no longer needed)
     for (int s = s0; s < s1; ++s)
@@ -1258,64 +1642,96 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         if (hd != s) atomicMin(&lcp[hd], lcp[s]);
     }
     __syncthreads();
-    int heads = 0;  // this thread's groups
+    // a chunk of n members is a row group when n x g <= kRowTile (n >= 2), else a
+    // tile group when n >= kMinGroupMembers; info = nb << 9 | row << 8 | n
+    int nt_heads = 0, nr_heads = 0;  // this thread's tile / row groups
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
         const int n = info[s], mn = lcp[s];
-        const int np = n >= kMinGroupMembers ? min(mn / bpp, kMaxGroupParts) : 0;
-        info[s] = (np << 8) | n;
-        if (np > 0) ++heads;
+        const bool row = n >= 2 && n * g <= kRowTile;
+        const bool tile = !row && p.tile_groups && n >= kMinGroupMembers;
+        const int nb = (row || tile) && mn >= bpp ? min(mn, kMaxGroupBlocks) : 0;
+        info[s] = (nb << 9) | ((row ? 1 : 0) << 8) | n;
+        if (nb > 0) {
+            if (row) ++nr_heads;
+            else ++nt_heads;
+        }
     }
-    const int g0 = block_scan(heads, 0, false);  // (the scan's barriers publish info)
-    // work estimate in (token, kv head) units: the group units' keys (measured on
-    // B200 to cost about 1.5 times a per-sequence key, their rows padding a
-    // 128-row tensor-core tile) against the per-sequence kernel's keys
-    __shared__ unsigned long long work[2];
-    if (threadIdx.x == 0) work[0] = work[1] = 0ull;
+    // both counts in one scan (each total <= 4096 fits 16 bits)
+    __shared__ int tot_groups;
+    const int mine = nt_heads + (nr_heads << 16);
+    const int ex = block_scan(mine, 0, false);  // (the scan's barriers publish info)
+    if (threadIdx.x == kDetectThreads - 1) tot_groups = ex + mine;
+    // work estimate in (token, kv head) units: group keys (measured on B200 to
+    // cost about 1.5 times a per-sequence key: a tile group's rows pad a 128-row
+    // tensor-core tile, a row group's 16 rows double the tiles of a block) against
+    // the per-sequence kernel's keys
+    __shared__ unsigned long long work[3];
+    if (threadIdx.x == 0) work[0] = work[1] = work[2] = 0ull;
     __syncthreads();
-    unsigned long long tw = 0, dw = 0;
+    const int n_tile = tot_groups & 0xffff, n_row = tot_groups >> 16;
+    unsigned long long tw = 0, rw = 0, dw = 0;
     for (int s = s0; s < s1; ++s) {
-        const int np = info[head_of[s - s0]] >> 8;
-        first_p[s] = np;
+        const int inf = info[head_of[s - s0]];
+        const int ft = (inf >> 9) * kBlockSize;
+        first_t[s] = ft;
         const int L = max(checked_len(p, s), 0);
-        dw += (unsigned long long)max(0, L - np * p.part_tokens);
-        if (head_of[s - s0] == s) tw += (unsigned long long)np * p.part_tokens;
+        dw += (unsigned long long)max(0, L - ft);
+        if (head_of[s - s0] == s) {
+            if ((inf >> 8) & 1) rw += (unsigned long long)ft;
+            else tw += (unsigned long long)ft;
+        }
     }
     // one shared-memory atomic per warp (1,024 on one word would serialise)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
         tw += __shfl_xor_sync(kFull, tw, o);
+        rw += __shfl_xor_sync(kFull, rw, o);
         dw += __shfl_xor_sync(kFull, dw, o);
     }
     if (lane == 0) {
         atomicAdd(&work[0], tw);
-        atomicAdd(&work[1], dw);
+        atomicAdd(&work[1], rw);
+        atomicAdd(&work[2], dw);
     }
-    int g = g0;
+    // records: tile groups first (the tile kernel reads groups[0, n_tile)), then
+    // the row groups
+    int gt = ex & 0xffff, gr = n_tile + (ex >> 16);
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
-        const int n = info[s] & 255, np = info[s] >> 8;
-        if (np > 0) {
-            groups[g] = make_int4(s, n, np, g * p.num_kv_heads);
-            ++g;
+        const int inf = info[s];
+        const int n = inf & 255, nb = inf >> 9;
+        if (nb == 0) continue;
+        if ((inf >> 8) & 1) {
+            groups[gr] = make_int4(s, n, nb * kBlockSize, (gr - n_tile) * p.num_kv_heads);
+            ++gr;
+        } else {
+            groups[gt] = make_int4(s, n, nb * kBlockSize, gt * p.num_kv_heads);
+            ++gt;
         }
     }
     __syncthreads();
-    if (threadIdx.x == kDetectThreads - 1) {  // its running count ends at the total
-        meta[0] = g;
-        meta[1] = g * p.num_kv_heads;
+    if (threadIdx.x == 0) {
+        meta[0] = n_tile;
+        meta[1] = n_tile * p.num_kv_heads;
         meta[2] = 0;   // the per-sequence kernel's work counter
         meta[3] = 0;   // the group tiles' work counter
-        // SMs for the group tiles, in proportion to their share of the work (the
-        // per-sequence kernel takes the rest), so that the two kernels end
-        // together; at least one per 2 group units (up to half the SMs), since a
-        // short unit's time is mostly latency
-        const double t = 1.5 * (double)work[0], d = (double)work[1];
+        meta[5] = n_row;
+        meta[6] = 0;   // the group-rows kernel's work counter
+        // SMs for the group tiles and the group rows, in proportion to their
+        // shares of the work (the per-sequence kernel takes the rest), so that the
+        // kernels end together; the tiles get at least one SM per 2 units (up to
+        // half the SMs), since a short tile unit's time is mostly latency
+        const double t = 1.5 * (double)work[0], r = 1.5 * (double)work[1], d = (double)work[2];
+        const double all = t + r + d + 1.0;
         const int sms = max(1, p.num_sms);
-        const int units = g * p.num_kv_heads;
-        int want = (int)ceil(sms * t / (t + d + 1.0));
-        want = max(want, min(sms / 2, (units + 1) / 2));
-        meta[4] = g == 0 ? 0 : min(sms, max(1, want));
+        int want_t = (int)ceil(sms * t / all);
+        want_t = max(want_t, min(sms / 2, (n_tile * p.num_kv_heads + 1) / 2));
+        want_t = n_tile == 0 ? 0 : min(sms, max(1, want_t));
+        int want_r = n_row == 0 ? 0 : max(1, (int)ceil(sms * r / all));
+        want_r = min(want_r, max(n_row == 0 ? 0 : 1, sms - want_t));
+        meta[4] = want_t;
+        meta[7] = want_r;
     }
 }
 
@@ -1355,9 +1771,9 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
     }
     int L = checked_len(p, s);
     if (L < 0) L = 0;
-    const int fp = first_part(p, s);
-    const int n = slot_base(fp) + seq_units(p, L, fp);  // slots written
-    if (fp == 0 && n <= 1) return;                       // finished by the decode kernel
+    const int ft = first_tok(p, s);
+    const int n = slot_base(ft) + seq_units(p, L, ft);  // slots written
+    if (ft == 0 && n <= 1) return;                       // finished by the decode kernel
     float M = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kPre; ++i)
@@ -1421,19 +1837,22 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
         const int want = (int64_t)a.num_seqs * a.cache.num_kv_heads < 4LL * sms ? 2048 : 1024;
         prm.seq_tokens = prm.part_tokens * std::max(1, want / prm.part_tokens);
     }
-    // shared-prefix groups: bf16, head_dim 128, split contexts.  Detection, the
-    // group tiles, this kernel and the combine follow one another with
-    // programmatic dependent launch (see the kernels for where each waits).
+    // shared-prefix groups: bf16 or fp8, head_dim 128, split contexts.  Detection,
+    // the group tiles (bf16 only), the group rows, this kernel and the combine
+    // follow one another with programmatic dependent launch (see the kernels for
+    // where each waits).
     bool grouped = false;
-    if constexpr (sizeof(T) == 2 && D == 128) {
+    if constexpr ((sizeof(T) == 2 || kIsFp8<T>) && D == 128) {
         if (split && a.ws_group && a.num_seqs <= kMaxGroupSeqs) {
             unsigned char *g = static_cast<unsigned char *>(a.ws_group);
-            // group area: first_p[S] (16-byte padded), groups[S], meta
+            // group area: first_t[S] (16-byte padded), groups[S], meta
             const size_t sa = ((size_t)a.num_seqs * 4 + 15) / 16 * 16;
-            prm.first_p = reinterpret_cast<int32_t *>(g);
+            prm.first_t = reinterpret_cast<int32_t *>(g);
             prm.groups = reinterpret_cast<int4 *>(g + sa);
             prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
+            constexpr bool kTiles = sizeof(T) == 2;  // the tcgen05 tile kernel reads bf16 pools
             prm.max_members = 128 / G;
+            prm.tile_groups = kTiles ? 1 : 0;
             StepWriteArgs wa;
             std::memset(&wa, 0, sizeof(wa));
             unsigned write_blocks = 0;
@@ -1454,38 +1873,53 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             }
             if (a.after_write) {
                 e = launch_after(group_detect_kernel, dim3(1 + write_blocks), dim3(kDetectThreads), 0, stream,
-                                 static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_p),
+                                 static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_t),
                                  const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta),
                                  static_cast<const StepWriteArgs &>(wa));
             } else {
                 group_detect_kernel<<<1 + write_blocks, kDetectThreads, 0, stream>>>(
-                    prm, const_cast<int32_t *>(prm.first_p), const_cast<int4 *>(prm.groups),
+                    prm, const_cast<int32_t *>(prm.first_t), const_cast<int4 *>(prm.groups),
                     const_cast<int32_t *>(prm.meta), wa);
                 e = cudaGetLastError();
             }
             if (e != cudaSuccess) return e;
-            GroupTileLaunch gl;
-            gl.query = a.query;
-            gl.num_seqs = a.num_seqs;
-            gl.key_cache = a.key_cache;
-            gl.value_cache = a.value_cache;
-            gl.block_tables = a.block_tables;
-            gl.max_blocks_per_seq = a.max_blocks_per_seq;
-            gl.groups = prm.groups;
-            gl.meta = prm.meta;
-            gl.ws_acc = prm.ws_acc;
-            gl.ws_ml = prm.ws_ml;
-            gl.num_q_heads = a.num_q_heads;
-            gl.num_kv_heads = a.cache.num_kv_heads;
-            gl.num_blocks = a.cache.num_blocks;
-            gl.partition_size = a.partition_size;
-            gl.max_partitions = a.max_partitions;
-            gl.scale = a.scale;
-            gl.err = a.err;
-            // The detection kernel picks how many SMs take the group units (ids drawn
-            // from a counter); the tile CTAs beyond that exit at once, and the
-            // per-sequence kernel starts on those SMs instead of waiting for them.
-            if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
+            if constexpr (kTiles) {
+                GroupTileLaunch gl;
+                gl.query = a.query;
+                gl.num_seqs = a.num_seqs;
+                gl.key_cache = a.key_cache;
+                gl.value_cache = a.value_cache;
+                gl.block_tables = a.block_tables;
+                gl.max_blocks_per_seq = a.max_blocks_per_seq;
+                gl.groups = prm.groups;
+                gl.meta = prm.meta;
+                gl.ws_acc = prm.ws_acc;
+                gl.ws_ml = prm.ws_ml;
+                gl.num_q_heads = a.num_q_heads;
+                gl.num_kv_heads = a.cache.num_kv_heads;
+                gl.num_blocks = a.cache.num_blocks;
+                gl.max_partitions = a.max_partitions;
+                gl.scale = a.scale;
+                gl.err = a.err;
+                // The detection kernel picks how many SMs take the group units (ids drawn
+                // from a counter); the tile CTAs beyond that exit at once, and the
+                // per-sequence kernel starts on those SMs instead of waiting for them.
+                if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
+            }
+            // Row groups (members x g <= 16 rows) on the group-rows mode of this
+            // kernel, launched behind the tiles the same way: its CTAs beyond the
+            // number the detection kernel chose leave at once.
+            using LayR = Layout<T, D, kRowTile>;
+            static_assert(LayR::smem_bytes(0) <= 232448, "group-rows smem over the sm_100 limit");
+            e = cudaFuncSetAttribute(decode_kernel<T, D, kRowTile>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)LayR::smem_bytes(0));
+            if (e != cudaSuccess) return e;
+            Params rp = prm;
+            rp.work_ctr = const_cast<int32_t *>(prm.meta) + 6;
+            rp.wait_first = kTiles ? 0 : 1;  // the tiles start only after the detection ends
+            e = launch_after(decode_kernel<T, D, kRowTile>, dim3((unsigned)sms), dim3(kThreads), LayR::smem_bytes(0),
+                             stream, static_cast<const Params &>(rp));
+            if (e != cudaSuccess) return e;
             grouped = true;
             prm.work_ctr = const_cast<int32_t *>(prm.meta) + 2;
         }

@@ -166,8 +166,10 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
 int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype, int32_t partition_size) {
     if (num_seqs <= 0) return 0;
     if (partition_size <= 0) return 1;
-    const bool grouped = dtype == PA_BF16 && head_dim == 128 && num_seqs <= kMaxSplitSeqs;
-    return grouped ? 4 : 2;
+    if (head_dim != 128 || num_seqs > kMaxSplitSeqs) return 2;
+    if (dtype == PA_BF16) return 5;       // detection, group tiles, group rows, decode, combine
+    if (dtype == PA_FP8_E4M3) return 4;   // no tile kernel for fp8 pools
+    return 2;
 }
 
 namespace {

@@ -103,8 +103,8 @@ cudaError_t launch_prefill(const PrefillLaunch &a, cudaStream_t stream);
 
 // Shared-prefix group units of a split bf16 / head_dim 128 decode, on the tcgen05
 // tile kernel: one unit per (group, kv head), rows = the group's members x g query
-// heads, keys = every partition the members share; it writes one partial (slot 0
-// of each member).  groups / meta are the decode's detection output (device memory).
+// heads, keys = the leading full blocks the members share; it writes one partial
+// (slot 0 of each member).  groups / meta are the decode's detection output (device memory).
 struct GroupTileLaunch {
     const void *query;       // [num_seqs, num_q_heads, 128] bf16
     int32_t num_seqs;
@@ -119,7 +119,6 @@ struct GroupTileLaunch {
     int32_t num_q_heads;
     int32_t num_kv_heads;
     int32_t num_blocks;
-    int32_t partition_size;
     int32_t max_partitions;
     float scale;
     int32_t *err;

@@ -120,11 +120,10 @@ struct Params {
     int32_t pairs;     // prefill: 256-row jobs per (sequence, kv head)
     float scale_log2;
     // shared-prefix group units of the split decode
-    const int4 *groups;    // (first seq, members, shared partitions, units before)
+    const int4 *groups;    // (first seq, members, shared tokens, units before)
     const int32_t *meta;   // [0] groups, [1] units, [3] work counter, [4] CTAs that take units
     float *ws_acc;
     float2 *ws_ml;
-    int32_t part_tokens;
     int32_t max_parts;
     unsigned long long wait_ns;  // bound of every in-kernel wait
 };
@@ -260,7 +259,7 @@ struct Job {
     int first, part;
 };
 
-// Group unit u's record (first seq, members, shared partitions, kv head), from
+// Group unit u's record (first seq, members, shared tokens, kv head), from
 // the group list copied to shared memory.
 __device__ __forceinline__ int4 group_record(int u, const int4 *sgroups, int ngroups) {
     int lo = 0, hi = ngroups;  // groups[lo].w <= u < groups[hi].w
@@ -268,7 +267,7 @@ __device__ __forceinline__ int4 group_record(int u, const int4 *sgroups, int ngr
         const int mid = (lo + hi) >> 1;
         if (sgroups[mid].w <= u) lo = mid; else hi = mid;
     }
-    const int4 gr = sgroups[lo];  // (first seq, members, shared partitions, units before)
+    const int4 gr = sgroups[lo];  // (first seq, members, shared tokens, units before)
     return make_int4(gr.x, gr.y, gr.z, u - gr.w);
 }
 
@@ -279,14 +278,14 @@ __device__ __forceinline__ bool make_job(const Params &p, int u, int4 rec, Job &
     if constexpr (kGroup) {
         const int4 gr = rec;
         jb.h = gr.w;                   // one unit per kv head
-        jb.part = 0;                   // workspace slot 0 holds the shared partitions' partial
+        jb.part = 0;                   // workspace slot 0 holds the shared tokens' partial
         jb.first = gr.x;
         jb.two = false;
         jb.nrows[0] = gr.y * G;
         jb.nrows[1] = 0;
         jb.qz[0] = jb.qz[1] = gr.x;
         jb.trow = p.tables + (int64_t)gr.x * p.max_blocks;
-        jb.nkeys = gr.z * p.part_tokens;
+        jb.nkeys = gr.z;               // the group's shared tokens (whole blocks)
         jb.lim0[0] = jb.lim0[1] = jb.nkeys - 1;
         jb.lim_step = 0;
         jb.ntiles = (jb.nkeys + kTileN - 1) / kTileN;
@@ -1035,7 +1034,6 @@ cudaError_t launch_group_tiles(const GroupTileLaunch &a, int sms, cudaStream_t s
     prm.meta = a.meta;
     prm.ws_acc = a.ws_acc;
     prm.ws_ml = a.ws_ml;
-    prm.part_tokens = a.partition_size;
     prm.max_parts = a.max_partitions;
     prm.wait_ns = wait_limit_ns();
     if (!encode_map(&prm.qmap, a.query, (uint64_t)a.num_q_heads, (uint64_t)a.num_seqs,

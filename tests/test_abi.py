@@ -108,7 +108,7 @@ def test_host_validation_launches_nothing(pa):
 
 def test_workspace_size_formula(pa):
     # partials: rows = S * Hq * ceil(maxctx / part), each head_dim fp32 + (m, l);
-    # then the shared-prefix group area: S int32 first partitions (16-byte
+    # then the shared-prefix group area: S int32 shared-token counts (16-byte
     # padded), S int4 group records, 32 bytes of counts.
     def a16(x):
         return (x + 15) // 16 * 16
@@ -128,8 +128,8 @@ def test_decode_launch_count(pa):
     assert pa.pa_decode_launches(8, 128, pa.PA_BF16, 0) == 1
     assert pa.pa_decode_launches(8, 128, pa.PA_F32, 512) == 2
     assert pa.pa_decode_launches(8, 64, pa.PA_BF16, 512) == 2
-    assert pa.pa_decode_launches(4096, 128, pa.PA_BF16, 512) == 4
-    assert pa.pa_decode_launches(4096, 128, pa.PA_FP8_E4M3, 512) == 2   # no shared-prefix groups
+    assert pa.pa_decode_launches(4096, 128, pa.PA_BF16, 512) == 5
+    assert pa.pa_decode_launches(4096, 128, pa.PA_FP8_E4M3, 512) == 4   # detection, group rows, decode, combine
     assert pa.pa_decode_launches(8, 128, pa.PA_FP8_E4M3, 0) == 1
 
 

@@ -207,20 +207,21 @@ def test_device_index_errors_are_flagged_not_fatal():
 
 def _grouped_workload(g=4):
     """Sibling structures the shared-prefix grouping must get right (g query heads
-    per kv head; a group takes at most 64 / g sequences)."""
+    per kv head): large families become tile groups of at most 128 / g members,
+    families with members x g <= 16 rows become row groups."""
     rng = np.random.default_rng(21)
     hkv, d = 4, 128
     hq = g * hkv
     # (parent tokens, [suffix lengths]) per family; forked parents end on a block
-    # boundary so that no sibling's first append needs a copy.  A group needs at
-    # least 4 members and takes at most 128 / g.
+    # boundary so that no sibling's first append needs a copy.  A tile group needs
+    # at least 4 members and takes at most 128 / g; a row group 2 to 16 / g.
     spec = []
     spec.append((1104, [int(x) for x in rng.integers(0, 300, size=20)]))   # 20 siblings
     spec.append((608, [5, 77, 130, 3, 9, 27, 81, 1, 40]))   # 9 siblings sharing 38 full blocks
     spec.append((208, [40, 41, 0, 7, 13, 90, 5, 60]))        # shares 13 blocks: < one 256-token partition
     spec.append((512, [0] * 8))                  # members entirely inside the shared prefix
     spec.append((333, []))                       # singleton (parent kept, partly filled last block)
-    spec.append((400, [3, 9, 27]))               # 3 siblings: too few to group
+    spec.append((400, [3, 9, 27]))               # 3 siblings: a row group for g <= 4, none for g = 8
     nb = 20 + sum(-(-(pt + max(sx, default=0) + 2) // 16) * (len(sx) + 1) for pt, sx in spec)
     wl = workloads.Workload(0, "groups", "bf16", nb, hq, hkv, d, 1.0 / np.sqrt(d),
                             rng.permutation(nb).astype(np.int32))
@@ -400,16 +401,19 @@ def ts_free_decode(pa, torch, q_np, gpu, t, l, scale, part):
     return to_host(out)
 
 
-def _expected_groups(tables, lens, part, g, hkv, min_members=4):
+def _expected_groups(tables, lens, part, g, hkv, min_members=4, tile_groups=True):
     """The shared-prefix grouping rule, written out on the host: lcp[s] = leading
     full blocks of s's table equal to those of s - 1; a run is a stretch of
-    sequences each sharing >= one whole partition with its predecessor; runs are
-    cut into chunks of 128 / g counted from the run's start; a chunk of >= 4
-    sequences shares min(lcp over its members after the first) // blocks per
-    partition whole partitions (np) and is a group when np > 0."""
+    sequences each sharing >= part tokens of full blocks with its predecessor; a
+    run of n sequences with n * g <= 16 stays whole, a longer one is cut into
+    chunks of 128 / g (16 / g without tile groups) counted from its start; a
+    chunk shares nb = min(lcp over its members after the first) blocks and is a
+    row group when 2 <= n and n * g <= 16, else a tile group when n >= 4.
+    Returns first_t (shared tokens per sequence), the tile groups' records, then
+    the row groups' records."""
     S = len(lens)
     bpp = part // 16
-    M = 128 // g
+    M = 128 // g if tile_groups else 16 // g
     lcp = [0] * S
     for s in range(1, S):
         n = min(int(lens[s]), int(lens[s - 1])) // 16
@@ -417,22 +421,33 @@ def _expected_groups(tables, lens, part, g, hkv, min_members=4):
         while k < n and tables[s, k] == tables[s - 1, k]:
             k += 1
         lcp[s] = k
-    first_p, groups = [0] * S, []
-    rs = 0
-    heads = {}
+    runs, rs = {}, 0
     for s in range(S):
         if s == 0 or lcp[s] < bpp:
             rs = s
-        heads.setdefault(rs + ((s - rs) // M) * M, []).append(s)
-    for hd in sorted(heads):
-        members = heads[hd]
-        n = len(members)
-        np_ = min(lcp[m] for m in members[1:]) // bpp if n >= min_members else 0
-        for m in members:
-            first_p[m] = np_
-        if np_ > 0:
-            groups.append((hd, n, np_, len(groups) * hkv))
-    return first_p, groups
+        runs.setdefault(rs, []).append(s)
+    chunks = []
+    for r0, mem in sorted(runs.items()):
+        if len(mem) * g <= 16:
+            chunks.append(mem)
+        else:
+            chunks += [mem[i:i + M] for i in range(0, len(mem), M)]
+    first_t, tiles, rows = [0] * S, [], []
+    for mem in chunks:
+        n = len(mem)
+        row = n >= 2 and n * g <= 16
+        tile = not row and tile_groups and n >= min_members
+        mn = min(lcp[m] for m in mem[1:]) if n > 1 else 0
+        nb = min(mn, (1 << 22) - 1) if (row or tile) and mn >= bpp else 0
+        if nb == 0:
+            continue
+        for m in mem:
+            first_t[m] = nb * 16
+        if row:
+            rows.append((mem[0], n, nb * 16, len(rows) * hkv))
+        else:
+            tiles.append((mem[0], n, nb * 16, len(tiles) * hkv))
+    return first_t, tiles, rows
 
 
 @pytest.mark.parametrize("cid,part", [(3, 512), (4, 512), (3, 64)])
@@ -458,18 +473,28 @@ def test_group_detection_matches_the_rule(cid, part):
     rows = S * wl.num_q_heads * parts
     at = -(-(rows * wl.head_dim * 4 + rows * 8) // 16) * 16
     raw = ws.cpu().numpy()
-    first_p = raw[at:at + 4 * S].view(np.int32)
+    first_t = raw[at:at + 4 * S].view(np.int32)
     gat = at + -(-4 * S // 16) * 16
     meta = raw[gat + 16 * S:gat + 16 * S + 32].view(np.int32)
-    want_fp, want_groups = _expected_groups(t, l, part, wl.num_q_heads // wl.num_kv_heads, wl.num_kv_heads)
-    assert first_p.tolist() == want_fp
-    assert meta[0] == len(want_groups) and meta[1] == len(want_groups) * wl.num_kv_heads
-    got_groups = raw[gat:gat + 16 * len(want_groups)].view(np.int32).reshape(-1, 4)
-    assert [tuple(int(x) for x in r) for r in got_groups] == want_groups
+    want_ft, want_tiles, want_rows = _expected_groups(t, l, part, wl.num_q_heads // wl.num_kv_heads,
+                                                      wl.num_kv_heads)
+    assert first_t.tolist() == want_ft
+    assert meta[0] == len(want_tiles) and meta[1] == len(want_tiles) * wl.num_kv_heads
+    assert meta[5] == len(want_rows)
+    n_g = len(want_tiles) + len(want_rows)
+    got = raw[gat:gat + 16 * n_g].view(np.int32).reshape(-1, 4)
+    assert [tuple(int(x) for x in r) for r in got] == want_tiles + want_rows
     sms = torch.cuda.get_device_properties(0).multi_processor_count
-    if want_groups:   # SMs the detection kernel gave the group tiles
+    if want_tiles:   # SMs the detection kernel gave the group tiles
         assert 1 <= meta[4] <= sms
     else:
         assert meta[4] == 0
+    if want_rows:    # and the group rows
+        assert 1 <= meta[7] <= sms
+    else:
+        assert meta[7] == 0
+    want_groups = want_tiles + want_rows
     if cid == 3:
         assert len(want_groups) > 0
+    if cid == 4:   # four forked siblings of g = 4: 16 query rows, one row group each
+        assert len(want_rows) > 0
