@@ -162,14 +162,14 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
 /*
  * Number of kernels one pa_decode call with these arguments launches on its
  * stream (for launch accounting and graph planning): 1 unsplit; 2 split (the
- * partition kernel and the combine); 5 split with dtype PA_BF16, head_dim 128 and
- * num_seqs <= 4096 (the shared-prefix detection kernel and the two group kernels,
- * tensor-core tiles for large groups and 16-row units for small ones, run
- * first); 4 for the same with PA_FP8_E4M3 (no tile kernel: every group takes
- * 16-row units).  0 when num_seqs <= 0.  Pure host function.
+ * partition kernel and the combine); with a split, dtype PA_BF16, head_dim 128 and
+ * num_seqs <= 4096 the shared-prefix detection kernel and the tcgen05 group tiles
+ * run first (4), and for g = num_q_heads / num_kv_heads <= 4 also the 16-row
+ * group kernel for small sibling groups (5).  0 when num_seqs <= 0 or the head
+ * counts are not positive.  Pure host function.
  */
-PA_API int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype,
-                                  int32_t partition_size);
+PA_API int32_t pa_decode_launches(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t dtype, int32_t partition_size);
 
 /*
  * Decode attention over the paged cache, one query token per sequence:
@@ -184,15 +184,16 @@ PA_API int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dt
  * l_p and unnormalised accumulator o_p in `workspace`, and a second kernel
  * combines them: out = sum_p e^{m_p - M} o_p / sum_p e^{m_p - M} l_p with
  * M = max_p m_p.  Sequences with a single partition are finished by the first
- * kernel.  With a split, bf16 or fp8 caches, head_dim 128 and num_seqs <= 4096, adjacent
+ * kernel.  With a split, bf16 caches, head_dim 128 and num_seqs <= 4096, adjacent
  * sequences whose block tables begin with the same block ids (forked siblings, a
  * common prompt; at least partition_size tokens of full blocks shared with the
  * previous sequence) read those shared full blocks once per group, with all the
- * group's queries against each K/V tile: groups of 2 to 16 / g members on
- * 16-row tensor-core tiles, larger ones (at least 4 members, at most 128 / g) on
- * the tcgen05 tile kernel (bf16; fp8 pools cut every run into 16-row groups).  The result is the same sum, and the shared blocks
- * cross the memory bus once instead of once per sibling (devpress teardown,
- * 关键设计二: siblings point at the same physical blocks).  workspace_bytes must be >= pa_decode_workspace_size(...) for the same
+ * group's queries against each K/V tile: for g = num_q_heads / num_kv_heads <= 4,
+ * groups of 2 to 16 / g members on 16-row tensor-core tiles; groups of at least 4
+ * members (at most 128 / g) on the tcgen05 tile kernel.  The result is the same
+ * sum, and the shared blocks cross the memory bus once instead of once per
+ * sibling (devpress teardown, 关键设计二: siblings point at the same physical
+ * blocks).  workspace_bytes must be >= pa_decode_workspace_size(...) for the same
  * num_seqs, num_q_heads, head_dim, max_context_len and partition_size.
  * max_context_len bounds every context_lens[s] (larger sets PA_DEVERR_CONTEXT_LEN
  * and that sequence's outputs are unspecified).  num_seqs <= 16384.

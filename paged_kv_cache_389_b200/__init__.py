@@ -49,7 +49,7 @@ def _load():
         "pa_copy_blocks": (C.c_int, [vp, vp, vp, i32, desc, vp, vp]),
         "pa_check_copy_pairs": (C.c_int, [vp, i32, i32]),
         "pa_decode_workspace_size": (sz, [i32, i32, i32, i32, i32]),
-        "pa_decode_launches": (i32, [i32, i32, i32, i32]),
+        "pa_decode_launches": (i32, [i32, i32, i32, i32, i32, i32]),
         "pa_decode": (C.c_int, [vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, i32, vp, sz, vp, desc,
                                 vp, vp]),
         "pa_append_decode": (C.c_int, [vp, vp, vp, i32, vp, vp, vp, vp, i32, vp, i32, i32, i32, f32, i32,
@@ -201,9 +201,9 @@ def pa_decode_workspace_size(num_seqs, num_q_heads, head_dim, max_context_len, p
                                              partition_size))
 
 
-def pa_decode_launches(num_seqs, head_dim, dtype, partition_size) -> int:
+def pa_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, dtype, partition_size) -> int:
     """Kernels one pa_decode call launches; dtype PA_F32 / PA_BF16 / PA_FP8_E4M3."""
-    return int(_lib.pa_decode_launches(num_seqs, head_dim, dtype, partition_size))
+    return int(_lib.pa_decode_launches(num_seqs, num_q_heads, num_kv_heads, head_dim, dtype, partition_size))
 
 
 def pa_decode(query, key_cache, value_cache, block_tables, context_lens, max_context_len, scale,

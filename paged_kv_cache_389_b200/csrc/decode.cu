@@ -173,7 +173,7 @@ struct Params {
                             // per-sequence and tile kernels, [4] tile CTAs, [5] row groups,
                             // [6] group-rows work counter, [7] group-rows CTAs
     int32_t max_members;    // sequences per tile group: query rows members x g <= 128
-    int32_t tile_groups;    // detection may form tile groups (bf16 pools); else row groups only
+    int32_t row_groups;     // detection may form row groups (the group-rows kernel runs)
     int32_t wait_first;     // launched right behind a cache write: wait for it first
     float v_scale;          // fp8 pools: value dequantisation scale (1 otherwise)
     unsigned long long wait_ns;  // bound of every in-kernel wait
@@ -645,19 +645,23 @@ __device__ __forceinline__ void mma_block_rows(uint32_t kb, unsigned char *vgen,
     auto addr = [&](uint32_t base, int row, int chunk) {
         return base + row * kRow + ((((chunk & ~7) | ((chunk ^ row) & 7))) << 4);
     };
+    // two accumulators per column tile (even / odd k steps) halve the MMA chains
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float s2[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     const int krow = ((mat & 1) << 3) + r8;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
         uint32_t a[4];
         ldsm_x4(a, addr(kb, krow, kk * 2 + (mat >> 1)));
-        mma_bf16_16816(s[0], a, st.qb[kk][0][0], st.qb[kk][0][1]);
-        mma_bf16_16816(s[1], a, st.qb[kk][1][0], st.qb[kk][1][1]);
+        float(&d0)[4] = (kk & 1) ? s2[0] : s[0];
+        float(&d1)[4] = (kk & 1) ? s2[1] : s[1];
+        mma_bf16_16816(d0, a, st.qb[kk][0][0], st.qb[kk][0][1]);
+        mma_bf16_16816(d1, a, st.qb[kk][1][0], st.qb[kk][1][1]);
     }
 #pragma unroll
     for (int n = 0; n < 2; ++n)
 #pragma unroll
-        for (int k = 0; k < 4; ++k) s[n][k] *= sl2;
+        for (int k = 0; k < 4; ++k) s[n][k] = (s[n][k] + s2[n][k]) * sl2;
     softmax_rows<D>(s, ntok, st, lane);
     // P^T operand fragments of both column tiles, transposed in registers
     uint32_t pb[2][2];
@@ -773,72 +777,6 @@ __device__ __forceinline__ void mma_tiles_fp8(unsigned char *const (&kb)[NT], co
             e4m3x4_to_f16x2x2(f23, a[2], a[3]);
             mma_f16_16816(st.o[2 * w + 1], a, pb0[b], pb1[b]);
         }
-    }
-}
-
-// Group-rows mode on an fp8 pool: one 16-token block against 16 query rows, with
-// the dim maps of mma_tiles_fp8 (each converted K or V fragment feeds both column
-// tiles).  kb: the block's stage (K slab, V slab behind it).
-template <int D>
-__device__ __forceinline__ void mma_block_rows_fp8(unsigned char *kb, int ntok, MmaRows<D> &st, float sl2,
-                                                   int lane) {
-    static_assert(D == 128, "the fp8 fragment map assumes 128-byte rows");
-    constexpr int kSlab = kBlockSize * D;
-    const int g = lane >> 2, t = lane & 3;
-    auto chunk = [&](const unsigned char *base, int row, int c) {
-        return *reinterpret_cast<const uint4 *>(base + row * D + ((c ^ (row & 7)) << 4));
-    };
-    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const uint4 lo = chunk(kb, g, 2 * t + j), hi = chunk(kb, g + 8, 2 * t + j);
-        const uint32_t wl[4] = {lo.x, lo.y, lo.z, lo.w}, wh[4] = {hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int kk = 4 * j + i;
-            uint32_t a[4];
-            e4m3x4_to_f16x2x2(wl[i], a[0], a[2]);
-            e4m3x4_to_f16x2x2(wh[i], a[1], a[3]);
-            mma_f16_16816(s[0], a, st.qb[kk][0][0], st.qb[kk][0][1]);
-            mma_f16_16816(s[1], a, st.qb[kk][1][0], st.qb[kk][1][1]);
-        }
-    }
-#pragma unroll
-    for (int n = 0; n < 2; ++n)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) s[n][k] *= sl2;
-    softmax_rows<D>(s, ntok, st, lane);
-    uint32_t pb[2][2];
-#pragma unroll
-    for (int n = 0; n < 2; ++n) {
-        pb[n][0] = movmatrix_trans(pack_f16x2(s[n][0], s[n][1]));
-        pb[n][1] = movmatrix_trans(pack_f16x2(s[n][2], s[n][3]));
-    }
-    unsigned char *vb = kb + kSlab;
-    if (ntok < kBlockSize) {
-        // codes past the keys may be NaN: zero those V rows
-        for (int idx = lane; idx < (kBlockSize - ntok) * (D / 16); idx += 32)
-            *reinterpret_cast<uint4 *>(vb + (ntok + idx / (D / 16)) * D + (idx % (D / 16)) * 16) =
-                make_uint4(0, 0, 0, 0);
-        __syncwarp();
-    }
-    const uint4 v0 = chunk(vb, 2 * t, g), v1 = chunk(vb, 2 * t + 1, g);
-    const uint4 v2 = chunk(vb, 2 * t + 8, g), v3 = chunk(vb, 2 * t + 9, g);
-    const uint32_t r0[4] = {v0.x, v0.y, v0.z, v0.w}, r1[4] = {v1.x, v1.y, v1.z, v1.w};
-    const uint32_t r2[4] = {v2.x, v2.y, v2.z, v2.w}, r3[4] = {v3.x, v3.y, v3.z, v3.w};
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const uint32_t e01 = __byte_perm(r0[w], r1[w], 0x5140), f01 = __byte_perm(r0[w], r1[w], 0x7362);
-        const uint32_t e23 = __byte_perm(r2[w], r3[w], 0x5140), f23 = __byte_perm(r2[w], r3[w], 0x7362);
-        uint32_t a[4];
-        e4m3x4_to_f16x2x2(e01, a[0], a[1]);
-        e4m3x4_to_f16x2x2(e23, a[2], a[3]);
-        mma_f16_16816(st.o[2 * w][0], a, pb[0][0], pb[0][1]);
-        mma_f16_16816(st.o[2 * w][1], a, pb[1][0], pb[1][1]);
-        e4m3x4_to_f16x2x2(f01, a[0], a[1]);
-        e4m3x4_to_f16x2x2(f23, a[2], a[3]);
-        mma_f16_16816(st.o[2 * w + 1][0], a, pb[0][0], pb[0][1]);
-        mma_f16_16816(st.o[2 * w + 1][1], a, pb[1][0], pb[1][1]);
     }
 }
 
@@ -988,22 +926,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
     constexpr bool kRows = Lay::kRows;
     static_assert(Lay::kMergeBufs == 2 || kRows, "the deferred merge needs two slots");
-    static_assert(!kRows || kMma, "group-rows mode runs on tensor-core tiles");
+    static_assert(!kRows || (kMma && !kFp8), "group-rows mode runs on bf16 tensor-core tiles");
     // The combine may start launching now; it waits for this grid to finish.
     // When launched behind the group tiles, this grid reads only what the
     // detection wrote (complete before the tiles let it start) and writes other
     // partitions; it waits for the tiles only before exiting, so that its
     // completion implies theirs.  Launched right behind a cache write instead
     // (pa_append_decode without groups), it waits for the write first.
-    if (kRows && p.wait_first) {
-        // group-rows mode right behind the detection (no tile kernel between): the
-        // next kernel reads the detection output, so it may launch only after it
-        grid_dep_wait();
-        grid_dep_launch();
-    } else {
-        grid_dep_launch();
-        if (p.wait_first) grid_dep_wait();
-    }
+    grid_dep_launch();
+    if (p.wait_first) grid_dep_wait();
     // Group-rows mode: the detection kernel chose how many CTAs take row-group
     // units (ids from the counter meta[6]); the others leave their SM at once.
     // CTA 0 always stays until the previous kernel of the call has finished, so
@@ -1177,28 +1108,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
                 const unsigned char *qr =
                     p.q + ((int64_t)(cur.un.s + r / g) * p.num_q_heads + (int64_t)cur.un.h * g + r % g) *
                               Lay::kQRowBytes;
-                if constexpr (kFp8) {
-                    // bf16 -> f16 in the k-slot map of mma_tiles_fp8, clamped to the f16 range
 #pragma unroll
-                    for (int j = 0; j < 2; ++j)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int d0 = 32 * q4 + 16 * j + 4 * i;
-                            uint2 x = make_uint2(0u, 0u);
-                            if (rv) x = __ldg(reinterpret_cast<const uint2 *>(qr + d0 * 2));
-                            const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.x));
-                            const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.y));
-                            auto c = [](float v) { return fminf(fmaxf(v, -65504.f), 65504.f); };
-                            mr.qb[4 * j + i][n][0] = pack_f16x2(c(a.x), c(a.y));
-                            mr.qb[4 * j + i][n][1] = pack_f16x2(c(b.x), c(b.y));
-                        }
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const int d0 = kk * 16 + 2 * q4;
-                        mr.qb[kk][n][0] = rv ? __ldg(reinterpret_cast<const uint32_t *>(qr + d0 * 2)) : 0u;
-                        mr.qb[kk][n][1] = rv ? __ldg(reinterpret_cast<const uint32_t *>(qr + (d0 + 8) * 2)) : 0u;
-                    }
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const int d0 = kk * 16 + 2 * q4;
+                    mr.qb[kk][n][0] = rv ? __ldg(reinterpret_cast<const uint32_t *>(qr + d0 * 2)) : 0u;
+                    mr.qb[kk][n][1] = rv ? __ldg(reinterpret_cast<const uint32_t *>(qr + (d0 + 8) * 2)) : 0u;
                 }
             }
 #pragma unroll
@@ -1297,9 +1211,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             const int stage = n_cmp % NS;
             if ((okmask >> stage) & 1u) {
                 const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
-                if constexpr (kRows && kFp8)
-                    mma_block_rows_fp8<D>(wring + stage * Lay::kStageBytes, ntok, mr, p.scale_log2, lane);
-                else if constexpr (kRows)
+                if constexpr (kRows)
                     mma_block_rows<D>(wring_s + stage * Lay::kStageBytes,
                                       wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, mr,
                                       p.scale_log2, lane);
@@ -1333,8 +1245,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             for (int mt = 0; mt < D / 16; ++mt)
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
-                    // accumulator row dr + 8 half of tile mt (fp8: the dim map of mma_tiles_fp8)
-                    const int d = kFp8 ? 16 * dr + 2 * mt + half : mt * 16 + dr + 8 * half;
+                    const int d = mt * 16 + dr + 8 * half;  // accumulator row dr + 8 half of tile mt
 #pragma unroll
                     for (int n = 0; n < 2; ++n) {
                         wacc[(8 * n + 2 * q4) * D + d] = mr.o[mt][n][2 * half];
@@ -1609,25 +1520,23 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     for (int s = s0; s < s1; ++s)
         if (s == 0 || lcp[s] < bpp) mx = s;
     int rs = block_scan(mx, -1, true);
-    int rs_of[4], head_of[4];
+    // With row groups, a run of at most K = kRowTile / g sequences (its rows fit
+    // one group-rows unit) stays whole: its next run start lies within K after its
+    // start.  Other runs are cut, from their start, into chunks of M.
+    const int g = p.num_q_heads / p.num_kv_heads;
+    const int K = kRowTile / g;
+    int head_of[4];
+    int short_rs = -1, short_ok = 0;  // the last run start tested, and its result
     for (int s = s0; s < s1; ++s) {
         if (s == 0 || lcp[s] < bpp) rs = s;
-        rs_of[s - s0] = rs;
-        if (rs == s) info[s] = 0;
+        if (p.row_groups && rs != short_rs) {
+            short_rs = rs;
+            short_ok = rs + K >= S;
+            for (int k = 1; k <= K && !short_ok; ++k) short_ok = lcp[rs + k] < bpp;
+        }
+        head_of[s - s0] = short_ok ? rs : rs + ((s - rs) & ~(M - 1));
     }
-    __syncthreads();
-    for (int s = s0; s < s1; ++s) atomicAdd(&info[rs_of[s - s0]], 1);  // run sizes
-    __syncthreads();
-    // A run whose rows (members x g) fit one group-rows unit stays whole; a longer
-    // one is cut, from its start, into chunks of M (tile groups) or, without tile
-    // groups, of kRowTile / g members.
-    const int g = p.num_q_heads / p.num_kv_heads;
-    const int chunk = p.tile_groups ? M : kRowTile / g;  // powers of two
-    for (int s = s0; s < s1; ++s) {
-        const int r0 = rs_of[s - s0];
-        head_of[s - s0] = info[r0] * g <= kRowTile ? r0 : r0 + ((s - r0) & ~(chunk - 1));
-    }
-    __syncthreads();  // run sizes read; info is reused below
+    __syncthreads();  // every lcp read; heads' entries are reset below
     // chunk heads collect their size and the smallest shared length of the
     // members after them (a head's own lcp is no longer needed)
     for (int s = s0; s < s1; ++s)
@@ -1648,8 +1557,8 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
         const int n = info[s], mn = lcp[s];
-        const bool row = n >= 2 && n * g <= kRowTile;
-        const bool tile = !row && p.tile_groups && n >= kMinGroupMembers;
+        const bool row = p.row_groups && n >= 2 && n * g <= kRowTile;
+        const bool tile = !row && n >= kMinGroupMembers;
         const int nb = (row || tile) && mn >= bpp ? min(mn, kMaxGroupBlocks) : 0;
         info[s] = (nb << 9) | ((row ? 1 : 0) << 8) | n;
         if (nb > 0) {
@@ -1721,8 +1630,12 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         // SMs for the group tiles and the group rows, in proportion to their
         // shares of the work (the per-sequence kernel takes the rest), so that the
         // kernels end together; the tiles get at least one SM per 2 units (up to
-        // half the SMs), since a short tile unit's time is mostly latency
-        const double t = 1.5 * (double)work[0], r = 1.5 * (double)work[1], d = (double)work[2];
+        // half the SMs), since a short tile unit's time is mostly latency.  A
+        // group-rows key costs about 1.7 per-sequence keys (measured on B200), and
+        // each of its units about 64 more for the meeting and merge at its end.
+        const double t = 1.5 * (double)work[0];
+        const double r = 1.7 * (double)work[1] + 64.0 * n_row * p.num_kv_heads;
+        const double d = (double)work[2];
         const double all = t + r + d + 1.0;
         const int sms = max(1, p.num_sms);
         int want_t = (int)ceil(sms * t / all);
@@ -1837,12 +1750,12 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
         const int want = (int64_t)a.num_seqs * a.cache.num_kv_heads < 4LL * sms ? 2048 : 1024;
         prm.seq_tokens = prm.part_tokens * std::max(1, want / prm.part_tokens);
     }
-    // shared-prefix groups: bf16 or fp8, head_dim 128, split contexts.  Detection,
-    // the group tiles (bf16 only), the group rows, this kernel and the combine
-    // follow one another with programmatic dependent launch (see the kernels for
-    // where each waits).
+    // shared-prefix groups: bf16, head_dim 128, split contexts.  Detection, the
+    // group tiles, the group rows (g <= 4), this kernel and the combine follow one
+    // another with programmatic dependent launch (see the kernels for where each
+    // waits).
     bool grouped = false;
-    if constexpr ((sizeof(T) == 2 || kIsFp8<T>) && D == 128) {
+    if constexpr (sizeof(T) == 2 && D == 128) {
         if (split && a.ws_group && a.num_seqs <= kMaxGroupSeqs) {
             unsigned char *g = static_cast<unsigned char *>(a.ws_group);
             // group area: first_t[S] (16-byte padded), groups[S], meta
@@ -1850,9 +1763,12 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             prm.first_t = reinterpret_cast<int32_t *>(g);
             prm.groups = reinterpret_cast<int4 *>(g + sa);
             prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
-            constexpr bool kTiles = sizeof(T) == 2;  // the tcgen05 tile kernel reads bf16 pools
+            // Row groups need 2 <= members <= 16 / g; at g = 8 only pairs qualify,
+            // whose gain does not pay for the extra launch, so the group-rows kernel
+            // runs for g <= 4 only.
+            constexpr bool kRowsLaunch = G <= 4;
             prm.max_members = 128 / G;
-            prm.tile_groups = kTiles ? 1 : 0;
+            prm.row_groups = kRowsLaunch ? 1 : 0;
             StepWriteArgs wa;
             std::memset(&wa, 0, sizeof(wa));
             unsigned write_blocks = 0;
@@ -1883,43 +1799,43 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
                 e = cudaGetLastError();
             }
             if (e != cudaSuccess) return e;
-            if constexpr (kTiles) {
-                GroupTileLaunch gl;
-                gl.query = a.query;
-                gl.num_seqs = a.num_seqs;
-                gl.key_cache = a.key_cache;
-                gl.value_cache = a.value_cache;
-                gl.block_tables = a.block_tables;
-                gl.max_blocks_per_seq = a.max_blocks_per_seq;
-                gl.groups = prm.groups;
-                gl.meta = prm.meta;
-                gl.ws_acc = prm.ws_acc;
-                gl.ws_ml = prm.ws_ml;
-                gl.num_q_heads = a.num_q_heads;
-                gl.num_kv_heads = a.cache.num_kv_heads;
-                gl.num_blocks = a.cache.num_blocks;
-                gl.max_partitions = a.max_partitions;
-                gl.scale = a.scale;
-                gl.err = a.err;
-                // The detection kernel picks how many SMs take the group units (ids drawn
-                // from a counter); the tile CTAs beyond that exit at once, and the
-                // per-sequence kernel starts on those SMs instead of waiting for them.
-                if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
-            }
+            GroupTileLaunch gl;
+            gl.query = a.query;
+            gl.num_seqs = a.num_seqs;
+            gl.key_cache = a.key_cache;
+            gl.value_cache = a.value_cache;
+            gl.block_tables = a.block_tables;
+            gl.max_blocks_per_seq = a.max_blocks_per_seq;
+            gl.groups = prm.groups;
+            gl.meta = prm.meta;
+            gl.ws_acc = prm.ws_acc;
+            gl.ws_ml = prm.ws_ml;
+            gl.num_q_heads = a.num_q_heads;
+            gl.num_kv_heads = a.cache.num_kv_heads;
+            gl.num_blocks = a.cache.num_blocks;
+            gl.max_partitions = a.max_partitions;
+            gl.scale = a.scale;
+            gl.err = a.err;
+            // The detection kernel picks how many SMs take the group units (ids drawn
+            // from a counter); the tile CTAs beyond that exit at once, and the
+            // per-sequence kernel starts on those SMs instead of waiting for them.
+            if ((e = launch_group_tiles(gl, sms, stream)) != cudaSuccess) return e;
             // Row groups (members x g <= 16 rows) on the group-rows mode of this
             // kernel, launched behind the tiles the same way: its CTAs beyond the
             // number the detection kernel chose leave at once.
-            using LayR = Layout<T, D, kRowTile>;
-            static_assert(LayR::smem_bytes(0) <= 232448, "group-rows smem over the sm_100 limit");
-            e = cudaFuncSetAttribute(decode_kernel<T, D, kRowTile>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)LayR::smem_bytes(0));
-            if (e != cudaSuccess) return e;
-            Params rp = prm;
-            rp.work_ctr = const_cast<int32_t *>(prm.meta) + 6;
-            rp.wait_first = kTiles ? 0 : 1;  // the tiles start only after the detection ends
-            e = launch_after(decode_kernel<T, D, kRowTile>, dim3((unsigned)sms), dim3(kThreads), LayR::smem_bytes(0),
-                             stream, static_cast<const Params &>(rp));
-            if (e != cudaSuccess) return e;
+            if constexpr (kRowsLaunch) {
+                using LayR = Layout<T, D, kRowTile>;
+                static_assert(LayR::smem_bytes(0) <= 232448, "group-rows smem over the sm_100 limit");
+                e = cudaFuncSetAttribute(decode_kernel<T, D, kRowTile>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)LayR::smem_bytes(0));
+                if (e != cudaSuccess) return e;
+                Params rp = prm;
+                rp.work_ctr = const_cast<int32_t *>(prm.meta) + 6;
+                rp.wait_first = 0;  // the tiles start only after the detection ends
+                e = launch_after(decode_kernel<T, D, kRowTile>, dim3((unsigned)sms), dim3(kThreads), LayR::smem_bytes(0),
+                                 stream, static_cast<const Params &>(rp));
+                if (e != cudaSuccess) return e;
+            }
             grouped = true;
             prm.work_ctr = const_cast<int32_t *>(prm.meta) + 2;
         }

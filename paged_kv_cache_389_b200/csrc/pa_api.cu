@@ -65,7 +65,7 @@ using namespace pa;
 
 extern "C" {
 
-int32_t pa_abi_version(void) { return 2; }
+int32_t pa_abi_version(void) { return 3; }
 
 uint64_t pa_set_wait_timeout_ns(uint64_t ns) {
     if (ns == 0) ns = kWaitTimeoutNs;
@@ -163,13 +163,13 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
     return (size_t)((partials + 15) / 16 * 16 + group);
 }
 
-int32_t pa_decode_launches(int32_t num_seqs, int32_t head_dim, int32_t dtype, int32_t partition_size) {
-    if (num_seqs <= 0) return 0;
+int32_t pa_decode_launches(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t dtype, int32_t partition_size) {
+    if (num_seqs <= 0 || num_q_heads <= 0 || num_kv_heads <= 0) return 0;
     if (partition_size <= 0) return 1;
-    if (head_dim != 128 || num_seqs > kMaxSplitSeqs) return 2;
-    if (dtype == PA_BF16) return 5;       // detection, group tiles, group rows, decode, combine
-    if (dtype == PA_FP8_E4M3) return 4;   // no tile kernel for fp8 pools
-    return 2;
+    if (head_dim != 128 || num_seqs > kMaxSplitSeqs || dtype != PA_BF16) return 2;
+    // detection, group tiles, [group rows: g <= 4], decode, combine
+    return num_q_heads / num_kv_heads <= 4 ? 5 : 4;
 }
 
 namespace {

@@ -23,7 +23,7 @@
     } while (0)
 
 int main(void) {
-    CHECK(1, pa_abi_version() == 2);
+    CHECK(1, pa_abi_version() == 3);
     CHECK(2, strcmp(pa_status_string(PA_OK), "ok") == 0);
 
     /* host validation of a device call: an unsupported block size fails first */
@@ -35,7 +35,7 @@ int main(void) {
     CHECK(4, pa_cache_write(fake, fake, (const int64_t *)fake, 1, fake, fake, &fp8, NULL, NULL) ==
                  PA_ERR_INVALID_ARG);
     CHECK(5, pa_decode_workspace_size(3, 4, 64, 100, 0) == 0);
-    CHECK(6, pa_decode_launches(8, 128, PA_BF16, 0) == 1);
+    CHECK(6, pa_decode_launches(8, 32, 8, 128, PA_BF16, 0) == 1);
 
     /* copy pairs: one source may feed several destinations; a repeated dst may not */
     const int32_t ok_pairs[] = {0, 1, 0, 2, 5, 4};

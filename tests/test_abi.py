@@ -42,7 +42,7 @@ def test_only_the_abi_is_exported(pa):
 
 
 def test_version_and_status_strings(pa):
-    assert pa.abi_version() == 2
+    assert pa.abi_version() == 3
     assert pa.status_string(pa.PA_OK) == "ok"
     assert "out of" in pa.status_string(pa.PA_ERR_OOM)
     assert pa.status_string(99) == "unknown status"
@@ -124,13 +124,17 @@ def test_workspace_size_formula(pa):
 
 
 def test_decode_launch_count(pa):
-    assert pa.pa_decode_launches(0, 128, pa.PA_BF16, 512) == 0
-    assert pa.pa_decode_launches(8, 128, pa.PA_BF16, 0) == 1
-    assert pa.pa_decode_launches(8, 128, pa.PA_F32, 512) == 2
-    assert pa.pa_decode_launches(8, 64, pa.PA_BF16, 512) == 2
-    assert pa.pa_decode_launches(4096, 128, pa.PA_BF16, 512) == 5
-    assert pa.pa_decode_launches(4096, 128, pa.PA_FP8_E4M3, 512) == 4   # detection, group rows, decode, combine
-    assert pa.pa_decode_launches(8, 128, pa.PA_FP8_E4M3, 0) == 1
+    L = pa.pa_decode_launches
+    assert L(0, 32, 8, 128, pa.PA_BF16, 512) == 0
+    assert L(8, 0, 8, 128, pa.PA_BF16, 512) == 0
+    assert L(8, 32, 8, 128, pa.PA_BF16, 0) == 1
+    assert L(8, 32, 8, 128, pa.PA_F32, 512) == 2
+    assert L(8, 32, 8, 64, pa.PA_BF16, 512) == 2
+    assert L(4096, 32, 8, 128, pa.PA_BF16, 512) == 5    # detection, tiles, group rows, decode, combine
+    assert L(4096, 64, 8, 128, pa.PA_BF16, 512) == 4    # g = 8: no group rows
+    assert L(4097, 32, 8, 128, pa.PA_BF16, 512) == 2
+    assert L(4096, 32, 8, 128, pa.PA_FP8_E4M3, 512) == 2   # no shared-prefix path for fp8 pools
+    assert L(8, 32, 8, 128, pa.PA_FP8_E4M3, 0) == 1
 
 
 

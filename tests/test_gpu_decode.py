@@ -401,19 +401,20 @@ def ts_free_decode(pa, torch, q_np, gpu, t, l, scale, part):
     return to_host(out)
 
 
-def _expected_groups(tables, lens, part, g, hkv, min_members=4, tile_groups=True):
+def _expected_groups(tables, lens, part, g, hkv, min_members=4):
     """The shared-prefix grouping rule, written out on the host: lcp[s] = leading
     full blocks of s's table equal to those of s - 1; a run is a stretch of
-    sequences each sharing >= part tokens of full blocks with its predecessor; a
-    run of n sequences with n * g <= 16 stays whole, a longer one is cut into
-    chunks of 128 / g (16 / g without tile groups) counted from its start; a
-    chunk shares nb = min(lcp over its members after the first) blocks and is a
-    row group when 2 <= n and n * g <= 16, else a tile group when n >= 4.
-    Returns first_t (shared tokens per sequence), the tile groups' records, then
-    the row groups' records."""
+    sequences each sharing >= part tokens of full blocks with its predecessor.
+    With row groups (g <= 4) a run of n sequences with n * g <= 16 stays whole;
+    other runs are cut into chunks of 128 / g counted from their start.  A chunk
+    shares nb = min(lcp over its members after the first) blocks and is a row
+    group when row groups are on, 2 <= n and n * g <= 16, else a tile group when
+    n >= 4.  Returns first_t (shared tokens per sequence), the tile groups'
+    records, then the row groups' records."""
     S = len(lens)
     bpp = part // 16
-    M = 128 // g if tile_groups else 16 // g
+    M = 128 // g
+    row_groups = g <= 4
     lcp = [0] * S
     for s in range(1, S):
         n = min(int(lens[s]), int(lens[s - 1])) // 16
@@ -428,15 +429,15 @@ def _expected_groups(tables, lens, part, g, hkv, min_members=4, tile_groups=True
         runs.setdefault(rs, []).append(s)
     chunks = []
     for r0, mem in sorted(runs.items()):
-        if len(mem) * g <= 16:
+        if row_groups and len(mem) * g <= 16:
             chunks.append(mem)
         else:
             chunks += [mem[i:i + M] for i in range(0, len(mem), M)]
     first_t, tiles, rows = [0] * S, [], []
     for mem in chunks:
         n = len(mem)
-        row = n >= 2 and n * g <= 16
-        tile = not row and tile_groups and n >= min_members
+        row = row_groups and n >= 2 and n * g <= 16
+        tile = not row and n >= min_members
         mn = min(lcp[m] for m in mem[1:]) if n > 1 else 0
         nb = min(mn, (1 << 22) - 1) if (row or tile) and mn >= bpp else 0
         if nb == 0:

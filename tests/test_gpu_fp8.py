@@ -93,6 +93,23 @@ def test_fp8_fork_copy_on_write():
     assert ts.model.num_free() == ts.gpu.manager.num_free()
 
 
+@pytest.mark.parametrize("g", [1, 2, 4, 8])
+def test_fp8_sibling_families_match_oracle(g):
+    """The sibling families of the bf16 grouping test on fp8 pools (no grouping:
+    every sequence reads its shared blocks itself), at several partitions, against
+    the oracle over the same codes."""
+    from test_gpu_decode import _grouped_workload
+    wl = _grouped_workload(g)
+    ts = TwoSided(wl, (K_SCALE, V_SCALE))
+    step = wl.steps[0]
+    ts.append_step(step)
+    assert ts.pools_equal()
+    ref = ts.oracle_decode(step)
+    for part in (0, 48, 256, 512, 1024):
+        check_close(ts.gpu_decode(step, part), ref, "bf16", f"fp8 g{g} grouped decode partition {part}")
+    assert ts.err_flag() == 0
+
+
 def _custom(lens, hq, hkv, seed=5):
     rng = np.random.default_rng(seed)
     need = sum(-(-L // 16) for L in lens) + 4
