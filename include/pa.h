@@ -49,6 +49,17 @@
  *     affected outputs are then unspecified.  Read the flag with pa_wait().
  *   - Every wait inside a kernel is bounded; a wait that runs out sets
  *     PA_DEVERR_TIMEOUT and the kernel returns early.
+ *   - Programmatic dependent launch: the kernels of a call are chained with it,
+ *     and the last kernel of a split decode signals early that a dependent may
+ *     launch.  A kernel the caller launches right after a call, with
+ *     cudaLaunchAttributeProgrammaticStreamSerialization, must call
+ *     cudaGridDependencySynchronize() before it reads the call's outputs (stream
+ *     order is unchanged for every other kernel and for copies).  The first
+ *     kernel of a split bf16 decode is itself launched that way: until the
+ *     kernel before it has finished it only reads block_tables and context_lens,
+ *     so the kernel just before the call must not write those two after it has
+ *     called cudaTriggerProgrammaticLaunchCompletion() (kernels that never call
+ *     it count as finished before the call starts).
  */
 #ifndef PA_H_
 #define PA_H_

@@ -1473,10 +1473,15 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     __shared__ int lcp[kMaxGroupSeqs];
     __shared__ int info[kMaxGroupSeqs];  // run sizes, then at a chunk head: its size, then
                                          // nb << 9 | row group << 8 | size (size <= 128)
+    // Launched with programmatic serialization: this grid may start while the
+    // kernel before it in the stream (the previous call's combine, say) is still
+    // running.  Until grid_dep_wait() it only reads the block tables and lengths
+    // (inputs no kernel of this library writes); every write comes after it.
     grid_dep_launch();  // the group tiles set up while this runs, then wait for it
     if (blockIdx.x > 0) {
         // the step's new K/V (pa_append_decode): the tiles and the decode wait for
         // this whole grid, so they see it; detection reads no cache bytes
+        grid_dep_wait();
         for (int64_t i = (int64_t)(blockIdx.x - 1) * kDetectThreads + threadIdx.x; i < w.chunks;
              i += (int64_t)(gridDim.x - 1) * kDetectThreads)
             write_chunk(i, w.key, w.value, w.slot_mapping, w.num_tokens, w.key_cache, w.value_cache,
@@ -1486,9 +1491,10 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     const int S = p.num_seqs;
     shared_prefix_lengths(p, lcp);
     __syncthreads();
-    // Behind a cache write (pa_append_decode) this kernel neither reads nor writes
-    // the cache, so it runs alongside the write, but it finishes only after it:
-    // the group tiles wait for this kernel and so see the new tokens' K/V.
+    // The previous kernel must be complete before this grid writes anything.  Behind
+    // a cache write (pa_decode after pa_cache_write) this also means: this kernel
+    // finishes only after the write, and the group tiles, which wait for this
+    // kernel, see the new tokens' K/V.
     grid_dep_wait();
     // Every thread owns a contiguous run of at most 4 sequences [s0, s1).
     __shared__ int wtot[kDetectThreads / 32];
@@ -1655,7 +1661,8 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
 // round trip after the decode ends.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Params p) {
-    grid_dep_wait();  // every partial is written
+    grid_dep_launch();  // the next call's detection may start reading its tables
+    grid_dep_wait();    // every partial is written
     constexpr int kDpl = D / 32;
     constexpr int kPre = 4;
     const int lane = threadIdx.x & 31;
@@ -1787,17 +1794,12 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
                 write_blocks = (unsigned)std::min<int64_t>((wa.chunks + kDetectThreads - 1) / kDetectThreads,
                                                            4 * sms);
             }
-            if (a.after_write) {
-                e = launch_after(group_detect_kernel, dim3(1 + write_blocks), dim3(kDetectThreads), 0, stream,
-                                 static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_t),
-                                 const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta),
-                                 static_cast<const StepWriteArgs &>(wa));
-            } else {
-                group_detect_kernel<<<1 + write_blocks, kDetectThreads, 0, stream>>>(
-                    prm, const_cast<int32_t *>(prm.first_t), const_cast<int4 *>(prm.groups),
-                    const_cast<int32_t *>(prm.meta), wa);
-                e = cudaGetLastError();
-            }
+            // always with programmatic serialization: its table comparison may
+            // overlap the end of whatever kernel precedes it (see the kernel)
+            e = launch_after(group_detect_kernel, dim3(1 + write_blocks), dim3(kDetectThreads), 0, stream,
+                             static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_t),
+                             const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta),
+                             static_cast<const StepWriteArgs &>(wa));
             if (e != cudaSuccess) return e;
             GroupTileLaunch gl;
             gl.query = a.query;
