@@ -183,7 +183,7 @@ TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "decode_gqa8b_prefix_traffic.jso
 def kernel_sources_sha256():
     """sha256 of every kernel source that one pa_append_decode call runs."""
     out = {}
-    for name in ("cache_ops.cu", "decode.cu", "prefill.cu", "pa_common.cuh"):
+    for name in ("cache_ops.cu", "cache_write.cuh", "decode.cu", "prefill.cu", "pa_common.cuh"):
         src = os.path.join(ROOT, "paged_kv_cache_389_b200", "csrc", name)
         out[name] = hashlib.sha256(open(src, "rb").read()).hexdigest()
     return out
@@ -440,7 +440,7 @@ def run_ours(args):
             "pct_of_measured_hbm": round(100 * value / world / peak, 2),
             "logical_gbs": round(world * (logical_b + cw_b) * K / (ms_max * 1e-3) / 1e9, 2),
             "bytes_per_step": {"decode_unique": unique_b, "decode_logical": logical_b, "cache_write": cw_b},
-            "roofline": {"bound": "hbm", "kernel": "pa_append_decode call (cache write fused with group detection, tcgen05 group tiles, decode_kernel, lse reduce)",
+            "roofline": {"bound": "hbm", "kernel": "pa_append_decode call (cache write fused with group detection, tcgen05 group tiles, 16-row group units, decode_kernel, lse reduce)",
                          "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4),
                          "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)" if peaks else "fallback",

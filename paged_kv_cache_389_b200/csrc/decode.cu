@@ -1476,7 +1476,8 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     // Launched with programmatic serialization: this grid may start while the
     // kernel before it in the stream (the previous call's combine, say) is still
     // running.  Until grid_dep_wait() it only reads the block tables and lengths
-    // (inputs no kernel of this library writes); every write comes after it.
+    // (inputs no kernel of this library writes) and works in shared memory (the
+    // whole grouping); every global write comes after it.
     grid_dep_launch();  // the group tiles set up while this runs, then wait for it
     if (blockIdx.x > 0) {
         // the step's new K/V (pa_append_decode): the tiles and the decode wait for
@@ -1491,11 +1492,6 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     const int S = p.num_seqs;
     shared_prefix_lengths(p, lcp);
     __syncthreads();
-    // The previous kernel must be complete before this grid writes anything.  Behind
-    // a cache write (pa_decode after pa_cache_write) this also means: this kernel
-    // finishes only after the write, and the group tiles, which wait for this
-    // kernel, see the new tokens' K/V.
-    grid_dep_wait();
     // Every thread owns a contiguous run of at most 4 sequences [s0, s1).
     __shared__ int wtot[kDetectThreads / 32];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -1503,6 +1499,11 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     const int M = p.max_members;  // 128 / g: a power of two
     const int per = (S + kDetectThreads - 1) / kDetectThreads;
     const int s0 = min(S, (int)threadIdx.x * per), s1 = min(S, s0 + per);
+    // this thread's context lengths, loaded now for the work estimate at the end
+    // (their latency hides behind the grouping's scans)
+    int len_of[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) len_of[i] = s0 + i < s1 ? __ldg(p.lens + s0 + i) : 0;
     // block-wide exclusive scan of one value per thread (sum, or max when kMax)
     auto block_scan = [&](int x, int identity, bool is_max) -> int {
         const int wex = is_max ? warp_exclusive_scan<true>(x, identity) : warp_exclusive_scan<false>(x, identity);
@@ -1585,12 +1586,18 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     if (threadIdx.x == 0) work[0] = work[1] = work[2] = 0ull;
     __syncthreads();
     const int n_tile = tot_groups & 0xffff, n_row = tot_groups >> 16;
+    // Everything so far ran in shared memory and registers.  The previous kernel
+    // must be complete before this grid writes anything; behind a cache write
+    // (pa_decode after pa_cache_write) this also means that this kernel finishes
+    // only after the write, and the group tiles, which wait for this kernel, see
+    // the new tokens' K/V.
+    grid_dep_wait();
     unsigned long long tw = 0, rw = 0, dw = 0;
     for (int s = s0; s < s1; ++s) {
         const int inf = info[head_of[s - s0]];
         const int ft = (inf >> 9) * kBlockSize;
         first_t[s] = ft;
-        const int L = max(checked_len(p, s), 0);
+        const int L = max(check_len(p, len_of[s - s0]), 0);
         dw += (unsigned long long)max(0, L - ft);
         if (head_of[s - s0] == s) {
             if ((inf >> 8) & 1) rw += (unsigned long long)ft;
