@@ -106,6 +106,9 @@ constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
 // the members x g query heads of a small sibling group, two 8-column tensor-core
 // tiles.
 constexpr int kRowTile = 16;
+// Longest private tail (blocks past the shared ones) a group-rows unit takes per
+// member, so that its members need no per-sequence unit.
+constexpr int kTailBlocks = 4;
 constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Shared-memory carve-up (byte offsets from the dynamic shared memory base).
@@ -125,7 +128,10 @@ struct Layout {
     static constexpr size_t kLimit = 232448;                    // sm_100 max dynamic smem per CTA
     static constexpr size_t kPBytes = sizeof(T) == 4 ? (size_t)kWarps * (16 * G + G) * 4 : 64;
     static constexpr size_t kMergeBytes = (size_t)kWarps * G * (D * 4 + 8);
-    static constexpr size_t kFixed = kPBytes + 16 + 48 + 96 + (kRows ? 0 : (size_t)(kMaxSplitSeqs + 1) * 4) + 64;
+    // prefix sums of the split path: the extra units per sequence, and on the
+    // shared-prefix path (bf16, head_dim 128) also the first units
+    static constexpr int kCumArrays = kRows ? 0 : (sizeof(T) == 2 && D == 128 ? 2 : 1);
+    static constexpr size_t kFixed = kPBytes + 16 + 48 + 96 + (size_t)kCumArrays * (kMaxSplitSeqs + 1) * 4 + 64;
     static constexpr int stages_fit(int bufs) {
         return (int)((kLimit - kFixed - bufs * kMergeBytes) / ((size_t)kWarps * kStageBytes));
     }
@@ -165,10 +171,12 @@ struct Params {
     int32_t seq_tokens;   // split: tokens per per-sequence unit (a multiple of part_tokens)
     float scale_log2;
     // shared-prefix groups (split contexts only; nullptr = none): first_t[s] is the
-    // number of leading tokens of s computed by its group's unit (a multiple of 16,
-    // at least part_tokens; 0 outside a group)
+    // number of leading tokens of s computed by its group's unit (the shared full
+    // blocks, at least part_tokens; all of s when the group-rows unit also takes
+    // the members' tails; 0 outside a group)
     const int32_t *first_t;
-    const int4 *groups;     // (first seq, members, shared tokens, units before)
+    const int4 *groups;     // (first seq, members, shared tokens, units before: tile groups;
+                            //  1 when the unit takes the members' tails: row groups)
     const int32_t *meta;    // [0] tile groups, [1] their units, [2] / [3] work counters of the
                             // per-sequence and tile kernels, [4] tile CTAs, [5] row groups,
                             // [6] group-rows work counter, [7] group-rows CTAs
@@ -220,14 +228,25 @@ __device__ __forceinline__ int first_tok(const Params &p, int s) {
 // Unit u -> (sequence, slot, kv head).  Units [0, n_extra) are the further
 // units of long sequences (slots after their first unit's), sequence-major, kv
 // head innermost, using cum[s] = sum_{s' < s} (seq_units(s') - 1)^+; after them
-// comes the first per-sequence unit of every sequence (slot slot_base(ft)).  The
-// further units are all full-length, so putting them first leaves the shorter
-// first units for the end of the queue, where they even out the CTAs' finish.
+// comes the first per-sequence unit (slot slot_base(ft)) of every sequence that
+// has one, using cum[S + 1 + s] (their count before s).  The further units are
+// all full-length, so putting them first leaves the shorter first units for the
+// end of the queue, where they even out the CTAs' finish.
 __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t n_extra, int hkv,
                                         const int *cum, int S) {
     if (u >= n_extra) {
         const int64_t f = u - n_extra;
-        const int s = (int)(f / hkv);
+        const int fi = (int)(f / hkv);
+        int s = fi;  // identity when every sequence has a first unit
+        if (p.first_t != nullptr && cum[2 * S + 1] != S) {
+            const int *cumf = cum + S + 1;
+            int lo = 0, hi = S;  // cumf[lo] <= fi < cumf[hi]
+            while (hi - lo > 1) {
+                const int mid = (lo + hi) >> 1;
+                if (cumf[mid] <= fi) lo = mid; else hi = mid;
+            }
+            s = lo;
+        }
         const int ft = first_tok(p, s);
         return Unit{s, slot_base(ft), (int)(f % hkv), ft};
     }
@@ -254,19 +273,27 @@ struct WarpUnit {
     const int32_t *trow;
     bool skip;  // partition past the end (every partition was covered by a group unit)
     int nrow;   // group-rows mode: query rows in use (members x g)
+    int nsh;    // group-rows mode: shared blocks (items [0, nsh)); items after them are the
+                // members' tails, kTailBlocks slots per member (empty past a member's tail)
+    int mlen;   // group-rows mode with tails: lane m holds member m's context length
 };
+
+// A tail slot past its member's tail: no block to load (not an error).
+constexpr int kEmptyItem = -2;
 
 // Group-rows mode: unit v = (row group v / Hkv, kv head v % Hkv).  Its keys are
 // the group's shared tokens (whole blocks of the first member's table); its rows
 // are members x g query heads, member-major.
 __device__ __forceinline__ void load_unit_rows(const Params &p, int64_t v, int gbase, WarpUnit &w, int lane) {
     const int hkv = p.num_kv_heads;
-    const int4 gr = __ldg(p.groups + gbase + (int)(v / hkv));  // (first seq, members, shared tokens, -)
+    const int4 gr = __ldg(p.groups + gbase + (int)(v / hkv));  // (first seq, members, shared tokens, tails)
     w.un = Unit{gr.x, 0, (int)(v % hkv), gr.z};
     w.L = gr.z;
     w.t0 = 0;
     w.nt = gr.z;
-    w.nb = gr.z / kBlockSize;
+    w.nsh = gr.z / kBlockSize;
+    w.nb = w.nsh + (gr.w ? gr.y * kTailBlocks : 0);
+    w.mlen = gr.w && lane < gr.y ? max(checked_len(p, gr.x + lane), 0) : 0;
     w.trow = p.tables + (int64_t)gr.x * p.max_blocks;
     w.tab = lane < p.max_blocks ? __ldg(w.trow + lane) : -1;
     w.skip = false;
@@ -301,36 +328,57 @@ __device__ __forceinline__ void load_unit(const Params &p, int64_t u, int64_t n_
     w.nb = (w.nt + kBlockSize - 1) / kBlockSize;
 }
 
-// Prologue: cum[s] = sum_{s' < s} (seq_units(s') - 1)^+ (exclusive
-// scan, one chunk of sequences per thread).  Ends with __syncthreads.
+// Prologue (split contexts): cum[s] = sum_{s' < s} (seq_units(s') - 1)^+ and, at
+// cum[S + 1 + s], the number of s' < s with seq_units(s') >= 1 (sequences whose
+// every token is covered by a group unit have no per-sequence unit at all);
+// exclusive scans, one chunk of sequences per thread.  Ends with __syncthreads.
 __device__ __forceinline__ void prologue(const Params &p, int *cum, int *scratch) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (p.part_tokens > 0) {
         const int S = p.num_seqs;
+        int *cumf = cum + S + 1;  // written only on the shared-prefix path (first_t set)
+        const bool wf = p.first_t != nullptr;
         const int per = (S + kThreads - 1) / kThreads;
         const int beg = min(S, (int)threadIdx.x * per), end = min(S, beg + per);
-        int local = 0;
+        int local = 0, localf = 0;
         for (int s = beg; s < end; ++s) {
             const int L = checked_len(p, s);
-            local += max(0, seq_units(p, L < 0 ? 0 : L, first_tok(p, s)) - 1);
+            const int su = seq_units(p, L < 0 ? 0 : L, first_tok(p, s));
+            local += max(0, su - 1);
+            localf += su > 0 ? 1 : 0;
         }
-        int incl = local;
+        int incl = local, inclf = localf;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += y;
+            const int y = __shfl_up_sync(kFull, incl, o), yf = __shfl_up_sync(kFull, inclf, o);
+            if (lane >= o) {
+                incl += y;
+                inclf += yf;
+            }
         }
-        if (lane == 31) scratch[warp] = incl;
+        if (lane == 31) {
+            scratch[warp] = incl;
+            scratch[kWarps + warp] = inclf;
+        }
         __syncthreads();
-        int off = 0;
-        for (int w = 0; w < warp; ++w) off += scratch[w];
-        int run = off + incl - local;
+        int off = 0, offf = 0;
+        for (int w = 0; w < warp; ++w) {
+            off += scratch[w];
+            offf += scratch[kWarps + w];
+        }
+        int run = off + incl - local, runf = offf + inclf - localf;
         for (int s = beg; s < end; ++s) {
             cum[s] = run;
+            if (wf) cumf[s] = runf;
             const int L = checked_len(p, s);
-            run += max(0, seq_units(p, L < 0 ? 0 : L, first_tok(p, s)) - 1);
+            const int su = seq_units(p, L < 0 ? 0 : L, first_tok(p, s));
+            run += max(0, su - 1);
+            runf += su > 0 ? 1 : 0;
         }
-        if ((int)threadIdx.x == kThreads - 1) cum[S] = run;
+        if ((int)threadIdx.x == kThreads - 1) {
+            cum[S] = run;
+            if (wf) cumf[S] = runf;
+        }
     }
     __syncthreads();
 }
@@ -578,9 +626,11 @@ struct MmaRows {
 
 // Group-rows mode: one online-softmax step per column over one 16-token block.
 // s[n]: column tile n's scores in log2 units as S^T fragments (tokens lane/4 and
-// lane/4 + 8, columns 2(lane%4) and 2(lane%4)+1).  Masks tokens at or past ntok
-// (>= 1), updates m and l, rescales the O^T accumulators and leaves the
-// unnormalised probabilities in s.
+// lane/4 + 8, columns 2(lane%4) and 2(lane%4)+1), -inf where a column does not
+// see the block.  Masks tokens at or past ntok (>= 1), updates m and l, rescales
+// the O^T accumulators and leaves the unnormalised probabilities in s.  A column
+// that has seen no key yet keeps m = -inf and contributes nothing (its reference
+// point is taken as 0, so no -inf - -inf arises).
 template <int D>
 __device__ __forceinline__ void softmax_rows(float (&s)[2][4], int ntok, MmaRows<D> &st, int lane) {
     constexpr int KS = D / 16;
@@ -597,19 +647,21 @@ __device__ __forceinline__ void softmax_rows(float (&s)[2][4], int ntok, MmaRows
     for (int off = 4; off < 32; off <<= 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) c[i] = fmaxf(c[i], __shfl_xor_sync(kFull, c[i], off));
+    float ref[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const float mn = fmaxf(st.m[i], c[i]);
-        al[i] = fast_exp2(st.m[i] - mn);
+        ref[i] = mn == -INFINITY ? 0.f : mn;
+        al[i] = fast_exp2(st.m[i] - ref[i]);
         st.m[i] = mn;
     }
     float r[4];
 #pragma unroll
     for (int n = 0; n < 2; ++n) {
-        s[n][0] = fast_exp2(s[n][0] - st.m[2 * n]);
-        s[n][1] = fast_exp2(s[n][1] - st.m[2 * n + 1]);
-        s[n][2] = fast_exp2(s[n][2] - st.m[2 * n]);
-        s[n][3] = fast_exp2(s[n][3] - st.m[2 * n + 1]);
+        s[n][0] = fast_exp2(s[n][0] - ref[2 * n]);
+        s[n][1] = fast_exp2(s[n][1] - ref[2 * n + 1]);
+        s[n][2] = fast_exp2(s[n][2] - ref[2 * n]);
+        s[n][3] = fast_exp2(s[n][3] - ref[2 * n + 1]);
         r[2 * n] = s[n][0] + s[n][2];
         r[2 * n + 1] = s[n][1] + s[n][3];
     }
@@ -636,8 +688,8 @@ __device__ __forceinline__ void softmax_rows(float (&s)[2][4], int ntok, MmaRows
 // sharing every K fragment, one online-softmax step per column, then
 // O^T += V^T P^T with every V fragment feeding both column tiles.
 template <int D>
-__device__ __forceinline__ void mma_block_rows(uint32_t kb, unsigned char *vgen, int ntok, MmaRows<D> &st,
-                                               float sl2, int lane) {
+__device__ __forceinline__ void mma_block_rows(uint32_t kb, unsigned char *vgen, int ntok, int c_lo, int c_hi,
+                                               MmaRows<D> &st, float sl2, int lane) {
     constexpr int KS = D / 16;
     constexpr int kRow = 2 * D;
     const uint32_t vb = kb + kBlockSize * kRow;
@@ -659,9 +711,14 @@ __device__ __forceinline__ void mma_block_rows(uint32_t kb, unsigned char *vgen,
         mma_bf16_16816(d1, a, st.qb[kk][1][0], st.qb[kk][1][1]);
     }
 #pragma unroll
-    for (int n = 0; n < 2; ++n)
+    for (int n = 0; n < 2; ++n) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) s[n][k] = (s[n][k] + s2[n][k]) * sl2;
+        // columns (query rows) outside [c_lo, c_hi) do not see this block
+        const int c0 = 8 * n + 2 * (lane & 3);
+        if (c0 < c_lo || c0 >= c_hi) s[n][0] = s[n][2] = -INFINITY;
+        if (c0 + 1 < c_lo || c0 + 1 >= c_hi) s[n][1] = s[n][3] = -INFINITY;
+    }
     softmax_rows<D>(s, ntok, st, lane);
     // P^T operand fragments of both column tiles, transposed in registers
     uint32_t pb[2][2];
@@ -989,7 +1046,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     const int S = p.num_seqs, hkv = p.num_kv_heads;
     const int64_t n_extra = !kRows && p.part_tokens > 0 ? (int64_t)cum[S] * hkv : 0;
     const int gbase = kRows ? __ldg(p.meta) : 0;  // row groups follow the tile groups
-    const int64_t total = kRows ? (int64_t)__ldg(p.meta + 5) * hkv : (int64_t)S * hkv + n_extra;
+    const int64_t total = kRows ? (int64_t)__ldg(p.meta + 5) * hkv
+                                : (p.first_t != nullptr ? (int64_t)cum[2 * S + 1] : (int64_t)S) * hkv + n_extra;
     auto load_any = [&](int64_t u, WarpUnit &w) {
         if constexpr (kRows) load_unit_rows(p, u, gbase, w, lane);
         else load_unit(p, u, n_extra, cum, w, lane, warp == 0);
@@ -1049,9 +1107,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     bool have_nxt = u_nxt < total;
     if (have_nxt) load_any(u_nxt, nxt);
 
-    // table entry of logical block j of a unit (the first 32 come from registers)
+    // table entry of logical block j of a unit (the first 32 come from registers);
+    // a group-rows unit's items past its shared blocks are its members' tail blocks
     auto phys_of = [&](const WarpUnit &w, int j) {
         const int v = __shfl_sync(kFull, w.tab, j & 31);
+        if constexpr (kRows) {
+            if (j >= w.nsh) {
+                const int m = (j - w.nsh) / kTailBlocks, i = (j - w.nsh) % kTailBlocks;
+                const int Lm = __shfl_sync(kFull, w.mlen, m & 31);
+                if (i >= (Lm + kBlockSize - 1) / kBlockSize - w.nsh) return kEmptyItem;
+                return __ldg(p.tables + (int64_t)(w.un.s + m) * p.max_blocks + w.nsh + i);
+            }
+        }
         return j < 32 ? v : __ldg(w.trow + j);
     };
     // normalise a cursor (iu: 0 = cur, 1 = nxt) onto an existing item, skipping
@@ -1080,7 +1147,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
         const int blk = phys_of(w, iss_j);
         const bool ok = blk >= 0 && blk < p.num_blocks;
         if (ok) issue_slabs<T, D, G>(p, wring_s + stage * Lay::kStageBytes, blk, w.un.h, lane);
-        else if (lane == 0) flag_error(p.err, PA_DEVERR_BLOCK_ID);
+        else if (lane == 0 && blk != kEmptyItem) flag_error(p.err, PA_DEVERR_BLOCK_ID);
         cp_async_commit();
         okmask = (okmask & ~(1u << stage)) | ((ok ? 1u : 0u) << stage);
         iss_j += kWarps;
@@ -1210,11 +1277,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
             __syncwarp();
             const int stage = n_cmp % NS;
             if ((okmask >> stage) & 1u) {
-                const int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
-                if constexpr (kRows)
+                int ntok = min(kBlockSize, cur.nt - j * kBlockSize);
+                if constexpr (kRows) {
+                    // a tail block counts for its member's g rows only
+                    int c_lo = 0, c_hi = kRowTile;
+                    if (j >= cur.nsh) {
+                        const int m = (j - cur.nsh) / kTailBlocks, i = (j - cur.nsh) % kTailBlocks;
+                        const int Lm = __shfl_sync(kFull, cur.mlen, m & 31);
+                        const int g = p.num_q_heads / hkv;
+                        ntok = min(kBlockSize, Lm - (cur.nsh + i) * kBlockSize);
+                        c_lo = m * g;
+                        c_hi = c_lo + g;
+                    }
                     mma_block_rows<D>(wring_s + stage * Lay::kStageBytes,
-                                      wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, mr,
+                                      wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, c_lo, c_hi, mr,
                                       p.scale_log2, lane);
+                }
                 else if constexpr (kMma)
                     mma_block<D>(wring_s + stage * Lay::kStageBytes,
                                  wring + stage * Lay::kStageBytes + Lay::kSlabBytes, ntok, ms,
@@ -1353,7 +1431,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
 constexpr int kDetectThreads = 1024;
 constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
-constexpr int kMaxGroupBlocks = (1 << 22) - 1;  // fits info's packing (nb << 9)
+constexpr int kMaxGroupBlocks = (1 << 21) - 1;  // fits info's packing (nb << 10)
 // Groups of fewer members do not pay for the group unit's fixed cost (its rows
 // pad a 128-row tensor-core tile).
 constexpr int kMinGroupMembers = 4;
@@ -1471,8 +1549,8 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
                                                                       int32_t *meta,
                                                                       const __grid_constant__ StepWriteArgs w) {
     __shared__ int lcp[kMaxGroupSeqs];
-    __shared__ int info[kMaxGroupSeqs];  // run sizes, then at a chunk head: its size, then
-                                         // nb << 9 | row group << 8 | size (size <= 128)
+    __shared__ int info[kMaxGroupSeqs];  // at a chunk head: its size, then nb << 10 |
+                                         // tails << 9 | row group << 8 | size (size <= 128)
     // Launched with programmatic serialization: this grid may start while the
     // kernel before it in the stream (the previous call's combine, say) is still
     // running.  Until grid_dep_wait() it only reads the block tables and lengths
@@ -1559,7 +1637,10 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     }
     __syncthreads();
     // a chunk of n members is a row group when n x g <= kRowTile (n >= 2), else a
-    // tile group when n >= kMinGroupMembers; info = nb << 9 | row << 8 | n
+    // tile group when n >= kMinGroupMembers.  A row group whose members' private
+    // tails (blocks past the shared ones) are all at most kTailBlocks long takes
+    // the tails too (its unit masks each tail block to its member's rows), so its
+    // members need no per-sequence unit.  info = nb << 10 | tails << 9 | row << 8 | n
     int nt_heads = 0, nr_heads = 0;  // this thread's tile / row groups
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
@@ -1567,7 +1648,16 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         const bool row = p.row_groups && n >= 2 && n * g <= kRowTile;
         const bool tile = !row && n >= kMinGroupMembers;
         const int nb = (row || tile) && mn >= bpp ? min(mn, kMaxGroupBlocks) : 0;
-        info[s] = (nb << 9) | ((row ? 1 : 0) << 8) | n;
+        bool tails = false;
+        if (row && nb > 0) {
+            int tmax = 0;
+            for (int k = 0; k < n; ++k) {
+                const int L = max(checked_len(p, s + k), 0);
+                tmax = max(tmax, (L + kBlockSize - 1) / kBlockSize - nb);
+            }
+            tails = tmax <= kTailBlocks;
+        }
+        info[s] = (nb << 10) | ((tails ? 1 : 0) << 9) | ((row ? 1 : 0) << 8) | n;
         if (nb > 0) {
             if (row) ++nr_heads;
             else ++nt_heads;
@@ -1595,14 +1685,13 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     unsigned long long tw = 0, rw = 0, dw = 0;
     for (int s = s0; s < s1; ++s) {
         const int inf = info[head_of[s - s0]];
-        const int ft = (inf >> 9) * kBlockSize;
-        first_t[s] = ft;
         const int L = max(check_len(p, len_of[s - s0]), 0);
+        const int fs = (inf >> 10) * kBlockSize;                // shared tokens
+        const int ft = ((inf >> 9) & 1) ? max(L, fs) : fs;      // tails: all of it
+        first_t[s] = ft;
         dw += (unsigned long long)max(0, L - ft);
-        if (head_of[s - s0] == s) {
-            if ((inf >> 8) & 1) rw += (unsigned long long)ft;
-            else tw += (unsigned long long)ft;
-        }
+        if ((inf >> 8) & 1) rw += (unsigned long long)(max(0, ft - fs) + (head_of[s - s0] == s ? fs : 0));
+        else if (head_of[s - s0] == s) tw += (unsigned long long)fs;
     }
     // one shared-memory atomic per warp (1,024 on one word would serialise)
 #pragma unroll
@@ -1622,10 +1711,10 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
         const int inf = info[s];
-        const int n = inf & 255, nb = inf >> 9;
+        const int n = inf & 255, nb = inf >> 10;
         if (nb == 0) continue;
-        if ((inf >> 8) & 1) {
-            groups[gr] = make_int4(s, n, nb * kBlockSize, (gr - n_tile) * p.num_kv_heads);
+        if ((inf >> 8) & 1) {  // row groups: the fourth field says whether the unit takes the tails
+            groups[gr] = make_int4(s, n, nb * kBlockSize, (inf >> 9) & 1);
             ++gr;
         } else {
             groups[gt] = make_int4(s, n, nb * kBlockSize, gt * p.num_kv_heads);
@@ -1746,13 +1835,13 @@ template <typename T, int D, int G>
 cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
     using Lay = Layout<T, D, G>;
     const bool split = prm.part_tokens > 0;
-    const size_t smem = Lay::smem_bytes(split ? a.num_seqs + 1 : 0);
+    const size_t smem = Lay::smem_bytes(split ? Lay::kCumArrays * (a.num_seqs + 1) : 0);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    static_assert(Lay::smem_bytes(kMaxSplitSeqs + 1) <= 232448, "decode smem over the sm_100 limit");
+    static_assert(Lay::smem_bytes(Lay::kCumArrays * (kMaxSplitSeqs + 1)) <= 232448, "decode smem over the sm_100 limit");
     e = cudaFuncSetAttribute(decode_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)Lay::smem_bytes(kMaxSplitSeqs + 1));
+                             (int)Lay::smem_bytes(Lay::kCumArrays * (kMaxSplitSeqs + 1)));
     if (e != cudaSuccess) return e;
     const int sms = num_sms(dev);
     prm.num_sms = sms;

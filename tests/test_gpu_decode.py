@@ -409,8 +409,10 @@ def _expected_groups(tables, lens, part, g, hkv, min_members=4):
     other runs are cut into chunks of 128 / g counted from their start.  A chunk
     shares nb = min(lcp over its members after the first) blocks and is a row
     group when row groups are on, 2 <= n and n * g <= 16, else a tile group when
-    n >= 4.  Returns first_t (shared tokens per sequence), the tile groups'
-    records, then the row groups' records."""
+    n >= 4.  A row group whose members' tails (blocks past the nb shared ones) are
+    at most 4 blocks long covers its members entirely.  Returns first_t (tokens
+    per sequence covered by its group), the tile groups' records, then the row
+    groups' records (their last field: 1 when they take the tails)."""
     S = len(lens)
     bpp = part // 16
     M = 128 // g
@@ -439,13 +441,15 @@ def _expected_groups(tables, lens, part, g, hkv, min_members=4):
         row = row_groups and n >= 2 and n * g <= 16
         tile = not row and n >= min_members
         mn = min(lcp[m] for m in mem[1:]) if n > 1 else 0
-        nb = min(mn, (1 << 22) - 1) if (row or tile) and mn >= bpp else 0
+        nb = min(mn, (1 << 21) - 1) if (row or tile) and mn >= bpp else 0
         if nb == 0:
             continue
+        # a row group takes its members' private tails when none is longer than 4 blocks
+        tails = row and max(-(-int(lens[m]) // 16) - nb for m in mem) <= 4
         for m in mem:
-            first_t[m] = nb * 16
+            first_t[m] = max(int(lens[m]), nb * 16) if tails else nb * 16
         if row:
-            rows.append((mem[0], n, nb * 16, len(rows) * hkv))
+            rows.append((mem[0], n, nb * 16, 1 if tails else 0))
         else:
             tiles.append((mem[0], n, nb * 16, len(tiles) * hkv))
     return first_t, tiles, rows
