@@ -1705,17 +1705,40 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         atomicAdd(&work[1], rw);
         atomicAdd(&work[2], dw);
     }
-    // records: tile groups first (the tile kernel reads groups[0, n_tile)), then
-    // the row groups
-    int gt = ex & 0xffff, gr = n_tile + (ex >> 16);
+    // records: tile groups first (the tile kernel reads groups[0, n_tile)), in
+    // sequence order; then the row groups, longest first by buckets of 32 shared
+    // blocks (the group-rows kernel draws its units in record order, so the
+    // longest start first and the short ones even out the end; the order within a
+    // bucket does not affect any result)
+    constexpr int kBuckets = 8;
+    __shared__ int rcount[kBuckets], rbase[kBuckets];
+    auto bucket = [](int nb) { return kBuckets - 1 - min(kBuckets - 1, nb >> 5); };  // 0: longest
+    if (n_row > 0) {  // (uniform)
+        if (threadIdx.x < kBuckets) rcount[threadIdx.x] = 0;
+        __syncthreads();
+        for (int s = s0; s < s1; ++s)
+            if (head_of[s - s0] == s && ((info[s] >> 8) & 1) && (info[s] >> 10) > 0)
+                atomicAdd(&rcount[bucket(info[s] >> 10)], 1);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            int run = n_tile;
+            for (int b = 0; b < kBuckets; ++b) {
+                rbase[b] = run;
+                run += rcount[b];
+                rcount[b] = 0;
+            }
+        }
+        __syncthreads();
+    }
+    int gt = ex & 0xffff;
     for (int s = s0; s < s1; ++s) {
         if (head_of[s - s0] != s) continue;
         const int inf = info[s];
         const int n = inf & 255, nb = inf >> 10;
         if (nb == 0) continue;
         if ((inf >> 8) & 1) {  // row groups: the fourth field says whether the unit takes the tails
-            groups[gr] = make_int4(s, n, nb * kBlockSize, (inf >> 9) & 1);
-            ++gr;
+            const int b = bucket(nb);
+            groups[rbase[b] + atomicAdd(&rcount[b], 1)] = make_int4(s, n, nb * kBlockSize, (inf >> 9) & 1);
         } else {
             groups[gt] = make_int4(s, n, nb * kBlockSize, gt * p.num_kv_heads);
             ++gt;

@@ -487,8 +487,12 @@ def test_group_detection_matches_the_rule(cid, part):
     assert meta[0] == len(want_tiles) and meta[1] == len(want_tiles) * wl.num_kv_heads
     assert meta[5] == len(want_rows)
     n_g = len(want_tiles) + len(want_rows)
-    got = raw[gat:gat + 16 * n_g].view(np.int32).reshape(-1, 4)
-    assert [tuple(int(x) for x in r) for r in got] == want_tiles + want_rows
+    got = [tuple(int(x) for x in r) for r in raw[gat:gat + 16 * n_g].view(np.int32).reshape(-1, 4)]
+    assert got[:len(want_tiles)] == want_tiles            # tile groups in sequence order
+    got_rows = got[len(want_tiles):]
+    assert sorted(got_rows) == sorted(want_rows)          # row groups: longest first by buckets
+    keys = [7 - min(7, (r[2] // 16) >> 5) for r in got_rows]
+    assert keys == sorted(keys)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     if want_tiles:   # SMs the detection kernel gave the group tiles
         assert 1 <= meta[4] <= sms
