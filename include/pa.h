@@ -163,8 +163,9 @@ PA_API pa_status pa_check_copy_pairs(const int32_t *src_dst_pairs, int32_t num_p
  * Bytes of workspace pa_decode needs for a split (partitioned) context:
  * partials of num_seqs * num_q_heads * ceil(max_context_len / partition_size)
  * partitions (head_dim fp32 accumulators plus a running max and sum each), then
- * the shared-prefix group area (a shared-token count and a 16-byte group record
- * per sequence, and 32 bytes of counts).  Returns 0 when partition_size <= 0
+ * the shared-prefix group area (a shared-token count, a 16-byte group record and
+ * a table-comparison result per sequence, 32 bytes of counts and 512 bytes of
+ * flags).  Returns 0 when partition_size <= 0
  * (no split, no workspace).
  */
 PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t head_dim,

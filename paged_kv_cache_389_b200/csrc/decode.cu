@@ -56,7 +56,9 @@
 //  * Every wait that depends on another warp or kernel (the merge slots' mbarrier,
 //    the ring of unit ids) is bounded by %globaltimer; on a timeout the CTA sets
 //    PA_DEVERR_TIMEOUT, raises its abort flag and every warp leaves its loop.
+#include <atomic>
 #include <cfloat>
+#include <chrono>
 #include <climits>
 #include <cstring>
 #include <type_traits>
@@ -188,6 +190,14 @@ struct Params {
     int32_t *work_ctr;      // units handed out beyond the first gridDim.x (zeroed by the
                             // detection kernel of this call), or nullptr: static order
     int32_t num_sms;        // SMs of the device (the detection kernel splits them)
+    // detection: blocks 1..lcp_blocks compare the tables of a slice of sequences
+    // each, write lcp_g[s] and then lflags[block - 1] = epoch (a 64-bit value unique
+    // to the call, so stale workspace contents never match); block 0 waits for those
+    // flags (0 blocks: block 0 compares all)
+    int32_t *lcp_g;
+    unsigned long long *lflags;
+    unsigned long long epoch;
+    int32_t lcp_blocks;
 };
 
 // Context length, or -1 when outside [0, max_context] or longer than its table.
@@ -221,8 +231,11 @@ struct Unit {
 // partial into slot 0.
 __device__ __forceinline__ int slot_base(int ft) { return ft > 0 ? 1 : 0; }
 
+// first_t[s] carries kDoneBit for the members of a group-rows unit that takes the
+// tails: that unit covers all of s and writes s's output itself.
+constexpr int kDoneBit = 1 << 30;
 __device__ __forceinline__ int first_tok(const Params &p, int s) {
-    return p.first_t ? __ldg(p.first_t + s) : 0;
+    return p.first_t ? (__ldg(p.first_t + s) & (kDoneBit - 1)) : 0;
 }
 
 // Unit u -> (sequence, slot, kv head).  Units [0, n_extra) are the further
@@ -276,6 +289,7 @@ struct WarpUnit {
     int nsh;    // group-rows mode: shared blocks (items [0, nsh)); items after them are the
                 // members' tails, kTailBlocks slots per member (empty past a member's tail)
     int mlen;   // group-rows mode with tails: lane m holds member m's context length
+    bool full;  // group-rows mode: the unit covers its members entirely (writes the output)
 };
 
 // A tail slot past its member's tail: no block to load (not an error).
@@ -294,6 +308,7 @@ __device__ __forceinline__ void load_unit_rows(const Params &p, int64_t v, int g
     w.nsh = gr.z / kBlockSize;
     w.nb = w.nsh + (gr.w ? gr.y * kTailBlocks : 0);
     w.mlen = gr.w && lane < gr.y ? max(checked_len(p, gr.x + lane), 0) : 0;
+    w.full = gr.w != 0;
     w.trow = p.tables + (int64_t)gr.x * p.max_blocks;
     w.tab = lane < p.max_blocks ? __ldg(w.trow + lane) : -1;
     w.skip = false;
@@ -479,9 +494,14 @@ __device__ __forceinline__ void finish_unit_rows(const Params &p, const WarpUnit
             }
         }
         if constexpr (kIsFp8<T>) o *= p.v_scale;
-        const int64_t row = ((int64_t)(w.un.s + r / g) * p.num_q_heads + (int64_t)w.un.h * g + r % g) * p.max_parts;
-        p.ws_acc[row * D + dd] = o;
-        if (dd == 0) p.ws_ml[row] = make_float2(M, lsum);
+        const int64_t qrow = (int64_t)(w.un.s + r / g) * p.num_q_heads + (int64_t)w.un.h * g + r % g;
+        if (w.full) {  // the unit covered every key of its members: the output itself
+            store_out<IoT<T>>(p.out, qrow * D + dd, lsum > 0.f ? o * (1.f / lsum) : 0.f);
+        } else {
+            const int64_t row = qrow * p.max_parts;
+            p.ws_acc[row * D + dd] = o;
+            if (dd == 0) p.ws_ml[row] = make_float2(M, lsum);
+        }
     }
 }
 
@@ -1430,6 +1450,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 // (launch_group_tiles).
 
 constexpr int kDetectThreads = 1024;
+constexpr int kLcpBlocksMax = 64;  // detection blocks that compare tables (flags in the workspace)
+
+// A 64-bit value unique to each call of this process (the high half drawn from
+// the clock once per process), so that detection flags left in a reused
+// workspace by an earlier call -- or by another process -- never match.
+unsigned long long next_epoch() {
+    static std::atomic<unsigned long long> ctr{
+        (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() << 20};
+    unsigned long long e = ++ctr;
+    return e == 0 ? ++ctr : e;
+}
 constexpr int kMaxGroupSeqs = 4096;  // == kMaxSplitSeqs
 constexpr int kMaxGroupBlocks = (1 << 21) - 1;  // fits info's packing (nb << 10)
 // Groups of fewer members do not pay for the group unit's fixed cost (its rows
@@ -1505,6 +1536,43 @@ __device__ __forceinline__ void shared_prefix_lengths(const Params &p, int *lcp)
     }
 }
 
+// lcp of the pair (s - 1, s) (s > 0) by one warp: leading entries of s's table
+// equal to those of s - 1, over the blocks both contexts fill completely.  Rounds
+// of 256 entries (8 loads per lane and table); the first round's loads go out
+// together with the lengths'.
+__device__ __forceinline__ int pair_lcp(const Params &p, int s, int lane) {
+    const int32_t *ta = p.tables + (int64_t)s * p.max_blocks;
+    const int32_t *tb = ta - p.max_blocks;
+    const int la = __ldg(p.lens + s), lb = __ldg(p.lens + s - 1);
+    int va[8], vb[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int i = 32 * k + lane;
+        va[k] = i < p.max_blocks ? __ldg(ta + i) : 0;
+        vb[k] = i < p.max_blocks ? __ldg(tb + i) : 0;
+    }
+    const int La = check_len(p, la), Lb = check_len(p, lb);
+    const int n = min(max(La, 0), max(Lb, 0)) / kBlockSize;
+    for (int c0 = 0;; c0 += 256) {
+        if (c0 > 0) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int i = c0 + 32 * k + lane;
+                va[k] = i < n ? __ldg(ta + i) : 0;
+                vb[k] = i < n ? __ldg(tb + i) : 0;
+            }
+        }
+        int mis = n;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = c0 + 32 * k + lane;
+            if (i < n && va[k] != vb[k]) mis = min(mis, i);
+        }
+        mis = __reduce_min_sync(kFull, mis);
+        if (mis < n || c0 + 256 >= n) return mis;
+    }
+}
+
 // Warp-wide exclusive scan (sum, or max when kMax) of one int per lane.
 template <bool kMax>
 __device__ __forceinline__ int warp_exclusive_scan(int x, int identity) {
@@ -1519,17 +1587,19 @@ __device__ __forceinline__ int warp_exclusive_scan(int x, int identity) {
     return lane == 0 ? identity : exc;
 }
 
-// Block 0: all warps compare tables, then the groups are formed block-parallel.
-// A run is a maximal stretch of sequences each sharing at least part_tokens
-// tokens of full blocks with its predecessor.  A run of n sequences with
-// n x g <= 16 query rows stays whole; a longer run is cut into chunks of
-// max_members (128 / g) sequences counted from its start (kRowTile / g without
-// tile groups).  A chunk shares its nb = min(lcp over its members after the
-// first) leading blocks; it becomes a row group when 2 <= n and n x g <= 16
-// (one group-rows unit per kv head, on decode_kernel<T, D, kRowTile>), else a
-// tile group when n >= kMinGroupMembers (one tcgen05 tile unit per kv head);
-// each unit covers the 16 nb shared tokens.  first_t[s] = 16 nb of s's group (0
-// outside one).
+// Detection.  lcp[s] = leading full blocks of s's table equal to those of s - 1
+// (compared by blocks 1.. of the grid for more than 64 sequences, else by block
+// 0); then block 0 forms the groups block-parallel.  A run is a maximal stretch of
+// sequences each sharing at least part_tokens tokens of full blocks with its
+// predecessor.  With row groups, a run of n sequences with n x g <= 16 query rows
+// stays whole; other runs are cut into chunks of max_members (128 / g) sequences
+// counted from their start.  A chunk shares its nb = min(lcp over its members
+// after the first) leading blocks; it becomes a row group when 2 <= n and
+// n x g <= 16 (one group-rows unit per kv head, on decode_kernel<T, D, kRowTile>),
+// else a tile group when n >= kMinGroupMembers (one tcgen05 tile unit per kv head);
+// each unit covers the 16 nb shared tokens, a row group's unit also its members'
+// private tails when none is longer than kTailBlocks.  first_t[s] = 16 nb of s's
+// group, or s's length with kDoneBit for a row group with tails (0 outside one).
 // The one-call step's cache write, done by blocks 1.. of the detection grid.
 struct StepWriteArgs {
     const uint4 *key;
@@ -1558,6 +1628,21 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     // whole grouping); every global write comes after it.
     grid_dep_launch();  // the group tiles set up while this runs, then wait for it
     if (blockIdx.x > 0) {
+        if ((int)blockIdx.x <= p.lcp_blocks) {
+            // this block's slice of the table comparison, one pair per warp
+            const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+            const int per = (p.num_seqs + p.lcp_blocks - 1) / p.lcp_blocks;
+            const int b0 = ((int)blockIdx.x - 1) * per, b1 = min(p.num_seqs, b0 + per);
+            for (int s = b0 + warp; s < b1; s += kDetectThreads / 32) {
+                const int v = s > 0 ? pair_lcp(p, s, lane) : 0;
+                if (lane == 0) p.lcp_g[s] = v;
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                __threadfence();
+                *reinterpret_cast<volatile unsigned long long *>(p.lflags + blockIdx.x - 1) = p.epoch;
+            }
+        }
         // the step's new K/V (pa_append_decode): the tiles and the decode wait for
         // this whole grid, so they see it; detection reads no cache bytes
         grid_dep_wait();
@@ -1568,7 +1653,29 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         return;
     }
     const int S = p.num_seqs;
-    shared_prefix_lengths(p, lcp);
+    __shared__ int lcp_ok;  // 0: the wait for the other blocks' comparisons ran out
+    if (threadIdx.x == 0) lcp_ok = 1;
+    if (p.lcp_blocks > 0) {
+        // the other blocks compare the tables; wait (bounded) for their flags.  On a
+        // timeout no sequence is grouped (lcp 0): slower, the same result.
+        __syncthreads();
+        if ((int)threadIdx.x < p.lcp_blocks) {
+            const volatile unsigned long long *f =
+                reinterpret_cast<const volatile unsigned long long *>(p.lflags + threadIdx.x);
+            const unsigned long long t0 = global_ns();
+            while (*f != p.epoch) {
+                if (global_ns() - t0 > p.wait_ns) {
+                    lcp_ok = 0;
+                    break;
+                }
+            }
+        }
+        __syncthreads();
+        __threadfence();
+        for (int s = threadIdx.x; s < S; s += kDetectThreads) lcp[s] = lcp_ok ? __ldcg(p.lcp_g + s) : 0;
+    } else {
+        shared_prefix_lengths(p, lcp);
+    }
     __syncthreads();
     // Every thread owns a contiguous run of at most 4 sequences [s0, s1).
     __shared__ int wtot[kDetectThreads / 32];
@@ -1656,6 +1763,7 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
                 tmax = max(tmax, (L + kBlockSize - 1) / kBlockSize - nb);
             }
             tails = tmax <= kTailBlocks;
+            for (int k = 0; k < n && tails; ++k) tails = checked_len(p, s + k) < kDoneBit;
         }
         info[s] = (nb << 10) | ((tails ? 1 : 0) << 9) | ((row ? 1 : 0) << 8) | n;
         if (nb > 0) {
@@ -1682,13 +1790,14 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
     // only after the write, and the group tiles, which wait for this kernel, see
     // the new tokens' K/V.
     grid_dep_wait();
+    if (threadIdx.x == 0 && !lcp_ok) flag_error(p.err, PA_DEVERR_TIMEOUT);
     unsigned long long tw = 0, rw = 0, dw = 0;
     for (int s = s0; s < s1; ++s) {
         const int inf = info[head_of[s - s0]];
         const int L = max(check_len(p, len_of[s - s0]), 0);
         const int fs = (inf >> 10) * kBlockSize;                // shared tokens
         const int ft = ((inf >> 9) & 1) ? max(L, fs) : fs;      // tails: all of it
-        first_t[s] = ft;
+        first_t[s] = ((inf >> 9) & 1) ? (ft | kDoneBit) : ft;
         dw += (unsigned long long)max(0, L - ft);
         if ((inf >> 8) & 1) rw += (unsigned long long)(max(0, ft - fs) + (head_of[s - s0] == s ? fs : 0));
         else if (head_of[s - s0] == s) tw += (unsigned long long)fs;
@@ -1810,7 +1919,9 @@ __global__ void __launch_bounds__(128) reduce_kernel(const __grid_constant__ Par
     }
     int L = checked_len(p, s);
     if (L < 0) L = 0;
-    const int ft = first_tok(p, s);
+    const int ftr = p.first_t ? __ldg(p.first_t + s) : 0;
+    if (ftr & kDoneBit) return;                          // written by its group-rows unit
+    const int ft = ftr;
     const int n = slot_base(ft) + seq_units(p, L, ft);  // slots written
     if (ft == 0 && n <= 1) return;                       // finished by the decode kernel
     float M = -INFINITY;
@@ -1889,6 +2000,14 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             prm.first_t = reinterpret_cast<int32_t *>(g);
             prm.groups = reinterpret_cast<int4 *>(g + sa);
             prm.meta = reinterpret_cast<int32_t *>(const_cast<int4 *>(prm.groups) + a.num_seqs);
+            // then lcp_g[S] (16-byte padded) and the comparison blocks' flags (64 x 8 bytes)
+            unsigned char *gl_area = reinterpret_cast<unsigned char *>(const_cast<int32_t *>(prm.meta)) + 32;
+            prm.lcp_g = reinterpret_cast<int32_t *>(gl_area);
+            prm.lflags = reinterpret_cast<unsigned long long *>(gl_area + sa);
+            // more than 64 sequences: the comparison is spread over one block per 32
+            // sequences (up to kLcpBlocksMax); the epoch makes each call's flags unique
+            prm.lcp_blocks = a.num_seqs > 64 ? std::min(kLcpBlocksMax, (a.num_seqs + 31) / 32) : 0;
+            prm.epoch = next_epoch();
             // Row groups need 2 <= members <= 16 / g; at g = 8 only pairs qualify,
             // whose gain does not pay for the extra launch, so the group-rows kernel
             // runs for g <= 4 only.
@@ -1915,7 +2034,8 @@ cudaError_t launch_t(const DecodeLaunch &a, Params &prm, cudaStream_t stream) {
             }
             // always with programmatic serialization: its table comparison may
             // overlap the end of whatever kernel precedes it (see the kernel)
-            e = launch_after(group_detect_kernel, dim3(1 + write_blocks), dim3(kDetectThreads), 0, stream,
+            e = launch_after(group_detect_kernel, dim3(1 + std::max<unsigned>(write_blocks, (unsigned)prm.lcp_blocks)),
+                             dim3(kDetectThreads), 0, stream,
                              static_cast<const Params &>(prm), const_cast<int32_t *>(prm.first_t),
                              const_cast<int4 *>(prm.groups), const_cast<int32_t *>(prm.meta),
                              static_cast<const StepWriteArgs &>(wa));

@@ -156,10 +156,12 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t h
     const int64_t parts = ((int64_t)max_context_len + partition_size - 1) / partition_size;
     const int64_t rows = (int64_t)num_seqs * num_q_heads * parts;
     // partials (fp32 acc, then (m, l)), then the shared-prefix group bookkeeping:
-    // first partition per sequence (16-byte padded), group list (16 bytes each),
-    // 32 bytes of counts and counters
+    // shared tokens per sequence (16-byte padded), group list (16 bytes each), 32
+    // bytes of counts and counters, the table comparison's per-sequence results
+    // (16-byte padded) and its blocks' flags (64 x 8 bytes)
     const int64_t partials = rows * head_dim * 4 + rows * 8;
-    const int64_t group = ((int64_t)num_seqs * 4 + 15) / 16 * 16 + (int64_t)num_seqs * 16 + 32;
+    const int64_t s16 = ((int64_t)num_seqs * 4 + 15) / 16 * 16;
+    const int64_t group = s16 + (int64_t)num_seqs * 16 + 32 + s16 + 64 * 8;
     return (size_t)((partials + 15) / 16 * 16 + group);
 }
 

@@ -109,17 +109,18 @@ def test_host_validation_launches_nothing(pa):
 def test_workspace_size_formula(pa):
     # partials: rows = S * Hq * ceil(maxctx / part), each head_dim fp32 + (m, l);
     # then the shared-prefix group area: S int32 shared-token counts (16-byte
-    # padded), S int4 group records, 32 bytes of counts.
+    # padded), S int4 group records, 32 bytes of counts, S int32 table-comparison
+    # results (16-byte padded), 64 x 8 bytes of flags.
     def a16(x):
         return (x + 15) // 16 * 16
 
     def expect(S, hq, d, ctx, part):
         rows = S * hq * (-(-ctx // part))
-        return a16(rows * (d * 4 + 8)) + a16(S * 4) + S * 16 + 32
+        return a16(rows * (d * 4 + 8)) + a16(S * 4) + S * 16 + 32 + a16(S * 4) + 512
 
     assert pa.pa_decode_workspace_size(8, 64, 128, 32768, 512) == expect(8, 64, 128, 32768, 512)
     assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == expect(3, 4, 64, 100, 32)
-    assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == 3 * 4 * 4 * (64 * 4 + 8) + 16 + 48 + 32
+    assert pa.pa_decode_workspace_size(3, 4, 64, 100, 32) == 3 * 4 * 4 * (64 * 4 + 8) + 16 + 48 + 32 + 16 + 512
     assert pa.pa_decode_workspace_size(3, 4, 64, 100, 0) == 0
 
 

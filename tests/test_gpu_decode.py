@@ -447,7 +447,9 @@ def _expected_groups(tables, lens, part, g, hkv, min_members=4):
         # a row group takes its members' private tails when none is longer than 4 blocks
         tails = row and max(-(-int(lens[m]) // 16) - nb for m in mem) <= 4
         for m in mem:
-            first_t[m] = max(int(lens[m]), nb * 16) if tails else nb * 16
+            # members of a row group with tails carry bit 30 (their output is written
+            # by the group's unit; the combine skips them)
+            first_t[m] = (max(int(lens[m]), nb * 16) | (1 << 30)) if tails else nb * 16
         if row:
             rows.append((mem[0], n, nb * 16, 1 if tails else 0))
         else:
