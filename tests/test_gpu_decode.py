@@ -281,6 +281,85 @@ def test_shared_prefix_groups_match_oracle(g):
     assert ts.err_flag() == 0
 
 
+def _families_workload(spec, g, n_loners, seed=31):
+    """Sibling families (parent tokens, [suffix lengths]) followed by n_loners unrelated
+    sequences of 40 tokens, g query heads per kv head, 2 kv heads, head_dim 128."""
+    rng = np.random.default_rng(seed)
+    hkv, d = 2, 128
+    hq = g * hkv
+    nb = 16 + sum(-(-(pt + max(sx, default=0) + 2) // 16) * (len(sx) + 1) for pt, sx in spec) + 4 * n_loners
+    wl = workloads.Workload(0, "families", "bf16", nb, hq, hkv, d, 1.0 / np.sqrt(d),
+                            rng.permutation(nb).astype(np.int32))
+    seq, seqs = 0, []
+    for fi, (pt, sx) in enumerate(spec):
+        parent = 10000 + fi
+        wl.ops.append(("add", parent))
+        wl.ops.append(("append", parent, workloads.normal(rng, (pt, hkv, d), "bf16"),
+                       workloads.normal(rng, (pt, hkv, d), "bf16")))
+        kids = []
+        for _ in sx:
+            wl.ops.append(("fork", parent, seq))
+            kids.append(seq)
+            seq += 1
+        wl.ops.append(("free", parent))
+        for kid, n in zip(kids, sx):
+            if n:
+                wl.ops.append(("append", kid, workloads.normal(rng, (n, hkv, d), "bf16"),
+                               workloads.normal(rng, (n, hkv, d), "bf16")))
+        seqs.extend(kids)
+    for _ in range(n_loners):
+        wl.ops.append(("add", seq))
+        wl.ops.append(("append", seq, workloads.normal(rng, (40, hkv, d), "bf16"),
+                       workloads.normal(rng, (40, hkv, d), "bf16")))
+        seqs.append(seq)
+        seq += 1
+    S = len(seqs)
+    wl.steps.append(workloads.Step(seqs, workloads.normal(rng, (S, hkv, d), "bf16"),
+                                   workloads.normal(rng, (S, hkv, d), "bf16"),
+                                   workloads.normal(rng, (S, hq, d), "bf16")))
+    return wl
+
+
+@pytest.mark.parametrize("g", [1, 2, 4])
+def test_long_shared_runs_and_tail_boundaries(g):
+    """More than 64 sequences (the table comparison runs in the detection grid's extra
+    blocks), siblings sharing 4800 tokens (300 blocks: more than one 256-entry round),
+    and 4-sibling families whose private tails are exactly 4 blocks (taken by the
+    group-rows unit) or 5 blocks (left to the per-sequence kernel), against the oracle;
+    the detection output against the rule."""
+    spec = [(4800, [1, 17, 40, 3]),          # 300 shared blocks
+            (512, [63, 48, 10, 1]),          # tails of at most 4 blocks
+            (512, [64, 80, 5, 0]),           # a 5-block tail: no tails
+            (1040, [15, 16, 47, 63])]        # 65 shared blocks, tails 1..4 blocks
+    wl = _families_workload(spec, g, n_loners=60)
+    ts = TwoSided(wl)
+    step = wl.steps[0]
+    ts.append_step(step)
+    assert ts.pools_equal()
+    ref = ts.oracle_decode(step)
+    for part in (256, 512):
+        check_close(ts.gpu_decode(step, part), ref, "bf16", f"g{g} families partition {part}")
+    assert ts.err_flag() == 0
+    # the detection's output in a fresh workspace against the rule
+    torch = torch_mod()
+    t, l = ts.tables(step.seqs)
+    S, part = len(step.seqs), 512
+    maxc = int(l.max())
+    ws = torch.zeros(ts.pa.pa_decode_workspace_size(S, wl.num_q_heads, wl.head_dim, maxc, part),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty((S, wl.num_q_heads, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    ts.pa.pa_decode(to_dev(step.q), ts.gpu.key_cache, ts.gpu.value_cache, torch.from_numpy(t).cuda(),
+                    torch.from_numpy(l).cuda(), maxc, wl.scale, out, part, ws, ts.gpu.err_flag)
+    assert ts.err_flag() == 0
+    rows = S * wl.num_q_heads * -(-maxc // part)
+    at = -(-(rows * wl.head_dim * 4 + rows * 8) // 16) * 16
+    raw = ws.cpu().numpy()
+    want_ft, want_tiles, want_rows = _expected_groups(t, l, part, g, wl.num_kv_heads)
+    assert raw[at:at + 4 * S].view(np.int32).tolist() == want_ft
+    assert sum(1 for r in want_rows if r[3] == 1) == 3      # three families take their tails
+    assert any(r[3] == 0 for r in want_rows)                # the 5-block tail does not
+
+
 @pytest.mark.parametrize("cid,part", [(1, 0), (1, 16), (2, 256), (3, 0), (3, 256), (4, 256)])
 def test_append_decode_one_call(cid, part):
     """pa_append_decode (cache write + decode in one call, chained launches) gives the
