@@ -143,3 +143,24 @@ def test_speculative_verify_chunks(hq, hkv):
     mask = rows_mask(ks, 8)
     check_close(got[mask], ref[mask], "bf16", f"verify {hq}/{hkv}")
     assert ts.err_flag() == 0
+
+
+def test_many_short_chunks_static_jobs():
+    """256 sequences x 8 kv heads = 2048 one-tile jobs, more than 8 per CTA: the launch
+    takes the static round robin of jobs (fewer per CTA are drawn from a counter, as
+    in every other case here).  Ragged draft counts in [0, 8] (0: an empty job) over
+    contexts of 20..400 tokens."""
+    rng = np.random.default_rng(29)
+    S, hq, hkv = 256, 32, 8
+    lens = rng.integers(20, 401, size=S).tolist()
+    ks = [int(min(k, L)) for k, L in zip(rng.integers(0, 9, size=S), lens)]
+    wl, rng2 = _custom(lens, hq, hkv, seed=31)
+    ts = TwoSided(wl)
+    t, l = ts.tables(list(range(S)))
+    q = workloads.normal(rng2, (S, 8, hq, 128), "bf16")
+    got = gpu_prefill(ts, q, ks, t, l)
+    ref = oracle.prefill(q, ts.kc, ts.vc, t, l, np.array(ks, np.int32), wl.scale)
+    mask = rows_mask(ks, 8)
+    check_close(got[mask], ref[mask], "bf16", "2048 static jobs")
+    assert np.isnan(workloads.bf16_bits_to_f32(got[~mask])).all(), "rows past the chunk must not be written"
+    assert ts.err_flag() == 0
