@@ -1815,13 +1815,13 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         atomicAdd(&work[2], dw);
     }
     // records: tile groups first (the tile kernel reads groups[0, n_tile)), in
-    // sequence order; then the row groups, longest first by buckets of 32 shared
+    // sequence order; then the row groups, longest first by buckets of 8 shared
     // blocks (the group-rows kernel draws its units in record order, so the
     // longest start first and the short ones even out the end; the order within a
     // bucket does not affect any result)
-    constexpr int kBuckets = 8;
+    constexpr int kBuckets = 32;
     __shared__ int rcount[kBuckets], rbase[kBuckets];
-    auto bucket = [](int nb) { return kBuckets - 1 - min(kBuckets - 1, nb >> 5); };  // 0: longest
+    auto bucket = [](int nb) { return kBuckets - 1 - min(kBuckets - 1, nb >> 3); };  // 0: longest
     if (n_row > 0) {  // (uniform)
         if (threadIdx.x < kBuckets) rcount[threadIdx.x] = 0;
         __syncthreads();
@@ -1831,6 +1831,7 @@ __global__ void __launch_bounds__(kDetectThreads) group_detect_kernel(const __gr
         __syncthreads();
         if (threadIdx.x == 0) {
             int run = n_tile;
+#pragma unroll
             for (int b = 0; b < kBuckets; ++b) {
                 rbase[b] = run;
                 run += rcount[b];

@@ -572,7 +572,7 @@ def test_group_detection_matches_the_rule(cid, part):
     assert got[:len(want_tiles)] == want_tiles            # tile groups in sequence order
     got_rows = got[len(want_tiles):]
     assert sorted(got_rows) == sorted(want_rows)          # row groups: longest first by buckets
-    keys = [7 - min(7, (r[2] // 16) >> 5) for r in got_rows]
+    keys = [31 - min(31, (r[2] // 16) >> 3) for r in got_rows]
     assert keys == sorted(keys)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     if want_tiles:   # SMs the detection kernel gave the group tiles
