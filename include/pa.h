@@ -36,7 +36,9 @@
  *
  * Conventions:
  *   - Ownership: the caller owns every buffer, the decode workspace included.
- *     The library allocates no device memory.
+ *     The library allocates no device memory; its module holds two static device
+ *     arrays (the scratch of pa_decode_static_scratch, 32 MiB, and the job
+ *     counters of pa_prefill_chunk, 8 KB), set up when the library is loaded.
  *   - Asynchrony: each call validates its arguments on the host and enqueues its
  *     kernels on `stream` (a cudaStream_t; NULL = legacy default stream).
  *     PA_OK means "validated and launched", not "finished".
@@ -284,6 +286,14 @@ PA_API pa_status pa_decode_static_scratch(const void *query, const void *key_cac
  * its k_s draft tokens (pa_cache_write), then the k_s new positions attend
  * causally with chunk_lens[s] = k_s (chenxutan 5.4, speculative decoding: the
  * target model checks several proposed tokens in one pass).
+ * Work distribution (no effect on results): a job is (sequence, kv head, 256
+ * packed rows).  With at most 8 jobs per SM they are handed out from a work
+ * counter, one of a static pool of 1,024; each call tags its counter with a
+ * per-process ticket, so calls need no ordering between them and nothing is
+ * reset.  A call whose kernel still runs after 1,024 later pa_prefill_chunk
+ * calls of the process have started (impossible on one stream) sets
+ * PA_DEVERR_TIMEOUT and its outputs are unspecified.  With more jobs per SM the
+ * order is a fixed round robin.
  * Source: chenxutan 2.3 (prefill computes a whole prompt and is compute bound)
  * and 4.3/5.1 (long prompts are cut into chunks that run between decodes).
  */
