@@ -242,9 +242,9 @@ __device__ __forceinline__ int first_tok(const Params &p, int s) {
 // units of long sequences (slots after their first unit's), sequence-major, kv
 // head innermost, using cum[s] = sum_{s' < s} (seq_units(s') - 1)^+; after them
 // comes the first per-sequence unit (slot slot_base(ft)) of every sequence that
-// has one, using cum[S + 1 + s] (their count before s).  The further units are
-// all full-length, so putting them first leaves the shorter first units for the
-// end of the queue, where they even out the CTAs' finish.
+// has one, using cum[S + 1 + s] (their count before s).  Most sequences have a
+// first unit only, often short, so the queue tends to end on short units (a strict
+// longest-first order of the first units was measured slower on B200).
 __device__ __forceinline__ Unit unit_of(const Params &p, int64_t u, int64_t n_extra, int hkv,
                                         const int *cum, int S) {
     if (u >= n_extra) {
