@@ -51,6 +51,16 @@
  *     affected outputs are then unspecified.  Read the flag with pa_wait().
  *   - Every wait inside a kernel is bounded; a wait that runs out sets
  *     PA_DEVERR_TIMEOUT and the kernel returns early.
+ *   - CUDA graphs: a captured call replays the values its host side chose at
+ *     capture time.  Cache writes, block copies, unsplit decodes, split decodes of
+ *     fp32 or fp8 pools or head_dim 64, and prefills with more than 8 jobs per
+ *     SM (jobs = num_seqs * num_kv_heads * ceil(max_chunk * g / 256)) replay
+ *     correctly.  Issue directly, not from a graph: a split decode (pa_decode,
+ *     pa_append_decode, pa_decode_static_scratch) of bf16 pools with head_dim 128,
+ *     whose shared-prefix detection tags its flags with a per-call value (a replay
+ *     would read the previous replay's table comparison), and a pa_prefill_chunk
+ *     with at most 8 jobs per SM, whose work counter is tagged per call (a replay
+ *     would find its count spent and skip jobs).
  *   - Programmatic dependent launch: the kernels of a call are chained with it,
  *     and the last kernel of a split decode signals early that a dependent may
  *     launch.  A kernel the caller launches right after a call, with
@@ -175,7 +185,7 @@ PA_API size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, in
 
 /*
  * Number of kernels one pa_decode call with these arguments launches on its
- * stream (for launch accounting and graph planning): 1 unsplit; 2 split (the
+ * stream (for launch accounting): 1 unsplit; 2 split (the
  * partition kernel and the combine); with a split, dtype PA_BF16, head_dim 128 and
  * num_seqs <= 4096 the shared-prefix detection kernel and the tcgen05 group tiles
  * run first (4), and for g = num_q_heads / num_kv_heads <= 4 also the 16-row
