@@ -47,3 +47,33 @@ def test_fp8_pools_count_one_byte_per_cached_element():
     # cache write: bf16 read, e4m3 written
     assert bench.cache_write_bytes(wl, 3) == 3 * 2 * 8 * 2 * (2 + 2)
     assert bench.cache_write_bytes(wl, 3, kv_elem=1) == 3 * 2 * 8 * 2 * (2 + 1)
+
+
+def _record():
+    import json
+    return json.load(open(bench.TRAFFIC_RECORD))
+
+
+def test_traffic_record_is_self_consistent():
+    """The committed DRAM-traffic record: one entry per kernel of the call, summing to
+    the call's total, and hashes for every kernel source the bench checks."""
+    rec = _record()
+    assert sum(rec["per_kernel_bytes"].values()) == rec["dram_bytes_per_call"]
+    assert len(rec["per_kernel_bytes"]) == 5
+    assert set(rec["sources_sha256"]) == set(bench.kernel_sources_sha256())
+
+
+def test_traffic_is_dropped_once_a_kernel_source_changes(monkeypatch):
+    """A record taken for other kernel sources is not reported (traffic null)."""
+    cur = bench.kernel_sources_sha256()
+    changed = dict(cur, **{"decode.cu": "0" * 64})
+    monkeypatch.setattr(bench, "kernel_sources_sha256", lambda: changed)
+    assert bench.recorded_traffic() is None
+
+
+def test_traffic_is_reported_for_the_sources_it_was_taken_on():
+    rec = _record()
+    if rec["sources_sha256"] != bench.kernel_sources_sha256():
+        import pytest
+        pytest.skip("kernel sources changed since the capture: the bench reports traffic null")
+    assert bench.recorded_traffic() == rec["dram_bytes_per_call"]
